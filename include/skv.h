@@ -1,0 +1,194 @@
+/*
+ * skv.h -- C ABI of libskv: equal-variation KV-cache coarsening and compressed
+ * (macro-node) single-query decode attention on one NVIDIA B200 (sm_100a).
+ *
+ * Two operations, from two web pages:
+ *
+ *  1. skv_coarsen: "Equal-Variation KV Cache" (synthcore idea 664),
+ *     "Mathematical statement" and "Implementation notes". Per (sequence, KV
+ *     head) unit the first n_sink tokens and the last n_recent tokens stay
+ *     exact; the middle span is cut into N segments of equal cumulative
+ *     variation of the projected trajectory z_t = P [k_t; v_t] (first token
+ *     whose cumulative variation reaches j c_T / N starts segment j); each
+ *     nonempty segment becomes one macro-node. Node statistics follow the
+ *     "SPICY-KV" demo page, Independent Claims 2-3 and section 2: mass m =
+ *     member count, mean key, mean value, per-dimension key variance sigma^2
+ *     averaged over the d dimensions, alpha = ln m, beta = sigma^2 / (2 d).
+ *
+ *  2. skv_decode_attn: "SPICY-KV" demo page, section 2 ("FlashAttention-2/3 &
+ *     PagedAttention Online-Softmax Kernel Fusion") and Claim 3. For each
+ *     query row q and each entry j of its KV head's compressed cache,
+ *     s_j = q.k_j / sqrt(d) + alpha_j + |q|^2 beta_j; out = softmax(s) V and
+ *     lse = ln sum_j exp(s_j).
+ *
+ * Conventions shared by every entry point:
+ *  - All tensor arguments are DEVICE pointers unless the name ends in _host.
+ *    The caller owns every buffer (inputs, outputs, node pool, page table,
+ *    workspace). No entry point allocates device memory or synchronises the
+ *    stream, except skv_workspace_error, which synchronises to read a flag.
+ *  - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Work is enqueued on it in order; the call returns before it finishes.
+ *  - Host-detectable errors return before anything is enqueued. Errors that
+ *    only the device can see (a page id outside the pool, a lens entry above
+ *    the page table's capacity, a variation overflow) set a flag in the
+ *    workspace header that skv_workspace_error reports; the offending write is
+ *    skipped, never performed out of bounds.
+ *  - Supported: d in {64, 128}; dtype SKV_F32 or SKV_BF16 (keys, values,
+ *    queries, node vectors and outputs share the dtype; alpha/beta and lse are
+ *    fp32); at most SKV_MAX_SEQS sequences per call.
+ *
+ * Node pool layout (produced by skv_coarsen, consumed by skv_decode_attn):
+ *  A page holds SKV_PAGE_NODES = 16 consecutive entries of ONE unit.
+ *    pool.k, pool.v : [num_pages][16][d] in the dtype. Within a page the
+ *                     16-byte chunk c of slot n's vector is stored at chunk
+ *                     position c ^ (n & 7) (a bank-conflict-free order for
+ *                     the tensor-core fragment loads; d * elem >= 128 bytes).
+ *    pool.ab        : [num_pages][16] pairs {alpha, beta} (fp32).
+ *  page_table : [B][Hkv][max_pages] int32 physical page ids; entry e of unit
+ *               (b, h) lives in page page_table[b][h][e / 16], slot e % 16.
+ *  lens       : [B][Hkv] int32 entries per unit, in the order sinks, nonempty
+ *               middle segments (in token order), recents.
+ *  Every pool pointer must be 16-byte aligned.
+ */
+#ifndef SKV_H
+#define SKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    SKV_OK = 0,
+    SKV_ERR_INVALID_ARG = -1, /* null pointer, bad size, misaligned buffer */
+    SKV_ERR_UNSUPPORTED = -2, /* valid but outside the built configurations */
+    SKV_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
+    SKV_ERR_OVERFLOW = -4,    /* variation step above 2^20 or too many tokens */
+    SKV_ERR_WORKSPACE = -6,   /* workspace smaller than the *_workspace_bytes query */
+    SKV_ERR_DEVICE = -7       /* device-detected bad page id or lens (see flags) */
+} skv_status;
+
+typedef enum { SKV_F32 = 0, SKV_BF16 = 1 } skv_dtype;
+
+#define SKV_PAGE_NODES 16
+#define SKV_PROJ_DIM 16
+#define SKV_MAX_SEQS 512
+#define SKV_MAX_TOKENS ((1 << 22) - 1) /* per sequence */
+
+typedef struct {
+    void *k;           /* [num_pages][16][d] mean keys (device) */
+    void *v;           /* [num_pages][16][d] mean values (device) */
+    float *ab;         /* [num_pages][16][2] alpha, beta (device) */
+    int64_t num_pages; /* capacity of the three arrays, in pages */
+} skv_node_pool;
+
+/* Human-readable name of a status code (static storage; never NULL). */
+const char *skv_status_string(int status);
+
+/* ABI version of this header (major * 100 + minor). */
+int skv_abi_version(void);
+
+/*
+ * The projection the coarsener draws from proj_seed ("Equal-Variation KV
+ * Cache", "Implementation notes": z_t = P [k_t; v_t] with P a fixed random
+ * projection). P_host: [16][2d] fp32 row-major, written on the host; no GPU
+ * work. Entry e consumes two SplitMix64 words a, b of the stream seeded by
+ * proj_seed: u1 = ((a >> 11) + 1) 2^-53, u2 = (b >> 11) 2^-53, entry =
+ * fp32(sqrt(-2 ln u1) cos(2 pi u2) / 4).
+ * Errors: SKV_ERR_INVALID_ARG for P_host == NULL or d not in {64, 128}.
+ */
+skv_status skv_projection_matrix(uint64_t proj_seed, int d, float *P_host);
+
+/*
+ * Bytes of device workspace skv_coarsen needs for this batch (0 on invalid
+ * arguments). T_host, N_host: [B] host arrays of sequence lengths and segment
+ * counts.
+ */
+size_t skv_coarsen_workspace_bytes(int B, int Hkv, int d, const int32_t *T_host, const int32_t *N_host,
+                                   int n_sink, int n_recent);
+
+/*
+ * Coarsen B sequences x Hkv KV heads into the node pool.
+ *
+ * k, v      : raw keys/values in dtype. Sequence b occupies the contiguous
+ *             block [Hkv][T_b][d] starting at element offset
+ *             (T_0 + ... + T_{b-1}) * Hkv * d (for equal T this is
+ *             [B][Hkv][T][d]). Read only.
+ * T_host    : [B] host, tokens per sequence, 0 <= T_b <= SKV_MAX_TOKENS.
+ * n_sink, n_recent : exact tokens kept at the start / end (>= 0). When
+ *             T_b < n_sink + n_recent the sinks take priority.
+ * N_host    : [B] host, middle segments per sequence, 1 <= N_b <= 2^20.
+ * proj_seed : seed of the projection P (see skv_projection_matrix).
+ * pool, page_table, max_pages : output node pool and the caller's page
+ *             assignment ([B][Hkv][max_pages] int32, device). Unit (b, h)
+ *             needs ceil((S_eff + N_b + W_eff) / 16) pages (host-checked
+ *             against max_pages; page ids device-checked against num_pages).
+ * lens      : [B][Hkv] int32 device output, entries written per unit.
+ * boundaries: optional ([B][Hkv][Nmax+1] int32 device, Nmax = max_b N_b):
+ *             middle-local segment boundaries b_0 = 0 <= ... <= b_N = M_b.
+ * cumvar    : optional int64 device array with the token layout of k (one
+ *             value per token and head); position t < M_b of unit (b, h)
+ *             receives the cumulative quantised variation c_t of middle
+ *             token t. Other positions are left untouched.
+ * workspace : device scratch of at least skv_coarsen_workspace_bytes bytes,
+ *             256-byte aligned; its header holds the device error flags.
+ *
+ * The variation step d_t = ||z_t - z_{t-1}||_2 is quantised to
+ * D_t = rne(d_t * 2^20) (int64) through one fixed fp32 recipe: each z_i is an
+ * fp32 fma chain over j = 0..2d-1 ascending from 0; d_t = sqrtf of an fma
+ * chain of squared differences over i = 0..15 ascending. The boundaries are
+ * therefore exact integers: b_j = min{ t : N c_t >= j c_T } (128-bit
+ * products). Node statistics are fp32 (two-pass variance), node vectors are
+ * stored in dtype (round to nearest even).
+ *
+ * Errors: SKV_ERR_INVALID_ARG (null pointers, negative sizes, B > SKV_MAX_SEQS,
+ * misalignment, workspace too small -> SKV_ERR_WORKSPACE), SKV_ERR_UNSUPPORTED
+ * (d, dtype), SKV_ERR_CUDA (launch failure). A step above 2^20 sets the
+ * device overflow flag (SKV_ERR_OVERFLOW from skv_workspace_error).
+ */
+skv_status skv_coarsen(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d,
+                       const int32_t *T_host, int n_sink, int n_recent, const int32_t *N_host,
+                       uint64_t proj_seed, const skv_node_pool *pool, const int32_t *page_table,
+                       int max_pages, int32_t *lens, int32_t *boundaries, int64_t *cumvar,
+                       void *workspace, size_t ws_bytes, void *stream);
+
+/* Bytes of device workspace skv_decode_attn needs (0 on invalid arguments). */
+size_t skv_decode_workspace_bytes(int B, int R, int Hq, int Hkv, int d, int max_pages);
+
+/*
+ * Compressed decode attention.
+ *
+ * q     : [B][R][Hq][d] queries in dtype (R independent query rows per
+ *         sequence, pre-RoPE basis). Query head hq reads KV head hq / (Hq/Hkv).
+ * pool, page_table, max_pages, lens : the compressed cache (layout above).
+ * out   : [B][R][Hq][d] in dtype, softmax(s) V.
+ * lse   : [B][R][Hq] fp32, natural-log partition ln sum_j exp(s_j); a unit
+ *         with zero entries gives out = 0 and lse = -inf.
+ * workspace : device scratch of at least skv_decode_workspace_bytes bytes,
+ *         256-byte aligned (split partials and the device error flags).
+ *
+ * Errors: SKV_ERR_INVALID_ARG, SKV_ERR_UNSUPPORTED (d, dtype, Hq % Hkv != 0),
+ * SKV_ERR_WORKSPACE, SKV_ERR_CUDA. Device-detected bad page ids or lens above
+ * max_pages * 16 set the device flag (SKV_ERR_DEVICE from
+ * skv_workspace_error); those pages are skipped.
+ */
+skv_status skv_decode_attn(const void *q, skv_dtype dtype, int B, int R, int Hq, int Hkv, int d,
+                           const skv_node_pool *pool, const int32_t *page_table, int max_pages,
+                           const int32_t *lens, void *out, float *lse, void *workspace, size_t ws_bytes,
+                           void *stream);
+
+/*
+ * Synchronise stream and report the device error flags that the last
+ * skv_coarsen or skv_decode_attn call on this workspace raised: SKV_OK,
+ * SKV_ERR_OVERFLOW or SKV_ERR_DEVICE (SKV_ERR_CUDA if synchronisation fails).
+ * *flags_host (optional) receives the raw flag bits.
+ */
+skv_status skv_workspace_error(const void *workspace, void *stream, uint32_t *flags_host);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SKV_H */
