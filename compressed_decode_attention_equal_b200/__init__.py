@@ -1,0 +1,197 @@
+"""Equal-variation KV-cache coarsening and compressed decode attention for B200.
+
+A thin binding over libskv's C ABI (include/skv.h): torch tensors are checked
+and passed as raw device pointers with the current CUDA stream. Every step of
+both operations runs in libskv's sm_100a kernels; there is no CPU or PyTorch
+fallback, and a missing library raises at the first call.
+
+  coarsen(...)      "Equal-Variation KV Cache" (synthcore idea 664) segmentation
+                    of each (sequence, KV head) history into macro-nodes with
+                    "SPICY-KV" node statistics (mass, mean key/value, variance)
+  decode_attn(...)  "SPICY-KV" section 2 decode logit
+                    q.k/sqrt(d) + ln m + |q|^2 sigma^2/(2d) with online softmax
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+
+import torch
+
+from . import _lib
+from ._lib import PAGE_NODES, SkvError
+
+__all__ = ["NodePool", "coarsen", "decode_attn", "coarsen_workspace_bytes", "decode_workspace_bytes",
+           "workspace_error", "projection_matrix", "entries_bound", "pages_for", "read_entries", "SkvError",
+           "PAGE_NODES", "library_path"]
+
+
+def library_path() -> str:
+    return _lib.LIB_PATH
+
+
+def _code(dtype: torch.dtype) -> int:
+    if dtype == torch.bfloat16:
+        return _lib.SKV_BF16
+    if dtype == torch.float32:
+        return _lib.SKV_F32
+    raise TypeError(f"unsupported dtype {dtype}; use torch.bfloat16 or torch.float32")
+
+
+def _stream_handle(stream) -> int:
+    s = torch.cuda.current_stream() if stream is None else stream
+    return int(s.cuda_stream)
+
+
+def _dev(t: torch.Tensor, name: str):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _i32(xs):
+    return (ctypes.c_int32 * len(xs))(*[int(x) for x in xs])
+
+
+def entries_bound(T: int, N: int, n_sink: int, n_recent: int) -> int:
+    """Upper bound on the entries one unit produces: sinks + N segments (if any middle) + recents."""
+    s = min(n_sink, T)
+    r = min(n_recent, T - s)
+    return s + (N if T - s - r > 0 else 0) + r
+
+
+def pages_for(T: int, N: int, n_sink: int, n_recent: int) -> int:
+    return -(-entries_bound(T, N, n_sink, n_recent) // PAGE_NODES)
+
+
+class NodePool:
+    """Paged macro-node storage: k, v [num_pages, 16, d] (dtype) and ab [num_pages, 16, 2] fp32
+    (alpha = ln m, beta = sigma^2 / (2d)). Within a page, 16-byte chunk c of slot n is stored at
+    chunk c ^ (n & 7)."""
+
+    def __init__(self, num_pages: int, d: int, dtype: torch.dtype, device="cuda"):
+        self.num_pages, self.d, self.dtype = int(num_pages), int(d), dtype
+        self.k = torch.empty(self.num_pages, PAGE_NODES, d, dtype=dtype, device=device)
+        self.v = torch.empty(self.num_pages, PAGE_NODES, d, dtype=dtype, device=device)
+        self.ab = torch.empty(self.num_pages, PAGE_NODES, 2, dtype=torch.float32, device=device)
+
+    def struct(self) -> _lib.SkvNodePool:
+        return _lib.SkvNodePool(self.k.data_ptr(), self.v.data_ptr(), self.ab.data_ptr(), self.num_pages)
+
+    def nbytes(self) -> int:
+        return self.k.numel() * self.k.element_size() * 2 + self.ab.numel() * 4
+
+
+def projection_matrix(seed: int, d: int) -> torch.Tensor:
+    """The 16 x 2d projection skv_coarsen draws from `seed` (computed on the host)."""
+    out = torch.empty(16, 2 * d, dtype=torch.float32)
+    _lib.check(_lib.load().skv_projection_matrix(ctypes.c_uint64(seed), d,
+                                                  ctypes.cast(out.data_ptr(), ctypes.POINTER(ctypes.c_float))),
+               "skv_projection_matrix")
+    return out
+
+
+def coarsen_workspace_bytes(Hkv: int, d: int, T_list, N_list, n_sink: int, n_recent: int) -> int:
+    B = len(T_list)
+    return int(_lib.load().skv_coarsen_workspace_bytes(B, Hkv, d, _i32(T_list), _i32(N_list), n_sink, n_recent))
+
+
+def coarsen(k: torch.Tensor, v: torch.Tensor, Hkv: int, T_list, N_list, n_sink: int, n_recent: int,
+            proj_seed: int, pool: NodePool, page_table: torch.Tensor, lens: torch.Tensor | None = None,
+            boundaries: torch.Tensor | None = None, cumvar: torch.Tensor | None = None,
+            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Coarsen B sequences (k, v: [sum_b Hkv*T_b, d], sequence b a contiguous [Hkv, T_b, d] block)
+    into `pool` through `page_table` [B, Hkv, max_pages] int32. Returns lens [B, Hkv] int32."""
+    B = len(T_list)
+    d = k.shape[-1]
+    if v.shape != k.shape or v.dtype != k.dtype:
+        raise ValueError("k and v must have the same shape and dtype")
+    if pool.dtype != k.dtype or pool.d != d:
+        raise ValueError("pool dtype / d must match k")
+    if page_table.dtype != torch.int32 or page_table.dim() != 3 or tuple(page_table.shape[:2]) != (B, Hkv):
+        raise ValueError("page_table must be int32 [B, Hkv, max_pages]")
+    dev = k.device
+    if lens is None:
+        lens = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
+    ws_bytes = coarsen_workspace_bytes(Hkv, d, T_list, N_list, n_sink, n_recent)
+    if ws_bytes == 0:
+        raise SkvError(_lib.SKV_ERR_INVALID_ARG, "skv_coarsen_workspace_bytes")
+    if workspace is None:
+        workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
+    ps = pool.struct()
+    null = ctypes.c_void_p(0)
+    st = _lib.load().skv_coarsen(
+        _dev(k, "k") if k.numel() else null, _dev(v, "v") if v.numel() else null, _code(k.dtype), B, Hkv, d,
+        _i32(T_list), n_sink, n_recent, _i32(N_list), ctypes.c_uint64(proj_seed), ctypes.byref(ps),
+        _dev(page_table, "page_table"), page_table.shape[2], _dev(lens, "lens"),
+        _dev(boundaries, "boundaries") if boundaries is not None else null,
+        _dev(cumvar, "cumvar") if cumvar is not None else null,
+        _dev(workspace, "workspace"), workspace.numel(), ctypes.c_void_p(_stream_handle(stream)))
+    _lib.check(st, "skv_coarsen")
+    return lens
+
+
+def decode_workspace_bytes(B: int, R: int, Hq: int, Hkv: int, d: int, max_pages: int) -> int:
+    return int(_lib.load().skv_decode_workspace_bytes(B, R, Hq, Hkv, d, max_pages))
+
+
+def decode_attn(q: torch.Tensor, Hkv: int, pool: NodePool, page_table: torch.Tensor, lens: torch.Tensor,
+                out: torch.Tensor | None = None, lse: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None, stream=None):
+    """q [B, R, Hq, d] against the compressed cache. Returns (out [B, R, Hq, d], lse [B, R, Hq] fp32)."""
+    B, R, Hq, d = q.shape
+    if pool.dtype != q.dtype or pool.d != d:
+        raise ValueError("pool dtype / d must match q")
+    if page_table.dtype != torch.int32 or page_table.dim() != 3 or tuple(page_table.shape[:2]) != (B, Hkv):
+        raise ValueError("page_table must be int32 [B, Hkv, max_pages]")
+    if lens.dtype != torch.int32 or tuple(lens.shape) != (B, Hkv):
+        raise ValueError("lens must be int32 [B, Hkv]")
+    max_pages = page_table.shape[2]
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, R, Hq, dtype=torch.float32, device=q.device)
+    if workspace is None:
+        workspace = torch.zeros(decode_workspace_bytes(B, R, Hq, Hkv, d, max_pages), dtype=torch.uint8,
+                                device=q.device)
+    ps = pool.struct()
+    st = _lib.load().skv_decode_attn(
+        _dev(q, "q"), _code(q.dtype), B, R, Hq, Hkv, d, ctypes.byref(ps), _dev(page_table, "page_table"),
+        max_pages, _dev(lens, "lens"), _dev(out, "out"), _dev(lse, "lse"), _dev(workspace, "workspace"),
+        workspace.numel(), ctypes.c_void_p(_stream_handle(stream)))
+    _lib.check(st, "skv_decode_attn")
+    return out, lse
+
+
+def workspace_error(workspace: torch.Tensor, stream=None):
+    """Synchronise and read-and-clear the device error flags of a workspace: (status, flags)."""
+    flags = ctypes.c_uint32(0)
+    st = _lib.load().skv_workspace_error(_dev(workspace, "workspace"), ctypes.c_void_p(_stream_handle(stream)),
+                                         ctypes.byref(flags))
+    return st, flags.value
+
+
+def read_entries(pool: NodePool, page_table: torch.Tensor, lens: torch.Tensor, b: int, h: int):
+    """Entries of unit (b, h) in entry order, un-swizzled: (kt [E, d], vt [E, d], alpha [E], beta [E]).
+    A layout view for inspection (indexing only)."""
+    E = int(lens[b, h])
+    d = pool.d
+    if E == 0:
+        z = pool.k.new_zeros(0, d)
+        return z, z.clone(), pool.ab.new_zeros(0), pool.ab.new_zeros(0)
+    n_pages = -(-E // PAGE_NODES)
+    pages = page_table[b, h, :n_pages].long()
+    rows = (pages[:, None] * PAGE_NODES + torch.arange(PAGE_NODES, device=pages.device)).reshape(-1)[:E]
+    epc = 16 // pool.k.element_size()
+    ch = d // epc
+    slot = torch.arange(E, device=pages.device) % PAGE_NODES
+    phys = torch.arange(ch, device=pages.device)[None, :] ^ (slot[:, None] & 7)
+    kr = pool.k.reshape(-1, ch, epc)[rows]
+    vr = pool.v.reshape(-1, ch, epc)[rows]
+    idx = phys[:, :, None].expand(E, ch, epc)
+    kt = torch.gather(kr, 1, idx).reshape(E, d)
+    vt = torch.gather(vr, 1, idx).reshape(E, d)
+    ab = pool.ab.reshape(-1, 2)[rows]
+    return kt, vt, ab[:, 0], ab[:, 1]

@@ -1,0 +1,493 @@
+// Equal-variation coarsening of a KV cache into macro-nodes.
+//
+// "Equal-Variation KV Cache" (synthcore idea 664), Mathematical statement and
+// Implementation notes: the middle span of each (sequence, KV head) unit is cut
+// at the first tokens whose cumulative variation of z_t = P [k_t; v_t] reaches
+// j c_T / N. "SPICY-KV" demo page, Claims 2-3 and section 2: each segment keeps
+// its mass m, mean key, mean value and per-dimension key variance, stored as
+// alpha = ln m and beta = sigma^2 / (2 d).
+//
+// Pipeline (stream-ordered launches, all integer stages exact):
+//   k_setup          copy the host-built per-sequence plan into the workspace
+//   k_project_scan   TMA-staged tiles of 255 middle tokens (+1 halo): z via the
+//                    fixed fp32 fma recipe, D_t = rne(d_t 2^20), tile-local
+//                    inclusive int64 scan and tile totals
+//   k_tile_prefix    exclusive scan of tile totals per unit, c_T
+//   k_boundaries     every token writes the thresholds it crosses:
+//                    b_j = t for N c_{t-1} < j c_T <= N c_t (128-bit products)
+//   k_plan_entries   drop empty segments, lay out entries (sinks, segments,
+//                    recents) and write lens
+//   k_segment_reduce one warp per entry: two-pass mean / variance, node write
+//                    into the paged pool (swizzled 16-byte chunks)
+#include "skv_common.cuh"
+#include "skv_internal.h"
+
+namespace skv {
+
+// ---------------------------------------------------------------------------
+// k_setup: per-sequence plan -> workspace; clear the error flags
+// ---------------------------------------------------------------------------
+__global__ void k_setup(const __grid_constant__ SeqTable table, SeqRow *dst, int B, uint32_t *flags) {
+    for (int b = threadIdx.x; b < B; b += blockDim.x) dst[b] = table.rows[b];
+    if (threadIdx.x == 0) *flags = 0u;
+}
+
+// ---------------------------------------------------------------------------
+// k_project_scan
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ float elem_of(const uint4 &w, int e);
+
+template <>
+__device__ __forceinline__ float elem_of<__nv_bfloat16>(const uint4 &w, int e) {
+    const uint32_t x = (e >> 1) == 0 ? w.x : (e >> 1) == 1 ? w.y : (e >> 1) == 2 ? w.z : w.w;
+    return (e & 1) ? bf16hi(x) : bf16lo(x);
+}
+
+template <>
+__device__ __forceinline__ float elem_of<float>(const uint4 &w, int e) {
+    const uint32_t x = e == 0 ? w.x : e == 1 ? w.y : e == 2 ? w.z : w.w;
+    return __uint_as_float(x);
+}
+
+// D = rne(||zc - zp||_2 * 2^20) by the fixed recipe (fp32, i ascending); -1 on overflow.
+__device__ __forceinline__ long long quantised_step(const float *zp, const float *zc) {
+    float s = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kProjDim; ++i) {
+        const float di = __fsub_rn(zc[i], zp[i]);
+        s = __fmaf_rn(di, di, s);
+    }
+    const float dd = __fsqrt_rn(s);
+    const float scaled = __fmul_rn(dd, 1048576.0f);
+    if (!(scaled <= 0x1p40f)) return -1;
+    return __float2ll_rn(scaled);
+}
+
+constexpr int kK1Threads = 128;
+constexpr int kK1Stages = 2;
+constexpr int kK1StageBytes = kTileRows * 128;   // one 128-byte column chunk of 256 rows
+constexpr int kZStride = 20;                     // floats per row of the z buffer (conflict-free)
+
+template <int D>
+constexpr size_t k1_smem_bytes() {
+    return 1024 /*alignment slack*/ + kK1Stages * kK1StageBytes + 2 * D * kProjDim * sizeof(float) + 64 + 64;
+}
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kK1Threads, 2)
+    k_project_scan(const CoarsenArgs a, const __grid_constant__ CUtensorMap map_k,
+                   const __grid_constant__ CUtensorMap map_v, const __grid_constant__ ProjT proj) {
+    constexpr int ELEM = sizeof(T);
+    constexpr int KCHUNK = D * ELEM / 128;    // 128-byte chunks of one key row
+    constexpr int NCHUNK = 2 * KCHUNK;        // key chunks, then value chunks
+    constexpr int JPC = 128 / ELEM;           // feature index j per chunk
+    constexpr int EPS = 16 / ELEM;            // elements per 16-byte sub-chunk
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t *stages = smem;
+    float *pt = reinterpret_cast<float *>(smem + kK1Stages * kK1StageBytes);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(pt + 2 * D * kProjDim);
+    long long *warp_sum = reinterpret_cast<long long *>(bar + 8);
+
+    const int u = blockIdx.y;
+    const int tile = blockIdx.x;
+    const int b = u / a.Hkv, h = u % a.Hkv;
+    const SeqRow sr = a.seq[b];
+    if (tile >= sr.tiles) return;
+    const int tid = threadIdx.x;
+
+    const int y0 = static_cast<int>(sr.row_off + static_cast<int64_t>(h) * sr.T + sr.s_eff) + tile * kTileOut - 1;
+    if (tid == 0) {
+        prefetch_tensormap(&map_k);
+        prefetch_tensormap(&map_v);
+        for (int s = 0; s < kK1Stages; ++s) mbar_init(&bar[s], 1);
+        fence_mbar_init();
+        for (int c = 0; c < NCHUNK && c < kK1Stages; ++c) {
+            mbar_arrive_expect_tx(&bar[c], kK1StageBytes);
+            tma_load_2d(stages + c * kK1StageBytes, c < KCHUNK ? &map_k : &map_v, (c % KCHUNK) * JPC, y0, &bar[c]);
+        }
+    }
+    for (int i = tid; i < 2 * D * kProjDim; i += kK1Threads) pt[i] = proj.pt[i];
+    __syncthreads();
+
+    const uint32_t pt_addr = smem_u32(pt);
+    const int r0 = tid, r1 = tid + kK1Threads;
+    uint64_t acc0[kProjDim / 2], acc1[kProjDim / 2];
+#pragma unroll
+    for (int i = 0; i < kProjDim / 2; ++i) acc0[i] = acc1[i] = 0ull;
+
+    bool ok = true;
+    for (int c = 0; c < NCHUNK; ++c) {
+        const int s = c % kK1Stages;
+        if (ok && !mbar_wait(&bar[s], (c / kK1Stages) & 1)) ok = false;
+        const uint32_t base = smem_u32(stages + s * kK1StageBytes);
+#pragma unroll 1
+        for (int sc = 0; sc < 8; ++sc) {
+            const uint4 xa = lds128(base + r0 * 128 + ((sc ^ (r0 & 7)) << 4));
+            const uint4 xb = lds128(base + r1 * 128 + ((sc ^ (r1 & 7)) << 4));
+#pragma unroll
+            for (int e = 0; e < EPS; ++e) {
+                const int j = c * JPC + sc * EPS + e;
+                const float va = elem_of<T>(xa, e), vb = elem_of<T>(xb, e);
+                const uint64_t xa2 = f2pack(va, va), xb2 = f2pack(vb, vb);
+                const uint32_t prow = pt_addr + j * kProjDim * 4;
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) {
+                    const float4 p = lds128f(prow + q4 * 16);
+                    const uint64_t pa = f2pack(p.x, p.y), pb = f2pack(p.z, p.w);
+                    acc0[2 * q4] = ffma2(pa, xa2, acc0[2 * q4]);
+                    acc0[2 * q4 + 1] = ffma2(pb, xa2, acc0[2 * q4 + 1]);
+                    acc1[2 * q4] = ffma2(pa, xb2, acc1[2 * q4]);
+                    acc1[2 * q4 + 1] = ffma2(pb, xb2, acc1[2 * q4 + 1]);
+                }
+            }
+        }
+        __syncthreads();
+        if (tid == 0 && c + kK1Stages < NCHUNK) {
+            const int cn = c + kK1Stages;
+            mbar_arrive_expect_tx(&bar[s], kK1StageBytes);
+            tma_load_2d(stages + s * kK1StageBytes, cn < KCHUNK ? &map_k : &map_v, (cn % KCHUNK) * JPC, y0, &bar[s]);
+        }
+    }
+    if (!ok) {
+        raise_flag(a.flags, FLAG_TIMEOUT);
+    }
+
+    // z of both rows -> shared (stage 0 is free: every chunk has been consumed and synced)
+    float *zb = reinterpret_cast<float *>(stages);
+#pragma unroll
+    for (int i = 0; i < kProjDim / 2; ++i) {
+        f2unpack(acc0[i], zb[r0 * kZStride + 2 * i], zb[r0 * kZStride + 2 * i + 1]);
+        f2unpack(acc1[i], zb[r1 * kZStride + 2 * i], zb[r1 * kZStride + 2 * i + 1]);
+    }
+    __syncthreads();
+
+    // outputs l = 2 tid + 1, 2 tid + 2 (rows of the tile; row 0 is the halo)
+    long long Dv[2];
+#pragma unroll
+    for (int q = 0; q < 2; ++q) {
+        const int l = 2 * tid + 1 + q;
+        const int t = tile * kTileOut + l - 1;
+        long long D_ = 0;
+        if (l <= kTileOut && t < sr.M && t > 0) {
+            D_ = quantised_step(zb + (l - 1) * kZStride, zb + l * kZStride);
+            if (D_ < 0) {
+                raise_flag(a.flags, FLAG_OVERFLOW);
+                D_ = 0;
+            }
+        }
+        Dv[q] = D_;
+    }
+    // block inclusive scan of the pair sums
+    const int lane = tid & 31, warp = tid >> 5;
+    long long v = Dv[0] + Dv[1];
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const long long n = __shfl_up_sync(0xffffffffu, v, off);
+        if (lane >= off) v += n;
+    }
+    if (lane == 31) warp_sum[warp] = v;
+    __syncthreads();
+    long long wp = 0;
+    for (int w = 0; w < warp; ++w) wp += warp_sum[w];
+    const long long incl = wp + v;
+    const long long excl = incl - Dv[0] - Dv[1];
+    int64_t *ls = a.local_scan + sr.mid_off + static_cast<int64_t>(h) * sr.M;
+    const int t0 = tile * kTileOut + 2 * tid;   // middle index of output l = 2 tid + 1
+    if (2 * tid + 1 <= kTileOut && t0 < sr.M) ls[t0] = excl + Dv[0];
+    if (2 * tid + 2 <= kTileOut && t0 + 1 < sr.M) ls[t0 + 1] = excl + Dv[0] + Dv[1];
+    if (tid == kK1Threads - 1) a.tile_total[static_cast<int64_t>(u) * a.max_tiles + tile] = incl;
+}
+
+// ---------------------------------------------------------------------------
+// k_tile_prefix: exclusive scan of the tile totals of one unit; c_T
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) k_tile_prefix(const CoarsenArgs a) {
+    __shared__ long long wsum[8];
+    __shared__ long long carry_s;
+    const int u = blockIdx.x;
+    const int b = u / a.Hkv;
+    const SeqRow sr = a.seq[b];
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t rowb = static_cast<int64_t>(u) * a.max_tiles;
+    long long carry = 0;
+    for (int base = 0; base < sr.tiles; base += 256) {
+        const int i = base + tid;
+        const long long x = i < sr.tiles ? a.tile_total[rowb + i] : 0;
+        long long v = x;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const long long n = __shfl_up_sync(0xffffffffu, v, off);
+            if (lane >= off) v += n;
+        }
+        if (lane == 31) wsum[warp] = v;
+        __syncthreads();
+        long long wp = 0;
+        for (int w = 0; w < warp; ++w) wp += wsum[w];
+        if (i < sr.tiles) a.tile_prefix[rowb + i] = carry + wp + v - x;
+        if (tid == 255) carry_s = carry + wp + v;
+        __syncthreads();
+        carry = carry_s;
+        __syncthreads();
+    }
+    if (tid == 0) a.unit_total[u] = carry;
+}
+
+// ---------------------------------------------------------------------------
+// k_boundaries: b_j = first t with N c_t >= j c_T  (j = 1 .. N-1)
+// ---------------------------------------------------------------------------
+// floor(N * C / CT) for CT > 0, exact (the double estimate is off by at most one)
+__device__ __forceinline__ long long floor_ratio(long long N, long long C, long long CT) {
+    long long q = static_cast<long long>(static_cast<double>(N) * static_cast<double>(C) / static_cast<double>(CT));
+    if (q < 0) q = 0;
+    while (prod_ge(static_cast<uint64_t>(N), static_cast<uint64_t>(C), static_cast<uint64_t>(q + 1),
+                   static_cast<uint64_t>(CT)))
+        ++q;
+    while (q > 0 && !prod_ge(static_cast<uint64_t>(N), static_cast<uint64_t>(C), static_cast<uint64_t>(q),
+                             static_cast<uint64_t>(CT)))
+        --q;
+    return q;
+}
+
+__global__ void __launch_bounds__(256) k_boundaries(const CoarsenArgs a) {
+    const int u = blockIdx.y, tile = blockIdx.x;
+    const int b = u / a.Hkv, h = u % a.Hkv;
+    const SeqRow sr = a.seq[b];
+    if (tile >= sr.tiles || threadIdx.x >= kTileOut) return;
+    const int t = tile * kTileOut + threadIdx.x;
+    if (t >= sr.M) return;
+    const int64_t *ls = a.local_scan + sr.mid_off + static_cast<int64_t>(h) * sr.M;
+    const long long tp = a.tile_prefix[static_cast<int64_t>(u) * a.max_tiles + tile];
+    const long long CT = a.unit_total[u];
+    const long long Ct = tp + ls[t];
+    const long long Cprev = threadIdx.x == 0 ? tp : tp + ls[t - 1];
+    if (a.cumvar) a.cumvar[sr.row_off + static_cast<int64_t>(h) * sr.T + t] = Ct;
+    const int N = sr.N;
+    int32_t *bnd = a.bounds + sr.bnd_off + static_cast<int64_t>(h) * (N + 1);
+    if (CT == 0) {
+        if (t == 0)
+            for (int j = 1; j < N; ++j) bnd[j] = 0;
+        return;
+    }
+    if (t == 0) return;
+    long long jhi = floor_ratio(N, Ct, CT);
+    if (jhi > N - 1) jhi = N - 1;
+    const long long jlo = floor_ratio(N, Cprev, CT) + 1;
+    for (long long j = jlo; j <= jhi; ++j) bnd[j] = t;
+}
+
+// ---------------------------------------------------------------------------
+// k_plan_entries: entries (start, mass) in the order sinks, nonempty segments, recents
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(512) k_plan_entries(const CoarsenArgs a) {
+    __shared__ int wsum[16];
+    __shared__ int carry_s;
+    const int u = blockIdx.x;
+    const int b = u / a.Hkv, h = u % a.Hkv;
+    const SeqRow sr = a.seq[b];
+    const int N = sr.N, M = sr.M;
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    int32_t *bnd = a.bounds + sr.bnd_off + static_cast<int64_t>(h) * (N + 1);
+    if (M == 0) {
+        for (int j = tid; j <= N; j += 512) bnd[j] = 0;
+    } else if (tid == 0) {
+        bnd[0] = 0;
+        bnd[N] = M;
+    }
+    __syncthreads();
+    int2 *ents = a.ents + sr.ent_off + static_cast<int64_t>(h) * sr.emax;
+    for (int e = tid; e < sr.s_eff; e += 512) ents[e] = make_int2(e, 1);
+    int carry = 0;
+    for (int base = 0; base < N; base += 512) {
+        const int j = base + tid;
+        int lo = 0, hi = 0;
+        if (j < N) {
+            lo = bnd[j];
+            hi = bnd[j + 1];
+        }
+        const int f = (j < N && hi > lo) ? 1 : 0;
+        int v = f;
+#pragma unroll
+        for (int off = 1; off < 32; off <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, v, off);
+            if (lane >= off) v += n;
+        }
+        if (lane == 31) wsum[warp] = v;
+        __syncthreads();
+        int wp = 0;
+        for (int w = 0; w < warp; ++w) wp += wsum[w];
+        if (f) ents[sr.s_eff + carry + wp + v - 1] = make_int2(sr.s_eff + lo, hi - lo);
+        if (tid == 511) carry_s = carry + wp + v;
+        __syncthreads();
+        carry = carry_s;
+        __syncthreads();
+    }
+    for (int i = tid; i < sr.w_eff; i += 512) ents[sr.s_eff + carry + i] = make_int2(sr.s_eff + M + i, 1);
+    if (tid == 0) a.lens[u] = sr.s_eff + carry + sr.w_eff;
+    if (a.user_bounds)
+        for (int j = tid; j <= N; j += 512) a.user_bounds[static_cast<int64_t>(u) * (a.Nmax + 1) + j] = bnd[j];
+}
+
+// ---------------------------------------------------------------------------
+// k_segment_reduce: one warp per entry
+// ---------------------------------------------------------------------------
+template <typename T>
+struct Vec16;   // 16 bytes of elements as fp32
+
+template <>
+struct Vec16<__nv_bfloat16> {
+    static constexpr int N = 8;
+    __device__ static void load(const void *p, float (&x)[8]) {
+        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p));
+        x[0] = bf16lo(w.x); x[1] = bf16hi(w.x); x[2] = bf16lo(w.y); x[3] = bf16hi(w.y);
+        x[4] = bf16lo(w.z); x[5] = bf16hi(w.z); x[6] = bf16lo(w.w); x[7] = bf16hi(w.w);
+    }
+    __device__ static void store(void *p, const float (&x)[8]) {
+        uint4 w;
+        w.x = pack_bf16x2(x[0], x[1]); w.y = pack_bf16x2(x[2], x[3]);
+        w.z = pack_bf16x2(x[4], x[5]); w.w = pack_bf16x2(x[6], x[7]);
+        *reinterpret_cast<uint4 *>(p) = w;
+    }
+};
+
+template <>
+struct Vec16<float> {
+    static constexpr int N = 4;
+    __device__ static void load(const void *p, float (&x)[4]) {
+        const float4 w = __ldg(reinterpret_cast<const float4 *>(p));
+        x[0] = w.x; x[1] = w.y; x[2] = w.z; x[3] = w.w;
+    }
+    __device__ static void store(void *p, const float (&x)[4]) {
+        *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+    }
+};
+
+constexpr int kK3Warps = 8;
+
+template <int D, typename T>
+__global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenArgs a) {
+    constexpr int ELEM = sizeof(T);
+    constexpr int ROWB = D * ELEM;        // bytes of one key row
+    constexpr int CH = ROWB / 16;         // 16-byte chunks per row = lanes per token
+    constexpr int TPS = 32 / CH;          // tokens per warp step
+    constexpr int EPL = 16 / ELEM;        // elements per lane
+    static_assert(CH >= 8 && CH <= 32, "row must span 8..32 chunks");
+
+    const int u = blockIdx.y;
+    const int b = u / a.Hkv, h = u % a.Hkv;
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int e = blockIdx.x * kK3Warps + warp;
+    const int n_ent = a.lens[u];
+    if (e >= n_ent) return;
+    const SeqRow sr = a.seq[b];
+    const int2 ent = a.ents[sr.ent_off + static_cast<int64_t>(h) * sr.emax + e];
+    const int start = ent.x, m = ent.y;
+    const int sub = lane / CH, ch = lane % CH;
+
+    const int64_t row0 = sr.row_off + static_cast<int64_t>(h) * sr.T + start;
+    const uint8_t *kp = static_cast<const uint8_t *>(a.k) + row0 * ROWB + ch * 16;
+    const uint8_t *vp = static_cast<const uint8_t *>(a.v) + row0 * ROWB + ch * 16;
+
+    float sk[EPL], sv[EPL], x[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) sk[i] = sv[i] = 0.0f;
+#pragma unroll 4
+    for (int t = sub; t < m; t += TPS) {
+        Vec16<T>::load(kp + static_cast<int64_t>(t) * ROWB, x);
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) sk[i] += x[i];
+        Vec16<T>::load(vp + static_cast<int64_t>(t) * ROWB, x);
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) sv[i] += x[i];
+    }
+#pragma unroll
+    for (int off = CH; off < 32; off <<= 1)
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], off);
+            sv[i] += __shfl_xor_sync(0xffffffffu, sv[i], off);
+        }
+    const float fm = static_cast<float>(m);
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        sk[i] = __fdiv_rn(sk[i], fm);   // mean key
+        sv[i] = __fdiv_rn(sv[i], fm);   // mean value
+    }
+    float q2[EPL];
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) q2[i] = 0.0f;
+#pragma unroll 4
+    for (int t = sub; t < m; t += TPS) {
+        Vec16<T>::load(kp + static_cast<int64_t>(t) * ROWB, x);
+#pragma unroll
+        for (int i = 0; i < EPL; ++i) {
+            const float dv = x[i] - sk[i];
+            q2[i] = __fmaf_rn(dv, dv, q2[i]);
+        }
+    }
+    float var_lane = 0.0f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        float qi = q2[i];
+#pragma unroll
+        for (int off = CH; off < 32; off <<= 1) qi += __shfl_xor_sync(0xffffffffu, qi, off);
+        var_lane += __fdiv_rn(qi, fm);   // population variance of dimension i
+    }
+#pragma unroll
+    for (int off = 1; off < CH; off <<= 1) var_lane += __shfl_xor_sync(0xffffffffu, var_lane, off);
+    const float sigma2 = var_lane / static_cast<float>(D);
+
+    const int32_t page = a.page_table[static_cast<int64_t>(u) * a.max_pages + e / kPageNodes];
+    const int slot = e % kPageNodes;
+    if (page < 0 || page >= a.num_pages) {
+        if (lane == 0) raise_flag(a.flags, FLAG_BAD_PAGE);
+        return;
+    }
+    if (sub == 0) {
+        const int64_t off = (static_cast<int64_t>(page) * kPageNodes + slot) * ROWB + swz(ch, slot) * 16;
+        Vec16<T>::store(a.pool_k + off, sk);
+        Vec16<T>::store(a.pool_v + off, sv);
+    }
+    if (lane == 0) {
+        const float alpha = m == 1 ? 0.0f : logf(fm);
+        a.pool_ab[static_cast<int64_t>(page) * kPageNodes + slot] = make_float2(alpha, sigma2 / (2.0f * D));
+    }
+}
+
+// ---------------------------------------------------------------------------
+// host launcher
+// ---------------------------------------------------------------------------
+template <int D, typename T>
+static cudaError_t launch_typed(const CoarsenArgs &a, const SeqTable &table, const ProjT &proj,
+                                const CUtensorMap &map_k, const CUtensorMap &map_v, cudaStream_t s) {
+    const int units = a.B * a.Hkv;
+    k_setup<<<1, 512, 0, s>>>(table, const_cast<SeqRow *>(a.seq), a.B, a.flags);
+    if (a.max_tiles > 0) {
+        constexpr size_t smem = k1_smem_bytes<D>();
+        cudaError_t e = cudaFuncSetAttribute(k_project_scan<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                             static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        k_project_scan<D, T><<<dim3(a.max_tiles, units), kK1Threads, smem, s>>>(a, map_k, map_v, proj);
+        k_tile_prefix<<<units, 256, 0, s>>>(a);
+        k_boundaries<<<dim3(a.max_tiles, units), 256, 0, s>>>(a);
+    }
+    k_plan_entries<<<units, 512, 0, s>>>(a);
+    if (a.max_emax > 0)
+        k_segment_reduce<D, T><<<dim3((a.max_emax + kK3Warps - 1) / kK3Warps, units), kK3Warps * 32, 0, s>>>(a);
+    return cudaGetLastError();
+}
+
+cudaError_t launch_coarsen(const CoarsenArgs &a, const SeqTable &table, const ProjT &proj,
+                           const CUtensorMap &map_k, const CUtensorMap &map_v, cudaStream_t s) {
+    if (a.dtype == SKV_BF16) {
+        if (a.d == 128) return launch_typed<128, __nv_bfloat16>(a, table, proj, map_k, map_v, s);
+        return launch_typed<64, __nv_bfloat16>(a, table, proj, map_k, map_v, s);
+    }
+    if (a.d == 128) return launch_typed<128, float>(a, table, proj, map_k, map_v, s);
+    return launch_typed<64, float>(a, table, proj, map_k, map_v, s);
+}
+
+}  // namespace skv

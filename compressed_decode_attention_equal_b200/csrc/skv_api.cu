@@ -1,0 +1,369 @@
+// C ABI of libskv (declared in include/skv.h): argument checks, the projection
+// generator, workspace plans, TMA descriptors and kernel launches. No entry
+// point allocates device memory; only skv_workspace_error synchronises.
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "skv_common.cuh"
+#include "skv_internal.h"
+
+using namespace skv;
+
+namespace {
+
+size_t align256(size_t x) { return (x + 255) & ~static_cast<size_t>(255); }
+
+bool aligned(const void *p, size_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+// ---------------------------------------------------------------------------
+// projection P (16 x 2d): SplitMix64 words -> Box-Muller (cosine branch) / 4
+// ---------------------------------------------------------------------------
+struct SplitMix64 {
+    uint64_t state;
+    uint64_t next() {
+        state += 0x9e3779b97f4a7c15ULL;
+        uint64_t z = state;
+        z = (z ^ (z >> 30)) * 0xbf58476d1ce4e5b9ULL;
+        z = (z ^ (z >> 27)) * 0x94d049bb133111ebULL;
+        return z ^ (z >> 31);
+    }
+};
+
+void make_projection(uint64_t seed, int d, float *P) {
+    const int cols = 2 * d;
+    const double two_pi = 6.283185307179586476925286766559;
+    const double scale = 1.0 / std::sqrt(static_cast<double>(kProjDim));
+    SplitMix64 g{seed};
+    for (int idx = 0; idx < kProjDim * cols; ++idx) {
+        const uint64_t w1 = g.next();
+        const uint64_t w2 = g.next();
+        const double u1 = static_cast<double>((w1 >> 11) + 1) * 0x1p-53;   // (0, 1]
+        const double u2 = static_cast<double>(w2 >> 11) * 0x1p-53;         // [0, 1)
+        const double gauss = std::sqrt(-2.0 * std::log(u1)) * std::cos(two_pi * u2);
+        P[idx] = static_cast<float>(gauss * scale);
+    }
+}
+
+// Small cache of transposed projections, keyed by (seed, d).
+struct ProjCache {
+    std::mutex mu;
+    struct Entry {
+        uint64_t seed;
+        int d;
+        ProjT pt;
+    };
+    std::vector<Entry> entries;
+    void get(uint64_t seed, int d, ProjT &out) {
+        std::lock_guard<std::mutex> lock(mu);
+        for (auto &e : entries)
+            if (e.seed == seed && e.d == d) {
+                out = e.pt;
+                return;
+            }
+        std::vector<float> P(static_cast<size_t>(kProjDim) * 2 * d);
+        make_projection(seed, d, P.data());
+        Entry e;
+        e.seed = seed;
+        e.d = d;
+        std::memset(&e.pt, 0, sizeof e.pt);
+        for (int i = 0; i < kProjDim; ++i)
+            for (int j = 0; j < 2 * d; ++j) e.pt.pt[j * kProjDim + i] = P[static_cast<size_t>(i) * 2 * d + j];
+        if (entries.size() >= 16) entries.erase(entries.begin());
+        entries.push_back(e);
+        out = e.pt;
+    }
+};
+ProjCache g_proj;
+
+// ---------------------------------------------------------------------------
+// driver entry point for TMA descriptors (resolved once through the runtime)
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *, const cuuint64_t *,
+                                  const cuuint64_t *, const cuuint32_t *, const cuuint32_t *, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+    static EncodeTiledFn fn = nullptr;
+    static std::once_flag once;
+    std::call_once(once, [] {
+        void *p = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<EncodeTiledFn>(p);
+    });
+    return fn;
+}
+
+// Rows x d matrix of raw keys or values; boxes of 256 rows x 128 bytes, 128-byte swizzle.
+bool make_row_map(CUtensorMap *map, const void *base, int dtype, int d, int64_t rows) {
+    EncodeTiledFn fn = encode_fn();
+    if (!fn) return false;
+    const int elem = dtype == SKV_BF16 ? 2 : 4;
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * elem};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem), static_cast<cuuint32_t>(kTileRows)};
+    cuuint32_t estr[2] = {1, 1};
+    const CUresult r = fn(map, dtype == SKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
+                          const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    return r == CUDA_SUCCESS;
+}
+
+// ---------------------------------------------------------------------------
+// coarsening plan
+// ---------------------------------------------------------------------------
+struct CoarsenPlan {
+    int max_tiles = 0, max_emax = 0, Nmax = 0;
+    int64_t rows = 0, mid = 0, bnd = 0, ent = 0;
+    CoarsenLayout lay{};
+};
+
+skv_status plan_coarsen(int B, int Hkv, int d, const int32_t *T_host, const int32_t *N_host, int n_sink,
+                        int n_recent, SeqTable *table, CoarsenPlan *plan) {
+    if (B < 1 || B > SKV_MAX_SEQS || Hkv < 1 || !T_host || !N_host || n_sink < 0 || n_recent < 0)
+        return SKV_ERR_INVALID_ARG;
+    if (static_cast<int64_t>(B) * Hkv > 65535) return SKV_ERR_UNSUPPORTED;
+    if (d != 64 && d != 128) return SKV_ERR_UNSUPPORTED;
+    CoarsenPlan p;
+    for (int b = 0; b < B; ++b) {
+        const int T = T_host[b], N = N_host[b];
+        if (T < 0 || T > SKV_MAX_TOKENS || N < 1 || N > (1 << 20)) return SKV_ERR_INVALID_ARG;
+        SeqRow r{};
+        r.T = T;
+        r.N = N;
+        r.s_eff = n_sink < T ? n_sink : T;
+        r.w_eff = n_recent < T - r.s_eff ? n_recent : T - r.s_eff;
+        r.M = T - r.s_eff - r.w_eff;
+        r.tiles = (r.M + kTileOut - 1) / kTileOut;
+        r.emax = r.s_eff + (r.M > 0 ? N : 0) + r.w_eff;
+        r.row_off = p.rows;
+        r.mid_off = p.mid;
+        if (p.bnd > INT32_MAX - static_cast<int64_t>(Hkv) * (N + 1) ||
+            p.ent > INT32_MAX - static_cast<int64_t>(Hkv) * r.emax)
+            return SKV_ERR_UNSUPPORTED;
+        r.bnd_off = static_cast<int32_t>(p.bnd);
+        r.ent_off = static_cast<int32_t>(p.ent);
+        p.rows += static_cast<int64_t>(Hkv) * T;
+        p.mid += static_cast<int64_t>(Hkv) * r.M;
+        p.bnd += static_cast<int64_t>(Hkv) * (N + 1);
+        p.ent += static_cast<int64_t>(Hkv) * r.emax;
+        if (r.tiles > p.max_tiles) p.max_tiles = r.tiles;
+        if (r.emax > p.max_emax) p.max_emax = r.emax;
+        if (N > p.Nmax) p.Nmax = N;
+        if (table) table->rows[b] = r;
+    }
+    if (p.rows > INT32_MAX) return SKV_ERR_UNSUPPORTED;   // TMA row coordinates are int32
+    const int64_t units = static_cast<int64_t>(B) * Hkv;
+    size_t off = kWsHeader;
+    p.lay.seq = off;
+    off += align256(sizeof(SeqRow) * B);
+    p.lay.tile_total = off;
+    off += align256(static_cast<size_t>(units) * p.max_tiles * 8);
+    p.lay.tile_prefix = off;
+    off += align256(static_cast<size_t>(units) * p.max_tiles * 8);
+    p.lay.unit_total = off;
+    off += align256(static_cast<size_t>(units) * 8);
+    p.lay.local_scan = off;
+    off += align256(static_cast<size_t>(p.mid) * 8);
+    p.lay.bounds = off;
+    off += align256(static_cast<size_t>(p.bnd) * 4);
+    p.lay.ents = off;
+    off += align256(static_cast<size_t>(p.ent) * 8);
+    p.lay.total = off;
+    *plan = p;
+    return SKV_OK;
+}
+
+// ---------------------------------------------------------------------------
+// decode plan
+// ---------------------------------------------------------------------------
+struct DecodePlan {
+    int rows, row_passes, pass_rows, n_vunits;
+    DecodeLayout lay;
+};
+
+skv_status plan_decode(int dtype, int B, int R, int Hq, int Hkv, int d, int max_pages, DecodePlan *plan) {
+    if (B < 1 || R < 1 || Hq < 1 || Hkv < 1 || max_pages < 1) return SKV_ERR_INVALID_ARG;
+    if (Hq % Hkv != 0 || (d != 64 && d != 128) || (dtype != SKV_BF16 && dtype != SKV_F32))
+        return SKV_ERR_UNSUPPORTED;
+    if (static_cast<int64_t>(max_pages) * kPageNodes > INT32_MAX / 2) return SKV_ERR_UNSUPPORTED;
+    DecodePlan p{};
+    const int64_t rows = static_cast<int64_t>(R) * (Hq / Hkv);
+    if (rows > (1 << 20)) return SKV_ERR_UNSUPPORTED;
+    p.rows = static_cast<int>(rows);
+    p.row_passes = (p.rows + kRowsPerPass - 1) / kRowsPerPass;
+    p.pass_rows = p.rows > kRowsPerPass ? kRowsPerPass : ((p.rows + 7) / 8) * 8;
+    const int64_t nv = static_cast<int64_t>(B) * Hkv * p.row_passes;
+    if (nv > kMaxVUnits) return SKV_ERR_UNSUPPORTED;
+    // the page prefix is an int32 sum over all units
+    if (static_cast<int64_t>(B) * Hkv * max_pages * p.row_passes > INT32_MAX / 2) return SKV_ERR_UNSUPPORTED;
+    p.n_vunits = static_cast<int>(nv);
+    size_t off = kWsHeader;
+    p.lay.vu_prefix = off;
+    off += align256(static_cast<size_t>(nv + 1) * 4);
+    p.lay.part = off;
+    if (dtype == SKV_BF16) off += align256(static_cast<size_t>(kMaxDecodeCtas) * 2 * p.pass_rows * (d + 1) * 4);
+    p.lay.total = off;
+    *plan = p;
+    return SKV_OK;
+}
+
+}  // namespace
+
+// ===========================================================================
+extern "C" {
+
+const char *skv_status_string(int status) {
+    switch (status) {
+        case SKV_OK: return "SKV_OK";
+        case SKV_ERR_INVALID_ARG: return "SKV_ERR_INVALID_ARG: invalid argument";
+        case SKV_ERR_UNSUPPORTED: return "SKV_ERR_UNSUPPORTED: configuration not supported";
+        case SKV_ERR_CUDA: return "SKV_ERR_CUDA: CUDA runtime error";
+        case SKV_ERR_OVERFLOW: return "SKV_ERR_OVERFLOW: variation step above 2^20 (or not finite)";
+        case SKV_ERR_WORKSPACE: return "SKV_ERR_WORKSPACE: workspace too small or misaligned";
+        case SKV_ERR_DEVICE: return "SKV_ERR_DEVICE: device detected a bad page id, lens entry or stuck wait";
+        default: return "unknown skv status";
+    }
+}
+
+int skv_abi_version(void) { return 100; }
+
+skv_status skv_projection_matrix(uint64_t proj_seed, int d, float *P_host) {
+    if (!P_host || (d != 64 && d != 128)) return SKV_ERR_INVALID_ARG;
+    make_projection(proj_seed, d, P_host);
+    return SKV_OK;
+}
+
+size_t skv_coarsen_workspace_bytes(int B, int Hkv, int d, const int32_t *T_host, const int32_t *N_host, int n_sink,
+                                   int n_recent) {
+    CoarsenPlan p;
+    if (plan_coarsen(B, Hkv, d, T_host, N_host, n_sink, n_recent, nullptr, &p) != SKV_OK) return 0;
+    return p.lay.total;
+}
+
+skv_status skv_coarsen(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d, const int32_t *T_host,
+                       int n_sink, int n_recent, const int32_t *N_host, uint64_t proj_seed,
+                       const skv_node_pool *pool, const int32_t *page_table, int max_pages, int32_t *lens,
+                       int32_t *boundaries, int64_t *cumvar, void *workspace, size_t ws_bytes, void *stream) {
+    if (dtype != SKV_BF16 && dtype != SKV_F32) return SKV_ERR_UNSUPPORTED;
+    static SeqTable table;   // host staging; guarded by the mutex below
+    static std::mutex table_mu;
+    std::lock_guard<std::mutex> lock(table_mu);
+    CoarsenPlan plan;
+    skv_status st = plan_coarsen(B, Hkv, d, T_host, N_host, n_sink, n_recent, &table, &plan);
+    if (st != SKV_OK) return st;
+    if (!pool || !page_table || !lens || max_pages < 1) return SKV_ERR_INVALID_ARG;
+    if (!pool->k || !pool->v || !pool->ab || pool->num_pages < 0) return SKV_ERR_INVALID_ARG;
+    if (!aligned(pool->k, 16) || !aligned(pool->v, 16) || !aligned(pool->ab, 16)) return SKV_ERR_INVALID_ARG;
+    if (plan.rows > 0 && (!k || !v || !aligned(k, 16) || !aligned(v, 16))) return SKV_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < plan.lay.total) return SKV_ERR_WORKSPACE;
+    for (int b = 0; b < B; ++b)
+        if (table.rows[b].emax > static_cast<int64_t>(max_pages) * kPageNodes) return SKV_ERR_INVALID_ARG;
+
+    ProjT proj;
+    g_proj.get(proj_seed, d, proj);
+    CUtensorMap map_k, map_v;
+    std::memset(&map_k, 0, sizeof map_k);
+    std::memset(&map_v, 0, sizeof map_v);
+    if (plan.max_tiles > 0) {
+        if (!make_row_map(&map_k, k, dtype, d, plan.rows) || !make_row_map(&map_v, v, dtype, d, plan.rows))
+            return SKV_ERR_CUDA;
+    }
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    CoarsenArgs a{};
+    a.k = k;
+    a.v = v;
+    a.B = B;
+    a.Hkv = Hkv;
+    a.d = d;
+    a.dtype = dtype;
+    a.max_tiles = plan.max_tiles;
+    a.max_emax = plan.max_emax;
+    a.Nmax = plan.Nmax;
+    a.seq = reinterpret_cast<const SeqRow *>(ws + plan.lay.seq);
+    a.tile_total = reinterpret_cast<int64_t *>(ws + plan.lay.tile_total);
+    a.tile_prefix = reinterpret_cast<int64_t *>(ws + plan.lay.tile_prefix);
+    a.unit_total = reinterpret_cast<int64_t *>(ws + plan.lay.unit_total);
+    a.local_scan = reinterpret_cast<int64_t *>(ws + plan.lay.local_scan);
+    a.bounds = reinterpret_cast<int32_t *>(ws + plan.lay.bounds);
+    a.ents = reinterpret_cast<int2 *>(ws + plan.lay.ents);
+    a.flags = reinterpret_cast<uint32_t *>(ws);
+    a.pool_k = static_cast<uint8_t *>(pool->k);
+    a.pool_v = static_cast<uint8_t *>(pool->v);
+    a.pool_ab = reinterpret_cast<float2 *>(pool->ab);
+    a.num_pages = pool->num_pages;
+    a.page_table = page_table;
+    a.max_pages = max_pages;
+    a.lens = lens;
+    a.user_bounds = boundaries;
+    a.cumvar = cumvar;
+    const cudaError_t e = launch_coarsen(a, table, proj, map_k, map_v, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SKV_OK : SKV_ERR_CUDA;
+}
+
+size_t skv_decode_workspace_bytes(int B, int R, int Hq, int Hkv, int d, int max_pages) {
+    DecodePlan p;
+    if (plan_decode(SKV_BF16, B, R, Hq, Hkv, d, max_pages, &p) != SKV_OK) return 0;
+    return p.lay.total;
+}
+
+skv_status skv_decode_attn(const void *q, skv_dtype dtype, int B, int R, int Hq, int Hkv, int d,
+                           const skv_node_pool *pool, const int32_t *page_table, int max_pages, const int32_t *lens,
+                           void *out, float *lse, void *workspace, size_t ws_bytes, void *stream) {
+    DecodePlan plan;
+    skv_status st = plan_decode(dtype, B, R, Hq, Hkv, d, max_pages, &plan);
+    if (st != SKV_OK) return st;
+    if (!q || !out || !lse || !pool || !page_table || !lens) return SKV_ERR_INVALID_ARG;
+    if (!pool->k || !pool->v || !pool->ab || pool->num_pages < 0) return SKV_ERR_INVALID_ARG;
+    if (!aligned(pool->k, 16) || !aligned(pool->v, 16) || !aligned(pool->ab, 16) || !aligned(q, 16) ||
+        !aligned(out, 16) || !aligned(lse, 4))
+        return SKV_ERR_INVALID_ARG;
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < plan.lay.total) return SKV_ERR_WORKSPACE;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    DecodeArgs a{};
+    a.q = q;
+    a.pool_k = static_cast<const uint8_t *>(pool->k);
+    a.pool_v = static_cast<const uint8_t *>(pool->v);
+    a.pool_ab = reinterpret_cast<const float2 *>(pool->ab);
+    a.num_pages = pool->num_pages;
+    a.page_table = page_table;
+    a.max_pages = max_pages;
+    a.lens = lens;
+    a.out = out;
+    a.lse = lse;
+    a.B = B;
+    a.R = R;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.G = Hq / Hkv;
+    a.d = d;
+    a.dtype = dtype;
+    a.rows = plan.rows;
+    a.row_passes = plan.row_passes;
+    a.pass_rows = plan.pass_rows;
+    a.n_vunits = plan.n_vunits;
+    a.part = reinterpret_cast<float *>(ws + plan.lay.part);
+    a.vu_prefix = reinterpret_cast<int32_t *>(ws + plan.lay.vu_prefix);
+    a.flags = reinterpret_cast<uint32_t *>(ws);
+    const cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream));
+    return e == cudaSuccess ? SKV_OK : SKV_ERR_CUDA;
+}
+
+skv_status skv_workspace_error(const void *workspace, void *stream, uint32_t *flags_host) {
+    if (!workspace) return SKV_ERR_INVALID_ARG;
+    cudaStream_t s = static_cast<cudaStream_t>(stream);
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SKV_ERR_CUDA;
+    uint32_t f = 0;
+    if (cudaMemcpy(&f, workspace, sizeof f, cudaMemcpyDeviceToHost) != cudaSuccess) return SKV_ERR_CUDA;
+    if (cudaMemset(const_cast<void *>(workspace), 0, sizeof f) != cudaSuccess) return SKV_ERR_CUDA;
+    if (flags_host) *flags_host = f;
+    if (f & FLAG_OVERFLOW) return SKV_ERR_OVERFLOW;
+    if (f) return SKV_ERR_DEVICE;
+    return SKV_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,106 @@
+// Internal declarations shared by the C-ABI host code and the kernels.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include "skv.h"
+
+namespace skv {
+
+// ---------------------------------------------------------------------------
+// coarsening
+// ---------------------------------------------------------------------------
+constexpr int kTileRows = 256;              // rows a projection tile computes (1 halo + outputs)
+constexpr int kTileOut = kTileRows - 1;     // middle tokens per projection tile
+
+// Per-sequence plan, computed on the host and copied into the workspace.
+struct SeqRow {
+    int64_t row_off;   // first row of the sequence in the packed [rows][d] view of k / v
+    int64_t mid_off;   // first index of the sequence in the per-middle-token scratch arrays
+    int32_t T, N;      // tokens, middle segments
+    int32_t s_eff, w_eff, M;
+    int32_t tiles;     // projection tiles per head: ceil(M / kTileOut)
+    int32_t bnd_off;   // first index of the sequence in the boundary scratch (Hkv * (N + 1) each)
+    int32_t ent_off;   // first index of the sequence in the entry scratch (Hkv * emax each)
+    int32_t emax;      // entries a head can produce: s_eff + (M > 0 ? N : 0) + w_eff
+    int32_t pad;
+};
+static_assert(sizeof(SeqRow) == 56, "SeqRow layout");
+
+struct SeqTable {
+    SeqRow rows[SKV_MAX_SEQS];
+};
+
+// Projection transposed for the kernels: pt[j][i] = P[i][j], j < 2d, i < 16.
+struct ProjT {
+    float pt[2 * 128 * SKV_PROJ_DIM];
+};
+
+struct CoarsenArgs {
+    const void *k, *v;
+    int B, Hkv, d, dtype;
+    int max_tiles;   // largest tiles per head over the batch
+    int max_emax;    // largest emax over the batch
+    int Nmax;        // largest N over the batch
+    const SeqRow *seq;
+    int64_t *tile_total, *tile_prefix, *unit_total, *local_scan;
+    int32_t *bounds;
+    int2 *ents;
+    uint32_t *flags;
+    uint8_t *pool_k, *pool_v;
+    float2 *pool_ab;
+    int64_t num_pages;
+    const int32_t *page_table;
+    int max_pages;
+    int32_t *lens;
+    int32_t *user_bounds;
+    int64_t *cumvar;
+};
+
+// Workspace carve-up (offsets in bytes from the workspace start).
+struct CoarsenLayout {
+    size_t seq, tile_total, tile_prefix, unit_total, local_scan, bounds, ents, total;
+};
+
+// Host-side launchers (coarsen.cu).
+cudaError_t launch_coarsen(const CoarsenArgs &a, const SeqTable &table, const ProjT &proj,
+                           const CUtensorMap &map_k, const CUtensorMap &map_v, cudaStream_t s);
+
+// ---------------------------------------------------------------------------
+// decode
+// ---------------------------------------------------------------------------
+constexpr int kRowsPerPass = 32;    // query rows one pass over a unit's pages serves
+constexpr int kMaxDecodeCtas = 1024;
+constexpr int kMaxVUnits = 8192;
+
+struct DecodeArgs {
+    const void *q;
+    const uint8_t *pool_k, *pool_v;
+    const float2 *pool_ab;
+    int64_t num_pages;
+    const int32_t *page_table;
+    int max_pages;
+    const int32_t *lens;
+    void *out;
+    float *lse;
+    int B, R, Hq, Hkv, G, d, dtype;
+    int rows;         // R * G query rows per unit
+    int row_passes;   // ceil(rows / kRowsPerPass)
+    int pass_rows;    // rows a pass holds: min(kRowsPerPass, rows rounded up to 8)
+    int n_vunits;     // B * Hkv * row_passes
+    int ncta;         // CTAs of the split kernel
+    float *part;      // [ncta][2][pass_rows][d + 1] split partials
+    int32_t *vu_prefix;  // [n_vunits + 1] page prefix over virtual units
+    uint32_t *flags;
+};
+
+struct DecodeLayout {
+    size_t vu_prefix, part, total;
+};
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+
+}  // namespace skv

@@ -1,0 +1,130 @@
+"""Helpers shared by the GPU parity tests: pool / page-table set-up, writing synthetic
+entries into the pool layout, reading GPU nodes back for the oracle, and the
+tolerance checks the parity bar fixes:
+  fp32: relative L2 <= 1e-5;
+  bf16: relative L2 <= 5e-3 and max-abs <= 2e-2 on outputs, |lse error| <= 1e-3.
+"""
+from __future__ import annotations
+
+import math
+
+import numpy as np
+import torch
+
+import compressed_decode_attention_equal_b200 as skv
+import workloads
+
+TOL_F32_REL_L2 = 1e-5
+TOL_BF16_REL_L2 = 5e-3
+TOL_BF16_MAX_ABS = 2e-2
+TOL_LSE_ABS = 1e-3
+
+
+def pool_for_units(entries_per_unit, B, Hkv, d, dtype, shuffle=False, seed=0, spare_pages=0, device="cuda"):
+    """Pool and page table with ceil(E/16) pages for each unit (entries_per_unit[b] per head)."""
+    pages = [max(1, -(-int(e) // skv.PAGE_NODES)) for e in entries_per_unit]
+    table, total = workloads.page_assignment(B, Hkv, pages, shuffle, seed)
+    pool = skv.NodePool(total + spare_pages, d, dtype, device=device)
+    pool.k.zero_()
+    pool.v.zero_()
+    pool.ab.zero_()
+    return pool, table.to(device)
+
+
+def write_entries(pool, table, b, h, kt, vt, alpha, beta):
+    """Write entries of unit (b, h) into the pool's swizzled page layout (inverse of read_entries)."""
+    E, d = kt.shape
+    if E == 0:
+        return
+    dev = pool.k.device
+    n_pages = -(-E // skv.PAGE_NODES)
+    pages = table[b, h, :n_pages].long()
+    rows = (pages[:, None] * skv.PAGE_NODES + torch.arange(skv.PAGE_NODES, device=dev)).reshape(-1)[:E]
+    epc = 16 // pool.k.element_size()
+    ch = d // epc
+    slot = torch.arange(E, device=dev) % skv.PAGE_NODES
+    phys = torch.arange(ch, device=dev)[None, :] ^ (slot[:, None] & 7)
+    kflat = pool.k.view(-1, ch, epc)
+    vflat = pool.v.view(-1, ch, epc)
+    ridx = rows[:, None].expand(E, ch)
+    kflat[ridx, phys] = kt.to(pool.dtype).reshape(E, ch, epc).to(dev)
+    vflat[ridx, phys] = vt.to(pool.dtype).reshape(E, ch, epc).to(dev)
+    abflat = pool.ab.view(-1, 2)
+    abflat[rows, 0] = alpha.float().to(dev)
+    abflat[rows, 1] = beta.float().to(dev)
+
+
+class GpuUnit:
+    """A unit's GPU-stored entries as fp64 numpy arrays (attribute names the oracle expects)."""
+
+    def __init__(self, kt, vt, alpha, beta):
+        self.kt, self.vt, self.alpha, self.beta = kt, vt, alpha, beta
+
+
+def gpu_units(pool, table, lens, B, Hkv):
+    out = []
+    for b in range(B):
+        row = []
+        for h in range(Hkv):
+            kt, vt, al, be = skv.read_entries(pool, table, lens, b, h)
+            row.append(GpuUnit(kt.double().cpu().numpy(), vt.double().cpu().numpy(), al.double().cpu().numpy(),
+                               be.double().cpu().numpy()))
+        out.append(row)
+    return out
+
+
+def rel_l2(a, b):
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    den = np.linalg.norm(b)
+    return float(np.linalg.norm(a - b) / (den if den > 0 else 1.0))
+
+
+def check_decode(out_gpu, lse_gpu, out_ref, lse_ref, dtype, what=""):
+    og = out_gpu.double().cpu().numpy() if isinstance(out_gpu, torch.Tensor) else np.asarray(out_gpu)
+    lg = lse_gpu.double().cpu().numpy() if isinstance(lse_gpu, torch.Tensor) else np.asarray(lse_gpu)
+    inf_ref = np.isneginf(lse_ref)
+    assert np.array_equal(np.isneginf(lg), inf_ref), f"{what}: empty-unit pattern differs"
+    fin = ~inf_ref
+    if dtype == torch.float32:
+        assert rel_l2(og, out_ref) <= TOL_F32_REL_L2, f"{what}: out rel-L2 {rel_l2(og, out_ref):.3e}"
+        assert rel_l2(lg[fin], lse_ref[fin]) <= TOL_F32_REL_L2, f"{what}: lse rel-L2"
+    else:
+        r = rel_l2(og, out_ref)
+        m = float(np.abs(og - out_ref).max()) if og.size else 0.0
+        assert r <= TOL_BF16_REL_L2, f"{what}: out rel-L2 {r:.3e}"
+        assert m <= TOL_BF16_MAX_ABS, f"{what}: out max-abs {m:.3e}"
+        if fin.any():
+            le = float(np.abs(lg[fin] - lse_ref[fin]).max())
+            assert le <= TOL_LSE_ABS, f"{what}: lse max-abs {le:.3e}"
+    assert np.all(og[inf_ref] == 0), f"{what}: empty units must give zero output"
+
+
+def bf16_ulp(x):
+    ax = np.abs(np.asarray(x, np.float64))
+    e = np.floor(np.log2(np.maximum(ax, 1e-38)))
+    return np.exp2(e - 7)
+
+
+def check_nodes(gpu_unit, orc_unit, dtype, d, what=""):
+    """Node statistics of one unit: GPU (stored) vs oracle fp64."""
+    assert gpu_unit.kt.shape == orc_unit.kt.shape, f"{what}: entry count"
+    al_err = np.abs(gpu_unit.alpha - orc_unit.alpha)
+    assert np.all(al_err <= 1e-6 * np.maximum(1.0, np.abs(orc_unit.alpha))), f"{what}: alpha"
+    be_ref = orc_unit.beta
+    be_err = np.abs(gpu_unit.beta - be_ref)
+    assert np.all(be_err <= 1e-5 * np.abs(be_ref) + 1e-12), f"{what}: beta max rel {np.max(be_err / (be_ref + 1e-30)):.2e}"
+    for name in ("kt", "vt"):
+        g, o = getattr(gpu_unit, name), getattr(orc_unit, name)
+        if dtype == torch.float32:
+            assert rel_l2(g, o) <= TOL_F32_REL_L2, f"{what}: {name} rel-L2 {rel_l2(g, o):.2e}"
+        else:
+            # the fp32 mean rounded once to bf16: within half an ulp of the fp64 mean, plus fp32 error
+            err = np.abs(g - o)
+            bound = 0.5 * bf16_ulp(o) + 1e-6 * np.abs(o) + 1e-30
+            assert np.all(err <= bound), f"{what}: {name} worst excess {np.max(err / bound):.3f}"
+            assert rel_l2(g, o) <= TOL_BF16_REL_L2
+
+
+def to_np32(t: torch.Tensor) -> np.ndarray:
+    return t.float().cpu().numpy()

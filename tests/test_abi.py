@@ -1,0 +1,97 @@
+"""The C-ABI library loads, exports every symbol include/skv.h declares, and rejects bad
+arguments on the host before touching the GPU (not gpu: no compute calls)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from compressed_decode_attention_equal_b200 import build, _lib
+    build.build()
+    return _lib.load()
+
+
+def _declared():
+    src = open(os.path.join(ROOT, "include", "skv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(skv_[a-z_]+)\s*\(", src)))
+
+
+def test_header_declares_the_binding_exports():
+    from compressed_decode_attention_equal_b200 import _lib
+    assert sorted(_lib.EXPORTS) == _declared()
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared():
+        assert hasattr(lib, name), name
+
+
+def test_status_strings(lib):
+    for code in (0, -1, -2, -3, -4, -6, -7):
+        s = lib.skv_status_string(code).decode()
+        assert s.startswith("SKV_")
+    assert "unknown" in lib.skv_status_string(12345).decode()
+    assert lib.skv_abi_version() == 100
+
+
+def test_workspace_queries_are_host_arithmetic(lib):
+    from compressed_decode_attention_equal_b200 import coarsen_workspace_bytes, decode_workspace_bytes
+    a = coarsen_workspace_bytes(4, 128, [32768] * 32, [1091] * 32, 8, 48)
+    b = coarsen_workspace_bytes(4, 128, [32768] * 33, [1091] * 33, 8, 48)
+    assert 0 < a < b
+    assert coarsen_workspace_bytes(4, 96, [100], [4], 8, 48) == 0         # d unsupported
+    assert coarsen_workspace_bytes(4, 128, [100], [0], 8, 48) == 0        # N < 1
+    assert coarsen_workspace_bytes(4, 128, [1 << 22], [4], 8, 48) == 0    # too many tokens
+    assert decode_workspace_bytes(32, 1, 28, 4, 128, 72) > 0
+    assert decode_workspace_bytes(32, 1, 28, 5, 128, 72) == 0             # Hq % Hkv != 0
+    assert decode_workspace_bytes(32, 1, 28, 4, 80, 72) == 0              # d unsupported
+
+
+def test_bad_arguments_rejected_before_any_launch(lib):
+    from compressed_decode_attention_equal_b200 import _lib
+    null = ctypes.c_void_p(0)
+    pool = _lib.SkvNodePool(0, 0, 0, 0)
+    st = lib.skv_decode_attn(null, 1, 1, 1, 7, 1, 128, ctypes.byref(pool), null, 4, null, null, null, null, 0, null)
+    assert st == _lib.SKV_ERR_INVALID_ARG
+    st = lib.skv_decode_attn(null, 1, 1, 1, 7, 2, 128, ctypes.byref(pool), null, 4, null, null, null, null, 0, null)
+    assert st == _lib.SKV_ERR_UNSUPPORTED
+    st = lib.skv_decode_attn(null, 7, 1, 1, 7, 1, 128, ctypes.byref(pool), null, 4, null, null, null, null, 0, null)
+    assert st == _lib.SKV_ERR_UNSUPPORTED
+    T = (ctypes.c_int32 * 1)(100)
+    N = (ctypes.c_int32 * 1)(4)
+    st = lib.skv_coarsen(null, null, 1, 1, 1, 128, T, 8, 48, N, 0, None, null, 4, null, null, null, null, 0, null)
+    assert st == _lib.SKV_ERR_INVALID_ARG
+    st = lib.skv_coarsen(null, null, 3, 1, 1, 128, T, 8, 48, N, 0, None, null, 4, null, null, null, null, 0, null)
+    assert st == _lib.SKV_ERR_UNSUPPORTED
+    Tbad = (ctypes.c_int32 * 1)(-1)
+    pool2 = _lib.SkvNodePool(16, 16, 16, 1)
+    st = lib.skv_coarsen(null, null, 1, 1, 1, 128, Tbad, 8, 48, N, 0, ctypes.byref(pool2), ctypes.c_void_p(16), 4,
+                         ctypes.c_void_p(16), null, null, null, 0, null)
+    assert st == _lib.SKV_ERR_INVALID_ARG
+    # workspace too small is reported before any launch
+    st = lib.skv_coarsen(ctypes.c_void_p(256), ctypes.c_void_p(256), 1, 1, 1, 128, T, 8, 48, N, 0,
+                         ctypes.byref(pool2), ctypes.c_void_p(16), 4, ctypes.c_void_p(16), null, null,
+                         ctypes.c_void_p(256), 16, null)
+    assert st == _lib.SKV_ERR_WORKSPACE
+    # page capacity: 8 + 4 + 48 = 60 entries need 4 pages of 16
+    st = lib.skv_coarsen(ctypes.c_void_p(256), ctypes.c_void_p(256), 1, 1, 1, 128, T, 8, 48, N, 0,
+                         ctypes.byref(pool2), ctypes.c_void_p(16), 3, ctypes.c_void_p(16), null, null,
+                         ctypes.c_void_p(256), 1 << 30, null)
+    assert st == _lib.SKV_ERR_INVALID_ARG
+
+
+def test_binding_fails_loudly_without_library(tmp_path):
+    from compressed_decode_attention_equal_b200 import _lib
+    saved = _lib._lib
+    try:
+        _lib._lib = None
+        with pytest.raises(OSError):
+            _lib.load(str(tmp_path / "missing.so"))
+    finally:
+        _lib._lib = saved

@@ -1,0 +1,183 @@
+"""GPU parity of equal-variation coarsening against the oracle.
+
+Bit-exact: the projection P, every unit's cumulative quantised variation c_t, the segment
+boundaries, the entry counts. Within tolerance: node statistics (mean key / value, alpha = ln m,
+beta = sigma^2 / (2d)). Sizes span several projection tiles (255 tokens each) with ragged tails,
+plus the degenerate cases: T <= n_sink + n_recent, empty middle, M < N (empty segments dropped),
+constant middle (c_T = 0), N = 1, one jump crossing many thresholds, d = 64 / 128, fp32 / bf16."""
+import numpy as np
+import pytest
+import torch
+
+import compressed_decode_attention_equal_b200 as skv
+import oracle
+import workloads
+from gpu_helpers import check_decode, check_nodes, gpu_units, pool_for_units, to_np32
+
+pytestmark = pytest.mark.gpu
+
+S, W = workloads.N_SINK, workloads.N_RECENT
+
+
+def run_coarsen(k, v, Hkv, T_list, N_list, seed, n_sink=S, n_recent=W, shuffle=True):
+    B = len(T_list)
+    d = k.shape[-1]
+    ent = [skv.entries_bound(T, N, n_sink, n_recent) for T, N in zip(T_list, N_list)]
+    pool, table = pool_for_units(ent, B, Hkv, d, k.dtype, shuffle=shuffle, seed=seed)
+    Nmax = max(N_list)
+    bnd = torch.full((B, Hkv, Nmax + 1), -7, dtype=torch.int32, device="cuda")
+    cum = torch.full((k.shape[0],), -7, dtype=torch.int64, device="cuda")
+    ws = torch.zeros(skv.coarsen_workspace_bytes(Hkv, d, T_list, N_list, n_sink, n_recent), dtype=torch.uint8,
+                     device="cuda")
+    lens = skv.coarsen(k, v, Hkv, T_list, N_list, n_sink, n_recent, seed, pool, table, boundaries=bnd, cumvar=cum,
+                       workspace=ws)
+    st, flags = skv.workspace_error(ws)
+    return dict(pool=pool, table=table, lens=lens, bnd=bnd, cum=cum, status=st, flags=flags)
+
+
+def oracle_units(k, v, Hkv, T_list, N_list, seed, units=None, n_sink=S, n_recent=W):
+    d = k.shape[-1]
+    P = oracle.projection(seed, d)
+    res = {}
+    for b, T in enumerate(T_list):
+        for h in range(Hkv):
+            if units is not None and (b, h) not in units:
+                continue
+            kk = to_np32(workloads.unit_rows(k, T_list, Hkv, b, h))
+            vv = to_np32(workloads.unit_rows(v, T_list, Hkv, b, h))
+            res[(b, h)] = oracle.coarsen_unit(kk, vv, n_sink, n_recent, int(N_list[b]), P)
+    return res
+
+
+def compare_units(r, orc, k, T_list, Hkv, N_list, dtype):
+    d = k.shape[-1]
+    for (b, h), u in orc.items():
+        what = f"unit ({b},{h}) T={T_list[b]} N={N_list[b]}"
+        # cumulative variation, bit for bit
+        off = sum(T_list[:b]) * Hkv + h * T_list[b]
+        cg = r["cum"][off:off + u.M].cpu().numpy()
+        assert np.array_equal(cg, u.C), f"{what}: c_t differs at {np.flatnonzero(cg != u.C)[:5]}"
+        # boundaries and entry counts, bit for bit
+        bg = r["bnd"][b, h, :N_list[b] + 1].cpu().numpy()
+        assert np.array_equal(bg, u.bounds), f"{what}: boundaries differ"
+        assert int(r["lens"][b, h]) == u.kt.shape[0], f"{what}: lens"
+        kt, vt, al, be = skv.read_entries(r["pool"], r["table"], r["lens"], b, h)
+
+        class G:
+            pass
+
+        gu = G()
+        gu.kt, gu.vt = kt.double().cpu().numpy(), vt.double().cpu().numpy()
+        gu.alpha, gu.beta = al.double().cpu().numpy(), be.double().cpu().numpy()
+        check_nodes(gu, u, dtype, d, what)
+
+
+def test_projection_matches_oracle_bitwise():
+    for seed in (0, 1, 2, 3, 4, 12345678901234):
+        for d in (64, 128):
+            a = skv.projection_matrix(seed, d).numpy()
+            b = oracle.projection(seed, d)
+            assert np.array_equal(a.view(np.uint32), b.view(np.uint32))
+
+
+CASES = [
+    # name, dtype, d, Hkv, T_list, N_list, values
+    ("bf16_d128_multi_tile", torch.bfloat16, 128, 2, [1000, 777], [37, 20], "normal"),
+    ("bf16_d64", torch.bfloat16, 64, 3, [600, 256, 1301], [11, 5, 40], "normal"),
+    ("f32_d64", torch.float32, 64, 1, [1024, 511], [32, 9], "normal"),
+    ("f32_d128", torch.float32, 128, 2, [700], [21], "walk"),
+    ("key_only_variation", torch.bfloat16, 128, 2, [2000, 900], [50, 30], "zero"),
+    ("short_sequences", torch.bfloat16, 128, 2, [0, 1, 8, 55, 56, 57, 60, 63], [4, 4, 4, 4, 4, 4, 4, 4], "normal"),
+    ("more_segments_than_tokens", torch.bfloat16, 128, 1, [70, 200], [40, 500], "normal"),
+    ("single_segment", torch.bfloat16, 128, 2, [3000], [1], "normal"),
+    ("tile_edges", torch.bfloat16, 128, 1, [56 + 255, 56 + 256, 56 + 510, 56 + 511, 56 + 254], [7, 7, 7, 7, 7],
+     "normal"),
+]
+
+
+@pytest.mark.parametrize("name,dtype,d,Hkv,T_list,N_list,values", CASES, ids=[c[0] for c in CASES])
+def test_coarsen_matches_oracle(name, dtype, d, Hkv, T_list, N_list, values):
+    seed = sum(T_list) + d
+    w = workloads.Workload(name, seed, B=len(T_list), Hq=Hkv, Hkv=Hkv, d=d, R=1,
+                           dtype="bf16" if dtype == torch.bfloat16 else "f32", T=0, regimes=12)
+    k, v, _ = workloads.make_kv(w, "cuda", T_list=T_list, values=values)
+    r = run_coarsen(k, v, Hkv, T_list, N_list, seed)
+    assert r["status"] == 0, f"device flags {r['flags']}"
+    orc = oracle_units(k, v, Hkv, T_list, N_list, seed)
+    compare_units(r, orc, k, T_list, Hkv, N_list, dtype)
+
+
+def test_constant_middle_gives_one_node():
+    """c_T = 0: every threshold is hit at the first middle token; one node holds the middle."""
+    T, d, Hkv = 700, 128, 1
+    k = torch.ones(T, d, dtype=torch.bfloat16, device="cuda") * 0.5
+    v = torch.zeros(T, d, dtype=torch.bfloat16, device="cuda")
+    k[:S] = torch.randn(S, d, device="cuda").bfloat16()
+    r = run_coarsen(k, v, Hkv, [T], [16], seed=1)
+    assert int(r["lens"][0, 0]) == S + 1 + W
+    orc = oracle_units(k, v, Hkv, [T], [16], seed=1)
+    compare_units(r, orc, k, [T], Hkv, [16], torch.bfloat16)
+
+
+def test_jump_crosses_many_thresholds():
+    """One huge step takes several thresholds at once: their segments are empty and dropped."""
+    T, d = 400, 128
+    g = torch.Generator(device="cuda").manual_seed(3)
+    k = (torch.randn(T, d, device="cuda", generator=g) * 0.01).bfloat16()
+    v = torch.zeros(T, d, dtype=torch.bfloat16, device="cuda")
+    k[200:] += 50.0
+    r = run_coarsen(k, v, 1, [T], [30], seed=2)
+    orc = oracle_units(k, v, 1, [T], [30], seed=2)
+    assert orc[(0, 0)].kt.shape[0] < S + 30 + W
+    compare_units(r, orc, k, [T], 1, [30], torch.bfloat16)
+
+
+def test_overflow_is_flagged():
+    T, d = 300, 128
+    k = torch.zeros(T, d, dtype=torch.float32, device="cuda")
+    v = torch.zeros(T, d, dtype=torch.float32, device="cuda")
+    k[150:] = 1e30
+    r = run_coarsen(k, v, 1, [T], [8], seed=2)
+    assert r["status"] == skv._lib.SKV_ERR_OVERFLOW and r["flags"] & skv._lib.FLAG_OVERFLOW
+
+
+def test_tiny_f32_end_to_end():
+    """The tiny fp32 workload: 1 KV head, 2 query heads, d=64, T=1024, N=32; nodes and decode
+    against the oracle's own nodes (fp32 bar: relative L2 <= 1e-5)."""
+    w = workloads.WORKLOADS["tiny_f32"]
+    k, v, T_list = workloads.make_kv(w, "cuda")
+    N_list = workloads.segment_counts(w, T_list)
+    r = run_coarsen(k, v, w.Hkv, T_list, N_list, w.seed)
+    assert r["status"] == 0
+    orc = oracle_units(k, v, w.Hkv, T_list, N_list, w.seed)
+    compare_units(r, orc, k, T_list, w.Hkv, N_list, torch.float32)
+    q = workloads.make_queries(w, "cuda")
+    out, lse = skv.decode_attn(q, w.Hkv, r["pool"], r["table"], r["lens"])
+    units = [[orc[(0, 0)]]]
+    ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), units)
+    check_decode(out, lse, ref_out, ref_lse, torch.float32, "tiny_f32 end to end")
+
+
+def test_gqa6_10k5_prefill_then_decode():
+    """1.5B-shaped: 12/2 heads, d=128, T=10,500, N=365: bit-exact segmentation of both heads,
+    node statistics, then decode over the GPU nodes."""
+    w = workloads.WORKLOADS["gqa6_10k5_prefill_decode"]
+    k, v, T_list = workloads.make_kv(w, "cuda")
+    N_list = workloads.segment_counts(w, T_list)
+    r = run_coarsen(k, v, w.Hkv, T_list, N_list, w.seed)
+    assert r["status"] == 0
+    orc = oracle_units(k, v, w.Hkv, T_list, N_list, w.seed)
+    compare_units(r, orc, k, T_list, w.Hkv, N_list, torch.bfloat16)
+    q = workloads.make_queries(w, "cuda")
+    out, lse = skv.decode_attn(q, w.Hkv, r["pool"], r["table"], r["lens"])
+    ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), gpu_units(r["pool"], r["table"], r["lens"], 1, 2))
+    check_decode(out, lse, ref_out, ref_lse, torch.bfloat16, "gqa6 decode")
+
+
+def test_coarsen_is_deterministic():
+    w = workloads.Workload("det", 9, B=2, Hq=4, Hkv=2, d=128, R=1, dtype="bf16", T=0, regimes=20)
+    k, v, T_list = workloads.make_kv(w, "cuda", T_list=[3000, 1700])
+    a = run_coarsen(k, v, 2, T_list, [90, 40], seed=9, shuffle=False)
+    b = run_coarsen(k, v, 2, T_list, [90, 40], seed=9, shuffle=False)
+    assert torch.equal(a["cum"], b["cum"]) and torch.equal(a["bnd"], b["bnd"])
+    assert torch.equal(a["pool"].k, b["pool"].k) and torch.equal(a["pool"].ab, b["pool"].ab)

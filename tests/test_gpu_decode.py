@@ -1,0 +1,108 @@
+"""GPU parity of compressed decode attention ("SPICY-KV" section 2 logit with online softmax)
+against the fp64 oracle, on synthetic entry sets written straight into the pool: GQA groups of
+1..8 heads, 1..5 query rows per sequence (row passes above 32 rows), d = 64 / 128, ragged and
+empty units, partial last pages, shuffled page tables and split units."""
+import math
+
+import numpy as np
+import pytest
+import torch
+
+import compressed_decode_attention_equal_b200 as skv
+import oracle
+from gpu_helpers import check_decode, gpu_units, pool_for_units, write_entries
+
+pytestmark = pytest.mark.gpu
+
+
+def _synthetic(B, Hq, Hkv, R, d, lens_list, dtype, seed, key_scale=3.0, shuffle=True, spare=0):
+    g = torch.Generator(device="cpu").manual_seed(seed)
+    pool, table = pool_for_units(lens_list, B, Hkv, d, dtype, shuffle=shuffle, seed=seed, spare_pages=spare)
+    for b in range(B):
+        for h in range(Hkv):
+            E = int(lens_list[b])
+            kt = torch.randn(E, d, generator=g) * key_scale
+            vt = torch.randn(E, d, generator=g)
+            mass = torch.randint(1, 200, (E,), generator=g).double()
+            alpha = torch.log(mass)
+            beta = torch.rand(E, generator=g) * 0.02
+            write_entries(pool, table, b, h, kt, vt, alpha, beta)
+    lens = torch.tensor([[int(lens_list[b])] * Hkv for b in range(B)], dtype=torch.int32, device="cuda")
+    q = (torch.randn(B, R, Hq, d, generator=g)).to(dtype).cuda()
+    return pool, table, lens, q
+
+
+def _run(B, Hq, Hkv, R, d, lens_list, dtype, seed, **kw):
+    pool, table, lens, q = _synthetic(B, Hq, Hkv, R, d, lens_list, dtype, seed, **kw)
+    out, lse = skv.decode_attn(q, Hkv, pool, table, lens)
+    torch.cuda.synchronize()
+    units = gpu_units(pool, table, lens, B, Hkv)
+    ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), units)
+    check_decode(out, lse, ref_out, ref_lse, dtype, what=f"B{B} Hq{Hq} Hkv{Hkv} R{R} d{d}")
+    return out, lse
+
+
+@pytest.mark.parametrize("Hq,Hkv,R", [(28, 4, 1), (12, 2, 1), (4, 4, 1), (16, 8, 1), (28, 4, 4), (16, 2, 5),
+                                      (14, 2, 2), (8, 1, 3)])
+def test_decode_bf16_gqa_shapes(Hq, Hkv, R):
+    B = 3
+    lens = [1147, 37, 300]
+    _run(B, Hq, Hkv, R, 128, lens, torch.bfloat16, seed=Hq * 10 + R)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_bf16_ragged_and_empty(d):
+    lens = [0, 1, 15, 16, 17, 31, 33, 250, 0, 2677]
+    _run(len(lens), 14, 2, 1, d, lens, torch.bfloat16, seed=d)
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_decode_f32_path(d):
+    lens = [88, 1, 0, 200]
+    _run(len(lens), 2, 1, 1, d, lens, torch.float32, seed=5 + d, key_scale=1.0)
+
+
+def test_decode_single_unit_many_ctas():
+    """One long unit split across every CTA (partials merged by the combine kernel)."""
+    _run(1, 7, 1, 1, 128, [20000], torch.bfloat16, seed=11)
+
+
+def test_decode_peaked_softmax():
+    """Large key scale: one entry dominates (online max updates across pages and CTAs)."""
+    _run(4, 28, 4, 1, 128, [500, 1500, 64, 3000], torch.bfloat16, seed=12, key_scale=12.0)
+
+
+def test_decode_is_deterministic():
+    a, la = _run(2, 28, 4, 1, 128, [900, 2000], torch.bfloat16, seed=13)
+    b, lb = _run(2, 28, 4, 1, 128, [900, 2000], torch.bfloat16, seed=13)
+    assert torch.equal(a, b) and torch.equal(la, lb)
+
+
+def test_decode_bad_page_id_is_flagged_not_read():
+    """A page id outside the pool raises the device flag and is skipped (no out-of-bounds read)."""
+    B, Hq, Hkv, d = 2, 7, 1, 128
+    pool, table, lens, q = _synthetic(B, Hq, Hkv, 1, d, [64, 64], torch.bfloat16, seed=3)
+    table[1, 0, 2] = pool.num_pages + 5
+    ws = torch.zeros(skv.decode_workspace_bytes(B, 1, Hq, Hkv, d, table.shape[2]), dtype=torch.uint8,
+                     device="cuda")
+    out, lse = skv.decode_attn(q, Hkv, pool, table, lens, workspace=ws)
+    st, flags = skv.workspace_error(ws)
+    assert st == skv._lib.SKV_ERR_DEVICE and flags & skv._lib.FLAG_BAD_PAGE
+    # unit 0 is untouched by the bad page
+    units = gpu_units(pool, table, lens, 1, Hkv)
+    ref_out, ref_lse = oracle.decode(q[:1].double().cpu().numpy(), units)
+    check_decode(out[:1], lse[:1], ref_out, ref_lse, torch.bfloat16)
+    st, flags = skv.workspace_error(ws)
+    assert st == 0 and flags == 0          # read-and-clear
+
+
+def test_decode_lens_above_capacity_is_clamped_and_flagged():
+    B, Hq, Hkv, d = 1, 7, 1, 128
+    pool, table, lens, q = _synthetic(B, Hq, Hkv, 1, d, [40], torch.bfloat16, seed=4, shuffle=False)
+    ws = torch.zeros(skv.decode_workspace_bytes(B, 1, Hq, Hkv, d, table.shape[2]), dtype=torch.uint8,
+                     device="cuda")
+    lens_bad = lens.clone()
+    lens_bad[0, 0] = table.shape[2] * 16 + 100
+    skv.decode_attn(q, Hkv, pool, table, lens_bad, workspace=ws)
+    st, flags = skv.workspace_error(ws)
+    assert flags & skv._lib.FLAG_BAD_LENS
