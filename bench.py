@@ -1,0 +1,527 @@
+"""Benchmark: compressed decode attention on the 7B-shaped GQA workload at 3.5% KV.
+
+Workload (one step = one decode-attention call for the whole batch):
+  B = 32 sequences, 28 query / 4 KV heads (GQA 7), d = 128, T = 32,768 tokens per sequence,
+  coarsened by this library's own kernels to 8 sink + N = 1,091 equal-variation nodes + 48
+  recent entries per KV head (regime-walk keys with 200 regimes, N(0,1) values, bf16). One
+  query row per query head: 896 query rows per step.
+  The caches of L layers (distinct seeds, 76 MB each) are built once; step i decodes layer
+  i % L, so consecutive steps never find their cache in the 126 MB L2.
+
+Output: one JSON line (rank 0) with the decode throughput (`value`, query rows/s), the decode
+op's achieved HBM bandwidth against the measured copy peak (`roofline`), an end-to-end figure
+with pinned host queries / outputs copied every step (`e2e`), the SM clocks sampled during the
+timed region, the CPU oracle timed on the host (`cpu_baseline`), and the coarsener's own
+throughput on the 8 x 4 x 131,072-token workload (`coarsen`).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+Multi-GPU (torchrun, one rank per GPU): every rank decodes its own batch (weak scaling, no
+collective on the data path); the timed duration is the max over ranks.
+"""
+from __future__ import annotations
+
+import argparse
+import dataclasses
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn query-rows/s & HBM GB/s (% of peak), 7B GQA shape, 3.5% KV"
+UNIT = "query-rows/s"
+WORKLOAD = "gqa7_32k_decode_3p5pct"
+COARSEN_WORKLOAD = "coarsen_131k"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def _peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as fh:
+            p = json.load(fh)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+def _source_sha(files):
+    h = hashlib.sha256()
+    for f in files:
+        with open(os.path.join(ROOT, f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+DECODE_SOURCES = ["compressed_decode_attention_equal_b200/csrc/decode.cu",
+                  "compressed_decode_attention_equal_b200/csrc/skv_common.cuh",
+                  "compressed_decode_attention_equal_b200/csrc/skv_internal.h"]
+COARSEN_SOURCES = ["compressed_decode_attention_equal_b200/csrc/coarsen.cu",
+                   "compressed_decode_attention_equal_b200/csrc/skv_common.cuh",
+                   "compressed_decode_attention_equal_b200/csrc/skv_internal.h"]
+
+
+def _profile_traffic(summary: str, sources):
+    """DRAM bytes per launch from a committed ncu summary, if it was taken on the current source."""
+    path = os.path.join(ROOT, "profiles", summary)
+    try:
+        text = open(path).read()
+    except OSError:
+        return None
+    m_sha = re.search(r"source_sha256_16:\s*([0-9a-f]+)", text)
+    m_b = re.search(r"dram_bytes_per_launch:\s*([0-9.eE+]+)", text)
+    if not m_sha or not m_b or m_sha.group(1) != _source_sha(sources):
+        return None
+    return float(m_b.group(1))
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples taken while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        if not rows:
+            return None
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, flags in rows for i, f in enumerate(flags) if f.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ---------------------------------------------------------------------------
+# workload set-up (untimed)
+# ---------------------------------------------------------------------------
+def build_layer_caches(w, layers: int, device):
+    import torch
+    import compressed_decode_attention_equal_b200 as skv
+    import workloads
+    T_list = workloads.seq_lengths(w)
+    N_list = workloads.segment_counts(w, T_list)
+    pages = [skv.pages_for(T, N, workloads.N_SINK, workloads.N_RECENT) for T, N in zip(T_list, N_list)]
+    table, num_pages = workloads.page_assignment(w.B, w.Hkv, pages, w.shuffle_pages, w.seed)
+    table = table.to(device)
+    ws = torch.zeros(skv.coarsen_workspace_bytes(w.Hkv, w.d, T_list, N_list, workloads.N_SINK, workloads.N_RECENT),
+                     dtype=torch.uint8, device=device)
+    caches, coarsen_ms = [], []
+    for layer in range(layers):
+        wl = dataclasses.replace(w, seed=w.seed + 1000 * layer)
+        k, v, _ = workloads.make_kv(wl, device, T_list=T_list)
+        pool = skv.NodePool(num_pages, w.d, w.torch_dtype, device=device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        lens = skv.coarsen(k, v, w.Hkv, T_list, N_list, workloads.N_SINK, workloads.N_RECENT, wl.seed, pool, table,
+                           workspace=ws)
+        e1.record()
+        torch.cuda.synchronize()
+        coarsen_ms.append(e0.elapsed_time(e1))
+        st, flags = skv.workspace_error(ws)
+        if st != 0:
+            raise RuntimeError(f"coarsening raised device flags {flags}")
+        q = workloads.make_queries(wl, device)
+        caches.append(dict(pool=pool, lens=lens, q=q, seed=wl.seed))
+        del k, v
+    torch.cuda.empty_cache()
+    return caches, table, T_list, N_list, coarsen_ms
+
+
+def algorithmic_decode_bytes(w, lens_list):
+    """HBM bytes one decode call must move: every entry's key, value and (alpha, beta) once,
+    the queries once, the outputs and lse once."""
+    ent = sum(int(x) for x in lens_list)
+    node = 2 * w.d * 2 + 8
+    rows = w.B * w.R * w.Hq
+    return ent * node + rows * w.d * 2 * 2 + rows * 4, ent
+
+
+def _graph_steps(fn, steps: int, chunk: int):
+    """Capture `fn(i)` for i in [0, chunk) into a CUDA graph (replayed for exactly `steps`)."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        with torch.cuda.graph(g, stream=s):
+            for i in range(chunk):
+                fn(i)
+    torch.cuda.current_stream().wait_stream(s)
+    return g
+
+
+def time_graphs(fn, steps: int, layers: int, dist_on: bool):
+    """Device time (ms) of exactly `steps` calls fn(i), replayed from CUDA graphs."""
+    import torch
+    chunk = max(layers, min(steps, 60 * layers))
+    chunk -= chunk % layers
+    full, rem = divmod(steps, chunk)
+    g_full = _graph_steps(fn, chunk, chunk) if full else None
+    g_rem = _graph_steps(fn, rem, rem) if rem else None
+    if g_full is not None:
+        g_full.replay()   # first replay uploads the graph
+    if g_rem is not None:
+        g_rem.replay()
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(full):
+        g_full.replay()
+    if g_rem is not None:
+        g_rem.replay()
+    e1.record()
+    torch.cuda.synchronize()
+    if dist_on:
+        torch.distributed.barrier()
+    return e0.elapsed_time(e1)
+
+
+def coarsen_stage(device, reps: int = 5):
+    """Coarsener throughput on the 8 x 4 x 131,072-token workload (tokens/s, GB/s of raw KV)."""
+    import torch
+    import compressed_decode_attention_equal_b200 as skv
+    import workloads
+    w = workloads.WORKLOADS[COARSEN_WORKLOAD]
+    T_list = workloads.seq_lengths(w)
+    N_list = workloads.segment_counts(w, T_list)
+    k, v, _ = workloads.make_kv(w, device, T_list=T_list)
+    pages = [skv.pages_for(T, N, workloads.N_SINK, workloads.N_RECENT) for T, N in zip(T_list, N_list)]
+    table, num_pages = workloads.page_assignment(w.B, w.Hkv, pages, False, w.seed)
+    table = table.to(device)
+    pool = skv.NodePool(num_pages, w.d, w.torch_dtype, device=device)
+    lens = torch.empty(w.B, w.Hkv, dtype=torch.int32, device=device)
+    ws = torch.zeros(skv.coarsen_workspace_bytes(w.Hkv, w.d, T_list, N_list, workloads.N_SINK, workloads.N_RECENT),
+                     dtype=torch.uint8, device=device)
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
+
+    def call():
+        skv.coarsen(k, v, w.Hkv, T_list, N_list, workloads.N_SINK, workloads.N_RECENT, w.seed, pool, table,
+                    lens=lens, workspace=ws)
+
+    for _ in range(2):
+        call()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(reps):
+        flush.zero_()                      # evict the raw KV from L2 between calls
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        call()
+        e1.record()
+        torch.cuda.synchronize()
+        times.append(e0.elapsed_time(e1))
+    st, flags = skv.workspace_error(ws)
+    if st != 0:
+        raise RuntimeError(f"coarsening raised device flags {flags}")
+    ms = statistics.median(times)
+    tokens = sum(T_list) * w.Hkv
+    raw_bytes = 2 * tokens * w.d * 2
+    ent = int(lens.sum())
+    node_bytes = ent * (2 * w.d * 2 + 8)
+    alg = raw_bytes + node_bytes
+    peak, src = _peaks()
+    middle = sum(max(0, T - workloads.N_SINK - workloads.N_RECENT) for T in T_list) * w.Hkv
+    fma = middle * 16 * 2 * w.d
+    sm_clock_ghz = 1.965
+    alu_peak_tfma = 148 * 128 * sm_clock_ghz / 1000.0
+    del k, v, flush
+    torch.cuda.empty_cache()
+    return {
+        "workload": COARSEN_WORKLOAD, "ms": ms, "tokens_per_s": tokens / (ms / 1e3),
+        "raw_kv_gbs": raw_bytes / (ms / 1e3) / 1e9,
+        "roofline": {"bound": "hbm", "achieved": alg / (ms / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                     "frac": alg / (ms / 1e3) / 1e9 / peak, "peak_source": src, "traffic": _profile_traffic(
+                         "coarsen_131k_summary.md", COARSEN_SOURCES), "algorithmic_bytes": alg},
+        "projection_alu": {"fma_per_call": fma, "achieved_tfma_s": fma / (ms / 1e3) / 1e12,
+                           "peak_tfma_s_at_max_clock": alu_peak_tfma},
+        "frac_of_8tbs": alg / (ms / 1e3) / 8e12,
+    }
+
+
+def cpu_baseline(w, caches, table, budget_s: float = 12.0):
+    """The fp64 CPU oracle decoding the same cache (nodes read back from the GPU) on the host
+    cores: whole batches of one layer, repeated until `budget_s` of work."""
+    import numpy as np
+    import torch
+    import compressed_decode_attention_equal_b200 as skv
+    import oracle
+
+    class U:
+        def __init__(self, kt, vt, al, be):
+            self.kt, self.vt, self.alpha, self.beta = kt, vt, al, be
+
+    c = caches[0]
+    units = []
+    for b in range(w.B):
+        row = []
+        for h in range(w.Hkv):
+            kt, vt, al, be = skv.read_entries(c["pool"], table, c["lens"], b, h)
+            row.append(U(kt.double().cpu().numpy(), vt.double().cpu().numpy(), al.double().cpu().numpy(),
+                         be.double().cpu().numpy()))
+        units.append(row)
+    q = c["q"].double().cpu().numpy()
+    threads = os.cpu_count() or 1
+    rows = 0
+    t0 = time.perf_counter()
+    reps = 0
+    while True:
+        oracle.decode(q, units, threads=threads)
+        rows += w.B * w.R * w.Hq
+        reps += 1
+        if time.perf_counter() - t0 >= budget_s:
+            break
+    dt = time.perf_counter() - t0
+    return {"value": rows / dt, "unit": UNIT, "cores": threads, "kind": "oracle",
+            "sample": f"{reps} full decode batches of one layer ({w.B} x {w.Hq} query rows over "
+                      f"{int(c['lens'].sum())} entries), fp64, nodes read back from the GPU"}
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+def run_ours(args, rank: int, world: int, device):
+    import torch
+    import compressed_decode_attention_equal_b200 as skv
+    import workloads
+
+    dist_on = world > 1
+    w = workloads.WORKLOADS[WORKLOAD]
+    if dist_on:   # each rank decodes its own, independently seeded batch
+        w = dataclasses.replace(w, seed=w.seed + 100000 * rank)
+    caches, table, T_list, N_list, coarsen_ms = build_layer_caches(w, args.layers, device)
+    L = len(caches)
+    rows_per_step = w.B * w.R * w.Hq
+    alg_bytes, ent = algorithmic_decode_bytes(w, [int(c["lens"].sum()) for c in caches][:1])
+    outs = [torch.empty_like(c["q"]) for c in caches]
+    lses = [torch.empty(w.B, w.R, w.Hq, dtype=torch.float32, device=device) for _ in caches]
+    ws = torch.zeros(skv.decode_workspace_bytes(w.B, w.R, w.Hq, w.Hkv, w.d, table.shape[2]), dtype=torch.uint8,
+                     device=device)
+
+    def step(i):
+        c = caches[i % L]
+        skv.decode_attn(c["q"], w.Hkv, c["pool"], table, c["lens"], out=outs[i % L], lse=lses[i % L], workspace=ws)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    st, flags = skv.workspace_error(ws)
+    if st != 0:
+        raise RuntimeError(f"decode raised device flags {flags}")
+
+    sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    ms = time_graphs(step, args.steps, L, dist_on)
+    clocks = sampler.stop() if sampler else None
+    if dist_on:
+        t = torch.tensor([ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    ms_per_step = ms / args.steps
+    value = rows_per_step * world * args.steps / (ms / 1e3)
+
+    # end to end: pinned host queries in, pinned host outputs back, every step
+    q_host = [c["q"].cpu().pin_memory() for c in caches]
+    out_host = [torch.empty_like(q, device="cpu").pin_memory() for q in q_host]
+    lse_host = [torch.empty(w.B, w.R, w.Hq, dtype=torch.float32).pin_memory() for _ in caches]
+    q_dev = [torch.empty_like(c["q"]) for c in caches]
+
+    def e2e_step(i):
+        j = i % L
+        q_dev[j].copy_(q_host[j], non_blocking=True)
+        c = caches[j]
+        skv.decode_attn(q_dev[j], w.Hkv, c["pool"], table, c["lens"], out=outs[j], lse=lses[j], workspace=ws)
+        out_host[j].copy_(outs[j], non_blocking=True)
+        lse_host[j].copy_(lses[j], non_blocking=True)
+
+    for i in range(min(args.warmup, 3 * L)):
+        e2e_step(i)
+    e2e_steps = max(L, min(args.steps, 20000))
+    e2e_ms = time_graphs(e2e_step, e2e_steps, L, dist_on)
+    if dist_on:
+        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    # the timed copies are real: the last step's outputs match the device results
+    torch.cuda.synchronize()
+    assert torch.equal(out_host[(e2e_steps - 1) % L], outs[(e2e_steps - 1) % L].cpu())
+
+    result = None
+    if rank == 0:
+        peak, src = _peaks()
+        achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
+        launches_per_step = 1   # one decode kernel per call
+        result = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16",
+            "data": "synthetic: regime-walk keys, N(0,1) values and queries, coarsened on the GPU by this library",
+            "config": {"workload": WORKLOAD, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "d": w.d,
+                       "context": w.T, "middle_nodes": w.N, "entries_per_head": ent // (w.B * w.Hkv),
+                       "query_rows_per_step": rows_per_step, "parallelism": f"dp{world}" if world > 1 else "single",
+                       "l2": f"inputs larger than L2: {L} layer caches of {alg_bytes / 1e6:.1f} MB rotated",
+                       "timing": "CUDA graphs of back-to-back decode calls, CUDA events around the replay"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
+                         "traffic": _profile_traffic("decode_gqa7_32k_summary.md", DECODE_SOURCES),
+                         "peak_source": f"{src} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
+                         if src == "measured" else "fallback 6.65 TB/s",
+                         "frac_of_8tbs": achieved / 8000.0, "algorithmic_bytes_per_launch": alg_bytes,
+                         "kernel": "k_decode_split (one launch per call), time per call"},
+            "e2e": {"value": rows_per_step * world * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+                    "h2d_bytes_per_step": q_host[0].numel() * q_host[0].element_size(),
+                    "d2h_bytes_per_step": out_host[0].numel() * out_host[0].element_size() + lse_host[0].numel() * 4,
+                    "steps": e2e_steps},
+            "gpu_launches": launches_per_step * args.steps,
+            "clocks": clocks,
+            "coarsen_build_ms_per_layer": coarsen_ms,
+        }
+    return result, caches, table, w
+
+
+def run_reference(args, rank: int):
+    """The oracle on the host cores, on this arm's workload, metric and unit (rank 0 only)."""
+    if rank != 0:
+        return None
+    import numpy as np
+    import oracle
+    import workloads
+    w = workloads.WORKLOADS[WORKLOAD]
+    rng = np.random.default_rng(w.seed)
+    # the oracle decodes units whose entries have the workload's shape: E = 8 + 1091 + 48 per head
+    E = workloads.N_SINK + w.N + workloads.N_RECENT
+    T, N = w.T, w.N
+    sizes = np.full(N, (T - workloads.N_SINK - workloads.N_RECENT) // N)
+    sizes[: (T - workloads.N_SINK - workloads.N_RECENT) % N] += 1
+    mass = np.concatenate([np.ones(workloads.N_SINK), sizes, np.ones(workloads.N_RECENT)])
+
+    class U:
+        pass
+
+    def unit():
+        u = U()
+        u.kt = rng.standard_normal((E, w.d)) * 3
+        u.vt = rng.standard_normal((E, w.d))
+        u.alpha = np.log(mass)
+        u.beta = rng.random(E) * 1e-3
+        return u
+
+    units = [[unit() for _ in range(w.Hkv)] for _ in range(w.B)]
+    q = rng.standard_normal((w.B, w.R, w.Hq, w.d))
+    threads = os.cpu_count() or 1
+    # calibrate: one step decodes `n` sequences so that warmup + steps fit in ~60 s
+    t0 = time.perf_counter()
+    oracle.decode(q[:1], units[:1], threads=threads)
+    per_seq = max(time.perf_counter() - t0, 1e-4)
+    budget = 60.0 / max(1, args.steps + args.warmup)
+    n = int(max(1, min(w.B, budget / per_seq)))
+    for i in range(args.warmup):
+        oracle.decode(q[:n], units[:n], threads=threads)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        oracle.decode(q[:n], units[:n], threads=threads)
+    dt = time.perf_counter() - t0
+    rows = n * w.R * w.Hq * args.steps
+    value = rows / dt
+    return {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": 1, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic entries with the workload's shape", "impl": "reference",
+        "config": {"workload": WORKLOAD, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "d": w.d,
+                   "context": w.T, "middle_nodes": w.N, "entries_per_head": E},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": f"{n} of {w.B} sequences per step ({n * w.Hq} query rows x {E} entries)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=60000)
+    ap.add_argument("--warmup", type=int, default=600)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--layers", type=int, default=6)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-coarsen", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        res = run_reference(args, rank)
+        if res is not None:
+            print(json.dumps(res), flush=True)
+        return
+
+    import torch
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device")
+    torch.cuda.set_device(local)
+    device = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=device)
+    from compressed_decode_attention_equal_b200 import build
+    build.build()
+    res, caches, table, w = run_ours(args, rank, world, device)
+    if rank == 0:
+        if not args.no_coarsen:
+            res["coarsen"] = coarsen_stage(device)
+        if not args.no_cpu_baseline:
+            res["cpu_baseline"] = cpu_baseline(w, caches, table)
+        print(json.dumps(res), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

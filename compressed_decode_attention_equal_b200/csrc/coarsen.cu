@@ -467,9 +467,16 @@ static cudaError_t launch_typed(const CoarsenArgs &a, const SeqTable &table, con
     k_setup<<<1, 512, 0, s>>>(table, const_cast<SeqRow *>(a.seq), a.B, a.flags);
     if (a.max_tiles > 0) {
         constexpr size_t smem = k1_smem_bytes<D>();
-        cudaError_t e = cudaFuncSetAttribute(k_project_scan<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                             static_cast<int>(smem));
+        static thread_local int configured_dev = -1;
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return e;
+        if (configured_dev != dev) {
+            e = cudaFuncSetAttribute(k_project_scan<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem));
+            if (e != cudaSuccess) return e;
+            configured_dev = dev;
+        }
         k_project_scan<D, T><<<dim3(a.max_tiles, units), kK1Threads, smem, s>>>(a, map_k, map_v, proj);
         k_tile_prefix<<<units, 256, 0, s>>>(a);
         k_boundaries<<<dim3(a.max_tiles, units), 256, 0, s>>>(a);

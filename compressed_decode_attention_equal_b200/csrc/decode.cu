@@ -8,7 +8,7 @@
 // proceeds as for exact tokens. Claim 3: the beta term is the second-order
 // cumulant closure of the partition Z.
 //
-// bf16 path (k_decode_split + k_decode_combine), split-K over pages:
+// bf16 path (k_decode_split, one launch per call), split-K over pages:
 //  * the flat page space of all (unit, row-pass) "virtual units" is cut into
 //    ncta equal ranges (one per CTA, a stream-K style split), so every CTA
 //    streams the same number of 16-node pages whatever the length mix;
@@ -19,10 +19,17 @@
 //    N = 8 (a GQA group of 7 rows wastes 1/8), softmax on the accumulator, P^T
 //    transposed in registers (movmatrix) into the B operand of O^T = V^T P^T;
 //  * a piece that covers a whole unit writes out / lse directly; pieces of a
-//    unit split across CTAs write (lse, out) partials that k_decode_combine
-//    merges with a log-sum-exp.
+//    unit split across CTAs write (lse, out) partials, and the CTA that
+//    finishes a unit last (an atomic per-unit counter, reset after use) merges
+//    them with a log-sum-exp;
+//  * launched with programmatic stream serialisation: the next launch's CTAs
+//    become resident while this grid drains; each grid reads its inputs only
+//    after griddepcontrol.wait, so data from any preceding kernel is visible.
 // fp32 path (k_decode_f32): a plain CUDA-core kernel (exact fp32 arithmetic),
 // one CTA per unit, for fp32 caches.
+#include <mutex>
+#include <vector>
+
 #include "skv_common.cuh"
 #include "skv_internal.h"
 
@@ -76,7 +83,11 @@ __device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, i
     const int per = (nv + nth - 1) / nth;
     const int lo = min(tid * per, nv), hi = min(lo + per, nv);
     int local = 0;
-    for (int v = lo; v < hi; ++v) local += (clamp_entries(a, v / a.row_passes) + kPageNodes - 1) / kPageNodes;
+    for (int v = lo; v < hi; ++v) {
+        const int pages = (clamp_entries(a, v / a.row_passes) + kPageNodes - 1) / kPageNodes;
+        prefix[v] = pages;   // page count for now; made exclusive below
+        local += pages;
+    }
     // block exclusive scan of `local`
     const int lane = tid & 31, warp = tid >> 5;
     int x = local;
@@ -91,11 +102,52 @@ __device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, i
     for (int w = 0; w < warp; ++w) wp += scratch[w];
     int run = wp + x - local;
     for (int v = lo; v < hi; ++v) {
+        const int pages = prefix[v];
         prefix[v] = run;
-        run += (clamp_entries(a, v / a.row_passes) + kPageNodes - 1) / kPageNodes;
+        run += pages;
     }
     if (tid == nth - 1) prefix[nv] = wp + x;
     __syncthreads();
+}
+
+// First flat page of CTA c's range, and the CTA whose (nonempty) range holds page f.
+__device__ __forceinline__ long long cta_begin(long long c, long long ptot, int ncta) { return ptot * c / ncta; }
+__device__ __forceinline__ long long cta_of(long long f, long long ptot, int ncta) {
+    return ((f + 1) * ncta + ptot - 1) / ptot - 1;
+}
+
+// Log-sum-exp merge of every piece of virtual unit v (run by the CTA that completed it).
+template <int D>
+__device__ void merge_unit(const DecodeArgs &a, int v, int b, int h, int rpass, long long ps, long long pe,
+                           long long ptot, int tid, int nth) {
+    const long long c_first = cta_of(ps, ptot, a.ncta), c_last = cta_of(pe - 1, ptot, a.ncta);
+    const int rows_here = min(a.pass_rows, a.rows - rpass * kRowsPerPass);
+    __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(a.out);
+    for (int idx = tid; idx < rows_here * D; idx += nth) {
+        const int rr = idx / D, dim = idx % D;
+        const int row = rpass * kRowsPerPass + rr;
+        float M = -INFINITY;
+        for (long long cc = c_first; cc <= c_last; ++cc) {
+            const long long a_c = cta_begin(cc, ptot, a.ncta);
+            if (a_c >= cta_begin(cc + 1, ptot, a.ncta)) continue;   // an empty range wrote no partial
+            const int slot = ps < a_c ? 0 : 1;
+            M = fmaxf(M, __ldcg(a.part + ((cc * 2 + slot) * a.pass_rows + rr) * (D + 1)));
+        }
+        const float Mb = M == -INFINITY ? 0.0f : M;
+        float Ls = 0.0f, Os = 0.0f;
+        for (long long cc = c_first; cc <= c_last; ++cc) {
+            const long long a_c = cta_begin(cc, ptot, a.ncta);
+            if (a_c >= cta_begin(cc + 1, ptot, a.ncta)) continue;
+            const int slot = ps < a_c ? 0 : 1;
+            const float *pp = a.part + ((cc * 2 + slot) * a.pass_rows + rr) * (D + 1);
+            const float w = ex2(__ldcg(pp) - Mb);
+            Ls += w;
+            Os = fmaf(__ldcg(pp + 1 + dim), w, Os);
+        }
+        const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
+        outp[oi * D + dim] = __float2bfloat16_rn(Ls > 0.0f ? __fdividef(Os, Ls) : 0.0f);
+        if (dim == 0) a.lse[oi] = Ls > 0.0f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
+    }
 }
 
 template <int D, int NT>
@@ -116,12 +168,28 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nv = a.n_vunits;
+    // let the next launch in the stream become resident as our CTAs retire; then wait for every
+    // preceding grid to complete (its writes visible) before reading any input
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+    asm volatile("griddepcontrol.wait;" ::: "memory");
     build_prefix(a, prefix, scan_scratch);
-    if (blockIdx.x == 0)
-        for (int v = tid; v <= nv; v += kDecThreads) a.vu_prefix[v] = prefix[v];
     const long long ptot = prefix[nv];
     const long long ra = ptot * blockIdx.x / a.ncta;
     const long long rb = ptot * (blockIdx.x + 1) / a.ncta;
+    // units with no entries get out = 0, lse = -inf (spread over the CTAs)
+    for (int v = blockIdx.x; v < nv; v += a.ncta) {
+        if (prefix[v + 1] != prefix[v]) continue;
+        const int u = v / a.row_passes, rpass = v % a.row_passes;
+        const int b = u / a.Hkv, h = u % a.Hkv;
+        for (int idx = tid; idx < a.pass_rows * D; idx += kDecThreads) {
+            const int rr = idx / D, dim = idx % D;
+            const int row = rpass * kRowsPerPass + rr;
+            if (row >= a.rows) continue;
+            const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
+            static_cast<__nv_bfloat16 *>(a.out)[oi * D + dim] = __float2bfloat16_rn(0.0f);
+            if (dim == 0) a.lse[oi] = -INFINITY;
+        }
+    }
     if (ra >= rb) return;
     const int v0 = find_vunit(prefix, nv, ra);
     const int n_my = static_cast<int>(rb - ra);
@@ -292,12 +360,28 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                 // O^T (D x 8) += V^T (D x 16) P^T (16 x 8)
                 {
                     const int mi = lane >> 3, node = (lane & 7) + 8 * (mi >> 1);
+                    if (nvalid == kPageNodes) {
 #pragma unroll
-                    for (int mt = 0; mt < NKS; ++mt) {
-                        const int chunk = 2 * mt + (mi & 1);
-                        uint32_t a0, a1, a2, a3;
-                        ldsm_x4_t(vb + node * G::ROWB + (swz(chunk, node) << 4), a0, a1, a2, a3);
-                        mma_bf16(o[mt], a0, a1, a2, a3, bp0, bp1);
+                        for (int mt = 0; mt < NKS; ++mt) {
+                            const int chunk = 2 * mt + (mi & 1);
+                            uint32_t a0, a1, a2, a3;
+                            ldsm_x4_t(vb + node * G::ROWB + (swz(chunk, node) << 4), a0, a1, a2, a3);
+                            mma_bf16(o[mt], a0, a1, a2, a3, bp0, bp1);
+                        }
+                    } else {
+                        // slots past the unit's last entry may hold anything (NaN included):
+                        // zero their V^T elements, since P = 0 does not cancel NaN in the product.
+                        // This thread's fragment holds nodes 2c, 2c+1 (a0..a3) and 2c+8, 2c+9 (a4..a7).
+                        const uint32_t m_lo = (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
+                        const uint32_t m_hi =
+                            (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
+#pragma unroll
+                        for (int mt = 0; mt < NKS; ++mt) {
+                            const int chunk = 2 * mt + (mi & 1);
+                            uint32_t a0, a1, a2, a3;
+                            ldsm_x4_t(vb + node * G::ROWB + (swz(chunk, node) << 4), a0, a1, a2, a3);
+                            mma_bf16(o[mt], a0 & m_lo, a1 & m_lo, a2 & m_hi, a3 & m_hi, bp0, bp1);
+                        }
                     }
                 }
             }
@@ -348,7 +432,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                 Ls = fmaf(st[D + 1], w, Ls);
                 Os = fmaf(st[dim], w, Os);
             }
-            const float val = Ls > 0.0f ? Os / Ls : 0.0f;
+            const float val = Ls > 0.0f ? __fdividef(Os, Ls) : 0.0f;
             const float lse2 = Ls > 0.0f ? M + __log2f(Ls) : -INFINITY;
             if (complete) {
                 const int r = row / a.G, gg = row % a.G;
@@ -361,59 +445,27 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                 if (dim == 0) pp[0] = lse2;
             }
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
-    }
-}
-
-// Merge the partials of units split across CTAs; write empty units.
-template <int D, typename TOut>
-__global__ void __launch_bounds__(128) k_decode_combine(const DecodeArgs a) {
-    const int v = blockIdx.x;
-    const long long ps = a.vu_prefix[v], pe = a.vu_prefix[v + 1], ptot = a.vu_prefix[a.n_vunits];
-    const int u = v / a.row_passes, rpass = v % a.row_passes;
-    const int b = u / a.Hkv, h = u % a.Hkv;
-    const int rows_here = min(a.pass_rows, a.rows - rpass * kRowsPerPass);
-    TOut *outp = static_cast<TOut *>(a.out);
-    auto cta_of = [&](long long f) -> long long { return ((f + 1) * a.ncta + ptot - 1) / ptot - 1; };
-    long long c_first = 0, c_last = -1;
-    if (pe > ps) {
-        c_first = cta_of(ps);
-        c_last = cta_of(pe - 1);
-        if (c_first == c_last) return;   // written whole by the split kernel
-    }
-    for (int idx = threadIdx.x; idx < rows_here * D; idx += blockDim.x) {
-        const int rr = idx / D, dim = idx % D;
-        const int row = rpass * kRowsPerPass + rr;
-        float val = 0.0f, lse2 = -INFINITY;
-        if (pe > ps) {
-            float M = -INFINITY;
-            for (long long cc = c_first; cc <= c_last; ++cc) {
-                const long long a_c = ptot * cc / a.ncta, b_c = ptot * (cc + 1) / a.ncta;
-                if (a_c >= b_c) continue;   // an empty range wrote no partial
-                const int slot = ps < a_c ? 0 : 1;
-                M = fmaxf(M, a.part[((cc * 2 + slot) * a.pass_rows + rr) * (D + 1)]);
+        if (!complete) {
+            // publish this piece; the CTA that completes the unit merges all of its pieces
+            __threadfence();
+            asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
+            int *last = reinterpret_cast<int *>(mbuf);   // mbuf is free again after the barrier
+            if (ctid == 0) {
+                const long long c_first = cta_of(ps, ptot, a.ncta), c_last = cta_of(pe - 1, ptot, a.ncta);
+                int pieces = 0;
+                for (long long cc = c_first; cc <= c_last; ++cc) pieces += cta_begin(cc, ptot, a.ncta) <
+                                                                            cta_begin(cc + 1, ptot, a.ncta);
+                const int prev = atomicAdd(a.counters + v, 1);
+                *last = (prev == pieces - 1) ? 1 : 0;
             }
-            const float Mb = M == -INFINITY ? 0.0f : M;
-            float Ls = 0.0f, Os = 0.0f;
-            for (long long cc = c_first; cc <= c_last; ++cc) {
-                const long long a_c = ptot * cc / a.ncta, b_c = ptot * (cc + 1) / a.ncta;
-                if (a_c >= b_c) continue;
-                const int slot = ps < a_c ? 0 : 1;
-                const float *pp = a.part + ((cc * 2 + slot) * a.pass_rows + rr) * (D + 1);
-                const float w = exp2f(pp[0] - Mb);
-                Ls += w;
-                Os = fmaf(pp[1 + dim], w, Os);
-            }
-            if (Ls > 0.0f) {
-                val = Os / Ls;
-                lse2 = M + log2f(Ls);
+            asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
+            if (*last) {
+                __threadfence();
+                merge_unit<D>(a, v, b, h, rpass, ps, pe, ptot, ctid, kDecConsumers * 32);
+                if (ctid == 0) a.counters[v] = 0;   // ready for the next call
             }
         }
-        const int r = row / a.G, gg = row % a.G;
-        const long long oi = (static_cast<long long>(b) * a.R + r) * a.Hq + h * a.G + gg;
-        if constexpr (sizeof(TOut) == 2) outp[oi * D + dim] = __float2bfloat16_rn(val);
-        else outp[oi * D + dim] = val;
-        if (dim == 0) a.lse[oi] = lse2 * kLn2;
+        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
     }
 }
 
@@ -487,24 +539,63 @@ static size_t split_smem(int n_vunits) {
     return dec_smem_fixed<D>() + static_cast<size_t>(n_vunits + 1) * 4;
 }
 
+// Grid size of the split kernel for one (device, shared-memory size): SMs x resident CTAs.
+// Queried once and cached, so that later calls (and stream capture) issue no attribute queries.
 template <int D, int NT>
-static cudaError_t launch_split(const DecodeArgs &a0, cudaStream_t s) {
-    DecodeArgs a = a0;
-    const size_t smem = split_smem<D, NT>(a.n_vunits);
-    cudaError_t e = cudaFuncSetAttribute(k_decode_split<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(smem));
+static cudaError_t split_grid(size_t smem, int *ncta) {
+    struct Entry {
+        int dev;
+        size_t smem;
+        int ncta;
+    };
+    static std::mutex mu;
+    static std::vector<Entry> cache;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
-    int dev = 0, sms = 0, occ = 0;
-    if ((e = cudaGetDevice(&dev)) != cudaSuccess) return e;
+    std::lock_guard<std::mutex> lock(mu);
+    for (const Entry &c : cache)
+        if (c.dev == dev && c.smem == smem) {
+            *ncta = c.ncta;
+            return cudaSuccess;
+        }
+    bool configured = false;
+    for (const Entry &c : cache) configured |= (c.dev == dev);
+    if (!configured) {
+        // the largest request any call can make (the page prefix of kMaxVUnits virtual units)
+        e = cudaFuncSetAttribute(k_decode_split<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(split_smem<D, NT>(kMaxVUnits)));
+        if (e != cudaSuccess) return e;
+    }
+    int sms = 0, occ = 0;
     if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
     if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_split<D, NT>, kDecThreads, smem)) !=
         cudaSuccess)
         return e;
-    a.ncta = sms * (occ > 0 ? occ : 1);
-    if (a.ncta > kMaxDecodeCtas) a.ncta = kMaxDecodeCtas;
-    k_decode_split<D, NT><<<a.ncta, kDecThreads, smem, s>>>(a);
-    k_decode_combine<D, __nv_bfloat16><<<a.n_vunits, 128, 0, s>>>(a);
-    return cudaGetLastError();
+    int n = sms * (occ > 0 ? occ : 1);
+    if (n > kMaxDecodeCtas) n = kMaxDecodeCtas;
+    cache.push_back({dev, smem, n});
+    *ncta = n;
+    return cudaSuccess;
+}
+
+template <int D, int NT>
+static cudaError_t launch_split(const DecodeArgs &a0, cudaStream_t s) {
+    DecodeArgs a = a0;
+    const size_t smem = split_smem<D, NT>(a.n_vunits);
+    cudaError_t e = split_grid<D, NT>(smem, &a.ncta);
+    if (e != cudaSuccess) return e;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(a.ncta);
+    cfg.blockDim = dim3(kDecThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k_decode_split<D, NT>, a);
 }
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {

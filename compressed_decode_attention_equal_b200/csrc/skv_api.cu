@@ -203,8 +203,8 @@ skv_status plan_decode(int dtype, int B, int R, int Hq, int Hkv, int d, int max_
     if (static_cast<int64_t>(B) * Hkv * max_pages * p.row_passes > INT32_MAX / 2) return SKV_ERR_UNSUPPORTED;
     p.n_vunits = static_cast<int>(nv);
     size_t off = kWsHeader;
-    p.lay.vu_prefix = off;
-    off += align256(static_cast<size_t>(nv + 1) * 4);
+    p.lay.counters = off;
+    off += align256(static_cast<size_t>(nv) * 4);
     p.lay.part = off;
     if (dtype == SKV_BF16) off += align256(static_cast<size_t>(kMaxDecodeCtas) * 2 * p.pass_rows * (d + 1) * 4);
     p.lay.total = off;
@@ -347,7 +347,7 @@ skv_status skv_decode_attn(const void *q, skv_dtype dtype, int B, int R, int Hq,
     a.pass_rows = plan.pass_rows;
     a.n_vunits = plan.n_vunits;
     a.part = reinterpret_cast<float *>(ws + plan.lay.part);
-    a.vu_prefix = reinterpret_cast<int32_t *>(ws + plan.lay.vu_prefix);
+    a.counters = reinterpret_cast<int32_t *>(ws + plan.lay.counters);
     a.flags = reinterpret_cast<uint32_t *>(ws);
     const cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SKV_OK : SKV_ERR_CUDA;

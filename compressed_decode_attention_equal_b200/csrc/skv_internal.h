@@ -93,12 +93,12 @@ struct DecodeArgs {
     int n_vunits;     // B * Hkv * row_passes
     int ncta;         // CTAs of the split kernel
     float *part;      // [ncta][2][pass_rows][d + 1] split partials
-    int32_t *vu_prefix;  // [n_vunits + 1] page prefix over virtual units
+    int32_t *counters;   // [n_vunits] pieces finished per virtual unit (zero between calls)
     uint32_t *flags;
 };
 
 struct DecodeLayout {
-    size_t vu_prefix, part, total;
+    size_t counters, part, total;
 };
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);

@@ -31,8 +31,13 @@
  *  - Host-detectable errors return before anything is enqueued. Errors that
  *    only the device can see (a page id outside the pool, a lens entry above
  *    the page table's capacity, a variation overflow) set a flag in the
- *    workspace header that skv_workspace_error reports; the offending write is
- *    skipped, never performed out of bounds.
+ *    workspace header that skv_workspace_error reports; the offending access
+ *    is skipped, never performed out of bounds. Flags are sticky: they
+ *    accumulate until skv_workspace_error reads and clears them (skv_coarsen
+ *    also clears them when it starts).
+ *  - A workspace must be zero-filled before its first use (cudaMemsetAsync or
+ *    torch.zeros); every call leaves it ready for the next call. Calls that
+ *    share a workspace must be ordered on one stream.
  *  - Supported: d in {64, 128}; dtype SKV_F32 or SKV_BF16 (keys, values,
  *    queries, node vectors and outputs share the dtype; alpha/beta and lse are
  *    fp32); at most SKV_MAX_SEQS sequences per call.
@@ -167,7 +172,12 @@ size_t skv_decode_workspace_bytes(int B, int R, int Hq, int Hkv, int d, int max_
  * lse   : [B][R][Hq] fp32, natural-log partition ln sum_j exp(s_j); a unit
  *         with zero entries gives out = 0 and lse = -inf.
  * workspace : device scratch of at least skv_decode_workspace_bytes bytes,
- *         256-byte aligned (split partials and the device error flags).
+ *         256-byte aligned (split partials, per-unit completion counters that
+ *         every call returns to zero, and the device error flags).
+ *
+ * One kernel launch per call (programmatic stream serialisation: it becomes
+ * resident while the previous launch drains, and reads its inputs only after
+ * every preceding grid in the stream has completed). Graph-capturable.
  *
  * Errors: SKV_ERR_INVALID_ARG, SKV_ERR_UNSUPPORTED (d, dtype, Hq % Hkv != 0),
  * SKV_ERR_WORKSPACE, SKV_ERR_CUDA. Device-detected bad page ids or lens above
@@ -180,10 +190,11 @@ skv_status skv_decode_attn(const void *q, skv_dtype dtype, int B, int R, int Hq,
                            void *stream);
 
 /*
- * Synchronise stream and report the device error flags that the last
- * skv_coarsen or skv_decode_attn call on this workspace raised: SKV_OK,
- * SKV_ERR_OVERFLOW or SKV_ERR_DEVICE (SKV_ERR_CUDA if synchronisation fails).
- * *flags_host (optional) receives the raw flag bits.
+ * Synchronise stream, then read and clear the device error flags raised on
+ * this workspace since they were last cleared: SKV_OK, SKV_ERR_OVERFLOW or
+ * SKV_ERR_DEVICE (SKV_ERR_CUDA if synchronisation fails). *flags_host
+ * (optional) receives the raw bits: 1 overflow, 2 bad page id, 4 lens above
+ * capacity, 8 a bounded wait gave up.
  */
 skv_status skv_workspace_error(const void *workspace, void *stream, uint32_t *flags_host);
 

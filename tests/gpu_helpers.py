@@ -25,9 +25,10 @@ def pool_for_units(entries_per_unit, B, Hkv, d, dtype, shuffle=False, seed=0, sp
     pages = [max(1, -(-int(e) // skv.PAGE_NODES)) for e in entries_per_unit]
     table, total = workloads.page_assignment(B, Hkv, pages, shuffle, seed)
     pool = skv.NodePool(total + spare_pages, d, dtype, device=device)
-    pool.k.zero_()
-    pool.v.zero_()
-    pool.ab.zero_()
+    # slots no entry uses hold NaN: a kernel that lets them leak into a result fails the checks
+    pool.k.fill_(float("nan"))
+    pool.v.fill_(float("nan"))
+    pool.ab.fill_(float("nan"))
     return pool, table.to(device)
 
 
