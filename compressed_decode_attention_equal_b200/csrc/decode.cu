@@ -11,17 +11,20 @@
 // bf16 path (k_decode_split, one launch per call), split-K over pages:
 //  * the flat page space of all (unit, row-pass) "virtual units" is cut into
 //    ncta equal ranges (one per CTA, a stream-K style split), so every CTA
-//    streams the same number of 16-node pages whatever the length mix;
+//    streams the same number of 16-node pages whatever the length mix; the
+//    part of one virtual unit inside one CTA's range is a "piece";
 //  * one producer warp copies each page (K 4 KB, V 4 KB, alpha/beta 128 B at
-//    d = 128) with three TMA bulk copies into an 8-stage mbarrier ring;
+//    d = 128) with three TMA bulk copies into an 8-stage mbarrier ring, and
+//    each piece's query rows into a double-buffered slot;
 //  * four consumer warps run the GQA group's query rows through tensor cores:
 //    S^T = K Q^T with nodes as the M = 16 dimension and up to 8 query rows as
 //    N = 8 (a GQA group of 7 rows wastes 1/8), softmax on the accumulator, P^T
 //    transposed in registers (movmatrix) into the B operand of O^T = V^T P^T;
 //  * a piece that covers a whole unit writes out / lse directly; pieces of a
-//    unit split across CTAs write (lse, out) partials, and the CTA that
-//    finishes a unit last (an atomic per-unit counter, reset after use) merges
-//    them with a log-sum-exp;
+//    unit split across CTAs write normalised partials (out, log2 partition);
+//    after streaming, each CTA counts its split pieces in per-unit counters,
+//    and the CTA that completes a unit merges its pieces (log-sum-exp) and
+//    resets the counter;
 //  * launched with programmatic stream serialisation: the next launch's CTAs
 //    become resident while this grid drains; each grid reads its inputs only
 //    after griddepcontrol.wait, so data from any preceding kernel is visible.
@@ -37,23 +40,32 @@ namespace skv {
 
 constexpr int kDecConsumers = 4;
 constexpr int kDecThreads = (kDecConsumers + 1) * 32;
+// Ring depth: a multiple of every page-group count (1, 2, 4), so that the pages i and
+// i + kDecStages that share a stage always go to the same consumer warp, in order. A warp that
+// could poll a stage for page i + kDecStages while it still held page i would see the previous
+// phase's parity as complete (mbarrier parity aliasing) and read stale data.
 constexpr int kDecStages = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 template <int D>
 struct PageGeom {
-    static constexpr int ROWB = D * 2;                 // bytes of one bf16 node vector
+    static constexpr int ROWB = D * 2;                    // bytes of one bf16 node vector
     static constexpr int VEC_BYTES = kPageNodes * ROWB;   // K (or V) bytes of a page
     static constexpr int AB_BYTES = kPageNodes * 8;
     static constexpr int STAGE = 2 * VEC_BYTES + AB_BYTES;
 };
 
-template <int D>
-constexpr size_t dec_smem_fixed() {
-    return 16 /*align*/ + kDecStages * PageGeom<D>::STAGE + 2 * kDecStages * 8 + kDecStages * 4 +
-           kDecConsumers * 8 * (D + 2) * 4;
-}
+template <int D, int NT>
+struct SplitSmem {
+    static constexpr int QROWB = D * 2 + 16;              // padded query row: conflict-free ldmatrix
+    static constexpr int QBUF = NT * 8 * QROWB;           // the query rows of one piece
+    static constexpr int STAGES_BYTES = kDecStages * PageGeom<D>::STAGE;
+    static constexpr int MBUF_FLOATS = kDecConsumers * 8 * (D + 2);
+    static constexpr int BARS = 2 * kDecStages + 4;
+    static constexpr size_t FIXED =
+        16 + STAGES_BYTES + 2 * QBUF + BARS * 8 + kDecStages * 4 + MBUF_FLOATS * 4 + 16 * 4;
+};
 
 __device__ __forceinline__ int clamp_entries(const DecodeArgs &a, int u) {
     int L = a.lens[u];
@@ -88,7 +100,6 @@ __device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, i
         prefix[v] = pages;   // page count for now; made exclusive below
         local += pages;
     }
-    // block exclusive scan of `local`
     const int lane = tid & 31, warp = tid >> 5;
     int x = local;
 #pragma unroll
@@ -116,66 +127,184 @@ __device__ __forceinline__ long long cta_of(long long f, long long ptot, int nct
     return ((f + 1) * ncta + ptot - 1) / ptot - 1;
 }
 
-// Log-sum-exp merge of every piece of virtual unit v (run by the CTA that completed it).
+// Pieces of the unit covering flat pages [ps, pe): their count, and the partial-slot code
+// (cta * 2 + slot) of piece i. With ptot >= ncta every CTA range is nonempty: the pieces sit in
+// CTAs c_first..c_last, the first in its tail slot (1), the others in their head slot (0). With
+// ptot < ncta every nonempty range holds exactly one page: piece i is page ps + i's CTA.
+__device__ __forceinline__ int piece_count(long long ps, long long pe, long long ptot, int ncta) {
+    if (ptot < ncta) return static_cast<int>(pe - ps);
+    return static_cast<int>(cta_of(pe - 1, ptot, ncta) - cta_of(ps, ptot, ncta) + 1);
+}
+
+__device__ __forceinline__ int piece_code(int i, long long ps, long long ptot, int ncta, long long c_first) {
+    const long long c = ptot < ncta ? cta_of(ps + i, ptot, ncta) : c_first + i;
+    return static_cast<int>(c * 2 + (i == 0 ? 1 : 0));
+}
+
+// Log-sum-exp merge of the n pieces (partial-slot codes in shared memory) of virtual unit v,
+// by the CTA that completed it: one warp per query row, lanes over dimensions. Up to kFastPieces
+// pieces, every load of two rows is issued before any is used (one round trip to L2).
+constexpr int kFastPieces = 6;
+
 template <int D>
-__device__ void merge_unit(const DecodeArgs &a, int v, int b, int h, int rpass, long long ps, long long pe,
-                           long long ptot, int tid, int nth) {
-    const long long c_first = cta_of(ps, ptot, a.ncta), c_last = cta_of(pe - 1, ptot, a.ncta);
+__device__ __forceinline__ void merge_store(const DecodeArgs &a, int b, int h, int row, int lane, const float *acc,
+                                            float M, float Ls) {
+    constexpr int DPL = D / 32;
+    const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
+    const float inv = Ls > 0.0f ? 1.0f / Ls : 0.0f;
+    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) + oi * D + lane * DPL;
+    if constexpr (DPL == 4) {
+        uint2 w;
+        w.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+        w.y = pack_bf16x2(acc[2] * inv, acc[3] * inv);
+        *reinterpret_cast<uint2 *>(dst) = w;
+    } else {
+        *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
+    }
+    if (lane == 0) a.lse[oi] = Ls > 0.0f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
+}
+
+template <int D>
+__device__ void merge_unit(const DecodeArgs &a, int v, const int *codes, int n, int warp, int lane) {
+    constexpr int DPL = D / 32;   // dimensions per lane
+    const int u = v / a.row_passes, rpass = v % a.row_passes;
+    const int b = u / a.Hkv, h = u % a.Hkv;
     const int rows_here = min(a.pass_rows, a.rows - rpass * kRowsPerPass);
-    __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(a.out);
-    for (int idx = tid; idx < rows_here * D; idx += nth) {
-        const int rr = idx / D, dim = idx % D;
-        const int row = rpass * kRowsPerPass + rr;
+    if (n <= kFastPieces) {
+        for (int r0 = warp; r0 < rows_here; r0 += 2 * kDecConsumers) {
+            float lv[2][kFastPieces], xv[2][kFastPieces][DPL];
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int rr = r0 + t * kDecConsumers;
+#pragma unroll
+                for (int i = 0; i < kFastPieces; ++i) {
+                    lv[t][i] = -INFINITY;
+#pragma unroll
+                    for (int j = 0; j < DPL; ++j) xv[t][i][j] = 0.0f;
+                    if (i < n && rr < rows_here) {
+                        const long long pr = static_cast<long long>(codes[i]) * a.pass_rows + rr;
+                        lv[t][i] = __ldcg(a.part_l + pr);
+                        const float *src = a.part_v + pr * D + lane * DPL;
+                        if constexpr (DPL == 4) {
+                            const float4 x = __ldcg(reinterpret_cast<const float4 *>(src));
+                            xv[t][i][0] = x.x; xv[t][i][1] = x.y; xv[t][i][2] = x.z; xv[t][i][3] = x.w;
+                        } else {
+                            const float2 x = __ldcg(reinterpret_cast<const float2 *>(src));
+                            xv[t][i][0] = x.x; xv[t][i][1] = x.y;
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < 2; ++t) {
+                const int rr = r0 + t * kDecConsumers;
+                if (rr >= rows_here) continue;
+                float M = -INFINITY;
+#pragma unroll
+                for (int i = 0; i < kFastPieces; ++i) M = fmaxf(M, lv[t][i]);
+                const float Mb = M == -INFINITY ? 0.0f : M;
+                float acc[DPL], Ls = 0.0f;
+#pragma unroll
+                for (int j = 0; j < DPL; ++j) acc[j] = 0.0f;
+#pragma unroll
+                for (int i = 0; i < kFastPieces; ++i) {
+                    const float w = ex2(lv[t][i] - Mb);   // -inf (absent piece) gives 0
+                    Ls += w;
+#pragma unroll
+                    for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w, xv[t][i][j], acc[j]);
+                }
+                merge_store<D>(a, b, h, rpass * kRowsPerPass + rr, lane, acc, M, Ls);
+            }
+        }
+        return;
+    }
+    for (int rr = warp; rr < rows_here; rr += kDecConsumers) {
         float M = -INFINITY;
-        for (long long cc = c_first; cc <= c_last; ++cc) {
-            const long long a_c = cta_begin(cc, ptot, a.ncta);
-            if (a_c >= cta_begin(cc + 1, ptot, a.ncta)) continue;   // an empty range wrote no partial
-            const int slot = ps < a_c ? 0 : 1;
-            M = fmaxf(M, __ldcg(a.part + ((cc * 2 + slot) * a.pass_rows + rr) * (D + 1)));
+        for (int base = 0; base < n; base += 32) {
+            const int i = base + lane;
+            M = fmaxf(M, i < n ? __ldcg(a.part_l + static_cast<long long>(codes[i]) * a.pass_rows + rr) : -INFINITY);
         }
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
         const float Mb = M == -INFINITY ? 0.0f : M;
-        float Ls = 0.0f, Os = 0.0f;
-        for (long long cc = c_first; cc <= c_last; ++cc) {
-            const long long a_c = cta_begin(cc, ptot, a.ncta);
-            if (a_c >= cta_begin(cc + 1, ptot, a.ncta)) continue;
-            const int slot = ps < a_c ? 0 : 1;
-            const float *pp = a.part + ((cc * 2 + slot) * a.pass_rows + rr) * (D + 1);
-            const float w = ex2(__ldcg(pp) - Mb);
-            Ls += w;
-            Os = fmaf(__ldcg(pp + 1 + dim), w, Os);
+        float acc[DPL], Ls = 0.0f;
+#pragma unroll
+        for (int j = 0; j < DPL; ++j) acc[j] = 0.0f;
+        for (int base = 0; base < n; base += 32) {
+            const int i = base + lane;
+            const float wi =
+                i < n ? ex2(__ldcg(a.part_l + static_cast<long long>(codes[i]) * a.pass_rows + rr) - Mb) : 0.0f;
+            Ls += wi;
+            const int cnt = min(32, n - base);
+#pragma unroll 4
+            for (int k = 0; k < cnt; ++k) {
+                const float w = __shfl_sync(0xffffffffu, wi, k);
+                const float *src =
+                    a.part_v + (static_cast<long long>(codes[base + k]) * a.pass_rows + rr) * D + lane * DPL;
+                if constexpr (DPL == 4) {
+                    const float4 x = __ldcg(reinterpret_cast<const float4 *>(src));
+                    acc[0] = fmaf(w, x.x, acc[0]);
+                    acc[1] = fmaf(w, x.y, acc[1]);
+                    acc[2] = fmaf(w, x.z, acc[2]);
+                    acc[3] = fmaf(w, x.w, acc[3]);
+                } else {
+                    const float2 x = __ldcg(reinterpret_cast<const float2 *>(src));
+                    acc[0] = fmaf(w, x.x, acc[0]);
+                    acc[1] = fmaf(w, x.y, acc[1]);
+                }
+            }
         }
-        const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
-        outp[oi * D + dim] = __float2bfloat16_rn(Ls > 0.0f ? __fdividef(Os, Ls) : 0.0f);
-        if (dim == 0) a.lse[oi] = Ls > 0.0f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
+#pragma unroll
+        for (int off = 16; off > 0; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
+        merge_store<D>(a, b, h, rpass * kRowsPerPass + rr, lane, acc, M, Ls);
     }
 }
 
 template <int D, int NT>
 __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArgs a) {
     using G = PageGeom<D>;
+    using L = SplitSmem<D, NT>;
     constexpr int PG = kDecConsumers / NT;   // page groups: warps sharing a row tile split the pages
     constexpr int NKS = D / 16;              // QK k-steps over dims == PV m-tiles over dims
+    static_assert(kDecStages % PG == 0, "a stage's successive pages must go to one consumer warp");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((16 - (smem_u32(smem_raw) & 15)) & 15);
     uint8_t *stages = smem;
-    uint64_t *full = reinterpret_cast<uint64_t *>(stages + kDecStages * G::STAGE);
+    uint8_t *qbuf = stages + L::STAGES_BYTES;
+    uint64_t *full = reinterpret_cast<uint64_t *>(qbuf + 2 * L::QBUF);
     uint64_t *empty = full + kDecStages;
-    int *svalid = reinterpret_cast<int *>(empty + kDecStages);
+    uint64_t *qfull = empty + kDecStages;
+    uint64_t *qempty = qfull + 2;
+    int *svalid = reinterpret_cast<int *>(qempty + 2);
     float *mbuf = reinterpret_cast<float *>(svalid + kDecStages);
-    int *prefix = reinterpret_cast<int *>(mbuf + kDecConsumers * 8 * (D + 2));
+    int *misc = reinterpret_cast<int *>(mbuf + L::MBUF_FLOATS);
+    int *prefix = misc + 16;
     __shared__ int scan_scratch[kDecThreads / 32];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nv = a.n_vunits;
+    if (tid == 0) {   // independent of the inputs: overlaps the wait below
+        for (int s = 0; s < kDecStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&empty[s], NT);
+        }
+        for (int s = 0; s < 2; ++s) {
+            mbar_init(&qfull[s], 1);
+            mbar_init(&qempty[s], kDecConsumers);
+        }
+        fence_mbar_init();
+    }
+    for (int i = tid; i < 2 * L::QBUF / 4; i += kDecThreads) reinterpret_cast<uint32_t *>(qbuf)[i] = 0u;
     // let the next launch in the stream become resident as our CTAs retire; then wait for every
     // preceding grid to complete (its writes visible) before reading any input
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    build_prefix(a, prefix, scan_scratch);
+    build_prefix(a, prefix, scan_scratch);   // ends with __syncthreads: barriers and qbuf are ready
     const long long ptot = prefix[nv];
     const long long ra = ptot * blockIdx.x / a.ncta;
     const long long rb = ptot * (blockIdx.x + 1) / a.ncta;
+    __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(a.out);
     // units with no entries get out = 0, lse = -inf (spread over the CTAs)
     for (int v = blockIdx.x; v < nv; v += a.ncta) {
         if (prefix[v + 1] != prefix[v]) continue;
@@ -186,37 +315,51 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
             const int row = rpass * kRowsPerPass + rr;
             if (row >= a.rows) continue;
             const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
-            static_cast<__nv_bfloat16 *>(a.out)[oi * D + dim] = __float2bfloat16_rn(0.0f);
+            outp[oi * D + dim] = __float2bfloat16_rn(0.0f);
             if (dim == 0) a.lse[oi] = -INFINITY;
         }
     }
     if (ra >= rb) return;
     const int v0 = find_vunit(prefix, nv, ra);
     const int n_my = static_cast<int>(rb - ra);
-
-    if (tid == 0) {
-        for (int s = 0; s < kDecStages; ++s) {
-            mbar_init(&full[s], 1);
-            mbar_init(&empty[s], NT);
-        }
-        fence_mbar_init();
-    }
-    __syncthreads();
+    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
 
     if (warp == kDecConsumers) {
         // ----------------------------- producer -----------------------------
         bool alive = true;
+        int v = -1, pi = -1;   // current (nonempty) piece
         for (int base = 0; base < n_my && alive; base += 32) {
             int my_page = -1;
             if (base + lane < n_my) {
                 const long long f = ra + base + lane;
-                const int v = find_vunit(prefix, nv, f);
-                const int u = v / a.row_passes;
-                my_page = a.page_table[static_cast<long long>(u) * a.max_pages + (f - prefix[v])];
+                const int vv = find_vunit(prefix, nv, f);
+                my_page = a.page_table[static_cast<long long>(vv / a.row_passes) * a.max_pages + (f - prefix[vv])];
             }
             const int cnt = min(32, n_my - base);
             for (int k = 0; k < cnt; ++k) {
                 const int i = base + k;
+                const long long f = ra + i;
+                if (v < 0 || f >= prefix[v + 1]) {
+                    // first page of the next piece: copy its query rows first
+                    v = find_vunit(prefix, nv, f);
+                    ++pi;
+                    const int slot = pi & 1;
+                    if (pi >= 2 && !mbar_wait(&qempty[slot], ((pi >> 1) - 1) & 1)) {
+                        if (lane == 0) raise_flag(a.flags, FLAG_TIMEOUT);
+                        alive = false;
+                        break;
+                    }
+                    const int u = v / a.row_passes, rpass = v % a.row_passes;
+                    const int b = u / a.Hkv, h = u % a.Hkv;
+                    const int p0 = rpass * kRowsPerPass, p1 = min(p0 + a.pass_rows, a.rows);
+                    if (lane == 0) mbar_arrive_expect_tx(&qfull[slot], (p1 - p0) * D * 2);
+                    __syncwarp();
+                    for (int row = p0 + lane; row < p1; row += 32) {
+                        const __nv_bfloat16 *src =
+                            q + ((static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G) * D;
+                        bulk_g2s(qbuf + slot * L::QBUF + (row - p0) * L::QROWB, src, D * 2, &qfull[slot]);
+                    }
+                }
                 const int s = i % kDecStages;
                 const int phys = __shfl_sync(0xffffffffu, my_page, k);
                 if (i >= kDecStages && !mbar_wait(&empty[s], ((i / kDecStages) - 1) & 1)) {
@@ -249,39 +392,39 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
     // ------------------------------- consumers -------------------------------
     const int nt = warp % NT, pg = warp / NT;
     const int g = lane >> 2, c = lane & 3;
+    const int ctid = tid;   // 0 .. 127
     const float c_scale = kLog2e * rsqrtf(static_cast<float>(D));
-    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
-    __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(a.out);
-    int i0 = 0;
+    int i0 = 0, pi = 0;
     bool alive = true;
+    int split_v[2] = {0, 0}, split_ps[2] = {0, 0}, split_pe[2] = {0, 0}, n_split = 0;   // (thread 0)
     for (int v = v0; v < nv && prefix[v] < rb; ++v) {
         const long long ps = prefix[v], pe = prefix[v + 1];
         const int lo = static_cast<int>(max(ra, ps) - ps), hi = static_cast<int>(min(rb, pe) - ps);
         const int npg = hi - lo;
+        if (npg <= 0) continue;   // an empty unit: written in the prologue
         const int u = v / a.row_passes, rpass = v % a.row_passes;
         const int b = u / a.Hkv, h = u % a.Hkv;
-        const int L = clamp_entries(a, u);
+        const int Lent = clamp_entries(a, u);
 
-        // Q^T fragments of rows rpass*32 + nt*8 + g, and |q|^2 of rows 2c, 2c+1
-        const int my_row = rpass * kRowsPerPass + nt * 8 + g;
-        const bool row_ok = (nt * 8 + g) < a.pass_rows && my_row < a.rows;
+        // Q^T fragments of rows nt*8 + g of this piece (ldmatrix from the producer's copy), |q|^2
         uint32_t qf[NKS][2];
         float qn = 0.0f;
         {
-            const __nv_bfloat16 *qr = q;
-            if (row_ok) {
-                const int r = my_row / a.G, gg = my_row % a.G;
-                qr = q + ((static_cast<long long>(b) * a.R + r) * a.Hq + h * a.G + gg) * D;
+            const int slot = pi & 1;
+            if (alive && !mbar_wait(&qfull[slot], (pi >> 1) & 1)) {
+                if (lane == 0) raise_flag(a.flags, FLAG_TIMEOUT);
+                alive = false;
             }
+            const uint32_t qb = smem_u32(qbuf + slot * L::QBUF) + (nt * 8 + (lane & 7)) * L::QROWB;
+#pragma unroll
+            for (int k2 = 0; k2 < NKS / 2; ++k2)
+                ldsm_x4(qb + ((4 * k2 + (lane >> 3)) << 4), qf[2 * k2][0], qf[2 * k2][1], qf[2 * k2 + 1][0],
+                        qf[2 * k2 + 1][1]);
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&qempty[slot]);
 #pragma unroll
             for (int ks = 0; ks < NKS; ++ks) {
-                uint32_t w0 = 0, w1 = 0;
-                if (row_ok) {
-                    w0 = *reinterpret_cast<const uint32_t *>(qr + 16 * ks + 2 * c);
-                    w1 = *reinterpret_cast<const uint32_t *>(qr + 16 * ks + 8 + 2 * c);
-                }
-                qf[ks][0] = w0;
-                qf[ks][1] = w1;
+                const uint32_t w0 = qf[ks][0], w1 = qf[ks][1];
                 qn = fmaf(bf16lo(w0), bf16lo(w0), qn);
                 qn = fmaf(bf16hi(w0), bf16hi(w0), qn);
                 qn = fmaf(bf16lo(w1), bf16lo(w1), qn);
@@ -298,7 +441,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
 #pragma unroll
         for (int mt = 0; mt < NKS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.0f;
 
-        for (int k = pg; k < npg && alive; k += PG) {
+        // page i of the CTA's range goes to page group i % PG (global index, not piece-local)
+        for (int k = ((pg - i0 % PG) + PG) % PG; k < npg && alive; k += PG) {
             const int i = i0 + k;
             const int s = i % kDecStages;
             if (!mbar_wait(&full[s], (i / kDecStages) & 1)) {
@@ -307,7 +451,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                 break;
             }
             if (svalid[s]) {
-                const int nvalid = min(kPageNodes, L - (lo + k) * kPageNodes);
+                const int nvalid = min(kPageNodes, Lent - (lo + k) * kPageNodes);
                 const uint32_t kb = smem_u32(stages + s * G::STAGE);
                 const uint32_t vb = kb + G::VEC_BYTES;
                 const float2 *ab = reinterpret_cast<const float2 *>(stages + s * G::STAGE + 2 * G::VEC_BYTES);
@@ -372,7 +516,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                         // slots past the unit's last entry may hold anything (NaN included):
                         // zero their V^T elements, since P = 0 does not cancel NaN in the product.
                         // This thread's fragment holds nodes 2c, 2c+1 (a0..a3) and 2c+8, 2c+9 (a4..a7).
-                        const uint32_t m_lo = (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
+                        const uint32_t m_lo =
+                            (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
                         const uint32_t m_hi =
                             (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
 #pragma unroll
@@ -389,14 +534,14 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
             if (lane == 0) mbar_arrive(&empty[s]);
         }
         i0 += npg;
+        ++pi;
 
         // ---- piece epilogue: merge the page groups through shared memory ----
-        l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], 4);
-        l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], 4);
-        l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], 8);
-        l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], 8);
-        l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], 16);
-        l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], 16);
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
+            l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
+        }
         float *mw = mbuf + warp * 8 * (D + 2);
 #pragma unroll
         for (int mt = 0; mt < NKS; ++mt) {
@@ -414,7 +559,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
         asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
         const bool complete = (ps >= ra) && (pe <= rb);
         const int slot = ps < ra ? 0 : 1;
-        const int ctid = tid;   // 0 .. 127
         for (int idx = ctid; idx < NT * 8 * D; idx += kDecConsumers * 32) {
             const int rr = idx / D, dim = idx % D;
             const int ntr = rr >> 3, j = rr & 7;
@@ -435,36 +579,58 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
             const float val = Ls > 0.0f ? __fdividef(Os, Ls) : 0.0f;
             const float lse2 = Ls > 0.0f ? M + __log2f(Ls) : -INFINITY;
             if (complete) {
-                const int r = row / a.G, gg = row % a.G;
-                const long long oi = (static_cast<long long>(b) * a.R + r) * a.Hq + h * a.G + gg;
+                const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
                 outp[oi * D + dim] = __float2bfloat16_rn(val);
                 if (dim == 0) a.lse[oi] = lse2 * kLn2;
             } else {
-                float *pp = a.part + ((static_cast<long long>(blockIdx.x) * 2 + slot) * a.pass_rows + rr) * (D + 1);
-                pp[1 + dim] = val;
-                if (dim == 0) pp[0] = lse2;
+                const long long pr = (static_cast<long long>(blockIdx.x) * 2 + slot) * a.pass_rows + rr;
+                a.part_v[pr * D + dim] = val;
+                if (dim == 0) a.part_l[pr] = lse2;
             }
         }
-        if (!complete) {
-            // publish this piece; the CTA that completes the unit merges all of its pieces
+        if (!complete && ctid == 0 && n_split < 2) {
+            split_v[n_split] = v;
+            split_ps[n_split] = static_cast<int>(ps);
+            split_pe[n_split] = static_cast<int>(pe);
+            ++n_split;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));   // mbuf free for the next piece
+    }
+
+    // ---- count this CTA's split pieces; merge the units it completes ----
+    // (the barrier above ordered every thread's partial stores before thread 0's fence)
+    int *pend = misc;   // pend[0] = count, then (v, ps, pe) per unit to merge
+    if (ctid == 0) {
+        int np = 0;
+        if (n_split > 0) {
             __threadfence();
-            asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
-            int *last = reinterpret_cast<int *>(mbuf);   // mbuf is free again after the barrier
-            if (ctid == 0) {
-                const long long c_first = cta_of(ps, ptot, a.ncta), c_last = cta_of(pe - 1, ptot, a.ncta);
-                int pieces = 0;
-                for (long long cc = c_first; cc <= c_last; ++cc) pieces += cta_begin(cc, ptot, a.ncta) <
-                                                                            cta_begin(cc + 1, ptot, a.ncta);
-                const int prev = atomicAdd(a.counters + v, 1);
-                *last = (prev == pieces - 1) ? 1 : 0;
-            }
-            asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
-            if (*last) {
-                __threadfence();
-                merge_unit<D>(a, v, b, h, rpass, ps, pe, ptot, ctid, kDecConsumers * 32);
-                if (ctid == 0) a.counters[v] = 0;   // ready for the next call
+            // both counters in flight at once: one round trip
+            const int prev0 = atomicAdd(a.counters + split_v[0], 1);
+            const int prev1 = n_split > 1 ? atomicAdd(a.counters + split_v[1], 1) : 0;
+            for (int k = 0; k < n_split; ++k) {
+                if ((k == 0 ? prev0 : prev1) == piece_count(split_ps[k], split_pe[k], ptot, a.ncta) - 1) {
+                    pend[1 + 3 * np] = split_v[k];
+                    pend[2 + 3 * np] = split_ps[k];
+                    pend[3 + 3 * np] = split_pe[k];
+                    ++np;
+                }
             }
         }
+        pend[0] = np;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
+    const int np = pend[0];
+    int *codes = reinterpret_cast<int *>(mbuf);
+    for (int k = 0; k < np; ++k) {
+        const int v = pend[1 + 3 * k];
+        const long long ps = pend[2 + 3 * k], pe = pend[3 + 3 * k];
+        const int n = piece_count(ps, pe, ptot, a.ncta);
+        const long long c_first = cta_of(ps, ptot, a.ncta);
+        for (int i = ctid; i < n; i += kDecConsumers * 32) codes[i] = piece_code(i, ps, ptot, a.ncta, c_first);
+        __threadfence();   // acquire: the other pieces' partials are visible after their counts
+        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
+        merge_unit<D>(a, v, codes, n, warp, lane);
+        if (ctid == 0) a.counters[v] = 0;   // ready for the next call
         asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
     }
 }
@@ -536,7 +702,7 @@ __global__ void __launch_bounds__(128) k_decode_f32(const DecodeArgs a) {
 // ---------------------------------------------------------------------------
 template <int D, int NT>
 static size_t split_smem(int n_vunits) {
-    return dec_smem_fixed<D>() + static_cast<size_t>(n_vunits + 1) * 4;
+    return SplitSmem<D, NT>::FIXED + static_cast<size_t>(n_vunits + 1) * 4;
 }
 
 // Grid size of the split kernel for one (device, shared-memory size): SMs x resident CTAs.

@@ -205,8 +205,10 @@ skv_status plan_decode(int dtype, int B, int R, int Hq, int Hkv, int d, int max_
     size_t off = kWsHeader;
     p.lay.counters = off;
     off += align256(static_cast<size_t>(nv) * 4);
-    p.lay.part = off;
-    if (dtype == SKV_BF16) off += align256(static_cast<size_t>(kMaxDecodeCtas) * 2 * p.pass_rows * (d + 1) * 4);
+    p.lay.part_v = off;
+    if (dtype == SKV_BF16) off += align256(static_cast<size_t>(kMaxDecodeCtas) * 2 * p.pass_rows * d * 4);
+    p.lay.part_l = off;
+    if (dtype == SKV_BF16) off += align256(static_cast<size_t>(kMaxDecodeCtas) * 2 * p.pass_rows * 4);
     p.lay.total = off;
     *plan = p;
     return SKV_OK;
@@ -346,7 +348,8 @@ skv_status skv_decode_attn(const void *q, skv_dtype dtype, int B, int R, int Hq,
     a.row_passes = plan.row_passes;
     a.pass_rows = plan.pass_rows;
     a.n_vunits = plan.n_vunits;
-    a.part = reinterpret_cast<float *>(ws + plan.lay.part);
+    a.part_v = reinterpret_cast<float *>(ws + plan.lay.part_v);
+    a.part_l = reinterpret_cast<float *>(ws + plan.lay.part_l);
     a.counters = reinterpret_cast<int32_t *>(ws + plan.lay.counters);
     a.flags = reinterpret_cast<uint32_t *>(ws);
     const cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream));

@@ -92,13 +92,14 @@ struct DecodeArgs {
     int pass_rows;    // rows a pass holds: min(kRowsPerPass, rows rounded up to 8)
     int n_vunits;     // B * Hkv * row_passes
     int ncta;         // CTAs of the split kernel
-    float *part;      // [ncta][2][pass_rows][d + 1] split partials
+    float *part_v;    // [ncta][2][pass_rows][d] split partial outputs (normalised)
+    float *part_l;    // [ncta][2][pass_rows] split partial log2-partitions
     int32_t *counters;   // [n_vunits] pieces finished per virtual unit (zero between calls)
     uint32_t *flags;
 };
 
 struct DecodeLayout {
-    size_t counters, part, total;
+    size_t counters, part_v, part_l, total;
 };
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);

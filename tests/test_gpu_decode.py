@@ -106,3 +106,33 @@ def test_decode_lens_above_capacity_is_clamped_and_flagged():
     skv.decode_attn(q, Hkv, pool, table, lens_bad, workspace=ws)
     st, flags = skv.workspace_error(ws)
     assert flags & skv._lib.FLAG_BAD_LENS
+
+
+def test_decode_repeated_calls_at_bench_shape_are_identical():
+    """The 7B-shaped 3.5% workload's launch configuration (32 x 4 units of 1,147 entries, split
+    across every CTA): 24 back-to-back calls alternating two caches give bit-identical outputs,
+    and sampled units match the oracle. Catches pipeline races that depend on timing."""
+    B, Hq, Hkv, d = 32, 28, 4, 128
+    lens = [1147] * B
+    caches = [_synthetic(B, Hq, Hkv, 1, d, lens, torch.bfloat16, seed=100 + i, shuffle=False) for i in range(2)]
+    ws = torch.zeros(skv.decode_workspace_bytes(B, 1, Hq, Hkv, d, caches[0][1].shape[2]), dtype=torch.uint8,
+                     device="cuda")
+    firsts = [None, None]
+    outs = [(torch.empty_like(c[3]), torch.empty(B, 1, Hq, dtype=torch.float32, device="cuda")) for c in caches]
+    for it in range(24):
+        pool, table, ln, q = caches[it % 2]
+        out, lse = outs[it % 2]
+        skv.decode_attn(q, Hkv, pool, table, ln, out=out, lse=lse, workspace=ws)
+        if firsts[it % 2] is None:
+            torch.cuda.synchronize()
+            firsts[it % 2] = (out.clone(), lse.clone())
+        elif it >= 22:
+            torch.cuda.synchronize()
+            assert torch.equal(out, firsts[it % 2][0]) and torch.equal(lse, firsts[it % 2][1])
+    st, flags = skv.workspace_error(ws)
+    assert st == 0, flags
+    pool, table, ln, q = caches[0]
+    sample = [0, 13, 31]
+    units = gpu_units(pool, table, ln, B, Hkv)
+    ref_out, ref_lse = oracle.decode(q[sample].double().cpu().numpy(), [units[b] for b in sample])
+    check_decode(firsts[0][0][sample], firsts[0][1][sample], ref_out, ref_lse, torch.bfloat16, "bench shape")
