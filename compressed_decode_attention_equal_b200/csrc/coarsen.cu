@@ -71,7 +71,8 @@ constexpr int kZStride = 20;                     // floats per row of the z buff
 
 template <int D>
 constexpr size_t k1_smem_bytes() {
-    return 1024 /*alignment slack*/ + kK1Stages * kK1StageBytes + 2 * D * kProjDim * sizeof(float) + 64 + 64;
+    // stages + P^T with one zero row of padding (the pipelined loop reads row j + 1) + barriers
+    return 1024 /*alignment slack*/ + kK1Stages * kK1StageBytes + (2 * D + 1) * kProjDim * sizeof(float) + 64 + 64;
 }
 
 template <int D, typename T>
@@ -89,7 +90,7 @@ __global__ void __launch_bounds__(kK1Threads, 2)
     uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
     uint8_t *stages = smem;
     float *pt = reinterpret_cast<float *>(smem + kK1Stages * kK1StageBytes);
-    uint64_t *bar = reinterpret_cast<uint64_t *>(pt + 2 * D * kProjDim);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(pt + (2 * D + 1) * kProjDim);
     long long *warp_sum = reinterpret_cast<long long *>(bar + 8);
 
     const int u = blockIdx.y;
@@ -110,40 +111,53 @@ __global__ void __launch_bounds__(kK1Threads, 2)
             tma_load_2d(stages + c * kK1StageBytes, c < KCHUNK ? &map_k : &map_v, (c % KCHUNK) * JPC, y0, &bar[c]);
         }
     }
-    for (int i = tid; i < 2 * D * kProjDim; i += kK1Threads) pt[i] = proj.pt[i];
+    for (int i = tid; i < (2 * D + 1) * kProjDim; i += kK1Threads) pt[i] = i < 2 * D * kProjDim ? proj.pt[i] : 0.0f;
     __syncthreads();
 
-    const uint32_t pt_addr = smem_u32(pt);
     const int r0 = tid, r1 = tid + kK1Threads;
     uint64_t acc0[kProjDim / 2], acc1[kProjDim / 2];
 #pragma unroll
     for (int i = 0; i < kProjDim / 2; ++i) acc0[i] = acc1[i] = 0ull;
+    const float4 *ptv = reinterpret_cast<const float4 *>(pt);   // P^T row j = ptv[4 j .. 4 j + 3]
+    // software pipeline: the P^T row of feature j + 1 and the next 16-byte sub-chunk of both rows
+    // are read while feature j is accumulated (plain shared loads: never hoisted above the wait)
+    float4 pc[4];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) pc[q4] = ptv[q4];
 
     bool ok = true;
     for (int c = 0; c < NCHUNK; ++c) {
         const int s = c % kK1Stages;
         if (ok && !mbar_wait(&bar[s], (c / kK1Stages) & 1)) ok = false;
-        const uint32_t base = smem_u32(stages + s * kK1StageBytes);
+        const uint4 *st = reinterpret_cast<const uint4 *>(stages + s * kK1StageBytes);
+        uint4 xa = st[r0 * 8 + (0 ^ (r0 & 7))];
+        uint4 xb = st[r1 * 8 + (0 ^ (r1 & 7))];
 #pragma unroll 1
         for (int sc = 0; sc < 8; ++sc) {
-            const uint4 xa = lds128(base + r0 * 128 + ((sc ^ (r0 & 7)) << 4));
-            const uint4 xb = lds128(base + r1 * 128 + ((sc ^ (r1 & 7)) << 4));
+            const int scn = sc < 7 ? sc + 1 : 7;
+            const uint4 nxa = st[r0 * 8 + (scn ^ (r0 & 7))];
+            const uint4 nxb = st[r1 * 8 + (scn ^ (r1 & 7))];
 #pragma unroll
             for (int e = 0; e < EPS; ++e) {
                 const int j = c * JPC + sc * EPS + e;
+                float4 pn[4];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) pn[q4] = ptv[4 * (j + 1) + q4];
                 const float va = elem_of<T>(xa, e), vb = elem_of<T>(xb, e);
                 const uint64_t xa2 = f2pack(va, va), xb2 = f2pack(vb, vb);
-                const uint32_t prow = pt_addr + j * kProjDim * 4;
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) {
-                    const float4 p = lds128f(prow + q4 * 16);
-                    const uint64_t pa = f2pack(p.x, p.y), pb = f2pack(p.z, p.w);
+                    const uint64_t pa = f2pack(pc[q4].x, pc[q4].y), pb = f2pack(pc[q4].z, pc[q4].w);
                     acc0[2 * q4] = ffma2(pa, xa2, acc0[2 * q4]);
                     acc0[2 * q4 + 1] = ffma2(pb, xa2, acc0[2 * q4 + 1]);
                     acc1[2 * q4] = ffma2(pa, xb2, acc1[2 * q4]);
                     acc1[2 * q4 + 1] = ffma2(pb, xb2, acc1[2 * q4 + 1]);
                 }
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) pc[q4] = pn[q4];
             }
+            xa = nxa;
+            xb = nxb;
         }
         __syncthreads();
         if (tid == 0 && c + kK1Stages < NCHUNK) {
@@ -340,11 +354,11 @@ struct Vec16;   // 16 bytes of elements as fp32
 template <>
 struct Vec16<__nv_bfloat16> {
     static constexpr int N = 8;
-    __device__ static void load(const void *p, float (&x)[8]) {
-        const uint4 w = __ldg(reinterpret_cast<const uint4 *>(p));
+    __device__ static void cvt(const uint4 &w, float (&x)[8]) {
         x[0] = bf16lo(w.x); x[1] = bf16hi(w.x); x[2] = bf16lo(w.y); x[3] = bf16hi(w.y);
         x[4] = bf16lo(w.z); x[5] = bf16hi(w.z); x[6] = bf16lo(w.w); x[7] = bf16hi(w.w);
     }
+    __device__ static void load(const void *p, float (&x)[8]) { cvt(__ldg(reinterpret_cast<const uint4 *>(p)), x); }
     __device__ static void store(void *p, const float (&x)[8]) {
         uint4 w;
         w.x = pack_bf16x2(x[0], x[1]); w.y = pack_bf16x2(x[2], x[3]);
@@ -356,10 +370,11 @@ struct Vec16<__nv_bfloat16> {
 template <>
 struct Vec16<float> {
     static constexpr int N = 4;
-    __device__ static void load(const void *p, float (&x)[4]) {
-        const float4 w = __ldg(reinterpret_cast<const float4 *>(p));
-        x[0] = w.x; x[1] = w.y; x[2] = w.z; x[3] = w.w;
+    __device__ static void cvt(const uint4 &w, float (&x)[4]) {
+        x[0] = __uint_as_float(w.x); x[1] = __uint_as_float(w.y);
+        x[2] = __uint_as_float(w.z); x[3] = __uint_as_float(w.w);
     }
+    __device__ static void load(const void *p, float (&x)[4]) { cvt(__ldg(reinterpret_cast<const uint4 *>(p)), x); }
     __device__ static void store(void *p, const float (&x)[4]) {
         *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
     }
@@ -391,17 +406,31 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
     const uint8_t *kp = static_cast<const uint8_t *>(a.k) + row0 * ROWB + ch * 16;
     const uint8_t *vp = static_cast<const uint8_t *>(a.v) + row0 * ROWB + ch * 16;
 
+    // loads are issued kUnroll token steps at a time (2 x kUnroll 16-byte loads in flight per lane)
+    constexpr int kUnroll = 8;
     float sk[EPL], sv[EPL], x[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) sk[i] = sv[i] = 0.0f;
-#pragma unroll 4
-    for (int t = sub; t < m; t += TPS) {
-        Vec16<T>::load(kp + static_cast<int64_t>(t) * ROWB, x);
+    for (int t0 = sub; t0 < m; t0 += TPS * kUnroll) {
+        uint4 kw[kUnroll], vw[kUnroll];
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) sk[i] += x[i];
-        Vec16<T>::load(vp + static_cast<int64_t>(t) * ROWB, x);
+        for (int r = 0; r < kUnroll; ++r) {
+            const int t = t0 + r * TPS;
+            kw[r] = vw[r] = make_uint4(0u, 0u, 0u, 0u);   // zero bits: +0.0 in both dtypes
+            if (t < m) {
+                kw[r] = __ldg(reinterpret_cast<const uint4 *>(kp + static_cast<int64_t>(t) * ROWB));
+                vw[r] = __ldg(reinterpret_cast<const uint4 *>(vp + static_cast<int64_t>(t) * ROWB));
+            }
+        }
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) sv[i] += x[i];
+        for (int r = 0; r < kUnroll; ++r) {
+            Vec16<T>::cvt(kw[r], x);
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) sk[i] += x[i];
+            Vec16<T>::cvt(vw[r], x);
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) sv[i] += x[i];
+        }
     }
 #pragma unroll
     for (int off = CH; off < 32; off <<= 1)
@@ -416,16 +445,27 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
         sk[i] = __fdiv_rn(sk[i], fm);   // mean key
         sv[i] = __fdiv_rn(sv[i], fm);   // mean value
     }
+    // second pass over the keys (just read: served from L1 / L2)
     float q2[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) q2[i] = 0.0f;
-#pragma unroll 4
-    for (int t = sub; t < m; t += TPS) {
-        Vec16<T>::load(kp + static_cast<int64_t>(t) * ROWB, x);
+    for (int t0 = sub; t0 < m; t0 += TPS * kUnroll) {
+        uint4 kw[kUnroll];
 #pragma unroll
-        for (int i = 0; i < EPL; ++i) {
-            const float dv = x[i] - sk[i];
-            q2[i] = __fmaf_rn(dv, dv, q2[i]);
+        for (int r = 0; r < kUnroll; ++r) {
+            const int t = t0 + r * TPS;
+            kw[r] = make_uint4(0u, 0u, 0u, 0u);
+            if (t < m) kw[r] = __ldg(reinterpret_cast<const uint4 *>(kp + static_cast<int64_t>(t) * ROWB));
+        }
+#pragma unroll
+        for (int r = 0; r < kUnroll; ++r) {
+            if (t0 + r * TPS >= m) break;
+            Vec16<T>::cvt(kw[r], x);
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                const float dv = x[i] - sk[i];
+                q2[i] = __fmaf_rn(dv, dv, q2[i]);
+            }
         }
     }
     float var_lane = 0.0f;
