@@ -9,7 +9,7 @@
 //
 // Pipeline (stream-ordered launches, all integer stages exact):
 //   k_setup          copy the host-built per-sequence plan into the workspace
-//   k_project_scan   TMA-staged tiles of 255 middle tokens (+1 halo): z via the
+//   k_project_scan   TMA-staged tiles of 511 middle tokens (+1 halo): z via the
 //                    fixed fp32 fma recipe, D_t = rne(d_t 2^20), tile-local
 //                    inclusive int64 scan and tile totals
 //   k_tile_prefix    exclusive scan of tile totals per unit, c_T
@@ -35,21 +35,6 @@ __global__ void k_setup(const __grid_constant__ SeqTable table, SeqRow *dst, int
 // ---------------------------------------------------------------------------
 // k_project_scan
 // ---------------------------------------------------------------------------
-template <typename T>
-__device__ __forceinline__ float elem_of(const uint4 &w, int e);
-
-template <>
-__device__ __forceinline__ float elem_of<__nv_bfloat16>(const uint4 &w, int e) {
-    const uint32_t x = (e >> 1) == 0 ? w.x : (e >> 1) == 1 ? w.y : (e >> 1) == 2 ? w.z : w.w;
-    return (e & 1) ? bf16hi(x) : bf16lo(x);
-}
-
-template <>
-__device__ __forceinline__ float elem_of<float>(const uint4 &w, int e) {
-    const uint32_t x = e == 0 ? w.x : e == 1 ? w.y : e == 2 ? w.z : w.w;
-    return __uint_as_float(x);
-}
-
 // D = rne(||zc - zp||_2 * 2^20) by the fixed recipe (fp32, i ascending); -1 on overflow.
 __device__ __forceinline__ long long quantised_step(const float *zp, const float *zc) {
     float s = 0.0f;
@@ -65,9 +50,13 @@ __device__ __forceinline__ long long quantised_step(const float *zp, const float
 }
 
 constexpr int kK1Threads = 128;
+constexpr int kK1Tok = kTileRows / kK1Threads;   // token rows per thread (4)
 constexpr int kK1Stages = 2;
-constexpr int kK1StageBytes = kTileRows * 128;   // one 128-byte column chunk of 256 rows
+constexpr int kK1ColBytes = 64;                  // column chunk of every row per stage (64-byte swizzle)
+constexpr int kK1BoxRows = 256;                  // TMA box height (two boxes per stage)
+constexpr int kK1StageBytes = kTileRows * kK1ColBytes;
 constexpr int kZStride = 20;                     // floats per row of the z buffer (conflict-free)
+static_assert(kTileRows % kK1BoxRows == 0 && kTileRows * kZStride * 4 <= kK1Stages * kK1StageBytes, "tile");
 
 template <int D>
 constexpr size_t k1_smem_bytes() {
@@ -75,15 +64,43 @@ constexpr size_t k1_smem_bytes() {
     return 1024 /*alignment slack*/ + kK1Stages * kK1StageBytes + (2 * D + 1) * kProjDim * sizeof(float) + 64 + 64;
 }
 
+// x duplicated into both halves of an f32x2 operand, built with two different ALU operations (the
+// pair then needs no register move): the bf16 in the low / high half of a 32-bit word as fp32.
+__device__ __forceinline__ uint64_t dup_bf16lo(uint32_t w) {
+    return f2pack(__uint_as_float(w << 16), __uint_as_float(__byte_perm(w, 0u, 0x1044)));
+}
+__device__ __forceinline__ uint64_t dup_bf16hi(uint32_t w) {
+    return f2pack(__uint_as_float(w & 0xffff0000u), __uint_as_float(__byte_perm(w, 0u, 0x3244)));
+}
+
+template <typename T>
+__device__ __forceinline__ uint64_t dup_elem(const uint4 &w, int e);
+
+template <>
+__device__ __forceinline__ uint64_t dup_elem<__nv_bfloat16>(const uint4 &w, int e) {
+    const uint32_t x = (e >> 1) == 0 ? w.x : (e >> 1) == 1 ? w.y : (e >> 1) == 2 ? w.z : w.w;
+    return (e & 1) ? dup_bf16hi(x) : dup_bf16lo(x);
+}
+
+template <>
+__device__ __forceinline__ uint64_t dup_elem<float>(const uint4 &w, int e) {
+    const uint32_t x = e == 0 ? w.x : e == 1 ? w.y : e == 2 ? w.z : w.w;
+    return f2pack(__uint_as_float(x), __uint_as_float(x));
+}
+
+// 16-byte sub-chunk cc (0..3) of row r in a stage written by TMA with the 64-byte swizzle
+// (sub-chunk index XOR bits [1:2] of the row: bank-conflict free for 8 consecutive rows)
+__device__ __forceinline__ int k1_sub(int r, int cc) { return r * 4 + (cc ^ ((r >> 1) & 3)); }
+
 template <int D, typename T>
 __global__ void __launch_bounds__(kK1Threads, 2)
     k_project_scan(const CoarsenArgs a, const __grid_constant__ CUtensorMap map_k,
                    const __grid_constant__ CUtensorMap map_v, const __grid_constant__ ProjT proj) {
     constexpr int ELEM = sizeof(T);
-    constexpr int KCHUNK = D * ELEM / 128;    // 128-byte chunks of one key row
-    constexpr int NCHUNK = 2 * KCHUNK;        // key chunks, then value chunks
-    constexpr int JPC = 128 / ELEM;           // feature index j per chunk
-    constexpr int EPS = 16 / ELEM;            // elements per 16-byte sub-chunk
+    constexpr int KCHUNK = D * ELEM / kK1ColBytes;   // column chunks of one key row
+    constexpr int NCHUNK = 2 * KCHUNK;               // key chunks, then value chunks
+    constexpr int JPC = kK1ColBytes / ELEM;          // feature index j per chunk
+    constexpr int EPS = 16 / ELEM;                   // elements per 16-byte sub-chunk
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
@@ -101,25 +118,32 @@ __global__ void __launch_bounds__(kK1Threads, 2)
     const int tid = threadIdx.x;
 
     const int y0 = static_cast<int>(sr.row_off + static_cast<int64_t>(h) * sr.T + sr.s_eff) + tile * kTileOut - 1;
+    auto issue = [&](int c, int s) {
+        mbar_arrive_expect_tx(&bar[s], kK1StageBytes);
+        const CUtensorMap *map = c < KCHUNK ? &map_k : &map_v;
+#pragma unroll
+        for (int hb = 0; hb < kTileRows / kK1BoxRows; ++hb)
+            tma_load_2d(stages + s * kK1StageBytes + hb * kK1BoxRows * kK1ColBytes, map, (c % KCHUNK) * JPC,
+                        y0 + hb * kK1BoxRows, &bar[s]);
+    };
     if (tid == 0) {
         prefetch_tensormap(&map_k);
         prefetch_tensormap(&map_v);
         for (int s = 0; s < kK1Stages; ++s) mbar_init(&bar[s], 1);
         fence_mbar_init();
-        for (int c = 0; c < NCHUNK && c < kK1Stages; ++c) {
-            mbar_arrive_expect_tx(&bar[c], kK1StageBytes);
-            tma_load_2d(stages + c * kK1StageBytes, c < KCHUNK ? &map_k : &map_v, (c % KCHUNK) * JPC, y0, &bar[c]);
-        }
+        for (int c = 0; c < NCHUNK && c < kK1Stages; ++c) issue(c, c);
     }
     for (int i = tid; i < (2 * D + 1) * kProjDim; i += kK1Threads) pt[i] = i < 2 * D * kProjDim ? proj.pt[i] : 0.0f;
     __syncthreads();
 
-    const int r0 = tid, r1 = tid + kK1Threads;
-    uint64_t acc0[kProjDim / 2], acc1[kProjDim / 2];
+    // rows tid + 128 t (t < 4) of the tile; each feature's P^T row is read once per 4 tokens
+    uint64_t acc[kK1Tok][kProjDim / 2];
 #pragma unroll
-    for (int i = 0; i < kProjDim / 2; ++i) acc0[i] = acc1[i] = 0ull;
+    for (int t = 0; t < kK1Tok; ++t)
+#pragma unroll
+        for (int i = 0; i < kProjDim / 2; ++i) acc[t][i] = 0ull;
     const float4 *ptv = reinterpret_cast<const float4 *>(pt);   // P^T row j = ptv[4 j .. 4 j + 3]
-    // software pipeline: the P^T row of feature j + 1 and the next 16-byte sub-chunk of both rows
+    // software pipeline: the P^T row of feature j + 1 and the next 16-byte sub-chunk of the rows
     // are read while feature j is accumulated (plain shared loads: never hoisted above the wait)
     float4 pc[4];
 #pragma unroll
@@ -130,60 +154,56 @@ __global__ void __launch_bounds__(kK1Threads, 2)
         const int s = c % kK1Stages;
         if (ok && !mbar_wait(&bar[s], (c / kK1Stages) & 1)) ok = false;
         const uint4 *st = reinterpret_cast<const uint4 *>(stages + s * kK1StageBytes);
-        uint4 xa = st[r0 * 8 + (0 ^ (r0 & 7))];
-        uint4 xb = st[r1 * 8 + (0 ^ (r1 & 7))];
+        uint4 x[kK1Tok];
+#pragma unroll
+        for (int t = 0; t < kK1Tok; ++t) x[t] = st[k1_sub(tid + t * kK1Threads, 0)];
 #pragma unroll 1
-        for (int sc = 0; sc < 8; ++sc) {
-            const int scn = sc < 7 ? sc + 1 : 7;
-            const uint4 nxa = st[r0 * 8 + (scn ^ (r0 & 7))];
-            const uint4 nxb = st[r1 * 8 + (scn ^ (r1 & 7))];
+        for (int cc = 0; cc < 4; ++cc) {
+            const int ccn = cc < 3 ? cc + 1 : 3;
+            uint4 xn[kK1Tok];
+#pragma unroll
+            for (int t = 0; t < kK1Tok; ++t) xn[t] = st[k1_sub(tid + t * kK1Threads, ccn)];
 #pragma unroll
             for (int e = 0; e < EPS; ++e) {
-                const int j = c * JPC + sc * EPS + e;
+                const int j = c * JPC + cc * EPS + e;
                 float4 pn[4];
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) pn[q4] = ptv[4 * (j + 1) + q4];
-                const float va = elem_of<T>(xa, e), vb = elem_of<T>(xb, e);
-                const uint64_t xa2 = f2pack(va, va), xb2 = f2pack(vb, vb);
 #pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) {
-                    const uint64_t pa = f2pack(pc[q4].x, pc[q4].y), pb = f2pack(pc[q4].z, pc[q4].w);
-                    acc0[2 * q4] = ffma2(pa, xa2, acc0[2 * q4]);
-                    acc0[2 * q4 + 1] = ffma2(pb, xa2, acc0[2 * q4 + 1]);
-                    acc1[2 * q4] = ffma2(pa, xb2, acc1[2 * q4]);
-                    acc1[2 * q4 + 1] = ffma2(pb, xb2, acc1[2 * q4 + 1]);
+                for (int t = 0; t < kK1Tok; ++t) {
+                    const uint64_t xx = dup_elem<T>(x[t], e);
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        acc[t][2 * q4] = ffma2(f2pack(pc[q4].x, pc[q4].y), xx, acc[t][2 * q4]);
+                        acc[t][2 * q4 + 1] = ffma2(f2pack(pc[q4].z, pc[q4].w), xx, acc[t][2 * q4 + 1]);
+                    }
                 }
 #pragma unroll
                 for (int q4 = 0; q4 < 4; ++q4) pc[q4] = pn[q4];
             }
-            xa = nxa;
-            xb = nxb;
+#pragma unroll
+            for (int t = 0; t < kK1Tok; ++t) x[t] = xn[t];
         }
         __syncthreads();
-        if (tid == 0 && c + kK1Stages < NCHUNK) {
-            const int cn = c + kK1Stages;
-            mbar_arrive_expect_tx(&bar[s], kK1StageBytes);
-            tma_load_2d(stages + s * kK1StageBytes, cn < KCHUNK ? &map_k : &map_v, (cn % KCHUNK) * JPC, y0, &bar[s]);
-        }
+        if (tid == 0 && c + kK1Stages < NCHUNK) issue(c + kK1Stages, s);
     }
-    if (!ok) {
-        raise_flag(a.flags, FLAG_TIMEOUT);
-    }
+    if (!ok) raise_flag(a.flags, FLAG_TIMEOUT);
 
-    // z of both rows -> shared (stage 0 is free: every chunk has been consumed and synced)
+    // z of the rows -> shared (the stages are free: every chunk has been consumed and synced)
     float *zb = reinterpret_cast<float *>(stages);
 #pragma unroll
-    for (int i = 0; i < kProjDim / 2; ++i) {
-        f2unpack(acc0[i], zb[r0 * kZStride + 2 * i], zb[r0 * kZStride + 2 * i + 1]);
-        f2unpack(acc1[i], zb[r1 * kZStride + 2 * i], zb[r1 * kZStride + 2 * i + 1]);
+    for (int t = 0; t < kK1Tok; ++t) {
+        const int r = tid + t * kK1Threads;
+#pragma unroll
+        for (int i = 0; i < kProjDim / 2; ++i) f2unpack(acc[t][i], zb[r * kZStride + 2 * i], zb[r * kZStride + 2 * i + 1]);
     }
     __syncthreads();
 
-    // outputs l = 2 tid + 1, 2 tid + 2 (rows of the tile; row 0 is the halo)
-    long long Dv[2];
+    // outputs l = 4 tid + 1 .. 4 tid + 4 (rows of the tile; row 0 is the halo)
+    long long Dv[kK1Tok];
 #pragma unroll
-    for (int q = 0; q < 2; ++q) {
-        const int l = 2 * tid + 1 + q;
+    for (int q = 0; q < kK1Tok; ++q) {
+        const int l = kK1Tok * tid + 1 + q;
         const int t = tile * kTileOut + l - 1;
         long long D_ = 0;
         if (l <= kTileOut && t < sr.M && t > 0) {
@@ -195,9 +215,12 @@ __global__ void __launch_bounds__(kK1Threads, 2)
         }
         Dv[q] = D_;
     }
-    // block inclusive scan of the pair sums
+    // block inclusive scan of the per-thread sums
     const int lane = tid & 31, warp = tid >> 5;
-    long long v = Dv[0] + Dv[1];
+    long long own = 0;
+#pragma unroll
+    for (int q = 0; q < kK1Tok; ++q) own += Dv[q];
+    long long v = own;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
         const long long n = __shfl_up_sync(0xffffffffu, v, off);
@@ -208,11 +231,15 @@ __global__ void __launch_bounds__(kK1Threads, 2)
     long long wp = 0;
     for (int w = 0; w < warp; ++w) wp += warp_sum[w];
     const long long incl = wp + v;
-    const long long excl = incl - Dv[0] - Dv[1];
+    long long run = incl - own;
     int64_t *ls = a.local_scan + sr.mid_off + static_cast<int64_t>(h) * sr.M;
-    const int t0 = tile * kTileOut + 2 * tid;   // middle index of output l = 2 tid + 1
-    if (2 * tid + 1 <= kTileOut && t0 < sr.M) ls[t0] = excl + Dv[0];
-    if (2 * tid + 2 <= kTileOut && t0 + 1 < sr.M) ls[t0 + 1] = excl + Dv[0] + Dv[1];
+#pragma unroll
+    for (int q = 0; q < kK1Tok; ++q) {
+        run += Dv[q];
+        const int l = kK1Tok * tid + 1 + q;
+        const int t = tile * kTileOut + l - 1;
+        if (l <= kTileOut && t < sr.M) ls[t] = run;
+    }
     if (tid == kK1Threads - 1) a.tile_total[static_cast<int64_t>(u) * a.max_tiles + tile] = incl;
 }
 
@@ -266,7 +293,7 @@ __device__ __forceinline__ long long floor_ratio(long long N, long long C, long 
     return q;
 }
 
-__global__ void __launch_bounds__(256) k_boundaries(const CoarsenArgs a) {
+__global__ void __launch_bounds__(kTileRows) k_boundaries(const CoarsenArgs a) {
     const int u = blockIdx.y, tile = blockIdx.x;
     const int b = u / a.Hkv, h = u % a.Hkv;
     const SeqRow sr = a.seq[b];
@@ -519,7 +546,7 @@ static cudaError_t launch_typed(const CoarsenArgs &a, const SeqTable &table, con
         }
         k_project_scan<D, T><<<dim3(a.max_tiles, units), kK1Threads, smem, s>>>(a, map_k, map_v, proj);
         k_tile_prefix<<<units, 256, 0, s>>>(a);
-        k_boundaries<<<dim3(a.max_tiles, units), 256, 0, s>>>(a);
+        k_boundaries<<<dim3(a.max_tiles, units), kTileRows, 0, s>>>(a);
     }
     k_plan_entries<<<units, 512, 0, s>>>(a);
     if (a.max_emax > 0)

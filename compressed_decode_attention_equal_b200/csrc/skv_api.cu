@@ -97,18 +97,18 @@ EncodeTiledFn encode_fn() {
     return fn;
 }
 
-// Rows x d matrix of raw keys or values; boxes of 256 rows x 128 bytes, 128-byte swizzle.
+// Rows x d matrix of raw keys or values; boxes of 256 rows x 64 bytes, 64-byte swizzle.
 bool make_row_map(CUtensorMap *map, const void *base, int dtype, int d, int64_t rows) {
     EncodeTiledFn fn = encode_fn();
     if (!fn) return false;
     const int elem = dtype == SKV_BF16 ? 2 : 4;
     cuuint64_t dims[2] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows)};
     cuuint64_t strides[1] = {static_cast<cuuint64_t>(d) * elem};
-    cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem), static_cast<cuuint32_t>(kTileRows)};
+    cuuint32_t box[2] = {static_cast<cuuint32_t>(64 / elem), 256u};
     cuuint32_t estr[2] = {1, 1};
     const CUresult r = fn(map, dtype == SKV_BF16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2,
                           const_cast<void *>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
-                          CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                          CU_TENSOR_MAP_SWIZZLE_64B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
     return r == CUDA_SUCCESS;
 }

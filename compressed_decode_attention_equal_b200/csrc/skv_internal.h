@@ -13,7 +13,7 @@ namespace skv {
 // ---------------------------------------------------------------------------
 // coarsening
 // ---------------------------------------------------------------------------
-constexpr int kTileRows = 256;              // rows a projection tile computes (1 halo + outputs)
+constexpr int kTileRows = 512;              // rows a projection tile computes (1 halo + outputs)
 constexpr int kTileOut = kTileRows - 1;     // middle tokens per projection tile
 
 // Per-sequence plan, computed on the host and copied into the workspace.
