@@ -14,6 +14,7 @@ SKV_F32, SKV_BF16 = 0, 1
 PAGE_NODES = 16
 PROJ_DIM = 16
 MAX_SEQS = 512
+NOALLOC_SCRATCH_BYTES = 4 << 20
 
 FLAG_OVERFLOW, FLAG_BAD_PAGE, FLAG_BAD_LENS, FLAG_TIMEOUT = 1, 2, 4, 8
 
@@ -31,7 +32,8 @@ class SkvError(RuntimeError):
 
 # The header declares every symbol below; tests check that the library exports all of them.
 EXPORTS = ("skv_status_string", "skv_abi_version", "skv_projection_matrix", "skv_coarsen_workspace_bytes",
-           "skv_coarsen", "skv_decode_workspace_bytes", "skv_decode_attn", "skv_workspace_error")
+           "skv_coarsen", "skv_decode_workspace_bytes", "skv_decode_attn", "skv_decode_attn_noalloc",
+           "skv_workspace_error")
 
 _lib = None
 
@@ -63,6 +65,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.skv_decode_attn.argtypes = [vp, i32, i32, i32, i32, i32, i32, ctypes.POINTER(SkvNodePool), vp, i32,
                                     vp, vp, vp, vp, sz, vp]
     lib.skv_decode_attn.restype = i32
+    lib.skv_decode_attn_noalloc.argtypes = [vp, i32, i32, i32, i32, i32, i32, ctypes.POINTER(SkvNodePool), vp,
+                                            i32, vp, vp, vp, vp]
+    lib.skv_decode_attn_noalloc.restype = i32
     lib.skv_workspace_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.skv_workspace_error.restype = i32
     _lib = lib

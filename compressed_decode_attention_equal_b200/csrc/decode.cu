@@ -782,3 +782,21 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
 }
 
 }  // namespace skv
+
+namespace skv {
+
+// The grid k_decode_split would use for these arguments (bf16 caches), for callers that must size
+// split-partial storage before launching. Queries (and caches) the same occupancy as the launcher.
+cudaError_t decode_split_ctas(const DecodeArgs &a, int *ncta) {
+    const int nt = a.pass_rows / 8 + (a.pass_rows % 8 ? 1 : 0);
+    if (a.d == 128) {
+        if (nt == 1) return split_grid<128, 1>(split_smem<128, 1>(a.n_vunits), ncta);
+        if (nt == 2) return split_grid<128, 2>(split_smem<128, 2>(a.n_vunits), ncta);
+        return split_grid<128, 4>(split_smem<128, 4>(a.n_vunits), ncta);
+    }
+    if (nt == 1) return split_grid<64, 1>(split_smem<64, 1>(a.n_vunits), ncta);
+    if (nt == 2) return split_grid<64, 2>(split_smem<64, 2>(a.n_vunits), ncta);
+    return split_grid<64, 4>(split_smem<64, 4>(a.n_vunits), ncta);
+}
+
+}  // namespace skv

@@ -103,5 +103,6 @@ struct DecodeLayout {
 };
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
+cudaError_t decode_split_ctas(const DecodeArgs &a, int *ncta);
 
 }  // namespace skv

@@ -190,6 +190,35 @@ skv_status skv_decode_attn(const void *q, skv_dtype dtype, int B, int R, int Hq,
                            void *stream);
 
 /*
+ * Decode attention without any caller-provided workspace. (The sources describe no such entry
+ * point; it exists for callers of this library that cannot allocate device memory.)
+ *
+ * Some callers cannot allocate: code recorded into a CUDA graph owned by someone else, a plugin
+ * that a host framework hands only its input and output buffers, or a runtime whose allocator is
+ * fixed when it starts. This entry point takes the same arguments and computes the same result
+ * as skv_decode_attn (the same kernel), but keeps its scratch -- device flags, per-unit
+ * completion counters and split partials -- in one array of SKV_NOALLOC_SCRATCH_BYTES that the
+ * library defines at file scope. Every GPU that loads the library reserves that array once and
+ * keeps it until the process exits.
+ *  - No cudaMalloc, cudaFree or other allocating call is made.
+ *  - The first call on each device looks up the array's device address (cudaGetSymbolAddress)
+ *    with that device current and caches it; make that first call before any stream capture.
+ *  - All calls on a device share the array: calls whose kernels may overlap on the GPU (other
+ *    streams, or other threads' streams) race on it and must be serialised by the caller. Each
+ *    call clears the flags and counters on `stream` before its kernel runs.
+ *  - A request whose scratch would exceed SKV_NOALLOC_SCRATCH_BYTES (bf16: split partials of
+ *    2 x grid x rows-per-pass x (d + 1) floats, plus 4 bytes per unit and row pass) returns
+ *    SKV_ERR_WORKSPACE before anything is enqueued; use skv_decode_attn for such sizes.
+ *  - Device-detected errors (bad page id, lens above capacity) still skip the bad access, but
+ *    their flags live in the library's array and are not reported; diagnose with skv_decode_attn.
+ * Other errors: as skv_decode_attn.
+ */
+#define SKV_NOALLOC_SCRATCH_BYTES (4u << 20)
+skv_status skv_decode_attn_noalloc(const void *q, skv_dtype dtype, int B, int R, int Hq, int Hkv, int d,
+                                   const skv_node_pool *pool, const int32_t *page_table, int max_pages,
+                                   const int32_t *lens, void *out, float *lse, void *stream);
+
+/*
  * Synchronise stream, then read and clear the device error flags raised on
  * this workspace since they were last cleared: SKV_OK, SKV_ERR_OVERFLOW or
  * SKV_ERR_DEVICE (SKV_ERR_CUDA if synchronisation fails). *flags_host
