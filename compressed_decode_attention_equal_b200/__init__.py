@@ -22,8 +22,8 @@ from . import _lib
 from ._lib import PAGE_NODES, SkvError
 
 __all__ = ["NodePool", "coarsen", "decode_attn", "coarsen_workspace_bytes", "decode_workspace_bytes",
-           "workspace_error", "projection_matrix", "entries_bound", "pages_for", "read_entries", "SkvError",
-           "PAGE_NODES", "library_path"]
+           "workspace_error", "projection_matrix", "entries_bound", "pages_for", "page_bytes", "read_entries",
+           "SkvError", "PAGE_NODES", "library_path"]
 
 
 def library_path() -> str:
@@ -67,21 +67,27 @@ def pages_for(T: int, N: int, n_sink: int, n_recent: int) -> int:
 
 
 class NodePool:
-    """Paged macro-node storage: k, v [num_pages, 16, d] (dtype) and ab [num_pages, 16, 2] fp32
-    (alpha = ln m, beta = sigma^2 / (2d)). Within a page, 16-byte chunk c of slot n is stored at
-    chunk c ^ (n & 7)."""
+    """Paged macro-node storage: one uint8 tensor `pages` [num_pages, page_bytes]; page p holds 16
+    entries of one unit as [keys 16 x d | values 16 x d | {alpha, beta} 16 x 2 fp32] (alpha = ln m,
+    beta = sigma^2 / (2d)). `k`, `v`, `ab` are strided views of those blocks. Within the key and value
+    blocks, 16-byte chunk c of slot n is stored at chunk c ^ (n & 7)."""
 
     def __init__(self, num_pages: int, d: int, dtype: torch.dtype, device="cuda"):
         self.num_pages, self.d, self.dtype = int(num_pages), int(d), dtype
-        self.k = torch.empty(self.num_pages, PAGE_NODES, d, dtype=dtype, device=device)
-        self.v = torch.empty(self.num_pages, PAGE_NODES, d, dtype=dtype, device=device)
-        self.ab = torch.empty(self.num_pages, PAGE_NODES, 2, dtype=torch.float32, device=device)
+        elem = torch.tensor([], dtype=dtype).element_size()
+        self.vec_bytes = PAGE_NODES * d * elem
+        self.page_bytes = 2 * self.vec_bytes + PAGE_NODES * 8
+        P = self.num_pages
+        self.pages = torch.empty(P, self.page_bytes, dtype=torch.uint8, device=device)
+        self.k = self.pages[:, :self.vec_bytes].view(dtype).view(P, PAGE_NODES, d)
+        self.v = self.pages[:, self.vec_bytes:2 * self.vec_bytes].view(dtype).view(P, PAGE_NODES, d)
+        self.ab = self.pages[:, 2 * self.vec_bytes:].view(torch.float32).view(P, PAGE_NODES, 2)
 
     def struct(self) -> _lib.SkvNodePool:
-        return _lib.SkvNodePool(self.k.data_ptr(), self.v.data_ptr(), self.ab.data_ptr(), self.num_pages)
+        return _lib.SkvNodePool(self.pages.data_ptr(), self.num_pages)
 
     def nbytes(self) -> int:
-        return self.k.numel() * self.k.element_size() * 2 + self.ab.numel() * 4
+        return self.pages.numel()
 
 
 def projection_matrix(seed: int, d: int) -> torch.Tensor:
@@ -173,6 +179,19 @@ def workspace_error(workspace: torch.Tensor, stream=None):
     return st, flags.value
 
 
+def page_bytes(dtype: torch.dtype, d: int) -> int:
+    return int(_lib.load().skv_page_bytes(_code(dtype), d))
+
+
+def _entry_rows(pool: NodePool, page_table: torch.Tensor, b: int, h: int, E: int):
+    n_pages = -(-E // PAGE_NODES)
+    pages = page_table[b, h, :n_pages].long()
+    slots = torch.arange(PAGE_NODES, device=pages.device)
+    pg = pages[:, None].expand(n_pages, PAGE_NODES).reshape(-1)[:E]
+    sl = slots[None, :].expand(n_pages, PAGE_NODES).reshape(-1)[:E]
+    return pg, sl
+
+
 def read_entries(pool: NodePool, page_table: torch.Tensor, lens: torch.Tensor, b: int, h: int):
     """Entries of unit (b, h) in entry order, un-swizzled: (kt [E, d], vt [E, d], alpha [E], beta [E]).
     A layout view for inspection (indexing only)."""
@@ -181,17 +200,13 @@ def read_entries(pool: NodePool, page_table: torch.Tensor, lens: torch.Tensor, b
     if E == 0:
         z = pool.k.new_zeros(0, d)
         return z, z.clone(), pool.ab.new_zeros(0), pool.ab.new_zeros(0)
-    n_pages = -(-E // PAGE_NODES)
-    pages = page_table[b, h, :n_pages].long()
-    rows = (pages[:, None] * PAGE_NODES + torch.arange(PAGE_NODES, device=pages.device)).reshape(-1)[:E]
+    pg, sl = _entry_rows(pool, page_table, b, h, E)
     epc = 16 // pool.k.element_size()
     ch = d // epc
-    slot = torch.arange(E, device=pages.device) % PAGE_NODES
-    phys = torch.arange(ch, device=pages.device)[None, :] ^ (slot[:, None] & 7)
-    kr = pool.k.reshape(-1, ch, epc)[rows]
-    vr = pool.v.reshape(-1, ch, epc)[rows]
-    idx = phys[:, :, None].expand(E, ch, epc)
-    kt = torch.gather(kr, 1, idx).reshape(E, d)
-    vt = torch.gather(vr, 1, idx).reshape(E, d)
-    ab = pool.ab.reshape(-1, 2)[rows]
+    phys = torch.arange(ch, device=pg.device)[None, :] ^ (sl[:, None] & 7)
+    k4 = pool.k.view(pool.num_pages, PAGE_NODES, ch, epc)
+    v4 = pool.v.view(pool.num_pages, PAGE_NODES, ch, epc)
+    kt = k4[pg[:, None], sl[:, None], phys].reshape(E, d)
+    vt = v4[pg[:, None], sl[:, None], phys].reshape(E, d)
+    ab = pool.ab[pg, sl]
     return kt, vt, ab[:, 0], ab[:, 1]

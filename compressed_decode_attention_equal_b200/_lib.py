@@ -20,8 +20,7 @@ FLAG_OVERFLOW, FLAG_BAD_PAGE, FLAG_BAD_LENS, FLAG_TIMEOUT = 1, 2, 4, 8
 
 
 class SkvNodePool(ctypes.Structure):
-    _fields_ = [("k", ctypes.c_void_p), ("v", ctypes.c_void_p), ("ab", ctypes.c_void_p),
-                ("num_pages", ctypes.c_int64)]
+    _fields_ = [("pages", ctypes.c_void_p), ("num_pages", ctypes.c_int64)]
 
 
 class SkvError(RuntimeError):
@@ -31,7 +30,8 @@ class SkvError(RuntimeError):
 
 
 # The header declares every symbol below; tests check that the library exports all of them.
-EXPORTS = ("skv_status_string", "skv_abi_version", "skv_projection_matrix", "skv_coarsen_workspace_bytes",
+EXPORTS = ("skv_status_string", "skv_abi_version", "skv_page_bytes", "skv_projection_matrix",
+           "skv_coarsen_workspace_bytes",
            "skv_coarsen", "skv_decode_workspace_bytes", "skv_decode_attn", "skv_decode_attn_noalloc",
            "skv_workspace_error")
 
@@ -53,6 +53,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.skv_status_string.restype = ctypes.c_char_p
     lib.skv_abi_version.argtypes = []
     lib.skv_abi_version.restype = i32
+    lib.skv_page_bytes.argtypes = [i32, i32]
+    lib.skv_page_bytes.restype = sz
     lib.skv_projection_matrix.argtypes = [u64, i32, ctypes.POINTER(ctypes.c_float)]
     lib.skv_projection_matrix.restype = i32
     lib.skv_coarsen_workspace_bytes.argtypes = [i32, i32, i32, pi32, pi32, i32, i32]

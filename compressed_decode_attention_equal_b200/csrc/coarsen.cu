@@ -513,14 +513,16 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
         if (lane == 0) raise_flag(a.flags, FLAG_BAD_PAGE);
         return;
     }
+    constexpr int VEC_BYTES = kPageNodes * ROWB;   // keys (then values) of one page
+    uint8_t *pg = a.pages + static_cast<int64_t>(page) * (2 * VEC_BYTES + kPageNodes * 8);
     if (sub == 0) {
-        const int64_t off = (static_cast<int64_t>(page) * kPageNodes + slot) * ROWB + swz(ch, slot) * 16;
-        Vec16<T>::store(a.pool_k + off, sk);
-        Vec16<T>::store(a.pool_v + off, sv);
+        const int off = slot * ROWB + swz(ch, slot) * 16;
+        Vec16<T>::store(pg + off, sk);
+        Vec16<T>::store(pg + VEC_BYTES + off, sv);
     }
     if (lane == 0) {
         const float alpha = m == 1 ? 0.0f : logf(fm);
-        a.pool_ab[static_cast<int64_t>(page) * kPageNodes + slot] = make_float2(alpha, sigma2 / (2.0f * D));
+        reinterpret_cast<float2 *>(pg + 2 * VEC_BYTES)[slot] = make_float2(alpha, sigma2 / (2.0f * D));
     }
 }
 

@@ -13,9 +13,9 @@
 //    ncta equal ranges (one per CTA, a stream-K style split), so every CTA
 //    streams the same number of 16-node pages whatever the length mix; the
 //    part of one virtual unit inside one CTA's range is a "piece";
-//  * one producer warp copies each page (K 4 KB, V 4 KB, alpha/beta 128 B at
-//    d = 128) with three TMA bulk copies into an 8-stage mbarrier ring, and
-//    each piece's query rows into a double-buffered slot;
+//  * one producer warp copies each page (keys 4 KB, values 4 KB, alpha/beta
+//    128 B at d = 128, contiguous) with one TMA bulk copy into an 8-stage
+//    mbarrier ring, and each piece's query rows into a double-buffered slot;
 //  * four consumer warps run the GQA group's query rows through tensor cores:
 //    S^T = K Q^T with nodes as the M = 16 dimension and up to 8 query rows as
 //    N = 8 (a GQA group of 7 rows wastes 1/8), softmax on the accumulator, P^T
@@ -374,13 +374,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                         mbar_arrive(&full[s]);
                     } else {
                         svalid[s] = 1;
-                        uint8_t *dst = stages + s * G::STAGE;
                         mbar_arrive_expect_tx(&full[s], G::STAGE);
-                        bulk_g2s(dst, a.pool_k + static_cast<long long>(phys) * G::VEC_BYTES, G::VEC_BYTES, &full[s]);
-                        bulk_g2s(dst + G::VEC_BYTES, a.pool_v + static_cast<long long>(phys) * G::VEC_BYTES,
-                                 G::VEC_BYTES, &full[s]);
-                        bulk_g2s(dst + 2 * G::VEC_BYTES, a.pool_ab + static_cast<long long>(phys) * kPageNodes,
-                                 G::AB_BYTES, &full[s]);
+                        // a page is one contiguous [keys | values | alpha,beta] block: one copy
+                        bulk_g2s(stages + s * G::STAGE, a.pages + static_cast<long long>(phys) * G::STAGE, G::STAGE,
+                                 &full[s]);
                     }
                 }
                 __syncwarp();
@@ -644,8 +641,9 @@ __global__ void __launch_bounds__(128) k_decode_f32(const DecodeArgs a) {
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int L = clamp_entries(a, u);
     const float *q = static_cast<const float *>(a.q);
-    const float *pk = reinterpret_cast<const float *>(a.pool_k);
-    const float *pv = reinterpret_cast<const float *>(a.pool_v);
+    constexpr int VEC_FLOATS = kPageNodes * D;   // fp32 keys (then values) of one page
+    constexpr long long PAGE_FLOATS = 2 * VEC_FLOATS + 2 * kPageNodes;
+    const float *pool = reinterpret_cast<const float *>(a.pages);
     float *outp = static_cast<float *>(a.out);
     const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
     for (int row = warp; row < a.rows; row += 4) {
@@ -669,7 +667,9 @@ __global__ void __launch_bounds__(128) k_decode_f32(const DecodeArgs a) {
                 continue;
             }
             const int slot = e % kPageNodes;
-            const long long nb = (static_cast<long long>(page) * kPageNodes + slot) * D;
+            const float *pk = pool + static_cast<long long>(page) * PAGE_FLOATS;
+            const float *pv = pk + VEC_FLOATS;
+            const long long nb = static_cast<long long>(slot) * D;
             float dot = 0.0f;
 #pragma unroll
             for (int i = 0; i < PER; ++i) {
@@ -678,7 +678,7 @@ __global__ void __launch_bounds__(128) k_decode_f32(const DecodeArgs a) {
             }
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-            const float2 ab = a.pool_ab[static_cast<long long>(page) * kPageNodes + slot];
+            const float2 ab = reinterpret_cast<const float2 *>(pk + 2 * VEC_FLOATS)[slot];
             const float s = fmaf(dot, inv_sqrt_d, fmaf(qn, ab.y, ab.x));
             const float mn = fmaxf(m, s);
             const float corr = expf(m - mn);

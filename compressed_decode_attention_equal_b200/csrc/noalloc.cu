@@ -55,10 +55,9 @@ extern "C" skv_status skv_decode_attn_noalloc(const void *q, skv_dtype dtype, in
     if (Hq % Hkv != 0 || (d != 64 && d != 128) || (dtype != SKV_BF16 && dtype != SKV_F32))
         return SKV_ERR_UNSUPPORTED;
     if (!q || !out || !lse || !pool || !page_table || !lens) return SKV_ERR_INVALID_ARG;
-    if (!pool->k || !pool->v || !pool->ab || pool->num_pages < 0) return SKV_ERR_INVALID_ARG;
+    if (!pool->pages || pool->num_pages < 0) return SKV_ERR_INVALID_ARG;
     const auto al = [](const void *p, uintptr_t m) { return (reinterpret_cast<uintptr_t>(p) & (m - 1)) == 0; };
-    if (!al(pool->k, 16) || !al(pool->v, 16) || !al(pool->ab, 16) || !al(q, 16) || !al(out, 16) || !al(lse, 4))
-        return SKV_ERR_INVALID_ARG;
+    if (!al(pool->pages, 16) || !al(q, 16) || !al(out, 16) || !al(lse, 4)) return SKV_ERR_INVALID_ARG;
     const int64_t rows = static_cast<int64_t>(R) * (Hq / Hkv);
     if (rows > (1 << 20) || static_cast<int64_t>(max_pages) * kPageNodes > INT32_MAX / 2) return SKV_ERR_UNSUPPORTED;
     DecodeArgs a{};
@@ -70,9 +69,7 @@ extern "C" skv_status skv_decode_attn_noalloc(const void *q, skv_dtype dtype, in
         return SKV_ERR_UNSUPPORTED;
     a.n_vunits = static_cast<int>(nv);
     a.q = q;
-    a.pool_k = static_cast<const uint8_t *>(pool->k);
-    a.pool_v = static_cast<const uint8_t *>(pool->v);
-    a.pool_ab = reinterpret_cast<const float2 *>(pool->ab);
+    a.pages = static_cast<const uint8_t *>(pool->pages);
     a.num_pages = pool->num_pages;
     a.page_table = page_table;
     a.max_pages = max_pages;

@@ -232,7 +232,13 @@ const char *skv_status_string(int status) {
     }
 }
 
-int skv_abi_version(void) { return 100; }
+int skv_abi_version(void) { return 200; }
+
+size_t skv_page_bytes(skv_dtype dtype, int d) {
+    if ((dtype != SKV_BF16 && dtype != SKV_F32) || (d != 64 && d != 128)) return 0;
+    const size_t elem = dtype == SKV_BF16 ? 2 : 4;
+    return 2 * static_cast<size_t>(kPageNodes) * d * elem + kPageNodes * 8;
+}
 
 skv_status skv_projection_matrix(uint64_t proj_seed, int d, float *P_host) {
     if (!P_host || (d != 64 && d != 128)) return SKV_ERR_INVALID_ARG;
@@ -259,8 +265,7 @@ skv_status skv_coarsen(const void *k, const void *v, skv_dtype dtype, int B, int
     skv_status st = plan_coarsen(B, Hkv, d, T_host, N_host, n_sink, n_recent, &table, &plan);
     if (st != SKV_OK) return st;
     if (!pool || !page_table || !lens || max_pages < 1) return SKV_ERR_INVALID_ARG;
-    if (!pool->k || !pool->v || !pool->ab || pool->num_pages < 0) return SKV_ERR_INVALID_ARG;
-    if (!aligned(pool->k, 16) || !aligned(pool->v, 16) || !aligned(pool->ab, 16)) return SKV_ERR_INVALID_ARG;
+    if (!pool->pages || pool->num_pages < 0 || !aligned(pool->pages, 16)) return SKV_ERR_INVALID_ARG;
     if (plan.rows > 0 && (!k || !v || !aligned(k, 16) || !aligned(v, 16))) return SKV_ERR_INVALID_ARG;
     if (!workspace || !aligned(workspace, 256) || ws_bytes < plan.lay.total) return SKV_ERR_WORKSPACE;
     for (int b = 0; b < B; ++b)
@@ -294,9 +299,7 @@ skv_status skv_coarsen(const void *k, const void *v, skv_dtype dtype, int B, int
     a.bounds = reinterpret_cast<int32_t *>(ws + plan.lay.bounds);
     a.ents = reinterpret_cast<int2 *>(ws + plan.lay.ents);
     a.flags = reinterpret_cast<uint32_t *>(ws);
-    a.pool_k = static_cast<uint8_t *>(pool->k);
-    a.pool_v = static_cast<uint8_t *>(pool->v);
-    a.pool_ab = reinterpret_cast<float2 *>(pool->ab);
+    a.pages = static_cast<uint8_t *>(pool->pages);
     a.num_pages = pool->num_pages;
     a.page_table = page_table;
     a.max_pages = max_pages;
@@ -320,17 +323,14 @@ skv_status skv_decode_attn(const void *q, skv_dtype dtype, int B, int R, int Hq,
     skv_status st = plan_decode(dtype, B, R, Hq, Hkv, d, max_pages, &plan);
     if (st != SKV_OK) return st;
     if (!q || !out || !lse || !pool || !page_table || !lens) return SKV_ERR_INVALID_ARG;
-    if (!pool->k || !pool->v || !pool->ab || pool->num_pages < 0) return SKV_ERR_INVALID_ARG;
-    if (!aligned(pool->k, 16) || !aligned(pool->v, 16) || !aligned(pool->ab, 16) || !aligned(q, 16) ||
-        !aligned(out, 16) || !aligned(lse, 4))
+    if (!pool->pages || pool->num_pages < 0) return SKV_ERR_INVALID_ARG;
+    if (!aligned(pool->pages, 16) || !aligned(q, 16) || !aligned(out, 16) || !aligned(lse, 4))
         return SKV_ERR_INVALID_ARG;
     if (!workspace || !aligned(workspace, 256) || ws_bytes < plan.lay.total) return SKV_ERR_WORKSPACE;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
     DecodeArgs a{};
     a.q = q;
-    a.pool_k = static_cast<const uint8_t *>(pool->k);
-    a.pool_v = static_cast<const uint8_t *>(pool->v);
-    a.pool_ab = reinterpret_cast<const float2 *>(pool->ab);
+    a.pages = static_cast<const uint8_t *>(pool->pages);
     a.num_pages = pool->num_pages;
     a.page_table = page_table;
     a.max_pages = max_pages;

@@ -50,8 +50,7 @@ struct CoarsenArgs {
     int32_t *bounds;
     int2 *ents;
     uint32_t *flags;
-    uint8_t *pool_k, *pool_v;
-    float2 *pool_ab;
+    uint8_t *pages;  // node pool: [num_pages][2 * 16 * d * elem + 128]
     int64_t num_pages;
     const int32_t *page_table;
     int max_pages;
@@ -78,8 +77,7 @@ constexpr int kMaxVUnits = 8192;
 
 struct DecodeArgs {
     const void *q;
-    const uint8_t *pool_k, *pool_v;
-    const float2 *pool_ab;
+    const uint8_t *pages;  // node pool: [num_pages][2 * 16 * d * elem + 128]
     int64_t num_pages;
     const int32_t *page_table;
     int max_pages;

@@ -43,17 +43,19 @@
  *    fp32); at most SKV_MAX_SEQS sequences per call.
  *
  * Node pool layout (produced by skv_coarsen, consumed by skv_decode_attn):
- *  A page holds SKV_PAGE_NODES = 16 consecutive entries of ONE unit.
- *    pool.k, pool.v : [num_pages][16][d] in the dtype. Within a page the
- *                     16-byte chunk c of slot n's vector is stored at chunk
- *                     position c ^ (n & 7) (a bank-conflict-free order for
- *                     the tensor-core fragment loads; d * elem >= 128 bytes).
- *    pool.ab        : [num_pages][16] pairs {alpha, beta} (fp32).
+ *  A page holds SKV_PAGE_NODES = 16 consecutive entries of ONE unit, stored
+ *  as one contiguous block of skv_page_bytes(dtype, d) bytes:
+ *    [0, V)        keys   [16][d] in the dtype         (V = 16 * d * elem)
+ *    [V, 2V)       values [16][d] in the dtype
+ *    [2V, 2V+128)  {alpha, beta} fp32 pairs [16]
+ *  Within the key and value blocks the 16-byte chunk c of slot n's vector is
+ *  stored at chunk position c ^ (n & 7) (a bank-conflict-free order for the
+ *  tensor-core fragment loads; d * elem >= 128 bytes). One page is one copy.
  *  page_table : [B][Hkv][max_pages] int32 physical page ids; entry e of unit
  *               (b, h) lives in page page_table[b][h][e / 16], slot e % 16.
  *  lens       : [B][Hkv] int32 entries per unit, in the order sinks, nonempty
  *               middle segments (in token order), recents.
- *  Every pool pointer must be 16-byte aligned.
+ *  The pool pointer must be 16-byte aligned.
  */
 #ifndef SKV_H
 #define SKV_H
@@ -83,10 +85,8 @@ typedef enum { SKV_F32 = 0, SKV_BF16 = 1 } skv_dtype;
 #define SKV_MAX_TOKENS ((1 << 22) - 1) /* per sequence */
 
 typedef struct {
-    void *k;           /* [num_pages][16][d] mean keys (device) */
-    void *v;           /* [num_pages][16][d] mean values (device) */
-    float *ab;         /* [num_pages][16][2] alpha, beta (device) */
-    int64_t num_pages; /* capacity of the three arrays, in pages */
+    void *pages;       /* [num_pages][skv_page_bytes(dtype, d)] (device) */
+    int64_t num_pages; /* capacity, in pages */
 } skv_node_pool;
 
 /* Human-readable name of a status code (static storage; never NULL). */
@@ -94,6 +94,9 @@ const char *skv_status_string(int status);
 
 /* ABI version of this header (major * 100 + minor). */
 int skv_abi_version(void);
+
+/* Bytes of one node-pool page: 2 * 16 * d * elem + 128 (0 for an unsupported dtype or d). */
+size_t skv_page_bytes(skv_dtype dtype, int d);
 
 /*
  * The projection the coarsener draws from proj_seed ("Equal-Variation KV

@@ -38,21 +38,16 @@ def write_entries(pool, table, b, h, kt, vt, alpha, beta):
     if E == 0:
         return
     dev = pool.k.device
-    n_pages = -(-E // skv.PAGE_NODES)
-    pages = table[b, h, :n_pages].long()
-    rows = (pages[:, None] * skv.PAGE_NODES + torch.arange(skv.PAGE_NODES, device=dev)).reshape(-1)[:E]
+    pg, sl = skv._entry_rows(pool, table, b, h, E)
     epc = 16 // pool.k.element_size()
     ch = d // epc
-    slot = torch.arange(E, device=dev) % skv.PAGE_NODES
-    phys = torch.arange(ch, device=dev)[None, :] ^ (slot[:, None] & 7)
-    kflat = pool.k.view(-1, ch, epc)
-    vflat = pool.v.view(-1, ch, epc)
-    ridx = rows[:, None].expand(E, ch)
-    kflat[ridx, phys] = kt.to(pool.dtype).reshape(E, ch, epc).to(dev)
-    vflat[ridx, phys] = vt.to(pool.dtype).reshape(E, ch, epc).to(dev)
-    abflat = pool.ab.view(-1, 2)
-    abflat[rows, 0] = alpha.float().to(dev)
-    abflat[rows, 1] = beta.float().to(dev)
+    phys = torch.arange(ch, device=dev)[None, :] ^ (sl[:, None] & 7)
+    k4 = pool.k.view(pool.num_pages, skv.PAGE_NODES, ch, epc)
+    v4 = pool.v.view(pool.num_pages, skv.PAGE_NODES, ch, epc)
+    k4[pg[:, None], sl[:, None], phys] = kt.to(pool.dtype).reshape(E, ch, epc).to(dev)
+    v4[pg[:, None], sl[:, None], phys] = vt.to(pool.dtype).reshape(E, ch, epc).to(dev)
+    pool.ab[pg, sl, 0] = alpha.float().to(dev)
+    pool.ab[pg, sl, 1] = beta.float().to(dev)
 
 
 class GpuUnit:

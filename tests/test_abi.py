@@ -37,7 +37,10 @@ def test_status_strings(lib):
         s = lib.skv_status_string(code).decode()
         assert s.startswith("SKV_")
     assert "unknown" in lib.skv_status_string(12345).decode()
-    assert lib.skv_abi_version() == 100
+    assert lib.skv_abi_version() == 200
+    assert lib.skv_page_bytes(1, 128) == 2 * 16 * 128 * 2 + 128
+    assert lib.skv_page_bytes(0, 64) == 2 * 16 * 64 * 4 + 128
+    assert lib.skv_page_bytes(1, 96) == 0
 
 
 def test_workspace_queries_are_host_arithmetic(lib):
@@ -56,7 +59,7 @@ def test_workspace_queries_are_host_arithmetic(lib):
 def test_bad_arguments_rejected_before_any_launch(lib):
     from compressed_decode_attention_equal_b200 import _lib
     null = ctypes.c_void_p(0)
-    pool = _lib.SkvNodePool(0, 0, 0, 0)
+    pool = _lib.SkvNodePool(0, 0)
     st = lib.skv_decode_attn(null, 1, 1, 1, 7, 1, 128, ctypes.byref(pool), null, 4, null, null, null, null, 0, null)
     assert st == _lib.SKV_ERR_INVALID_ARG
     st = lib.skv_decode_attn(null, 1, 1, 1, 7, 2, 128, ctypes.byref(pool), null, 4, null, null, null, null, 0, null)
@@ -70,7 +73,7 @@ def test_bad_arguments_rejected_before_any_launch(lib):
     st = lib.skv_coarsen(null, null, 3, 1, 1, 128, T, 8, 48, N, 0, None, null, 4, null, null, null, null, 0, null)
     assert st == _lib.SKV_ERR_UNSUPPORTED
     Tbad = (ctypes.c_int32 * 1)(-1)
-    pool2 = _lib.SkvNodePool(16, 16, 16, 1)
+    pool2 = _lib.SkvNodePool(16, 1)
     st = lib.skv_coarsen(null, null, 1, 1, 1, 128, Tbad, 8, 48, N, 0, ctypes.byref(pool2), ctypes.c_void_p(16), 4,
                          ctypes.c_void_p(16), null, null, null, 0, null)
     assert st == _lib.SKV_ERR_INVALID_ARG
