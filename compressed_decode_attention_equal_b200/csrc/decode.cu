@@ -302,8 +302,29 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
     asm volatile("griddepcontrol.wait;" ::: "memory");
     build_prefix(a, prefix, scan_scratch);   // ends with __syncthreads: barriers and qbuf are ready
     const long long ptot = prefix[nv];
-    const long long ra = ptot * blockIdx.x / a.ncta;
-    const long long rb = ptot * (blockIdx.x + 1) / a.ncta;
+    // Aligned split: when every unit has the same page count P0 and `cluster` CTAs per unit fit in
+    // the grid, the k = cluster CTAs of a thread-block cluster take equal page ranges of one unit
+    // and merge through distributed shared memory (no global partials, one piece per CTA).
+    // Otherwise the flat page space is cut into ncta equal ranges (stream-K style).
+    const int kcl = a.cluster;
+    const int P0 = prefix[1] - prefix[0];
+    bool uni = true;
+    {
+        const int per = (nv + kDecThreads - 1) / kDecThreads;
+        for (int v = min(tid * per, nv); v < min(tid * per + per, nv); ++v) uni &= (prefix[v + 1] - prefix[v] == P0);
+    }
+    const bool aligned =
+        __syncthreads_and(uni) && kcl > 1 && P0 >= kcl && static_cast<long long>(nv) * kcl <= a.ncta;
+    const int crank = blockIdx.x % kcl;   // rank in the cluster (clusters are consecutive blocks)
+    long long ra, rb;
+    if (aligned) {
+        const int vc = blockIdx.x / kcl;
+        ra = vc < nv ? prefix[vc] + static_cast<long long>(P0) * crank / kcl : 0;
+        rb = vc < nv ? prefix[vc] + static_cast<long long>(P0) * (crank + 1) / kcl : 0;
+    } else {
+        ra = ptot * blockIdx.x / a.ncta;
+        rb = ptot * (blockIdx.x + 1) / a.ncta;
+    }
     __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(a.out);
     // units with no entries get out = 0, lse = -inf (spread over the CTAs)
     for (int v = blockIdx.x; v < nv; v += a.ncta) {
@@ -382,6 +403,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                 }
                 __syncwarp();
             }
+        }
+        if (aligned) {   // the producer joins the consumers' two cluster barriers
+            cluster_sync();
+            cluster_sync();
         }
         return;
     }
@@ -579,19 +604,57 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                 const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
                 outp[oi * D + dim] = __float2bfloat16_rn(val);
                 if (dim == 0) a.lse[oi] = lse2 * kLn2;
+            } else if (aligned) {
+                // the CTA's only piece: keep it in the drained stage ring for the cluster merge
+                float *xl = reinterpret_cast<float *>(stages);
+                xl[rr * D + dim] = val;
+                if (dim == 0) xl[a.pass_rows * D + rr] = lse2;
             } else {
                 const long long pr = (static_cast<long long>(blockIdx.x) * 2 + slot) * a.pass_rows + rr;
                 a.part_v[pr * D + dim] = val;
                 if (dim == 0) a.part_l[pr] = lse2;
             }
         }
-        if (!complete && ctid == 0 && n_split < 2) {
+        if (!complete && !aligned && ctid == 0 && n_split < 2) {
             split_v[n_split] = v;
             split_ps[n_split] = static_cast<int>(ps);
             split_pe[n_split] = static_cast<int>(pe);
             ++n_split;
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));   // mbuf free for the next piece
+    }
+
+    if (aligned) {
+        // ---- cluster merge: rank 0 combines every rank's (out, log2 partition) of the unit ----
+        cluster_sync();   // every rank's piece is in its stage ring
+        if (crank == 0) {
+            const int vc = blockIdx.x / kcl;
+            const int u = vc / a.row_passes, rpass = vc % a.row_passes;
+            const int b = u / a.Hkv, h = u % a.Hkv;
+            const int rows_here = min(a.pass_rows, a.rows - rpass * kRowsPerPass);
+            const uint32_t xl = smem_u32(stages);
+            for (int idx = ctid; idx < rows_here * D; idx += kDecConsumers * 32) {
+                const int rr = idx / D, dim = idx % D;
+                float M = -INFINITY, Ls = 0.0f, Os = 0.0f;
+                for (int r = 0; r < kcl; ++r) {
+                    const uint32_t base = dsmem_addr(xl, r);
+                    const float l2 = ld_dsmem(base + (a.pass_rows * D + rr) * 4);
+                    const float x = ld_dsmem(base + (rr * D + dim) * 4);
+                    if (l2 == -INFINITY) continue;
+                    const float Mn = fmaxf(M, l2);
+                    const float sc = ex2(M - Mn), w = ex2(l2 - Mn);
+                    Ls = fmaf(Ls, sc, w);
+                    Os = fmaf(Os, sc, x * w);
+                    M = Mn;
+                }
+                const int row = rpass * kRowsPerPass + rr;
+                const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
+                outp[oi * D + dim] = __float2bfloat16_rn(Ls > 0.0f ? __fdividef(Os, Ls) : 0.0f);
+                if (dim == 0) a.lse[oi] = Ls > 0.0f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
+            }
+        }
+        cluster_sync();   // remote reads are done before any rank exits
+        return;
     }
 
     // ---- count this CTA's split pieces; merge the units it completes ----
@@ -751,16 +814,25 @@ static cudaError_t launch_split(const DecodeArgs &a0, cudaStream_t s) {
     const size_t smem = split_smem<D, NT>(a.n_vunits);
     cudaError_t e = split_grid<D, NT>(smem, &a.ncta);
     if (e != cudaSuccess) return e;
+    // cluster size for the aligned split (used only if the device finds every unit equally long):
+    // the largest power of two k <= 8 with k CTAs per virtual unit inside the grid
+    a.cluster = 1;
+    while (a.cluster < 8 && static_cast<long long>(a.n_vunits) * a.cluster * 2 <= a.ncta) a.cluster *= 2;
+    a.ncta -= a.ncta % a.cluster;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.ncta);
     cfg.blockDim = dim3(kDecThreads);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
-    cudaLaunchAttribute attr[1];
+    cudaLaunchAttribute attr[2];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = a.cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = a.cluster > 1 ? 2 : 1;
     return cudaLaunchKernelEx(&cfg, k_decode_split<D, NT>, a);
 }
 

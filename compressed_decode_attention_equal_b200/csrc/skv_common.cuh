@@ -176,6 +176,26 @@ __device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
 }
 
 // ---------------------------------------------------------------------------
+// thread-block clusters: barrier across the cluster, distributed shared memory
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+
+// Shared-memory address of the same location in cluster CTA `rank`.
+__device__ __forceinline__ uint32_t dsmem_addr(uint32_t local, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(local), "r"(rank));
+    return r;
+}
+
+__device__ __forceinline__ float ld_dsmem(uint32_t addr) {
+    float v;
+    asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+    return v;
+}
+
+// ---------------------------------------------------------------------------
 // 128-bit products for exact threshold comparisons: a1*b1 >= a2*b2 (all >= 0)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ bool prod_ge(uint64_t a1, uint64_t b1, uint64_t a2, uint64_t b2) {

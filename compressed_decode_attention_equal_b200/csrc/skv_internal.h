@@ -90,6 +90,7 @@ struct DecodeArgs {
     int pass_rows;    // rows a pass holds: min(kRowsPerPass, rows rounded up to 8)
     int n_vunits;     // B * Hkv * row_passes
     int ncta;         // CTAs of the split kernel
+    int cluster;      // CTAs per thread-block cluster (1: no clusters)
     float *part_v;    // [ncta][2][pass_rows][d] split partial outputs (normalised)
     float *part_l;    // [ncta][2][pass_rows] split partial log2-partitions
     int32_t *counters;   // [n_vunits] pieces finished per virtual unit (zero between calls)
