@@ -88,10 +88,11 @@ __device__ __forceinline__ int find_vunit(const int *prefix, int nv, long long f
     return lo;
 }
 
-// Every CTA rebuilds the page prefix over virtual units (lens are tiny and L2-resident).
+// Every CTA rebuilds the page prefix over virtual units (lens are tiny and L2-resident). Run by
+// the consumer warps alone (named barrier 1), so the producer can start copies meanwhile.
 __device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, int *scratch) {
     const int nv = a.n_vunits;
-    const int tid = threadIdx.x, nth = blockDim.x;
+    const int tid = threadIdx.x, nth = kDecConsumers * 32;
     const int per = (nv + nth - 1) / nth;
     const int lo = min(tid * per, nv), hi = min(lo + per, nv);
     int local = 0;
@@ -108,7 +109,7 @@ __device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, i
         if (lane >= off) x += n;
     }
     if (lane == 31) scratch[warp] = x;
-    __syncthreads();
+    asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
     int wp = 0;
     for (int w = 0; w < warp; ++w) wp += scratch[w];
     int run = wp + x - local;
@@ -118,7 +119,7 @@ __device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, i
         run += pages;
     }
     if (tid == nth - 1) prefix[nv] = wp + x;
-    __syncthreads();
+    asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
 }
 
 // First flat page of CTA c's range, and the CTA whose (nonempty) range holds page f.
@@ -284,6 +285,10 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nv = a.n_vunits;
+    // aligned split: rank r > 0 of a cluster stores its piece into rank 0's receive buffer
+    // (cluster - 1 blocks of pass_rows x (D + 1) floats behind the page prefix)
+    float *xbuf = reinterpret_cast<float *>(prefix + nv + 1);
+    cluster_arrive_relaxed();   // this CTA has started (waited on before any remote access)
     if (tid == 0) {   // independent of the inputs: overlaps the wait below
         for (int s = 0; s < kDecStages; ++s) {
             mbar_init(&full[s], 1);
@@ -296,68 +301,162 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
         fence_mbar_init();
     }
     for (int i = tid; i < 2 * L::QBUF / 4; i += kDecThreads) reinterpret_cast<uint32_t *>(qbuf)[i] = 0u;
+    fence_proxy_async_smem();   // the zeros land before the query-row copies
+    // Speculation, set up before the inputs may be read. The aligned split below, if every unit
+    // fills its page-table row (P0 = max_pages), gives this CTA the table columns [c0, c1) of
+    // virtual unit vc. As soon as the inputs are readable the producer copies that unit's query
+    // rows and the range's first pages while the consumers read the lens; if the lens confirm the
+    // guess the ring just continues, otherwise the copies are drained, the barriers re-armed and
+    // the general split runs (a wrong guess costs up to kDecStages page reads).
+    const int kcl = a.cluster;
+    const int crank = blockIdx.x % kcl, vc = blockIdx.x / kcl;   // clusters are consecutive blocks
+    const bool try_spec = kcl > 1 && vc < nv && a.max_pages >= kcl && static_cast<long long>(nv) * kcl <= a.ncta;
+    const int c0 = try_spec ? a.max_pages * crank / kcl : 0;   // max_pages * 8 fits in an int
+    const int c1 = try_spec ? a.max_pages * (crank + 1) / kcl : 0;
+    const int n_first = min(kDecStages, c1 - c0);
+    __syncthreads();   // barriers initialised, qbuf zeroed
     // let the next launch in the stream become resident as our CTAs retire; then wait for every
     // preceding grid to complete (its writes visible) before reading any input
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     asm volatile("griddepcontrol.wait;" ::: "memory");
-    build_prefix(a, prefix, scan_scratch);   // ends with __syncthreads: barriers and qbuf are ready
-    const long long ptot = prefix[nv];
-    // Aligned split: when every unit has the same page count P0 and `cluster` CTAs per unit fit in
-    // the grid, the k = cluster CTAs of a thread-block cluster take equal page ranges of one unit
-    // and merge through distributed shared memory (no global partials, one piece per CTA).
-    // Otherwise the flat page space is cut into ncta equal ranges (stream-K style).
-    const int kcl = a.cluster;
-    const int P0 = prefix[1] - prefix[0];
-    bool uni = true;
-    {
-        const int per = (nv + kDecThreads - 1) / kDecThreads;
-        for (int v = min(tid * per, nv); v < min(tid * per + per, nv); ++v) uni &= (prefix[v + 1] - prefix[v] == P0);
+    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
+    int spec_page = -1;      // producer lane j: page id of column c0 + j
+    uint32_t spec_bad = 0;   // producer: first pages whose id lies outside the pool
+    if (warp == kDecConsumers) {
+        if (try_spec) {
+            const int u = vc / a.row_passes, rpass = vc % a.row_passes;
+            if (lane < c1 - c0)
+                spec_page = ld_global_s32(a.page_table + static_cast<long long>(u) * a.max_pages + c0 + lane);
+            const int b = u / a.Hkv, h = u % a.Hkv;
+            const int p0 = rpass * kRowsPerPass, p1 = min(p0 + a.pass_rows, a.rows);
+            if (lane == 0) mbar_arrive_expect_tx(&qfull[0], (p1 - p0) * D * 2);
+            __syncwarp();
+            for (int row = p0 + lane; row < p1; row += 32) {
+                const __nv_bfloat16 *src =
+                    q + ((static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G) * D;
+                bulk_g2s(qbuf + (row - p0) * L::QROWB, src, D * 2, &qfull[0]);
+            }
+            for (int k = 0; k < n_first; ++k) {
+                const int phys = __shfl_sync(0xffffffffu, spec_page, k);
+                if (lane == 0) {
+                    if (phys < 0 || phys >= a.num_pages) {   // flagged only if the guess holds
+                        spec_bad |= 1u << k;
+                        svalid[k] = 0;
+                        mbar_arrive(&full[k]);
+                    } else {
+                        svalid[k] = 1;
+                        mbar_arrive_expect_tx(&full[k], G::STAGE);
+                        bulk_g2s(stages + k * G::STAGE, a.pages + static_cast<long long>(phys) * G::STAGE, G::STAGE,
+                                 &full[k]);
+                    }
+                }
+                __syncwarp();
+            }
+        }
+        cluster_wait();   // pairs with the arrival above (the producer touches no remote memory)
+        asm volatile("bar.sync 2, %0;" ::"n"(kDecThreads));   // the consumers' verdict and prefix
+    } else {
+        build_prefix(a, prefix, scan_scratch);
+        // Aligned split: when every unit has the same page count P0 and `cluster` CTAs per unit
+        // fit in the grid, the k = cluster CTAs of a thread-block cluster take equal page ranges of
+        // one unit and merge through distributed shared memory (no global partials, one piece per
+        // CTA). Otherwise the flat page space is cut into ncta equal ranges (stream-K style).
+        const int P0 = prefix[1] - prefix[0];
+        bool uni = true;
+        {
+            const int per = (nv + kDecConsumers * 32 - 1) / (kDecConsumers * 32);
+            for (int v = min(tid * per, nv); v < min(tid * per + per, nv); ++v)
+                uni &= (prefix[v + 1] - prefix[v] == P0);
+        }
+        uni = bar_and(1, kDecConsumers * 32, uni);
+        if (tid == 0) {
+            const bool al = uni && kcl > 1 && P0 >= kcl && static_cast<long long>(nv) * kcl <= a.ncta;
+            misc[8] = al ? 1 : 0;
+            misc[9] = (al && try_spec && P0 == a.max_pages) ? 1 : 0;
+        }
+        cluster_wait();   // every CTA of the cluster has started
+        asm volatile("bar.arrive 2, %0;" ::"n"(kDecThreads));
+        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));   // misc visible to every consumer
     }
-    const bool aligned =
-        __syncthreads_and(uni) && kcl > 1 && P0 >= kcl && static_cast<long long>(nv) * kcl <= a.ncta;
-    const int crank = blockIdx.x % kcl;   // rank in the cluster (clusters are consecutive blocks)
+    const bool aligned = misc[8] != 0;
+    const bool spec_ok = misc[9] != 0;
+    bool alive = true;
+    if (try_spec && !spec_ok) {
+        // wrong guess: wait for the speculative copies, then re-arm every barrier
+        if (warp == kDecConsumers) {
+            bool ok = true;
+            for (int k = 0; k < n_first; ++k) ok &= mbar_wait(&full[k], 0);
+            ok &= mbar_wait(&qfull[0], 0);
+            if (lane == 0) misc[10] = ok ? 1 : 0;
+            if (!ok && lane == 0) raise_flag(a.flags, FLAG_TIMEOUT);
+        }
+        __syncthreads();
+        alive = misc[10] != 0;
+        if (tid == 0 && alive) {
+            for (int s2 = 0; s2 < kDecStages; ++s2) {
+                mbar_inval(&full[s2]);
+                mbar_inval(&empty[s2]);
+                mbar_init(&full[s2], 1);
+                mbar_init(&empty[s2], NT);
+            }
+            for (int s2 = 0; s2 < 2; ++s2) {
+                mbar_inval(&qfull[s2]);
+                mbar_inval(&qempty[s2]);
+                mbar_init(&qfull[s2], 1);
+                mbar_init(&qempty[s2], kDecConsumers);
+            }
+            fence_mbar_init();
+        }
+        __syncthreads();
+    }
+    const long long ptot = prefix[nv];
+    const int P0 = prefix[1] - prefix[0];
     long long ra, rb;
     if (aligned) {
-        const int vc = blockIdx.x / kcl;
-        ra = vc < nv ? prefix[vc] + static_cast<long long>(P0) * crank / kcl : 0;
-        rb = vc < nv ? prefix[vc] + static_cast<long long>(P0) * (crank + 1) / kcl : 0;
+        ra = vc < nv ? prefix[vc] + P0 * crank / kcl : 0;
+        rb = vc < nv ? prefix[vc] + P0 * (crank + 1) / kcl : 0;
     } else {
         ra = ptot * blockIdx.x / a.ncta;
         rb = ptot * (blockIdx.x + 1) / a.ncta;
     }
     __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(a.out);
-    // units with no entries get out = 0, lse = -inf (spread over the CTAs)
-    for (int v = blockIdx.x; v < nv; v += a.ncta) {
-        if (prefix[v + 1] != prefix[v]) continue;
-        const int u = v / a.row_passes, rpass = v % a.row_passes;
-        const int b = u / a.Hkv, h = u % a.Hkv;
-        for (int idx = tid; idx < a.pass_rows * D; idx += kDecThreads) {
-            const int rr = idx / D, dim = idx % D;
-            const int row = rpass * kRowsPerPass + rr;
-            if (row >= a.rows) continue;
-            const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
-            outp[oi * D + dim] = __float2bfloat16_rn(0.0f);
-            if (dim == 0) a.lse[oi] = -INFINITY;
+    if (warp < kDecConsumers) {
+        // units with no entries get out = 0, lse = -inf (spread over the CTAs)
+        for (int v = blockIdx.x; v < nv; v += a.ncta) {
+            if (prefix[v + 1] != prefix[v]) continue;
+            const int u = v / a.row_passes, rpass = v % a.row_passes;
+            const int b = u / a.Hkv, h = u % a.Hkv;
+            for (int idx = tid; idx < a.pass_rows * D; idx += kDecConsumers * 32) {
+                const int rr = idx / D, dim = idx % D;
+                const int row = rpass * kRowsPerPass + rr;
+                if (row >= a.rows) continue;
+                const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
+                outp[oi * D + dim] = __float2bfloat16_rn(0.0f);
+                if (dim == 0) a.lse[oi] = -INFINITY;
+            }
         }
     }
     if (ra >= rb) return;
-    const int v0 = find_vunit(prefix, nv, ra);
+    const int v0 = aligned ? vc : find_vunit(prefix, nv, ra);
     const int n_my = static_cast<int>(rb - ra);
-    const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
 
     if (warp == kDecConsumers) {
         // ----------------------------- producer -----------------------------
-        bool alive = true;
-        int v = -1, pi = -1;   // current (nonempty) piece
+        // a confirmed guess has issued piece 0's query rows and pages [0, n_first) already
+        int v = spec_ok ? vc : -1, pi = spec_ok ? 0 : -1;   // current (nonempty) piece
+        const int i_first = spec_ok ? n_first : 0;
+        if (spec_ok && spec_bad != 0 && lane == 0) raise_flag(a.flags, FLAG_BAD_PAGE);
         for (int base = 0; base < n_my && alive; base += 32) {
             int my_page = -1;
-            if (base + lane < n_my) {
+            if (base == 0 && spec_ok) {
+                my_page = spec_page;   // the same columns, read before the lens were known
+            } else if (base + lane < n_my) {
                 const long long f = ra + base + lane;
                 const int vv = find_vunit(prefix, nv, f);
                 my_page = a.page_table[static_cast<long long>(vv / a.row_passes) * a.max_pages + (f - prefix[vv])];
             }
             const int cnt = min(32, n_my - base);
-            for (int k = 0; k < cnt; ++k) {
+            for (int k = base < i_first ? i_first - base : 0; k < cnt; ++k) {
                 const int i = base + k;
                 const long long f = ra + i;
                 if (v < 0 || f >= prefix[v + 1]) {
@@ -404,10 +503,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                 __syncwarp();
             }
         }
-        if (aligned) {   // the producer joins the consumers' two cluster barriers
-            cluster_sync();
-            cluster_sync();
-        }
+        if (aligned) cluster_sync();   // the producer joins the consumers' cluster barrier
         return;
     }
 
@@ -417,7 +513,6 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
     const int ctid = tid;   // 0 .. 127
     const float c_scale = kLog2e * rsqrtf(static_cast<float>(D));
     int i0 = 0, pi = 0;
-    bool alive = true;
     int split_v[2] = {0, 0}, split_ps[2] = {0, 0}, split_pe[2] = {0, 0}, n_split = 0;   // (thread 0)
     for (int v = v0; v < nv && prefix[v] < rb; ++v) {
         const long long ps = prefix[v], pe = prefix[v + 1];
@@ -605,10 +700,17 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                 outp[oi * D + dim] = __float2bfloat16_rn(val);
                 if (dim == 0) a.lse[oi] = lse2 * kLn2;
             } else if (aligned) {
-                // the CTA's only piece: keep it in the drained stage ring for the cluster merge
-                float *xl = reinterpret_cast<float *>(stages);
-                xl[rr * D + dim] = val;
-                if (dim == 0) xl[a.pass_rows * D + rr] = lse2;
+                // the CTA's only piece: rank 0 keeps it in its drained stage ring, the other ranks
+                // store it into rank 0's receive buffer (no remote round trips)
+                if (crank == 0) {
+                    float *xl = reinterpret_cast<float *>(stages);
+                    xl[rr * D + dim] = val;
+                    if (dim == 0) xl[a.pass_rows * D + rr] = lse2;
+                } else {
+                    const uint32_t xr = dsmem_addr(smem_u32(xbuf + (crank - 1) * a.pass_rows * (D + 1)), 0);
+                    st_dsmem(xr + (rr * D + dim) * 4, val);
+                    if (dim == 0) st_dsmem(xr + (a.pass_rows * D + rr) * 4, lse2);
+                }
             } else {
                 const long long pr = (static_cast<long long>(blockIdx.x) * 2 + slot) * a.pass_rows + rr;
                 a.part_v[pr * D + dim] = val;
@@ -626,34 +728,31 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
 
     if (aligned) {
         // ---- cluster merge: rank 0 combines every rank's (out, log2 partition) of the unit ----
-        cluster_sync();   // every rank's piece is in its stage ring
-        if (crank == 0) {
-            const int vc = blockIdx.x / kcl;
-            const int u = vc / a.row_passes, rpass = vc % a.row_passes;
-            const int b = u / a.Hkv, h = u % a.Hkv;
-            const int rows_here = min(a.pass_rows, a.rows - rpass * kRowsPerPass);
-            const uint32_t xl = smem_u32(stages);
-            for (int idx = ctid; idx < rows_here * D; idx += kDecConsumers * 32) {
-                const int rr = idx / D, dim = idx % D;
-                float M = -INFINITY, Ls = 0.0f, Os = 0.0f;
-                for (int r = 0; r < kcl; ++r) {
-                    const uint32_t base = dsmem_addr(xl, r);
-                    const float l2 = ld_dsmem(base + (a.pass_rows * D + rr) * 4);
-                    const float x = ld_dsmem(base + (rr * D + dim) * 4);
-                    if (l2 == -INFINITY) continue;
-                    const float Mn = fmaxf(M, l2);
-                    const float sc = ex2(M - Mn), w = ex2(l2 - Mn);
-                    Ls = fmaf(Ls, sc, w);
-                    Os = fmaf(Os, sc, x * w);
-                    M = Mn;
-                }
-                const int row = rpass * kRowsPerPass + rr;
-                const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
-                outp[oi * D + dim] = __float2bfloat16_rn(Ls > 0.0f ? __fdividef(Os, Ls) : 0.0f);
-                if (dim == 0) a.lse[oi] = Ls > 0.0f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
+        cluster_sync();   // release / acquire: the other ranks' stores into xbuf are visible
+        if (crank != 0) return;
+        const int u = vc / a.row_passes, rpass = vc % a.row_passes;
+        const int b = u / a.Hkv, h = u % a.Hkv;
+        const int rows_here = min(a.pass_rows, a.rows - rpass * kRowsPerPass);
+        const float *own = reinterpret_cast<const float *>(stages);
+        for (int idx = ctid; idx < rows_here * D; idx += kDecConsumers * 32) {
+            const int rr = idx / D, dim = idx % D;
+            float M = -INFINITY, Ls = 0.0f, Os = 0.0f;
+            for (int r = 0; r < kcl; ++r) {
+                const float *src = r == 0 ? own : xbuf + (r - 1) * a.pass_rows * (D + 1);
+                const float l2 = src[a.pass_rows * D + rr];
+                if (l2 == -INFINITY) continue;
+                const float x = src[rr * D + dim];
+                const float Mn = fmaxf(M, l2);
+                const float sc = ex2(M - Mn), w = ex2(l2 - Mn);
+                Ls = fmaf(Ls, sc, w);
+                Os = fmaf(Os, sc, x * w);
+                M = Mn;
             }
+            const int row = rpass * kRowsPerPass + rr;
+            const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
+            outp[oi * D + dim] = __float2bfloat16_rn(Ls > 0.0f ? __fdividef(Os, Ls) : 0.0f);
+            if (dim == 0) a.lse[oi] = Ls > 0.0f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
         }
-        cluster_sync();   // remote reads are done before any rank exits
         return;
     }
 
@@ -764,17 +863,30 @@ __global__ void __launch_bounds__(128) k_decode_f32(const DecodeArgs a) {
 // host side
 // ---------------------------------------------------------------------------
 template <int D, int NT>
-static size_t split_smem(int n_vunits) {
-    return SplitSmem<D, NT>::FIXED + static_cast<size_t>(n_vunits + 1) * 4;
+static size_t split_smem(int n_vunits, int cluster) {
+    return SplitSmem<D, NT>::FIXED + static_cast<size_t>(n_vunits + 1) * 4 +
+           static_cast<size_t>(cluster - 1) * (NT * 8) * (D + 1) * 4;   // aligned-split receive buffer
 }
 
-// Grid size of the split kernel for one (device, shared-memory size): SMs x resident CTAs.
-// Queried once and cached, so that later calls (and stream capture) issue no attribute queries.
+constexpr int kMaxCluster = 8;   // portable cluster size limit
+// cluster > 1 needs n_vunits * cluster <= ncta <= kMaxDecodeCtas
 template <int D, int NT>
-static cudaError_t split_grid(size_t smem, int *ncta) {
+static size_t split_smem_max() {
+    const size_t a = split_smem<D, NT>(kMaxVUnits, 1);
+    const size_t b = split_smem<D, NT>(kMaxDecodeCtas / 2, kMaxCluster);
+    return a > b ? a : b;
+}
+
+// Co-resident CTAs of the split kernel for one (device, shared-memory size, cluster size):
+// SMs x resident CTAs without clusters, resident clusters x cluster size with them (a cluster
+// must fit inside one GPC). Queried once and cached, so that later calls (and stream capture)
+// issue no attribute queries.
+template <int D, int NT>
+static cudaError_t split_grid(size_t smem, int cluster, int *ncta) {
     struct Entry {
         int dev;
         size_t smem;
+        int cluster;
         int ncta;
     };
     static std::mutex mu;
@@ -784,41 +896,82 @@ static cudaError_t split_grid(size_t smem, int *ncta) {
     if (e != cudaSuccess) return e;
     std::lock_guard<std::mutex> lock(mu);
     for (const Entry &c : cache)
-        if (c.dev == dev && c.smem == smem) {
+        if (c.dev == dev && c.smem == smem && c.cluster == cluster) {
             *ncta = c.ncta;
             return cudaSuccess;
         }
     bool configured = false;
     for (const Entry &c : cache) configured |= (c.dev == dev);
     if (!configured) {
-        // the largest request any call can make (the page prefix of kMaxVUnits virtual units)
+        // the largest request any call can make
         e = cudaFuncSetAttribute(k_decode_split<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(split_smem<D, NT>(kMaxVUnits)));
+                                 static_cast<int>(split_smem_max<D, NT>()));
         if (e != cudaSuccess) return e;
     }
-    int sms = 0, occ = 0;
-    if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-    if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_split<D, NT>, kDecThreads, smem)) !=
-        cudaSuccess)
-        return e;
-    int n = sms * (occ > 0 ? occ : 1);
-    if (n > kMaxDecodeCtas) n = kMaxDecodeCtas;
-    cache.push_back({dev, smem, n});
+    int n = 0;
+    if (cluster == 1) {
+        int sms = 0, occ = 0;
+        if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_split<D, NT>, kDecThreads, smem)) !=
+            cudaSuccess)
+            return e;
+        n = sms * (occ > 0 ? occ : 1);
+    } else {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(cluster);
+        cfg.blockDim = dim3(kDecThreads);
+        cfg.dynamicSmemBytes = smem;
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeClusterDimension;
+        attr.val.clusterDim.x = cluster;
+        attr.val.clusterDim.y = 1;
+        attr.val.clusterDim.z = 1;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        int nc = 0;
+        if (cudaOccupancyMaxActiveClusters(&nc, k_decode_split<D, NT>, &cfg) != cudaSuccess) {
+            (void)cudaGetLastError();   // this cluster size is not available: not an error of the call
+            nc = 0;
+        }
+        n = nc * cluster;
+    }
+    if (n > kMaxDecodeCtas) n = kMaxDecodeCtas - kMaxDecodeCtas % cluster;
+    cache.push_back({dev, smem, cluster, n});
     *ncta = n;
+    return cudaSuccess;
+}
+
+// Grid and cluster size of one call. The cluster size is the largest k <= 8 for which one
+// cluster of k CTAs per virtual unit is co-resident and keeps at least 3/4 of the grid busy
+// (an aligned split then streams at most 4/3 of the pages per CTA a stream-K split would, and
+// saves its global merges). It is used only if the device finds every unit equally long;
+// otherwise the same grid runs the stream-K split.
+template <int D, int NT>
+static cudaError_t split_config(DecodeArgs *a, size_t *smem) {
+    *smem = split_smem<D, NT>(a->n_vunits, 1);
+    cudaError_t e = split_grid<D, NT>(*smem, 1, &a->ncta);
+    if (e != cudaSuccess) return e;
+    a->cluster = 1;
+    for (int k = a->ncta / a->n_vunits < kMaxCluster ? a->ncta / a->n_vunits : kMaxCluster; k > 1; --k) {
+        const size_t sk = split_smem<D, NT>(a->n_vunits, k);
+        int n = 0;
+        if ((e = split_grid<D, NT>(sk, k, &n)) != cudaSuccess) return e;
+        if (static_cast<long long>(a->n_vunits) * k <= n && static_cast<long long>(a->n_vunits) * k * 4 >= 3LL * n) {
+            a->cluster = k;
+            a->ncta = n;
+            *smem = sk;
+            break;
+        }
+    }
     return cudaSuccess;
 }
 
 template <int D, int NT>
 static cudaError_t launch_split(const DecodeArgs &a0, cudaStream_t s) {
     DecodeArgs a = a0;
-    const size_t smem = split_smem<D, NT>(a.n_vunits);
-    cudaError_t e = split_grid<D, NT>(smem, &a.ncta);
+    size_t smem = 0;
+    cudaError_t e = split_config<D, NT>(&a, &smem);
     if (e != cudaSuccess) return e;
-    // cluster size for the aligned split (used only if the device finds every unit equally long):
-    // the largest power of two k <= 8 with k CTAs per virtual unit inside the grid
-    a.cluster = 1;
-    while (a.cluster < 8 && static_cast<long long>(a.n_vunits) * a.cluster * 2 <= a.ncta) a.cluster *= 2;
-    a.ncta -= a.ncta % a.cluster;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.ncta);
     cfg.blockDim = dim3(kDecThreads);
@@ -857,18 +1010,27 @@ cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
 
 namespace skv {
 
+template <int D, int NT>
+static cudaError_t split_ctas(const DecodeArgs &a0, int *ncta) {
+    DecodeArgs a = a0;
+    size_t smem = 0;
+    const cudaError_t e = split_config<D, NT>(&a, &smem);
+    *ncta = a.ncta;
+    return e;
+}
+
 // The grid k_decode_split would use for these arguments (bf16 caches), for callers that must size
 // split-partial storage before launching. Queries (and caches) the same occupancy as the launcher.
 cudaError_t decode_split_ctas(const DecodeArgs &a, int *ncta) {
     const int nt = a.pass_rows / 8 + (a.pass_rows % 8 ? 1 : 0);
     if (a.d == 128) {
-        if (nt == 1) return split_grid<128, 1>(split_smem<128, 1>(a.n_vunits), ncta);
-        if (nt == 2) return split_grid<128, 2>(split_smem<128, 2>(a.n_vunits), ncta);
-        return split_grid<128, 4>(split_smem<128, 4>(a.n_vunits), ncta);
+        if (nt == 1) return split_ctas<128, 1>(a, ncta);
+        if (nt == 2) return split_ctas<128, 2>(a, ncta);
+        return split_ctas<128, 4>(a, ncta);
     }
-    if (nt == 1) return split_grid<64, 1>(split_smem<64, 1>(a.n_vunits), ncta);
-    if (nt == 2) return split_grid<64, 2>(split_smem<64, 2>(a.n_vunits), ncta);
-    return split_grid<64, 4>(split_smem<64, 4>(a.n_vunits), ncta);
+    if (nt == 1) return split_ctas<64, 1>(a, ncta);
+    if (nt == 2) return split_ctas<64, 2>(a, ncta);
+    return split_ctas<64, 4>(a, ncta);
 }
 
 }  // namespace skv

@@ -136,3 +136,58 @@ def test_decode_repeated_calls_at_bench_shape_are_identical():
     units = gpu_units(pool, table, ln, B, Hkv)
     ref_out, ref_lse = oracle.decode(q[sample].double().cpu().numpy(), [units[b] for b in sample])
     check_decode(firsts[0][0][sample], firsts[0][1][sample], ref_out, ref_lse, torch.bfloat16, "bench shape")
+
+
+def _widen_table(table, extra, fill):
+    """The same page table with `extra` more columns holding `fill` (ids past every unit's pages)."""
+    B, Hkv, P = table.shape
+    wide = torch.full((B, Hkv, P + extra), fill, dtype=table.dtype, device=table.device)
+    wide[:, :, :P] = table
+    return wide
+
+
+def test_decode_uniform_lens_table_wider_than_units():
+    """Equal-length units in a page table wider than they need, its spare columns holding ids
+    outside the pool: pages read ahead for a full-width table are discarded, no flag is raised,
+    and the outputs match the oracle."""
+    B, Hq, Hkv, d = 16, 28, 4, 128
+    pool, table, lens, q = _synthetic(B, Hq, Hkv, 1, d, [700] * B, torch.bfloat16, seed=21)
+    wide = _widen_table(table, 13, pool.num_pages + 1000)
+    ws = torch.zeros(skv.decode_workspace_bytes(B, 1, Hq, Hkv, d, wide.shape[2]), dtype=torch.uint8, device="cuda")
+    for _ in range(3):
+        out, lse = skv.decode_attn(q, Hkv, pool, wide, lens, workspace=ws)
+        st, flags = skv.workspace_error(ws)
+        assert st == 0 and flags == 0, flags
+    units = gpu_units(pool, table, lens, B, Hkv)
+    ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), units)
+    check_decode(out, lse, ref_out, ref_lse, torch.bfloat16, "wide table")
+
+
+def test_decode_ragged_lens_few_units():
+    """Few units of different lengths (the launch a uniform batch of this size would use, with the
+    read-ahead discarded and the flat split taking over)."""
+    lens = [700, 1147, 33, 512, 900, 1, 0, 640, 16, 17, 300, 1147, 64, 65, 999, 250]
+    _run(len(lens), 28, 4, 1, 128, lens, torch.bfloat16, seed=22)
+
+
+def test_decode_bad_page_in_first_pages_is_flagged():
+    """A bad page id among the first pages of a full-width, equal-length batch (read before the
+    lens are known) raises the flag once the lens confirm the split; other units are exact."""
+    B, Hq, Hkv, d = 16, 28, 4, 128
+    pool, table, lens, q = _synthetic(B, Hq, Hkv, 1, d, [700] * B, torch.bfloat16, seed=23)
+    bad = table.clone()
+    bad[5, 1, 0] = pool.num_pages + 9
+    ws = torch.zeros(skv.decode_workspace_bytes(B, 1, Hq, Hkv, d, table.shape[2]), dtype=torch.uint8,
+                     device="cuda")
+    out, lse = skv.decode_attn(q, Hkv, pool, bad, lens, workspace=ws)
+    st, flags = skv.workspace_error(ws)
+    assert st == skv._lib.SKV_ERR_DEVICE and flags & skv._lib.FLAG_BAD_PAGE
+    keep = [b for b in range(B) if b != 5]
+    units = gpu_units(pool, table, lens, B, Hkv)
+    ref_out, ref_lse = oracle.decode(q[keep].double().cpu().numpy(), [units[b] for b in keep])
+    check_decode(out[keep], lse[keep], ref_out, ref_lse, torch.bfloat16, "bad first page")
+    out2, lse2 = skv.decode_attn(q, Hkv, pool, table, lens, workspace=ws)
+    st, flags = skv.workspace_error(ws)
+    assert st == 0 and flags == 0
+    ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), units)
+    check_decode(out2, lse2, ref_out, ref_lse, torch.bfloat16, "after bad page")
