@@ -61,10 +61,14 @@ struct SplitSmem {
     static constexpr int QROWB = D * 2 + 16;              // padded query row: conflict-free ldmatrix
     static constexpr int QBUF = NT * 8 * QROWB;           // the query rows of one piece
     static constexpr int STAGES_BYTES = kDecStages * PageGeom<D>::STAGE;
-    static constexpr int MBUF_FLOATS = kDecConsumers * 8 * (D + 2);
+    static constexpr int MST = D + 4;                     // mbuf row stride: 16-byte rows
+    static constexpr int MBUF_FLOATS = kDecConsumers * 8 * MST;
     static constexpr int BARS = 2 * kDecStages + 4;
-    static constexpr size_t FIXED =
-        16 + STAGES_BYTES + 2 * QBUF + BARS * 8 + kDecStages * 4 + MBUF_FLOATS * 4 + 16 * 4;
+    static constexpr int ROWS = NT * 8;                   // query rows of one piece
+    static constexpr int WST = 9;                         // merge weights per row (<= 8) + log2 partition
+    static constexpr int EPI_BYTES = ROWS * 8 + ROWS * WST * 4;
+    static constexpr size_t FIXED = 16 + STAGES_BYTES + 2 * QBUF + BARS * 8 + kDecStages * 4 + MBUF_FLOATS * 4 +
+                                    16 * 4 + ((EPI_BYTES + 15) / 16) * 16;
 };
 
 __device__ __forceinline__ int clamp_entries(const DecodeArgs &a, int u) {
@@ -280,14 +284,17 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
     int *svalid = reinterpret_cast<int *>(qempty + 2);
     float *mbuf = reinterpret_cast<float *>(svalid + kDecStages);
     int *misc = reinterpret_cast<int *>(mbuf + L::MBUF_FLOATS);
-    int *prefix = misc + 16;
+    // epilogue tables: output row index and merge weights per query row of the piece
+    long long *orow = reinterpret_cast<long long *>(misc + 16);
+    float *wrow = reinterpret_cast<float *>(orow + L::ROWS);
+    int *prefix = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(misc + 16) + ((L::EPI_BYTES + 15) / 16) * 16);
     __shared__ int scan_scratch[kDecThreads / 32];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nv = a.n_vunits;
     // aligned split: rank r > 0 of a cluster stores its piece into rank 0's receive buffer
     // (cluster - 1 blocks of pass_rows x (D + 1) floats behind the page prefix)
-    float *xbuf = reinterpret_cast<float *>(prefix + nv + 1);
+    float *xbuf = reinterpret_cast<float *>(prefix + ((nv + 1 + 3) & ~3));   // 16-byte aligned
     cluster_arrive_relaxed();   // this CTA has started (waited on before any remote access)
     if (tid == 0) {   // independent of the inputs: overlaps the wait below
         for (int s = 0; s < kDecStages; ++s) {
@@ -522,6 +529,11 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
         const int u = v / a.row_passes, rpass = v % a.row_passes;
         const int b = u / a.Hkv, h = u % a.Hkv;
         const int Lent = clamp_entries(a, u);
+        const int rows_here = min(a.pass_rows, a.rows - rpass * kRowsPerPass);
+        if (ctid < rows_here) {   // output row of each query row (read after the page loop)
+            const int row = rpass * kRowsPerPass + ctid;
+            orow[ctid] = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
+        }
 
         // Q^T fragments of rows nt*8 + g of this piece (ldmatrix from the producer's copy), |q|^2
         uint32_t qf[NKS][2];
@@ -659,62 +671,79 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
             l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
             l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
         }
-        float *mw = mbuf + warp * 8 * (D + 2);
+        constexpr int MST = L::MST, WST = L::WST;
+        float *mw = mbuf + warp * 8 * MST;
 #pragma unroll
         for (int mt = 0; mt < NKS; ++mt) {
-            mw[(2 * c) * (D + 2) + 16 * mt + g] = o[mt][0];
-            mw[(2 * c + 1) * (D + 2) + 16 * mt + g] = o[mt][1];
-            mw[(2 * c) * (D + 2) + 16 * mt + g + 8] = o[mt][2];
-            mw[(2 * c + 1) * (D + 2) + 16 * mt + g + 8] = o[mt][3];
+            mw[(2 * c) * MST + 16 * mt + g] = o[mt][0];
+            mw[(2 * c + 1) * MST + 16 * mt + g] = o[mt][1];
+            mw[(2 * c) * MST + 16 * mt + g + 8] = o[mt][2];
+            mw[(2 * c + 1) * MST + 16 * mt + g + 8] = o[mt][3];
         }
         if (g == 0) {
-            mw[(2 * c) * (D + 2) + D] = m_run[0];
-            mw[(2 * c) * (D + 2) + D + 1] = l_run[0];
-            mw[(2 * c + 1) * (D + 2) + D] = m_run[1];
-            mw[(2 * c + 1) * (D + 2) + D + 1] = l_run[1];
+            mw[(2 * c) * MST + D] = m_run[0];
+            mw[(2 * c) * MST + D + 1] = l_run[0];
+            mw[(2 * c + 1) * MST + D] = m_run[1];
+            mw[(2 * c + 1) * MST + D + 1] = l_run[1];
         }
         asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
         const bool complete = (ps >= ra) && (pe <= rb);
         const int slot = ps < ra ? 0 : 1;
-        for (int idx = ctid; idx < NT * 8 * D; idx += kDecConsumers * 32) {
-            const int rr = idx / D, dim = idx % D;
-            const int ntr = rr >> 3, j = rr & 7;
-            const int row = rpass * kRowsPerPass + rr;
-            if (rr >= a.pass_rows || row >= a.rows) continue;
+        // per query row: normalised page-group weights, log2 partition and output row
+        if (ctid < rows_here) {
+            const int rr = ctid, ntr = rr >> 3, j = rr & 7;
             float M = -INFINITY;
 #pragma unroll
-            for (int q2 = 0; q2 < PG; ++q2) M = fmaxf(M, mbuf[((q2 * NT + ntr) * 8 + j) * (D + 2) + D]);
-            float Ls = 0.0f, Os = 0.0f;
+            for (int q2 = 0; q2 < PG; ++q2) M = fmaxf(M, mbuf[((q2 * NT + ntr) * 8 + j) * MST + D]);
             const float Mb = M == -INFINITY ? 0.0f : M;
+            float wq[PG], Ls = 0.0f;
 #pragma unroll
             for (int q2 = 0; q2 < PG; ++q2) {
-                const float *st = mbuf + ((q2 * NT + ntr) * 8 + j) * (D + 2);
-                const float w = ex2(st[D] - Mb);
-                Ls = fmaf(st[D + 1], w, Ls);
-                Os = fmaf(st[dim], w, Os);
+                const float *st = mbuf + ((q2 * NT + ntr) * 8 + j) * MST;
+                wq[q2] = ex2(st[D] - Mb);
+                Ls = fmaf(st[D + 1], wq[q2], Ls);
             }
-            const float val = Ls > 0.0f ? __fdividef(Os, Ls) : 0.0f;
-            const float lse2 = Ls > 0.0f ? M + __log2f(Ls) : -INFINITY;
+            const float inv = Ls > 0.0f ? __fdividef(1.0f, Ls) : 0.0f;   // Ls <= entries of a unit
+#pragma unroll
+            for (int q2 = 0; q2 < PG; ++q2) wrow[rr * WST + q2] = wq[q2] * inv;
+            wrow[rr * WST + 8] = Ls > 0.0f ? M + __log2f(Ls) : -INFINITY;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
+        for (int it = ctid; it < rows_here * (D / 4); it += kDecConsumers * 32) {
+            const int rr = it / (D / 4), d4 = (it % (D / 4)) * 4;
+            const int ntr = rr >> 3, j = rr & 7;
+            float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+#pragma unroll
+            for (int q2 = 0; q2 < PG; ++q2) {
+                const float w = wrow[rr * WST + q2];
+                const float4 x = *reinterpret_cast<const float4 *>(mbuf + ((q2 * NT + ntr) * 8 + j) * MST + d4);
+                acc.x = fmaf(w, x.x, acc.x);
+                acc.y = fmaf(w, x.y, acc.y);
+                acc.z = fmaf(w, x.z, acc.z);
+                acc.w = fmaf(w, x.w, acc.w);
+            }
+            const float lse2 = wrow[rr * WST + 8];
             if (complete) {
-                const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
-                outp[oi * D + dim] = __float2bfloat16_rn(val);
-                if (dim == 0) a.lse[oi] = lse2 * kLn2;
+                const long long oi = orow[rr];
+                *reinterpret_cast<uint2 *>(outp + oi * D + d4) =
+                    make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+                if (d4 == 0) a.lse[oi] = lse2 * kLn2;
             } else if (aligned) {
                 // the CTA's only piece: rank 0 keeps it in its drained stage ring, the other ranks
                 // store it into rank 0's receive buffer (no remote round trips)
                 if (crank == 0) {
                     float *xl = reinterpret_cast<float *>(stages);
-                    xl[rr * D + dim] = val;
-                    if (dim == 0) xl[a.pass_rows * D + rr] = lse2;
+                    *reinterpret_cast<float4 *>(xl + rr * D + d4) = acc;
+                    if (d4 == 0) xl[a.pass_rows * D + rr] = lse2;
                 } else {
                     const uint32_t xr = dsmem_addr(smem_u32(xbuf + (crank - 1) * a.pass_rows * (D + 1)), 0);
-                    st_dsmem(xr + (rr * D + dim) * 4, val);
-                    if (dim == 0) st_dsmem(xr + (a.pass_rows * D + rr) * 4, lse2);
+                    st_dsmem_v4(xr + (rr * D + d4) * 4, acc);
+                    if (d4 == 0) st_dsmem(xr + (a.pass_rows * D + rr) * 4, lse2);
                 }
             } else {
                 const long long pr = (static_cast<long long>(blockIdx.x) * 2 + slot) * a.pass_rows + rr;
-                a.part_v[pr * D + dim] = val;
-                if (dim == 0) a.part_l[pr] = lse2;
+                *reinterpret_cast<float4 *>(a.part_v + pr * D + d4) = acc;
+                if (d4 == 0) a.part_l[pr] = lse2;
             }
         }
         if (!complete && !aligned && ctid == 0 && n_split < 2) {
@@ -730,28 +759,42 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
         // ---- cluster merge: rank 0 combines every rank's (out, log2 partition) of the unit ----
         cluster_sync();   // release / acquire: the other ranks' stores into xbuf are visible
         if (crank != 0) return;
-        const int u = vc / a.row_passes, rpass = vc % a.row_passes;
-        const int b = u / a.Hkv, h = u % a.Hkv;
-        const int rows_here = min(a.pass_rows, a.rows - rpass * kRowsPerPass);
+        // orow[] still holds this unit's output rows (written by the piece epilogue)
+        constexpr int WST = L::WST;
+        const int rows_here = min(a.pass_rows, a.rows - (vc % a.row_passes) * kRowsPerPass);
         const float *own = reinterpret_cast<const float *>(stages);
-        for (int idx = ctid; idx < rows_here * D; idx += kDecConsumers * 32) {
-            const int rr = idx / D, dim = idx % D;
-            float M = -INFINITY, Ls = 0.0f, Os = 0.0f;
+        const int blk = a.pass_rows * (D + 1);
+        if (ctid < rows_here) {
+            const int rr = ctid;
+            float M = -INFINITY;
+            for (int r = 0; r < kcl; ++r) M = fmaxf(M, (r == 0 ? own : xbuf + (r - 1) * blk)[a.pass_rows * D + rr]);
+            const float Mb = M == -INFINITY ? 0.0f : M;
+            float Ls = 0.0f;
             for (int r = 0; r < kcl; ++r) {
-                const float *src = r == 0 ? own : xbuf + (r - 1) * a.pass_rows * (D + 1);
-                const float l2 = src[a.pass_rows * D + rr];
-                if (l2 == -INFINITY) continue;
-                const float x = src[rr * D + dim];
-                const float Mn = fmaxf(M, l2);
-                const float sc = ex2(M - Mn), w = ex2(l2 - Mn);
-                Ls = fmaf(Ls, sc, w);
-                Os = fmaf(Os, sc, x * w);
-                M = Mn;
+                const float w = ex2((r == 0 ? own : xbuf + (r - 1) * blk)[a.pass_rows * D + rr] - Mb);
+                wrow[rr * WST + r] = w;
+                Ls += w;
             }
-            const int row = rpass * kRowsPerPass + rr;
-            const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
-            outp[oi * D + dim] = __float2bfloat16_rn(Ls > 0.0f ? __fdividef(Os, Ls) : 0.0f);
-            if (dim == 0) a.lse[oi] = Ls > 0.0f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
+            const float inv = Ls > 0.0f ? __fdividef(1.0f, Ls) : 0.0f;   // 1 <= Ls <= kcl
+            for (int r = 0; r < kcl; ++r) wrow[rr * WST + r] *= inv;
+            wrow[rr * WST + 8] = Ls > 0.0f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
+        }
+        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
+        for (int it = ctid; it < rows_here * (D / 4); it += kDecConsumers * 32) {
+            const int rr = it / (D / 4), d4 = (it % (D / 4)) * 4;
+            float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            for (int r = 0; r < kcl; ++r) {
+                const float w = wrow[rr * WST + r];
+                const float4 x = *reinterpret_cast<const float4 *>((r == 0 ? own : xbuf + (r - 1) * blk) + rr * D + d4);
+                acc.x = fmaf(w, x.x, acc.x);
+                acc.y = fmaf(w, x.y, acc.y);
+                acc.z = fmaf(w, x.z, acc.z);
+                acc.w = fmaf(w, x.w, acc.w);
+            }
+            const long long oi = orow[rr];
+            *reinterpret_cast<uint2 *>(outp + oi * D + d4) =
+                make_uint2(pack_bf16x2(acc.x, acc.y), pack_bf16x2(acc.z, acc.w));
+            if (d4 == 0) a.lse[oi] = wrow[rr * WST + 8];
         }
         return;
     }
@@ -864,7 +907,7 @@ __global__ void __launch_bounds__(128) k_decode_f32(const DecodeArgs a) {
 // ---------------------------------------------------------------------------
 template <int D, int NT>
 static size_t split_smem(int n_vunits, int cluster) {
-    return SplitSmem<D, NT>::FIXED + static_cast<size_t>(n_vunits + 1) * 4 +
+    return SplitSmem<D, NT>::FIXED + static_cast<size_t>((n_vunits + 1 + 3) & ~3) * 4 +
            static_cast<size_t>(cluster - 1) * (NT * 8) * (D + 1) * 4;   // aligned-split receive buffer
 }
 

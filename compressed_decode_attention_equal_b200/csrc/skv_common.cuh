@@ -222,6 +222,12 @@ __device__ __forceinline__ void st_dsmem(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
 
+__device__ __forceinline__ void st_dsmem_v4(uint32_t addr, float4 v) {
+    asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "f"(v.x), "f"(v.y), "f"(v.z),
+                 "f"(v.w)
+                 : "memory");
+}
+
 // Split cluster barrier: every thread arrives once early (no ordering) and waits before its first
 // access to another CTA's shared memory, so that every CTA of the cluster has started by then.
 __device__ __forceinline__ void cluster_arrive_relaxed() {
