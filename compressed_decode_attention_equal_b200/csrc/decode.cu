@@ -579,13 +579,16 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                 alive = false;
                 break;
             }
-            if (svalid[s]) {
-                const int nvalid = min(kPageNodes, Lent - (lo + k) * kPageNodes);
+            const bool valid = svalid[s] != 0;
+            const int nvalid = min(kPageNodes, Lent - (lo + k) * kPageNodes);
+            float sacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            uint32_t vf[NKS][4];
+            float2 ab0 = make_float2(0.0f, 0.0f), ab1 = ab0;
+            if (valid) {
                 const uint32_t kb = smem_u32(stages + s * G::STAGE);
                 const uint32_t vb = kb + G::VEC_BYTES;
                 const float2 *ab = reinterpret_cast<const float2 *>(stages + s * G::STAGE + 2 * G::VEC_BYTES);
                 // S^T (16 nodes x 8 rows) = K (16 x D) Q^T (D x 8)
-                float sacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
                 {
                     const int mi = lane >> 3, node = (lane & 7) + 8 * (mi & 1);
 #pragma unroll
@@ -596,7 +599,21 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                         mma_bf16(sacc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
                     }
                 }
-                const float2 ab0 = ab[g], ab1 = ab[g + 8];
+                // V^T fragments (A operand of O^T = V^T P^T) into registers now, so the stage goes
+                // back to the producer before the softmax
+                {
+                    const int mi = lane >> 3, node = (lane & 7) + 8 * (mi >> 1);
+#pragma unroll
+                    for (int mt = 0; mt < NKS; ++mt)
+                        ldsm_x4_t(vb + node * G::ROWB + (swz(2 * mt + (mi & 1), node) << 4), vf[mt][0], vf[mt][1],
+                                  vf[mt][2], vf[mt][3]);
+                }
+                ab0 = ab[g];
+                ab1 = ab[g + 8];
+            }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&empty[s]);   // the page is in registers: release the stage
+            if (valid) {
                 float sl[4];
                 sl[0] = g < nvalid ? fmaf(sacc[0], c_scale, kLog2e * fmaf(qn_r0, ab0.y, ab0.x)) : -INFINITY;
                 sl[1] = g < nvalid ? fmaf(sacc[1], c_scale, kLog2e * fmaf(qn_r1, ab0.y, ab0.x)) : -INFINITY;
@@ -631,36 +648,23 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                 const uint32_t bp0 = movmatrix_t(pack_bf16x2(p0, p1));
                 const uint32_t bp1 = movmatrix_t(pack_bf16x2(p2, p3));
                 // O^T (D x 8) += V^T (D x 16) P^T (16 x 8)
-                {
-                    const int mi = lane >> 3, node = (lane & 7) + 8 * (mi >> 1);
-                    if (nvalid == kPageNodes) {
+                if (nvalid == kPageNodes) {
 #pragma unroll
-                        for (int mt = 0; mt < NKS; ++mt) {
-                            const int chunk = 2 * mt + (mi & 1);
-                            uint32_t a0, a1, a2, a3;
-                            ldsm_x4_t(vb + node * G::ROWB + (swz(chunk, node) << 4), a0, a1, a2, a3);
-                            mma_bf16(o[mt], a0, a1, a2, a3, bp0, bp1);
-                        }
-                    } else {
-                        // slots past the unit's last entry may hold anything (NaN included):
-                        // zero their V^T elements, since P = 0 does not cancel NaN in the product.
-                        // This thread's fragment holds nodes 2c, 2c+1 (a0..a3) and 2c+8, 2c+9 (a4..a7).
-                        const uint32_t m_lo =
-                            (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
-                        const uint32_t m_hi =
-                            (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
+                    for (int mt = 0; mt < NKS; ++mt) mma_bf16(o[mt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], bp0, bp1);
+                } else {
+                    // slots past the unit's last entry may hold anything (NaN included): zero their
+                    // V^T elements, since P = 0 does not cancel NaN in the product. This thread's
+                    // fragment holds nodes 2c, 2c+1 (a0..a3) and 2c+8, 2c+9 (a4..a7).
+                    const uint32_t m_lo =
+                        (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
+                    const uint32_t m_hi =
+                        (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
 #pragma unroll
-                        for (int mt = 0; mt < NKS; ++mt) {
-                            const int chunk = 2 * mt + (mi & 1);
-                            uint32_t a0, a1, a2, a3;
-                            ldsm_x4_t(vb + node * G::ROWB + (swz(chunk, node) << 4), a0, a1, a2, a3);
-                            mma_bf16(o[mt], a0 & m_lo, a1 & m_lo, a2 & m_hi, a3 & m_hi, bp0, bp1);
-                        }
-                    }
+                    for (int mt = 0; mt < NKS; ++mt)
+                        mma_bf16(o[mt], vf[mt][0] & m_lo, vf[mt][1] & m_lo, vf[mt][2] & m_hi, vf[mt][3] & m_hi, bp0,
+                                 bp1);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);
         }
         i0 += npg;
         ++pi;
