@@ -107,9 +107,14 @@ def coarsen_workspace_bytes(Hkv: int, d: int, T_list, N_list, n_sink: int, n_rec
 def coarsen(k: torch.Tensor, v: torch.Tensor, Hkv: int, T_list, N_list, n_sink: int, n_recent: int,
             proj_seed: int, pool: NodePool, page_table: torch.Tensor, lens: torch.Tensor | None = None,
             boundaries: torch.Tensor | None = None, cumvar: torch.Tensor | None = None,
-            workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+            workspace: torch.Tensor | None = None, stream=None, representative: str = "mean") -> torch.Tensor:
     """Coarsen B sequences (k, v: [sum_b Hkv*T_b, d], sequence b a contiguous [Hkv, T_b, d] block)
-    into `pool` through `page_table` [B, Hkv, max_pages] int32. Returns lens [B, Hkv] int32."""
+    into `pool` through `page_table` [B, Hkv, max_pages] int32. Returns lens [B, Hkv] int32.
+    representative: "mean" (skv_coarsen) or "variation" (skv_coarsen_ex with the
+    variation-weighted segment key and value)."""
+    reps = {"mean": _lib.SKV_REP_MEAN, "variation": _lib.SKV_REP_VARIATION_WEIGHTED}
+    if representative not in reps:
+        raise ValueError(f"representative must be one of {sorted(reps)}")
     B = len(T_list)
     d = k.shape[-1]
     if v.shape != k.shape or v.dtype != k.dtype:
@@ -128,14 +133,19 @@ def coarsen(k: torch.Tensor, v: torch.Tensor, Hkv: int, T_list, N_list, n_sink: 
         workspace = torch.zeros(ws_bytes, dtype=torch.uint8, device=dev)
     ps = pool.struct()
     null = ctypes.c_void_p(0)
-    st = _lib.load().skv_coarsen(
-        _dev(k, "k") if k.numel() else null, _dev(v, "v") if v.numel() else null, _code(k.dtype), B, Hkv, d,
-        _i32(T_list), n_sink, n_recent, _i32(N_list), ctypes.c_uint64(proj_seed), ctypes.byref(ps),
-        _dev(page_table, "page_table"), page_table.shape[2], _dev(lens, "lens"),
-        _dev(boundaries, "boundaries") if boundaries is not None else null,
-        _dev(cumvar, "cumvar") if cumvar is not None else null,
-        _dev(workspace, "workspace"), workspace.numel(), ctypes.c_void_p(_stream_handle(stream)))
-    _lib.check(st, "skv_coarsen")
+    args = (_dev(k, "k") if k.numel() else null, _dev(v, "v") if v.numel() else null, _code(k.dtype), B, Hkv, d,
+            _i32(T_list), n_sink, n_recent, _i32(N_list), ctypes.c_uint64(proj_seed), ctypes.byref(ps),
+            _dev(page_table, "page_table"), page_table.shape[2], _dev(lens, "lens"),
+            _dev(boundaries, "boundaries") if boundaries is not None else null,
+            _dev(cumvar, "cumvar") if cumvar is not None else null,
+            _dev(workspace, "workspace"), workspace.numel())
+    if representative == "mean":
+        st = _lib.load().skv_coarsen(*args, ctypes.c_void_p(_stream_handle(stream)))
+        _lib.check(st, "skv_coarsen")
+    else:
+        opts = _lib.SkvCoarsenOptions(reps[representative])
+        st = _lib.load().skv_coarsen_ex(*args, ctypes.byref(opts), ctypes.c_void_p(_stream_handle(stream)))
+        _lib.check(st, "skv_coarsen_ex")
     return lens
 
 

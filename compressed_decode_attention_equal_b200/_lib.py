@@ -23,6 +23,13 @@ class SkvNodePool(ctypes.Structure):
     _fields_ = [("pages", ctypes.c_void_p), ("num_pages", ctypes.c_int64)]
 
 
+SKV_REP_MEAN, SKV_REP_VARIATION_WEIGHTED = 0, 1
+
+
+class SkvCoarsenOptions(ctypes.Structure):
+    _fields_ = [("representative", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
+
+
 class SkvError(RuntimeError):
     def __init__(self, status: int, what: str):
         self.status = status
@@ -32,7 +39,7 @@ class SkvError(RuntimeError):
 # The header declares every symbol below; tests check that the library exports all of them.
 EXPORTS = ("skv_status_string", "skv_abi_version", "skv_page_bytes", "skv_projection_matrix",
            "skv_coarsen_workspace_bytes",
-           "skv_coarsen", "skv_decode_workspace_bytes", "skv_decode_attn", "skv_decode_attn_noalloc",
+           "skv_coarsen", "skv_coarsen_ex", "skv_decode_workspace_bytes", "skv_decode_attn", "skv_decode_attn_noalloc",
            "skv_workspace_error")
 
 _lib = None
@@ -62,6 +69,10 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.skv_coarsen.argtypes = [vp, vp, i32, i32, i32, i32, pi32, i32, i32, pi32, u64,
                                 ctypes.POINTER(SkvNodePool), vp, i32, vp, vp, vp, vp, sz, vp]
     lib.skv_coarsen.restype = i32
+    lib.skv_coarsen_ex.argtypes = [vp, vp, i32, i32, i32, i32, pi32, i32, i32, pi32, u64,
+                                   ctypes.POINTER(SkvNodePool), vp, i32, vp, vp, vp, vp, sz,
+                                   ctypes.POINTER(SkvCoarsenOptions), vp]
+    lib.skv_coarsen_ex.restype = i32
     lib.skv_decode_workspace_bytes.argtypes = [i32, i32, i32, i32, i32, i32]
     lib.skv_decode_workspace_bytes.restype = sz
     lib.skv_decode_attn.argtypes = [vp, i32, i32, i32, i32, i32, i32, ctypes.POINTER(SkvNodePool), vp, i32,

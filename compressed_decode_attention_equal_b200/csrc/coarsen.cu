@@ -409,7 +409,9 @@ struct Vec16<float> {
 
 constexpr int kK3Warps = 8;
 
-template <int D, typename T>
+// W: the variation-weighted representative is compiled in (a separate instantiation, so the
+// plain-mean kernel keeps its register budget).
+template <int D, typename T, bool W>
 __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenArgs a) {
     constexpr int ELEM = sizeof(T);
     constexpr int ROWB = D * ELEM;        // bytes of one key row
@@ -433,44 +435,83 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
     const uint8_t *kp = static_cast<const uint8_t *>(a.k) + row0 * ROWB + ch * 16;
     const uint8_t *vp = static_cast<const uint8_t *>(a.v) + row0 * ROWB + ch * 16;
 
+    // A middle segment with the variation-weighted representative ("Equal-Variation KV Cache",
+    // "Implementation notes") also accumulates sum_r d_r k_r, sum_r d_r v_r and sum_r d_r with
+    // d_r = D_r 2^-20, D_r recovered from the tile-local scan of the projection kernel.
+    const int t_mid = start - sr.s_eff;   // middle index of the first member
+    const bool weighted = W && m > 1 && t_mid >= 0 && t_mid < sr.M;
+    const int64_t *ls = a.local_scan + sr.mid_off + static_cast<int64_t>(h) * sr.M;
+
     // loads are issued kUnroll token steps at a time (2 x kUnroll 16-byte loads in flight per lane)
-    constexpr int kUnroll = 8;
-    float sk[EPL], sv[EPL], x[EPL];
+    constexpr int kUnroll = W ? 4 : 8;
+    float sk[EPL], sv[EPL], wk[EPL], wv[EPL], x[EPL], wsum = 0.0f;
 #pragma unroll
-    for (int i = 0; i < EPL; ++i) sk[i] = sv[i] = 0.0f;
+    for (int i = 0; i < EPL; ++i) sk[i] = sv[i] = wk[i] = wv[i] = 0.0f;
     for (int t0 = sub; t0 < m; t0 += TPS * kUnroll) {
         uint4 kw[kUnroll], vw[kUnroll];
+        long long lc[kUnroll], lp[kUnroll];
 #pragma unroll
         for (int r = 0; r < kUnroll; ++r) {
             const int t = t0 + r * TPS;
             kw[r] = vw[r] = make_uint4(0u, 0u, 0u, 0u);   // zero bits: +0.0 in both dtypes
+            lc[r] = lp[r] = 0;
             if (t < m) {
                 kw[r] = __ldg(reinterpret_cast<const uint4 *>(kp + static_cast<int64_t>(t) * ROWB));
                 vw[r] = __ldg(reinterpret_cast<const uint4 *>(vp + static_cast<int64_t>(t) * ROWB));
+                if (W && weighted) {   // D of middle token tm: its tile-local inclusive scan minus the previous
+                    const int tm = t_mid + t;
+                    lc[r] = __ldg(reinterpret_cast<const long long *>(ls + tm));
+                    if (tm % kTileOut != 0) lp[r] = __ldg(reinterpret_cast<const long long *>(ls + tm - 1));
+                }
             }
         }
 #pragma unroll
         for (int r = 0; r < kUnroll; ++r) {
+            const float w = W && weighted ? __ll2float_rn(lc[r] - lp[r]) * 0x1p-20f : 0.0f;
+            if (W) wsum += w;
             Vec16<T>::cvt(kw[r], x);
 #pragma unroll
-            for (int i = 0; i < EPL; ++i) sk[i] += x[i];
+            for (int i = 0; i < EPL; ++i) {
+                sk[i] += x[i];
+                if (W) wk[i] = __fmaf_rn(w, x[i], wk[i]);
+            }
             Vec16<T>::cvt(vw[r], x);
 #pragma unroll
-            for (int i = 0; i < EPL; ++i) sv[i] += x[i];
+            for (int i = 0; i < EPL; ++i) {
+                sv[i] += x[i];
+                if (W) wv[i] = __fmaf_rn(w, x[i], wv[i]);
+            }
         }
     }
 #pragma unroll
-    for (int off = CH; off < 32; off <<= 1)
+    for (int off = CH; off < 32; off <<= 1) {
 #pragma unroll
         for (int i = 0; i < EPL; ++i) {
             sk[i] += __shfl_xor_sync(0xffffffffu, sk[i], off);
             sv[i] += __shfl_xor_sync(0xffffffffu, sv[i], off);
         }
+        if (W && weighted) {
+#pragma unroll
+            for (int i = 0; i < EPL; ++i) {
+                wk[i] += __shfl_xor_sync(0xffffffffu, wk[i], off);
+                wv[i] += __shfl_xor_sync(0xffffffffu, wv[i], off);
+            }
+            wsum += __shfl_xor_sync(0xffffffffu, wsum, off);
+        }
+    }
     const float fm = static_cast<float>(m);
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         sk[i] = __fdiv_rn(sk[i], fm);   // mean key
         sv[i] = __fdiv_rn(sv[i], fm);   // mean value
+    }
+    // the stored key and value: the mean, or the weighted average when the segment has variation
+    float rk[EPL], rv[EPL];
+    const bool use_w = W && weighted && wsum > 0.0f;
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) {
+        rk[i] = use_w ? __fdiv_rn(wk[i], wsum) : sk[i];
+        rv[i] = use_w ? __fdiv_rn(wv[i], wsum) : sv[i];
     }
     // second pass over the keys (just read: served from L1 / L2)
     float q2[EPL];
@@ -517,8 +558,8 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
     uint8_t *pg = a.pages + static_cast<int64_t>(page) * (2 * VEC_BYTES + kPageNodes * 8);
     if (sub == 0) {
         const int off = slot * ROWB + swz(ch, slot) * 16;
-        Vec16<T>::store(pg + off, sk);
-        Vec16<T>::store(pg + VEC_BYTES + off, sv);
+        Vec16<T>::store(pg + off, rk);
+        Vec16<T>::store(pg + VEC_BYTES + off, rv);
     }
     if (lane == 0) {
         const float alpha = m == 1 ? 0.0f : logf(fm);
@@ -551,8 +592,11 @@ static cudaError_t launch_typed(const CoarsenArgs &a, const SeqTable &table, con
         k_boundaries<<<dim3(a.max_tiles, units), kTileRows, 0, s>>>(a);
     }
     k_plan_entries<<<units, 512, 0, s>>>(a);
-    if (a.max_emax > 0)
-        k_segment_reduce<D, T><<<dim3((a.max_emax + kK3Warps - 1) / kK3Warps, units), kK3Warps * 32, 0, s>>>(a);
+    if (a.max_emax > 0) {
+        const dim3 g3((a.max_emax + kK3Warps - 1) / kK3Warps, units);
+        if (a.representative == SKV_REP_VARIATION_WEIGHTED) k_segment_reduce<D, T, true><<<g3, kK3Warps * 32, 0, s>>>(a);
+        else k_segment_reduce<D, T, false><<<g3, kK3Warps * 32, 0, s>>>(a);
+    }
     return cudaGetLastError();
 }
 

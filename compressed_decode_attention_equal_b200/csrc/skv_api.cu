@@ -232,7 +232,7 @@ const char *skv_status_string(int status) {
     }
 }
 
-int skv_abi_version(void) { return 200; }
+int skv_abi_version(void) { return 201; }
 
 size_t skv_page_bytes(skv_dtype dtype, int d) {
     if ((dtype != SKV_BF16 && dtype != SKV_F32) || (d != 64 && d != 128)) return 0;
@@ -253,10 +253,19 @@ size_t skv_coarsen_workspace_bytes(int B, int Hkv, int d, const int32_t *T_host,
     return p.lay.total;
 }
 
-skv_status skv_coarsen(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d, const int32_t *T_host,
-                       int n_sink, int n_recent, const int32_t *N_host, uint64_t proj_seed,
-                       const skv_node_pool *pool, const int32_t *page_table, int max_pages, int32_t *lens,
-                       int32_t *boundaries, int64_t *cumvar, void *workspace, size_t ws_bytes, void *stream) {
+skv_status skv_coarsen_ex(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d,
+                          const int32_t *T_host, int n_sink, int n_recent, const int32_t *N_host, uint64_t proj_seed,
+                          const skv_node_pool *pool, const int32_t *page_table, int max_pages, int32_t *lens,
+                          int32_t *boundaries, int64_t *cumvar, void *workspace, size_t ws_bytes,
+                          const skv_coarsen_options *options, void *stream) {
+    int representative = SKV_REP_MEAN;
+    if (options) {
+        if (options->representative != SKV_REP_MEAN && options->representative != SKV_REP_VARIATION_WEIGHTED)
+            return SKV_ERR_INVALID_ARG;
+        for (int i = 0; i < 7; ++i)
+            if (options->reserved[i] != 0) return SKV_ERR_INVALID_ARG;
+        representative = options->representative;
+    }
     if (dtype != SKV_BF16 && dtype != SKV_F32) return SKV_ERR_UNSUPPORTED;
     static SeqTable table;   // host staging; guarded by the mutex below
     static std::mutex table_mu;
@@ -306,8 +315,17 @@ skv_status skv_coarsen(const void *k, const void *v, skv_dtype dtype, int B, int
     a.lens = lens;
     a.user_bounds = boundaries;
     a.cumvar = cumvar;
+    a.representative = representative;
     const cudaError_t e = launch_coarsen(a, table, proj, map_k, map_v, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SKV_OK : SKV_ERR_CUDA;
+}
+
+skv_status skv_coarsen(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d, const int32_t *T_host,
+                       int n_sink, int n_recent, const int32_t *N_host, uint64_t proj_seed,
+                       const skv_node_pool *pool, const int32_t *page_table, int max_pages, int32_t *lens,
+                       int32_t *boundaries, int64_t *cumvar, void *workspace, size_t ws_bytes, void *stream) {
+    return skv_coarsen_ex(k, v, dtype, B, Hkv, d, T_host, n_sink, n_recent, N_host, proj_seed, pool, page_table,
+                          max_pages, lens, boundaries, cumvar, workspace, ws_bytes, nullptr, stream);
 }
 
 size_t skv_decode_workspace_bytes(int B, int R, int Hq, int Hkv, int d, int max_pages) {

@@ -57,6 +57,7 @@ struct CoarsenArgs {
     int32_t *lens;
     int32_t *user_bounds;
     int64_t *cumvar;
+    int representative;  // skv_representative of the middle segments' stored key and value
 };
 
 // Workspace carve-up (offsets in bytes from the workspace start).

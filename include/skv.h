@@ -162,6 +162,44 @@ skv_status skv_coarsen(const void *k, const void *v, skv_dtype dtype, int B, int
                        int max_pages, int32_t *lens, int32_t *boundaries, int64_t *cumvar,
                        void *workspace, size_t ws_bytes, void *stream);
 
+/*
+ * Options of skv_coarsen_ex.
+ *
+ * representative: the key and value a middle segment stores.
+ *   SKV_REP_MEAN (0): the plain member mean ("SPICY-KV" demo page, Claim 2),
+ *     what skv_coarsen stores.
+ *   SKV_REP_VARIATION_WEIGHTED (1): the variation-weighted average of
+ *     "Equal-Variation KV Cache", "Implementation notes":
+ *     k_j = sum_{r in S_j} d_r k_r / sum_{r in S_j} d_r, and the same for v,
+ *     with d_r the variation step into token r taken as the fixed-point step
+ *     D_r * 2^-20 (so both the weights and which segments have none are exact;
+ *     D_0 = 0 for the first middle token). A segment whose steps are all zero
+ *     stores the plain mean. Exact tokens (sinks, recents) are unchanged.
+ *   In both cases sigma^2 (and beta) is the members' population key variance
+ *   about their plain mean (Claim 3 defines it on the members), m and alpha are
+ *   unchanged, and the boundaries do not depend on the option.
+ * reserved: must be zero.
+ */
+typedef enum { SKV_REP_MEAN = 0, SKV_REP_VARIATION_WEIGHTED = 1 } skv_representative;
+
+typedef struct {
+    int32_t representative; /* skv_representative */
+    int32_t reserved[7];
+} skv_coarsen_options;
+
+/*
+ * skv_coarsen with options (NULL = defaults, identical to skv_coarsen). Same
+ * arguments, layouts, ownership and errors as skv_coarsen; additionally
+ * SKV_ERR_INVALID_ARG for an unknown representative or a nonzero reserved
+ * field.
+ */
+skv_status skv_coarsen_ex(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d,
+                          const int32_t *T_host, int n_sink, int n_recent, const int32_t *N_host,
+                          uint64_t proj_seed, const skv_node_pool *pool, const int32_t *page_table,
+                          int max_pages, int32_t *lens, int32_t *boundaries, int64_t *cumvar,
+                          void *workspace, size_t ws_bytes, const skv_coarsen_options *options,
+                          void *stream);
+
 /* Bytes of device workspace skv_decode_attn needs (0 on invalid arguments). */
 size_t skv_decode_workspace_bytes(int B, int R, int Hq, int Hkv, int d, int max_pages);
 

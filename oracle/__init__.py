@@ -76,6 +76,9 @@ def _load():
         lib.orc_split.argtypes = [ctypes.c_int] * 3 + [P(ctypes.c_int)] * 3
         lib.orc_coarsen_unit.argtypes = ([P(f32), P(f32)] + [ctypes.c_int] * 5 + [P(f32), P(i64), P(i64), P(f64),
                                          P(i32), P(i32), P(i32), P(f64), P(f64), P(f64), P(f64), P(f64), P(i32)])
+        lib.orc_coarsen_unit2.argtypes = ([P(f32), P(f32)] + [ctypes.c_int] * 5 + [P(f32), ctypes.c_int, P(i64),
+                                          P(i64), P(f64), P(i32), P(i32), P(i32), P(f64), P(f64), P(f64), P(f64),
+                                          P(f64), P(i32)])
         lib.orc_decode_rows.argtypes = [P(f64), ctypes.c_int, ctypes.c_int, P(f64), P(f64), P(f64), P(f64),
                                         ctypes.c_int, P(f64), P(f64)]
         _lib = lib
@@ -170,9 +173,16 @@ class UnitNodes:
     M: int
 
 
+REPRESENTATIVES = {"mean": 0, "variation": 1}
+
+
 def coarsen_unit(k: np.ndarray, v: np.ndarray, n_sink: int, n_recent: int, N: int,
-                 P: np.ndarray) -> UnitNodes:
-    """Coarsen one unit: k, v [T, d] (any float dtype holding fp32-representable values)."""
+                 P: np.ndarray, representative: str = "mean") -> UnitNodes:
+    """Coarsen one unit: k, v [T, d] (any float dtype holding fp32-representable values).
+    representative: "mean" (plain member mean, SPICY-KV Claim 2) or "variation" (the
+    variation-weighted average of the Equal-Variation page's implementation notes, weights D_r;
+    a segment without variation keeps the plain mean)."""
+    rep = REPRESENTATIVES[representative]
     k = np.ascontiguousarray(k, np.float32)
     v = np.ascontiguousarray(v, np.float32)
     P = np.ascontiguousarray(P, np.float32)
@@ -195,10 +205,10 @@ def coarsen_unit(k: np.ndarray, v: np.ndarray, n_sink: int, n_recent: int, N: in
     kk = k if T > 0 else np.zeros((1, d), np.float32)
     vv = v if T > 0 else np.zeros((1, d), np.float32)
     f32p, i64p, i32p, f64p = (ctypes.c_float, ctypes.c_int64, ctypes.c_int32, ctypes.c_double)
-    rc = _load().orc_coarsen_unit(_ptr(kk, f32p), _ptr(vv, f32p), T, d, n_sink, n_recent, N, _ptr(P, f32p),
-                                  _ptr(D, i64p), _ptr(C, i64p), _ptr(d64, f64p), _ptr(b, i32p), _ptr(st, i32p),
-                                  _ptr(ln, i32p), _ptr(kt, f64p), _ptr(vt, f64p), _ptr(s2, f64p), _ptr(al, f64p),
-                                  _ptr(be, f64p), _ptr(E, i32p))
+    rc = _load().orc_coarsen_unit2(_ptr(kk, f32p), _ptr(vv, f32p), T, d, n_sink, n_recent, N, _ptr(P, f32p), rep,
+                                   _ptr(D, i64p), _ptr(C, i64p), _ptr(d64, f64p), _ptr(b, i32p), _ptr(st, i32p),
+                                   _ptr(ln, i32p), _ptr(kt, f64p), _ptr(vt, f64p), _ptr(s2, f64p), _ptr(al, f64p),
+                                   _ptr(be, f64p), _ptr(E, i32p))
     _check(rc, "coarsen_unit")
     e = int(E[0])
     return UnitNodes(D[:M].copy(), C[:M].copy(), d64[:M].copy(), b, st[:e].copy(), ln[:e].copy(),
@@ -209,7 +219,8 @@ def _pool(threads: int | None):
     return ThreadPoolExecutor(max_workers=threads or os.cpu_count() or 1)
 
 
-def coarsen(seqs, n_sink: int, n_recent: int, N_list, seed: int, threads: int | None = None):
+def coarsen(seqs, n_sink: int, n_recent: int, N_list, seed: int, threads: int | None = None,
+            representative: str = "mean"):
     """Coarsen a batch. seqs: list over sequences b of (k_b, v_b) arrays [Hkv, T_b, d].
     Returns nested list [b][h] of UnitNodes. The projection P is drawn from ``seed``."""
     d = seqs[0][0].shape[-1]
@@ -217,7 +228,8 @@ def coarsen(seqs, n_sink: int, n_recent: int, N_list, seed: int, threads: int | 
     jobs = [(b, h) for b in range(len(seqs)) for h in range(seqs[b][0].shape[0])]
     res = {}
     with _pool(threads) as ex:
-        futs = {ex.submit(coarsen_unit, seqs[b][0][h], seqs[b][1][h], n_sink, n_recent, int(N_list[b]), P): (b, h)
+        futs = {ex.submit(coarsen_unit, seqs[b][0][h], seqs[b][1][h], n_sink, n_recent, int(N_list[b]), P,
+                          representative): (b, h)
                 for (b, h) in jobs}
         for f, key in futs.items():
             res[key] = f.result()

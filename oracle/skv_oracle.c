@@ -34,6 +34,12 @@
  *      boundary token starts the new segment; empty segments are dropped.
  *  R6  A node stores the plain member mean of keys and values, mass m, and
  *      the per-dimension population key variance averaged over dimensions.
+ *  R6b Option (orc_coarsen_unit2, rep = 1): a middle segment stores instead
+ *      the variation-weighted averages of [EV] "Implementation notes",
+ *      k = sum_r d_r k_r / sum_r d_r (same for v), with d_r the fixed-point
+ *      step D_r (the common 2^-20 scale cancels); a segment whose steps are
+ *      all zero keeps the plain mean. sigma^2, m and alpha stay as in R6
+ *      (the variance is about the plain mean of the members).
  *  R7  Decode logit s = q.k/sqrt(d) + ln m + |q|^2 sigma^2/(2d); lse is the
  *      natural-log partition; an empty entry list gives out = 0, lse = -inf.
  */
@@ -193,8 +199,11 @@ int orc_split(int T, int S, int W, int *S_eff, int *W_eff, int *M)
 
 /* Node statistics of tokens [start, start + m) ([SK] Claim 2: mass, mean key,
  * mean value; Claim 3: subgrid key variance; section 2: alpha = log m,
- * beta = sigma^2 / (2 d_k)). Two-pass population variance in fp64. */
-static void orc_node_stats(const float *k, const float *v, int d, int start, int m,
+ * beta = sigma^2 / (2 d_k)). Two-pass population variance in fp64.
+ * w (may be NULL): the members' variation steps D; when given and not all
+ * zero, the stored key and value are the D-weighted averages ([EV]
+ * "Implementation notes"), the variance still being about the plain mean. */
+static void orc_node_stats(const float *k, const float *v, int d, int start, int m, const int64_t *w,
                            double *kt, double *vt, double *sig2, double *alpha, double *beta)
 {
     for (int i = 0; i < d; ++i) {
@@ -218,6 +227,21 @@ static void orc_node_stats(const float *k, const float *v, int d, int start, int
     *sig2 = var_sum / d;
     *alpha = log((double)m);
     *beta = *sig2 / (2.0 * d);
+    if (w) {
+        double W = 0.0;
+        for (int r = 0; r < m; ++r) W += (double)w[r];
+        if (W > 0.0) {
+            for (int i = 0; i < d; ++i) {
+                double wk = 0.0, wv = 0.0;
+                for (int r = 0; r < m; ++r) {
+                    wk += (double)w[r] * (double)k[(long)(start + r) * d + i];
+                    wv += (double)w[r] * (double)v[(long)(start + r) * d + i];
+                }
+                kt[i] = wk / W;
+                vt[i] = wv / W;
+            }
+        }
+    }
 }
 
 /*
@@ -227,13 +251,14 @@ static void orc_node_stats(const float *k, const float *v, int d, int start, int
  * [S_eff+N+W_eff]. *E receives the number of entries (sinks, nonempty
  * segments in order, recents). d64 (may be NULL) is the fp64 variation.
  */
-int orc_coarsen_unit(const float *k, const float *v, int T, int d, int S, int W, int N,
-                     const float *P, int64_t *D, int64_t *C, double *d64, int32_t *b,
-                     int32_t *ent_start, int32_t *ent_len, double *kt, double *vt,
-                     double *sig2, double *alpha, double *beta, int32_t *E)
+int orc_coarsen_unit2(const float *k, const float *v, int T, int d, int S, int W, int N,
+                      const float *P, int rep, int64_t *D, int64_t *C, double *d64, int32_t *b,
+                      int32_t *ent_start, int32_t *ent_len, double *kt, double *vt,
+                      double *sig2, double *alpha, double *beta, int32_t *E)
 {
     int s_eff, w_eff, M;
     if (d <= 0 || N < 1 || !P || !b || !E) return ORC_ERR_ARG;
+    if (rep != 0 && (rep != 1 || !D)) return ORC_ERR_ARG;
     if (orc_split(T, S, W, &s_eff, &w_eff, &M) != ORC_OK) return ORC_ERR_ARG;
     if (M >= ORC_M_MAX) return ORC_ERR_OVERFLOW;
 
@@ -291,10 +316,24 @@ int orc_coarsen_unit(const float *k, const float *v, int T, int d, int S, int W,
     }
     for (int t = 0; t < w_eff; ++t, ++e) { ent_start[e] = s_eff + M + t; ent_len[e] = 1; }
     *E = e;
-    for (int i = 0; i < e; ++i)
-        orc_node_stats(k, v, d, ent_start[i], ent_len[i], kt + (long)i * d, vt + (long)i * d,
+    for (int i = 0; i < e; ++i) {
+        /* weights only for middle segments (exact tokens are their own representative) */
+        const int mid = ent_start[i] - s_eff;
+        const int64_t *w = (rep == 1 && mid >= 0 && mid < M) ? D + mid : NULL;
+        orc_node_stats(k, v, d, ent_start[i], ent_len[i], w, kt + (long)i * d, vt + (long)i * d,
                        sig2 + i, alpha + i, beta + i);
+    }
     return ORC_OK;
+}
+
+/* orc_coarsen_unit2 with the plain-mean representative (R6). */
+int orc_coarsen_unit(const float *k, const float *v, int T, int d, int S, int W, int N,
+                     const float *P, int64_t *D, int64_t *C, double *d64, int32_t *b,
+                     int32_t *ent_start, int32_t *ent_len, double *kt, double *vt,
+                     double *sig2, double *alpha, double *beta, int32_t *E)
+{
+    return orc_coarsen_unit2(k, v, T, d, S, W, N, P, 0, D, C, d64, b, ent_start, ent_len, kt, vt, sig2, alpha,
+                             beta, E);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -37,7 +37,7 @@ def test_status_strings(lib):
         s = lib.skv_status_string(code).decode()
         assert s.startswith("SKV_")
     assert "unknown" in lib.skv_status_string(12345).decode()
-    assert lib.skv_abi_version() == 200
+    assert lib.skv_abi_version() == 201
     assert lib.skv_page_bytes(1, 128) == 2 * 16 * 128 * 2 + 128
     assert lib.skv_page_bytes(0, 64) == 2 * 16 * 64 * 4 + 128
     assert lib.skv_page_bytes(1, 96) == 0
@@ -87,6 +87,25 @@ def test_bad_arguments_rejected_before_any_launch(lib):
                          ctypes.byref(pool2), ctypes.c_void_p(16), 3, ctypes.c_void_p(16), null, null,
                          ctypes.c_void_p(256), 1 << 30, null)
     assert st == _lib.SKV_ERR_INVALID_ARG
+
+
+def test_coarsen_options_validated_before_any_launch(lib):
+    from compressed_decode_attention_equal_b200 import _lib
+    null = ctypes.c_void_p(0)
+    T = (ctypes.c_int32 * 1)(100)
+    N = (ctypes.c_int32 * 1)(4)
+    pool2 = _lib.SkvNodePool(16, 1)
+    args = (ctypes.c_void_p(256), ctypes.c_void_p(256), 1, 1, 1, 128, T, 8, 48, N, 0, ctypes.byref(pool2),
+            ctypes.c_void_p(16), 4, ctypes.c_void_p(16), null, null, ctypes.c_void_p(256), 16)
+    bad_rep = _lib.SkvCoarsenOptions(2)
+    assert lib.skv_coarsen_ex(*args, ctypes.byref(bad_rep), null) == _lib.SKV_ERR_INVALID_ARG
+    bad_res = _lib.SkvCoarsenOptions(1)
+    bad_res.reserved[3] = 1
+    assert lib.skv_coarsen_ex(*args, ctypes.byref(bad_res), null) == _lib.SKV_ERR_INVALID_ARG
+    # valid options fall through to the same checks as skv_coarsen (here: workspace too small)
+    ok = _lib.SkvCoarsenOptions(_lib.SKV_REP_VARIATION_WEIGHTED)
+    assert lib.skv_coarsen_ex(*args, ctypes.byref(ok), null) == _lib.SKV_ERR_WORKSPACE
+    assert lib.skv_coarsen_ex(*args, None, null) == _lib.SKV_ERR_WORKSPACE
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

@@ -4,7 +4,8 @@ Bit-exact: the projection P, every unit's cumulative quantised variation c_t, th
 boundaries, the entry counts. Within tolerance: node statistics (mean key / value, alpha = ln m,
 beta = sigma^2 / (2d)). Sizes span several projection tiles (255 tokens each) with ragged tails,
 plus the degenerate cases: T <= n_sink + n_recent, empty middle, M < N (empty segments dropped),
-constant middle (c_T = 0), N = 1, one jump crossing many thresholds, d = 64 / 128, fp32 / bf16."""
+constant middle (c_T = 0), N = 1, one jump crossing many thresholds, d = 64 / 128, fp32 / bf16;
+every case also with the variation-weighted segment representative."""
 import numpy as np
 import pytest
 import torch
@@ -12,14 +13,14 @@ import torch
 import compressed_decode_attention_equal_b200 as skv
 import oracle
 import workloads
-from gpu_helpers import check_decode, check_nodes, gpu_units, pool_for_units, to_np32
+from gpu_helpers import check_decode, check_nodes, gpu_units, pool_for_units, to_np32, weighted_slack
 
 pytestmark = pytest.mark.gpu
 
 S, W = workloads.N_SINK, workloads.N_RECENT
 
 
-def run_coarsen(k, v, Hkv, T_list, N_list, seed, n_sink=S, n_recent=W, shuffle=True):
+def run_coarsen(k, v, Hkv, T_list, N_list, seed, n_sink=S, n_recent=W, shuffle=True, representative="mean"):
     B = len(T_list)
     d = k.shape[-1]
     ent = [skv.entries_bound(T, N, n_sink, n_recent) for T, N in zip(T_list, N_list)]
@@ -30,12 +31,12 @@ def run_coarsen(k, v, Hkv, T_list, N_list, seed, n_sink=S, n_recent=W, shuffle=T
     ws = torch.zeros(skv.coarsen_workspace_bytes(Hkv, d, T_list, N_list, n_sink, n_recent), dtype=torch.uint8,
                      device="cuda")
     lens = skv.coarsen(k, v, Hkv, T_list, N_list, n_sink, n_recent, seed, pool, table, boundaries=bnd, cumvar=cum,
-                       workspace=ws)
+                       workspace=ws, representative=representative)
     st, flags = skv.workspace_error(ws)
     return dict(pool=pool, table=table, lens=lens, bnd=bnd, cum=cum, status=st, flags=flags)
 
 
-def oracle_units(k, v, Hkv, T_list, N_list, seed, units=None, n_sink=S, n_recent=W):
+def oracle_units(k, v, Hkv, T_list, N_list, seed, units=None, n_sink=S, n_recent=W, representative="mean"):
     d = k.shape[-1]
     P = oracle.projection(seed, d)
     res = {}
@@ -45,11 +46,11 @@ def oracle_units(k, v, Hkv, T_list, N_list, seed, units=None, n_sink=S, n_recent
                 continue
             kk = to_np32(workloads.unit_rows(k, T_list, Hkv, b, h))
             vv = to_np32(workloads.unit_rows(v, T_list, Hkv, b, h))
-            res[(b, h)] = oracle.coarsen_unit(kk, vv, n_sink, n_recent, int(N_list[b]), P)
+            res[(b, h)] = oracle.coarsen_unit(kk, vv, n_sink, n_recent, int(N_list[b]), P, representative)
     return res
 
 
-def compare_units(r, orc, k, T_list, Hkv, N_list, dtype):
+def compare_units(r, orc, k, v, T_list, Hkv, N_list, dtype):
     d = k.shape[-1]
     for (b, h), u in orc.items():
         what = f"unit ({b},{h}) T={T_list[b]} N={N_list[b]}"
@@ -69,7 +70,9 @@ def compare_units(r, orc, k, T_list, Hkv, N_list, dtype):
         gu = G()
         gu.kt, gu.vt = kt.double().cpu().numpy(), vt.double().cpu().numpy()
         gu.alpha, gu.beta = al.double().cpu().numpy(), be.double().cpu().numpy()
-        check_nodes(gu, u, dtype, d, what)
+        kk = to_np32(workloads.unit_rows(k, T_list, Hkv, b, h))
+        vv = to_np32(workloads.unit_rows(v, T_list, Hkv, b, h))
+        check_nodes(gu, u, dtype, d, what, slack=weighted_slack(u, kk, vv))
 
 
 def test_projection_matches_oracle_bitwise():
@@ -95,16 +98,36 @@ CASES = [
 ]
 
 
+@pytest.mark.parametrize("representative", ["mean", "variation"])
 @pytest.mark.parametrize("name,dtype,d,Hkv,T_list,N_list,values", CASES, ids=[c[0] for c in CASES])
-def test_coarsen_matches_oracle(name, dtype, d, Hkv, T_list, N_list, values):
+def test_coarsen_matches_oracle(name, dtype, d, Hkv, T_list, N_list, values, representative):
     seed = sum(T_list) + d
     w = workloads.Workload(name, seed, B=len(T_list), Hq=Hkv, Hkv=Hkv, d=d, R=1,
                            dtype="bf16" if dtype == torch.bfloat16 else "f32", T=0, regimes=12)
     k, v, _ = workloads.make_kv(w, "cuda", T_list=T_list, values=values)
-    r = run_coarsen(k, v, Hkv, T_list, N_list, seed)
+    r = run_coarsen(k, v, Hkv, T_list, N_list, seed, representative=representative)
     assert r["status"] == 0, f"device flags {r['flags']}"
-    orc = oracle_units(k, v, Hkv, T_list, N_list, seed)
-    compare_units(r, orc, k, T_list, Hkv, N_list, dtype)
+    orc = oracle_units(k, v, Hkv, T_list, N_list, seed, representative=representative)
+    compare_units(r, orc, k, v, T_list, Hkv, N_list, dtype)
+
+
+def test_weighted_representative_on_flat_and_jump_segments():
+    """Piecewise-constant keys and values with jumps: a segment's steps sit on its jump tokens, so
+    the weighted key differs from the plain mean, and segments inside a flat run (no steps) keep
+    the plain mean; both against the oracle."""
+    T, d = 1500, 128
+    g = torch.Generator(device="cuda").manual_seed(5)
+    levels = torch.randn(12, 2, d, device="cuda", generator=g)
+    idx = torch.div(torch.arange(T, device="cuda") * 12, T, rounding_mode="floor")
+    k = (levels[idx, 0] + 0.02 * torch.randn(T, d, device="cuda", generator=g)).bfloat16()
+    v = levels[idx, 1].bfloat16()
+    k[600:900] = k[600]
+    r = run_coarsen(k, v, 1, [T], [40], seed=7, representative="variation")
+    assert r["status"] == 0
+    orc = oracle_units(k, v, 1, [T], [40], seed=7, representative="variation")
+    plain = oracle_units(k, v, 1, [T], [40], seed=7)
+    assert np.abs(orc[(0, 0)].kt - plain[(0, 0)].kt).max() > 1e-2
+    compare_units(r, orc, k, v, [T], 1, [40], torch.bfloat16)
 
 
 def test_constant_middle_gives_one_node():
@@ -116,7 +139,7 @@ def test_constant_middle_gives_one_node():
     r = run_coarsen(k, v, Hkv, [T], [16], seed=1)
     assert int(r["lens"][0, 0]) == S + 1 + W
     orc = oracle_units(k, v, Hkv, [T], [16], seed=1)
-    compare_units(r, orc, k, [T], Hkv, [16], torch.bfloat16)
+    compare_units(r, orc, k, v, [T], Hkv, [16], torch.bfloat16)
 
 
 def test_jump_crosses_many_thresholds():
@@ -129,7 +152,7 @@ def test_jump_crosses_many_thresholds():
     r = run_coarsen(k, v, 1, [T], [30], seed=2)
     orc = oracle_units(k, v, 1, [T], [30], seed=2)
     assert orc[(0, 0)].kt.shape[0] < S + 30 + W
-    compare_units(r, orc, k, [T], 1, [30], torch.bfloat16)
+    compare_units(r, orc, k, v, [T], 1, [30], torch.bfloat16)
 
 
 def test_overflow_is_flagged():
@@ -150,7 +173,7 @@ def test_tiny_f32_end_to_end():
     r = run_coarsen(k, v, w.Hkv, T_list, N_list, w.seed)
     assert r["status"] == 0
     orc = oracle_units(k, v, w.Hkv, T_list, N_list, w.seed)
-    compare_units(r, orc, k, T_list, w.Hkv, N_list, torch.float32)
+    compare_units(r, orc, k, v, T_list, w.Hkv, N_list, torch.float32)
     q = workloads.make_queries(w, "cuda")
     out, lse = skv.decode_attn(q, w.Hkv, r["pool"], r["table"], r["lens"])
     units = [[orc[(0, 0)]]]
@@ -167,7 +190,7 @@ def test_gqa6_10k5_prefill_then_decode():
     r = run_coarsen(k, v, w.Hkv, T_list, N_list, w.seed)
     assert r["status"] == 0
     orc = oracle_units(k, v, w.Hkv, T_list, N_list, w.seed)
-    compare_units(r, orc, k, T_list, w.Hkv, N_list, torch.bfloat16)
+    compare_units(r, orc, k, v, T_list, w.Hkv, N_list, torch.bfloat16)
     q = workloads.make_queries(w, "cuda")
     out, lse = skv.decode_attn(q, w.Hkv, r["pool"], r["table"], r["lens"])
     ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), gpu_units(r["pool"], r["table"], r["lens"], 1, 2))

@@ -191,3 +191,31 @@ def test_decode_bad_page_in_first_pages_is_flagged():
     assert st == 0 and flags == 0
     ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), units)
     check_decode(out2, lse2, ref_out, ref_lse, torch.bfloat16, "after bad page")
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,R,d,E", [
+    (24, 28, 4, 1, 128, 700),   # 96 virtual units: clusters of 3 CTAs
+    (16, 28, 4, 1, 64, 1147),   # 64 units, d = 64: clusters of 4
+    (16, 16, 2, 2, 128, 500),   # 16 query rows per unit (two row tiles)
+    (8, 32, 4, 4, 64, 900),     # 32 query rows per unit (four row tiles), d = 64
+    (8, 16, 4, 5, 128, 333),    # 20 query rows
+    (4, 32, 4, 5, 128, 640),    # 40 query rows: two row passes per unit
+])
+def test_decode_equal_lengths_cluster_split(B, Hq, Hkv, R, d, E):
+    """Equal-length units in a full-width page table (the read-ahead and cluster-merge path when a
+    cluster size fits), across GQA group sizes, query-row counts and head dims."""
+    _run(B, Hq, Hkv, R, d, [E] * B, torch.bfloat16, seed=B * 100 + R * 10 + d // 64, shuffle=True)
+
+
+def test_decode_equal_lengths_wide_table_two_row_passes():
+    """Equal lengths, 40 query rows (two row passes), page table wider than the units."""
+    B, Hq, Hkv, R, d = 4, 32, 4, 5, 128
+    pool, table, lens, q = _synthetic(B, Hq, Hkv, R, d, [640] * B, torch.bfloat16, seed=31)
+    wide = _widen_table(table, 7, -1)
+    ws = torch.zeros(skv.decode_workspace_bytes(B, R, Hq, Hkv, d, wide.shape[2]), dtype=torch.uint8, device="cuda")
+    out, lse = skv.decode_attn(q, Hkv, pool, wide, lens, workspace=ws)
+    st, flags = skv.workspace_error(ws)
+    assert st == 0 and flags == 0, flags
+    units = gpu_units(pool, table, lens, B, Hkv)
+    ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), units)
+    check_decode(out, lse, ref_out, ref_lse, torch.bfloat16, "wide table, two row passes")

@@ -12,14 +12,14 @@ import torch
 import compressed_decode_attention_equal_b200 as skv
 import oracle
 import workloads
-from gpu_helpers import check_decode, check_nodes, gpu_units, to_np32
+from gpu_helpers import check_decode, check_nodes, gpu_units, to_np32, weighted_slack
 
 pytestmark = pytest.mark.gpu
 
 S, W = workloads.N_SINK, workloads.N_RECENT
 
 
-def _coarsen_full(w, values="normal"):
+def _coarsen_full(w, values="normal", representative="mean"):
     T_list = workloads.seq_lengths(w)
     N_list = workloads.segment_counts(w, T_list)
     k, v, _ = workloads.make_kv(w, "cuda", T_list=T_list, values=values)
@@ -35,18 +35,18 @@ def _coarsen_full(w, values="normal"):
     ws = torch.zeros(skv.coarsen_workspace_bytes(w.Hkv, w.d, T_list, N_list, S, W), dtype=torch.uint8,
                      device="cuda")
     lens = skv.coarsen(k, v, w.Hkv, T_list, N_list, S, W, w.seed, pool, table, boundaries=bnd, cumvar=cum,
-                       workspace=ws)
+                       workspace=ws, representative=representative)
     st, flags = skv.workspace_error(ws)
     assert st == 0, flags
     return dict(k=k, v=v, T=T_list, N=N_list, pool=pool, table=table, lens=lens, bnd=bnd, cum=cum)
 
 
-def _check_units(w, r, units):
+def _check_units(w, r, units, representative="mean"):
     P = oracle.projection(w.seed, w.d)
     for (b, h) in units:
         kk = to_np32(workloads.unit_rows(r["k"], r["T"], w.Hkv, b, h))
         vv = to_np32(workloads.unit_rows(r["v"], r["T"], w.Hkv, b, h))
-        u = oracle.coarsen_unit(kk, vv, S, W, r["N"][b], P)
+        u = oracle.coarsen_unit(kk, vv, S, W, r["N"][b], P, representative)
         what = f"{w.name} unit ({b},{h}) T={r['T'][b]}"
         off = sum(r["T"][:b]) * w.Hkv + h * r["T"][b]
         assert np.array_equal(r["cum"][off:off + u.M].cpu().numpy(), u.C), f"{what}: c_t"
@@ -60,7 +60,7 @@ def _check_units(w, r, units):
         g = G()
         g.kt, g.vt = kt.double().cpu().numpy(), vt.double().cpu().numpy()
         g.alpha, g.beta = al.double().cpu().numpy(), be.double().cpu().numpy()
-        check_nodes(g, u, w.torch_dtype, w.d, what)
+        check_nodes(g, u, w.torch_dtype, w.d, what, slack=weighted_slack(u, kk, vv))
 
 
 def _check_decode(w, r, sample_b):
@@ -111,3 +111,11 @@ def test_coarsen_131k_full():
     w = workloads.WORKLOADS["coarsen_131k"]
     r = _coarsen_full(w)
     _check_units(w, r, [(0, 0), (7, 3)])
+
+
+def test_gqa7_32k_3p5pct_variation_weighted_full():
+    """The 7B-shaped workload coarsened with the variation-weighted representative, then decoded."""
+    w = workloads.WORKLOADS["gqa7_32k_decode_3p5pct"]
+    r = _coarsen_full(w, representative="variation")
+    _check_units(w, r, [(3, 1), (30, 2)], representative="variation")
+    _check_decode(w, r, [3, 30])
