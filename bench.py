@@ -190,6 +190,51 @@ def _graph_steps(fn, steps: int, chunk: int):
     return g
 
 
+# ---------------------------------------------------------------------------
+# ranks (one process per GPU under torchrun; every rank takes the same collective steps)
+# ---------------------------------------------------------------------------
+def rank_workload(w, rank: int, world: int):
+    """The batch a rank decodes: the same shapes, an independent seed per rank (weak scaling;
+    no data-path collective)."""
+    if world <= 1:
+        return w
+    return dataclasses.replace(w, seed=w.seed + 100000 * rank)
+
+
+def max_over_ranks(x: float, device, world: int) -> float:
+    """The largest x over all ranks (the job's duration is set by its slowest rank)."""
+    if world <= 1:
+        return x
+    import torch
+    t = torch.tensor([x], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_step: int, world: int, steps: int, ms: float) -> float:
+    """Whole-job units per second: every rank's units over the max-over-ranks time."""
+    return units_per_step * world * steps / (ms / 1e3)
+
+
+def init_ranks(backend: str, device, world: int, timeout_s: int = 120):
+    """One process group per job (short timeout: ranks that wait on a dead peer end with an
+    error); NCCL binds the rank's device."""
+    if world <= 1:
+        return
+    import datetime
+    import torch
+    kw = {"device_id": device} if backend == "nccl" else {}
+    torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=timeout_s), **kw)
+
+
+def finish_ranks(world: int):
+    if world <= 1:
+        return
+    import torch
+    torch.distributed.barrier()
+    torch.distributed.destroy_process_group()
+
+
 def time_graphs(fn, steps: int, layers: int, dist_on: bool):
     """Device time (ms) of exactly `steps` calls fn(i), replayed from CUDA graphs."""
     import torch
@@ -336,8 +381,7 @@ def run_ours(args, rank: int, world: int, device):
 
     dist_on = world > 1
     w = workloads.WORKLOADS[WORKLOAD]
-    if dist_on:   # each rank decodes its own, independently seeded batch
-        w = dataclasses.replace(w, seed=w.seed + 100000 * rank)
+    w = rank_workload(w, rank, world)   # each rank decodes its own, independently seeded batch
     caches, table, T_list, N_list, coarsen_ms = build_layer_caches(w, args.layers, device)
     L = len(caches)
     rows_per_step = w.B * w.R * w.Hq
@@ -363,12 +407,9 @@ def run_ours(args, rank: int, world: int, device):
         sampler.start()
     ms = time_graphs(step, args.steps, L, dist_on)
     clocks = sampler.stop() if sampler else None
-    if dist_on:
-        t = torch.tensor([ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, device, world)
     ms_per_step = ms / args.steps
-    value = rows_per_step * world * args.steps / (ms / 1e3)
+    value = job_throughput(rows_per_step, world, args.steps, ms)
 
     # end to end: pinned host queries in, pinned host outputs back, every step
     q_host = [c["q"].cpu().pin_memory() for c in caches]
@@ -388,10 +429,7 @@ def run_ours(args, rank: int, world: int, device):
         e2e_step(i)
     e2e_steps = max(L, min(args.steps, 20000))
     e2e_ms = time_graphs(e2e_step, e2e_steps, L, dist_on)
-    if dist_on:
-        t = torch.tensor([e2e_ms], device=device, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        e2e_ms = float(t.item())
+    e2e_ms = max_over_ranks(e2e_ms, device, world)
     # the timed copies are real: the last step's outputs match the device results
     torch.cuda.synchronize()
     assert torch.equal(out_host[(e2e_steps - 1) % L], outs[(e2e_steps - 1) % L].cpu())
@@ -417,7 +455,7 @@ def run_ours(args, rank: int, world: int, device):
                          if src == "measured" else "fallback 6.65 TB/s",
                          "frac_of_8tbs": achieved / 8000.0, "algorithmic_bytes_per_launch": alg_bytes,
                          "kernel": "k_decode_split (one launch per call), time per call"},
-            "e2e": {"value": rows_per_step * world * e2e_steps / (e2e_ms / 1e3), "unit": UNIT,
+            "e2e": {"value": job_throughput(rows_per_step, world, e2e_steps, e2e_ms), "unit": UNIT,
                     "h2d_bytes_per_step": q_host[0].numel() * q_host[0].element_size(),
                     "d2h_bytes_per_step": out_host[0].numel() * out_host[0].element_size() + lse_host[0].numel() * 4,
                     "steps": e2e_steps},
@@ -512,10 +550,7 @@ def main():
         raise SystemExit("bench.py needs a CUDA device")
     torch.cuda.set_device(local)
     device = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=device)
+    init_ranks("nccl", device, world)
     from compressed_decode_attention_equal_b200 import build
     build.build()
     res, caches, table, w = run_ours(args, rank, world, device)
@@ -525,9 +560,7 @@ def main():
         if not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(w, caches, table)
         print(json.dumps(res), flush=True)
-    if world > 1:
-        torch.distributed.barrier()
-        torch.distributed.destroy_process_group()
+    finish_ranks(world)
 
 
 if __name__ == "__main__":
