@@ -78,7 +78,9 @@ def _load():
                                          P(i32), P(i32), P(i32), P(f64), P(f64), P(f64), P(f64), P(f64), P(i32)])
         lib.orc_coarsen_unit2.argtypes = ([P(f32), P(f32)] + [ctypes.c_int] * 5 + [P(f32), ctypes.c_int, P(i64),
                                           P(i64), P(f64), P(i32), P(i32), P(i32), P(f64), P(f64), P(f64), P(f64),
-                                          P(f64), P(i32)])
+                                          P(f64), P(f64), P(i32)])
+        lib.orc_decode_rows2.argtypes = [P(f64), ctypes.c_int, ctypes.c_int, P(f64), P(f64), P(f64), P(f64),
+                                         P(f64), ctypes.c_int, P(f64), P(f64)]
         lib.orc_decode_rows.argtypes = [P(f64), ctypes.c_int, ctypes.c_int, P(f64), P(f64), P(f64), P(f64),
                                         ctypes.c_int, P(f64), P(f64)]
         _lib = lib
@@ -166,6 +168,7 @@ class UnitNodes:
     kt: np.ndarray         # [E, d] fp64 mean key
     vt: np.ndarray         # [E, d] fp64 mean value
     sigma2: np.ndarray     # [E] fp64 per-dimension key variance averaged over d
+    var: np.ndarray        # [E, d] fp64 per-dimension key variance (the diagonal closure's vector)
     alpha: np.ndarray      # [E] fp64 ln m
     beta: np.ndarray       # [E] fp64 sigma2 / (2 d)
     s_eff: int
@@ -199,6 +202,7 @@ def coarsen_unit(k: np.ndarray, v: np.ndarray, n_sink: int, n_recent: int, N: in
     kt = np.zeros((max(Emax, 1), d), np.float64)
     vt = np.zeros((max(Emax, 1), d), np.float64)
     s2 = np.zeros(max(Emax, 1), np.float64)
+    vv_ = np.zeros((max(Emax, 1), d), np.float64)
     al = np.zeros(max(Emax, 1), np.float64)
     be = np.zeros(max(Emax, 1), np.float64)
     E = np.zeros(1, np.int32)
@@ -207,12 +211,12 @@ def coarsen_unit(k: np.ndarray, v: np.ndarray, n_sink: int, n_recent: int, N: in
     f32p, i64p, i32p, f64p = (ctypes.c_float, ctypes.c_int64, ctypes.c_int32, ctypes.c_double)
     rc = _load().orc_coarsen_unit2(_ptr(kk, f32p), _ptr(vv, f32p), T, d, n_sink, n_recent, N, _ptr(P, f32p), rep,
                                    _ptr(D, i64p), _ptr(C, i64p), _ptr(d64, f64p), _ptr(b, i32p), _ptr(st, i32p),
-                                   _ptr(ln, i32p), _ptr(kt, f64p), _ptr(vt, f64p), _ptr(s2, f64p), _ptr(al, f64p),
-                                   _ptr(be, f64p), _ptr(E, i32p))
+                                   _ptr(ln, i32p), _ptr(kt, f64p), _ptr(vt, f64p), _ptr(vv_, f64p), _ptr(s2, f64p),
+                                   _ptr(al, f64p), _ptr(be, f64p), _ptr(E, i32p))
     _check(rc, "coarsen_unit")
     e = int(E[0])
     return UnitNodes(D[:M].copy(), C[:M].copy(), d64[:M].copy(), b, st[:e].copy(), ln[:e].copy(),
-                     kt[:e].copy(), vt[:e].copy(), s2[:e].copy(), al[:e].copy(), be[:e].copy(), s_eff, w_eff, M)
+                     kt[:e].copy(), vt[:e].copy(), s2[:e].copy(), vv_[:e].copy(), al[:e].copy(), be[:e].copy(), s_eff, w_eff, M)
 
 
 def _pool(threads: int | None):
@@ -239,8 +243,11 @@ def coarsen(seqs, n_sink: int, n_recent: int, N_list, seed: int, threads: int | 
 # --------------------------------------------------------------------------
 # decode
 # --------------------------------------------------------------------------
-def decode_rows(q: np.ndarray, kt: np.ndarray, vt: np.ndarray, alpha: np.ndarray, beta: np.ndarray):
+def decode_rows(q: np.ndarray, kt: np.ndarray, vt: np.ndarray, alpha: np.ndarray, beta: np.ndarray,
+                var: np.ndarray | None = None):
     """Compressed decode attention of query rows q [rows, d] against one unit's entries.
+    var [E, d] (optional): per-dimension key variances for the diagonal closure
+    sum_i q_i^2 var_i / (2d) in place of |q|^2 beta.
     Returns (out [rows, d] fp64, lse [rows] fp64, natural log)."""
     q = np.ascontiguousarray(q, np.float64)
     rows, d = q.shape
@@ -250,21 +257,26 @@ def decode_rows(q: np.ndarray, kt: np.ndarray, vt: np.ndarray, alpha: np.ndarray
         vt = np.ascontiguousarray(vt, np.float64)
         al = np.ascontiguousarray(alpha, np.float64)
         be = np.ascontiguousarray(beta, np.float64)
+        va = np.ascontiguousarray(var, np.float64) if var is not None else None
     else:
         kt, vt, al, be = np.zeros((1, d)), np.zeros((1, d)), np.zeros(1), np.zeros(1)
+        va = np.zeros((1, d)) if var is not None else None
     out = np.zeros((max(rows, 1), d), np.float64)
     lse = np.zeros(max(rows, 1), np.float64)
     qq = q if rows > 0 else np.zeros((1, d))
     f64p = ctypes.c_double
-    _check(_load().orc_decode_rows(_ptr(qq, f64p), rows, d, _ptr(kt, f64p), _ptr(vt, f64p), _ptr(al, f64p),
-                                   _ptr(be, f64p), E, _ptr(out, f64p), _ptr(lse, f64p)), "decode_rows")
+    vp = _ptr(va, f64p) if va is not None else None
+    _check(_load().orc_decode_rows2(_ptr(qq, f64p), rows, d, _ptr(kt, f64p), _ptr(vt, f64p), _ptr(al, f64p),
+                                    _ptr(be, f64p), vp, E, _ptr(out, f64p), _ptr(lse, f64p)), "decode_rows")
     return out[:rows], lse[:rows]
 
 
-def decode(q: np.ndarray, units, threads: int | None = None):
+def decode(q: np.ndarray, units, threads: int | None = None, closure: str = "scalar"):
     """Decode a batch. q [B, R, Hq, d]; units[b][h] supplies (kt, vt, alpha, beta) for KV head h
-    (a UnitNodes or any object with those attributes). Query head hq reads KV head hq // G.
-    Returns out [B, R, Hq, d] fp64 and lse [B, R, Hq] fp64."""
+    (a UnitNodes or any object with those attributes; `var` too for closure="diagonal"). Query head
+    hq reads KV head hq // G. Returns out [B, R, Hq, d] fp64 and lse [B, R, Hq] fp64."""
+    if closure not in ("scalar", "diagonal"):
+        raise ValueError("closure must be 'scalar' or 'diagonal'")
     B, R, Hq, d = q.shape
     Hkv = len(units[0])
     G = Hq // Hkv
@@ -274,7 +286,7 @@ def decode(q: np.ndarray, units, threads: int | None = None):
     def one(b, h):
         rows = q[b, :, h * G:(h + 1) * G, :].reshape(R * G, d)
         u = units[b][h]
-        o, l = decode_rows(rows, u.kt, u.vt, u.alpha, u.beta)
+        o, l = decode_rows(rows, u.kt, u.vt, u.alpha, u.beta, u.var if closure == "diagonal" else None)
         out[b, :, h * G:(h + 1) * G, :] = o.reshape(R, G, d)
         lse[b, :, h * G:(h + 1) * G] = l.reshape(R, G)
 

@@ -42,6 +42,12 @@
  *      (the variance is about the plain mean of the members).
  *  R7  Decode logit s = q.k/sqrt(d) + ln m + |q|^2 sigma^2/(2d); lse is the
  *      natural-log partition; an empty entry list gives out = 0, lse = -inf.
+ *  R7b Option (orc_decode_rows2 with var): the diagonal closure of [SK]
+ *      Claim 3 ("diagonal vector sigma_m^2"): the second cumulant of
+ *      q.eps/sqrt(d) for independent per-dimension deviations,
+ *      s = q.k/sqrt(d) + ln m + sum_i q_i^2 var_i / (2d), var_i the members'
+ *      population variance of key dimension i (orc_coarsen_unit2's var). With
+ *      var_i = sigma^2 for every i it is the scalar form of R7.
  */
 #include <math.h>
 #include <stdint.h>
@@ -204,7 +210,7 @@ int orc_split(int T, int S, int W, int *S_eff, int *W_eff, int *M)
  * zero, the stored key and value are the D-weighted averages ([EV]
  * "Implementation notes"), the variance still being about the plain mean. */
 static void orc_node_stats(const float *k, const float *v, int d, int start, int m, const int64_t *w,
-                           double *kt, double *vt, double *sig2, double *alpha, double *beta)
+                           double *kt, double *vt, double *var_vec, double *sig2, double *alpha, double *beta)
 {
     for (int i = 0; i < d; ++i) {
         double sk = 0.0, sv = 0.0;
@@ -223,6 +229,7 @@ static void orc_node_stats(const float *k, const float *v, int d, int start, int
             acc += dev * dev;
         }
         var_sum += acc / m;
+        if (var_vec) var_vec[i] = acc / m;
     }
     *sig2 = var_sum / d;
     *alpha = log((double)m);
@@ -253,7 +260,7 @@ static void orc_node_stats(const float *k, const float *v, int d, int start, int
  */
 int orc_coarsen_unit2(const float *k, const float *v, int T, int d, int S, int W, int N,
                       const float *P, int rep, int64_t *D, int64_t *C, double *d64, int32_t *b,
-                      int32_t *ent_start, int32_t *ent_len, double *kt, double *vt,
+                      int32_t *ent_start, int32_t *ent_len, double *kt, double *vt, double *var_vec,
                       double *sig2, double *alpha, double *beta, int32_t *E)
 {
     int s_eff, w_eff, M;
@@ -321,7 +328,7 @@ int orc_coarsen_unit2(const float *k, const float *v, int T, int d, int S, int W
         const int mid = ent_start[i] - s_eff;
         const int64_t *w = (rep == 1 && mid >= 0 && mid < M) ? D + mid : NULL;
         orc_node_stats(k, v, d, ent_start[i], ent_len[i], w, kt + (long)i * d, vt + (long)i * d,
-                       sig2 + i, alpha + i, beta + i);
+                       var_vec ? var_vec + (long)i * d : NULL, sig2 + i, alpha + i, beta + i);
     }
     return ORC_OK;
 }
@@ -332,8 +339,8 @@ int orc_coarsen_unit(const float *k, const float *v, int T, int d, int S, int W,
                      int32_t *ent_start, int32_t *ent_len, double *kt, double *vt,
                      double *sig2, double *alpha, double *beta, int32_t *E)
 {
-    return orc_coarsen_unit2(k, v, T, d, S, W, N, P, 0, D, C, d64, b, ent_start, ent_len, kt, vt, sig2, alpha,
-                             beta, E);
+    return orc_coarsen_unit2(k, v, T, d, S, W, N, P, 0, D, C, d64, b, ent_start, ent_len, kt, vt, NULL, sig2,
+                             alpha, beta, E);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -344,8 +351,9 @@ int orc_coarsen_unit(const float *k, const float *v, int T, int d, int S, int W,
 
 /* rows query rows q [rows][d] against E entries (kt, vt [E][d]; alpha, beta
  * [E]). out [rows][d], lse [rows]. fp64 throughout, max-shifted. */
-int orc_decode_rows(const double *q, int rows, int d, const double *kt, const double *vt,
-                    const double *alpha, const double *beta, int E, double *out, double *lse)
+int orc_decode_rows2(const double *q, int rows, int d, const double *kt, const double *vt,
+                     const double *alpha, const double *beta, const double *var, int E, double *out,
+                     double *lse)
 {
     if (rows < 0 || d <= 0 || E < 0) return ORC_ERR_ARG;
     double *s = (double *)malloc(sizeof(double) * (size_t)(E > 0 ? E : 1));
@@ -362,7 +370,13 @@ int orc_decode_rows(const double *q, int rows, int d, const double *kt, const do
         for (int j = 0; j < E; ++j) {
             double dot = 0.0;
             for (int i = 0; i < d; ++i) dot += qr[i] * kt[(long)j * d + i];
-            s[j] = dot * inv_sqrt_d + alpha[j] + qn2 * beta[j];
+            double closure = qn2 * beta[j];
+            if (var) {   /* R7b: sum_i q_i^2 var_i / (2d) */
+                double c = 0.0;
+                for (int i = 0; i < d; ++i) c += qr[i] * qr[i] * var[(long)j * d + i];
+                closure = c / (2.0 * d);
+            }
+            s[j] = dot * inv_sqrt_d + alpha[j] + closure;
             if (s[j] > mx) mx = s[j];
         }
         double Z = 0.0;
@@ -376,4 +390,11 @@ int orc_decode_rows(const double *q, int rows, int d, const double *kt, const do
     }
     free(s);
     return ORC_OK;
+}
+
+/* orc_decode_rows2 with the scalar closure (R7). */
+int orc_decode_rows(const double *q, int rows, int d, const double *kt, const double *vt,
+                    const double *alpha, const double *beta, int E, double *out, double *lse)
+{
+    return orc_decode_rows2(q, rows, d, kt, vt, alpha, beta, NULL, E, out, lse);
 }
