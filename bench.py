@@ -134,7 +134,7 @@ class ClockSampler:
 # ---------------------------------------------------------------------------
 # workload set-up (untimed)
 # ---------------------------------------------------------------------------
-def build_layer_caches(w, layers: int, device):
+def build_layer_caches(w, layers: int, device, closure: str = "scalar"):
     import torch
     import compressed_decode_attention_equal_b200 as skv
     import workloads
@@ -149,7 +149,7 @@ def build_layer_caches(w, layers: int, device):
     for layer in range(layers):
         wl = dataclasses.replace(w, seed=w.seed + 1000 * layer)
         k, v, _ = workloads.make_kv(wl, device, T_list=T_list)
-        pool = skv.NodePool(num_pages, w.d, w.torch_dtype, device=device)
+        pool = skv.NodePool(num_pages, w.d, w.torch_dtype, device=device, closure=closure)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record()
         lens = skv.coarsen(k, v, w.Hkv, T_list, N_list, workloads.N_SINK, workloads.N_RECENT, wl.seed, pool, table,
@@ -167,11 +167,11 @@ def build_layer_caches(w, layers: int, device):
     return caches, table, T_list, N_list, coarsen_ms
 
 
-def algorithmic_decode_bytes(w, lens_list):
-    """HBM bytes one decode call must move: every entry's key, value and (alpha, beta) once,
-    the queries once, the outputs and lse once."""
+def algorithmic_decode_bytes(w, lens_list, closure: str = "scalar"):
+    """HBM bytes one decode call must move: every entry's key, value and (alpha, beta) once (and its
+    per-dimension variances with the diagonal closure), the queries once, the outputs and lse once."""
     ent = sum(int(x) for x in lens_list)
-    node = 2 * w.d * 2 + 8
+    node = (3 if closure == "diagonal" else 2) * w.d * 2 + 8
     rows = w.B * w.R * w.Hq
     return ent * node + rows * w.d * 2 * 2 + rows * 4, ent
 
@@ -371,6 +371,40 @@ def cpu_baseline(w, caches, table, budget_s: float = 12.0):
                       f"{int(c['lens'].sum())} entries), fp64, nodes read back from the GPU"}
 
 
+def diagonal_closure_stage(w, device, layers: int, steps: int = 6000):
+    """Decode with the diagonal closure (per-dimension variances in every node) on the same workload:
+    layer caches coarsened into diagonal pools, graph replays, CUDA events (rank 0 only)."""
+    import torch
+    import compressed_decode_attention_equal_b200 as skv
+    caches, table, _, _, _ = build_layer_caches(w, layers, device, closure="diagonal")
+    L = len(caches)
+    alg, _ = algorithmic_decode_bytes(w, [int(caches[0]["lens"].sum())], closure="diagonal")
+    outs = [torch.empty_like(c["q"]) for c in caches]
+    lses = [torch.empty(w.B, w.R, w.Hq, dtype=torch.float32, device=device) for _ in caches]
+    ws = torch.zeros(skv.decode_workspace_bytes(w.B, w.R, w.Hq, w.Hkv, w.d, table.shape[2]), dtype=torch.uint8,
+                     device=device)
+
+    def step(i):
+        c = caches[i % L]
+        skv.decode_attn(c["q"], w.Hkv, c["pool"], table, c["lens"], out=outs[i % L], lse=lses[i % L], workspace=ws)
+
+    for i in range(3 * L):
+        step(i)
+    torch.cuda.synchronize()
+    st, flags = skv.workspace_error(ws)
+    if st != 0:
+        raise RuntimeError(f"diagonal-closure decode raised device flags {flags}")
+    ms = time_graphs(step, steps, L, False)
+    us = ms / steps * 1e3
+    peak, src = _peaks()
+    del caches
+    torch.cuda.empty_cache()
+    return {"us_per_call": us, "query_rows_per_s": w.B * w.R * w.Hq / (us * 1e-6),
+            "achieved_gbs": alg / (us * 1e-6) / 1e9, "frac": alg / (us * 1e-6) / 1e9 / peak,
+            "algorithmic_bytes_per_launch": alg,
+            "note": "same workload and call with diagonal-closure pools (per-dimension key variances)"}
+
+
 # ---------------------------------------------------------------------------
 # arms
 # ---------------------------------------------------------------------------
@@ -531,6 +565,7 @@ def main():
     ap.add_argument("--layers", type=int, default=6)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-coarsen", action="store_true")
+    ap.add_argument("--no-diagonal", action="store_true", help="skip the diagonal-closure decode timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -557,6 +592,8 @@ def main():
     if rank == 0:
         if not args.no_coarsen:
             res["coarsen"] = coarsen_stage(device)
+        if not args.no_diagonal:
+            res["diagonal_closure"] = diagonal_closure_stage(w, device, args.layers)
         if not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(w, caches, table)
         print(json.dumps(res), flush=True)

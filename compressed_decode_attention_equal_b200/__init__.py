@@ -66,22 +66,32 @@ def pages_for(T: int, N: int, n_sink: int, n_recent: int) -> int:
     return -(-entries_bound(T, N, n_sink, n_recent) // PAGE_NODES)
 
 
+CLOSURES = {"scalar": _lib.SKV_CLOSURE_SCALAR, "diagonal": _lib.SKV_CLOSURE_DIAGONAL}
+
+
 class NodePool:
     """Paged macro-node storage: one uint8 tensor `pages` [num_pages, page_bytes]; page p holds 16
     entries of one unit as [keys 16 x d | values 16 x d | {alpha, beta} 16 x 2 fp32] (alpha = ln m,
-    beta = sigma^2 / (2d)). `k`, `v`, `ab` are strided views of those blocks. Within the key and value
-    blocks, 16-byte chunk c of slot n is stored at chunk c ^ (n & 7)."""
+    beta = sigma^2 / (2d)), followed for closure="diagonal" by [per-dimension key variances 16 x d].
+    `k`, `v`, `ab` (and `var`) are strided views of those blocks. Within the vector blocks, 16-byte
+    chunk c of slot n is stored at chunk c ^ (n & 7). coarsen() and decode_attn() use the pool's
+    closure."""
 
-    def __init__(self, num_pages: int, d: int, dtype: torch.dtype, device="cuda"):
-        self.num_pages, self.d, self.dtype = int(num_pages), int(d), dtype
+    def __init__(self, num_pages: int, d: int, dtype: torch.dtype, device="cuda", closure: str = "scalar"):
+        if closure not in CLOSURES:
+            raise ValueError(f"closure must be one of {sorted(CLOSURES)}")
+        self.num_pages, self.d, self.dtype, self.closure = int(num_pages), int(d), dtype, closure
         elem = torch.tensor([], dtype=dtype).element_size()
         self.vec_bytes = PAGE_NODES * d * elem
-        self.page_bytes = 2 * self.vec_bytes + PAGE_NODES * 8
+        self.page_bytes = (3 if closure == "diagonal" else 2) * self.vec_bytes + PAGE_NODES * 8
         P = self.num_pages
         self.pages = torch.empty(P, self.page_bytes, dtype=torch.uint8, device=device)
-        self.k = self.pages[:, :self.vec_bytes].view(dtype).view(P, PAGE_NODES, d)
-        self.v = self.pages[:, self.vec_bytes:2 * self.vec_bytes].view(dtype).view(P, PAGE_NODES, d)
-        self.ab = self.pages[:, 2 * self.vec_bytes:].view(torch.float32).view(P, PAGE_NODES, 2)
+        vb = self.vec_bytes
+        self.k = self.pages[:, :vb].view(dtype).view(P, PAGE_NODES, d)
+        self.v = self.pages[:, vb:2 * vb].view(dtype).view(P, PAGE_NODES, d)
+        self.ab = self.pages[:, 2 * vb:2 * vb + PAGE_NODES * 8].view(torch.float32).view(P, PAGE_NODES, 2)
+        self.var = (self.pages[:, 2 * vb + PAGE_NODES * 8:].view(dtype).view(P, PAGE_NODES, d)
+                    if closure == "diagonal" else None)
 
     def struct(self) -> _lib.SkvNodePool:
         return _lib.SkvNodePool(self.pages.data_ptr(), self.num_pages)
@@ -139,11 +149,11 @@ def coarsen(k: torch.Tensor, v: torch.Tensor, Hkv: int, T_list, N_list, n_sink: 
             _dev(boundaries, "boundaries") if boundaries is not None else null,
             _dev(cumvar, "cumvar") if cumvar is not None else null,
             _dev(workspace, "workspace"), workspace.numel())
-    if representative == "mean":
+    if representative == "mean" and pool.closure == "scalar":
         st = _lib.load().skv_coarsen(*args, ctypes.c_void_p(_stream_handle(stream)))
         _lib.check(st, "skv_coarsen")
     else:
-        opts = _lib.SkvCoarsenOptions(reps[representative])
+        opts = _lib.SkvCoarsenOptions(reps[representative], CLOSURES[pool.closure])
         st = _lib.load().skv_coarsen_ex(*args, ctypes.byref(opts), ctypes.c_void_p(_stream_handle(stream)))
         _lib.check(st, "skv_coarsen_ex")
     return lens
@@ -173,11 +183,16 @@ def decode_attn(q: torch.Tensor, Hkv: int, pool: NodePool, page_table: torch.Ten
         workspace = torch.zeros(decode_workspace_bytes(B, R, Hq, Hkv, d, max_pages), dtype=torch.uint8,
                                 device=q.device)
     ps = pool.struct()
-    st = _lib.load().skv_decode_attn(
-        _dev(q, "q"), _code(q.dtype), B, R, Hq, Hkv, d, ctypes.byref(ps), _dev(page_table, "page_table"),
-        max_pages, _dev(lens, "lens"), _dev(out, "out"), _dev(lse, "lse"), _dev(workspace, "workspace"),
-        workspace.numel(), ctypes.c_void_p(_stream_handle(stream)))
-    _lib.check(st, "skv_decode_attn")
+    args = (_dev(q, "q"), _code(q.dtype), B, R, Hq, Hkv, d, ctypes.byref(ps), _dev(page_table, "page_table"),
+            max_pages, _dev(lens, "lens"), _dev(out, "out"), _dev(lse, "lse"), _dev(workspace, "workspace"),
+            workspace.numel())
+    if pool.closure == "scalar":
+        st = _lib.load().skv_decode_attn(*args, ctypes.c_void_p(_stream_handle(stream)))
+        _lib.check(st, "skv_decode_attn")
+    else:
+        opts = _lib.SkvDecodeOptions(CLOSURES[pool.closure])
+        st = _lib.load().skv_decode_attn_ex(*args, ctypes.byref(opts), ctypes.c_void_p(_stream_handle(stream)))
+        _lib.check(st, "skv_decode_attn_ex")
     return out, lse
 
 
@@ -189,8 +204,8 @@ def workspace_error(workspace: torch.Tensor, stream=None):
     return st, flags.value
 
 
-def page_bytes(dtype: torch.dtype, d: int) -> int:
-    return int(_lib.load().skv_page_bytes(_code(dtype), d))
+def page_bytes(dtype: torch.dtype, d: int, closure: str = "scalar") -> int:
+    return int(_lib.load().skv_page_bytes_ex(_code(dtype), d, CLOSURES[closure]))
 
 
 def _entry_rows(pool: NodePool, page_table: torch.Tensor, b: int, h: int, E: int):
@@ -200,6 +215,21 @@ def _entry_rows(pool: NodePool, page_table: torch.Tensor, b: int, h: int, E: int
     pg = pages[:, None].expand(n_pages, PAGE_NODES).reshape(-1)[:E]
     sl = slots[None, :].expand(n_pages, PAGE_NODES).reshape(-1)[:E]
     return pg, sl
+
+
+def read_variances(pool: NodePool, page_table: torch.Tensor, lens: torch.Tensor, b: int, h: int):
+    """Per-dimension key variances [E, d] of unit (b, h) in entry order (a diagonal pool)."""
+    if pool.var is None:
+        raise ValueError("the pool holds no per-dimension variances (closure='scalar')")
+    E = int(lens[b, h])
+    d = pool.d
+    if E == 0:
+        return pool.var.new_zeros(0, d)
+    pg, sl = _entry_rows(pool, page_table, b, h, E)
+    epc = 16 // pool.var.element_size()
+    ch = d // epc
+    phys = torch.arange(ch, device=pg.device)[None, :] ^ (sl[:, None] & 7)
+    return pool.var.view(pool.num_pages, PAGE_NODES, ch, epc)[pg[:, None], sl[:, None], phys].reshape(E, d)
 
 
 def read_entries(pool: NodePool, page_table: torch.Tensor, lens: torch.Tensor, b: int, h: int):

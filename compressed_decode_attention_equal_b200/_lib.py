@@ -24,10 +24,15 @@ class SkvNodePool(ctypes.Structure):
 
 
 SKV_REP_MEAN, SKV_REP_VARIATION_WEIGHTED = 0, 1
+SKV_CLOSURE_SCALAR, SKV_CLOSURE_DIAGONAL = 0, 1
 
 
 class SkvCoarsenOptions(ctypes.Structure):
-    _fields_ = [("representative", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
+    _fields_ = [("representative", ctypes.c_int32), ("closure", ctypes.c_int32), ("reserved", ctypes.c_int32 * 6)]
+
+
+class SkvDecodeOptions(ctypes.Structure):
+    _fields_ = [("closure", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7)]
 
 
 class SkvError(RuntimeError):
@@ -37,9 +42,9 @@ class SkvError(RuntimeError):
 
 
 # The header declares every symbol below; tests check that the library exports all of them.
-EXPORTS = ("skv_status_string", "skv_abi_version", "skv_page_bytes", "skv_projection_matrix",
+EXPORTS = ("skv_status_string", "skv_abi_version", "skv_page_bytes", "skv_page_bytes_ex", "skv_projection_matrix",
            "skv_coarsen_workspace_bytes",
-           "skv_coarsen", "skv_coarsen_ex", "skv_decode_workspace_bytes", "skv_decode_attn", "skv_decode_attn_noalloc",
+           "skv_coarsen", "skv_coarsen_ex", "skv_decode_workspace_bytes", "skv_decode_attn", "skv_decode_attn_ex", "skv_decode_attn_noalloc",
            "skv_workspace_error")
 
 _lib = None
@@ -62,6 +67,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.skv_abi_version.restype = i32
     lib.skv_page_bytes.argtypes = [i32, i32]
     lib.skv_page_bytes.restype = sz
+    lib.skv_page_bytes_ex.argtypes = [i32, i32, i32]
+    lib.skv_page_bytes_ex.restype = sz
     lib.skv_projection_matrix.argtypes = [u64, i32, ctypes.POINTER(ctypes.c_float)]
     lib.skv_projection_matrix.restype = i32
     lib.skv_coarsen_workspace_bytes.argtypes = [i32, i32, i32, pi32, pi32, i32, i32]
@@ -78,6 +85,9 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.skv_decode_attn.argtypes = [vp, i32, i32, i32, i32, i32, i32, ctypes.POINTER(SkvNodePool), vp, i32,
                                     vp, vp, vp, vp, sz, vp]
     lib.skv_decode_attn.restype = i32
+    lib.skv_decode_attn_ex.argtypes = [vp, i32, i32, i32, i32, i32, i32, ctypes.POINTER(SkvNodePool), vp, i32,
+                                       vp, vp, vp, vp, sz, ctypes.POINTER(SkvDecodeOptions), vp]
+    lib.skv_decode_attn_ex.restype = i32
     lib.skv_decode_attn_noalloc.argtypes = [vp, i32, i32, i32, i32, i32, i32, ctypes.POINTER(SkvNodePool), vp,
                                             i32, vp, vp, vp, vp]
     lib.skv_decode_attn_noalloc.restype = i32

@@ -536,13 +536,14 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
             }
         }
     }
-    float var_lane = 0.0f;
+    float var_lane = 0.0f, vd[EPL];
 #pragma unroll
     for (int i = 0; i < EPL; ++i) {
         float qi = q2[i];
 #pragma unroll
         for (int off = CH; off < 32; off <<= 1) qi += __shfl_xor_sync(0xffffffffu, qi, off);
-        var_lane += __fdiv_rn(qi, fm);   // population variance of dimension i
+        vd[i] = __fdiv_rn(qi, fm);   // population variance of dimension i
+        var_lane += vd[i];
     }
 #pragma unroll
     for (int off = 1; off < CH; off <<= 1) var_lane += __shfl_xor_sync(0xffffffffu, var_lane, off);
@@ -554,12 +555,14 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
         if (lane == 0) raise_flag(a.flags, FLAG_BAD_PAGE);
         return;
     }
-    constexpr int VEC_BYTES = kPageNodes * ROWB;   // keys (then values) of one page
-    uint8_t *pg = a.pages + static_cast<int64_t>(page) * (2 * VEC_BYTES + kPageNodes * 8);
+    constexpr int VEC_BYTES = kPageNodes * ROWB;   // keys (then values, then variances) of one page
+    const bool diag = a.closure == SKV_CLOSURE_DIAGONAL;
+    uint8_t *pg = a.pages + static_cast<int64_t>(page) * ((diag ? 3 : 2) * VEC_BYTES + kPageNodes * 8);
     if (sub == 0) {
         const int off = slot * ROWB + swz(ch, slot) * 16;
         Vec16<T>::store(pg + off, rk);
         Vec16<T>::store(pg + VEC_BYTES + off, rv);
+        if (diag) Vec16<T>::store(pg + 2 * VEC_BYTES + kPageNodes * 8 + off, vd);   // per-dimension variances
     }
     if (lane == 0) {
         const float alpha = m == 1 ? 0.0f : logf(fm);

@@ -48,26 +48,30 @@ constexpr int kDecStages = 8;
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-template <int D>
+// DIAG: the page also carries per-dimension key variances (the diagonal closure) after alpha/beta
+template <int D, bool DIAG = false>
 struct PageGeom {
     static constexpr int ROWB = D * 2;                    // bytes of one bf16 node vector
-    static constexpr int VEC_BYTES = kPageNodes * ROWB;   // K (or V) bytes of a page
+    static constexpr int VEC_BYTES = kPageNodes * ROWB;   // K (or V, or variance) bytes of a page
     static constexpr int AB_BYTES = kPageNodes * 8;
-    static constexpr int STAGE = 2 * VEC_BYTES + AB_BYTES;
+    static constexpr int VAR_OFF = 2 * VEC_BYTES + AB_BYTES;
+    static constexpr int STAGE = 2 * VEC_BYTES + AB_BYTES + (DIAG ? VEC_BYTES : 0);
 };
 
-template <int D, int NT>
+template <int D, int NT, bool DIAG = false>
 struct SplitSmem {
     static constexpr int QROWB = D * 2 + 16;              // padded query row: conflict-free ldmatrix
     static constexpr int QBUF = NT * 8 * QROWB;           // the query rows of one piece
-    static constexpr int STAGES_BYTES = kDecStages * PageGeom<D>::STAGE;
+    // ring depth: pages 1.5x larger with the variances, so a shallower ring keeps 3 CTAs per SM
+    static constexpr int STAGES = DIAG ? 4 : kDecStages;
+    static constexpr int STAGES_BYTES = STAGES * PageGeom<D, DIAG>::STAGE;
     static constexpr int MST = D + 4;                     // mbuf row stride: 16-byte rows
     static constexpr int MBUF_FLOATS = kDecConsumers * 8 * MST;
-    static constexpr int BARS = 2 * kDecStages + 4;
+    static constexpr int BARS = 2 * STAGES + 4;
     static constexpr int ROWS = NT * 8;                   // query rows of one piece
     static constexpr int WST = 9;                         // merge weights per row (<= 8) + log2 partition
     static constexpr int EPI_BYTES = ROWS * 8 + ROWS * WST * 4;
-    static constexpr size_t FIXED = 16 + STAGES_BYTES + 2 * QBUF + BARS * 8 + kDecStages * 4 + MBUF_FLOATS * 4 +
+    static constexpr size_t FIXED = 16 + STAGES_BYTES + 2 * QBUF + BARS * 8 + STAGES * 4 + MBUF_FLOATS * 4 +
                                     16 * 4 + ((EPI_BYTES + 15) / 16) * 16;
 };
 
@@ -265,24 +269,25 @@ __device__ void merge_unit(const DecodeArgs &a, int v, const int *codes, int n, 
     }
 }
 
-template <int D, int NT>
-__global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArgs a) {
-    using G = PageGeom<D>;
-    using L = SplitSmem<D, NT>;
+template <int D, int NT, bool DIAG>
+__global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(const DecodeArgs a) {
+    using G = PageGeom<D, DIAG>;
+    using L = SplitSmem<D, NT, DIAG>;
     constexpr int PG = kDecConsumers / NT;   // page groups: warps sharing a row tile split the pages
     constexpr int NKS = D / 16;              // QK k-steps over dims == PV m-tiles over dims
-    static_assert(kDecStages % PG == 0, "a stage's successive pages must go to one consumer warp");
+    constexpr int NS = L::STAGES;            // ring depth
+    static_assert(NS % PG == 0, "a stage's successive pages must go to one consumer warp");
 
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = smem_raw + ((16 - (smem_u32(smem_raw) & 15)) & 15);
     uint8_t *stages = smem;
     uint8_t *qbuf = stages + L::STAGES_BYTES;
     uint64_t *full = reinterpret_cast<uint64_t *>(qbuf + 2 * L::QBUF);
-    uint64_t *empty = full + kDecStages;
-    uint64_t *qfull = empty + kDecStages;
+    uint64_t *empty = full + NS;
+    uint64_t *qfull = empty + NS;
     uint64_t *qempty = qfull + 2;
     int *svalid = reinterpret_cast<int *>(qempty + 2);
-    float *mbuf = reinterpret_cast<float *>(svalid + kDecStages);
+    float *mbuf = reinterpret_cast<float *>(svalid + NS);
     int *misc = reinterpret_cast<int *>(mbuf + L::MBUF_FLOATS);
     // epilogue tables: output row index and merge weights per query row of the piece
     long long *orow = reinterpret_cast<long long *>(misc + 16);
@@ -297,7 +302,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
     float *xbuf = reinterpret_cast<float *>(prefix + ((nv + 1 + 3) & ~3));   // 16-byte aligned
     cluster_arrive_relaxed();   // this CTA has started (waited on before any remote access)
     if (tid == 0) {   // independent of the inputs: overlaps the wait below
-        for (int s = 0; s < kDecStages; ++s) {
+        for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
             mbar_init(&empty[s], NT);
         }
@@ -314,13 +319,13 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
     // virtual unit vc. As soon as the inputs are readable the producer copies that unit's query
     // rows and the range's first pages while the consumers read the lens; if the lens confirm the
     // guess the ring just continues, otherwise the copies are drained, the barriers re-armed and
-    // the general split runs (a wrong guess costs up to kDecStages page reads).
+    // the general split runs (a wrong guess costs up to NS page reads).
     const int kcl = a.cluster;
     const int crank = blockIdx.x % kcl, vc = blockIdx.x / kcl;   // clusters are consecutive blocks
     const bool try_spec = kcl > 1 && vc < nv && a.max_pages >= kcl && static_cast<long long>(nv) * kcl <= a.ncta;
     const int c0 = try_spec ? a.max_pages * crank / kcl : 0;   // max_pages * 8 fits in an int
     const int c1 = try_spec ? a.max_pages * (crank + 1) / kcl : 0;
-    const int n_first = min(kDecStages, c1 - c0);
+    const int n_first = min(NS, c1 - c0);
     __syncthreads();   // barriers initialised, qbuf zeroed
     // let the next launch in the stream become resident as our CTAs retire; then wait for every
     // preceding grid to complete (its writes visible) before reading any input
@@ -400,7 +405,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
         __syncthreads();
         alive = misc[10] != 0;
         if (tid == 0 && alive) {
-            for (int s2 = 0; s2 < kDecStages; ++s2) {
+            for (int s2 = 0; s2 < NS; ++s2) {
                 mbar_inval(&full[s2]);
                 mbar_inval(&empty[s2]);
                 mbar_init(&full[s2], 1);
@@ -487,9 +492,9 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                         bulk_g2s(qbuf + slot * L::QBUF + (row - p0) * L::QROWB, src, D * 2, &qfull[slot]);
                     }
                 }
-                const int s = i % kDecStages;
+                const int s = i % NS;
                 const int phys = __shfl_sync(0xffffffffu, my_page, k);
-                if (i >= kDecStages && !mbar_wait(&empty[s], ((i / kDecStages) - 1) & 1)) {
+                if (i >= NS && !mbar_wait(&empty[s], ((i / NS) - 1) & 1)) {
                     if (lane == 0) raise_flag(a.flags, FLAG_TIMEOUT);
                     alive = false;
                     break;
@@ -560,6 +565,21 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                 qn = fmaf(bf16hi(w1), bf16hi(w1), qn);
             }
         }
+        // diagonal closure: q_i^2 as the B operand of Var (16 x D) (q^2)^T, split into bf16 hi + lo
+        // (q^2 of a bf16 q has at most 16 significant bits: hi + lo holds it exactly)
+        uint32_t q2h[DIAG ? NKS : 1][2], q2l[DIAG ? NKS : 1][2];
+        if constexpr (DIAG) {
+#pragma unroll
+            for (int ks = 0; ks < NKS; ++ks)
+#pragma unroll
+                for (int r2 = 0; r2 < 2; ++r2) {
+                    const float lo = bf16lo(qf[ks][r2]), hi = bf16hi(qf[ks][r2]);
+                    const float slo = lo * lo, shi = hi * hi;
+                    const uint32_t h2 = pack_bf16x2(slo, shi);
+                    q2h[ks][r2] = h2;
+                    q2l[ks][r2] = pack_bf16x2(slo - bf16lo(h2), shi - bf16hi(h2));
+                }
+        }
         qn += __shfl_xor_sync(0xffffffffu, qn, 1);
         qn += __shfl_xor_sync(0xffffffffu, qn, 2);
         const float qn_r0 = __shfl_sync(0xffffffffu, qn, (2 * c) * 4);
@@ -573,8 +593,8 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
         // page i of the CTA's range goes to page group i % PG (global index, not piece-local)
         for (int k = ((pg - i0 % PG) + PG) % PG; k < npg && alive; k += PG) {
             const int i = i0 + k;
-            const int s = i % kDecStages;
-            if (!mbar_wait(&full[s], (i / kDecStages) & 1)) {
+            const int s = i % NS;
+            if (!mbar_wait(&full[s], (i / NS) & 1)) {
                 if (lane == 0) raise_flag(a.flags, FLAG_TIMEOUT);
                 alive = false;
                 break;
@@ -582,6 +602,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
             const bool valid = svalid[s] != 0;
             const int nvalid = min(kPageNodes, Lent - (lo + k) * kPageNodes);
             float sacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+            float cacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // diagonal closure: sum_i q_i^2 var_i
             uint32_t vf[NKS][4];
             float2 ab0 = make_float2(0.0f, 0.0f), ab1 = ab0;
             if (valid) {
@@ -597,6 +618,17 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
                         uint32_t a0, a1, a2, a3;
                         ldsm_x4(kb + node * G::ROWB + (swz(chunk, node) << 4), a0, a1, a2, a3);
                         mma_bf16(sacc, a0, a1, a2, a3, qf[ks][0], qf[ks][1]);
+                    }
+                    if constexpr (DIAG) {   // C^T (16 nodes x 8 rows) = Var (16 x D) (q^2)^T
+                        const uint32_t varb = kb + G::VAR_OFF;
+#pragma unroll
+                        for (int ks = 0; ks < NKS; ++ks) {
+                            const int chunk = 2 * ks + (mi >> 1);
+                            uint32_t a0, a1, a2, a3;
+                            ldsm_x4(varb + node * G::ROWB + (swz(chunk, node) << 4), a0, a1, a2, a3);
+                            mma_bf16(cacc, a0, a1, a2, a3, q2h[ks][0], q2h[ks][1]);
+                            mma_bf16(cacc, a0, a1, a2, a3, q2l[ks][0], q2l[ks][1]);
+                        }
                     }
                 }
                 // V^T fragments (A operand of O^T = V^T P^T) into registers now, so the stage goes
@@ -615,10 +647,16 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
             if (lane == 0) mbar_arrive(&empty[s]);   // the page is in registers: release the stage
             if (valid) {
                 float sl[4];
-                sl[0] = g < nvalid ? fmaf(sacc[0], c_scale, kLog2e * fmaf(qn_r0, ab0.y, ab0.x)) : -INFINITY;
-                sl[1] = g < nvalid ? fmaf(sacc[1], c_scale, kLog2e * fmaf(qn_r1, ab0.y, ab0.x)) : -INFINITY;
-                sl[2] = g + 8 < nvalid ? fmaf(sacc[2], c_scale, kLog2e * fmaf(qn_r0, ab1.y, ab1.x)) : -INFINITY;
-                sl[3] = g + 8 < nvalid ? fmaf(sacc[3], c_scale, kLog2e * fmaf(qn_r1, ab1.y, ab1.x)) : -INFINITY;
+                // closure: |q|^2 beta, or sum_i q_i^2 var_i / (2d) with the diagonal variances
+                constexpr float kInv2d = 0.5f / D;
+                const float cl0 = DIAG ? fmaf(cacc[0], kInv2d, ab0.x) : fmaf(qn_r0, ab0.y, ab0.x);
+                const float cl1 = DIAG ? fmaf(cacc[1], kInv2d, ab0.x) : fmaf(qn_r1, ab0.y, ab0.x);
+                const float cl2 = DIAG ? fmaf(cacc[2], kInv2d, ab1.x) : fmaf(qn_r0, ab1.y, ab1.x);
+                const float cl3 = DIAG ? fmaf(cacc[3], kInv2d, ab1.x) : fmaf(qn_r1, ab1.y, ab1.x);
+                sl[0] = g < nvalid ? fmaf(sacc[0], c_scale, kLog2e * cl0) : -INFINITY;
+                sl[1] = g < nvalid ? fmaf(sacc[1], c_scale, kLog2e * cl1) : -INFINITY;
+                sl[2] = g + 8 < nvalid ? fmaf(sacc[2], c_scale, kLog2e * cl2) : -INFINITY;
+                sl[3] = g + 8 < nvalid ? fmaf(sacc[3], c_scale, kLog2e * cl3) : -INFINITY;
                 float mx0 = fmaxf(sl[0], sl[2]), mx1 = fmaxf(sl[1], sl[3]);
 #pragma unroll
                 for (int off = 4; off < 32; off <<= 1) {
@@ -842,7 +880,7 @@ __global__ void __launch_bounds__(kDecThreads, 2) k_decode_split(const DecodeArg
 }
 
 // fp32 caches: exact fp32 CUDA-core path, one CTA per unit, one warp per query row.
-template <int D>
+template <int D, bool DIAG>
 __global__ void __launch_bounds__(128) k_decode_f32(const DecodeArgs a) {
     constexpr int PER = D / 32;
     const int u = blockIdx.x;
@@ -851,7 +889,7 @@ __global__ void __launch_bounds__(128) k_decode_f32(const DecodeArgs a) {
     const int L = clamp_entries(a, u);
     const float *q = static_cast<const float *>(a.q);
     constexpr int VEC_FLOATS = kPageNodes * D;   // fp32 keys (then values) of one page
-    constexpr long long PAGE_FLOATS = 2 * VEC_FLOATS + 2 * kPageNodes;
+    constexpr long long PAGE_FLOATS = (DIAG ? 3 : 2) * VEC_FLOATS + 2 * kPageNodes;
     const float *pool = reinterpret_cast<const float *>(a.pages);
     float *outp = static_cast<float *>(a.out);
     const float inv_sqrt_d = 1.0f / sqrtf(static_cast<float>(D));
@@ -888,7 +926,20 @@ __global__ void __launch_bounds__(128) k_decode_f32(const DecodeArgs a) {
 #pragma unroll
             for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
             const float2 ab = reinterpret_cast<const float2 *>(pk + 2 * VEC_FLOATS)[slot];
-            const float s = fmaf(dot, inv_sqrt_d, fmaf(qn, ab.y, ab.x));
+            float closure = qn * ab.y;   // |q|^2 beta
+            if constexpr (DIAG) {        // sum_i q_i^2 var_i / (2d)
+                const float *pvar = pk + 2 * VEC_FLOATS + 2 * kPageNodes;
+                float c = 0.0f;
+#pragma unroll
+                for (int i = 0; i < PER; ++i) {
+                    const int dim = lane + 32 * i;
+                    c = fmaf(qv[i] * qv[i], pvar[nb + swz(dim >> 2, slot) * 4 + (dim & 3)], c);
+                }
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) c += __shfl_xor_sync(0xffffffffu, c, off);
+                closure = c * (0.5f / D);
+            }
+            const float s = fmaf(dot, inv_sqrt_d, ab.x + closure);
             const float mn = fmaxf(m, s);
             const float corr = expf(m - mn);
             const float p = expf(s - mn);
@@ -909,18 +960,18 @@ __global__ void __launch_bounds__(128) k_decode_f32(const DecodeArgs a) {
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-template <int D, int NT>
+template <int D, int NT, bool DIAG>
 static size_t split_smem(int n_vunits, int cluster) {
-    return SplitSmem<D, NT>::FIXED + static_cast<size_t>((n_vunits + 1 + 3) & ~3) * 4 +
+    return SplitSmem<D, NT, DIAG>::FIXED + static_cast<size_t>((n_vunits + 1 + 3) & ~3) * 4 +
            static_cast<size_t>(cluster - 1) * (NT * 8) * (D + 1) * 4;   // aligned-split receive buffer
 }
 
 constexpr int kMaxCluster = 8;   // portable cluster size limit
 // cluster > 1 needs n_vunits * cluster <= ncta <= kMaxDecodeCtas
-template <int D, int NT>
+template <int D, int NT, bool DIAG>
 static size_t split_smem_max() {
-    const size_t a = split_smem<D, NT>(kMaxVUnits, 1);
-    const size_t b = split_smem<D, NT>(kMaxDecodeCtas / 2, kMaxCluster);
+    const size_t a = split_smem<D, NT, DIAG>(kMaxVUnits, 1);
+    const size_t b = split_smem<D, NT, DIAG>(kMaxDecodeCtas / 2, kMaxCluster);
     return a > b ? a : b;
 }
 
@@ -928,7 +979,7 @@ static size_t split_smem_max() {
 // SMs x resident CTAs without clusters, resident clusters x cluster size with them (a cluster
 // must fit inside one GPC). Queried once and cached, so that later calls (and stream capture)
 // issue no attribute queries.
-template <int D, int NT>
+template <int D, int NT, bool DIAG>
 static cudaError_t split_grid(size_t smem, int cluster, int *ncta) {
     struct Entry {
         int dev;
@@ -947,19 +998,33 @@ static cudaError_t split_grid(size_t smem, int cluster, int *ncta) {
             *ncta = c.ncta;
             return cudaSuccess;
         }
-    bool configured = false;
-    for (const Entry &c : cache) configured |= (c.dev == dev);
-    if (!configured) {
-        // the largest request any call can make
-        e = cudaFuncSetAttribute(k_decode_split<D, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(split_smem_max<D, NT>()));
+    static std::vector<std::pair<int, size_t>> limits;   // per device: the largest launchable request
+    size_t limit = 0;
+    for (const auto &l : limits)
+        if (l.first == dev) limit = l.second;
+    if (limit == 0) {
+        // the largest request any call can make, within the device's opt-in maximum
+        // (the opt-in maximum covers static and dynamic shared memory together)
+        int optin = 0;
+        if ((e = cudaDeviceGetAttribute(&optin, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev)) != cudaSuccess)
+            return e;
+        cudaFuncAttributes fa;
+        if ((e = cudaFuncGetAttributes(&fa, k_decode_split<D, NT, DIAG>)) != cudaSuccess) return e;
+        const size_t room = static_cast<size_t>(optin) - fa.sharedSizeBytes;
+        limit = split_smem_max<D, NT, DIAG>();
+        if (limit > room) limit = room;
+        e = cudaFuncSetAttribute(k_decode_split<D, NT, DIAG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(limit));
         if (e != cudaSuccess) return e;
+        limits.emplace_back(dev, limit);
     }
     int n = 0;
-    if (cluster == 1) {
+    if (smem > limit) {
+        n = 0;   // does not fit this device: not launchable
+    } else if (cluster == 1) {
         int sms = 0, occ = 0;
         if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_split<D, NT>, kDecThreads, smem)) !=
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_split<D, NT, DIAG>, kDecThreads, smem)) !=
             cudaSuccess)
             return e;
         n = sms * (occ > 0 ? occ : 1);
@@ -976,7 +1041,7 @@ static cudaError_t split_grid(size_t smem, int cluster, int *ncta) {
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
         int nc = 0;
-        if (cudaOccupancyMaxActiveClusters(&nc, k_decode_split<D, NT>, &cfg) != cudaSuccess) {
+        if (cudaOccupancyMaxActiveClusters(&nc, k_decode_split<D, NT, DIAG>, &cfg) != cudaSuccess) {
             (void)cudaGetLastError();   // this cluster size is not available: not an error of the call
             nc = 0;
         }
@@ -993,16 +1058,17 @@ static cudaError_t split_grid(size_t smem, int cluster, int *ncta) {
 // (an aligned split then streams at most 4/3 of the pages per CTA a stream-K split would, and
 // saves its global merges). It is used only if the device finds every unit equally long;
 // otherwise the same grid runs the stream-K split.
-template <int D, int NT>
+template <int D, int NT, bool DIAG>
 static cudaError_t split_config(DecodeArgs *a, size_t *smem) {
-    *smem = split_smem<D, NT>(a->n_vunits, 1);
-    cudaError_t e = split_grid<D, NT>(*smem, 1, &a->ncta);
+    *smem = split_smem<D, NT, DIAG>(a->n_vunits, 1);
+    cudaError_t e = split_grid<D, NT, DIAG>(*smem, 1, &a->ncta);
     if (e != cudaSuccess) return e;
+    if (a->ncta < 1) return cudaErrorInvalidValue;
     a->cluster = 1;
     for (int k = a->ncta / a->n_vunits < kMaxCluster ? a->ncta / a->n_vunits : kMaxCluster; k > 1; --k) {
-        const size_t sk = split_smem<D, NT>(a->n_vunits, k);
+        const size_t sk = split_smem<D, NT, DIAG>(a->n_vunits, k);
         int n = 0;
-        if ((e = split_grid<D, NT>(sk, k, &n)) != cudaSuccess) return e;
+        if ((e = split_grid<D, NT, DIAG>(sk, k, &n)) != cudaSuccess) return e;
         if (static_cast<long long>(a->n_vunits) * k <= n && static_cast<long long>(a->n_vunits) * k * 4 >= 3LL * n) {
             a->cluster = k;
             a->ncta = n;
@@ -1013,11 +1079,11 @@ static cudaError_t split_config(DecodeArgs *a, size_t *smem) {
     return cudaSuccess;
 }
 
-template <int D, int NT>
+template <int D, int NT, bool DIAG>
 static cudaError_t launch_split(const DecodeArgs &a0, cudaStream_t s) {
     DecodeArgs a = a0;
     size_t smem = 0;
-    cudaError_t e = split_config<D, NT>(&a, &smem);
+    cudaError_t e = split_config<D, NT, DIAG>(&a, &smem);
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.ncta);
@@ -1033,51 +1099,61 @@ static cudaError_t launch_split(const DecodeArgs &a0, cudaStream_t s) {
     attr[1].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = a.cluster > 1 ? 2 : 1;
-    return cudaLaunchKernelEx(&cfg, k_decode_split<D, NT>, a);
+    return cudaLaunchKernelEx(&cfg, k_decode_split<D, NT, DIAG>, a);
 }
 
-cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
+template <bool DIAG>
+static cudaError_t launch_decode_t(const DecodeArgs &a, cudaStream_t s) {
     if (a.dtype == SKV_F32) {
-        if (a.d == 128) k_decode_f32<128><<<a.B * a.Hkv, 128, 0, s>>>(a);
-        else k_decode_f32<64><<<a.B * a.Hkv, 128, 0, s>>>(a);
+        if (a.d == 128) k_decode_f32<128, DIAG><<<a.B * a.Hkv, 128, 0, s>>>(a);
+        else k_decode_f32<64, DIAG><<<a.B * a.Hkv, 128, 0, s>>>(a);
         return cudaGetLastError();
     }
     const int nt = a.pass_rows / 8 + (a.pass_rows % 8 ? 1 : 0);
     if (a.d == 128) {
-        if (nt == 1) return launch_split<128, 1>(a, s);
-        if (nt == 2) return launch_split<128, 2>(a, s);
-        return launch_split<128, 4>(a, s);
+        if (nt == 1) return launch_split<128, 1, DIAG>(a, s);
+        if (nt == 2) return launch_split<128, 2, DIAG>(a, s);
+        return launch_split<128, 4, DIAG>(a, s);
     }
-    if (nt == 1) return launch_split<64, 1>(a, s);
-    if (nt == 2) return launch_split<64, 2>(a, s);
-    return launch_split<64, 4>(a, s);
+    if (nt == 1) return launch_split<64, 1, DIAG>(a, s);
+    if (nt == 2) return launch_split<64, 2, DIAG>(a, s);
+    return launch_split<64, 4, DIAG>(a, s);
+}
+
+cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s) {
+    return a.closure == SKV_CLOSURE_DIAGONAL ? launch_decode_t<true>(a, s) : launch_decode_t<false>(a, s);
 }
 
 }  // namespace skv
 
 namespace skv {
 
-template <int D, int NT>
+template <int D, int NT, bool DIAG>
 static cudaError_t split_ctas(const DecodeArgs &a0, int *ncta) {
     DecodeArgs a = a0;
     size_t smem = 0;
-    const cudaError_t e = split_config<D, NT>(&a, &smem);
+    const cudaError_t e = split_config<D, NT, DIAG>(&a, &smem);
     *ncta = a.ncta;
     return e;
 }
 
 // The grid k_decode_split would use for these arguments (bf16 caches), for callers that must size
 // split-partial storage before launching. Queries (and caches) the same occupancy as the launcher.
-cudaError_t decode_split_ctas(const DecodeArgs &a, int *ncta) {
+template <bool DIAG>
+static cudaError_t split_ctas_t(const DecodeArgs &a, int *ncta) {
     const int nt = a.pass_rows / 8 + (a.pass_rows % 8 ? 1 : 0);
     if (a.d == 128) {
-        if (nt == 1) return split_ctas<128, 1>(a, ncta);
-        if (nt == 2) return split_ctas<128, 2>(a, ncta);
-        return split_ctas<128, 4>(a, ncta);
+        if (nt == 1) return split_ctas<128, 1, DIAG>(a, ncta);
+        if (nt == 2) return split_ctas<128, 2, DIAG>(a, ncta);
+        return split_ctas<128, 4, DIAG>(a, ncta);
     }
-    if (nt == 1) return split_ctas<64, 1>(a, ncta);
-    if (nt == 2) return split_ctas<64, 2>(a, ncta);
-    return split_ctas<64, 4>(a, ncta);
+    if (nt == 1) return split_ctas<64, 1, DIAG>(a, ncta);
+    if (nt == 2) return split_ctas<64, 2, DIAG>(a, ncta);
+    return split_ctas<64, 4, DIAG>(a, ncta);
+}
+
+cudaError_t decode_split_ctas(const DecodeArgs &a, int *ncta) {
+    return a.closure == SKV_CLOSURE_DIAGONAL ? split_ctas_t<true>(a, ncta) : split_ctas_t<false>(a, ncta);
 }
 
 }  // namespace skv

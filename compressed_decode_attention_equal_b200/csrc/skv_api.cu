@@ -232,12 +232,16 @@ const char *skv_status_string(int status) {
     }
 }
 
-int skv_abi_version(void) { return 201; }
+int skv_abi_version(void) { return 202; }
 
-size_t skv_page_bytes(skv_dtype dtype, int d) {
+size_t skv_page_bytes(skv_dtype dtype, int d) { return skv_page_bytes_ex(dtype, d, SKV_CLOSURE_SCALAR); }
+
+size_t skv_page_bytes_ex(skv_dtype dtype, int d, skv_closure closure) {
     if ((dtype != SKV_BF16 && dtype != SKV_F32) || (d != 64 && d != 128)) return 0;
+    if (closure != SKV_CLOSURE_SCALAR && closure != SKV_CLOSURE_DIAGONAL) return 0;
     const size_t elem = dtype == SKV_BF16 ? 2 : 4;
-    return 2 * static_cast<size_t>(kPageNodes) * d * elem + kPageNodes * 8;
+    const size_t vec = static_cast<size_t>(kPageNodes) * d * elem;
+    return (closure == SKV_CLOSURE_DIAGONAL ? 3 : 2) * vec + kPageNodes * 8;
 }
 
 skv_status skv_projection_matrix(uint64_t proj_seed, int d, float *P_host) {
@@ -258,13 +262,16 @@ skv_status skv_coarsen_ex(const void *k, const void *v, skv_dtype dtype, int B, 
                           const skv_node_pool *pool, const int32_t *page_table, int max_pages, int32_t *lens,
                           int32_t *boundaries, int64_t *cumvar, void *workspace, size_t ws_bytes,
                           const skv_coarsen_options *options, void *stream) {
-    int representative = SKV_REP_MEAN;
+    int representative = SKV_REP_MEAN, closure = SKV_CLOSURE_SCALAR;
     if (options) {
         if (options->representative != SKV_REP_MEAN && options->representative != SKV_REP_VARIATION_WEIGHTED)
             return SKV_ERR_INVALID_ARG;
-        for (int i = 0; i < 7; ++i)
+        if (options->closure != SKV_CLOSURE_SCALAR && options->closure != SKV_CLOSURE_DIAGONAL)
+            return SKV_ERR_INVALID_ARG;
+        for (int i = 0; i < 6; ++i)
             if (options->reserved[i] != 0) return SKV_ERR_INVALID_ARG;
         representative = options->representative;
+        closure = options->closure;
     }
     if (dtype != SKV_BF16 && dtype != SKV_F32) return SKV_ERR_UNSUPPORTED;
     static SeqTable table;   // host staging; guarded by the mutex below
@@ -316,6 +323,7 @@ skv_status skv_coarsen_ex(const void *k, const void *v, skv_dtype dtype, int B, 
     a.user_bounds = boundaries;
     a.cumvar = cumvar;
     a.representative = representative;
+    a.closure = closure;
     const cudaError_t e = launch_coarsen(a, table, proj, map_k, map_v, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SKV_OK : SKV_ERR_CUDA;
 }
@@ -334,9 +342,18 @@ size_t skv_decode_workspace_bytes(int B, int R, int Hq, int Hkv, int d, int max_
     return p.lay.total;
 }
 
-skv_status skv_decode_attn(const void *q, skv_dtype dtype, int B, int R, int Hq, int Hkv, int d,
-                           const skv_node_pool *pool, const int32_t *page_table, int max_pages, const int32_t *lens,
-                           void *out, float *lse, void *workspace, size_t ws_bytes, void *stream) {
+skv_status skv_decode_attn_ex(const void *q, skv_dtype dtype, int B, int R, int Hq, int Hkv, int d,
+                              const skv_node_pool *pool, const int32_t *page_table, int max_pages,
+                              const int32_t *lens, void *out, float *lse, void *workspace, size_t ws_bytes,
+                              const skv_decode_options *options, void *stream) {
+    int closure = SKV_CLOSURE_SCALAR;
+    if (options) {
+        if (options->closure != SKV_CLOSURE_SCALAR && options->closure != SKV_CLOSURE_DIAGONAL)
+            return SKV_ERR_INVALID_ARG;
+        for (int i = 0; i < 7; ++i)
+            if (options->reserved[i] != 0) return SKV_ERR_INVALID_ARG;
+        closure = options->closure;
+    }
     DecodePlan plan;
     skv_status st = plan_decode(dtype, B, R, Hq, Hkv, d, max_pages, &plan);
     if (st != SKV_OK) return st;
@@ -370,8 +387,16 @@ skv_status skv_decode_attn(const void *q, skv_dtype dtype, int B, int R, int Hq,
     a.part_l = reinterpret_cast<float *>(ws + plan.lay.part_l);
     a.counters = reinterpret_cast<int32_t *>(ws + plan.lay.counters);
     a.flags = reinterpret_cast<uint32_t *>(ws);
+    a.closure = closure;
     const cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SKV_OK : SKV_ERR_CUDA;
+}
+
+skv_status skv_decode_attn(const void *q, skv_dtype dtype, int B, int R, int Hq, int Hkv, int d,
+                           const skv_node_pool *pool, const int32_t *page_table, int max_pages, const int32_t *lens,
+                           void *out, float *lse, void *workspace, size_t ws_bytes, void *stream) {
+    return skv_decode_attn_ex(q, dtype, B, R, Hq, Hkv, d, pool, page_table, max_pages, lens, out, lse, workspace,
+                              ws_bytes, nullptr, stream);
 }
 
 skv_status skv_workspace_error(const void *workspace, void *stream, uint32_t *flags_host) {

@@ -58,6 +58,7 @@ struct CoarsenArgs {
     int32_t *user_bounds;
     int64_t *cumvar;
     int representative;  // skv_representative of the middle segments' stored key and value
+    int closure;         // skv_closure: SKV_CLOSURE_DIAGONAL also writes per-dimension variances
 };
 
 // Workspace carve-up (offsets in bytes from the workspace start).
@@ -96,6 +97,7 @@ struct DecodeArgs {
     float *part_l;    // [ncta][2][pass_rows] split partial log2-partitions
     int32_t *counters;   // [n_vunits] pieces finished per virtual unit (zero between calls)
     uint32_t *flags;
+    int closure;         // skv_closure of the pool (SKV_CLOSURE_DIAGONAL: pages carry variances)
 };
 
 struct DecodeLayout {

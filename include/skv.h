@@ -48,7 +48,10 @@
  *    [0, V)        keys   [16][d] in the dtype         (V = 16 * d * elem)
  *    [V, 2V)       values [16][d] in the dtype
  *    [2V, 2V+128)  {alpha, beta} fp32 pairs [16]
- *  Within the key and value blocks the 16-byte chunk c of slot n's vector is
+ *  and, in a pool built for the diagonal closure (SKV_CLOSURE_DIAGONAL), also
+ *    [2V+128, 3V+128)  per-dimension key variances [16][d] in the dtype
+ *  (skv_page_bytes_ex gives the page size of either layout). Within the key,
+ *  value and variance blocks the 16-byte chunk c of slot n's vector is
  *  stored at chunk position c ^ (n & 7) (a bank-conflict-free order for the
  *  tensor-core fragment loads; d * elem >= 128 bytes). One page is one copy.
  *  page_table : [B][Hkv][max_pages] int32 physical page ids; entry e of unit
@@ -97,6 +100,24 @@ int skv_abi_version(void);
 
 /* Bytes of one node-pool page: 2 * 16 * d * elem + 128 (0 for an unsupported dtype or d). */
 size_t skv_page_bytes(skv_dtype dtype, int d);
+
+/*
+ * The variance a node carries into the decode logit ("SPICY-KV" Independent
+ * Claim 3: a scalar sigma_m^2 or a diagonal vector):
+ *   SKV_CLOSURE_SCALAR (0): beta = sigma^2 / (2d), logit term |q|^2 beta.
+ *   SKV_CLOSURE_DIAGONAL (1): the node also stores var_i, the members'
+ *     population variance of key dimension i; logit term
+ *     sum_i q_i^2 var_i / (2d) (the second cumulant of q.eps/sqrt(d) for
+ *     independent per-dimension deviations; equal to the scalar term when
+ *     every var_i equals sigma^2). The pages grow by 16 * d * elem bytes.
+ * A pool is built for one closure: skv_coarsen_ex and skv_decode_attn_ex must
+ * be given the closure its pages were sized for.
+ */
+typedef enum { SKV_CLOSURE_SCALAR = 0, SKV_CLOSURE_DIAGONAL = 1 } skv_closure;
+
+/* Bytes of one page for a closure: skv_page_bytes, plus 16 * d * elem for
+ * SKV_CLOSURE_DIAGONAL (0 for an unsupported dtype, d or closure). */
+size_t skv_page_bytes_ex(skv_dtype dtype, int d, skv_closure closure);
 
 /*
  * The projection the coarsener draws from proj_seed ("Equal-Variation KV
@@ -178,20 +199,23 @@ skv_status skv_coarsen(const void *k, const void *v, skv_dtype dtype, int B, int
  *   In both cases sigma^2 (and beta) is the members' population key variance
  *   about their plain mean (Claim 3 defines it on the members), m and alpha are
  *   unchanged, and the boundaries do not depend on the option.
+ * closure: the pool's skv_closure; SKV_CLOSURE_DIAGONAL also writes each
+ *   node's per-dimension key variances (zero for exact tokens).
  * reserved: must be zero.
  */
 typedef enum { SKV_REP_MEAN = 0, SKV_REP_VARIATION_WEIGHTED = 1 } skv_representative;
 
 typedef struct {
     int32_t representative; /* skv_representative */
-    int32_t reserved[7];
+    int32_t closure;        /* skv_closure */
+    int32_t reserved[6];
 } skv_coarsen_options;
 
 /*
  * skv_coarsen with options (NULL = defaults, identical to skv_coarsen). Same
  * arguments, layouts, ownership and errors as skv_coarsen; additionally
- * SKV_ERR_INVALID_ARG for an unknown representative or a nonzero reserved
- * field.
+ * SKV_ERR_INVALID_ARG for an unknown representative or closure or a nonzero
+ * reserved field.
  */
 skv_status skv_coarsen_ex(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d,
                           const int32_t *T_host, int n_sink, int n_recent, const int32_t *N_host,
@@ -229,6 +253,27 @@ skv_status skv_decode_attn(const void *q, skv_dtype dtype, int B, int R, int Hq,
                            const skv_node_pool *pool, const int32_t *page_table, int max_pages,
                            const int32_t *lens, void *out, float *lse, void *workspace, size_t ws_bytes,
                            void *stream);
+
+/*
+ * Options of skv_decode_attn_ex. closure: the pool's skv_closure
+ * (SKV_CLOSURE_DIAGONAL reads each node's per-dimension variances and uses
+ * sum_i q_i^2 var_i / (2d) in place of |q|^2 beta). reserved: must be zero.
+ */
+typedef struct {
+    int32_t closure; /* skv_closure */
+    int32_t reserved[7];
+} skv_decode_options;
+
+/*
+ * skv_decode_attn with options (NULL = defaults, identical to
+ * skv_decode_attn). Same arguments, layouts, ownership, workspace and errors;
+ * additionally SKV_ERR_INVALID_ARG for an unknown closure or a nonzero
+ * reserved field.
+ */
+skv_status skv_decode_attn_ex(const void *q, skv_dtype dtype, int B, int R, int Hq, int Hkv, int d,
+                              const skv_node_pool *pool, const int32_t *page_table, int max_pages,
+                              const int32_t *lens, void *out, float *lse, void *workspace, size_t ws_bytes,
+                              const skv_decode_options *options, void *stream);
 
 /*
  * Decode attention without any caller-provided workspace. (The sources describe no such entry

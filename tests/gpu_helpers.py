@@ -20,19 +20,22 @@ TOL_BF16_MAX_ABS = 2e-2
 TOL_LSE_ABS = 1e-3
 
 
-def pool_for_units(entries_per_unit, B, Hkv, d, dtype, shuffle=False, seed=0, spare_pages=0, device="cuda"):
+def pool_for_units(entries_per_unit, B, Hkv, d, dtype, shuffle=False, seed=0, spare_pages=0, device="cuda",
+                   closure="scalar"):
     """Pool and page table with ceil(E/16) pages for each unit (entries_per_unit[b] per head)."""
     pages = [max(1, -(-int(e) // skv.PAGE_NODES)) for e in entries_per_unit]
     table, total = workloads.page_assignment(B, Hkv, pages, shuffle, seed)
-    pool = skv.NodePool(total + spare_pages, d, dtype, device=device)
+    pool = skv.NodePool(total + spare_pages, d, dtype, device=device, closure=closure)
     # slots no entry uses hold NaN: a kernel that lets them leak into a result fails the checks
     pool.k.fill_(float("nan"))
     pool.v.fill_(float("nan"))
     pool.ab.fill_(float("nan"))
+    if pool.var is not None:
+        pool.var.fill_(float("nan"))
     return pool, table.to(device)
 
 
-def write_entries(pool, table, b, h, kt, vt, alpha, beta):
+def write_entries(pool, table, b, h, kt, vt, alpha, beta, var=None):
     """Write entries of unit (b, h) into the pool's swizzled page layout (inverse of read_entries)."""
     E, d = kt.shape
     if E == 0:
@@ -48,25 +51,27 @@ def write_entries(pool, table, b, h, kt, vt, alpha, beta):
     v4[pg[:, None], sl[:, None], phys] = vt.to(pool.dtype).reshape(E, ch, epc).to(dev)
     pool.ab[pg, sl, 0] = alpha.float().to(dev)
     pool.ab[pg, sl, 1] = beta.float().to(dev)
+    if var is not None:
+        r4 = pool.var.view(pool.num_pages, skv.PAGE_NODES, ch, epc)
+        r4[pg[:, None], sl[:, None], phys] = var.to(pool.dtype).reshape(E, ch, epc).to(dev)
 
 
 class GpuUnit:
     """A unit's GPU-stored entries as fp64 numpy arrays (attribute names the oracle expects)."""
 
-    def __init__(self, kt, vt, alpha, beta):
-        self.kt, self.vt, self.alpha, self.beta = kt, vt, alpha, beta
+    def __init__(self, kt, vt, alpha, beta, var=None):
+        self.kt, self.vt, self.alpha, self.beta, self.var = kt, vt, alpha, beta, var
+
+
+def gpu_unit(pool, table, lens, b, h):
+    kt, vt, al, be = skv.read_entries(pool, table, lens, b, h)
+    var = skv.read_variances(pool, table, lens, b, h).double().cpu().numpy() if pool.var is not None else None
+    return GpuUnit(kt.double().cpu().numpy(), vt.double().cpu().numpy(), al.double().cpu().numpy(),
+                   be.double().cpu().numpy(), var)
 
 
 def gpu_units(pool, table, lens, B, Hkv):
-    out = []
-    for b in range(B):
-        row = []
-        for h in range(Hkv):
-            kt, vt, al, be = skv.read_entries(pool, table, lens, b, h)
-            row.append(GpuUnit(kt.double().cpu().numpy(), vt.double().cpu().numpy(), al.double().cpu().numpy(),
-                               be.double().cpu().numpy()))
-        out.append(row)
-    return out
+    return [[gpu_unit(pool, table, lens, b, h) for h in range(Hkv)] for b in range(B)]
 
 
 def rel_l2(a, b):
@@ -146,6 +151,15 @@ def check_nodes(gpu_unit, orc_unit, dtype, d, what="", slack=None):
                 bound = bound + slack[i]
             assert np.all(err <= bound), f"{what}: {name} worst excess {np.max(err / bound):.3f}"
             assert rel_l2(g, o) <= TOL_BF16_REL_L2
+    if getattr(gpu_unit, "var", None) is not None:
+        # per-dimension variances: an fp32 two-pass variance rounded once to the dtype
+        g, o = gpu_unit.var, orc_unit.var
+        err = np.abs(g - o)
+        if dtype == torch.float32:
+            bound = 2e-6 * np.abs(o) + 1e-12
+        else:
+            bound = 0.5 * bf16_ulp(o) + 2e-6 * np.abs(o) + 1e-12
+        assert np.all(err <= bound), f"{what}: var worst excess {np.max(err / bound):.3f}"
 
 
 def to_np32(t: torch.Tensor) -> np.ndarray:

@@ -37,7 +37,7 @@ def test_status_strings(lib):
         s = lib.skv_status_string(code).decode()
         assert s.startswith("SKV_")
     assert "unknown" in lib.skv_status_string(12345).decode()
-    assert lib.skv_abi_version() == 201
+    assert lib.skv_abi_version() == 202
     assert lib.skv_page_bytes(1, 128) == 2 * 16 * 128 * 2 + 128
     assert lib.skv_page_bytes(0, 64) == 2 * 16 * 64 * 4 + 128
     assert lib.skv_page_bytes(1, 96) == 0
@@ -106,6 +106,32 @@ def test_coarsen_options_validated_before_any_launch(lib):
     ok = _lib.SkvCoarsenOptions(_lib.SKV_REP_VARIATION_WEIGHTED)
     assert lib.skv_coarsen_ex(*args, ctypes.byref(ok), null) == _lib.SKV_ERR_WORKSPACE
     assert lib.skv_coarsen_ex(*args, None, null) == _lib.SKV_ERR_WORKSPACE
+
+
+def test_page_bytes_and_closure_options(lib):
+    from compressed_decode_attention_equal_b200 import _lib
+    # [K | V | alpha,beta] and, for the diagonal closure, [K | V | alpha,beta | var]
+    assert lib.skv_page_bytes_ex(1, 128, 0) == lib.skv_page_bytes(1, 128) == 2 * 16 * 128 * 2 + 128
+    assert lib.skv_page_bytes_ex(1, 128, 1) == 3 * 16 * 128 * 2 + 128
+    assert lib.skv_page_bytes_ex(0, 64, 1) == 3 * 16 * 64 * 4 + 128
+    assert lib.skv_page_bytes_ex(1, 128, 2) == 0 and lib.skv_page_bytes_ex(1, 96, 1) == 0
+    null = ctypes.c_void_p(0)
+    pool = _lib.SkvNodePool(16, 1)
+    args = (ctypes.c_void_p(256), 1, 1, 1, 7, 1, 128, ctypes.byref(pool), ctypes.c_void_p(16), 4,
+            ctypes.c_void_p(16), ctypes.c_void_p(256), ctypes.c_void_p(256), ctypes.c_void_p(256), 16)
+    bad = _lib.SkvDecodeOptions(2)
+    assert lib.skv_decode_attn_ex(*args, ctypes.byref(bad), null) == _lib.SKV_ERR_INVALID_ARG
+    bad_res = _lib.SkvDecodeOptions(1)
+    bad_res.reserved[0] = 3
+    assert lib.skv_decode_attn_ex(*args, ctypes.byref(bad_res), null) == _lib.SKV_ERR_INVALID_ARG
+    ok = _lib.SkvDecodeOptions(_lib.SKV_CLOSURE_DIAGONAL)
+    assert lib.skv_decode_attn_ex(*args, ctypes.byref(ok), null) == _lib.SKV_ERR_WORKSPACE
+    T = (ctypes.c_int32 * 1)(100)
+    N = (ctypes.c_int32 * 1)(4)
+    cargs = (ctypes.c_void_p(256), ctypes.c_void_p(256), 1, 1, 1, 128, T, 8, 48, N, 0, ctypes.byref(pool),
+             ctypes.c_void_p(16), 4, ctypes.c_void_p(16), null, null, ctypes.c_void_p(256), 16)
+    assert lib.skv_coarsen_ex(*cargs, ctypes.byref(_lib.SkvCoarsenOptions(0, 2)), null) == _lib.SKV_ERR_INVALID_ARG
+    assert lib.skv_coarsen_ex(*cargs, ctypes.byref(_lib.SkvCoarsenOptions(1, 1)), null) == _lib.SKV_ERR_WORKSPACE
 
 
 def test_binding_fails_loudly_without_library(tmp_path):

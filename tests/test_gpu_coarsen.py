@@ -13,18 +13,19 @@ import torch
 import compressed_decode_attention_equal_b200 as skv
 import oracle
 import workloads
-from gpu_helpers import check_decode, check_nodes, gpu_units, pool_for_units, to_np32, weighted_slack
+from gpu_helpers import check_decode, check_nodes, gpu_unit, gpu_units, pool_for_units, to_np32, weighted_slack
 
 pytestmark = pytest.mark.gpu
 
 S, W = workloads.N_SINK, workloads.N_RECENT
 
 
-def run_coarsen(k, v, Hkv, T_list, N_list, seed, n_sink=S, n_recent=W, shuffle=True, representative="mean"):
+def run_coarsen(k, v, Hkv, T_list, N_list, seed, n_sink=S, n_recent=W, shuffle=True, representative="mean",
+                closure="scalar"):
     B = len(T_list)
     d = k.shape[-1]
     ent = [skv.entries_bound(T, N, n_sink, n_recent) for T, N in zip(T_list, N_list)]
-    pool, table = pool_for_units(ent, B, Hkv, d, k.dtype, shuffle=shuffle, seed=seed)
+    pool, table = pool_for_units(ent, B, Hkv, d, k.dtype, shuffle=shuffle, seed=seed, closure=closure)
     Nmax = max(N_list)
     bnd = torch.full((B, Hkv, Nmax + 1), -7, dtype=torch.int32, device="cuda")
     cum = torch.full((k.shape[0],), -7, dtype=torch.int64, device="cuda")
@@ -62,14 +63,7 @@ def compare_units(r, orc, k, v, T_list, Hkv, N_list, dtype):
         bg = r["bnd"][b, h, :N_list[b] + 1].cpu().numpy()
         assert np.array_equal(bg, u.bounds), f"{what}: boundaries differ"
         assert int(r["lens"][b, h]) == u.kt.shape[0], f"{what}: lens"
-        kt, vt, al, be = skv.read_entries(r["pool"], r["table"], r["lens"], b, h)
-
-        class G:
-            pass
-
-        gu = G()
-        gu.kt, gu.vt = kt.double().cpu().numpy(), vt.double().cpu().numpy()
-        gu.alpha, gu.beta = al.double().cpu().numpy(), be.double().cpu().numpy()
+        gu = gpu_unit(r["pool"], r["table"], r["lens"], b, h)
         kk = to_np32(workloads.unit_rows(k, T_list, Hkv, b, h))
         vv = to_np32(workloads.unit_rows(v, T_list, Hkv, b, h))
         check_nodes(gu, u, dtype, d, what, slack=weighted_slack(u, kk, vv))
@@ -109,6 +103,42 @@ def test_coarsen_matches_oracle(name, dtype, d, Hkv, T_list, N_list, values, rep
     assert r["status"] == 0, f"device flags {r['flags']}"
     orc = oracle_units(k, v, Hkv, T_list, N_list, seed, representative=representative)
     compare_units(r, orc, k, v, T_list, Hkv, N_list, dtype)
+
+
+DIAG_CASES = [c for c in CASES if c[0] in ("bf16_d128_multi_tile", "bf16_d64", "f32_d64", "short_sequences",
+                                           "tile_edges", "single_segment")]
+
+
+@pytest.mark.parametrize("name,dtype,d,Hkv,T_list,N_list,values", DIAG_CASES, ids=[c[0] for c in DIAG_CASES])
+def test_coarsen_diagonal_closure_matches_oracle(name, dtype, d, Hkv, T_list, N_list, values):
+    """A pool for the diagonal closure: the same boundaries and statistics plus every node's
+    per-dimension key variances (zero for exact tokens)."""
+    seed = sum(T_list) + d + 1
+    w = workloads.Workload(name, seed, B=len(T_list), Hq=Hkv, Hkv=Hkv, d=d, R=1,
+                           dtype="bf16" if dtype == torch.bfloat16 else "f32", T=0, regimes=12)
+    k, v, _ = workloads.make_kv(w, "cuda", T_list=T_list, values=values)
+    r = run_coarsen(k, v, Hkv, T_list, N_list, seed, closure="diagonal")
+    assert r["status"] == 0, f"device flags {r['flags']}"
+    orc = oracle_units(k, v, Hkv, T_list, N_list, seed)
+    compare_units(r, orc, k, v, T_list, Hkv, N_list, dtype)
+
+
+def test_tiny_f32_diagonal_closure_end_to_end():
+    """tiny_f32 coarsened into a diagonal pool and decoded with the diagonal closure, against the
+    oracle's own nodes (fp32 bar)."""
+    w = workloads.WORKLOADS["tiny_f32"]
+    k, v, T_list = workloads.make_kv(w, "cuda")
+    N_list = workloads.segment_counts(w, T_list)
+    r = run_coarsen(k, v, w.Hkv, T_list, N_list, w.seed, closure="diagonal")
+    assert r["status"] == 0
+    orc = oracle_units(k, v, w.Hkv, T_list, N_list, w.seed)
+    compare_units(r, orc, k, v, T_list, w.Hkv, N_list, torch.float32)
+    q = workloads.make_queries(w, "cuda")
+    out, lse = skv.decode_attn(q, w.Hkv, r["pool"], r["table"], r["lens"])
+    ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), [[orc[(0, 0)]]], closure="diagonal")
+    check_decode(out, lse, ref_out, ref_lse, torch.float32, "tiny_f32 diagonal end to end")
+    scal_out, _ = oracle.decode(q.double().cpu().numpy(), [[orc[(0, 0)]]])
+    assert np.abs(ref_out - scal_out).max() > 1e-5      # the two closures differ on this cache
 
 
 def test_weighted_representative_on_flat_and_jump_segments():

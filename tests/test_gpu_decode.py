@@ -15,9 +15,10 @@ from gpu_helpers import check_decode, gpu_units, pool_for_units, write_entries
 pytestmark = pytest.mark.gpu
 
 
-def _synthetic(B, Hq, Hkv, R, d, lens_list, dtype, seed, key_scale=3.0, shuffle=True, spare=0):
+def _synthetic(B, Hq, Hkv, R, d, lens_list, dtype, seed, key_scale=3.0, shuffle=True, spare=0, closure="scalar"):
     g = torch.Generator(device="cpu").manual_seed(seed)
-    pool, table = pool_for_units(lens_list, B, Hkv, d, dtype, shuffle=shuffle, seed=seed, spare_pages=spare)
+    pool, table = pool_for_units(lens_list, B, Hkv, d, dtype, shuffle=shuffle, seed=seed, spare_pages=spare,
+                                 closure=closure)
     for b in range(B):
         for h in range(Hkv):
             E = int(lens_list[b])
@@ -26,18 +27,20 @@ def _synthetic(B, Hq, Hkv, R, d, lens_list, dtype, seed, key_scale=3.0, shuffle=
             mass = torch.randint(1, 200, (E,), generator=g).double()
             alpha = torch.log(mass)
             beta = torch.rand(E, generator=g) * 0.02
-            write_entries(pool, table, b, h, kt, vt, alpha, beta)
+            # per-dimension variances spread over two decades (diagonal pools only)
+            var = torch.rand(E, d, generator=g).pow(3) * 2.0 if closure == "diagonal" else None
+            write_entries(pool, table, b, h, kt, vt, alpha, beta, var)
     lens = torch.tensor([[int(lens_list[b])] * Hkv for b in range(B)], dtype=torch.int32, device="cuda")
     q = (torch.randn(B, R, Hq, d, generator=g)).to(dtype).cuda()
     return pool, table, lens, q
 
 
-def _run(B, Hq, Hkv, R, d, lens_list, dtype, seed, **kw):
-    pool, table, lens, q = _synthetic(B, Hq, Hkv, R, d, lens_list, dtype, seed, **kw)
+def _run(B, Hq, Hkv, R, d, lens_list, dtype, seed, closure="scalar", **kw):
+    pool, table, lens, q = _synthetic(B, Hq, Hkv, R, d, lens_list, dtype, seed, closure=closure, **kw)
     out, lse = skv.decode_attn(q, Hkv, pool, table, lens)
     torch.cuda.synchronize()
     units = gpu_units(pool, table, lens, B, Hkv)
-    ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), units)
+    ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), units, closure=closure)
     check_decode(out, lse, ref_out, ref_lse, dtype, what=f"B{B} Hq{Hq} Hkv{Hkv} R{R} d{d}")
     return out, lse
 
@@ -219,3 +222,19 @@ def test_decode_equal_lengths_wide_table_two_row_passes():
     units = gpu_units(pool, table, lens, B, Hkv)
     ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), units)
     check_decode(out, lse, ref_out, ref_lse, torch.bfloat16, "wide table, two row passes")
+
+
+@pytest.mark.parametrize("B,Hq,Hkv,R,d,lens,dtype", [
+    (32, 28, 4, 1, 128, [1147] * 32, torch.bfloat16),        # the 7B 3.5% shape
+    (3, 28, 4, 1, 128, [1147, 37, 300], torch.bfloat16),
+    (10, 14, 2, 1, 64, [0, 1, 15, 16, 17, 31, 33, 250, 0, 2677], torch.bfloat16),
+    (4, 32, 4, 4, 128, [640, 17, 900, 64], torch.bfloat16),  # 32 query rows per unit
+    (4, 32, 4, 5, 64, [333] * 4, torch.bfloat16),            # two row passes
+    (4, 2, 1, 1, 128, [88, 1, 0, 200], torch.float32),
+    (2, 4, 2, 1, 64, [300, 45], torch.float32),
+])
+def test_decode_diagonal_closure(B, Hq, Hkv, R, d, lens, dtype):
+    """Diagonal-closure pools: logit q.k/sqrt(d) + alpha + sum_i q_i^2 var_i/(2d) against the oracle
+    fed the GPU's stored nodes and variances."""
+    kw = {"key_scale": 1.0} if dtype == torch.float32 else {}
+    _run(B, Hq, Hkv, R, d, lens, dtype, seed=B * 7 + d + R, closure="diagonal", **kw)
