@@ -159,6 +159,59 @@ def coarsen(k: torch.Tensor, v: torch.Tensor, Hkv: int, T_list, N_list, n_sink: 
     return lens
 
 
+def stream_state_bytes(Hkv: int, d: int, N_list, n_sink: int, n_recent: int) -> int:
+    return int(_lib.load().skv_stream_state_bytes(len(N_list), Hkv, d, _i32(N_list), n_sink, n_recent))
+
+
+def stream_capacity(N_list, n_sink: int, n_recent: int) -> int:
+    """Entries a streamed unit may hold at once (its page-table row must cover them)."""
+    return n_sink + max(int(n) for n in N_list) + 1 + n_recent
+
+
+def stream_init(k: torch.Tensor, v: torch.Tensor, Hkv: int, T_list, N_list, n_sink: int, n_recent: int,
+                proj_seed: int, pool: NodePool, page_table: torch.Tensor, lens: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None, state: torch.Tensor | None = None, stream=None):
+    """Coarsen the prompts (as coarsen()) and build the streaming state. Returns (lens, state, workspace);
+    pass all three to stream_append."""
+    B = len(T_list)
+    d = k.shape[-1]
+    if pool.closure != "scalar":
+        raise ValueError("streaming coarsening keeps scalar-closure pools")
+    dev = k.device
+    if lens is None:
+        lens = torch.empty(B, Hkv, dtype=torch.int32, device=dev)
+    ws_bytes = coarsen_workspace_bytes(Hkv, d, T_list, N_list, n_sink, n_recent)
+    if workspace is None:
+        workspace = torch.zeros(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+    st_bytes = stream_state_bytes(Hkv, d, N_list, n_sink, n_recent)
+    if st_bytes == 0:
+        raise SkvError(_lib.SKV_ERR_INVALID_ARG, "skv_stream_state_bytes")
+    if state is None:
+        state = torch.zeros(st_bytes, dtype=torch.uint8, device=dev)
+    ps = pool.struct()
+    st = _lib.load().skv_stream_init(
+        _dev(k, "k"), _dev(v, "v"), _code(k.dtype), B, Hkv, d, _i32(T_list), n_sink, n_recent, _i32(N_list),
+        ctypes.c_uint64(proj_seed), ctypes.byref(ps), _dev(page_table, "page_table"), page_table.shape[2],
+        _dev(lens, "lens"), _dev(workspace, "workspace"), workspace.numel(), _dev(state, "state"), state.numel(),
+        ctypes.c_void_p(_stream_handle(stream)))
+    _lib.check(st, "skv_stream_init")
+    return lens, state, workspace
+
+
+def stream_append(k_new: torch.Tensor, v_new: torch.Tensor, N_list, n_sink: int, n_recent: int, proj_seed: int,
+                  pool: NodePool, page_table: torch.Tensor, lens: torch.Tensor, state: torch.Tensor,
+                  workspace: torch.Tensor, stream=None):
+    """Append one token per unit (k_new, v_new: [B, Hkv, d]) to streamed caches."""
+    B, Hkv, d = k_new.shape
+    ps = pool.struct()
+    st = _lib.load().skv_stream_append(
+        _dev(k_new, "k_new"), _dev(v_new, "v_new"), _code(k_new.dtype), B, Hkv, d, _i32(N_list), n_sink, n_recent,
+        ctypes.c_uint64(proj_seed), ctypes.byref(ps), _dev(page_table, "page_table"), page_table.shape[2],
+        _dev(lens, "lens"), _dev(state, "state"), state.numel(), _dev(workspace, "workspace"), workspace.numel(),
+        ctypes.c_void_p(_stream_handle(stream)))
+    _lib.check(st, "skv_stream_append")
+
+
 def decode_workspace_bytes(B: int, R: int, Hq: int, Hkv: int, d: int, max_pages: int) -> int:
     return int(_lib.load().skv_decode_workspace_bytes(B, R, Hq, Hkv, d, max_pages))
 

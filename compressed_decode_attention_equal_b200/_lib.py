@@ -45,6 +45,7 @@ class SkvError(RuntimeError):
 EXPORTS = ("skv_status_string", "skv_abi_version", "skv_page_bytes", "skv_page_bytes_ex", "skv_projection_matrix",
            "skv_coarsen_workspace_bytes",
            "skv_coarsen", "skv_coarsen_ex", "skv_decode_workspace_bytes", "skv_decode_attn", "skv_decode_attn_ex", "skv_decode_attn_noalloc",
+           "skv_stream_state_bytes", "skv_stream_init", "skv_stream_append",
            "skv_workspace_error")
 
 _lib = None
@@ -88,6 +89,14 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.skv_decode_attn_ex.argtypes = [vp, i32, i32, i32, i32, i32, i32, ctypes.POINTER(SkvNodePool), vp, i32,
                                        vp, vp, vp, vp, sz, ctypes.POINTER(SkvDecodeOptions), vp]
     lib.skv_decode_attn_ex.restype = i32
+    lib.skv_stream_state_bytes.argtypes = [i32, i32, i32, pi32, i32, i32]
+    lib.skv_stream_state_bytes.restype = sz
+    lib.skv_stream_init.argtypes = [vp, vp, i32, i32, i32, i32, pi32, i32, i32, pi32, u64,
+                                    ctypes.POINTER(SkvNodePool), vp, i32, vp, vp, sz, vp, sz, vp]
+    lib.skv_stream_init.restype = i32
+    lib.skv_stream_append.argtypes = [vp, vp, i32, i32, i32, i32, pi32, i32, i32, u64,
+                                      ctypes.POINTER(SkvNodePool), vp, i32, vp, vp, sz, vp, sz, vp]
+    lib.skv_stream_append.restype = i32
     lib.skv_decode_attn_noalloc.argtypes = [vp, i32, i32, i32, i32, i32, i32, ctypes.POINTER(SkvNodePool), vp,
                                             i32, vp, vp, vp, vp]
     lib.skv_decode_attn_noalloc.restype = i32

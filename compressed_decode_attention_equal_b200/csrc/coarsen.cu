@@ -35,19 +35,6 @@ __global__ void k_setup(const __grid_constant__ SeqTable table, SeqRow *dst, int
 // ---------------------------------------------------------------------------
 // k_project_scan
 // ---------------------------------------------------------------------------
-// D = rne(||zc - zp||_2 * 2^20) by the fixed recipe (fp32, i ascending); -1 on overflow.
-__device__ __forceinline__ long long quantised_step(const float *zp, const float *zc) {
-    float s = 0.0f;
-#pragma unroll
-    for (int i = 0; i < kProjDim; ++i) {
-        const float di = __fsub_rn(zc[i], zp[i]);
-        s = __fmaf_rn(di, di, s);
-    }
-    const float dd = __fsqrt_rn(s);
-    const float scaled = __fmul_rn(dd, 1048576.0f);
-    if (!(scaled <= 0x1p40f)) return -1;
-    return __float2ll_rn(scaled);
-}
 
 constexpr int kK1Threads = 128;
 constexpr int kK1Tok = kTileRows / kK1Threads;   // token rows per thread (4)

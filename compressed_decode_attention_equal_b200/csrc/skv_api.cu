@@ -257,6 +257,13 @@ size_t skv_coarsen_workspace_bytes(int B, int Hkv, int d, const int32_t *T_host,
     return p.lay.total;
 }
 
+// The coarsening pipeline; with `streaming` set, it also builds the streaming state (same stream).
+static skv_status coarsen_impl(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d,
+                               const int32_t *T_host, int n_sink, int n_recent, const int32_t *N_host,
+                               uint64_t proj_seed, const skv_node_pool *pool, const int32_t *page_table, int max_pages,
+                               int32_t *lens, int32_t *boundaries, int64_t *cumvar, void *workspace, size_t ws_bytes,
+                               int representative, int closure, StreamArgs *streaming, void *stream);
+
 skv_status skv_coarsen_ex(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d,
                           const int32_t *T_host, int n_sink, int n_recent, const int32_t *N_host, uint64_t proj_seed,
                           const skv_node_pool *pool, const int32_t *page_table, int max_pages, int32_t *lens,
@@ -273,6 +280,16 @@ skv_status skv_coarsen_ex(const void *k, const void *v, skv_dtype dtype, int B, 
         representative = options->representative;
         closure = options->closure;
     }
+    return coarsen_impl(k, v, dtype, B, Hkv, d, T_host, n_sink, n_recent, N_host, proj_seed, pool, page_table,
+                        max_pages, lens, boundaries, cumvar, workspace, ws_bytes, representative, closure, nullptr,
+                        stream);
+}
+
+static skv_status coarsen_impl(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d,
+                               const int32_t *T_host, int n_sink, int n_recent, const int32_t *N_host,
+                               uint64_t proj_seed, const skv_node_pool *pool, const int32_t *page_table, int max_pages,
+                               int32_t *lens, int32_t *boundaries, int64_t *cumvar, void *workspace, size_t ws_bytes,
+                               int representative, int closure, StreamArgs *streaming, void *stream) {
     if (dtype != SKV_BF16 && dtype != SKV_F32) return SKV_ERR_UNSUPPORTED;
     static SeqTable table;   // host staging; guarded by the mutex below
     static std::mutex table_mu;
@@ -324,8 +341,94 @@ skv_status skv_coarsen_ex(const void *k, const void *v, skv_dtype dtype, int B, 
     a.cumvar = cumvar;
     a.representative = representative;
     a.closure = closure;
-    const cudaError_t e = launch_coarsen(a, table, proj, map_k, map_v, static_cast<cudaStream_t>(stream));
+    cudaError_t e = launch_coarsen(a, table, proj, map_k, map_v, static_cast<cudaStream_t>(stream));
+    if (e == cudaSuccess && streaming) {
+        streaming->flags = a.flags;
+        streaming->pages = a.pages;
+        streaming->num_pages = a.num_pages;
+        streaming->page_table = page_table;
+        streaming->max_pages = max_pages;
+        streaming->lens = lens;
+        e = launch_stream_init(a, *streaming, proj, static_cast<cudaStream_t>(stream));
+    }
     return e == cudaSuccess ? SKV_OK : SKV_ERR_CUDA;
+}
+
+// ---------------------------------------------------------------------------
+// streaming coarsening
+// ---------------------------------------------------------------------------
+static bool stream_geometry(int B, int Hkv, int d, const int32_t *N_host, int n_sink, int n_recent, StreamArgs *s) {
+    if (B < 1 || Hkv < 1 || B > SKV_MAX_SEQS || !N_host || n_sink < 0 || n_recent < 1 || (d != 64 && d != 128))
+        return false;
+    int Nmax = 0;
+    for (int b = 0; b < B; ++b) {
+        if (N_host[b] < 1 || N_host[b] > (1 << 20)) return false;
+        Nmax = N_host[b] > Nmax ? N_host[b] : Nmax;
+    }
+    const int64_t ecap = static_cast<int64_t>(n_sink) + Nmax + 1 + n_recent;
+    if (ecap > (1 << 22)) return false;
+    stream_layout(d, static_cast<int>(ecap), n_recent, s);
+    return true;
+}
+
+size_t skv_stream_state_bytes(int B, int Hkv, int d, const int32_t *N_host, int n_sink, int n_recent) {
+    StreamArgs s{};
+    if (!stream_geometry(B, Hkv, d, N_host, n_sink, n_recent, &s)) return 0;
+    return static_cast<size_t>(s.unit_bytes) * B * Hkv;
+}
+
+skv_status skv_stream_init(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d,
+                           const int32_t *T_host, int n_sink, int n_recent, const int32_t *N_host,
+                           uint64_t proj_seed, const skv_node_pool *pool, const int32_t *page_table, int max_pages,
+                           int32_t *lens, void *workspace, size_t ws_bytes, void *state, size_t state_bytes,
+                           void *stream) {
+    if (dtype != SKV_BF16 && dtype != SKV_F32) return SKV_ERR_UNSUPPORTED;
+    StreamArgs s{};
+    if (!T_host || !stream_geometry(B, Hkv, d, N_host, n_sink, n_recent, &s)) return SKV_ERR_INVALID_ARG;
+    for (int b = 0; b < B; ++b)
+        if (T_host[b] <= n_sink + n_recent) return SKV_ERR_UNSUPPORTED;   // streaming needs a middle
+    if (!state || !aligned(state, 256) || state_bytes < static_cast<size_t>(s.unit_bytes) * B * Hkv)
+        return SKV_ERR_WORKSPACE;
+    if (static_cast<int64_t>(max_pages) * kPageNodes < s.Ecap) return SKV_ERR_INVALID_ARG;
+    s.B = B;
+    s.Hkv = Hkv;
+    s.d = d;
+    s.dtype = dtype;
+    s.state = static_cast<uint8_t *>(state);
+    return coarsen_impl(k, v, dtype, B, Hkv, d, T_host, n_sink, n_recent, N_host, proj_seed, pool, page_table,
+                        max_pages, lens, nullptr, nullptr, workspace, ws_bytes, SKV_REP_MEAN, SKV_CLOSURE_SCALAR, &s,
+                        stream);
+}
+
+skv_status skv_stream_append(const void *k_new, const void *v_new, skv_dtype dtype, int B, int Hkv, int d,
+                             const int32_t *N_host, int n_sink, int n_recent, uint64_t proj_seed,
+                             const skv_node_pool *pool, const int32_t *page_table, int max_pages, int32_t *lens,
+                             void *state, size_t state_bytes, void *workspace, size_t ws_bytes, void *stream) {
+    if (dtype != SKV_BF16 && dtype != SKV_F32) return SKV_ERR_UNSUPPORTED;
+    StreamArgs s{};
+    if (!stream_geometry(B, Hkv, d, N_host, n_sink, n_recent, &s)) return SKV_ERR_INVALID_ARG;
+    if (!k_new || !v_new || !pool || !pool->pages || pool->num_pages < 0 || !page_table || !lens)
+        return SKV_ERR_INVALID_ARG;
+    if (!aligned(pool->pages, 16) || static_cast<int64_t>(max_pages) * kPageNodes < s.Ecap) return SKV_ERR_INVALID_ARG;
+    if (!state || !aligned(state, 256) || state_bytes < static_cast<size_t>(s.unit_bytes) * B * Hkv)
+        return SKV_ERR_WORKSPACE;
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < kWsHeader) return SKV_ERR_WORKSPACE;
+    s.k_new = k_new;
+    s.v_new = v_new;
+    s.B = B;
+    s.Hkv = Hkv;
+    s.d = d;
+    s.dtype = dtype;
+    s.pages = static_cast<uint8_t *>(pool->pages);
+    s.num_pages = pool->num_pages;
+    s.page_table = page_table;
+    s.max_pages = max_pages;
+    s.lens = lens;
+    s.state = static_cast<uint8_t *>(state);
+    s.flags = static_cast<uint32_t *>(workspace);
+    ProjT proj;
+    g_proj.get(proj_seed, d, proj);
+    return launch_stream_append(s, proj, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SKV_OK : SKV_ERR_CUDA;
 }
 
 skv_status skv_coarsen(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d, const int32_t *T_host,

@@ -236,6 +236,23 @@ __device__ __forceinline__ void cluster_arrive_relaxed() {
 __device__ __forceinline__ void cluster_wait() { asm volatile("barrier.cluster.wait.aligned;" ::: "memory"); }
 
 // ---------------------------------------------------------------------------
+// the variation step of the equal-variation coarsener (offline and streaming)
+// ---------------------------------------------------------------------------
+// D = rne(||zc - zp||_2 * 2^20) by the fixed recipe (fp32, i ascending); -1 on overflow.
+__device__ __forceinline__ long long quantised_step(const float *zp, const float *zc) {
+    float s = 0.0f;
+#pragma unroll
+    for (int i = 0; i < kProjDim; ++i) {
+        const float di = __fsub_rn(zc[i], zp[i]);
+        s = __fmaf_rn(di, di, s);
+    }
+    const float dd = __fsqrt_rn(s);
+    const float scaled = __fmul_rn(dd, 1048576.0f);
+    if (!(scaled <= 0x1p40f)) return -1;
+    return __float2ll_rn(scaled);
+}
+
+// ---------------------------------------------------------------------------
 // 128-bit products for exact threshold comparisons: a1*b1 >= a2*b2 (all >= 0)
 // ---------------------------------------------------------------------------
 __device__ __forceinline__ bool prod_ge(uint64_t a1, uint64_t b1, uint64_t a2, uint64_t b2) {

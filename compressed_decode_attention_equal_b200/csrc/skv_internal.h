@@ -67,6 +67,42 @@ struct CoarsenLayout {
 };
 
 // Host-side launchers (coarsen.cu).
+// ---------------------------------------------------------------------------
+// streaming coarsening state (per unit, one block of unit_bytes in the caller's state buffer)
+// ---------------------------------------------------------------------------
+struct StreamHdr {
+    long long cT;      // cumulative quantised variation of the middle
+    int n_nodes;       // middle nodes
+    int T;             // tokens so far
+    int ring;          // recent ring position of the oldest recent token
+    int n_ent;         // entries (= lens)
+    int N, S, W;       // segment count, sinks, recent window
+    int pad[7];
+    float z_last[16];  // feature of the last middle token
+};
+static_assert(sizeof(StreamHdr) == 128, "StreamHdr layout");
+
+struct StreamArgs {
+    const void *k_new, *v_new;   // [B][Hkv][d] (append)
+    int B, Hkv, d, dtype;
+    uint8_t *pages;
+    int64_t num_pages;
+    const int32_t *page_table;
+    int max_pages;
+    int32_t *lens;
+    uint8_t *state;
+    int64_t unit_bytes;          // state bytes per unit
+    int NM, Ecap;                // node-order capacity, entry capacity per unit
+    int64_t off_order, off_recent, off_owner, off_m, off_start, off_V, off_M2, off_mk, off_mv;
+    uint32_t *flags;
+};
+
+// Byte layout of one unit's state for entry capacity Ecap and recent window W (offsets 256-aligned).
+void stream_layout(int d, int Ecap, int W, StreamArgs *s);
+
+cudaError_t launch_stream_init(const CoarsenArgs &a, const StreamArgs &s, const ProjT &proj, cudaStream_t st);
+cudaError_t launch_stream_append(const StreamArgs &s, const ProjT &proj, cudaStream_t st);
+
 cudaError_t launch_coarsen(const CoarsenArgs &a, const SeqTable &table, const ProjT &proj,
                            const CUtensorMap &map_k, const CUtensorMap &map_v, cudaStream_t s);
 

@@ -224,6 +224,57 @@ skv_status skv_coarsen_ex(const void *k, const void *v, skv_dtype dtype, int B, 
                           void *workspace, size_t ws_bytes, const skv_coarsen_options *options,
                           void *stream);
 
+/*
+ * Streaming coarsening ("Equal-Variation KV Cache", "Implementation notes":
+ * in streaming inference a segment that exceeds its variation budget is
+ * split at the first threshold crossing and adjacent low-variation segments
+ * are merged; node merges follow the law of total variance, "SPICY-KV"
+ * dependent Claim 10). The page leaves the policy open; this library fixes:
+ *  - skv_stream_init coarsens the prompt exactly as skv_coarsen (plain mean,
+ *    scalar closure) and records per-unit streaming state: each middle node's
+ *    mass m, variation V (sum of its steps D), first token and fp64 mean key,
+ *    mean value and summed squared key deviations M2, in token order; c_T;
+ *    the last middle token's feature; the recent window's pool slots.
+ *  - skv_stream_append appends one token per unit (k_new, v_new: [B][Hkv][d]
+ *    in dtype, device). The oldest recent token y enters the middle: its step
+ *    D_y (the offline fixed fp32 recipe against the previous middle token) is
+ *    added to c_T; if N (V_open + D_y) >= c_T (exact 128-bit comparison; the
+ *    open node is the last middle node) y starts a new node with V = D_y,
+ *    otherwise it joins the open node. While more than N middle nodes exist
+ *    the adjacent pair with the smallest V_j + V_{j+1} merges (leftmost on
+ *    ties): masses and variations add, means and M2 combine by the pairwise
+ *    update. The new token takes y's pool slot as an exact recent entry.
+ *    Node outputs as offline: alpha = ln m (0 for m = 1),
+ *    beta = M2 / (m d) / (2 d); lens is updated.
+ * Entries of a streamed unit are kept in no particular order in its pool
+ * slots [0, lens) (decode attention does not depend on their order): a merge
+ * frees a slot, which the unit's last entry then fills.
+ * Requirements: bf16 or fp32, d in {64, 128}, n_recent >= 1; every sequence
+ * has T_b > n_sink + n_recent at init (a non-empty middle; else
+ * SKV_ERR_UNSUPPORTED); each unit's page table row holds
+ * n_sink + max_b N_b + 1 + n_recent entries (host-checked). skv_stream_append
+ * takes the N_host, n_sink and n_recent given to skv_stream_init (they fix
+ * the state layout).
+ * state: device buffer of skv_stream_state_bytes bytes (caller-owned, written
+ * by skv_stream_init, read and updated by each skv_stream_append; calls that
+ * share a state must be ordered on one stream).
+ * workspace (append): any zero-filled device buffer of >= 256 bytes whose
+ * header holds the device error flags (see skv_workspace_error), e.g. the
+ * coarsen workspace.
+ */
+size_t skv_stream_state_bytes(int B, int Hkv, int d, const int32_t *N_host, int n_sink, int n_recent);
+
+skv_status skv_stream_init(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d,
+                           const int32_t *T_host, int n_sink, int n_recent, const int32_t *N_host,
+                           uint64_t proj_seed, const skv_node_pool *pool, const int32_t *page_table,
+                           int max_pages, int32_t *lens, void *workspace, size_t ws_bytes, void *state,
+                           size_t state_bytes, void *stream);
+
+skv_status skv_stream_append(const void *k_new, const void *v_new, skv_dtype dtype, int B, int Hkv, int d,
+                             const int32_t *N_host, int n_sink, int n_recent, uint64_t proj_seed,
+                             const skv_node_pool *pool, const int32_t *page_table, int max_pages, int32_t *lens,
+                             void *state, size_t state_bytes, void *workspace, size_t ws_bytes, void *stream);
+
 /* Bytes of device workspace skv_decode_attn needs (0 on invalid arguments). */
 size_t skv_decode_workspace_bytes(int B, int R, int Hq, int Hkv, int d, int max_pages);
 
