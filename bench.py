@@ -405,6 +405,51 @@ def diagonal_closure_stage(w, device, layers: int, steps: int = 6000):
             "note": "same workload and call with diagonal-closure pools (per-dimension key variances)"}
 
 
+def stream_stage(w, device, steps: int = 3000, distinct: int = 60):
+    """Streaming coarsening on the decode workload: skv_stream_init on the prompts, then appends of
+    one token per unit replayed from CUDA graphs (rank 0 only). The append is latency-bound (one CTA
+    per unit, a 4,096-FMA projection chain and O(N) merge search per call)."""
+    import torch
+    import compressed_decode_attention_equal_b200 as skv
+    import workloads
+    T_list = workloads.seq_lengths(w)
+    N_list = workloads.segment_counts(w, T_list)
+    cap = skv.stream_capacity(N_list, workloads.N_SINK, workloads.N_RECENT)
+    table, num_pages = workloads.page_assignment(w.B, w.Hkv, [-(-cap // 16)] * w.B, w.shuffle_pages, w.seed)
+    table = table.to(device)
+    k, v, _ = workloads.make_kv(w, device, T_list=T_list)
+    pool = skv.NodePool(num_pages, w.d, w.torch_dtype, device=device)
+    t0 = time.perf_counter()
+    lens, state, ws = skv.stream_init(k, v, w.Hkv, T_list, N_list, workloads.N_SINK, workloads.N_RECENT, w.seed,
+                                      pool, table)
+    torch.cuda.synchronize()
+    init_s = time.perf_counter() - t0
+    del k, v
+    g = torch.Generator(device=device).manual_seed(w.seed + 5)
+    new_k = (torch.randn(distinct, w.B, w.Hkv, w.d, generator=g, device=device)).to(w.torch_dtype)
+    new_v = (torch.randn(distinct, w.B, w.Hkv, w.d, generator=g, device=device)).to(w.torch_dtype)
+
+    def step(i):
+        skv.stream_append(new_k[i % distinct], new_v[i % distinct], N_list, workloads.N_SINK, workloads.N_RECENT,
+                          pool, table, lens, state, ws)
+
+    for i in range(distinct):
+        step(i)
+    torch.cuda.synchronize()
+    ms = time_graphs(step, steps, distinct, False)
+    st, flags = skv.workspace_error(ws)
+    if st != 0:
+        raise RuntimeError(f"streaming append raised device flags {flags}")
+    us = ms / steps * 1e3
+    units = w.B * w.Hkv
+    del pool, state
+    torch.cuda.empty_cache()
+    return {"us_per_append": us, "tokens_per_s": units / (us * 1e-6), "units": units,
+            "init_s_host_clock": init_s,
+            "note": "one token appended to every (sequence, KV head) unit per call, N = "
+                    f"{N_list[0]} nodes per unit, graphs of {distinct} calls"}
+
+
 # ---------------------------------------------------------------------------
 # arms
 # ---------------------------------------------------------------------------
@@ -566,6 +611,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-coarsen", action="store_true")
     ap.add_argument("--no-diagonal", action="store_true", help="skip the diagonal-closure decode timing")
+    ap.add_argument("--no-stream", action="store_true", help="skip the streaming-append timing")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -594,6 +640,8 @@ def main():
             res["coarsen"] = coarsen_stage(device)
         if not args.no_diagonal:
             res["diagonal_closure"] = diagonal_closure_stage(w, device, args.layers)
+        if not args.no_stream:
+            res["streaming_append"] = stream_stage(w, device)
         if not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(w, caches, table)
         print(json.dumps(res), flush=True)

@@ -198,7 +198,7 @@ def stream_init(k: torch.Tensor, v: torch.Tensor, Hkv: int, T_list, N_list, n_si
     return lens, state, workspace
 
 
-def stream_append(k_new: torch.Tensor, v_new: torch.Tensor, N_list, n_sink: int, n_recent: int, proj_seed: int,
+def stream_append(k_new: torch.Tensor, v_new: torch.Tensor, N_list, n_sink: int, n_recent: int,
                   pool: NodePool, page_table: torch.Tensor, lens: torch.Tensor, state: torch.Tensor,
                   workspace: torch.Tensor, stream=None):
     """Append one token per unit (k_new, v_new: [B, Hkv, d]) to streamed caches."""
@@ -206,7 +206,7 @@ def stream_append(k_new: torch.Tensor, v_new: torch.Tensor, N_list, n_sink: int,
     ps = pool.struct()
     st = _lib.load().skv_stream_append(
         _dev(k_new, "k_new"), _dev(v_new, "v_new"), _code(k_new.dtype), B, Hkv, d, _i32(N_list), n_sink, n_recent,
-        ctypes.c_uint64(proj_seed), ctypes.byref(ps), _dev(page_table, "page_table"), page_table.shape[2],
+        ctypes.byref(ps), _dev(page_table, "page_table"), page_table.shape[2],
         _dev(lens, "lens"), _dev(state, "state"), state.numel(), _dev(workspace, "workspace"), workspace.numel(),
         ctypes.c_void_p(_stream_handle(stream)))
     _lib.check(st, "skv_stream_append")

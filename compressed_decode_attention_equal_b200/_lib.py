@@ -94,7 +94,7 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.skv_stream_init.argtypes = [vp, vp, i32, i32, i32, i32, pi32, i32, i32, pi32, u64,
                                     ctypes.POINTER(SkvNodePool), vp, i32, vp, vp, sz, vp, sz, vp]
     lib.skv_stream_init.restype = i32
-    lib.skv_stream_append.argtypes = [vp, vp, i32, i32, i32, i32, pi32, i32, i32, u64,
+    lib.skv_stream_append.argtypes = [vp, vp, i32, i32, i32, i32, pi32, i32, i32,
                                       ctypes.POINTER(SkvNodePool), vp, i32, vp, vp, sz, vp, sz, vp]
     lib.skv_stream_append.restype = i32
     lib.skv_decode_attn_noalloc.argtypes = [vp, i32, i32, i32, i32, i32, i32, ctypes.POINTER(SkvNodePool), vp,

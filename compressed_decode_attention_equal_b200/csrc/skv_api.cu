@@ -366,7 +366,7 @@ static bool stream_geometry(int B, int Hkv, int d, const int32_t *N_host, int n_
         Nmax = N_host[b] > Nmax ? N_host[b] : Nmax;
     }
     const int64_t ecap = static_cast<int64_t>(n_sink) + Nmax + 1 + n_recent;
-    if (ecap > (1 << 22)) return false;
+    if (ecap > 8192) return false;   // the append kernel stages the node order in shared memory
     stream_layout(d, static_cast<int>(ecap), n_recent, s);
     return true;
 }
@@ -374,7 +374,7 @@ static bool stream_geometry(int B, int Hkv, int d, const int32_t *N_host, int n_
 size_t skv_stream_state_bytes(int B, int Hkv, int d, const int32_t *N_host, int n_sink, int n_recent) {
     StreamArgs s{};
     if (!stream_geometry(B, Hkv, d, N_host, n_sink, n_recent, &s)) return 0;
-    return static_cast<size_t>(s.unit_bytes) * B * Hkv;
+    return static_cast<size_t>(kStreamProjBytes + s.unit_bytes * B * Hkv);
 }
 
 skv_status skv_stream_init(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d,
@@ -387,30 +387,33 @@ skv_status skv_stream_init(const void *k, const void *v, skv_dtype dtype, int B,
     if (!T_host || !stream_geometry(B, Hkv, d, N_host, n_sink, n_recent, &s)) return SKV_ERR_INVALID_ARG;
     for (int b = 0; b < B; ++b)
         if (T_host[b] <= n_sink + n_recent) return SKV_ERR_UNSUPPORTED;   // streaming needs a middle
-    if (!state || !aligned(state, 256) || state_bytes < static_cast<size_t>(s.unit_bytes) * B * Hkv)
+    if (!state || !aligned(state, 256) ||
+        state_bytes < static_cast<size_t>(kStreamProjBytes + s.unit_bytes * B * Hkv))
         return SKV_ERR_WORKSPACE;
     if (static_cast<int64_t>(max_pages) * kPageNodes < s.Ecap) return SKV_ERR_INVALID_ARG;
     s.B = B;
     s.Hkv = Hkv;
     s.d = d;
     s.dtype = dtype;
-    s.state = static_cast<uint8_t *>(state);
+    s.pt = static_cast<float *>(state);
+    s.state = static_cast<uint8_t *>(state) + kStreamProjBytes;
     return coarsen_impl(k, v, dtype, B, Hkv, d, T_host, n_sink, n_recent, N_host, proj_seed, pool, page_table,
                         max_pages, lens, nullptr, nullptr, workspace, ws_bytes, SKV_REP_MEAN, SKV_CLOSURE_SCALAR, &s,
                         stream);
 }
 
 skv_status skv_stream_append(const void *k_new, const void *v_new, skv_dtype dtype, int B, int Hkv, int d,
-                             const int32_t *N_host, int n_sink, int n_recent, uint64_t proj_seed,
-                             const skv_node_pool *pool, const int32_t *page_table, int max_pages, int32_t *lens,
-                             void *state, size_t state_bytes, void *workspace, size_t ws_bytes, void *stream) {
+                             const int32_t *N_host, int n_sink, int n_recent, const skv_node_pool *pool,
+                             const int32_t *page_table, int max_pages, int32_t *lens, void *state,
+                             size_t state_bytes, void *workspace, size_t ws_bytes, void *stream) {
     if (dtype != SKV_BF16 && dtype != SKV_F32) return SKV_ERR_UNSUPPORTED;
     StreamArgs s{};
     if (!stream_geometry(B, Hkv, d, N_host, n_sink, n_recent, &s)) return SKV_ERR_INVALID_ARG;
     if (!k_new || !v_new || !pool || !pool->pages || pool->num_pages < 0 || !page_table || !lens)
         return SKV_ERR_INVALID_ARG;
     if (!aligned(pool->pages, 16) || static_cast<int64_t>(max_pages) * kPageNodes < s.Ecap) return SKV_ERR_INVALID_ARG;
-    if (!state || !aligned(state, 256) || state_bytes < static_cast<size_t>(s.unit_bytes) * B * Hkv)
+    if (!state || !aligned(state, 256) ||
+        state_bytes < static_cast<size_t>(kStreamProjBytes + s.unit_bytes * B * Hkv))
         return SKV_ERR_WORKSPACE;
     if (!workspace || !aligned(workspace, 256) || ws_bytes < kWsHeader) return SKV_ERR_WORKSPACE;
     s.k_new = k_new;
@@ -424,11 +427,10 @@ skv_status skv_stream_append(const void *k_new, const void *v_new, skv_dtype dty
     s.page_table = page_table;
     s.max_pages = max_pages;
     s.lens = lens;
-    s.state = static_cast<uint8_t *>(state);
+    s.pt = static_cast<float *>(state);
+    s.state = static_cast<uint8_t *>(state) + kStreamProjBytes;
     s.flags = static_cast<uint32_t *>(workspace);
-    ProjT proj;
-    g_proj.get(proj_seed, d, proj);
-    return launch_stream_append(s, proj, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SKV_OK : SKV_ERR_CUDA;
+    return launch_stream_append(s, static_cast<cudaStream_t>(stream)) == cudaSuccess ? SKV_OK : SKV_ERR_CUDA;
 }
 
 skv_status skv_coarsen(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d, const int32_t *T_host,

@@ -90,7 +90,8 @@ struct StreamArgs {
     const int32_t *page_table;
     int max_pages;
     int32_t *lens;
-    uint8_t *state;
+    uint8_t *state;              // the units' blocks (after the projection block)
+    float *pt;                   // P^T [2d][16] kept in the state buffer's first block
     int64_t unit_bytes;          // state bytes per unit
     int NM, Ecap;                // node-order capacity, entry capacity per unit
     int64_t off_order, off_recent, off_owner, off_m, off_start, off_V, off_M2, off_mk, off_mv;
@@ -101,7 +102,10 @@ struct StreamArgs {
 void stream_layout(int d, int Ecap, int W, StreamArgs *s);
 
 cudaError_t launch_stream_init(const CoarsenArgs &a, const StreamArgs &s, const ProjT &proj, cudaStream_t st);
-cudaError_t launch_stream_append(const StreamArgs &s, const ProjT &proj, cudaStream_t st);
+cudaError_t launch_stream_append(const StreamArgs &s, cudaStream_t st);
+
+// bytes at the start of a streaming state buffer that hold P^T (then the units' blocks)
+constexpr int64_t kStreamProjBytes = 2 * 128 * SKV_PROJ_DIM * 4;
 
 cudaError_t launch_coarsen(const CoarsenArgs &a, const SeqTable &table, const ProjT &proj,
                            const CUtensorMap &map_k, const CUtensorMap &map_v, cudaStream_t s);

@@ -23,6 +23,7 @@
 namespace skv {
 
 constexpr int kStreamThreads = 128;
+constexpr int kStreamMaxNodes = 8192;   // node-order capacity the append kernel stages in shared memory
 
 template <typename T>
 struct Elem;
@@ -123,11 +124,14 @@ __device__ void write_node(const StreamArgs &s, const UnitState<D, T> &st, int u
     }
 }
 
-// z = P [k; v] by the fixed recipe (z_i an fp32 fma chain over j ascending from 0); thread i < 16
-__device__ __forceinline__ float feature_i(const ProjT &proj, const float *kx, const float *vx, int D, int i) {
+// z = P [k; v] by the fixed recipe (z_i an fp32 fma chain over j ascending from 0); thread i < 16.
+// pt: P^T (pt[j * 16 + i] = P[i][j]) in shared or parameter memory.
+__device__ __forceinline__ float feature_i(const float *pt, const float *kx, const float *vx, int D, int i) {
     float z = 0.0f;
-    for (int j = 0; j < D; ++j) z = __fmaf_rn(proj.pt[j * kProjDim + i], kx[j], z);
-    for (int j = 0; j < D; ++j) z = __fmaf_rn(proj.pt[(D + j) * kProjDim + i], vx[j], z);
+#pragma unroll 8
+    for (int j = 0; j < D; ++j) z = __fmaf_rn(pt[j * kProjDim + i], kx[j], z);
+#pragma unroll 8
+    for (int j = 0; j < D; ++j) z = __fmaf_rn(pt[(D + j) * kProjDim + i], vx[j], z);
     return z;
 }
 
@@ -197,6 +201,9 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_init(const CoarsenArg
             st.M2[e] = M2;
         }
     }
+    // the projection, kept for the appends (small kernel parameters keep their launches cheap)
+    if (u == 0)
+        for (int i = tid; i < 2 * D * kProjDim; i += kStreamThreads) s.pt[i] = proj.pt[i];
     // feature of the last middle token
     const int last = sr.s_eff + sr.M - 1;
     for (int dim = tid; dim < D; dim += kStreamThreads) {
@@ -204,7 +211,7 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_init(const CoarsenArg
         xv[dim] = static_cast<float>(vraw[static_cast<int64_t>(last) * D + dim]);
     }
     __syncthreads();
-    if (tid < kProjDim) st.hdr->z_last[tid] = feature_i(proj, xk, xv, D, tid);
+    if (tid < kProjDim) st.hdr->z_last[tid] = feature_i(proj.pt, xk, xv, D, tid);
     if (tid == 0) {
         st.hdr->cT = a.unit_total[u];
         st.hdr->n_nodes = n_mid;
@@ -220,8 +227,18 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_init(const CoarsenArg
 // ---------------------------------------------------------------------------
 // k_stream_append: one token per unit
 // ---------------------------------------------------------------------------
+// dynamic shared memory of the append kernel: P^T, the node order and the nodes' variations
+template <int D>
+__host__ __device__ constexpr size_t append_smem(int NM) {
+    return static_cast<size_t>(2 * D * kProjDim) * 4 + static_cast<size_t>(NM) * 8 + static_cast<size_t>(NM) * 4;
+}
+
 template <int D, typename T>
-__global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamArgs s, const __grid_constant__ ProjT proj) {
+__global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamArgs s) {
+    extern __shared__ __align__(16) uint8_t dsm[];
+    float *sP = reinterpret_cast<float *>(dsm);                               // [2D][16]
+    long long *sV = reinterpret_cast<long long *>(dsm + 2 * D * kProjDim * 4);  // [NM] V in node order
+    int *sOrder = reinterpret_cast<int *>(sV + s.NM);                          // [NM] node order
     __shared__ float ky[D], vy[D];
     __shared__ float zy[kProjDim];
     __shared__ double red_d[kStreamThreads / 32];
@@ -239,6 +256,7 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
     const int ring = H.ring;
 
     // 1. the oldest recent token y leaves the window: read it from its pool slot
+    for (int i = tid; i < 2 * D * kProjDim; i += kStreamThreads) sP[i] = s.pt[i];
     const int yslot = st.recent[ring];
     const uint8_t *ypg = entry_page<D, T>(s, u, yslot);
     if (tid == 0) sh_ok = ypg != nullptr && n_nodes >= 1;
@@ -250,7 +268,7 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
     }
     __syncthreads();
     // 2. its variation step, then first hitting on the open node's budget
-    if (tid < kProjDim) zy[tid] = feature_i(proj, ky, vy, D, tid);
+    if (tid < kProjDim) zy[tid] = feature_i(sP, ky, vy, D, tid);
     __syncthreads();
     if (tid == 0) {
         long long Dy = quantised_step(H.z_last, zy);
@@ -316,11 +334,18 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
     // 3. above N nodes: merge the adjacent pair with the smallest combined variation
     int merged = -1, moved = -1;
     if (n_nodes > N) {
+        // the node order and variations to shared memory (all loads in flight at once)
+        for (int j = tid; j < n_nodes; j += kStreamThreads) {
+            const int o = st.order[j];
+            sOrder[j] = o;
+            sV[j] = st.V[o];
+        }
+        __syncthreads();
         // the smallest V_j + V_{j+1} (all >= 0), then the smallest j attaining it
         long long best = LLONG_MAX;
         int bj = INT_MAX;
         for (int j = tid; j < n_nodes - 1; j += kStreamThreads) {
-            const long long v2 = st.V[st.order[j]] + st.V[st.order[j + 1]];
+            const long long v2 = sV[j] + sV[j + 1];
             if (v2 < best) {   // j ascending per thread: keeps the leftmost of equal sums
                 best = v2;
                 bj = j;
@@ -336,7 +361,7 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
         if (static_cast<unsigned long long>(best) == sh_bmin) atomicMin(&sh_merge_j, bj);
         __syncthreads();
         const int j = sh_merge_j;
-        const int ea = st.order[j], eb = st.order[j + 1];
+        const int ea = sOrder[j], eb = sOrder[j + 1];
         // pairwise update: a <- a + b
         const int ma = st.m[ea], mb = st.m[eb];
         const double wb = static_cast<double>(mb) / (ma + mb);
@@ -355,14 +380,9 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
             st.m[ea] = ma + mb;
             st.V[ea] += st.V[eb];
         }
-        // drop position j + 1 from the node order (chunks of one block: reads stay ahead of writes)
-        for (int base = j + 1; base < n_nodes - 1; base += kStreamThreads) {
-            const int t = base + tid;
-            const int val = t < n_nodes - 1 ? st.order[t + 1] : 0;
-            __syncthreads();
-            if (t < n_nodes - 1) st.order[t] = val;
-            __syncthreads();
-        }
+        // drop position j + 1 from the node order (from the shared copy)
+        for (int t = j + 1 + tid; t < n_nodes - 1; t += kStreamThreads) st.order[t] = sOrder[t + 1];
+        __syncthreads();
         --n_nodes;
         merged = ea;
         // the freed slot eb takes the unit's last entry
@@ -401,8 +421,9 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
                     sh_pos = -1;
                 }
                 __syncthreads();
-                for (int p = tid; p < n_nodes; p += kStreamThreads)
-                    if (st.order[p] == last) sh_pos = p;
+                // its position in the order before the shift (sOrder), then after it
+                for (int p = tid; p < n_nodes + 1; p += kStreamThreads)
+                    if (sOrder[p] == last) sh_pos = p > j + 1 ? p - 1 : p;
                 __syncthreads();
                 if (tid == 0 && sh_pos >= 0) st.order[sh_pos] = eb;
                 if (merged == last) merged = eb;
@@ -483,16 +504,23 @@ cudaError_t launch_stream_init(const CoarsenArgs &a, const StreamArgs &s, const 
     return cudaGetLastError();
 }
 
-cudaError_t launch_stream_append(const StreamArgs &s, const ProjT &proj, cudaStream_t st) {
-    const int units = s.B * s.Hkv;
-    if (s.dtype == SKV_BF16) {
-        if (s.d == 128) k_stream_append<128, __nv_bfloat16><<<units, kStreamThreads, 0, st>>>(s, proj);
-        else k_stream_append<64, __nv_bfloat16><<<units, kStreamThreads, 0, st>>>(s, proj);
-    } else {
-        if (s.d == 128) k_stream_append<128, float><<<units, kStreamThreads, 0, st>>>(s, proj);
-        else k_stream_append<64, float><<<units, kStreamThreads, 0, st>>>(s, proj);
+template <int D, typename T>
+static cudaError_t append_typed(const StreamArgs &s, cudaStream_t st) {
+    const size_t smem = append_smem<D>(s.NM);
+    if (smem > 48 * 1024) {
+        const cudaError_t e = cudaFuncSetAttribute(k_stream_append<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   static_cast<int>(append_smem<D>(kStreamMaxNodes)));
+        if (e != cudaSuccess) return e;
     }
+    k_stream_append<D, T><<<s.B * s.Hkv, kStreamThreads, smem, st>>>(s);
     return cudaGetLastError();
+}
+
+cudaError_t launch_stream_append(const StreamArgs &s, cudaStream_t st) {
+    if (s.NM > kStreamMaxNodes) return cudaErrorInvalidValue;
+    if (s.dtype == SKV_BF16)
+        return s.d == 128 ? append_typed<128, __nv_bfloat16>(s, st) : append_typed<64, __nv_bfloat16>(s, st);
+    return s.d == 128 ? append_typed<128, float>(s, st) : append_typed<64, float>(s, st);
 }
 
 }  // namespace skv

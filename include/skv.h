@@ -252,12 +252,14 @@ skv_status skv_coarsen_ex(const void *k, const void *v, skv_dtype dtype, int B, 
  * Requirements: bf16 or fp32, d in {64, 128}, n_recent >= 1; every sequence
  * has T_b > n_sink + n_recent at init (a non-empty middle; else
  * SKV_ERR_UNSUPPORTED); each unit's page table row holds
- * n_sink + max_b N_b + 1 + n_recent entries (host-checked). skv_stream_append
+ * n_sink + max_b N_b + 1 + n_recent <= 8192 entries (host-checked; larger
+ * capacities return SKV_ERR_INVALID_ARG). skv_stream_append
  * takes the N_host, n_sink and n_recent given to skv_stream_init (they fix
  * the state layout).
  * state: device buffer of skv_stream_state_bytes bytes (caller-owned, written
- * by skv_stream_init, read and updated by each skv_stream_append; calls that
- * share a state must be ordered on one stream).
+ * by skv_stream_init -- including the projection P drawn from proj_seed,
+ * which the appends reuse -- and read and updated by each skv_stream_append;
+ * calls that share a state must be ordered on one stream).
  * workspace (append): any zero-filled device buffer of >= 256 bytes whose
  * header holds the device error flags (see skv_workspace_error), e.g. the
  * coarsen workspace.
@@ -271,9 +273,9 @@ skv_status skv_stream_init(const void *k, const void *v, skv_dtype dtype, int B,
                            size_t state_bytes, void *stream);
 
 skv_status skv_stream_append(const void *k_new, const void *v_new, skv_dtype dtype, int B, int Hkv, int d,
-                             const int32_t *N_host, int n_sink, int n_recent, uint64_t proj_seed,
-                             const skv_node_pool *pool, const int32_t *page_table, int max_pages, int32_t *lens,
-                             void *state, size_t state_bytes, void *workspace, size_t ws_bytes, void *stream);
+                             const int32_t *N_host, int n_sink, int n_recent, const skv_node_pool *pool,
+                             const int32_t *page_table, int max_pages, int32_t *lens, void *state,
+                             size_t state_bytes, void *workspace, size_t ws_bytes, void *stream);
 
 /* Bytes of device workspace skv_decode_attn needs (0 on invalid arguments). */
 size_t skv_decode_workspace_bytes(int B, int R, int Hq, int Hkv, int d, int max_pages);

@@ -134,6 +134,34 @@ def test_page_bytes_and_closure_options(lib):
     assert lib.skv_coarsen_ex(*cargs, ctypes.byref(_lib.SkvCoarsenOptions(1, 1)), null) == _lib.SKV_ERR_WORKSPACE
 
 
+def test_stream_queries_and_validation(lib):
+    from compressed_decode_attention_equal_b200 import _lib
+    null = ctypes.c_void_p(0)
+    N = (ctypes.c_int32 * 2)(20, 31)
+    # projection block + 2 x 2 unit blocks; zero for invalid geometry
+    one = lib.skv_stream_state_bytes(2, 2, 128, N, 8, 48)
+    assert one > 16384 and (one - 16384) % 4 == 0 and (one - 16384) % 256 == 0
+    assert lib.skv_stream_state_bytes(2, 2, 96, N, 8, 48) == 0
+    assert lib.skv_stream_state_bytes(2, 2, 128, N, 8, 0) == 0           # needs a recent window
+    big = (ctypes.c_int32 * 2)(9000, 1)
+    assert lib.skv_stream_state_bytes(2, 2, 128, big, 8, 48) == 0        # above the node capacity
+    T = (ctypes.c_int32 * 2)(56, 900)                                     # sequence 0 has no middle
+    pool = _lib.SkvNodePool(16, 1)
+    st = lib.skv_stream_init(ctypes.c_void_p(256), ctypes.c_void_p(256), 1, 2, 2, 128, T, 8, 48, N, 0,
+                             ctypes.byref(pool), ctypes.c_void_p(16), 80, ctypes.c_void_p(16), ctypes.c_void_p(256),
+                             1 << 20, ctypes.c_void_p(256), one, null)
+    assert st == _lib.SKV_ERR_UNSUPPORTED
+    # append: a state smaller than the query, a workspace without the flag header, too few pages
+    args = (ctypes.c_void_p(256), ctypes.c_void_p(256), 1, 2, 2, 128, N, 8, 48, ctypes.byref(pool),
+            ctypes.c_void_p(16))
+    assert lib.skv_stream_append(*args, 80, ctypes.c_void_p(16), ctypes.c_void_p(256), one - 256,
+                                 ctypes.c_void_p(256), 256, null) == _lib.SKV_ERR_WORKSPACE
+    assert lib.skv_stream_append(*args, 80, ctypes.c_void_p(16), ctypes.c_void_p(256), one,
+                                 ctypes.c_void_p(256), 16, null) == _lib.SKV_ERR_WORKSPACE
+    assert lib.skv_stream_append(*args, 4, ctypes.c_void_p(16), ctypes.c_void_p(256), one,
+                                 ctypes.c_void_p(256), 256, null) == _lib.SKV_ERR_INVALID_ARG
+
+
 def test_binding_fails_loudly_without_library(tmp_path):
     from compressed_decode_attention_equal_b200 import _lib
     saved = _lib._lib

@@ -17,6 +17,7 @@ from oracle.stream import StreamUnit
 pytestmark = pytest.mark.gpu
 
 S, W = workloads.N_SINK, workloads.N_RECENT
+PROJ_BYTES = 2 * 128 * 16 * 4   # the state buffer starts with the projection P^T
 
 
 def _layout(d, Ecap, W_):
@@ -47,7 +48,7 @@ def _walk_units(B, Hkv, T_full, d, seed):
 
 def _gpu_entries(state, st_lay, unit, pool, table, lens, d):
     """{token: (m, V, kt, vt, alpha, beta)} of one unit, read back from the pool and the state."""
-    base = unit * st_lay["unit"]
+    base = PROJ_BYTES + unit * st_lay["unit"]
     raw = state[base:base + st_lay["unit"]].cpu().numpy()
     hdr = raw[:128]
     cT = int(hdr[0:8].view(np.int64)[0])
@@ -117,7 +118,7 @@ def test_stream_matches_oracle(d, N_list, T0, steps):
     pool.ab.fill_(float("nan"))
     lens, state, ws = skv.stream_init(k0, v0, Hkv, T0, N_list, S, W, seed, pool, table)
     st_lay = _layout(d, cap, W)
-    assert st_lay["unit"] * B * Hkv == state.numel()
+    assert PROJ_BYTES + st_lay["unit"] * B * Hkv == state.numel()
     P = oracle.projection(seed, d)
     ous = {(b, h): StreamUnit(units[(b, h)][0][:T0[b]].float().numpy(), units[(b, h)][1][:T0[b]].float().numpy(),
                               S, W, N_list[b], P) for b in range(B) for h in range(Hkv)}
@@ -131,7 +132,7 @@ def test_stream_matches_oracle(d, N_list, T0, steps):
             break
         k_new = torch.stack([torch.stack([units[(b, h)][0][T0[b] + step] for h in range(Hkv)]) for b in range(B)])
         v_new = torch.stack([torch.stack([units[(b, h)][1][T0[b] + step] for h in range(Hkv)]) for b in range(B)])
-        skv.stream_append(k_new.cuda(), v_new.cuda(), N_list, S, W, seed, pool, table, lens, state, ws)
+        skv.stream_append(k_new.cuda(), v_new.cuda(), N_list, S, W, pool, table, lens, state, ws)
         for (b, h), ou in ous.items():
             ou.append(units[(b, h)][0][T0[b] + step].float().numpy(), units[(b, h)][1][T0[b] + step].float().numpy())
     st, flags = skv.workspace_error(ws)
