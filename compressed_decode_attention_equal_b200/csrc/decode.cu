@@ -62,11 +62,15 @@ template <int D, int NT, bool DIAG = false>
 struct SplitSmem {
     static constexpr int QROWB = D * 2 + 16;              // padded query row: conflict-free ldmatrix
     static constexpr int QBUF = NT * 8 * QROWB;           // the query rows of one piece
-    // ring depth: pages 1.5x larger with the variances, so a shallower ring keeps 3 CTAs per SM
-    static constexpr int STAGES = DIAG ? 4 : kDecStages;
+    // with the variances a page carries 1.5x the bytes and 3x the MMAs before PV: one CTA per SM
+    // with 8 consumer warps and 8 stages takes a whole unit (measured 27.5 us against 32.2 us for
+    // 4 warps, 4 stages and 3 CTAs per SM on the 7B 3.5% shape)
+    static constexpr int CONS = DIAG ? 8 : kDecConsumers;   // consumer warps
+    static constexpr int THREADS = (CONS + 1) * 32;
+    static constexpr int STAGES = DIAG ? 8 : kDecStages;
     static constexpr int STAGES_BYTES = STAGES * PageGeom<D, DIAG>::STAGE;
     static constexpr int MST = D + 4;                     // mbuf row stride: 16-byte rows
-    static constexpr int MBUF_FLOATS = kDecConsumers * 8 * MST;
+    static constexpr int MBUF_FLOATS = CONS * 8 * MST;
     static constexpr int BARS = 2 * STAGES + 4;
     static constexpr int ROWS = NT * 8;                   // query rows of one piece
     static constexpr int WST = 9;                         // merge weights per row (<= 8) + log2 partition
@@ -98,9 +102,10 @@ __device__ __forceinline__ int find_vunit(const int *prefix, int nv, long long f
 
 // Every CTA rebuilds the page prefix over virtual units (lens are tiny and L2-resident). Run by
 // the consumer warps alone (named barrier 1), so the producer can start copies meanwhile.
+template <int NCONS>
 __device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, int *scratch) {
     const int nv = a.n_vunits;
-    const int tid = threadIdx.x, nth = kDecConsumers * 32;
+    const int tid = threadIdx.x, nth = NCONS * 32;
     const int per = (nv + nth - 1) / nth;
     const int lo = min(tid * per, nv), hi = min(lo + per, nv);
     int local = 0;
@@ -117,7 +122,7 @@ __device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, i
         if (lane >= off) x += n;
     }
     if (lane == 31) scratch[warp] = x;
-    asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
+    asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
     int wp = 0;
     for (int w = 0; w < warp; ++w) wp += scratch[w];
     int run = wp + x - local;
@@ -127,7 +132,7 @@ __device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, i
         run += pages;
     }
     if (tid == nth - 1) prefix[nv] = wp + x;
-    asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
+    asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
 }
 
 // First flat page of CTA c's range, and the CTA whose (nonempty) range holds page f.
@@ -173,18 +178,18 @@ __device__ __forceinline__ void merge_store(const DecodeArgs &a, int b, int h, i
     if (lane == 0) a.lse[oi] = Ls > 0.0f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
 }
 
-template <int D>
+template <int D, int NCONS>
 __device__ void merge_unit(const DecodeArgs &a, int v, const int *codes, int n, int warp, int lane) {
     constexpr int DPL = D / 32;   // dimensions per lane
     const int u = v / a.row_passes, rpass = v % a.row_passes;
     const int b = u / a.Hkv, h = u % a.Hkv;
     const int rows_here = min(a.pass_rows, a.rows - rpass * kRowsPerPass);
     if (n <= kFastPieces) {
-        for (int r0 = warp; r0 < rows_here; r0 += 2 * kDecConsumers) {
+        for (int r0 = warp; r0 < rows_here; r0 += 2 * NCONS) {
             float lv[2][kFastPieces], xv[2][kFastPieces][DPL];
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
-                const int rr = r0 + t * kDecConsumers;
+                const int rr = r0 + t * NCONS;
 #pragma unroll
                 for (int i = 0; i < kFastPieces; ++i) {
                     lv[t][i] = -INFINITY;
@@ -206,7 +211,7 @@ __device__ void merge_unit(const DecodeArgs &a, int v, const int *codes, int n, 
             }
 #pragma unroll
             for (int t = 0; t < 2; ++t) {
-                const int rr = r0 + t * kDecConsumers;
+                const int rr = r0 + t * NCONS;
                 if (rr >= rows_here) continue;
                 float M = -INFINITY;
 #pragma unroll
@@ -227,7 +232,7 @@ __device__ void merge_unit(const DecodeArgs &a, int v, const int *codes, int n, 
         }
         return;
     }
-    for (int rr = warp; rr < rows_here; rr += kDecConsumers) {
+    for (int rr = warp; rr < rows_here; rr += NCONS) {
         float M = -INFINITY;
         for (int base = 0; base < n; base += 32) {
             const int i = base + lane;
@@ -270,10 +275,12 @@ __device__ void merge_unit(const DecodeArgs &a, int v, const int *codes, int n, 
 }
 
 template <int D, int NT, bool DIAG>
-__global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(const DecodeArgs a) {
+__global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, DIAG ? 1 : 2) k_decode_split(const DecodeArgs a) {
     using G = PageGeom<D, DIAG>;
     using L = SplitSmem<D, NT, DIAG>;
-    constexpr int PG = kDecConsumers / NT;   // page groups: warps sharing a row tile split the pages
+    constexpr int NCONS = L::CONS;           // consumer warps (the producer is warp NCONS)
+    constexpr int NTHR = L::THREADS;
+    constexpr int PG = NCONS / NT;   // page groups: warps sharing a row tile split the pages
     constexpr int NKS = D / 16;              // QK k-steps over dims == PV m-tiles over dims
     constexpr int NS = L::STAGES;            // ring depth
     static_assert(NS % PG == 0, "a stage's successive pages must go to one consumer warp");
@@ -293,7 +300,7 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
     long long *orow = reinterpret_cast<long long *>(misc + 16);
     float *wrow = reinterpret_cast<float *>(orow + L::ROWS);
     int *prefix = reinterpret_cast<int *>(reinterpret_cast<uint8_t *>(misc + 16) + ((L::EPI_BYTES + 15) / 16) * 16);
-    __shared__ int scan_scratch[kDecThreads / 32];
+    __shared__ int scan_scratch[NTHR / 32];
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int nv = a.n_vunits;
@@ -308,11 +315,11 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&qfull[s], 1);
-            mbar_init(&qempty[s], kDecConsumers);
+            mbar_init(&qempty[s], NCONS);
         }
         fence_mbar_init();
     }
-    for (int i = tid; i < 2 * L::QBUF / 4; i += kDecThreads) reinterpret_cast<uint32_t *>(qbuf)[i] = 0u;
+    for (int i = tid; i < 2 * L::QBUF / 4; i += NTHR) reinterpret_cast<uint32_t *>(qbuf)[i] = 0u;
     fence_proxy_async_smem();   // the zeros land before the query-row copies
     // Speculation, set up before the inputs may be read. The aligned split below, if every unit
     // fills its page-table row (P0 = max_pages), gives this CTA the table columns [c0, c1) of
@@ -322,7 +329,10 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
     // the general split runs (a wrong guess costs up to NS page reads).
     const int kcl = a.cluster;
     const int crank = blockIdx.x % kcl, vc = blockIdx.x / kcl;   // clusters are consecutive blocks
-    const bool try_spec = kcl > 1 && vc < nv && a.max_pages >= kcl && static_cast<long long>(nv) * kcl <= a.ncta;
+    // (a cluster of one CTA per unit counts as aligned when it keeps 3/4 of the grid busy: every CTA
+    // then owns a whole unit and nothing is merged)
+    const bool try_spec = (kcl > 1 || 4LL * nv >= 3LL * a.ncta) && vc < nv && a.max_pages >= kcl &&
+                          static_cast<long long>(nv) * kcl <= a.ncta;
     const int c0 = try_spec ? a.max_pages * crank / kcl : 0;   // max_pages * 8 fits in an int
     const int c1 = try_spec ? a.max_pages * (crank + 1) / kcl : 0;
     const int n_first = min(NS, c1 - c0);
@@ -334,7 +344,7 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
     int spec_page = -1;      // producer lane j: page id of column c0 + j
     uint32_t spec_bad = 0;   // producer: first pages whose id lies outside the pool
-    if (warp == kDecConsumers) {
+    if (warp == NCONS) {
         if (try_spec) {
             const int u = vc / a.row_passes, rpass = vc % a.row_passes;
             if (lane < c1 - c0)
@@ -366,9 +376,9 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
             }
         }
         cluster_wait();   // pairs with the arrival above (the producer touches no remote memory)
-        asm volatile("bar.sync 2, %0;" ::"n"(kDecThreads));   // the consumers' verdict and prefix
+        asm volatile("bar.sync 2, %0;" ::"n"(NTHR));   // the consumers' verdict and prefix
     } else {
-        build_prefix(a, prefix, scan_scratch);
+        build_prefix<NCONS>(a, prefix, scan_scratch);
         // Aligned split: when every unit has the same page count P0 and `cluster` CTAs per unit
         // fit in the grid, the k = cluster CTAs of a thread-block cluster take equal page ranges of
         // one unit and merge through distributed shared memory (no global partials, one piece per
@@ -376,26 +386,27 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
         const int P0 = prefix[1] - prefix[0];
         bool uni = true;
         {
-            const int per = (nv + kDecConsumers * 32 - 1) / (kDecConsumers * 32);
+            const int per = (nv + NCONS * 32 - 1) / (NCONS * 32);
             for (int v = min(tid * per, nv); v < min(tid * per + per, nv); ++v)
                 uni &= (prefix[v + 1] - prefix[v] == P0);
         }
-        uni = bar_and(1, kDecConsumers * 32, uni);
+        uni = bar_and(1, NCONS * 32, uni);
         if (tid == 0) {
-            const bool al = uni && kcl > 1 && P0 >= kcl && static_cast<long long>(nv) * kcl <= a.ncta;
+            const bool al = uni && (kcl > 1 || 4LL * nv >= 3LL * a.ncta) && P0 >= kcl &&
+                            static_cast<long long>(nv) * kcl <= a.ncta;
             misc[8] = al ? 1 : 0;
             misc[9] = (al && try_spec && P0 == a.max_pages) ? 1 : 0;
         }
         cluster_wait();   // every CTA of the cluster has started
-        asm volatile("bar.arrive 2, %0;" ::"n"(kDecThreads));
-        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));   // misc visible to every consumer
+        asm volatile("bar.arrive 2, %0;" ::"n"(NTHR));
+        asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));   // misc visible to every consumer
     }
     const bool aligned = misc[8] != 0;
     const bool spec_ok = misc[9] != 0;
     bool alive = true;
     if (try_spec && !spec_ok) {
         // wrong guess: wait for the speculative copies, then re-arm every barrier
-        if (warp == kDecConsumers) {
+        if (warp == NCONS) {
             bool ok = true;
             for (int k = 0; k < n_first; ++k) ok &= mbar_wait(&full[k], 0);
             ok &= mbar_wait(&qfull[0], 0);
@@ -415,7 +426,7 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
                 mbar_inval(&qfull[s2]);
                 mbar_inval(&qempty[s2]);
                 mbar_init(&qfull[s2], 1);
-                mbar_init(&qempty[s2], kDecConsumers);
+                mbar_init(&qempty[s2], NCONS);
             }
             fence_mbar_init();
         }
@@ -432,13 +443,13 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
         rb = ptot * (blockIdx.x + 1) / a.ncta;
     }
     __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(a.out);
-    if (warp < kDecConsumers) {
+    if (warp < NCONS) {
         // units with no entries get out = 0, lse = -inf (spread over the CTAs)
         for (int v = blockIdx.x; v < nv; v += a.ncta) {
             if (prefix[v + 1] != prefix[v]) continue;
             const int u = v / a.row_passes, rpass = v % a.row_passes;
             const int b = u / a.Hkv, h = u % a.Hkv;
-            for (int idx = tid; idx < a.pass_rows * D; idx += kDecConsumers * 32) {
+            for (int idx = tid; idx < a.pass_rows * D; idx += NCONS * 32) {
                 const int rr = idx / D, dim = idx % D;
                 const int row = rpass * kRowsPerPass + rr;
                 if (row >= a.rows) continue;
@@ -452,7 +463,7 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
     const int v0 = aligned ? vc : find_vunit(prefix, nv, ra);
     const int n_my = static_cast<int>(rb - ra);
 
-    if (warp == kDecConsumers) {
+    if (warp == NCONS) {
         // ----------------------------- producer -----------------------------
         // a confirmed guess has issued piece 0's query rows and pages [0, n_first) already
         int v = spec_ok ? vc : -1, pi = spec_ok ? 0 : -1;   // current (nonempty) piece
@@ -515,7 +526,7 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
                 __syncwarp();
             }
         }
-        if (aligned) cluster_sync();   // the producer joins the consumers' cluster barrier
+        if (aligned && kcl > 1) cluster_sync();   // the producer joins the consumers' cluster barrier
         return;
     }
 
@@ -728,7 +739,7 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
             mw[(2 * c + 1) * MST + D] = m_run[1];
             mw[(2 * c + 1) * MST + D + 1] = l_run[1];
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
+        asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
         const bool complete = (ps >= ra) && (pe <= rb);
         const int slot = ps < ra ? 0 : 1;
         // per query row: normalised page-group weights, log2 partition and output row
@@ -750,8 +761,8 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
             for (int q2 = 0; q2 < PG; ++q2) wrow[rr * WST + q2] = wq[q2] * inv;
             wrow[rr * WST + 8] = Ls > 0.0f ? M + __log2f(Ls) : -INFINITY;
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
-        for (int it = ctid; it < rows_here * (D / 4); it += kDecConsumers * 32) {
+        asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
+        for (int it = ctid; it < rows_here * (D / 4); it += NCONS * 32) {
             const int rr = it / (D / 4), d4 = (it % (D / 4)) * 4;
             const int ntr = rr >> 3, j = rr & 7;
             float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
@@ -794,10 +805,10 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
             split_pe[n_split] = static_cast<int>(pe);
             ++n_split;
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));   // mbuf free for the next piece
+        asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));   // mbuf free for the next piece
     }
 
-    if (aligned) {
+    if (aligned && kcl > 1) {
         // ---- cluster merge: rank 0 combines every rank's (out, log2 partition) of the unit ----
         cluster_sync();   // release / acquire: the other ranks' stores into xbuf are visible
         if (crank != 0) return;
@@ -821,8 +832,8 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
             for (int r = 0; r < kcl; ++r) wrow[rr * WST + r] *= inv;
             wrow[rr * WST + 8] = Ls > 0.0f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
-        for (int it = ctid; it < rows_here * (D / 4); it += kDecConsumers * 32) {
+        asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
+        for (int it = ctid; it < rows_here * (D / 4); it += NCONS * 32) {
             const int rr = it / (D / 4), d4 = (it % (D / 4)) * 4;
             float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
             for (int r = 0; r < kcl; ++r) {
@@ -862,7 +873,7 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
         }
         pend[0] = np;
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
+    asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
     const int np = pend[0];
     int *codes = reinterpret_cast<int *>(mbuf);
     for (int k = 0; k < np; ++k) {
@@ -870,12 +881,12 @@ __global__ void __launch_bounds__(kDecThreads, DIAG ? 3 : 2) k_decode_split(cons
         const long long ps = pend[2 + 3 * k], pe = pend[3 + 3 * k];
         const int n = piece_count(ps, pe, ptot, a.ncta);
         const long long c_first = cta_of(ps, ptot, a.ncta);
-        for (int i = ctid; i < n; i += kDecConsumers * 32) codes[i] = piece_code(i, ps, ptot, a.ncta, c_first);
+        for (int i = ctid; i < n; i += NCONS * 32) codes[i] = piece_code(i, ps, ptot, a.ncta, c_first);
         __threadfence();   // acquire: the other pieces' partials are visible after their counts
-        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
-        merge_unit<D>(a, v, codes, n, warp, lane);
+        asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
+        merge_unit<D, NCONS>(a, v, codes, n, warp, lane);
         if (ctid == 0) a.counters[v] = 0;   // ready for the next call
-        asm volatile("bar.sync 1, %0;" ::"n"(kDecConsumers * 32));
+        asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
     }
 }
 
@@ -1024,14 +1035,14 @@ static cudaError_t split_grid(size_t smem, int cluster, int *ncta) {
     } else if (cluster == 1) {
         int sms = 0, occ = 0;
         if ((e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess) return e;
-        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_split<D, NT, DIAG>, kDecThreads, smem)) !=
+        if ((e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, k_decode_split<D, NT, DIAG>, (SplitSmem<D, NT, DIAG>::THREADS), smem)) !=
             cudaSuccess)
             return e;
         n = sms * (occ > 0 ? occ : 1);
     } else {
         cudaLaunchConfig_t cfg = {};
         cfg.gridDim = dim3(cluster);
-        cfg.blockDim = dim3(kDecThreads);
+        cfg.blockDim = dim3((SplitSmem<D, NT, DIAG>::THREADS));
         cfg.dynamicSmemBytes = smem;
         cudaLaunchAttribute attr;
         attr.id = cudaLaunchAttributeClusterDimension;
@@ -1087,7 +1098,7 @@ static cudaError_t launch_split(const DecodeArgs &a0, cudaStream_t s) {
     if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(a.ncta);
-    cfg.blockDim = dim3(kDecThreads);
+    cfg.blockDim = dim3((SplitSmem<D, NT, DIAG>::THREADS));
     cfg.dynamicSmemBytes = smem;
     cfg.stream = s;
     cudaLaunchAttribute attr[2];

@@ -203,6 +203,7 @@ def test_decode_bad_page_in_first_pages_is_flagged():
     (8, 32, 4, 4, 64, 900),     # 32 query rows per unit (four row tiles), d = 64
     (8, 16, 4, 5, 128, 333),    # 20 query rows
     (4, 32, 4, 5, 128, 640),    # 40 query rows: two row passes per unit
+    (64, 28, 4, 1, 128, 300),   # 256 units: one CTA owns each whole unit (no merge)
 ])
 def test_decode_equal_lengths_cluster_split(B, Hq, Hkv, R, d, E):
     """Equal-length units in a full-width page table (the read-ahead and cluster-merge path when a
