@@ -75,7 +75,10 @@ struct SplitSmem {
     static constexpr int ROWS = NT * 8;                   // query rows of one piece
     static constexpr int WST = 9;                         // merge weights per row (<= 8) + log2 partition
     static constexpr int EPI_BYTES = ROWS * 8 + ROWS * WST * 4;
-    static constexpr size_t FIXED = 16 + STAGES_BYTES + 2 * QBUF + BARS * 8 + STAGES * 4 + MBUF_FLOATS * 4 +
+    static constexpr int SVALID_INTS = (STAGES + 3) & ~3;   // padded: mbuf (read as float4) stays 16-byte aligned
+    static constexpr int MBUF_OFF = STAGES_BYTES + 2 * QBUF + BARS * 8 + SVALID_INTS * 4;
+    static_assert(MBUF_OFF % 16 == 0 && (MBUF_FLOATS * 4) % 16 == 0, "16-byte aligned epilogue buffers");
+    static constexpr size_t FIXED = 16 + STAGES_BYTES + 2 * QBUF + BARS * 8 + SVALID_INTS * 4 + MBUF_FLOATS * 4 +
                                     16 * 4 + ((EPI_BYTES + 15) / 16) * 16;
 };
 
@@ -294,7 +297,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, DIAG ? 1 : 2)
     uint64_t *qfull = empty + NS;
     uint64_t *qempty = qfull + 2;
     int *svalid = reinterpret_cast<int *>(qempty + 2);
-    float *mbuf = reinterpret_cast<float *>(svalid + NS);
+    float *mbuf = reinterpret_cast<float *>(svalid + L::SVALID_INTS);
     int *misc = reinterpret_cast<int *>(mbuf + L::MBUF_FLOATS);
     // epilogue tables: output row index and merge weights per query row of the piece
     long long *orow = reinterpret_cast<long long *>(misc + 16);

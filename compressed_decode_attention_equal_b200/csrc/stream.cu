@@ -105,10 +105,10 @@ __device__ long long block_sum_ll(long long x, long long *red) {
     return t;
 }
 
-// write node e's mean key, mean value, alpha, beta into its pool slot
+// write node e's mean key, mean value, alpha, beta into its pool slot (pg: its page if known)
 template <int D, typename T>
-__device__ void write_node(const StreamArgs &s, const UnitState<D, T> &st, int u, int e) {
-    uint8_t *pg = entry_page<D, T>(s, u, e);
+__device__ void write_node(const StreamArgs &s, const UnitState<D, T> &st, int u, int e, uint8_t *pg = nullptr) {
+    if (!pg) pg = entry_page<D, T>(s, u, e);
     if (!pg) return;
     constexpr int VEC = kPageNodes * D * Elem<T>::SIZE;
     const int slot = e % kPageNodes;
@@ -235,6 +235,7 @@ __host__ __device__ constexpr size_t append_smem(int NM) {
 
 template <int D, typename T>
 __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamArgs s) {
+    static_assert(D <= kStreamThreads, "one thread per dimension");
     extern __shared__ __align__(16) uint8_t dsm[];
     float *sP = reinterpret_cast<float *>(dsm);                               // [2D][16]
     long long *sV = reinterpret_cast<long long *>(dsm + 2 * D * kProjDim * 4);  // [NM] V in node order
@@ -243,25 +244,52 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
     __shared__ float zy[kProjDim];
     __shared__ double red_d[kStreamThreads / 32];
     __shared__ long long red_l[kStreamThreads / 32];
-    __shared__ int sh_split, sh_merge_j, sh_pos, sh_ok;
-    __shared__ long long sh_D;
+    __shared__ int sh_split, sh_merge_j, sh_pos, sh_ok, sh_yslot, sh_open, sh_mopen;
+    __shared__ long long sh_D, sh_Vopen;
+    __shared__ uint8_t *sh_opage;
     __shared__ unsigned long long sh_bmin;
+    __shared__ float zl[kProjDim];
     const int u = blockIdx.x;
     const int tid = threadIdx.x;
     UnitState<D, T> st(s, u);
     StreamHdr &H = *st.hdr;
     constexpr int VEC = kPageNodes * D * Elem<T>::SIZE;
+    // The loads are grouped into rounds of independent requests (every round is one L2 round trip):
+    // header; ring slot, open node, last feature and projection; page id and the open node's
+    // statistics; the leaving token.
     const int W = H.W, N = H.N;
     int n_nodes = H.n_nodes, n_ent = H.n_ent;
     const int ring = H.ring;
-
-    // 1. the oldest recent token y leaves the window: read it from its pool slot
-    for (int i = tid; i < 2 * D * kProjDim; i += kStreamThreads) sP[i] = s.pt[i];
-    const int yslot = st.recent[ring];
-    const uint8_t *ypg = entry_page<D, T>(s, u, yslot);
-    if (tid == 0) sh_ok = ypg != nullptr && n_nodes >= 1;
+    {   // the projection: every load in flight at once
+        constexpr int NV4 = 2 * D * kProjDim / 4 / kStreamThreads;
+        float4 p4[NV4];
+#pragma unroll
+        for (int r = 0; r < NV4; ++r) p4[r] = reinterpret_cast<const float4 *>(s.pt)[r * kStreamThreads + tid];
+#pragma unroll
+        for (int r = 0; r < NV4; ++r) reinterpret_cast<float4 *>(sP)[r * kStreamThreads + tid] = p4[r];
+    }
+    if (tid == 0) sh_yslot = st.recent[ring];
+    if (tid == 32) sh_open = n_nodes >= 1 ? st.order[n_nodes - 1] : -1;
+    if (tid >= 64 && tid < 64 + kProjDim) zl[tid - 64] = H.z_last[tid - 64];
+    __syncthreads();
+    const int yslot = sh_yslot, open = sh_open;
+    if (tid == 0) sh_ok = open >= 0 && entry_page<D, T>(s, u, yslot) != nullptr;
+    if (tid == 32 && open >= 0) {
+        sh_Vopen = st.V[open];
+        sh_mopen = st.m[open];
+        sh_opage = entry_page<D, T>(s, u, open);
+    }
+    // the open node's running means (used if y joins it)
+    double mk_o = 0.0, mv_o = 0.0;
+    if (tid < D && open >= 0) {
+        mk_o = st.mk[static_cast<int64_t>(open) * D + tid];
+        mv_o = st.mv[static_cast<int64_t>(open) * D + tid];
+    }
     __syncthreads();
     if (!sh_ok) return;
+
+    // 1. the oldest recent token y leaves the window: read it from its pool slot
+    const uint8_t *ypg = entry_page<D, T>(s, u, yslot);
     for (int dim = tid; dim < D; dim += kStreamThreads) {
         ky[dim] = Elem<T>::get(ypg + vec_off<D, T>(yslot % kPageNodes, dim));
         vy[dim] = Elem<T>::get(ypg + VEC + vec_off<D, T>(yslot % kPageNodes, dim));
@@ -271,7 +299,7 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
     if (tid < kProjDim) zy[tid] = feature_i(sP, ky, vy, D, tid);
     __syncthreads();
     if (tid == 0) {
-        long long Dy = quantised_step(H.z_last, zy);
+        long long Dy = quantised_step(zl, zy);
         if (Dy < 0) {
             raise_flag(s.flags, FLAG_OVERFLOW);
             Dy = 0;
@@ -279,7 +307,7 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
         const long long cT = H.cT + Dy;
         H.cT = cT;
         for (int i = 0; i < kProjDim; ++i) H.z_last[i] = zy[i];
-        const long long Vo = st.V[st.order[n_nodes - 1]];
+        const long long Vo = sh_Vopen;
         sh_split = prod_ge(static_cast<unsigned long long>(N), static_cast<unsigned long long>(Vo + Dy), 1ull,
                            static_cast<unsigned long long>(cT))
                        ? 1
@@ -310,23 +338,21 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
         ++n_nodes;
         ++n_ent;
     } else {   // y joins the open node (pairwise update with a one-member node)
-        const int e = st.order[n_nodes - 1];
-        const int m = st.m[e];
+        const int e = open;
+        const int m = sh_mopen;
         const double inv = 1.0 / (m + 1);
         double q = 0.0;
-        for (int dim = tid; dim < D; dim += kStreamThreads) {
-            double &mk = st.mk[static_cast<int64_t>(e) * D + dim];
-            double &mv = st.mv[static_cast<int64_t>(e) * D + dim];
-            const double dk = static_cast<double>(ky[dim]) - mk;
-            q += dk * dk;
-            mk += dk * inv;
-            mv += (static_cast<double>(vy[dim]) - mv) * inv;
+        if (tid < D) {
+            const double dk = static_cast<double>(ky[tid]) - mk_o;
+            q = dk * dk;
+            st.mk[static_cast<int64_t>(e) * D + tid] = mk_o + dk * inv;
+            st.mv[static_cast<int64_t>(e) * D + tid] = mv_o + (static_cast<double>(vy[tid]) - mv_o) * inv;
         }
         const double dd = block_sum(q, red_d);
         if (tid == 0) {
             st.M2[e] += dd * m * inv;
             st.m[e] = m + 1;
-            st.V[e] += Dy;
+            st.V[e] = sh_Vopen + Dy;
         }
     }
     __syncthreads();
@@ -334,11 +360,33 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
     // 3. above N nodes: merge the adjacent pair with the smallest combined variation
     int merged = -1, moved = -1;
     if (n_nodes > N) {
-        // the node order and variations to shared memory (all loads in flight at once)
-        for (int j = tid; j < n_nodes; j += kStreamThreads) {
-            const int o = st.order[j];
-            sOrder[j] = o;
-            sV[j] = st.V[o];
+        // the node order, then the nodes' variations, to shared memory (batches of loads in flight)
+        for (int j0 = 0; j0 < n_nodes; j0 += 4 * kStreamThreads) {
+            int o[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int j = j0 + r * kStreamThreads + tid;
+                o[r] = j < n_nodes ? st.order[j] : 0;
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int j = j0 + r * kStreamThreads + tid;
+                if (j < n_nodes) sOrder[j] = o[r];
+            }
+        }
+        __syncthreads();
+        for (int j0 = 0; j0 < n_nodes; j0 += 4 * kStreamThreads) {
+            long long vv[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int j = j0 + r * kStreamThreads + tid;
+                vv[r] = j < n_nodes ? st.V[sOrder[j]] : 0;
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int j = j0 + r * kStreamThreads + tid;
+                if (j < n_nodes) sV[j] = vv[r];
+            }
         }
         __syncthreads();
         // the smallest V_j + V_{j+1} (all >= 0), then the smallest j attaining it
@@ -436,8 +484,8 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
 
     // 4. the new token takes y's (possibly moved) slot as an exact recent entry
     {
-        const int ns = st.recent[ring];
-        uint8_t *pg = entry_page<D, T>(s, u, ns);
+        const int ns = merged >= 0 ? st.recent[ring] : yslot;   // entries move only in a merge
+        uint8_t *pg = ns == yslot ? const_cast<uint8_t *>(ypg) : entry_page<D, T>(s, u, ns);
         if (pg) {
             const T *kn = static_cast<const T *>(s.k_new) + static_cast<int64_t>(u) * D;
             const T *vn = static_cast<const T *>(s.v_new) + static_cast<int64_t>(u) * D;
@@ -449,7 +497,10 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
         }
     }
     // 5. changed middle nodes to the pool
-    write_node<D, T>(s, st, u, st.order[n_nodes - 1]);
+    {
+        const int last_node = merged >= 0 || sh_split ? st.order[n_nodes - 1] : open;
+        write_node<D, T>(s, st, u, last_node, last_node == open ? sh_opage : nullptr);
+    }
     if (merged >= 0) write_node<D, T>(s, st, u, merged);
     if (moved >= 0) write_node<D, T>(s, st, u, moved);
     __syncthreads();
