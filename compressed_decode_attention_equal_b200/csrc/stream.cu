@@ -243,7 +243,6 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
     __shared__ float ky[D], vy[D];
     __shared__ float zy[kProjDim];
     __shared__ double red_d[kStreamThreads / 32];
-    __shared__ long long red_l[kStreamThreads / 32];
     __shared__ int sh_split, sh_merge_j, sh_pos, sh_ok, sh_yslot, sh_open, sh_mopen;
     __shared__ long long sh_D, sh_Vopen;
     __shared__ uint8_t *sh_opage;

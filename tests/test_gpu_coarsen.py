@@ -89,6 +89,9 @@ CASES = [
     ("single_segment", torch.bfloat16, 128, 2, [3000], [1], "normal"),
     ("tile_edges", torch.bfloat16, 128, 1, [56 + 255, 56 + 256, 56 + 510, 56 + 511, 56 + 254], [7, 7, 7, 7, 7],
      "normal"),
+    # 21 units of ragged lengths: one sequence empty, one without a middle, one with N = 1
+    ("many_units_ragged", torch.bfloat16, 128, 3, [900, 40, 1500, 0, 700, 2100, 333], [30, 4, 60, 4, 1, 80, 9],
+     "normal"),
 ]
 
 
@@ -225,6 +228,42 @@ def test_gqa6_10k5_prefill_then_decode():
     out, lse = skv.decode_attn(q, w.Hkv, r["pool"], r["table"], r["lens"])
     ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), gpu_units(r["pool"], r["table"], r["lens"], 1, 2))
     check_decode(out, lse, ref_out, ref_lse, torch.bfloat16, "gqa6 decode")
+
+
+def test_captured_coarsen_matches_direct_call_bitwise():
+    """A coarsening call captured into a CUDA graph and replayed gives, bit for bit, the c_t,
+    boundaries, lens and stored nodes of a direct call (the launches carry every host-side plan
+    value with them), for both segment representatives."""
+    T_list, N_list, Hkv, d, seed = [900, 40, 1500, 0, 700, 2100, 333, 1200], [30, 4, 60, 4, 1, 80, 9, 44], 3, 128, 31
+    w = workloads.Workload("captured", seed, B=len(T_list), Hq=Hkv, Hkv=Hkv, d=d, R=1, dtype="bf16", T=0, regimes=12)
+    k, v, _ = workloads.make_kv(w, "cuda", T_list=T_list)
+    for representative in ("mean", "variation"):
+        r = run_coarsen(k, v, Hkv, T_list, N_list, seed, representative=representative)
+        assert r["status"] == 0, r["flags"]
+        pool2 = skv.NodePool(r["pool"].num_pages, d, torch.bfloat16)
+        lens2 = torch.full_like(r["lens"], -7)
+        bnd2 = torch.full_like(r["bnd"], -7)
+        cum2 = torch.full_like(r["cum"], -7)
+        ws2 = torch.zeros(skv.coarsen_workspace_bytes(Hkv, d, T_list, N_list, S, W), dtype=torch.uint8, device="cuda")
+        torch.cuda.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            skv.coarsen(k, v, Hkv, T_list, N_list, S, W, seed, pool2, r["table"], lens=lens2, boundaries=bnd2,
+                        cumvar=cum2, workspace=ws2, representative=representative)
+        g.replay()
+        torch.cuda.synchronize()
+        assert skv.workspace_error(ws2)[0] == 0
+        assert torch.equal(lens2, r["lens"]) and torch.equal(bnd2, r["bnd"])
+        for b, T in enumerate(T_list):
+            for h in range(Hkv):
+                off = sum(T_list[:b]) * Hkv + h * T
+                M = max(0, T - S - W)
+                assert torch.equal(cum2[off:off + M], r["cum"][off:off + M])
+                one = skv.read_entries(r["pool"], r["table"], r["lens"], b, h)
+                two = skv.read_entries(pool2, r["table"], lens2, b, h)
+                for x, y in zip(one, two):
+                    assert torch.equal(x, y), f"{representative}: unit ({b},{h}) differs"
+        del g
 
 
 def test_coarsen_is_deterministic():
