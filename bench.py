@@ -11,8 +11,10 @@ Workload (one step = one decode-attention call for the whole batch):
 Output: one JSON line (rank 0) with the decode throughput (`value`, query rows/s), the decode
 op's achieved HBM bandwidth against the measured copy peak (`roofline`), an end-to-end figure
 with pinned host queries / outputs copied every step (`e2e`), the SM clocks sampled during the
-timed region, the CPU oracle timed on the host (`cpu_baseline`), and the coarsener's own
-throughput on the 8 x 4 x 131,072-token workload (`coarsen`).
+timed region, the CPU oracle timed on the host (`cpu_baseline`), the coarsener's own
+throughput on the 8 x 4 x 131,072-token workload (`coarsen`), decode with the diagonal closure
+(`diagonal_closure`), streaming appends (`streaming_append`), and decode on the 1.5B-shaped
+10.5K-token and the ragged paged 2% workloads (`other_decode`).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
 Multi-GPU (torchrun, one rank per GPU): every rank decodes its own batch (weak scaling, no
@@ -405,6 +407,61 @@ def diagonal_closure_stage(w, device, layers: int, steps: int = 6000):
             "note": "same workload and call with diagonal-closure pools (per-dimension key variances)"}
 
 
+def other_decode_stage(device, steps: int = 6000):
+    """Decode on the two other decode workloads, each cache built by the coarsener and replayed from
+    CUDA graphs (rank 0 only):
+    - gqa6_10k5_prefill_decode: 1 sequence, 2 KV heads, 421 entries each, a 0.45 MB cache, so the
+      call is latency-bound (reported in us); the cache is copied into enough pools to exceed L2
+      and the copies rotate.
+    - gqa7_ragged_paged_2pct: 128 sequences of log-uniform lengths, 4 query rows per sequence,
+      shuffled page tables; HBM-bound. Two independently seeded caches (each larger than L2) rotate."""
+    import torch
+    import compressed_decode_attention_equal_b200 as skv
+    import workloads
+    peak, _ = _peaks()
+    res = {}
+    for name, layers in (("gqa6_10k5_prefill_decode", 1), ("gqa7_ragged_paged_2pct", 2)):
+        w = workloads.WORKLOADS[name]
+        caches, table, _, _, _ = build_layer_caches(w, layers, device)
+        base = caches[0]
+        copies = -(-(256 << 20) // base["pool"].nbytes()) if layers == 1 else 1
+        if copies > 1:
+            pools = []
+            for _ in range(copies):
+                p = skv.NodePool(base["pool"].num_pages, w.d, w.torch_dtype, device=device)
+                p.pages.copy_(base["pool"].pages)
+                pools.append(p)
+            caches = [dict(base, pool=p) for p in pools]
+        L = len(caches)
+        alg, ent = algorithmic_decode_bytes(w, [int(caches[0]["lens"].sum())])
+        outs = [torch.empty_like(c["q"]) for c in caches]
+        lses = [torch.empty(w.B, w.R, w.Hq, dtype=torch.float32, device=device) for _ in caches]
+        ws = torch.zeros(skv.decode_workspace_bytes(w.B, w.R, w.Hq, w.Hkv, w.d, table.shape[2]), dtype=torch.uint8,
+                         device=device)
+
+        def step(i):
+            c = caches[i % L]
+            skv.decode_attn(c["q"], w.Hkv, c["pool"], table, c["lens"], out=outs[i % L], lse=lses[i % L],
+                            workspace=ws)
+
+        for i in range(L + 3):
+            step(i)
+        torch.cuda.synchronize()
+        st, flags = skv.workspace_error(ws)
+        if st != 0:
+            raise RuntimeError(f"{name}: decode raised device flags {flags}")
+        ms = time_graphs(step, steps, L, False)
+        us = ms / steps * 1e3
+        rows = w.B * w.R * w.Hq
+        res[name] = {"us_per_call": us, "query_rows_per_call": rows, "query_rows_per_s": rows / (us * 1e-6),
+                     "entries_per_call": ent, "algorithmic_bytes_per_launch": alg,
+                     "achieved_gbs": alg / (us * 1e-6) / 1e9, "frac": alg / (us * 1e-6) / 1e9 / peak,
+                     "l2": f"{L} caches of {base['pool'].nbytes() / 1e6:.2f} MB pool each, rotated"}
+        del caches, outs, lses, base
+        torch.cuda.empty_cache()
+    return res
+
+
 def stream_stage(w, device, steps: int = 3000, distinct: int = 60):
     """Streaming coarsening on the decode workload: skv_stream_init on the prompts, then appends of
     one token per unit replayed from CUDA graphs (rank 0 only). The append is latency-bound (one CTA
@@ -612,6 +669,7 @@ def main():
     ap.add_argument("--no-coarsen", action="store_true")
     ap.add_argument("--no-diagonal", action="store_true", help="skip the diagonal-closure decode timing")
     ap.add_argument("--no-stream", action="store_true", help="skip the streaming-append timing")
+    ap.add_argument("--no-other", action="store_true", help="skip the decode timing on the other two workloads")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -642,6 +700,8 @@ def main():
             res["diagonal_closure"] = diagonal_closure_stage(w, device, args.layers)
         if not args.no_stream:
             res["streaming_append"] = stream_stage(w, device)
+        if not args.no_other:
+            res["other_decode"] = other_decode_stage(device)
         if not args.no_cpu_baseline:
             res["cpu_baseline"] = cpu_baseline(w, caches, table)
         print(json.dumps(res), flush=True)

@@ -39,7 +39,6 @@
 namespace skv {
 
 constexpr int kDecConsumers = 4;
-constexpr int kDecThreads = (kDecConsumers + 1) * 32;
 // Ring depth: a multiple of every page-group count (1, 2, 4), so that the pages i and
 // i + kDecStages that share a stage always go to the same consumer warp, in order. A warp that
 // could poll a stage for page i + kDecStages while it still held page i would see the previous
@@ -1072,6 +1071,11 @@ static cudaError_t split_grid(size_t smem, int cluster, int *ncta) {
 // (an aligned split then streams at most 4/3 of the pages per CTA a stream-K split would, and
 // saves its global merges). It is used only if the device finds every unit equally long;
 // otherwise the same grid runs the stream-K split.
+// Few pages (all units together, at max_pages pages each, give at most one page per CTA of the
+// full grid): a stream-K split would leave most CTAs idle and merge each unit's one-page pieces
+// through global partials. The grid then shrinks to exactly one cluster of k CTAs per virtual
+// unit, k <= max_pages the largest co-resident size, so each CTA streams about max_pages / k
+// pages and the pieces merge in distributed shared memory.
 template <int D, int NT, bool DIAG>
 static cudaError_t split_config(DecodeArgs *a, size_t *smem) {
     *smem = split_smem<D, NT, DIAG>(a->n_vunits, 1);
@@ -1079,13 +1083,17 @@ static cudaError_t split_config(DecodeArgs *a, size_t *smem) {
     if (e != cudaSuccess) return e;
     if (a->ncta < 1) return cudaErrorInvalidValue;
     a->cluster = 1;
-    for (int k = a->ncta / a->n_vunits < kMaxCluster ? a->ncta / a->n_vunits : kMaxCluster; k > 1; --k) {
+    const long long nv = a->n_vunits;
+    const bool few = nv * a->max_pages <= a->ncta;
+    int kmax = a->ncta / a->n_vunits < kMaxCluster ? a->ncta / a->n_vunits : kMaxCluster;
+    if (few && kmax > a->max_pages) kmax = a->max_pages;
+    for (int k = kmax; k > 1; --k) {
         const size_t sk = split_smem<D, NT, DIAG>(a->n_vunits, k);
         int n = 0;
         if ((e = split_grid<D, NT, DIAG>(sk, k, &n)) != cudaSuccess) return e;
-        if (static_cast<long long>(a->n_vunits) * k <= n && static_cast<long long>(a->n_vunits) * k * 4 >= 3LL * n) {
+        if (nv * k <= n && (few || nv * k * 4 >= 3LL * n)) {
             a->cluster = k;
-            a->ncta = n;
+            a->ncta = few ? static_cast<int>(nv * k) : n;
             *smem = sk;
             break;
         }
