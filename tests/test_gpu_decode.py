@@ -211,6 +211,18 @@ def test_decode_equal_lengths_cluster_split(B, Hq, Hkv, R, d, E):
     _run(B, Hq, Hkv, R, d, [E] * B, torch.bfloat16, seed=B * 100 + R * 10 + d // 64, shuffle=True)
 
 
+@pytest.mark.parametrize("B,Hq,Hkv,R,d,lens", [
+    (1, 12, 2, 1, 128, [421]),              # the 1.5B 10.5K shape: 2 units x 27 pages, clusters of 8
+    (3, 12, 2, 1, 128, [421, 37, 0]),       # unequal and empty units: stream-K over the small grid
+    (2, 28, 4, 4, 64, [100, 100]),          # 28 query rows, d = 64, 7 pages per unit: clusters of 7
+    (1, 7, 1, 1, 128, [17]),                # two pages: a cluster of 2
+])
+def test_decode_few_pages(B, Hq, Hkv, R, d, lens):
+    """Fewer pages in all units than the grid has CTAs: one cluster of up to 8 CTAs per unit and a
+    grid of exactly those clusters (equal lengths), or the stream-K split over that grid."""
+    _run(B, Hq, Hkv, R, d, lens, torch.bfloat16, seed=sum(lens) + Hq + d, shuffle=True)
+
+
 def test_decode_equal_lengths_wide_table_two_row_passes():
     """Equal lengths, 40 query rows (two row passes), page table wider than the units."""
     B, Hq, Hkv, R, d = 4, 32, 4, 5, 128
