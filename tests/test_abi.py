@@ -171,3 +171,28 @@ def test_binding_fails_loudly_without_library(tmp_path):
             _lib.load(str(tmp_path / "missing.so"))
     finally:
         _lib._lib = saved
+
+
+@pytest.mark.parametrize("compiler,std", [("gcc", "-std=c99"), ("g++", "-std=c++17")])
+def test_header_compiles_as_c_and_cpp_and_links(lib, tmp_path, compiler, std):
+    """A translation unit that includes include/skv.h and takes the address of every declared entry
+    point compiles warning-free as C99 and as C++17 (the extern "C" guards) and links against
+    libskv.so; the program only counts the entry points (no CUDA call)."""
+    import shutil
+    import subprocess
+    cc = shutil.which(compiler)
+    if cc is None:
+        pytest.skip(f"{compiler} not installed")
+    names = _declared()
+    body = ['#include "skv.h"', "#include <stdio.h>", "", "typedef void (*entry_fn)(void);", "",
+            "int main(void) {", "    const entry_fn entries[] = {"]
+    body += [f"        (entry_fn)&{n}," for n in names]
+    body += ["    };", '    printf("%d\\n", (int)(sizeof entries / sizeof entries[0]));', "    return 0;", "}", ""]
+    src = tmp_path / ("main.c" if compiler == "gcc" else "main.cpp")
+    src.write_text("\n".join(body))
+    libdir = os.path.dirname(lib._name)
+    exe = tmp_path / "prog"
+    subprocess.run([cc, std, "-Wall", "-Wextra", "-Werror", "-pedantic", "-I", os.path.join(ROOT, "include"),
+                    str(src), "-L", libdir, "-lskv", f"-Wl,-rpath,{libdir}", "-o", str(exe)], check=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout
+    assert int(out) == len(names)
