@@ -1,7 +1,6 @@
 """Host-side rules of bench.py (not gpu): the algorithmic bytes a decode call must move, and the
 ncu traffic figure, which is reported only while the profiled sources are unchanged."""
 import os
-import shutil
 import sys
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -26,21 +25,21 @@ def test_algorithmic_decode_bytes_of_the_headline_workload():
 
 
 def test_profile_traffic_follows_the_source_hash(tmp_path, monkeypatch):
-    """A summary whose source hash matches gives its DRAM bytes; once any covered source changes
-    (here: a copy of the tree with one byte appended to a kernel file) the figure is withheld."""
-    for name, sources in (("decode_gqa7_32k_summary.md", bench.DECODE_SOURCES),
-                          ("coarsen_131k_summary.md", bench.COARSEN_SOURCES)):
-        assert bench._profile_traffic(name, sources) is not None, f"{name}: hash does not match the sources"
-        tree = tmp_path / name
-        os.makedirs(tree / "profiles")
-        shutil.copy(os.path.join(ROOT, "profiles", name), tree / "profiles" / name)
-        for f in sources:
-            os.makedirs(os.path.dirname(tree / f), exist_ok=True)
-            shutil.copy(os.path.join(ROOT, f), tree / f)
-        monkeypatch.setattr(bench, "ROOT", str(tree))
-        assert bench._profile_traffic(name, sources) is not None
-        with open(tree / sources[0], "ab") as fh:
-            fh.write(b"\n")
-        assert bench._profile_traffic(name, sources) is None
-        monkeypatch.setattr(bench, "ROOT", ROOT)
-    assert bench._profile_traffic("no_such_summary.md", bench.DECODE_SOURCES) is None
+    """A summary whose recorded hash matches its sources gives its DRAM bytes; once any covered
+    source changes by one byte the figure is withheld (the bench then reports traffic null)."""
+    tree = tmp_path / "tree"
+    os.makedirs(tree / "profiles")
+    os.makedirs(tree / "src")
+    sources = ["src/kernel.cu", "src/common.cuh"]
+    for f, text in zip(sources, (b"__global__ void k() {}\n", b"// shared\n")):
+        (tree / f).write_bytes(text)
+    monkeypatch.setattr(bench, "ROOT", str(tree))
+    sha = bench._source_sha(sources)
+    (tree / "profiles" / "k_summary.md").write_text(
+        f"# k\n\nsource_sha256_16: {sha}\ndram_bytes_per_launch: 79030528\n")
+    assert bench._profile_traffic("k_summary.md", sources) == 79030528.0
+    assert bench._profile_traffic("k_summary.md", sources[:1]) is None     # other file set
+    with open(tree / sources[1], "ab") as fh:
+        fh.write(b" ")
+    assert bench._profile_traffic("k_summary.md", sources) is None
+    assert bench._profile_traffic("no_such_summary.md", sources) is None
