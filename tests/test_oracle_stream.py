@@ -2,7 +2,10 @@
 middle nodes tile the middle span in order (masses add up, starts are contiguous), their variations
 add up to c_T exactly, there are at most N of them, and each node's statistics equal numpy's direct
 ones over its members (which pins the pairwise merge); N = 1 keeps one node over the whole middle;
-a large jump entering the middle starts a new node exactly at the jump."""
+a large jump entering the middle starts a new node exactly at the jump. The split and merge
+decisions (readings S3-S5) match an independent replay over (start, m, V) after every append, on
+random walks and on caches whose steps repeat exactly (ties between pair sums), and the split
+rule is checked at its boundary (N (V_open + D) equal to c_T after the step, and one less)."""
 import numpy as np
 import pytest
 
@@ -82,3 +85,117 @@ def test_jump_starts_a_new_node():
         u.append(k[t], v[t])
     assert any(n.start == jump for n in u.nodes)
     _check_invariants(u, k, v)
+
+
+def _replay_decisions(nodes, cT, N, steps, first_token):
+    """Readings S3-S5 restated over (start, m, V) triples alone: c_T grows by the step, the token
+    opens a new segment when N (V_open + D) >= c_T and joins the open one otherwise, and while more
+    than N segments remain the adjacent pair with the smallest summed variation (leftmost on ties)
+    becomes one."""
+    segs = [tuple(x) for x in nodes]
+    for i, D in enumerate(steps):
+        tok = first_token + i
+        cT += D
+        start, m, V = segs[-1]
+        segs = segs + [(tok, 1, D)] if N * (V + D) >= cT else segs[:-1] + [(start, m + 1, V + D)]
+        while len(segs) > N:
+            pair = min(range(len(segs) - 1), key=lambda j: (segs[j][2] + segs[j + 1][2], j))
+            (s0, m0, v0), (_, m1, v1) = segs[pair], segs[pair + 1]
+            segs = segs[:pair] + [(s0, m0 + m1, v0 + v1)] + segs[pair + 2:]
+    return segs, cT
+
+
+@pytest.mark.parametrize("N,seed,jumps", [(1, 11, ()), (2, 12, (700,)), (5, 13, (650, 820)), (40, 14, ()),
+                                          (40, 15, (620, 640, 900)), (300, 16, (700,))])
+def test_split_and_merge_decisions_match_a_brute_force_replay(N, seed, jumps):
+    """After every append the oracle's segments (start, m, V) and c_T equal an independent replay of
+    the split and merge rules fed the same quantised steps (the steps come from the pinned fixed
+    fp32 recipe). Plausible slips -- '>' for '>=', comparing V_open without the new step, c_T before
+    the step, the single smallest V instead of the smallest pair, the rightmost tie -- change the
+    segments on these walks."""
+    T0, extra, d = 600, 420, 64
+    k, v = _walk(T0 + extra, d, seed=seed)
+    for j in jumps:
+        k[j:] += 6.0
+    P = oracle.projection(seed, d)
+    u = StreamUnit(k[:T0], v[:T0], S, W, N, P)
+    segs = [(n.start, n.m, n.V) for n in u.nodes]
+    cT = u.cT
+    first = T0 - W                                   # the token that enters the middle first
+    z_prev = oracle.feature_f32(P, k[first - 1], v[first - 1])
+    saw_split = saw_merge = False
+    for i in range(extra):
+        tok = first + i
+        z = oracle.feature_f32(P, k[tok], v[tok])
+        D = oracle.quantised_step(z_prev, z)
+        z_prev = z
+        splits, merges = u.splits, u.merges
+        u.append(k[T0 + i], v[T0 + i])
+        segs, cT = _replay_decisions(segs, cT, N, [D], tok)
+        assert [(n.start, n.m, n.V) for n in u.nodes] == segs, f"append {i}"
+        assert u.cT == cT
+        saw_split |= u.splits > splits
+        saw_merge |= u.merges > merges
+    if N > 1:
+        assert saw_split and saw_merge
+
+
+def _periodic(T, d, seed, flat):
+    """Tokens alternating between two fixed vectors, so every variation step is the same integer D
+    (the fp32 differences of a pair are exact negatives of each other), except a run `flat` of one
+    repeated token (steps 0). All c_T and V are then multiples of D: exact equalities
+    N (V_open + D) = c_T and exact ties between adjacent pair sums occur throughout."""
+    rng = np.random.default_rng(seed)
+    a, b = rng.standard_normal((2, 2, d)).astype(np.float32)
+    k = np.empty((T, d), np.float32)
+    v = np.empty((T, d), np.float32)
+    for t in range(T):
+        src = a if (t % 2 == 0 or t in flat) else b
+        k[t], v[t] = src[0], src[1]
+    return k, v
+
+
+@pytest.mark.parametrize("N", [2, 3, 4, 7, 12, 40])
+def test_split_and_merge_decisions_on_exact_ties(N):
+    """The replay above on caches whose steps repeat exactly: splits at N (V_open + D) = c_T and
+    merges among equal pair sums decide the segments, so '>' for '>=', c_T taken before the step and
+    the rightmost tie each give different segments."""
+    T0, extra, d = 300, 500, 32
+    k, v = _periodic(T0 + extra, d, seed=N, flat=range(T0 + 200, T0 + 260))
+    P = oracle.projection(N + 100, d)
+    u = StreamUnit(k[:T0], v[:T0], S, W, N, P)
+    segs = [(n.start, n.m, n.V) for n in u.nodes]
+    cT = u.cT
+    first = T0 - W
+    z_prev = oracle.feature_f32(P, k[first - 1], v[first - 1])
+    for i in range(extra):
+        tok = first + i
+        z = oracle.feature_f32(P, k[tok], v[tok])
+        D = oracle.quantised_step(z_prev, z)
+        z_prev = z
+        u.append(k[T0 + i], v[T0 + i])
+        segs, cT = _replay_decisions(segs, cT, N, [D], tok)
+        assert [(n.start, n.m, n.V) for n in u.nodes] == segs, f"append {i}"
+        assert u.cT == cT
+
+
+@pytest.mark.parametrize("N", [2, 5, 40])
+def test_split_rule_at_its_boundary(N):
+    """Reading S4 at its boundary, with the unit's open-node variation and c_T set so that the test
+    knows the exact comparison: N (V_open + D) equal to c_T after the step splits ('>=', and c_T
+    includes the step); one less does not split. D is the fixed-recipe step of the token that
+    enters the middle."""
+    T0, d = 300, 32
+    k, v = _walk(T0 + 1, d, seed=N + 40)
+    P = oracle.projection(N + 40, d)
+    y = T0 - W                                            # the token that enters the middle
+    D = oracle.quantised_step(oracle.feature_f32(P, k[y - 1], v[y - 1]), oracle.feature_f32(P, k[y], v[y]))
+    assert D > 0
+    V_open = 1_000_003
+    for slack, splits in ((0, True), (1, False)):
+        u = StreamUnit(k[:T0], v[:T0], S, W, N, P)
+        u.nodes[-1].V = V_open
+        u.cT = N * (V_open + D) - D + slack               # so that N (V_open + D) = c_T + D - slack
+        u.append(k[T0], v[T0])
+        assert u.splits == (1 if splits else 0), f"slack {slack}"
+        assert u.cT == N * (V_open + D) + slack
