@@ -24,6 +24,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
 C = "oracle/skv_oracle.c"
 STREAM = "oracle/stream.py"
+INIT = "oracle/__init__.py"
 
 MUTATIONS = [
     # projection (reading R2) and the fixed fp32 variation recipe
@@ -67,6 +68,13 @@ MUTATIONS = [
     ("dec_diag_d", C, "closure = c / (2.0 * d);", "closure = c / d;"),
     ("dec_lse_log2", C, "const double l = mx + log(Z);", "const double l = mx + log2(Z);"),
     ("dec_out_unnorm", C, "const double p = exp(s[j] - l);", "const double p = exp(s[j] - mx);"),
+    # the Python layer: GQA head mapping and option marshalling
+    ("gqa_interleaved", INIT, "        rows = q[b, :, h * G:(h + 1) * G, :].reshape(R * G, d)",
+     "        rows = q[b, :, h::Hkv, :].reshape(R * G, d)"),
+    ("rows_order", INIT, "        rows = q[b, :, h * G:(h + 1) * G, :].reshape(R * G, d)",
+     "        rows = q[b, :, h * G:(h + 1) * G, :].transpose(1, 0, 2).reshape(R * G, d)"),
+    ("rep_codes_swapped", INIT, 'REPRESENTATIVES = {"mean": 0, "variation": 1}',
+     'REPRESENTATIVES = {"mean": 1, "variation": 0}'),
     # streaming (readings S3-S5)
     ("stream_gt_for_ge", STREAM, "if self.N * (last.V + D) >= self.cT:", "if self.N * (last.V + D) > self.cT:"),
     ("stream_no_step_in_open", STREAM, "if self.N * (last.V + D) >= self.cT:", "if self.N * last.V >= self.cT:"),
@@ -82,9 +90,14 @@ MUTATIONS = [
 # the Box-Muller branch is part of reading R2's generator definition, which the pages leave open
 CONVENTIONS = {"proj_sin"}
 
-# applied after the main replacement (the c_T update moves to after the split decision)
+# applied after the main replacement (the c_T update moves to after the split decision; the
+# interleaved GQA mapping also writes its outputs back interleaved)
 EXTRA = {"stream_cT_after_split": ("        while len(self.nodes) > self.N:",
-                                   "        self.cT += D\n        while len(self.nodes) > self.N:")}
+                                   "        self.cT += D\n        while len(self.nodes) > self.N:"),
+         "gqa_interleaved": ("        out[b, :, h * G:(h + 1) * G, :] = o.reshape(R, G, d)\n"
+                             "        lse[b, :, h * G:(h + 1) * G] = l.reshape(R, G)",
+                             "        out[b, :, h::Hkv, :] = o.reshape(R, G, d)\n"
+                             "        lse[b, :, h::Hkv] = l.reshape(R, G)")}
 
 
 def _copy_tree(dst):

@@ -105,3 +105,38 @@ def test_logit_terms_closed_form(orc):
 def test_empty_cache(orc):
     out, lse = orc.decode_rows(np.ones((2, 64)), np.zeros((0, 64)), np.zeros((0, 64)), np.zeros(0), np.zeros(0))
     assert np.all(out == 0) and np.all(np.isneginf(lse))
+
+
+def test_gqa_batch_matches_dense_attention_over_repeat_kv(orc):
+    """The batched decode's head mapping: with m = 1 and sigma^2 = 0 everywhere, decoding a batch
+    (several query rows per sequence, G query heads per KV head) equals dense softmax attention
+    after expanding the KV heads with transformers' `repeat_kv` (the GQA expansion the Llama / Qwen
+    model code applies: KV head j serves query heads j G .. j G + G - 1)."""
+    import torch
+    from transformers.models.llama.modeling_llama import repeat_kv
+
+    rng = np.random.default_rng(7)
+    B, R, Hkv, G, d, E = 2, 3, 3, 4, 16, 11
+    Hq = Hkv * G
+    K = rng.standard_normal((B, Hkv, E, d)) * 2
+    V = rng.standard_normal((B, Hkv, E, d))
+    q = rng.standard_normal((B, R, Hq, d))
+
+    class U:
+        pass
+
+    units = []
+    for b in range(B):
+        row = []
+        for h in range(Hkv):
+            u = U()
+            u.kt, u.vt, u.alpha, u.beta = K[b, h], V[b, h], np.zeros(E), np.zeros(E)
+            row.append(u)
+        units.append(row)
+    out, lse = orc.decode(q, units, threads=2)
+
+    Kx = repeat_kv(torch.from_numpy(K), G).numpy()          # [B, Hq, E, d]
+    Vx = repeat_kv(torch.from_numpy(V), G).numpy()
+    s = np.einsum("brhd,bhed->brhe", q, Kx) / math.sqrt(d)   # [B, R, Hq, E]
+    np.testing.assert_allclose(lse, logsumexp(s, axis=-1), rtol=1e-13, atol=1e-12)
+    np.testing.assert_allclose(out, np.einsum("brhe,bhed->brhd", softmax(s, axis=-1), Vx), rtol=1e-11, atol=1e-12)
