@@ -178,16 +178,16 @@ def algorithmic_decode_bytes(w, lens_list, closure: str = "scalar"):
     return ent * node + rows * w.d * 2 * 2 + rows * 4, ent
 
 
-def _graph_steps(fn, steps: int, chunk: int):
-    """Capture `fn(i)` for i in [0, chunk) into a CUDA graph (replayed for exactly `steps`)."""
+def _graph_steps(fn, steps: int, start: int = 0):
+    """Capture `fn(start + i)` for i in [0, steps) into one CUDA graph."""
     import torch
     g = torch.cuda.CUDAGraph()
     s = torch.cuda.Stream()
     s.wait_stream(torch.cuda.current_stream())
     with torch.cuda.stream(s):
         with torch.cuda.graph(g, stream=s):
-            for i in range(chunk):
-                fn(i)
+            for i in range(steps):
+                fn(start + i)
     torch.cuda.current_stream().wait_stream(s)
     return g
 
@@ -237,33 +237,61 @@ def finish_ranks(world: int):
     torch.distributed.destroy_process_group()
 
 
-def time_graphs(fn, steps: int, layers: int, dist_on: bool):
-    """Device time (ms) of exactly `steps` calls fn(i), replayed from CUDA graphs."""
+GRAPH_MAX_STEPS = 20000   # calls per captured graph; longer regions replay several graphs back to back
+
+
+def region_graphs(fn, steps: int):
+    """Graphs that together run exactly `steps` calls fn(0) .. fn(steps - 1), in order."""
+    graphs, done = [], 0
+    while done < steps:
+        n = min(GRAPH_MAX_STEPS, steps - done)
+        graphs.append(_graph_steps(fn, n, done))
+        done += n
+    return graphs
+
+
+def summarise_regions(times_ms, steps: int):
+    """Per-call statistics (us) over the timed regions of `steps` calls each."""
+    per = sorted(t / steps * 1e3 for t in times_ms)
+    n = len(per)
+    return {"regions": n, "steps_per_region": steps, "median_us": statistics.median(per), "min_us": per[0],
+            "max_us": per[-1], "p10_us": per[int(0.1 * (n - 1))], "p90_us": per[int(0.9 * (n - 1))]}
+
+
+def time_regions(fn, steps: int, dist_on: bool, regions: int, flush=None):
+    """Device time (ms) of `regions` timed regions, each EXACTLY `steps` calls fn(0..steps-1)
+    replayed from CUDA graphs and bracketed by a barrier (multi-rank) and a synchronize on both
+    sides. Between regions (outside the timed interval) `flush`, a buffer larger than L2, is
+    rewritten so that no region starts with the previous region's data in L2."""
     import torch
-    chunk = max(layers, min(steps, 60 * layers))
-    chunk -= chunk % layers
-    full, rem = divmod(steps, chunk)
-    g_full = _graph_steps(fn, chunk, chunk) if full else None
-    g_rem = _graph_steps(fn, rem, rem) if rem else None
-    if g_full is not None:
-        g_full.replay()   # first replay uploads the graph
-    if g_rem is not None:
-        g_rem.replay()
+    graphs = region_graphs(fn, steps)
+    for g in graphs:
+        g.replay()   # the first replay uploads the graph
     torch.cuda.synchronize()
-    if dist_on:
-        torch.distributed.barrier()
-    torch.cuda.synchronize()
-    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for _ in range(full):
-        g_full.replay()
-    if g_rem is not None:
-        g_rem.replay()
-    e1.record()
-    torch.cuda.synchronize()
-    if dist_on:
-        torch.distributed.barrier()
-    return e0.elapsed_time(e1)
+    times = []
+    for _ in range(regions):
+        if flush is not None:
+            flush.add_(1)
+        torch.cuda.synchronize()
+        if dist_on:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for g in graphs:
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        if dist_on:
+            torch.distributed.barrier()
+        times.append(e0.elapsed_time(e1))
+    del graphs
+    return times
+
+
+def l2_flush_buffer(device):
+    import torch
+    return torch.zeros(64 << 20, dtype=torch.float32, device=device)   # 256 MB, twice the 126 MB L2
 
 
 def coarsen_stage(device, reps: int = 5):
@@ -373,7 +401,7 @@ def cpu_baseline(w, caches, table, budget_s: float = 12.0):
                       f"{int(c['lens'].sum())} entries), fp64, nodes read back from the GPU"}
 
 
-def diagonal_closure_stage(w, device, layers: int, steps: int = 6000):
+def diagonal_closure_stage(w, device, layers: int, steps: int = 2000, regions: int = 5):
     """Decode with the diagonal closure (per-dimension variances in every node) on the same workload:
     layer caches coarsened into diagonal pools, graph replays, CUDA events (rank 0 only)."""
     import torch
@@ -396,18 +424,18 @@ def diagonal_closure_stage(w, device, layers: int, steps: int = 6000):
     st, flags = skv.workspace_error(ws)
     if st != 0:
         raise RuntimeError(f"diagonal-closure decode raised device flags {flags}")
-    ms = time_graphs(step, steps, L, False)
-    us = ms / steps * 1e3
+    stats = summarise_regions(time_regions(step, steps, False, regions, flush=l2_flush_buffer(device)), steps)
+    us = stats["median_us"]
     peak, src = _peaks()
     del caches
     torch.cuda.empty_cache()
     return {"us_per_call": us, "query_rows_per_s": w.B * w.R * w.Hq / (us * 1e-6),
             "achieved_gbs": alg / (us * 1e-6) / 1e9, "frac": alg / (us * 1e-6) / 1e9 / peak,
-            "algorithmic_bytes_per_launch": alg,
+            "algorithmic_bytes_per_launch": alg, "timing": stats,
             "note": "same workload and call with diagonal-closure pools (per-dimension key variances)"}
 
 
-def other_decode_stage(device, steps: int = 6000):
+def other_decode_stage(device, steps: int = 2000, regions: int = 5):
     """Decode on the two other decode workloads, each cache built by the coarsener and replayed from
     CUDA graphs (rank 0 only):
     - gqa6_10k5_prefill_decode: 1 sequence, 2 KV heads, 421 entries each, a 0.45 MB cache, so the
@@ -450,19 +478,19 @@ def other_decode_stage(device, steps: int = 6000):
         st, flags = skv.workspace_error(ws)
         if st != 0:
             raise RuntimeError(f"{name}: decode raised device flags {flags}")
-        ms = time_graphs(step, steps, L, False)
-        us = ms / steps * 1e3
+        stats = summarise_regions(time_regions(step, steps, False, regions, flush=l2_flush_buffer(device)), steps)
+        us = stats["median_us"]
         rows = w.B * w.R * w.Hq
         res[name] = {"us_per_call": us, "query_rows_per_call": rows, "query_rows_per_s": rows / (us * 1e-6),
                      "entries_per_call": ent, "algorithmic_bytes_per_launch": alg,
                      "achieved_gbs": alg / (us * 1e-6) / 1e9, "frac": alg / (us * 1e-6) / 1e9 / peak,
-                     "l2": f"{L} caches of {base['pool'].nbytes() / 1e6:.2f} MB pool each, rotated"}
+                     "timing": stats, "l2": f"{L} caches of {base['pool'].nbytes() / 1e6:.2f} MB pool each, rotated"}
         del caches, outs, lses, base
         torch.cuda.empty_cache()
     return res
 
 
-def stream_stage(w, device, steps: int = 3000, distinct: int = 60):
+def stream_stage(w, device, steps: int = 3000, distinct: int = 60, regions: int = 5):
     """Streaming coarsening on the decode workload: skv_stream_init on the prompts, then appends of
     one token per unit replayed from CUDA graphs (rank 0 only). The append is latency-bound (one CTA
     per unit, a 4,096-FMA projection chain and O(N) merge search per call)."""
@@ -493,15 +521,15 @@ def stream_stage(w, device, steps: int = 3000, distinct: int = 60):
     for i in range(distinct):
         step(i)
     torch.cuda.synchronize()
-    ms = time_graphs(step, steps, distinct, False)
+    stats = summarise_regions(time_regions(step, steps, False, regions), steps)
     st, flags = skv.workspace_error(ws)
     if st != 0:
         raise RuntimeError(f"streaming append raised device flags {flags}")
-    us = ms / steps * 1e3
+    us = stats["median_us"]
     units = w.B * w.Hkv
     del pool, state
     torch.cuda.empty_cache()
-    return {"us_per_append": us, "tokens_per_s": units / (us * 1e-6), "units": units,
+    return {"us_per_append": us, "tokens_per_s": units / (us * 1e-6), "units": units, "timing": stats,
             "init_s_host_clock": init_s,
             "note": "one token appended to every (sequence, KV head) unit per call, N = "
                     f"{N_list[0]} nodes per unit, graphs of {distinct} calls"}
@@ -510,6 +538,124 @@ def stream_stage(w, device, steps: int = 3000, distinct: int = 60):
 # ---------------------------------------------------------------------------
 # arms
 # ---------------------------------------------------------------------------
+def bench_config(w, world: int):
+    """The `config` object of the JSON line: the workload, its sizes and how L2 is kept out of the
+    timing. Both arms print this same object."""
+    return {"workload": WORKLOAD, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "d": w.d, "context": w.T,
+            "middle_nodes": w.N, "entries_per_head": workloads_entries(w), "query_rows_per_step": w.B * w.R * w.Hq,
+            "parallelism": f"dp{world}" if world > 1 else "single",
+            "l2": "inputs larger than L2: 6 layer caches of 76.8 MB decoded in rotation, and a 256 MB buffer "
+                  "rewritten between timed regions",
+            "timing": "CUDA graphs of back-to-back decode calls; CUDA events around each region of exactly "
+                      "`steps` calls; median over the regions, then max over ranks"}
+
+
+def workloads_entries(w) -> int:
+    import workloads
+    return workloads.N_SINK + w.N + workloads.N_RECENT
+
+
+def e2e_pipeline(w, caches, table, ws, outs, lses, device):
+    """The end-to-end step through the public API with host buffers, pipelined the way a caller
+    overlaps transfers with compute: step i's queries are copied from pinned host memory on an
+    upload stream, the decode runs on the compute stream once they have landed, and out / lse are
+    copied back to pinned host memory on a download stream. Buffers rotate over the L layer
+    slots, so step i + 1's upload and step i - 1's download overlap step i's kernel; each reuse of
+    a slot waits for the previous user of that slot. One cudaMemcpyAsync per buffer."""
+    import torch
+    import compressed_decode_attention_equal_b200 as skv
+    L = len(caches)
+    q_host = [c["q"].cpu().pin_memory() for c in caches]
+    out_host = [torch.empty_like(q, device="cpu").pin_memory() for q in q_host]
+    lse_host = [torch.empty(w.B, w.R, w.Hq, dtype=torch.float32).pin_memory() for _ in caches]
+    q_dev = [torch.empty_like(c["q"]) for c in caches]
+    up, down = torch.cuda.Stream(device), torch.cuda.Stream(device)
+    h2d_done = [torch.cuda.Event() for _ in range(L)]
+    k_done = [torch.cuda.Event() for _ in range(L)]
+    d2h_done = [torch.cuda.Event() for _ in range(L)]
+
+    def step(i, start):
+        """Step i of a captured sequence that began at step `start` (slot waits reach back only to
+        steps of the same capture; a graph completes before the next one starts)."""
+        j = i % L
+        main = torch.cuda.current_stream()
+        if i - L >= start:
+            up.wait_event(k_done[j])            # step i - L's kernel has read q_dev[j]
+        with torch.cuda.stream(up):
+            q_dev[j].copy_(q_host[j], non_blocking=True)
+            h2d_done[j].record(up)
+        main.wait_event(h2d_done[j])
+        if i - L >= start:
+            main.wait_event(d2h_done[j])        # step i - L's outputs have left outs[j]
+        c = caches[j]
+        skv.decode_attn(q_dev[j], w.Hkv, c["pool"], table, c["lens"], out=outs[j], lse=lses[j], workspace=ws)
+        k_done[j].record(main)
+        down.wait_event(k_done[j])
+        with torch.cuda.stream(down):
+            out_host[j].copy_(outs[j], non_blocking=True)
+            lse_host[j].copy_(lses[j], non_blocking=True)
+            d2h_done[j].record(down)
+
+    def fork(main):
+        up.wait_stream(main)
+        down.wait_stream(main)
+
+    def join(main):
+        main.wait_stream(up)
+        main.wait_stream(down)
+
+    h2d = q_host[0].numel() * q_host[0].element_size()
+    d2h = out_host[0].numel() * out_host[0].element_size() + lse_host[0].numel() * 4
+    return step, fork, join, out_host, h2d, d2h
+
+
+def time_e2e_regions(step, fork, join, steps: int, dist_on: bool, regions: int, flush):
+    """time_regions for the pipelined end-to-end step: each captured graph forks the side streams
+    at its start and joins them at its end, so a region ends only when its last download has
+    landed."""
+    import torch
+
+    def graph(n, start):
+        g = torch.cuda.CUDAGraph()
+        s = torch.cuda.Stream()
+        s.wait_stream(torch.cuda.current_stream())
+        with torch.cuda.stream(s):
+            with torch.cuda.graph(g, stream=s):
+                fork(s)
+                for i in range(n):
+                    step(start + i, start)
+                join(s)
+        torch.cuda.current_stream().wait_stream(s)
+        return g
+
+    graphs, done = [], 0
+    while done < steps:
+        n = min(GRAPH_MAX_STEPS, steps - done)
+        graphs.append(graph(n, done))
+        done += n
+    for g in graphs:
+        g.replay()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(regions):
+        flush.add_(1)
+        torch.cuda.synchronize()
+        if dist_on:
+            torch.distributed.barrier()
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for g in graphs:
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize()
+        if dist_on:
+            torch.distributed.barrier()
+        times.append(e0.elapsed_time(e1))
+    del graphs
+    return times
+
+
 def run_ours(args, rank: int, world: int, device):
     import torch
     import compressed_decode_attention_equal_b200 as skv
@@ -526,6 +672,7 @@ def run_ours(args, rank: int, world: int, device):
     lses = [torch.empty(w.B, w.R, w.Hq, dtype=torch.float32, device=device) for _ in caches]
     ws = torch.zeros(skv.decode_workspace_bytes(w.B, w.R, w.Hq, w.Hkv, w.d, table.shape[2]), dtype=torch.uint8,
                      device=device)
+    flush = l2_flush_buffer(device)
 
     def step(i):
         c = caches[i % L]
@@ -541,50 +688,41 @@ def run_ours(args, rank: int, world: int, device):
     sampler = ClockSampler(torch.cuda.current_device()) if rank == 0 else None
     if sampler:
         sampler.start()
-    ms = time_graphs(step, args.steps, L, dist_on)
+    times = time_regions(step, args.steps, dist_on, args.regions, flush=flush)
     clocks = sampler.stop() if sampler else None
-    ms = max_over_ranks(ms, device, world)
+    stats = summarise_regions(times, args.steps)
+    ms = max_over_ranks(stats["median_us"] * args.steps / 1e3, device, world)   # median region, slowest rank
     ms_per_step = ms / args.steps
     value = job_throughput(rows_per_step, world, args.steps, ms)
 
-    # end to end: pinned host queries in, pinned host outputs back, every step
-    q_host = [c["q"].cpu().pin_memory() for c in caches]
-    out_host = [torch.empty_like(q, device="cpu").pin_memory() for q in q_host]
-    lse_host = [torch.empty(w.B, w.R, w.Hq, dtype=torch.float32).pin_memory() for _ in caches]
-    q_dev = [torch.empty_like(c["q"]) for c in caches]
-
-    def e2e_step(i):
-        j = i % L
-        q_dev[j].copy_(q_host[j], non_blocking=True)
-        c = caches[j]
-        skv.decode_attn(q_dev[j], w.Hkv, c["pool"], table, c["lens"], out=outs[j], lse=lses[j], workspace=ws)
-        out_host[j].copy_(outs[j], non_blocking=True)
-        lse_host[j].copy_(lses[j], non_blocking=True)
-
-    for i in range(min(args.warmup, 3 * L)):
-        e2e_step(i)
-    e2e_steps = max(L, min(args.steps, 20000))
-    e2e_ms = time_graphs(e2e_step, e2e_steps, L, dist_on)
-    e2e_ms = max_over_ranks(e2e_ms, device, world)
-    # the timed copies are real: the last step's outputs match the device results
+    # end to end through the public API with host buffers, transfers pipelined with the kernels
+    e2e_step, e2e_fork, e2e_join, out_host, h2d, d2h = e2e_pipeline(w, caches, table, ws, outs, lses, device)
+    e2e_steps = max(L, args.steps)
+    e2e_regions = max(3, min(args.regions, 10))
+    e2e_stats = summarise_regions(time_e2e_regions(e2e_step, e2e_fork, e2e_join, e2e_steps, dist_on, e2e_regions, flush),
+                                  e2e_steps)
+    e2e_ms = max_over_ranks(e2e_stats["median_us"] * e2e_steps / 1e3, device, world)
+    # the timed copies are real: the last step's outputs landed in host memory
     torch.cuda.synchronize()
-    assert torch.equal(out_host[(e2e_steps - 1) % L], outs[(e2e_steps - 1) % L].cpu())
+    last = (e2e_steps - 1) % L
+    assert torch.equal(out_host[last], outs[last].cpu())
 
     result = None
     if rank == 0:
         peak, src = _peaks()
         achieved = alg_bytes / (ms_per_step / 1e3) / 1e9
         launches_per_step = 1   # one decode kernel per call
+        sm_ghz = clocks["sm_mhz"] / 1e3 if clocks else None
         result = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
             "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "bf16",
             "data": "synthetic: regime-walk keys, N(0,1) values and queries, coarsened on the GPU by this library",
-            "config": {"workload": WORKLOAD, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "d": w.d,
-                       "context": w.T, "middle_nodes": w.N, "entries_per_head": ent // (w.B * w.Hkv),
-                       "query_rows_per_step": rows_per_step, "parallelism": f"dp{world}" if world > 1 else "single",
-                       "l2": f"inputs larger than L2: {L} layer caches of {alg_bytes / 1e6:.1f} MB rotated",
-                       "timing": "CUDA graphs of back-to-back decode calls, CUDA events around the replay"},
+            "config": bench_config(w, world),
+            "timing": dict(stats, note=f"{args.regions} timed regions of exactly {args.steps} calls; value uses "
+                                       "the median region (max over ranks)",
+                           us_x_sm_ghz=stats["median_us"] * sm_ghz if sm_ghz else None),
+            "entries_per_step": ent,
             "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                          "traffic": _profile_traffic("decode_gqa7_32k_summary.md", DECODE_SOURCES),
                          "peak_source": f"{src} HBM copy bandwidth (MEASURED_PEAKS.json hbm_gbs)"
@@ -592,10 +730,12 @@ def run_ours(args, rank: int, world: int, device):
                          "frac_of_8tbs": achieved / 8000.0, "algorithmic_bytes_per_launch": alg_bytes,
                          "kernel": "k_decode_split (one launch per call), time per call"},
             "e2e": {"value": job_throughput(rows_per_step, world, e2e_steps, e2e_ms), "unit": UNIT,
-                    "h2d_bytes_per_step": q_host[0].numel() * q_host[0].element_size(),
-                    "d2h_bytes_per_step": out_host[0].numel() * out_host[0].element_size() + lse_host[0].numel() * 4,
-                    "steps": e2e_steps},
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": e2e_steps,
+                    "timing": e2e_stats,
+                    "note": "pinned host queries in and out / lse back every step through the public API; "
+                            "uploads and downloads on their own streams overlap the neighbouring steps' kernels"},
             "gpu_launches": launches_per_step * args.steps,
+            "gpu_launches_note": "decode kernels per timed region (one per step)",
             "clocks": clocks,
             "coarsen_build_ms_per_layer": coarsen_ms,
         }
@@ -664,7 +804,7 @@ def run_reference(args, rank: int, world: int = 1):
         t0 = time.perf_counter()
         step(0, per_unit, ex)
         per_row = max((time.perf_counter() - t0) / per_unit, 1e-6)
-        budget = 60.0 / max(1, args.steps + args.warmup)
+        budget = args.ref_seconds / max(1, args.steps + args.warmup)
         n = int(max(1, min(total, budget / per_row)))
         pos, used = 0, 1
         for _ in range(args.warmup):
@@ -683,21 +823,36 @@ def run_reference(args, rank: int, world: int = 1):
         "warmup": args.warmup,
         "ms_per_step": dt * 1e3 / args.steps, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
         "dtype": "f64", "data": "synthetic entries with the workload's shape", "impl": "reference",
-        "config": {"workload": WORKLOAD, "batch": w.B, "q_heads": w.Hq, "kv_heads": w.Hkv, "d": w.d,
-                   "context": w.T, "middle_nodes": w.N, "entries_per_head": E},
+        "config": bench_config(w, world),
         "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
                          "sample": f"{n} of the batch's {total} query rows per step, each against {E} entries"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
 
 
+def free_port() -> int:
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def relaunch_command(args_argv, gpus: int, port: int):
+    """The torch.distributed.run command that runs this script as `gpus` ranks on this node."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={gpus}",
+            "--master-addr=127.0.0.1", f"--master-port={port}", os.path.abspath(__file__), *args_argv]
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=60000)
-    ap.add_argument("--warmup", type=int, default=600)
+    ap.add_argument("--steps", type=int, default=2000, help="calls per timed region")
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--regions", type=int, default=30, help="timed regions of --steps calls (median reported)")
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--layers", type=int, default=6)
+    ap.add_argument("--ref-seconds", type=float, default=60.0,
+                    help="reference arm: host seconds that warm-up plus steps are sized to")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-coarsen", action="store_true")
     ap.add_argument("--no-diagonal", action="store_true", help="skip the diagonal-closure decode timing")
@@ -706,8 +861,19 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+    if args.gpus < 1 or args.regions < 1 or args.steps < 1:
+        ap.error("--gpus, --regions and --steps must be >= 1")
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if "WORLD_SIZE" not in os.environ:
+        if args.gpus > 1:
+            # one process per GPU: run this script as --gpus ranks under torch.distributed.run
+            rc = subprocess.call(relaunch_command(sys.argv[1:], args.gpus, free_port()))
+            raise SystemExit(rc)
+        world = 1
+    else:
+        world = int(os.environ["WORLD_SIZE"])
+        if world != args.gpus:
+            raise SystemExit(f"bench.py: --gpus {args.gpus} but WORLD_SIZE={world}; launch one rank per GPU")
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
 

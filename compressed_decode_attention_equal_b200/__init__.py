@@ -117,14 +117,20 @@ def coarsen_workspace_bytes(Hkv: int, d: int, T_list, N_list, n_sink: int, n_rec
 def coarsen(k: torch.Tensor, v: torch.Tensor, Hkv: int, T_list, N_list, n_sink: int, n_recent: int,
             proj_seed: int, pool: NodePool, page_table: torch.Tensor, lens: torch.Tensor | None = None,
             boundaries: torch.Tensor | None = None, cumvar: torch.Tensor | None = None,
-            workspace: torch.Tensor | None = None, stream=None, representative: str = "mean") -> torch.Tensor:
+            workspace: torch.Tensor | None = None, stream=None, representative: str = "mean",
+            center_keys: bool = False, projection: str = "fixed") -> torch.Tensor:
     """Coarsen B sequences (k, v: [sum_b Hkv*T_b, d], sequence b a contiguous [Hkv, T_b, d] block)
     into `pool` through `page_table` [B, Hkv, max_pages] int32. Returns lens [B, Hkv] int32.
     representative: "mean" (skv_coarsen) or "variation" (skv_coarsen_ex with the
-    variation-weighted segment key and value)."""
+    variation-weighted segment key and value). center_keys: skv_coarsen_ex's common-mode mean
+    removal (every key of a unit enters with the unit's mean key subtracted). projection: "fixed"
+    (the fixed fp32 recipe) or "tensor" (skv_coarsen_ex's tensor-core bf16 projection)."""
     reps = {"mean": _lib.SKV_REP_MEAN, "variation": _lib.SKV_REP_VARIATION_WEIGHTED}
+    projs = {"fixed": _lib.SKV_PROJECTION_FIXED_FP32, "tensor": _lib.SKV_PROJECTION_TENSOR_BF16}
     if representative not in reps:
         raise ValueError(f"representative must be one of {sorted(reps)}")
+    if projection not in projs:
+        raise ValueError(f"projection must be one of {sorted(projs)}")
     B = len(T_list)
     d = k.shape[-1]
     if v.shape != k.shape or v.dtype != k.dtype:
@@ -149,11 +155,12 @@ def coarsen(k: torch.Tensor, v: torch.Tensor, Hkv: int, T_list, N_list, n_sink: 
             _dev(boundaries, "boundaries") if boundaries is not None else null,
             _dev(cumvar, "cumvar") if cumvar is not None else null,
             _dev(workspace, "workspace"), workspace.numel())
-    if representative == "mean" and pool.closure == "scalar":
+    if representative == "mean" and pool.closure == "scalar" and not center_keys and projection == "fixed":
         st = _lib.load().skv_coarsen(*args, ctypes.c_void_p(_stream_handle(stream)))
         _lib.check(st, "skv_coarsen")
     else:
-        opts = _lib.SkvCoarsenOptions(reps[representative], CLOSURES[pool.closure])
+        opts = _lib.SkvCoarsenOptions(reps[representative], CLOSURES[pool.closure], 1 if center_keys else 0,
+                                      projs[projection])
         st = _lib.load().skv_coarsen_ex(*args, ctypes.byref(opts), ctypes.c_void_p(_stream_handle(stream)))
         _lib.check(st, "skv_coarsen_ex")
     return lens

@@ -9,7 +9,7 @@ LIB_PATH = os.path.join(_PKG, "libskv.so")
 
 SKV_OK = 0
 SKV_ERR_INVALID_ARG, SKV_ERR_UNSUPPORTED, SKV_ERR_CUDA, SKV_ERR_OVERFLOW = -1, -2, -3, -4
-SKV_ERR_WORKSPACE, SKV_ERR_DEVICE = -6, -7
+SKV_ERR_TIMEOUT, SKV_ERR_WORKSPACE, SKV_ERR_DEVICE = -5, -6, -7
 SKV_F32, SKV_BF16 = 0, 1
 PAGE_NODES = 16
 PROJ_DIM = 16
@@ -25,10 +25,12 @@ class SkvNodePool(ctypes.Structure):
 
 SKV_REP_MEAN, SKV_REP_VARIATION_WEIGHTED = 0, 1
 SKV_CLOSURE_SCALAR, SKV_CLOSURE_DIAGONAL = 0, 1
+SKV_PROJECTION_FIXED_FP32, SKV_PROJECTION_TENSOR_BF16 = 0, 1
 
 
 class SkvCoarsenOptions(ctypes.Structure):
-    _fields_ = [("representative", ctypes.c_int32), ("closure", ctypes.c_int32), ("reserved", ctypes.c_int32 * 6)]
+    _fields_ = [("representative", ctypes.c_int32), ("closure", ctypes.c_int32), ("center_keys", ctypes.c_int32),
+                ("projection", ctypes.c_int32), ("reserved", ctypes.c_int32 * 4)]
 
 
 class SkvDecodeOptions(ctypes.Structure):
@@ -46,7 +48,7 @@ EXPORTS = ("skv_status_string", "skv_abi_version", "skv_page_bytes", "skv_page_b
            "skv_coarsen_workspace_bytes",
            "skv_coarsen", "skv_coarsen_ex", "skv_decode_workspace_bytes", "skv_decode_attn", "skv_decode_attn_ex", "skv_decode_attn_noalloc",
            "skv_stream_state_bytes", "skv_stream_init", "skv_stream_append",
-           "skv_workspace_error")
+           "skv_workspace_error", "skv_wait_selftest")
 
 _lib = None
 
@@ -102,6 +104,8 @@ def load(path: str = LIB_PATH) -> ctypes.CDLL:
     lib.skv_decode_attn_noalloc.restype = i32
     lib.skv_workspace_error.argtypes = [vp, vp, ctypes.POINTER(ctypes.c_uint32)]
     lib.skv_workspace_error.restype = i32
+    lib.skv_wait_selftest.argtypes = [vp, sz, ctypes.c_uint32, vp]
+    lib.skv_wait_selftest.restype = i32
     _lib = lib
     return lib
 

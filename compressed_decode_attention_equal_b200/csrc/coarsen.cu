@@ -33,6 +33,46 @@ __global__ void k_setup(const __grid_constant__ SeqTable table, SeqRow *dst, int
 }
 
 // ---------------------------------------------------------------------------
+// centring option ("SPICY-KV" Independent Claim 1(b), common-mode mean removal): the unit's
+// mean key in one fixed fp32 order -- per dimension, blocks of kMeanBlock consecutive tokens
+// summed in token order from 0, block sums added in block order from 0, total divided by T
+// -- so that the centred keys fl32(k - mu) are the same bits wherever they are formed.
+// ---------------------------------------------------------------------------
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) { return __bfloat162float(x); }
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) { return x; }
+
+// one thread per key dimension, one CTA per (block of kMeanBlock tokens, unit)
+template <int D, typename T>
+__global__ void __launch_bounds__(D) k_key_block_sums(const CoarsenArgs a) {
+    const int u = blockIdx.y, blk = blockIdx.x;
+    const int b = u / a.Hkv, h = u % a.Hkv;
+    const SeqRow sr = a.seq[b];
+    const int t0 = blk * kMeanBlock;
+    if (t0 >= sr.T) return;
+    const int n = min(kMeanBlock, sr.T - t0);
+    const T *kp = static_cast<const T *>(a.k) + (sr.row_off + static_cast<int64_t>(h) * sr.T + t0) * D + threadIdx.x;
+    float s = 0.0f;
+#pragma unroll 16
+    for (int t = 0; t < n; ++t) s = __fadd_rn(s, to_f32<T>(kp[static_cast<int64_t>(t) * D]));
+    a.key_blk[(static_cast<int64_t>(u) * a.max_blk + blk) * D + threadIdx.x] = s;
+}
+
+template <int D>
+__global__ void __launch_bounds__(D) k_key_mean(const CoarsenArgs a) {
+    const int u = blockIdx.x;
+    const SeqRow sr = a.seq[u / a.Hkv];
+    const int nblk = (sr.T + kMeanBlock - 1) / kMeanBlock;
+    const float *bs = a.key_blk + static_cast<int64_t>(u) * a.max_blk * D + threadIdx.x;
+    float tot = 0.0f;
+    for (int c = 0; c < nblk; ++c) tot = __fadd_rn(tot, bs[static_cast<int64_t>(c) * D]);
+    a.key_mu[static_cast<int64_t>(u) * D + threadIdx.x] = sr.T > 0 ? __fdiv_rn(tot, static_cast<float>(sr.T)) : 0.0f;
+}
+
+// ---------------------------------------------------------------------------
 // k_project_scan
 // ---------------------------------------------------------------------------
 
@@ -48,7 +88,8 @@ static_assert(kTileRows % kK1BoxRows == 0 && kTileRows * kZStride * 4 <= kK1Stag
 template <int D>
 constexpr size_t k1_smem_bytes() {
     // stages + P^T with one zero row of padding (the pipelined loop reads row j + 1) + barriers
-    return 1024 /*alignment slack*/ + kK1Stages * kK1StageBytes + (2 * D + 1) * kProjDim * sizeof(float) + 64 + 64;
+    return 1024 /*alignment slack*/ + kK1Stages * kK1StageBytes + (2 * D + 1) * kProjDim * sizeof(float) + 64 + 64 +
+           D * sizeof(float);
 }
 
 // x duplicated into both halves of an f32x2 operand, built with two different ALU operations (the
@@ -79,113 +120,12 @@ __device__ __forceinline__ uint64_t dup_elem<float>(const uint4 &w, int e) {
 // (sub-chunk index XOR bits [1:2] of the row: bank-conflict free for 8 consecutive rows)
 __device__ __forceinline__ int k1_sub(int r, int cc) { return r * 4 + (cc ^ ((r >> 1) & 3)); }
 
-template <int D, typename T>
-__global__ void __launch_bounds__(kK1Threads, 2)
-    k_project_scan(const CoarsenArgs a, const __grid_constant__ CUtensorMap map_k,
-                   const __grid_constant__ CUtensorMap map_v, const __grid_constant__ ProjT proj) {
-    constexpr int ELEM = sizeof(T);
-    constexpr int KCHUNK = D * ELEM / kK1ColBytes;   // column chunks of one key row
-    constexpr int NCHUNK = 2 * KCHUNK;               // key chunks, then value chunks
-    constexpr int JPC = kK1ColBytes / ELEM;          // feature index j per chunk
-    constexpr int EPS = 16 / ELEM;                   // elements per 16-byte sub-chunk
-
-    extern __shared__ uint8_t smem_raw[];
-    const uint32_t raw = smem_u32(smem_raw);
-    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
-    uint8_t *stages = smem;
-    float *pt = reinterpret_cast<float *>(smem + kK1Stages * kK1StageBytes);
-    uint64_t *bar = reinterpret_cast<uint64_t *>(pt + (2 * D + 1) * kProjDim);
-    long long *warp_sum = reinterpret_cast<long long *>(bar + 8);
-
-    const int u = blockIdx.y;
-    const int tile = blockIdx.x;
-    const int b = u / a.Hkv, h = u % a.Hkv;
-    const SeqRow sr = a.seq[b];
-    if (tile >= sr.tiles) return;
+// Quantised steps and the tile-local inclusive scan of one projection tile (z of its 512 rows in
+// shared memory, row 0 the halo): D_t = rne(||z_t - z_{t-1}|| 2^20) by the fixed recipe for the
+// tile's middle tokens, their running sums into local_scan, the tile total into tile_total.
+__device__ __forceinline__ void scan_tile(const CoarsenArgs &a, const SeqRow &sr, int u, int h, int tile,
+                                          const float *zb, long long *warp_sum) {
     const int tid = threadIdx.x;
-
-    const int y0 = static_cast<int>(sr.row_off + static_cast<int64_t>(h) * sr.T + sr.s_eff) + tile * kTileOut - 1;
-    auto issue = [&](int c, int s) {
-        mbar_arrive_expect_tx(&bar[s], kK1StageBytes);
-        const CUtensorMap *map = c < KCHUNK ? &map_k : &map_v;
-#pragma unroll
-        for (int hb = 0; hb < kTileRows / kK1BoxRows; ++hb)
-            tma_load_2d(stages + s * kK1StageBytes + hb * kK1BoxRows * kK1ColBytes, map, (c % KCHUNK) * JPC,
-                        y0 + hb * kK1BoxRows, &bar[s]);
-    };
-    if (tid == 0) {
-        prefetch_tensormap(&map_k);
-        prefetch_tensormap(&map_v);
-        for (int s = 0; s < kK1Stages; ++s) mbar_init(&bar[s], 1);
-        fence_mbar_init();
-        for (int c = 0; c < NCHUNK && c < kK1Stages; ++c) issue(c, c);
-    }
-    for (int i = tid; i < (2 * D + 1) * kProjDim; i += kK1Threads) pt[i] = i < 2 * D * kProjDim ? proj.pt[i] : 0.0f;
-    __syncthreads();
-
-    // rows tid + 128 t (t < 4) of the tile; each feature's P^T row is read once per 4 tokens
-    uint64_t acc[kK1Tok][kProjDim / 2];
-#pragma unroll
-    for (int t = 0; t < kK1Tok; ++t)
-#pragma unroll
-        for (int i = 0; i < kProjDim / 2; ++i) acc[t][i] = 0ull;
-    const float4 *ptv = reinterpret_cast<const float4 *>(pt);   // P^T row j = ptv[4 j .. 4 j + 3]
-    // software pipeline: the P^T row of feature j + 1 and the next 16-byte sub-chunk of the rows
-    // are read while feature j is accumulated (plain shared loads: never hoisted above the wait)
-    float4 pc[4];
-#pragma unroll
-    for (int q4 = 0; q4 < 4; ++q4) pc[q4] = ptv[q4];
-
-    bool ok = true;
-    for (int c = 0; c < NCHUNK; ++c) {
-        const int s = c % kK1Stages;
-        if (ok && !mbar_wait(&bar[s], (c / kK1Stages) & 1)) ok = false;
-        const uint4 *st = reinterpret_cast<const uint4 *>(stages + s * kK1StageBytes);
-        uint4 x[kK1Tok];
-#pragma unroll
-        for (int t = 0; t < kK1Tok; ++t) x[t] = st[k1_sub(tid + t * kK1Threads, 0)];
-#pragma unroll 1
-        for (int cc = 0; cc < 4; ++cc) {
-            const int ccn = cc < 3 ? cc + 1 : 3;
-            uint4 xn[kK1Tok];
-#pragma unroll
-            for (int t = 0; t < kK1Tok; ++t) xn[t] = st[k1_sub(tid + t * kK1Threads, ccn)];
-#pragma unroll
-            for (int e = 0; e < EPS; ++e) {
-                const int j = c * JPC + cc * EPS + e;
-                float4 pn[4];
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) pn[q4] = ptv[4 * (j + 1) + q4];
-#pragma unroll
-                for (int t = 0; t < kK1Tok; ++t) {
-                    const uint64_t xx = dup_elem<T>(x[t], e);
-#pragma unroll
-                    for (int q4 = 0; q4 < 4; ++q4) {
-                        acc[t][2 * q4] = ffma2(f2pack(pc[q4].x, pc[q4].y), xx, acc[t][2 * q4]);
-                        acc[t][2 * q4 + 1] = ffma2(f2pack(pc[q4].z, pc[q4].w), xx, acc[t][2 * q4 + 1]);
-                    }
-                }
-#pragma unroll
-                for (int q4 = 0; q4 < 4; ++q4) pc[q4] = pn[q4];
-            }
-#pragma unroll
-            for (int t = 0; t < kK1Tok; ++t) x[t] = xn[t];
-        }
-        __syncthreads();
-        if (tid == 0 && c + kK1Stages < NCHUNK) issue(c + kK1Stages, s);
-    }
-    if (!ok) raise_flag(a.flags, FLAG_TIMEOUT);
-
-    // z of the rows -> shared (the stages are free: every chunk has been consumed and synced)
-    float *zb = reinterpret_cast<float *>(stages);
-#pragma unroll
-    for (int t = 0; t < kK1Tok; ++t) {
-        const int r = tid + t * kK1Threads;
-#pragma unroll
-        for (int i = 0; i < kProjDim / 2; ++i) f2unpack(acc[t][i], zb[r * kZStride + 2 * i], zb[r * kZStride + 2 * i + 1]);
-    }
-    __syncthreads();
-
     // outputs l = 4 tid + 1 .. 4 tid + 4 (rows of the tile; row 0 is the halo)
     long long Dv[kK1Tok];
 #pragma unroll
@@ -228,6 +168,256 @@ __global__ void __launch_bounds__(kK1Threads, 2)
         if (l <= kTileOut && t < sr.M) ls[t] = run;
     }
     if (tid == kK1Threads - 1) a.tile_total[static_cast<int64_t>(u) * a.max_tiles + tile] = incl;
+}
+
+// CENTER: the key features enter as fl32(k - mu) (the centring option)
+template <int D, typename T, bool CENTER>
+__global__ void __launch_bounds__(kK1Threads, 2)
+    k_project_scan(const CoarsenArgs a, const __grid_constant__ CUtensorMap map_k,
+                   const __grid_constant__ CUtensorMap map_v, const __grid_constant__ ProjT proj) {
+    constexpr int ELEM = sizeof(T);
+    constexpr int KCHUNK = D * ELEM / kK1ColBytes;   // column chunks of one key row
+    constexpr int NCHUNK = 2 * KCHUNK;               // key chunks, then value chunks
+    constexpr int JPC = kK1ColBytes / ELEM;          // feature index j per chunk
+    constexpr int EPS = 16 / ELEM;                   // elements per 16-byte sub-chunk
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t *stages = smem;
+    float *pt = reinterpret_cast<float *>(smem + kK1Stages * kK1StageBytes);
+    uint64_t *bar = reinterpret_cast<uint64_t *>(pt + (2 * D + 1) * kProjDim);
+    long long *warp_sum = reinterpret_cast<long long *>(bar + 8);
+    float *mus = reinterpret_cast<float *>(warp_sum + 8);   // the unit's mean key (CENTER)
+
+    const int u = blockIdx.y;
+    const int tile = blockIdx.x;
+    const int b = u / a.Hkv, h = u % a.Hkv;
+    const SeqRow sr = a.seq[b];
+    if (tile >= sr.tiles) return;
+    const int tid = threadIdx.x;
+
+    const int y0 = static_cast<int>(sr.row_off + static_cast<int64_t>(h) * sr.T + sr.s_eff) + tile * kTileOut - 1;
+    auto issue = [&](int c, int s) {
+        mbar_arrive_expect_tx(&bar[s], kK1StageBytes);
+        const CUtensorMap *map = c < KCHUNK ? &map_k : &map_v;
+#pragma unroll
+        for (int hb = 0; hb < kTileRows / kK1BoxRows; ++hb)
+            tma_load_2d(stages + s * kK1StageBytes + hb * kK1BoxRows * kK1ColBytes, map, (c % KCHUNK) * JPC,
+                        y0 + hb * kK1BoxRows, &bar[s]);
+    };
+    if (tid == 0) {
+        prefetch_tensormap(&map_k);
+        prefetch_tensormap(&map_v);
+        for (int s = 0; s < kK1Stages; ++s) mbar_init(&bar[s], 1);
+        fence_mbar_init();
+        for (int c = 0; c < NCHUNK && c < kK1Stages; ++c) issue(c, c);
+    }
+    for (int i = tid; i < (2 * D + 1) * kProjDim; i += kK1Threads) pt[i] = i < 2 * D * kProjDim ? proj.pt[i] : 0.0f;
+    if constexpr (CENTER)
+        for (int i = tid; i < D; i += kK1Threads) mus[i] = a.key_mu[static_cast<int64_t>(u) * D + i];
+    __syncthreads();
+
+    // rows tid + 128 t (t < 4) of the tile; each feature's P^T row is read once per 4 tokens
+    uint64_t acc[kK1Tok][kProjDim / 2];
+#pragma unroll
+    for (int t = 0; t < kK1Tok; ++t)
+#pragma unroll
+        for (int i = 0; i < kProjDim / 2; ++i) acc[t][i] = 0ull;
+    const float4 *ptv = reinterpret_cast<const float4 *>(pt);   // P^T row j = ptv[4 j .. 4 j + 3]
+    // software pipeline: the P^T row of feature j + 1 and the next 16-byte sub-chunk of the rows
+    // are read while feature j is accumulated (plain shared loads: never hoisted above the wait)
+    float4 pc[4];
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) pc[q4] = ptv[q4];
+
+    for (int c = 0; c < NCHUNK; ++c) {
+        const int s = c % kK1Stages;
+        const bool got = mbar_wait(&bar[s], (c / kK1Stages) & 1);
+        const uint4 *st = reinterpret_cast<const uint4 *>(stages + s * kK1StageBytes);
+        uint4 x[kK1Tok];
+#pragma unroll
+        for (int t = 0; t < kK1Tok; ++t) x[t] = st[k1_sub(tid + t * kK1Threads, 0)];
+#pragma unroll 1
+        for (int cc = 0; cc < 4; ++cc) {
+            const int ccn = cc < 3 ? cc + 1 : 3;
+            uint4 xn[kK1Tok];
+#pragma unroll
+            for (int t = 0; t < kK1Tok; ++t) xn[t] = st[k1_sub(tid + t * kK1Threads, ccn)];
+#pragma unroll
+            for (int e = 0; e < EPS; ++e) {
+                const int j = c * JPC + cc * EPS + e;
+                float4 pn[4];
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) pn[q4] = ptv[4 * (j + 1) + q4];
+                float mu_j = 0.0f;
+                if constexpr (CENTER) mu_j = mus[c < KCHUNK ? j : 0];   // value chunks: unused
+#pragma unroll
+                for (int t = 0; t < kK1Tok; ++t) {
+                    uint64_t xx;
+                    if constexpr (CENTER) {
+                        float lo, hi;
+                        f2unpack(dup_elem<T>(x[t], e), lo, hi);
+                        const float xc = c < KCHUNK ? __fsub_rn(lo, mu_j) : lo;
+                        xx = f2pack(xc, xc);
+                    } else {
+                        xx = dup_elem<T>(x[t], e);
+                    }
+#pragma unroll
+                    for (int q4 = 0; q4 < 4; ++q4) {
+                        acc[t][2 * q4] = ffma2(f2pack(pc[q4].x, pc[q4].y), xx, acc[t][2 * q4]);
+                        acc[t][2 * q4 + 1] = ffma2(f2pack(pc[q4].z, pc[q4].w), xx, acc[t][2 * q4 + 1]);
+                    }
+                }
+#pragma unroll
+                for (int q4 = 0; q4 < 4; ++q4) pc[q4] = pn[q4];
+            }
+#pragma unroll
+            for (int t = 0; t < kK1Tok; ++t) x[t] = xn[t];
+        }
+        // every thread's wait verdict: if any wait gave up, the CTA issues no further copy, thread 0
+        // waits (bounded) for the copies already in flight into its shared memory (chunks c and
+        // c + 1), and the tile writes nothing
+        if (!__syncthreads_and(got)) {
+            if (tid == 0) {
+                for (int c2 = c; c2 < NCHUNK && c2 <= c + 1; ++c2)
+                    (void)mbar_wait(&bar[c2 % kK1Stages], (c2 / kK1Stages) & 1);
+                raise_flag(a.flags, FLAG_TIMEOUT);
+            }
+            return;
+        }
+        if (tid == 0 && c + kK1Stages < NCHUNK) issue(c + kK1Stages, s);
+    }
+
+    // z of the rows -> shared (the stages are free: every chunk has been consumed and synced)
+    float *zb = reinterpret_cast<float *>(stages);
+#pragma unroll
+    for (int t = 0; t < kK1Tok; ++t) {
+        const int r = tid + t * kK1Threads;
+#pragma unroll
+        for (int i = 0; i < kProjDim / 2; ++i) f2unpack(acc[t][i], zb[r * kZStride + 2 * i], zb[r * kZStride + 2 * i + 1]);
+    }
+    __syncthreads();
+
+    scan_tile(a, sr, u, h, tile, zb, warp_sum);
+}
+
+// ---------------------------------------------------------------------------
+// k_project_tc (option SKV_PROJECTION_TENSOR_BF16): the same tiles, TMA staging and scan, but
+// z = P16 x on the tensor cores: P16 = bf16(P), x the bf16 features, fp32 accumulation
+// (mma.sync m16n8k16; tokens as M, the 16 outputs as two n8 tiles, features as K). Each warp owns
+// 128 rows of the tile (8 m-tiles); P16's B fragments stay in registers for the whole tile. The
+// products are exact; only the accumulation order and rounding differ from the fixed recipe, so
+// the quantised steps differ from it by a bounded amount and the boundaries follow the steps the
+// tensor cores produced.
+// ---------------------------------------------------------------------------
+template <int D>
+__global__ void __launch_bounds__(kK1Threads, 2)
+    k_project_tc(const CoarsenArgs a, const __grid_constant__ CUtensorMap map_k,
+                 const __grid_constant__ CUtensorMap map_v, const __grid_constant__ ProjFrag pf) {
+    constexpr int KCHUNK = D * 2 / kK1ColBytes;      // bf16 column chunks of one key row
+    constexpr int NCHUNK = 2 * KCHUNK;               // key chunks, then value chunks
+    constexpr int KPC = kK1ColBytes / 32;            // k-steps of 16 features per chunk
+    constexpr int NKS = NCHUNK * KPC;                // k-steps over the 2d features
+    constexpr int MT = kTileRows / 16 / (kK1Threads / 32);   // m-tiles of 16 rows per warp (8)
+    static_assert(NKS * 16 == 2 * D, "k-steps cover the features");
+
+    extern __shared__ uint8_t smem_raw[];
+    const uint32_t raw = smem_u32(smem_raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t *stages = smem;
+    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kK1Stages * kK1StageBytes);
+    long long *warp_sum = reinterpret_cast<long long *>(bar + 8);
+
+    const int u = blockIdx.y;
+    const int tile = blockIdx.x;
+    const int b = u / a.Hkv, h = u % a.Hkv;
+    const SeqRow sr = a.seq[b];
+    if (tile >= sr.tiles) return;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+
+    const int y0 = static_cast<int>(sr.row_off + static_cast<int64_t>(h) * sr.T + sr.s_eff) + tile * kTileOut - 1;
+    auto issue = [&](int c, int s) {
+        mbar_arrive_expect_tx(&bar[s], kK1StageBytes);
+        const CUtensorMap *map = c < KCHUNK ? &map_k : &map_v;
+#pragma unroll
+        for (int hb = 0; hb < kTileRows / kK1BoxRows; ++hb)
+            tma_load_2d(stages + s * kK1StageBytes + hb * kK1BoxRows * kK1ColBytes, map, (c % KCHUNK) * 32,
+                        y0 + hb * kK1BoxRows, &bar[s]);
+    };
+    if (tid == 0) {
+        prefetch_tensormap(&map_k);
+        prefetch_tensormap(&map_v);
+        for (int s = 0; s < kK1Stages; ++s) mbar_init(&bar[s], 1);
+        fence_mbar_init();
+        for (int c = 0; c < NCHUNK && c < kK1Stages; ++c) issue(c, c);
+    }
+    uint32_t bf[NKS][2][2];   // P16^T fragments: k-step, n-tile, register
+#pragma unroll
+    for (int ks = 0; ks < NKS; ++ks)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            bf[ks][nt][0] = pf.w[((ks * 2 + nt) * 32 + lane) * 2];
+            bf[ks][nt][1] = pf.w[((ks * 2 + nt) * 32 + lane) * 2 + 1];
+        }
+    float zacc[MT][2][4];
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) zacc[mt][nt][0] = zacc[mt][nt][1] = zacc[mt][nt][2] = zacc[mt][nt][3] = 0.0f;
+    __syncthreads();   // barriers initialised
+
+    // ldmatrix rows of this lane: matrices 0 / 1 are rows 0-7 / 8-15 of an m-tile at the k-step's
+    // first 8 features, matrices 2 / 3 the same rows at its last 8
+    const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1), lhalf = lane >> 4;
+#pragma unroll
+    for (int c = 0; c < NCHUNK; ++c) {
+        const int s = c % kK1Stages;
+        const bool got = mbar_wait(&bar[s], (c / kK1Stages) & 1);
+        const uint32_t sb = smem_u32(stages + s * kK1StageBytes);
+#pragma unroll
+        for (int kk = 0; kk < KPC; ++kk) {
+            const int ks = c * KPC + kk;
+            const int cc = 2 * kk + lhalf;   // 16-byte sub-chunk of the 64-byte chunk row
+#pragma unroll
+            for (int mt = 0; mt < MT; ++mt) {
+                const int row = warp * (MT * 16) + mt * 16 + lrow;
+                uint32_t a0, a1, a2, a3;
+                ldsm_x4(sb + row * kK1ColBytes + ((cc ^ ((row >> 1) & 3)) << 4), a0, a1, a2, a3);
+                mma_bf16(zacc[mt][0], a0, a1, a2, a3, bf[ks][0][0], bf[ks][0][1]);
+                mma_bf16(zacc[mt][1], a0, a1, a2, a3, bf[ks][1][0], bf[ks][1][1]);
+            }
+        }
+        // as in k_project_scan: a wait that gave up stops the tile after the copies in flight land
+        if (!__syncthreads_and(got)) {
+            if (tid == 0) {
+                for (int c2 = c; c2 < NCHUNK && c2 <= c + 1; ++c2)
+                    (void)mbar_wait(&bar[c2 % kK1Stages], (c2 / kK1Stages) & 1);
+                raise_flag(a.flags, FLAG_TIMEOUT);
+            }
+            return;
+        }
+        if (tid == 0 && c + kK1Stages < NCHUNK) issue(c + kK1Stages, s);
+    }
+
+    // z of the rows -> shared: accumulator (mt, nt) holds tokens row0 + g, row0 + g + 8 and
+    // outputs 8 nt + 2 c4, 8 nt + 2 c4 + 1
+    float *zb = reinterpret_cast<float *>(stages);
+    const int g = lane >> 2, c4 = lane & 3;
+#pragma unroll
+    for (int mt = 0; mt < MT; ++mt) {
+        const int r = warp * (MT * 16) + mt * 16 + g;
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+            const int i = nt * 8 + 2 * c4;
+            zb[r * kZStride + i] = zacc[mt][nt][0];
+            zb[r * kZStride + i + 1] = zacc[mt][nt][1];
+            zb[(r + 8) * kZStride + i] = zacc[mt][nt][2];
+            zb[(r + 8) * kZStride + i + 1] = zacc[mt][nt][3];
+        }
+    }
+    __syncthreads();
+    scan_tile(a, sr, u, h, tile, zb, warp_sum);
 }
 
 // ---------------------------------------------------------------------------
@@ -398,7 +588,8 @@ constexpr int kK3Warps = 8;
 
 // W: the variation-weighted representative is compiled in (a separate instantiation, so the
 // plain-mean kernel keeps its register budget).
-template <int D, typename T, bool W>
+// CENTER: keys enter as fl32(k - mu), mu the unit's mean key (the centring option)
+template <int D, typename T, bool W, bool CENTER>
 __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenArgs a) {
     constexpr int ELEM = sizeof(T);
     constexpr int ROWB = D * ELEM;        // bytes of one key row
@@ -418,6 +609,9 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
     const int start = ent.x, m = ent.y;
     const int sub = lane / CH, ch = lane % CH;
 
+    float muv[EPL];   // the unit's mean key on this lane's dimensions (zero without centring)
+#pragma unroll
+    for (int i = 0; i < EPL; ++i) muv[i] = CENTER ? a.key_mu[static_cast<int64_t>(u) * D + ch * EPL + i] : 0.0f;
     const int64_t row0 = sr.row_off + static_cast<int64_t>(h) * sr.T + start;
     const uint8_t *kp = static_cast<const uint8_t *>(a.k) + row0 * ROWB + ch * 16;
     const uint8_t *vp = static_cast<const uint8_t *>(a.v) + row0 * ROWB + ch * 16;
@@ -457,6 +651,10 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
             const float w = W && weighted ? __ll2float_rn(lc[r] - lp[r]) * 0x1p-20f : 0.0f;
             if (W) wsum += w;
             Vec16<T>::cvt(kw[r], x);
+            if constexpr (CENTER) {
+#pragma unroll
+                for (int i = 0; i < EPL; ++i) x[i] = t0 + r * TPS < m ? __fsub_rn(x[i], muv[i]) : 0.0f;
+            }
 #pragma unroll
             for (int i = 0; i < EPL; ++i) {
                 sk[i] += x[i];
@@ -516,6 +714,10 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
         for (int r = 0; r < kUnroll; ++r) {
             if (t0 + r * TPS >= m) break;
             Vec16<T>::cvt(kw[r], x);
+            if constexpr (CENTER) {
+#pragma unroll
+                for (int i = 0; i < EPL; ++i) x[i] = __fsub_rn(x[i], muv[i]);
+            }
 #pragma unroll
             for (int i = 0; i < EPL; ++i) {
                 const float dv = x[i] - sk[i];
@@ -560,44 +762,85 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
 // ---------------------------------------------------------------------------
 // host launcher
 // ---------------------------------------------------------------------------
-template <int D, typename T>
-static cudaError_t launch_typed(const CoarsenArgs &a, const SeqTable &table, const ProjT &proj,
+template <int D>
+static cudaError_t launch_project_tc(const CoarsenArgs &a, const ProjFrag &frag, const CUtensorMap &map_k,
+                                    const CUtensorMap &map_v, cudaStream_t s) {
+    constexpr size_t smem = 1024 + kK1Stages * kK1StageBytes + 64 + 64;
+    static thread_local int configured_dev = -1;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (configured_dev != dev) {
+        e = cudaFuncSetAttribute(k_project_tc<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess) return e;
+        configured_dev = dev;
+    }
+    k_project_tc<D><<<dim3(a.max_tiles, a.B * a.Hkv), kK1Threads, smem, s>>>(a, map_k, map_v, frag);
+    return cudaSuccess;
+}
+
+template <int D, typename T, bool CENTER>
+static cudaError_t launch_typed(const CoarsenArgs &a, const SeqTable &table, const ProjT &proj, const ProjFrag &frag,
                                 const CUtensorMap &map_k, const CUtensorMap &map_v, cudaStream_t s) {
     const int units = a.B * a.Hkv;
     k_setup<<<1, 512, 0, s>>>(table, const_cast<SeqRow *>(a.seq), a.B, a.flags);
-    if (a.max_tiles > 0) {
+    if (CENTER && a.max_blk > 0) {
+        k_key_block_sums<D, T><<<dim3(a.max_blk, units), D, 0, s>>>(a);
+        k_key_mean<D><<<units, D, 0, s>>>(a);
+    }
+    if (a.max_tiles > 0 && a.projection == SKV_PROJECTION_TENSOR_BF16) {
+        // the variation is translation invariant: the tensor-core projection reads the raw keys
+        // even when they are centred (a common shift cancels in z_t - z_{t-1})
+        if constexpr (sizeof(T) == 2) {
+            cudaError_t e = launch_project_tc<D>(a, frag, map_k, map_v, s);
+            if (e != cudaSuccess) return e;
+        } else {
+            return cudaErrorInvalidValue;   // bf16 inputs only (host-checked)
+        }
+        k_tile_prefix<<<units, 256, 0, s>>>(a);
+        k_boundaries<<<dim3(a.max_tiles, units), kTileRows, 0, s>>>(a);
+    } else if (a.max_tiles > 0) {
         constexpr size_t smem = k1_smem_bytes<D>();
         static thread_local int configured_dev = -1;
         int dev = 0;
         cudaError_t e = cudaGetDevice(&dev);
         if (e != cudaSuccess) return e;
         if (configured_dev != dev) {
-            e = cudaFuncSetAttribute(k_project_scan<D, T>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+            e = cudaFuncSetAttribute(k_project_scan<D, T, CENTER>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(smem));
             if (e != cudaSuccess) return e;
             configured_dev = dev;
         }
-        k_project_scan<D, T><<<dim3(a.max_tiles, units), kK1Threads, smem, s>>>(a, map_k, map_v, proj);
+        k_project_scan<D, T, CENTER><<<dim3(a.max_tiles, units), kK1Threads, smem, s>>>(a, map_k, map_v, proj);
         k_tile_prefix<<<units, 256, 0, s>>>(a);
         k_boundaries<<<dim3(a.max_tiles, units), kTileRows, 0, s>>>(a);
     }
     k_plan_entries<<<units, 512, 0, s>>>(a);
     if (a.max_emax > 0) {
         const dim3 g3((a.max_emax + kK3Warps - 1) / kK3Warps, units);
-        if (a.representative == SKV_REP_VARIATION_WEIGHTED) k_segment_reduce<D, T, true><<<g3, kK3Warps * 32, 0, s>>>(a);
-        else k_segment_reduce<D, T, false><<<g3, kK3Warps * 32, 0, s>>>(a);
+        if (a.representative == SKV_REP_VARIATION_WEIGHTED)
+            k_segment_reduce<D, T, true, CENTER><<<g3, kK3Warps * 32, 0, s>>>(a);
+        else
+            k_segment_reduce<D, T, false, CENTER><<<g3, kK3Warps * 32, 0, s>>>(a);
     }
     return cudaGetLastError();
 }
 
-cudaError_t launch_coarsen(const CoarsenArgs &a, const SeqTable &table, const ProjT &proj,
+template <int D, typename T>
+static cudaError_t launch_dt(const CoarsenArgs &a, const SeqTable &table, const ProjT &proj, const ProjFrag &frag,
+                             const CUtensorMap &map_k, const CUtensorMap &map_v, cudaStream_t s) {
+    return a.center ? launch_typed<D, T, true>(a, table, proj, frag, map_k, map_v, s)
+                    : launch_typed<D, T, false>(a, table, proj, frag, map_k, map_v, s);
+}
+
+cudaError_t launch_coarsen(const CoarsenArgs &a, const SeqTable &table, const ProjT &proj, const ProjFrag &frag,
                            const CUtensorMap &map_k, const CUtensorMap &map_v, cudaStream_t s) {
     if (a.dtype == SKV_BF16) {
-        if (a.d == 128) return launch_typed<128, __nv_bfloat16>(a, table, proj, map_k, map_v, s);
-        return launch_typed<64, __nv_bfloat16>(a, table, proj, map_k, map_v, s);
+        if (a.d == 128) return launch_dt<128, __nv_bfloat16>(a, table, proj, frag, map_k, map_v, s);
+        return launch_dt<64, __nv_bfloat16>(a, table, proj, frag, map_k, map_v, s);
     }
-    if (a.d == 128) return launch_typed<128, float>(a, table, proj, map_k, map_v, s);
-    return launch_typed<64, float>(a, table, proj, map_k, map_v, s);
+    if (a.d == 128) return launch_dt<128, float>(a, table, proj, frag, map_k, map_v, s);
+    return launch_dt<64, float>(a, table, proj, frag, map_k, map_v, s);
 }
 
 }  // namespace skv

@@ -77,6 +77,32 @@ struct ProjCache {
 };
 ProjCache g_proj;
 
+// bf16 bits of an fp32 value, rounded to nearest even (the inputs here are finite)
+uint16_t bf16_rne_bits(float x) {
+    uint32_t u;
+    std::memcpy(&u, &x, 4);
+    return static_cast<uint16_t>((u + 0x7fffu + ((u >> 16) & 1u)) >> 16);
+}
+
+// P16 = bf16(P) laid out as the tensor-core projection's B fragments (see ProjFrag): register r of
+// lane (g = lane / 4, c = lane % 4) in k-step ks and n-tile nt packs P16[8 nt + g][16 ks + 2 c + 8 r]
+// (low half) and P16[8 nt + g][16 ks + 2 c + 8 r + 1] (high half).
+void make_projection_fragments(uint64_t seed, int d, ProjFrag &out) {
+    std::vector<float> P(static_cast<size_t>(kProjDim) * 2 * d);
+    make_projection(seed, d, P.data());
+    std::memset(&out, 0, sizeof out);
+    const int cols = 2 * d, nks = cols / 16;
+    for (int ks = 0; ks < nks; ++ks)
+        for (int nt = 0; nt < 2; ++nt)
+            for (int lane = 0; lane < 32; ++lane)
+                for (int r = 0; r < 2; ++r) {
+                    const int n = 8 * nt + lane / 4, k = 16 * ks + 2 * (lane % 4) + 8 * r;
+                    const uint32_t lo = bf16_rne_bits(P[static_cast<size_t>(n) * cols + k]);
+                    const uint32_t hi = bf16_rne_bits(P[static_cast<size_t>(n) * cols + k + 1]);
+                    out.w[((ks * 2 + nt) * 32 + lane) * 2 + r] = lo | (hi << 16);
+                }
+}
+
 // ---------------------------------------------------------------------------
 // driver entry point for TMA descriptors (resolved once through the runtime)
 // ---------------------------------------------------------------------------
@@ -117,7 +143,7 @@ bool make_row_map(CUtensorMap *map, const void *base, int dtype, int d, int64_t 
 // coarsening plan
 // ---------------------------------------------------------------------------
 struct CoarsenPlan {
-    int max_tiles = 0, max_emax = 0, Nmax = 0;
+    int max_tiles = 0, max_emax = 0, Nmax = 0, max_blk = 0;
     int64_t rows = 0, mid = 0, bnd = 0, ent = 0;
     CoarsenLayout lay{};
 };
@@ -152,6 +178,8 @@ skv_status plan_coarsen(int B, int Hkv, int d, const int32_t *T_host, const int3
         p.bnd += static_cast<int64_t>(Hkv) * (N + 1);
         p.ent += static_cast<int64_t>(Hkv) * r.emax;
         if (r.tiles > p.max_tiles) p.max_tiles = r.tiles;
+        const int nblk = (T + kMeanBlock - 1) / kMeanBlock;
+        if (nblk > p.max_blk) p.max_blk = nblk;
         if (r.emax > p.max_emax) p.max_emax = r.emax;
         if (N > p.Nmax) p.Nmax = N;
         if (table) table->rows[b] = r;
@@ -173,19 +201,22 @@ skv_status plan_coarsen(int B, int Hkv, int d, const int32_t *T_host, const int3
     off += align256(static_cast<size_t>(p.bnd) * 4);
     p.lay.ents = off;
     off += align256(static_cast<size_t>(p.ent) * 8);
+    p.lay.key_blk = off;   // the centring option's block sums and unit means
+    off += align256(static_cast<size_t>(units) * p.max_blk * d * 4);
+    p.lay.key_mu = off;
+    off += align256(static_cast<size_t>(units) * d * 4);
     p.lay.total = off;
     *plan = p;
     return SKV_OK;
 }
 
-// ---------------------------------------------------------------------------
-// decode plan
-// ---------------------------------------------------------------------------
-struct DecodePlan {
-    int rows, row_passes, pass_rows, n_vunits;
-    DecodeLayout lay;
-};
+}  // namespace
 
+namespace skv {
+
+// ---------------------------------------------------------------------------
+// decode plan (shared by skv_decode_attn_ex and skv_decode_attn_noalloc)
+// ---------------------------------------------------------------------------
 skv_status plan_decode(int dtype, int B, int R, int Hq, int Hkv, int d, int max_pages, DecodePlan *plan) {
     if (B < 1 || R < 1 || Hq < 1 || Hkv < 1 || max_pages < 1) return SKV_ERR_INVALID_ARG;
     if (Hq % Hkv != 0 || (d != 64 && d != 128) || (dtype != SKV_BF16 && dtype != SKV_F32))
@@ -202,19 +233,78 @@ skv_status plan_decode(int dtype, int B, int R, int Hq, int Hkv, int d, int max_
     // the page prefix is an int32 sum over all units
     if (static_cast<int64_t>(B) * Hkv * max_pages * p.row_passes > INT32_MAX / 2) return SKV_ERR_UNSUPPORTED;
     p.n_vunits = static_cast<int>(nv);
-    size_t off = kWsHeader;
-    p.lay.counters = off;
-    off += align256(static_cast<size_t>(nv) * 4);
-    p.lay.part_v = off;
-    if (dtype == SKV_BF16) off += align256(static_cast<size_t>(kMaxDecodeCtas) * 2 * p.pass_rows * d * 4);
-    p.lay.part_l = off;
-    if (dtype == SKV_BF16) off += align256(static_cast<size_t>(kMaxDecodeCtas) * 2 * p.pass_rows * 4);
-    p.lay.total = off;
+    p.lay = decode_layout(dtype, d, p, kMaxDecodeCtas);
     *plan = p;
     return SKV_OK;
 }
 
-}  // namespace
+DecodeLayout decode_layout(int dtype, int d, const DecodePlan &p, int ncta) {
+    const auto al = [](size_t x) { return (x + 255) & ~static_cast<size_t>(255); };
+    DecodeLayout lay{};
+    size_t off = kWsHeader;
+    lay.counters = off;
+    off += al(static_cast<size_t>(p.n_vunits) * 4);
+    lay.part_v = off;
+    if (dtype == SKV_BF16) off += al(static_cast<size_t>(ncta) * 2 * p.pass_rows * d * 4);
+    lay.part_l = off;
+    if (dtype == SKV_BF16) off += al(static_cast<size_t>(ncta) * 2 * p.pass_rows * 4);
+    lay.total = off;
+    return lay;
+}
+
+skv_status decode_args(const void *q, int dtype, int B, int R, int Hq, int Hkv, int d, const skv_node_pool *pool,
+                       const int32_t *page_table, int max_pages, const int32_t *lens, void *out, float *lse,
+                       int closure, DecodePlan *plan, DecodeArgs *args) {
+    skv_status st = plan_decode(dtype, B, R, Hq, Hkv, d, max_pages, plan);
+    if (st != SKV_OK) return st;
+    if (!q || !out || !lse || !pool || !page_table || !lens) return SKV_ERR_INVALID_ARG;
+    if (!pool->pages || pool->num_pages < 0) return SKV_ERR_INVALID_ARG;
+    const auto al = [](const void *ptr, uintptr_t m) { return (reinterpret_cast<uintptr_t>(ptr) & (m - 1)) == 0; };
+    if (!al(pool->pages, 16) || !al(q, 16) || !al(out, 16) || !al(lse, 4)) return SKV_ERR_INVALID_ARG;
+    DecodeArgs a{};
+    a.q = q;
+    a.pages = static_cast<const uint8_t *>(pool->pages);
+    a.num_pages = pool->num_pages;
+    a.page_table = page_table;
+    a.max_pages = max_pages;
+    a.lens = lens;
+    a.out = out;
+    a.lse = lse;
+    a.B = B;
+    a.R = R;
+    a.Hq = Hq;
+    a.Hkv = Hkv;
+    a.G = Hq / Hkv;
+    a.d = d;
+    a.dtype = dtype;
+    a.rows = plan->rows;
+    a.row_passes = plan->row_passes;
+    a.pass_rows = plan->pass_rows;
+    a.n_vunits = plan->n_vunits;
+    a.closure = closure;
+    *args = a;
+    return SKV_OK;
+}
+
+}  // namespace skv
+
+namespace skv {
+
+// One thread arms an mbarrier for one arrival that nothing makes (no copy targets it), polls it at
+// most `polls` times with the same try_wait the pipelines use, and raises FLAG_TIMEOUT when the
+// polls run out -- the path every bounded wait of the library's kernels takes when it gives up.
+__global__ void k_wait_selftest(uint32_t *flags, uint32_t polls) {
+    __shared__ uint64_t bar;
+    if (threadIdx.x != 0) return;
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    bool done = false;
+    for (uint32_t i = 0; i < polls && !done; ++i) done = mbar_try_wait(&bar, 0);
+    if (!done) raise_flag(flags, FLAG_TIMEOUT);
+    mbar_inval(&bar);
+}
+
+}  // namespace skv
 
 // ===========================================================================
 extern "C" {
@@ -226,13 +316,14 @@ const char *skv_status_string(int status) {
         case SKV_ERR_UNSUPPORTED: return "SKV_ERR_UNSUPPORTED: configuration not supported";
         case SKV_ERR_CUDA: return "SKV_ERR_CUDA: CUDA runtime error";
         case SKV_ERR_OVERFLOW: return "SKV_ERR_OVERFLOW: variation step above 2^20 (or not finite)";
+        case SKV_ERR_TIMEOUT: return "SKV_ERR_TIMEOUT: a bounded device wait gave up (work abandoned)";
         case SKV_ERR_WORKSPACE: return "SKV_ERR_WORKSPACE: workspace too small or misaligned";
         case SKV_ERR_DEVICE: return "SKV_ERR_DEVICE: device detected a bad page id, lens entry or stuck wait";
         default: return "unknown skv status";
     }
 }
 
-int skv_abi_version(void) { return 202; }
+int skv_abi_version(void) { return 203; }
 
 size_t skv_page_bytes(skv_dtype dtype, int d) { return skv_page_bytes_ex(dtype, d, SKV_CLOSURE_SCALAR); }
 
@@ -262,34 +353,42 @@ static skv_status coarsen_impl(const void *k, const void *v, skv_dtype dtype, in
                                const int32_t *T_host, int n_sink, int n_recent, const int32_t *N_host,
                                uint64_t proj_seed, const skv_node_pool *pool, const int32_t *page_table, int max_pages,
                                int32_t *lens, int32_t *boundaries, int64_t *cumvar, void *workspace, size_t ws_bytes,
-                               int representative, int closure, StreamArgs *streaming, void *stream);
+                               int representative, int closure, int center, int projection, StreamArgs *streaming,
+                               void *stream);
 
 skv_status skv_coarsen_ex(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d,
                           const int32_t *T_host, int n_sink, int n_recent, const int32_t *N_host, uint64_t proj_seed,
                           const skv_node_pool *pool, const int32_t *page_table, int max_pages, int32_t *lens,
                           int32_t *boundaries, int64_t *cumvar, void *workspace, size_t ws_bytes,
                           const skv_coarsen_options *options, void *stream) {
-    int representative = SKV_REP_MEAN, closure = SKV_CLOSURE_SCALAR;
+    int representative = SKV_REP_MEAN, closure = SKV_CLOSURE_SCALAR, center = 0, projection = SKV_PROJECTION_FIXED_FP32;
     if (options) {
         if (options->representative != SKV_REP_MEAN && options->representative != SKV_REP_VARIATION_WEIGHTED)
             return SKV_ERR_INVALID_ARG;
         if (options->closure != SKV_CLOSURE_SCALAR && options->closure != SKV_CLOSURE_DIAGONAL)
             return SKV_ERR_INVALID_ARG;
-        for (int i = 0; i < 6; ++i)
+        if (options->center_keys != 0 && options->center_keys != 1) return SKV_ERR_INVALID_ARG;
+        if (options->projection != SKV_PROJECTION_FIXED_FP32 && options->projection != SKV_PROJECTION_TENSOR_BF16)
+            return SKV_ERR_INVALID_ARG;
+        for (int i = 0; i < 4; ++i)
             if (options->reserved[i] != 0) return SKV_ERR_INVALID_ARG;
         representative = options->representative;
         closure = options->closure;
+        center = options->center_keys;
+        projection = options->projection;
+        if (projection == SKV_PROJECTION_TENSOR_BF16 && dtype != SKV_BF16) return SKV_ERR_UNSUPPORTED;
     }
     return coarsen_impl(k, v, dtype, B, Hkv, d, T_host, n_sink, n_recent, N_host, proj_seed, pool, page_table,
-                        max_pages, lens, boundaries, cumvar, workspace, ws_bytes, representative, closure, nullptr,
-                        stream);
+                        max_pages, lens, boundaries, cumvar, workspace, ws_bytes, representative, closure, center,
+                        projection, nullptr, stream);
 }
 
 static skv_status coarsen_impl(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d,
                                const int32_t *T_host, int n_sink, int n_recent, const int32_t *N_host,
                                uint64_t proj_seed, const skv_node_pool *pool, const int32_t *page_table, int max_pages,
                                int32_t *lens, int32_t *boundaries, int64_t *cumvar, void *workspace, size_t ws_bytes,
-                               int representative, int closure, StreamArgs *streaming, void *stream) {
+                               int representative, int closure, int center, int projection, StreamArgs *streaming,
+                               void *stream) {
     if (dtype != SKV_BF16 && dtype != SKV_F32) return SKV_ERR_UNSUPPORTED;
     static SeqTable table;   // host staging; guarded by the mutex below
     static std::mutex table_mu;
@@ -305,7 +404,14 @@ static skv_status coarsen_impl(const void *k, const void *v, skv_dtype dtype, in
         if (table.rows[b].emax > static_cast<int64_t>(max_pages) * kPageNodes) return SKV_ERR_INVALID_ARG;
 
     ProjT proj;
-    g_proj.get(proj_seed, d, proj);
+    static ProjFrag frag;   // host staging (guarded by table_mu)
+    if (projection == SKV_PROJECTION_TENSOR_BF16) {
+        std::memset(&proj, 0, sizeof proj);
+        make_projection_fragments(proj_seed, d, frag);
+    } else {
+        g_proj.get(proj_seed, d, proj);
+        std::memset(&frag, 0, sizeof frag);
+    }
     CUtensorMap map_k, map_v;
     std::memset(&map_k, 0, sizeof map_k);
     std::memset(&map_v, 0, sizeof map_v);
@@ -341,7 +447,12 @@ static skv_status coarsen_impl(const void *k, const void *v, skv_dtype dtype, in
     a.cumvar = cumvar;
     a.representative = representative;
     a.closure = closure;
-    cudaError_t e = launch_coarsen(a, table, proj, map_k, map_v, static_cast<cudaStream_t>(stream));
+    a.center = center;
+    a.projection = projection;
+    a.max_blk = plan.max_blk;
+    a.key_blk = reinterpret_cast<float *>(ws + plan.lay.key_blk);
+    a.key_mu = reinterpret_cast<float *>(ws + plan.lay.key_mu);
+    cudaError_t e = launch_coarsen(a, table, proj, frag, map_k, map_v, static_cast<cudaStream_t>(stream));
     if (e == cudaSuccess && streaming) {
         streaming->flags = a.flags;
         streaming->pages = a.pages;
@@ -398,8 +509,8 @@ skv_status skv_stream_init(const void *k, const void *v, skv_dtype dtype, int B,
     s.pt = static_cast<float *>(state);
     s.state = static_cast<uint8_t *>(state) + kStreamProjBytes;
     return coarsen_impl(k, v, dtype, B, Hkv, d, T_host, n_sink, n_recent, N_host, proj_seed, pool, page_table,
-                        max_pages, lens, nullptr, nullptr, workspace, ws_bytes, SKV_REP_MEAN, SKV_CLOSURE_SCALAR, &s,
-                        stream);
+                        max_pages, lens, nullptr, nullptr, workspace, ws_bytes, SKV_REP_MEAN, SKV_CLOSURE_SCALAR, 0,
+                        SKV_PROJECTION_FIXED_FP32, &s, stream);
 }
 
 skv_status skv_stream_append(const void *k_new, const void *v_new, skv_dtype dtype, int B, int Hkv, int d,
@@ -460,39 +571,16 @@ skv_status skv_decode_attn_ex(const void *q, skv_dtype dtype, int B, int R, int 
         closure = options->closure;
     }
     DecodePlan plan;
-    skv_status st = plan_decode(dtype, B, R, Hq, Hkv, d, max_pages, &plan);
+    DecodeArgs a;
+    skv_status st = decode_args(q, dtype, B, R, Hq, Hkv, d, pool, page_table, max_pages, lens, out, lse, closure,
+                                &plan, &a);
     if (st != SKV_OK) return st;
-    if (!q || !out || !lse || !pool || !page_table || !lens) return SKV_ERR_INVALID_ARG;
-    if (!pool->pages || pool->num_pages < 0) return SKV_ERR_INVALID_ARG;
-    if (!aligned(pool->pages, 16) || !aligned(q, 16) || !aligned(out, 16) || !aligned(lse, 4))
-        return SKV_ERR_INVALID_ARG;
     if (!workspace || !aligned(workspace, 256) || ws_bytes < plan.lay.total) return SKV_ERR_WORKSPACE;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    DecodeArgs a{};
-    a.q = q;
-    a.pages = static_cast<const uint8_t *>(pool->pages);
-    a.num_pages = pool->num_pages;
-    a.page_table = page_table;
-    a.max_pages = max_pages;
-    a.lens = lens;
-    a.out = out;
-    a.lse = lse;
-    a.B = B;
-    a.R = R;
-    a.Hq = Hq;
-    a.Hkv = Hkv;
-    a.G = Hq / Hkv;
-    a.d = d;
-    a.dtype = dtype;
-    a.rows = plan.rows;
-    a.row_passes = plan.row_passes;
-    a.pass_rows = plan.pass_rows;
-    a.n_vunits = plan.n_vunits;
     a.part_v = reinterpret_cast<float *>(ws + plan.lay.part_v);
     a.part_l = reinterpret_cast<float *>(ws + plan.lay.part_l);
     a.counters = reinterpret_cast<int32_t *>(ws + plan.lay.counters);
     a.flags = reinterpret_cast<uint32_t *>(ws);
-    a.closure = closure;
     const cudaError_t e = launch_decode(a, static_cast<cudaStream_t>(stream));
     return e == cudaSuccess ? SKV_OK : SKV_ERR_CUDA;
 }
@@ -504,15 +592,24 @@ skv_status skv_decode_attn(const void *q, skv_dtype dtype, int B, int R, int Hq,
                               ws_bytes, nullptr, stream);
 }
 
+skv_status skv_wait_selftest(void *workspace, size_t ws_bytes, uint32_t polls, void *stream) {
+    if (!workspace || !aligned(workspace, 256) || ws_bytes < kWsHeader) return SKV_ERR_WORKSPACE;
+    if (polls > kWaitLimit) return SKV_ERR_INVALID_ARG;
+    k_wait_selftest<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(static_cast<uint32_t *>(workspace), polls);
+    return cudaGetLastError() == cudaSuccess ? SKV_OK : SKV_ERR_CUDA;
+}
+
 skv_status skv_workspace_error(const void *workspace, void *stream, uint32_t *flags_host) {
     if (!workspace) return SKV_ERR_INVALID_ARG;
     cudaStream_t s = static_cast<cudaStream_t>(stream);
-    if (cudaStreamSynchronize(s) != cudaSuccess) return SKV_ERR_CUDA;
+    // read and clear on the caller's stream, after everything already enqueued there
     uint32_t f = 0;
-    if (cudaMemcpy(&f, workspace, sizeof f, cudaMemcpyDeviceToHost) != cudaSuccess) return SKV_ERR_CUDA;
-    if (cudaMemset(const_cast<void *>(workspace), 0, sizeof f) != cudaSuccess) return SKV_ERR_CUDA;
+    if (cudaMemcpyAsync(&f, workspace, sizeof f, cudaMemcpyDeviceToHost, s) != cudaSuccess) return SKV_ERR_CUDA;
+    if (cudaMemsetAsync(const_cast<void *>(workspace), 0, sizeof f, s) != cudaSuccess) return SKV_ERR_CUDA;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return SKV_ERR_CUDA;
     if (flags_host) *flags_host = f;
     if (f & FLAG_OVERFLOW) return SKV_ERR_OVERFLOW;
+    if (f & FLAG_TIMEOUT) return SKV_ERR_TIMEOUT;
     if (f) return SKV_ERR_DEVICE;
     return SKV_OK;
 }

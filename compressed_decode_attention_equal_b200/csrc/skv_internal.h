@@ -39,6 +39,13 @@ struct ProjT {
     float pt[2 * 128 * SKV_PROJ_DIM];
 };
 
+// The tensor-core projection's operand: P16 = bf16(P) (round to nearest even) as mma.sync
+// m16n8k16 B fragments, w[((ks * 2 + nt) * 32 + lane) * 2 + r] for k-step ks (features 16 ks ..
+// 16 ks + 15), n-tile nt (outputs 8 nt .. 8 nt + 7) and the fragment's register r.
+struct ProjFrag {
+    uint32_t w[(2 * 128 / 16) * 2 * 32 * 2];
+};
+
 struct CoarsenArgs {
     const void *k, *v;
     int B, Hkv, d, dtype;
@@ -59,11 +66,18 @@ struct CoarsenArgs {
     int64_t *cumvar;
     int representative;  // skv_representative of the middle segments' stored key and value
     int closure;         // skv_closure: SKV_CLOSURE_DIAGONAL also writes per-dimension variances
+    int center;          // 1: keys enter every stage with the unit's mean key removed
+    int projection;      // skv_projection: SKV_PROJECTION_TENSOR_BF16 selects k_project_tc
+    int max_blk;         // largest ceil(T / kMeanBlock) over the batch
+    float *key_blk;      // [units][max_blk][d] per-block key sums (centring only)
+    float *key_mu;       // [units][d] mean key of each unit (centring only)
 };
+
+constexpr int kMeanBlock = 256;   // tokens per block of the centring mean's fixed summation order
 
 // Workspace carve-up (offsets in bytes from the workspace start).
 struct CoarsenLayout {
-    size_t seq, tile_total, tile_prefix, unit_total, local_scan, bounds, ents, total;
+    size_t seq, tile_total, tile_prefix, unit_total, local_scan, bounds, ents, key_blk, key_mu, total;
 };
 
 // Host-side launchers (coarsen.cu).
@@ -107,7 +121,7 @@ cudaError_t launch_stream_append(const StreamArgs &s, cudaStream_t st);
 // bytes at the start of a streaming state buffer that hold P^T (then the units' blocks)
 constexpr int64_t kStreamProjBytes = 2 * 128 * SKV_PROJ_DIM * 4;
 
-cudaError_t launch_coarsen(const CoarsenArgs &a, const SeqTable &table, const ProjT &proj,
+cudaError_t launch_coarsen(const CoarsenArgs &a, const SeqTable &table, const ProjT &proj, const ProjFrag &frag,
                            const CUtensorMap &map_k, const CUtensorMap &map_v, cudaStream_t s);
 
 // ---------------------------------------------------------------------------
@@ -143,6 +157,23 @@ struct DecodeArgs {
 struct DecodeLayout {
     size_t counters, part_v, part_l, total;
 };
+
+// Query-row geometry of one decode call and its workspace layout (split partials sized for the
+// largest grid, kMaxDecodeCtas).
+struct DecodePlan {
+    int rows, row_passes, pass_rows, n_vunits;
+    DecodeLayout lay;
+};
+
+// Host-side checks and geometry shared by every decode entry point (skv_api.cu).
+skv_status plan_decode(int dtype, int B, int R, int Hq, int Hkv, int d, int max_pages, DecodePlan *plan);
+// Workspace layout for a grid of ncta CTAs (flags header, counters, split partials).
+DecodeLayout decode_layout(int dtype, int d, const DecodePlan &plan, int ncta);
+// plan_decode plus the buffer checks; fills every DecodeArgs field except the workspace pointers
+// (part_v, part_l, counters, flags) and the grid (ncta, cluster).
+skv_status decode_args(const void *q, int dtype, int B, int R, int Hq, int Hkv, int d, const skv_node_pool *pool,
+                       const int32_t *page_table, int max_pages, const int32_t *lens, void *out, float *lse,
+                       int closure, DecodePlan *plan, DecodeArgs *args);
 
 cudaError_t launch_decode(const DecodeArgs &a, cudaStream_t s);
 cudaError_t decode_split_ctas(const DecodeArgs &a, int *ncta);

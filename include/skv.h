@@ -76,6 +76,7 @@ typedef enum {
     SKV_ERR_UNSUPPORTED = -2, /* valid but outside the built configurations */
     SKV_ERR_CUDA = -3,        /* a CUDA runtime call or launch failed */
     SKV_ERR_OVERFLOW = -4,    /* variation step above 2^20 or too many tokens */
+    SKV_ERR_TIMEOUT = -5,     /* a bounded device wait gave up; that work was abandoned */
     SKV_ERR_WORKSPACE = -6,   /* workspace smaller than the *_workspace_bytes query */
     SKV_ERR_DEVICE = -7       /* device-detected bad page id or lens (see flags) */
 } skv_status;
@@ -201,21 +202,51 @@ skv_status skv_coarsen(const void *k, const void *v, skv_dtype dtype, int B, int
  *   unchanged, and the boundaries do not depend on the option.
  * closure: the pool's skv_closure; SKV_CLOSURE_DIAGONAL also writes each
  *   node's per-dimension key variances (zero for exact tokens).
+ * center_keys: 1 selects the common-mode mean removal of "SPICY-KV"
+ *   Independent Claim 1(b) (keys mapped into an anisotropy-reduced space
+ *   before coarsening): every key of a unit enters the pipeline -- the
+ *   projection, the segment statistics and the exact tokens alike -- as
+ *   fl32(k_t - mu) with mu the unit's mean key over all T_b tokens. mu follows
+ *   one fixed fp32 order (per dimension: blocks of 256 consecutive tokens
+ *   summed in token order, block sums added in block order, total divided by
+ *   T_b), so the centred keys, and hence the boundaries, are exact. The stored
+ *   keys are centred: decode outputs are unchanged up to rounding and each
+ *   lse moves by -q.mu/sqrt(d). Not available for streaming coarsening.
+ * projection: how z_t = P [k_t; v_t] is computed for the variation steps.
+ *   SKV_PROJECTION_FIXED_FP32 (0, default): the fixed fp32 fma recipe above;
+ *     steps, boundaries and node counts are reproducible bit for bit by any
+ *     IEEE fp32 implementation of the recipe.
+ *   SKV_PROJECTION_TENSOR_BF16 (1, bf16 inputs only): z = P16 [k; v] on the
+ *     tensor cores, P16 = P rounded to bf16 (nearest even), exact products
+ *     accumulated in fp32 in the hardware's order; d_t and D_t then follow the
+ *     same recipe from z. A different fixed random projection (P16) and a
+ *     different summation order: each step D_t stays within the fp32
+ *     accumulation bound of the exact P16 projection's step, and the
+ *     boundaries are the exact first-hitting boundaries of those steps (given
+ *     the steps, every later stage is exact), but the steps are not those of
+ *     the fixed recipe, so boundaries may differ from the default's. The
+ *     projection reads the raw keys even with center_keys (a common shift
+ *     cancels in z_t - z_{t-1}). fp32 inputs: SKV_ERR_UNSUPPORTED.
  * reserved: must be zero.
  */
 typedef enum { SKV_REP_MEAN = 0, SKV_REP_VARIATION_WEIGHTED = 1 } skv_representative;
 
+typedef enum { SKV_PROJECTION_FIXED_FP32 = 0, SKV_PROJECTION_TENSOR_BF16 = 1 } skv_projection;
+
 typedef struct {
     int32_t representative; /* skv_representative */
     int32_t closure;        /* skv_closure */
-    int32_t reserved[6];
+    int32_t center_keys;    /* 0 or 1: common-mode mean removal (see above) */
+    int32_t projection;     /* skv_projection (see above) */
+    int32_t reserved[4];
 } skv_coarsen_options;
 
 /*
  * skv_coarsen with options (NULL = defaults, identical to skv_coarsen). Same
  * arguments, layouts, ownership and errors as skv_coarsen; additionally
- * SKV_ERR_INVALID_ARG for an unknown representative or closure or a nonzero
- * reserved field.
+ * SKV_ERR_INVALID_ARG for an unknown representative, closure or projection,
+ * center_keys not 0 or 1, or a nonzero reserved field; SKV_ERR_UNSUPPORTED for
+ * the tensor-core projection on fp32 inputs.
  */
 skv_status skv_coarsen_ex(const void *k, const void *v, skv_dtype dtype, int B, int Hkv, int d,
                           const int32_t *T_host, int n_sink, int n_recent, const int32_t *N_host,
@@ -332,22 +363,26 @@ skv_status skv_decode_attn_ex(const void *q, skv_dtype dtype, int B, int R, int 
  * Decode attention without any caller-provided workspace. (The sources describe no such entry
  * point; it exists for callers of this library that cannot allocate device memory.)
  *
- * Some callers cannot allocate: code recorded into a CUDA graph owned by someone else, a plugin
- * that a host framework hands only its input and output buffers, or a runtime whose allocator is
- * fixed when it starts. This entry point takes the same arguments and computes the same result
- * as skv_decode_attn (the same kernel), but keeps its scratch -- device flags, per-unit
- * completion counters and split partials -- in one array of SKV_NOALLOC_SCRATCH_BYTES that the
- * library defines at file scope. Every GPU that loads the library reserves that array once and
- * keeps it until the process exits.
+ * Some callers cannot allocate: a plugin that a host framework hands only its input and output
+ * buffers, a runtime whose device allocator is fixed when it starts, or code on a latency-critical
+ * path where cudaMalloc, which may synchronise the device, is not allowed. This entry point takes
+ * the same arguments as skv_decode_attn minus the workspace, applies the same checks and launches
+ * the same kernel with the same grid, so its out and lse are bit-identical to skv_decode_attn's
+ * for the same inputs. Its scratch -- device flags, per-unit completion counters and split
+ * partials -- lives in one array of SKV_NOALLOC_SCRATCH_BYTES that the library defines at file
+ * scope. Every GPU that loads the library reserves that array once and keeps it until the
+ * process exits.
  *  - No cudaMalloc, cudaFree or other allocating call is made.
  *  - The first call on each device looks up the array's device address (cudaGetSymbolAddress)
  *    with that device current and caches it; make that first call before any stream capture.
- *  - All calls on a device share the array: calls whose kernels may overlap on the GPU (other
- *    streams, or other threads' streams) race on it and must be serialised by the caller. Each
- *    call clears the flags and counters on `stream` before its kernel runs.
+ *  - All calls on a device share the array and it keeps the last call's contents: each call
+ *    clears the flags and counters on `stream` before its kernel runs, and calls whose kernels
+ *    may overlap on the GPU (other streams, or other threads' streams) race on the array and
+ *    must be serialised by the caller.
  *  - A request whose scratch would exceed SKV_NOALLOC_SCRATCH_BYTES (bf16: split partials of
  *    2 x grid x rows-per-pass x (d + 1) floats, plus 4 bytes per unit and row pass) returns
  *    SKV_ERR_WORKSPACE before anything is enqueued; use skv_decode_attn for such sizes.
+ *  - Scalar-closure pools only (the pools skv_coarsen builds).
  *  - Device-detected errors (bad page id, lens above capacity) still skip the bad access, but
  *    their flags live in the library's array and are not reported; diagnose with skv_decode_attn.
  * Other errors: as skv_decode_attn.
@@ -358,11 +393,32 @@ skv_status skv_decode_attn_noalloc(const void *q, skv_dtype dtype, int B, int R,
                                    const int32_t *lens, void *out, float *lse, void *stream);
 
 /*
- * Synchronise stream, then read and clear the device error flags raised on
- * this workspace since they were last cleared: SKV_OK, SKV_ERR_OVERFLOW or
- * SKV_ERR_DEVICE (SKV_ERR_CUDA if synchronisation fails). *flags_host
- * (optional) receives the raw bits: 1 overflow, 2 bad page id, 4 lens above
- * capacity, 8 a bounded wait gave up.
+ * Check of the device error path that a stuck pipeline takes. Every wait of
+ * the library's kernels on an mbarrier (a copy landing, a stage being freed)
+ * polls at most 2^20 times; when the polls run out the kernel raises the
+ * timeout flag, abandons the work it cannot finish (after waiting, again
+ * bounded, for its copies in flight) and returns, so the context stays
+ * usable. This call launches one thread that waits in the same way on a
+ * barrier nothing ever arrives at, for `polls` polls (0 .. 2^20), no copy
+ * outstanding, and raises the flag in `workspace` (any zero-filled buffer of
+ * >= 256 bytes, 256-byte aligned, e.g. a decode workspace). Afterwards
+ * skv_workspace_error returns SKV_ERR_TIMEOUT with flag bit 8. No counterpart
+ * in the sources: it exists to test failure reporting without a GPU fault.
+ * Errors: SKV_ERR_WORKSPACE (NULL, misaligned or too small), SKV_ERR_INVALID_ARG
+ * (polls above 2^20), SKV_ERR_CUDA (launch failure).
+ */
+skv_status skv_wait_selftest(void *workspace, size_t ws_bytes, uint32_t polls, void *stream);
+
+/*
+ * Read and clear the device error flags raised on this workspace since they
+ * were last cleared. The read and the clear are enqueued on `stream` (after
+ * the work already there) and the call then synchronises that stream. Returns
+ * SKV_OK, SKV_ERR_OVERFLOW (a variation step above 2^20), SKV_ERR_TIMEOUT (a
+ * bounded wait gave up and its work was abandoned), or SKV_ERR_DEVICE (a bad
+ * page id or lens entry was skipped); in that order of precedence when
+ * several flags are set (SKV_ERR_CUDA if a copy or the synchronisation
+ * fails). *flags_host (optional) receives the raw bits: 1 overflow, 2 bad page
+ * id, 4 lens above capacity, 8 a bounded wait gave up.
  */
 skv_status skv_workspace_error(const void *workspace, void *stream, uint32_t *flags_host);
 

@@ -73,12 +73,16 @@ def _load():
         lib.orc_feature_f32.restype = None
         lib.orc_quantised_step.argtypes = [P(f32), P(f32), P(i64)]
         lib.orc_segment.argtypes = [P(i64), ctypes.c_int, ctypes.c_int, P(i32)]
+        lib.orc_key_mean_f32.argtypes = [P(f32), ctypes.c_int, ctypes.c_int, P(f32)]
         lib.orc_split.argtypes = [ctypes.c_int] * 3 + [P(ctypes.c_int)] * 3
         lib.orc_coarsen_unit.argtypes = ([P(f32), P(f32)] + [ctypes.c_int] * 5 + [P(f32), P(i64), P(i64), P(f64),
                                          P(i32), P(i32), P(i32), P(f64), P(f64), P(f64), P(f64), P(f64), P(i32)])
         lib.orc_coarsen_unit2.argtypes = ([P(f32), P(f32)] + [ctypes.c_int] * 5 + [P(f32), ctypes.c_int, P(i64),
                                           P(i64), P(f64), P(i32), P(i32), P(i32), P(f64), P(f64), P(f64), P(f64),
                                           P(f64), P(f64), P(i32)])
+        lib.orc_coarsen_unit_steps.argtypes = ([P(f32), P(f32)] + [ctypes.c_int] * 6 + [P(i64), P(i64), P(i64),
+                                               P(i32), P(i32), P(i32), P(f64), P(f64), P(f64), P(f64), P(f64),
+                                               P(f64), P(i32)])
         lib.orc_decode_rows2.argtypes = [P(f64), ctypes.c_int, ctypes.c_int, P(f64), P(f64), P(f64), P(f64),
                                          P(f64), ctypes.c_int, P(f64), P(f64)]
         lib.orc_decode_rows.argtypes = [P(f64), ctypes.c_int, ctypes.c_int, P(f64), P(f64), P(f64), P(f64),
@@ -152,6 +156,24 @@ def split(T: int, S: int, W: int):
     return s.value, w.value, m.value
 
 
+def key_mean_f32(k: np.ndarray) -> np.ndarray:
+    """The unit's mean key mu [d] in the fixed fp32 order of reading R8 (common-mode mean removal,
+    [SK] Independent Claim 1(b)): per dimension, blocks of 256 tokens summed in token order, block
+    sums added in block order, total divided by T; all IEEE fp32."""
+    k = np.ascontiguousarray(k, np.float32)
+    T, d = k.shape
+    mu = np.zeros(d, np.float32)
+    kk = k if T > 0 else np.zeros((1, d), np.float32)
+    _check(_load().orc_key_mean_f32(_ptr(kk, ctypes.c_float), T, d, _ptr(mu, ctypes.c_float)), "key_mean_f32")
+    return mu
+
+
+def center_keys(k: np.ndarray) -> np.ndarray:
+    """Keys with the unit's mean key removed: fl32(k_ti - mu_i) (IEEE fp32 subtraction)."""
+    k = np.ascontiguousarray(k, np.float32)
+    return (k - key_mean_f32(k)[None, :]).astype(np.float32)
+
+
 # --------------------------------------------------------------------------
 # coarsening
 # --------------------------------------------------------------------------
@@ -180,13 +202,15 @@ REPRESENTATIVES = {"mean": 0, "variation": 1}
 
 
 def coarsen_unit(k: np.ndarray, v: np.ndarray, n_sink: int, n_recent: int, N: int,
-                 P: np.ndarray, representative: str = "mean") -> UnitNodes:
+                 P: np.ndarray, representative: str = "mean", center: bool = False) -> UnitNodes:
     """Coarsen one unit: k, v [T, d] (any float dtype holding fp32-representable values).
     representative: "mean" (plain member mean, SPICY-KV Claim 2) or "variation" (the
     variation-weighted average of the Equal-Variation page's implementation notes, weights D_r;
-    a segment without variation keeps the plain mean)."""
+    a segment without variation keeps the plain mean). center: coarsen the keys with the unit's
+    mean key removed (center_keys; SPICY-KV Claim 1(b)); every key statistic, exact tokens
+    included, is then of the centred keys."""
     rep = REPRESENTATIVES[representative]
-    k = np.ascontiguousarray(k, np.float32)
+    k = center_keys(k) if center else np.ascontiguousarray(k, np.float32)
     v = np.ascontiguousarray(v, np.float32)
     P = np.ascontiguousarray(P, np.float32)
     T, d = k.shape
@@ -219,12 +243,92 @@ def coarsen_unit(k: np.ndarray, v: np.ndarray, n_sink: int, n_recent: int, N: in
                      kt[:e].copy(), vt[:e].copy(), s2[:e].copy(), vv_[:e].copy(), al[:e].copy(), be[:e].copy(), s_eff, w_eff, M)
 
 
+def coarsen_unit_from_steps(k: np.ndarray, v: np.ndarray, n_sink: int, n_recent: int, N: int, D: np.ndarray,
+                            representative: str = "mean", center: bool = False) -> UnitNodes:
+    """coarsen_unit with the middle tokens' quantised steps D [M] given (int64, D[0] = 0) instead of
+    the fixed fp32 recipe: prefix sums, first-hitting boundaries and node statistics follow D. The
+    stage-wise check of steps computed another way (the tensor-core projection option)."""
+    rep = REPRESENTATIVES[representative]
+    k = center_keys(k) if center else np.ascontiguousarray(k, np.float32)
+    v = np.ascontiguousarray(v, np.float32)
+    T, d = k.shape
+    s_eff, w_eff, M = split(T, n_sink, n_recent)
+    D_in = np.ascontiguousarray(D, np.int64)
+    if D_in.shape != (M,):
+        raise ValueError(f"D must have the middle's {M} steps")
+    Emax = s_eff + N + w_eff
+    Mb = max(M, 1)
+    Dout = np.zeros(Mb, np.int64)
+    C = np.zeros(Mb, np.int64)
+    b = np.zeros(N + 1, np.int32)
+    E1 = max(Emax, 1)
+    st, ln = np.zeros(E1, np.int32), np.zeros(E1, np.int32)
+    kt, vt, vv_ = np.zeros((E1, d)), np.zeros((E1, d)), np.zeros((E1, d))
+    s2, al, be = np.zeros(E1), np.zeros(E1), np.zeros(E1)
+    E = np.zeros(1, np.int32)
+    kk = k if T > 0 else np.zeros((1, d), np.float32)
+    vv = v if T > 0 else np.zeros((1, d), np.float32)
+    Dp = D_in if M > 0 else np.zeros(1, np.int64)
+    f32p, i64p, i32p, f64p = (ctypes.c_float, ctypes.c_int64, ctypes.c_int32, ctypes.c_double)
+    rc = _load().orc_coarsen_unit_steps(_ptr(kk, f32p), _ptr(vv, f32p), T, d, n_sink, n_recent, N, rep,
+                                        _ptr(Dp, i64p), _ptr(Dout, i64p), _ptr(C, i64p), _ptr(b, i32p), _ptr(st, i32p),
+                                        _ptr(ln, i32p), _ptr(kt, f64p), _ptr(vt, f64p), _ptr(vv_, f64p), _ptr(s2, f64p),
+                                        _ptr(al, f64p), _ptr(be, f64p), _ptr(E, i32p))
+    _check(rc, "coarsen_unit_from_steps")
+    e = int(E[0])
+    return UnitNodes(Dout[:M].copy(), C[:M].copy(), np.zeros(M), b, st[:e].copy(), ln[:e].copy(), kt[:e].copy(),
+                     vt[:e].copy(), s2[:e].copy(), vv_[:e].copy(), al[:e].copy(), be[:e].copy(), s_eff, w_eff, M)
+
+
+def bf16_round(x: np.ndarray) -> np.ndarray:
+    """fp32 values rounded to the nearest bf16 (ties to even), returned as fp32 (finite inputs)."""
+    u = np.ascontiguousarray(x, np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).reshape(np.shape(x))
+
+
+def projection_bf16(seed: int, d: int) -> np.ndarray:
+    """P16 = bf16(P): the projection of the tensor-core option (SKV_PROJECTION_TENSOR_BF16)."""
+    return bf16_round(projection(seed, d))
+
+
+def tensor_steps_reference(k: np.ndarray, v: np.ndarray, n_sink: int, n_recent: int, P16: np.ndarray,
+                           mma_k_steps: int | None = None):
+    """The tensor-core option's steps against the exact P16 projection. Returns (d, bound), both
+    [M] fp64 in units of 2^-20: d the exact step ||P16 (x_t - x_{t-1})|| * 2^20 of the middle tokens
+    (x = [k; v]; every product of a bf16 feature and a bf16 entry is exact in fp64 and 2d of them
+    sum with fp64 error far below the bound), and bound a limit on |D_t - d_t| for any fp32
+    accumulation of those products in at most `mma_k_steps` (default 2d/16) accumulate steps of 16
+    products each, rounding or truncating every step to fp32 (error at most 18 units of 2^-23 of
+    the sum of magnitudes per step), followed by the fixed recipe's fp32 difference, square sum,
+    square root and rne quantisation."""
+    k = np.ascontiguousarray(k, np.float32).astype(np.float64)
+    v = np.ascontiguousarray(v, np.float32).astype(np.float64)
+    T, d = k.shape
+    s_eff, w_eff, M = split(T, n_sink, n_recent)
+    x = np.concatenate([k, v], axis=1)[s_eff:s_eff + M]
+    P = np.asarray(P16, np.float64)
+    z = x @ P.T
+    S = np.abs(x) @ np.abs(P).T                    # sum of magnitudes per token and output
+    nks = mma_k_steps if mma_k_steps is not None else 2 * d // 16
+    e = nks * 18.0 * 2.0 ** -23 * S                # per-output accumulation bound
+    dd = np.zeros(M)
+    bound = np.zeros(M)
+    if M > 1:
+        dz = z[1:] - z[:-1]
+        dd[1:] = np.sqrt((dz * dz).sum(axis=1))
+        err_z = np.sqrt(((e[1:] + e[:-1]) ** 2).sum(axis=1))
+        # fp32 difference, 16 fma steps, sqrt and scaling: a few dozen units of 2^-24 of d
+        bound[1:] = (err_z + 64 * 2.0 ** -24 * (dd[1:] + err_z)) * 2.0 ** 20 + 1.0
+    return dd * 2.0 ** 20, bound
+
+
 def _pool(threads: int | None):
     return ThreadPoolExecutor(max_workers=threads or os.cpu_count() or 1)
 
 
 def coarsen(seqs, n_sink: int, n_recent: int, N_list, seed: int, threads: int | None = None,
-            representative: str = "mean"):
+            representative: str = "mean", center: bool = False):
     """Coarsen a batch. seqs: list over sequences b of (k_b, v_b) arrays [Hkv, T_b, d].
     Returns nested list [b][h] of UnitNodes. The projection P is drawn from ``seed``."""
     d = seqs[0][0].shape[-1]
@@ -233,7 +337,7 @@ def coarsen(seqs, n_sink: int, n_recent: int, N_list, seed: int, threads: int | 
     res = {}
     with _pool(threads) as ex:
         futs = {ex.submit(coarsen_unit, seqs[b][0][h], seqs[b][1][h], n_sink, n_recent, int(N_list[b]), P,
-                          representative): (b, h)
+                          representative, center): (b, h)
                 for (b, h) in jobs}
         for f, key in futs.items():
             res[key] = f.result()

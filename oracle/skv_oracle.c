@@ -48,6 +48,12 @@
  *      s = q.k/sqrt(d) + ln m + sum_i q_i^2 var_i / (2d), var_i the members'
  *      population variance of key dimension i (orc_coarsen_unit2's var). With
  *      var_i = sigma^2 for every i it is the scalar form of R7.
+ *  R8  Option (orc_key_mean_f32): common-mode mean removal of [SK]
+ *      Independent Claim 1(b) (keys mapped into an anisotropy-reduced space
+ *      before coarsening): every key of a unit has the unit's mean key mu
+ *      (over all T tokens) subtracted in fp32, and the coarsening then runs on
+ *      the centred keys. Because the centred keys feed the fixed fp32
+ *      variation recipe, mu itself follows one fixed fp32 order.
  */
 #include <math.h>
 #include <stdint.h>
@@ -203,6 +209,28 @@ int orc_split(int T, int S, int W, int *S_eff, int *W_eff, int *M)
     return ORC_OK;
 }
 
+/* R8: the unit's mean key in a fixed fp32 order. Per dimension i, blocks of
+ * ORC_MEAN_BLOCK consecutive tokens are summed in token order from 0 (each
+ * addition an IEEE fp32 addition), the block sums are added in block order
+ * from 0, and the total is divided by T (IEEE fp32 division); mu = 0 for
+ * T = 0. The centred key is then fl32(k_ti - mu_i). */
+#define ORC_MEAN_BLOCK 256
+int orc_key_mean_f32(const float *k, int T, int d, float *mu)
+{
+    if (T < 0 || d < 1 || !mu || (T > 0 && !k)) return ORC_ERR_ARG;
+    for (int i = 0; i < d; ++i) {
+        float total = 0.0f;
+        for (int b0 = 0; b0 < T; b0 += ORC_MEAN_BLOCK) {
+            const int b1 = b0 + ORC_MEAN_BLOCK < T ? b0 + ORC_MEAN_BLOCK : T;
+            float blk = 0.0f;
+            for (int t = b0; t < b1; ++t) blk = blk + k[(long)t * d + i];
+            total = total + blk;
+        }
+        mu[i] = T > 0 ? total / (float)T : 0.0f;
+    }
+    return ORC_OK;
+}
+
 /* Node statistics of tokens [start, start + m) ([SK] Claim 2: mass, mean key,
  * mean value; Claim 3: subgrid key variance; section 2: alpha = log m,
  * beta = sigma^2 / (2 d_k)). Two-pass population variance in fp64.
@@ -258,16 +286,34 @@ static void orc_node_stats(const float *k, const float *v, int d, int start, int
  * [S_eff+N+W_eff]. *E receives the number of entries (sinks, nonempty
  * segments in order, recents). d64 (may be NULL) is the fp64 variation.
  */
-int orc_coarsen_unit2(const float *k, const float *v, int T, int d, int S, int W, int N,
-                      const float *P, int rep, int64_t *D, int64_t *C, double *d64, int32_t *b,
-                      int32_t *ent_start, int32_t *ent_len, double *kt, double *vt, double *var_vec,
-                      double *sig2, double *alpha, double *beta, int32_t *E)
+/* The coarsening of one unit; D_in (may be NULL): quantised steps given by the caller for the
+ * middle tokens (D_in[0] the first middle token's), in place of the fixed fp32 recipe -- the
+ * integer stages (prefix sums, first-hitting boundaries) and the node statistics then follow
+ * those steps (the stage-wise check of a projection computed another way). */
+static int coarsen_core(const float *k, const float *v, int T, int d, int S, int W, int N,
+                        const float *P, int rep, const int64_t *D_in, int64_t *D, int64_t *C, double *d64,
+                        int32_t *b, int32_t *ent_start, int32_t *ent_len, double *kt, double *vt,
+                        double *var_vec, double *sig2, double *alpha, double *beta, int32_t *E)
 {
     int s_eff, w_eff, M;
-    if (d <= 0 || N < 1 || !P || !b || !E) return ORC_ERR_ARG;
+    if (d <= 0 || N < 1 || (!P && !D_in) || !b || !E) return ORC_ERR_ARG;
     if (rep != 0 && (rep != 1 || !D)) return ORC_ERR_ARG;
     if (orc_split(T, S, W, &s_eff, &w_eff, &M) != ORC_OK) return ORC_ERR_ARG;
     if (M >= ORC_M_MAX) return ORC_ERR_OVERFLOW;
+    if (D_in) {
+        int64_t run = 0;
+        for (int t = 0; t < M; ++t) {
+            if (D_in[t] < 0 || D_in[t] > ((int64_t)1 << 40)) return ORC_ERR_ARG;
+            run += D_in[t];
+            if (D) D[t] = D_in[t];
+            if (C) C[t] = run;
+            if (d64) d64[t] = 0.0;
+        }
+        if (!C && M > 0) return ORC_ERR_ARG;   /* the given-steps path needs C for the boundaries */
+        int rc = orc_segment(C, M, N, b);
+        if (rc != ORC_OK) return rc;
+        goto entries;
+    }
 
     /* variation on the middle span [s_eff, s_eff + M) */
     float zp[ORC_PROJ_DIM], zc[ORC_PROJ_DIM];
@@ -315,6 +361,7 @@ int orc_coarsen_unit2(const float *k, const float *v, int T, int d, int S, int W
     if (Cw != C) free(Cw);
     if (rc != ORC_OK) return rc;
 
+entries:;
     /* entries: sinks, nonempty middle segments in order, recents */
     int e = 0;
     for (int t = 0; t < s_eff; ++t, ++e) { ent_start[e] = t; ent_len[e] = 1; }
@@ -331,6 +378,26 @@ int orc_coarsen_unit2(const float *k, const float *v, int T, int d, int S, int W
                        var_vec ? var_vec + (long)i * d : NULL, sig2 + i, alpha + i, beta + i);
     }
     return ORC_OK;
+}
+
+int orc_coarsen_unit2(const float *k, const float *v, int T, int d, int S, int W, int N,
+                      const float *P, int rep, int64_t *D, int64_t *C, double *d64, int32_t *b,
+                      int32_t *ent_start, int32_t *ent_len, double *kt, double *vt, double *var_vec,
+                      double *sig2, double *alpha, double *beta, int32_t *E)
+{
+    return coarsen_core(k, v, T, d, S, W, N, P, rep, NULL, D, C, d64, b, ent_start, ent_len, kt, vt, var_vec,
+                        sig2, alpha, beta, E);
+}
+
+/* orc_coarsen_unit2 from given quantised steps D_in[0..M) (see coarsen_core). */
+int orc_coarsen_unit_steps(const float *k, const float *v, int T, int d, int S, int W, int N, int rep,
+                           const int64_t *D_in, int64_t *D, int64_t *C, int32_t *b, int32_t *ent_start,
+                           int32_t *ent_len, double *kt, double *vt, double *var_vec, double *sig2,
+                           double *alpha, double *beta, int32_t *E)
+{
+    if (!D_in) return ORC_ERR_ARG;
+    return coarsen_core(k, v, T, d, S, W, N, NULL, rep, D_in, D, C, NULL, b, ent_start, ent_len, kt, vt,
+                        var_vec, sig2, alpha, beta, E);
 }
 
 /* orc_coarsen_unit2 with the plain-mean representative (R6). */

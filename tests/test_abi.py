@@ -33,11 +33,11 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in (0, -1, -2, -3, -4, -6, -7):
+    for code in (0, -1, -2, -3, -4, -5, -6, -7):
         s = lib.skv_status_string(code).decode()
         assert s.startswith("SKV_")
     assert "unknown" in lib.skv_status_string(12345).decode()
-    assert lib.skv_abi_version() == 202
+    assert lib.skv_abi_version() == 203
     assert lib.skv_page_bytes(1, 128) == 2 * 16 * 128 * 2 + 128
     assert lib.skv_page_bytes(0, 64) == 2 * 16 * 64 * 4 + 128
     assert lib.skv_page_bytes(1, 96) == 0
@@ -87,6 +87,25 @@ def test_bad_arguments_rejected_before_any_launch(lib):
                          ctypes.byref(pool2), ctypes.c_void_p(16), 3, ctypes.c_void_p(16), null, null,
                          ctypes.c_void_p(256), 1 << 30, null)
     assert st == _lib.SKV_ERR_INVALID_ARG
+
+
+def test_wait_selftest_and_noalloc_validated_before_any_launch(lib):
+    """The wait check rejects a missing, misaligned or too small workspace and a poll count above
+    the kernels' 2^20 limit before launching; the no-allocation decode applies skv_decode_attn's
+    argument rules (shared planning code) before touching its scratch."""
+    from compressed_decode_attention_equal_b200 import _lib
+    null = ctypes.c_void_p(0)
+    assert lib.skv_wait_selftest(null, 4096, 10, null) == _lib.SKV_ERR_WORKSPACE
+    assert lib.skv_wait_selftest(ctypes.c_void_p(512 + 16), 4096, 10, null) == _lib.SKV_ERR_WORKSPACE
+    assert lib.skv_wait_selftest(ctypes.c_void_p(512), 255, 10, null) == _lib.SKV_ERR_WORKSPACE
+    assert lib.skv_wait_selftest(ctypes.c_void_p(512), 4096, (1 << 20) + 1, null) == _lib.SKV_ERR_INVALID_ARG
+    pool = _lib.SkvNodePool(0, 0)
+    for args, want in (((1, 1, 1, 7, 1, 128), _lib.SKV_ERR_INVALID_ARG),     # null buffers
+                       ((1, 1, 1, 7, 2, 128), _lib.SKV_ERR_UNSUPPORTED),     # Hq % Hkv != 0
+                       ((1, 1, 1, 7, 1, 96), _lib.SKV_ERR_UNSUPPORTED),      # d
+                       ((1, 0, 1, 7, 1, 128), _lib.SKV_ERR_INVALID_ARG)):    # B < 1
+        st = lib.skv_decode_attn_noalloc(null, *args, ctypes.byref(pool), null, 4, null, null, null, null)
+        assert st == want, (args, st)
 
 
 def test_coarsen_options_validated_before_any_launch(lib):

@@ -21,7 +21,7 @@ S, W = workloads.N_SINK, workloads.N_RECENT
 
 
 def run_coarsen(k, v, Hkv, T_list, N_list, seed, n_sink=S, n_recent=W, shuffle=True, representative="mean",
-                closure="scalar"):
+                closure="scalar", center_keys=False, projection="fixed"):
     B = len(T_list)
     d = k.shape[-1]
     ent = [skv.entries_bound(T, N, n_sink, n_recent) for T, N in zip(T_list, N_list)]
@@ -32,12 +32,14 @@ def run_coarsen(k, v, Hkv, T_list, N_list, seed, n_sink=S, n_recent=W, shuffle=T
     ws = torch.zeros(skv.coarsen_workspace_bytes(Hkv, d, T_list, N_list, n_sink, n_recent), dtype=torch.uint8,
                      device="cuda")
     lens = skv.coarsen(k, v, Hkv, T_list, N_list, n_sink, n_recent, seed, pool, table, boundaries=bnd, cumvar=cum,
-                       workspace=ws, representative=representative)
+                       workspace=ws, representative=representative, center_keys=center_keys,
+                       projection=projection)
     st, flags = skv.workspace_error(ws)
     return dict(pool=pool, table=table, lens=lens, bnd=bnd, cum=cum, status=st, flags=flags)
 
 
-def oracle_units(k, v, Hkv, T_list, N_list, seed, units=None, n_sink=S, n_recent=W, representative="mean"):
+def oracle_units(k, v, Hkv, T_list, N_list, seed, units=None, n_sink=S, n_recent=W, representative="mean",
+                 center=False):
     d = k.shape[-1]
     P = oracle.projection(seed, d)
     res = {}
@@ -47,11 +49,11 @@ def oracle_units(k, v, Hkv, T_list, N_list, seed, units=None, n_sink=S, n_recent
                 continue
             kk = to_np32(workloads.unit_rows(k, T_list, Hkv, b, h))
             vv = to_np32(workloads.unit_rows(v, T_list, Hkv, b, h))
-            res[(b, h)] = oracle.coarsen_unit(kk, vv, n_sink, n_recent, int(N_list[b]), P, representative)
+            res[(b, h)] = oracle.coarsen_unit(kk, vv, n_sink, n_recent, int(N_list[b]), P, representative, center)
     return res
 
 
-def compare_units(r, orc, k, v, T_list, Hkv, N_list, dtype):
+def compare_units(r, orc, k, v, T_list, Hkv, N_list, dtype, center=False):
     d = k.shape[-1]
     for (b, h), u in orc.items():
         what = f"unit ({b},{h}) T={T_list[b]} N={N_list[b]}"
@@ -65,6 +67,8 @@ def compare_units(r, orc, k, v, T_list, Hkv, N_list, dtype):
         assert int(r["lens"][b, h]) == u.kt.shape[0], f"{what}: lens"
         gu = gpu_unit(r["pool"], r["table"], r["lens"], b, h)
         kk = to_np32(workloads.unit_rows(k, T_list, Hkv, b, h))
+        if center:
+            kk = oracle.center_keys(kk)
         vv = to_np32(workloads.unit_rows(v, T_list, Hkv, b, h))
         check_nodes(gu, u, dtype, d, what, slack=weighted_slack(u, kk, vv))
 
@@ -276,3 +280,120 @@ def test_coarsen_is_deterministic():
     assert torch.equal(a["pool"].k.view(torch.int16), b["pool"].k.view(torch.int16))
     assert torch.equal(a["pool"].v.view(torch.int16), b["pool"].v.view(torch.int16))
     assert torch.equal(a["pool"].ab.view(torch.int32), b["pool"].ab.view(torch.int32))
+
+
+CENTER_CASES = [c for c in CASES if c[0] in ("bf16_d128_multi_tile", "bf16_d64", "f32_d64", "f32_d128",
+                                             "short_sequences", "tile_edges", "many_units_ragged")]
+
+
+@pytest.mark.parametrize("representative", ["mean", "variation"])
+@pytest.mark.parametrize("name,dtype,d,Hkv,T_list,N_list,values", CENTER_CASES, ids=[c[0] for c in CENTER_CASES])
+def test_coarsen_centred_keys_matches_oracle(name, dtype, d, Hkv, T_list, N_list, values, representative):
+    """Common-mode mean removal ("SPICY-KV" Claim 1(b)): the GPU's centred keys, built from its own
+    fixed-order mean key, give c_t and boundaries bit-exact with the oracle's pipeline on the
+    oracle's centred keys (a single differing bit of mu would move the fixed fp32 steps), and node
+    statistics of the centred keys within tolerance. Keys carry a strong common mode."""
+    seed = sum(T_list) + d + 5
+    w = workloads.Workload(name, seed, B=len(T_list), Hq=Hkv, Hkv=Hkv, d=d, R=1,
+                           dtype="bf16" if dtype == torch.bfloat16 else "f32", T=0, regimes=12)
+    k, v, _ = workloads.make_kv(w, "cuda", T_list=T_list, values=values)
+    g = torch.Generator(device="cuda").manual_seed(seed)
+    k = (k.float() + 6.0 * torch.randn(1, d, device="cuda", generator=g)).to(dtype)
+    r = run_coarsen(k, v, Hkv, T_list, N_list, seed, representative=representative, center_keys=True)
+    assert r["status"] == 0, f"device flags {r['flags']}"
+    orc = oracle_units(k, v, Hkv, T_list, N_list, seed, representative=representative, center=True)
+    compare_units(r, orc, k, v, T_list, Hkv, N_list, dtype, center=True)
+    # the stored keys are centred: per unit the plain means average to about zero, weighted by mass
+    for (b, h), u in orc.items():
+        if representative == "mean" and u.kt.shape[0] and T_list[b] > 0:
+            centre = (u.kt * u.mass[:, None]).sum(axis=0) / u.mass.sum()
+            assert np.abs(centre).max() < 1e-3 * (1 + np.abs(to_np32(workloads.unit_rows(k, T_list, Hkv, b, h))).max())
+
+
+def test_centred_tiny_f32_decode_keeps_outputs_and_shifts_lse():
+    """tiny_f32 with a common mode added to the keys, coarsened with and without centring: the
+    centred pool decodes to the same outputs (fp32 bar) and lse lower by q.mu/sqrt(d), mu the
+    oracle's fixed-order mean key, whenever the two segmentations agree; and the centred pool's
+    decode matches the oracle on the oracle's centred nodes."""
+    w = workloads.WORKLOADS["tiny_f32"]
+    k, v, T_list = workloads.make_kv(w, "cuda")
+    k = k + 4.0 * torch.randn(1, w.d, device="cuda", generator=torch.Generator(device="cuda").manual_seed(3))
+    N_list = workloads.segment_counts(w, T_list)
+    plain = run_coarsen(k, v, w.Hkv, T_list, N_list, w.seed)
+    cent = run_coarsen(k, v, w.Hkv, T_list, N_list, w.seed, center_keys=True)
+    assert plain["status"] == 0 and cent["status"] == 0
+    orc = oracle_units(k, v, w.Hkv, T_list, N_list, w.seed, center=True)
+    compare_units(cent, orc, k, v, T_list, w.Hkv, N_list, torch.float32, center=True)
+    q = workloads.make_queries(w, "cuda")
+    out_c, lse_c = skv.decode_attn(q, w.Hkv, cent["pool"], cent["table"], cent["lens"])
+    ref_out, ref_lse = oracle.decode(q.double().cpu().numpy(), [[orc[(0, 0)]]])
+    check_decode(out_c, lse_c, ref_out, ref_lse, torch.float32, "centred tiny_f32")
+    if torch.equal(plain["bnd"], cent["bnd"]):
+        out_p, lse_p = skv.decode_attn(q, w.Hkv, plain["pool"], plain["table"], plain["lens"])
+        mu = oracle.key_mean_f32(to_np32(k)).astype(np.float64)
+        qq = q.double().cpu().numpy()
+        shift = (qq @ mu) / np.sqrt(w.d)
+        np.testing.assert_allclose(out_c.double().cpu().numpy(), out_p.double().cpu().numpy(), rtol=0, atol=2e-5)
+        np.testing.assert_allclose(lse_p.double().cpu().numpy() - lse_c.double().cpu().numpy(), shift, rtol=0,
+                                   atol=2e-4 * (1 + np.abs(shift).max()))
+
+
+def tensor_units(r, k, v, Hkv, T_list, N_list, seed, representative="mean", center=False):
+    """The stage-wise oracle of the tensor-core projection: every step within the bound of the exact
+    bf16 projection's step, then the oracle's integer stages and statistics driven by the GPU's own
+    steps (recovered from its cumulative variation)."""
+    d = k.shape[-1]
+    P16 = oracle.projection_bf16(seed, d)
+    res = {}
+    for b, T in enumerate(T_list):
+        for h in range(Hkv):
+            kk = to_np32(workloads.unit_rows(k, T_list, Hkv, b, h))
+            vv = to_np32(workloads.unit_rows(v, T_list, Hkv, b, h))
+            M = max(0, T - min(S, T) - min(W, T - min(S, T)))
+            off = sum(T_list[:b]) * Hkv + h * T
+            C = r["cum"][off:off + M].cpu().numpy()
+            D = np.diff(C, prepend=0)
+            dref, bound = oracle.tensor_steps_reference(kk, vv, S, W, P16)
+            bad = np.flatnonzero(np.abs(D - dref) > bound)
+            assert bad.size == 0, f"unit ({b},{h}): steps outside the bound at {bad[:5]}"
+            assert M == 0 or D[0] == 0
+            res[(b, h)] = oracle.coarsen_unit_from_steps(kk, vv, S, W, int(N_list[b]), D, representative, center)
+    return res
+
+
+TC_CASES = [c for c in CASES if c[1] == torch.bfloat16]
+
+
+@pytest.mark.parametrize("name,dtype,d,Hkv,T_list,N_list,values", TC_CASES, ids=[c[0] for c in TC_CASES])
+def test_coarsen_tensor_projection_stagewise(name, dtype, d, Hkv, T_list, N_list, values):
+    """SKV_PROJECTION_TENSOR_BF16: steps within the fp32 accumulation bound of the exact bf16
+    projection; given those steps, c_t, boundaries and entry counts bit-exact and node statistics
+    within tolerance (the oracle's integer stages and statistics fed the GPU's steps)."""
+    seed = sum(T_list) + d + 9
+    w = workloads.Workload(name, seed, B=len(T_list), Hq=Hkv, Hkv=Hkv, d=d, R=1, dtype="bf16", T=0, regimes=12)
+    k, v, _ = workloads.make_kv(w, "cuda", T_list=T_list, values=values)
+    r = run_coarsen(k, v, Hkv, T_list, N_list, seed, projection="tensor")
+    assert r["status"] == 0, f"device flags {r['flags']}"
+    orc = tensor_units(r, k, v, Hkv, T_list, N_list, seed)
+    compare_units(r, orc, k, v, T_list, Hkv, N_list, dtype)
+
+
+def test_tensor_projection_with_centred_keys_and_weighted_representative():
+    """The option composes with centring (the projection reads the raw keys; statistics are of the
+    centred keys) and with the variation-weighted representative (weights are the GPU's steps)."""
+    T_list, N_list, Hkv, d = [1300, 700], [40, 20], 2, 128
+    seed = 77
+    w = workloads.Workload("tc_combo", seed, B=2, Hq=Hkv, Hkv=Hkv, d=d, R=1, dtype="bf16", T=0, regimes=12)
+    k, v, _ = workloads.make_kv(w, "cuda", T_list=T_list)
+    k = (k.float() + 5.0).bfloat16()
+    r = run_coarsen(k, v, Hkv, T_list, N_list, seed, projection="tensor", center_keys=True,
+                    representative="variation")
+    assert r["status"] == 0
+    orc = tensor_units(r, k, v, Hkv, T_list, N_list, seed, representative="variation", center=True)
+    compare_units(r, orc, k, v, T_list, Hkv, N_list, torch.bfloat16, center=True)
+
+
+def test_tensor_projection_rejects_fp32_inputs():
+    k = torch.zeros(200, 64, device="cuda")
+    with pytest.raises(skv.SkvError):
+        run_coarsen(k, k.clone(), 1, [200], [4], 1, projection="tensor")

@@ -78,3 +78,39 @@ def test_two_ranks_max_over_ranks_and_job_throughput(tmp_path):
 def test_rank_that_leaves_fails_the_next_collective(tmp_path):
     r0, r1 = _spawn(tmp_path, "leave")
     assert r1["left"] and r0["error"] is not None
+
+
+def _bench_json(stdout: str):
+    lines = [ln for ln in stdout.splitlines() if ln.startswith("{")]
+    assert len(lines) == 1, stdout
+    return json.loads(lines[0])
+
+
+def test_bench_gpus_flag_launches_that_many_ranks():
+    """`bench.py --gpus 2` outside torchrun runs itself as two ranks (torch.distributed.run on
+    127.0.0.1); the reference arm, which needs no GPU, prints one line from rank 0 with n_gpus 2
+    and the same `config` object the GPU arm prints."""
+    import subprocess
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_PORT")}
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "3", "--ref-seconds", "1"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert p.returncode == 0, p.stderr[-2000:]
+    res = _bench_json(p.stdout)
+    assert res["n_gpus"] == 2 and res["impl"] == "reference"
+    sys.path.insert(0, ROOT)
+    import bench
+    import workloads
+    assert res["config"] == bench.bench_config(workloads.WORKLOADS[bench.WORKLOAD], 2)
+    assert res["cpu_baseline"]["kind"] == "oracle" and res["e2e"]["h2d_bytes_per_step"] == 0
+
+
+def test_bench_refuses_a_rank_count_other_than_gpus():
+    """Under a launcher whose WORLD_SIZE differs from --gpus the bench stops with an error naming
+    the mismatch instead of timing a different number of GPUs."""
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="3", RANK="0", LOCAL_RANK="0")
+    p = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "3", "--ref-seconds", "1"],
+                       capture_output=True, text=True, timeout=120, env=env, cwd=ROOT)
+    assert p.returncode != 0 and "WORLD_SIZE=3" in (p.stderr + p.stdout)

@@ -59,3 +59,88 @@ def test_decode_is_invariant_to_a_common_key_shift():
         o2, l2 = oracle.decode_rows(q, kt - mu, vt, alpha, beta, extra)
         np.testing.assert_allclose(o2, o1, rtol=0, atol=1e-12)
         np.testing.assert_allclose(l1 - l2, q @ mu / np.sqrt(d), rtol=0, atol=1e-11)
+
+
+# ---------------------------------------------------------------------------
+# the centring option's mean key: one fixed fp32 order (reading R8)
+# ---------------------------------------------------------------------------
+from fractions import Fraction  # noqa: E402
+
+import exact_f32  # noqa: E402
+
+
+def _blocked_mean_exact_model(k):
+    """The R8 order evaluated with the exact-rational binary32 model: every addition and the final
+    division rounded once to binary32 (ties to even)."""
+    T, d = k.shape
+    mu = np.zeros(d, np.float32)
+    for i in range(d):
+        total = 0.0
+        for b0 in range(0, T, 256):
+            blk = 0.0
+            for t in range(b0, min(b0 + 256, T)):
+                blk = exact_f32.round_f32(exact_f32.f(blk) + exact_f32.f(k[t, i]))
+            total = exact_f32.round_f32(exact_f32.f(total) + exact_f32.f(blk))
+        mu[i] = exact_f32.round_f32(exact_f32.f(total) / T) if T else 0.0
+    return mu
+
+
+def _order_sensitive_keys(T, d, seed):
+    rng = np.random.default_rng(seed)
+    # mixed magnitudes, so that the rounding of each partial sum depends on the summation order
+    mag = 10.0 ** rng.integers(-3, 4, size=(T, d))
+    return (rng.standard_normal((T, d)) * mag + 37.0).astype(np.float32)
+
+
+def test_key_mean_bits_follow_the_blocked_fp32_order():
+    for T, seed in ((700, 1), (256, 2), (255, 3), (1, 4), (513, 5)):
+        k = _order_sensitive_keys(T, 4, seed)
+        got = oracle.key_mean_f32(k)
+        want = _blocked_mean_exact_model(k)
+        assert np.array_equal(got.view(np.uint32), want.view(np.uint32)), (T, got, want)
+    assert np.array_equal(oracle.key_mean_f32(np.zeros((0, 3), np.float32)), np.zeros(3, np.float32))
+
+
+def test_key_mean_order_is_what_the_pin_sees():
+    """The data above is order sensitive: one sequential fp32 sum over all tokens (no blocks) gives
+    other bits in some dimension, so the bit pin would catch a wrong order."""
+    k = _order_sensitive_keys(700, 8, 1)
+    seq = np.zeros(8, np.float32)
+    for t in range(700):
+        seq = (seq + k[t]).astype(np.float32)
+    naive = (seq / np.float32(700)).astype(np.float32)
+    assert not np.array_equal(naive.view(np.uint32), oracle.key_mean_f32(k).view(np.uint32))
+
+
+def test_key_mean_within_the_fp32_summation_bound_and_exact_on_integers():
+    k = _order_sensitive_keys(5000, 6, 7)
+    mu = oracle.key_mean_f32(k).astype(np.float64)
+    exact = np.array([float(sum(Fraction(float(x)) for x in k[:, i]) / 5000) for i in range(6)])
+    # blocked summation: at most (256 + 20) additions on any path, each within 2^-24 relative
+    bound = (256 + 20 + 1) * 2.0 ** -24 * np.abs(k.astype(np.float64)).sum(axis=0) / 5000 + 2.0 ** -24 * np.abs(exact)
+    assert np.all(np.abs(mu - exact) <= bound)
+    ints = np.random.default_rng(8).integers(-1000, 1000, size=(3000, 5)).astype(np.float32)
+    np.testing.assert_array_equal(oracle.key_mean_f32(ints),
+                                  (ints.astype(np.float64).sum(axis=0) / 3000).astype(np.float32))
+
+
+def test_centred_coarsening_runs_on_the_centred_keys():
+    """coarsen_unit(center=True) equals coarsen_unit on center_keys(k); the centred keys average to
+    about zero; the value statistics and masses do not depend on the option."""
+    rng = np.random.default_rng(23)
+    T, d, N = 2000, 64, 40
+    k = (rng.standard_normal(d) * 5 + np.cumsum(rng.standard_normal((T, d)) * 0.05, axis=0)).astype(np.float32)
+    v = rng.standard_normal((T, d)).astype(np.float32)
+    P = oracle.projection(9, d)
+    a = oracle.coarsen_unit(k, v, S, W, N, P, center=True)
+    kc = oracle.center_keys(k)
+    b = oracle.coarsen_unit(kc, v, S, W, N, P)
+    np.testing.assert_array_equal(a.C, b.C)
+    np.testing.assert_array_equal(a.bounds, b.bounds)
+    np.testing.assert_array_equal(a.kt, b.kt)
+    assert np.abs(kc.astype(np.float64).mean(axis=0)).max() < 1e-4 * np.abs(k).max()
+    plain = oracle.coarsen_unit(k, v, S, W, N, P)
+    if np.array_equal(plain.bounds, a.bounds):
+        np.testing.assert_allclose(a.vt, plain.vt, rtol=0, atol=0)
+        np.testing.assert_array_equal(a.mass, plain.mass)
+        np.testing.assert_allclose(a.sigma2, plain.sigma2, rtol=1e-4, atol=1e-9)
