@@ -312,20 +312,20 @@ def coarsen_stage(device, reps: int = 5):
                      dtype=torch.uint8, device=device)
     flush = torch.empty(256 << 20, dtype=torch.uint8, device=device)
 
-    def call(representative):
+    def call(**opts):
         skv.coarsen(k, v, w.Hkv, T_list, N_list, workloads.N_SINK, workloads.N_RECENT, w.seed, pool, table,
-                    lens=lens, workspace=ws, representative=representative)
+                    lens=lens, workspace=ws, **opts)
 
-    def timed(representative):
+    def timed(**opts):
         for _ in range(2):
-            call(representative)
+            call(**opts)
         torch.cuda.synchronize()
         times = []
         for _ in range(reps):
             flush.zero_()                      # evict the raw KV from L2 between calls
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record()
-            call(representative)
+            call(**opts)
             e1.record()
             torch.cuda.synchronize()
             times.append(e0.elapsed_time(e1))
@@ -334,8 +334,10 @@ def coarsen_stage(device, reps: int = 5):
             raise RuntimeError(f"coarsening raised device flags {flags}")
         return statistics.median(times)
 
-    ms_weighted = timed("variation")
-    ms = timed("mean")
+    ms_weighted = timed(representative="variation")
+    ms_centred = timed(center_keys=True)
+    ms_tensor = timed(projection="tensor")
+    ms = timed()
     tokens = sum(T_list) * w.Hkv
     raw_bytes = 2 * tokens * w.d * 2
     ent = int(lens.sum())
@@ -360,6 +362,16 @@ def coarsen_stage(device, reps: int = 5):
         "variation_weighted": {"ms": ms_weighted, "tokens_per_s": tokens / (ms_weighted / 1e3),
                                "frac": alg / (ms_weighted / 1e3) / 1e9 / peak,
                                "note": "same call with the variation-weighted segment representative"},
+        "centred_keys": {"ms": ms_centred, "tokens_per_s": tokens / (ms_centred / 1e3),
+                         "frac": alg / (ms_centred / 1e3) / 1e9 / peak,
+                         "note": "same call with common-mode mean removal (one more read of the keys)"},
+        "tensor_projection": {
+            "ms": ms_tensor, "tokens_per_s": tokens / (ms_tensor / 1e3),
+            "roofline": {"bound": "hbm", "achieved": alg / (ms_tensor / 1e3) / 1e9, "peak": peak, "unit": "GB/s",
+                         "frac": alg / (ms_tensor / 1e3) / 1e9 / peak, "peak_source": src,
+                         "algorithmic_bytes": alg},
+            "note": "same call with the tensor-core bf16 projection option (steps checked stage by stage, not "
+                    "bit-exact with the fixed fp32 recipe)"},
     }
 
 

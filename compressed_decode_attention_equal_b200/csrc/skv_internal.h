@@ -68,6 +68,7 @@ struct CoarsenArgs {
     int closure;         // skv_closure: SKV_CLOSURE_DIAGONAL also writes per-dimension variances
     int center;          // 1: keys enter every stage with the unit's mean key removed
     int projection;      // skv_projection: SKV_PROJECTION_TENSOR_BF16 selects k_project_tc
+    int unit0;           // first unit of the launch (the per-unit kernels run over a wave of units)
     int max_blk;         // largest ceil(T / kMeanBlock) over the batch
     float *key_blk;      // [units][max_blk][d] per-block key sums (centring only)
     float *key_mu;       // [units][d] mean key of each unit (centring only)
@@ -91,7 +92,9 @@ struct StreamHdr {
     int ring;          // recent ring position of the oldest recent token
     int n_ent;         // entries (= lens)
     int N, S, W;       // segment count, sinks, recent window
-    int pad[7];
+    int open;          // entry of the open (last) middle node
+    int open_page;     // its page id
+    int pad[5];
     float z_last[16];  // feature of the last middle token
 };
 static_assert(sizeof(StreamHdr) == 128, "StreamHdr layout");
@@ -109,6 +112,10 @@ struct StreamArgs {
     int64_t unit_bytes;          // state bytes per unit
     int NM, Ecap;                // node-order capacity, entry capacity per unit
     int64_t off_order, off_recent, off_owner, off_m, off_start, off_V, off_M2, off_mk, off_mv;
+    // kept so that an append finds everything it needs one round trip after the header:
+    int64_t off_vord;     // [NM] int64 V of the middle nodes in node order (beside order)
+    int64_t off_rpage;    // [W] int32 page id of each recent ring position's pool slot
+    int64_t off_ring;     // [W][2][d] fp32 raw key and value of each recent ring position
     uint32_t *flags;
 };
 

@@ -13,6 +13,12 @@
 //
 // k_stream_init builds the per-unit state after the offline coarsening of the prompt (same
 // workspace: entry list and tile-local variation scans); k_stream_append runs one CTA per unit.
+// The append is a chain of dependent memory round trips, so the state keeps beside each node
+// list what lets the append issue every load it needs right after reading the unit's header:
+// the nodes' variations in node order, the open node and its page, and the recent window's raw
+// keys and values with their pages. One more round trip fetches the merged pair when a merge
+// follows a split. A merge always follows a split (the node count is at most N before the
+// append), so the entry it frees is refilled by the new node, the last entry.
 // Entries of a unit live in pool slots [0, lens) in no particular order: a merge frees a slot,
 // which the unit's last entry then fills (decode attention does not depend on entry order).
 #include <climits>
@@ -51,7 +57,9 @@ template <int D, typename T>
 struct UnitState {
     StreamHdr *hdr;
     int *order, *recent, *owner, *m, *start;
-    long long *V;
+    long long *V, *vord;
+    int *rpage;
+    float *ring;
     double *M2, *mk, *mv;
     __device__ UnitState(const StreamArgs &s, int u) {
         uint8_t *base = s.state + static_cast<int64_t>(u) * s.unit_bytes;
@@ -65,20 +73,11 @@ struct UnitState {
         M2 = reinterpret_cast<double *>(base + s.off_M2);
         mk = reinterpret_cast<double *>(base + s.off_mk);
         mv = reinterpret_cast<double *>(base + s.off_mv);
+        vord = reinterpret_cast<long long *>(base + s.off_vord);
+        rpage = reinterpret_cast<int *>(base + s.off_rpage);
+        ring = reinterpret_cast<float *>(base + s.off_ring);
     }
 };
-
-// page of entry e of unit u, or nullptr (flag raised) if the page id is outside the pool
-template <int D, typename T>
-__device__ __forceinline__ uint8_t *entry_page(const StreamArgs &s, int u, int e) {
-    const int32_t page = s.page_table[static_cast<int64_t>(u) * s.max_pages + e / kPageNodes];
-    if (page < 0 || page >= s.num_pages) {
-        raise_flag(s.flags, FLAG_BAD_PAGE);
-        return nullptr;
-    }
-    constexpr int VEC = kPageNodes * D * Elem<T>::SIZE;
-    return s.pages + static_cast<int64_t>(page) * (2 * VEC + kPageNodes * 8);
-}
 
 // block-wide sum of a double (all threads return it)
 __device__ double block_sum(double x, double *red) {
@@ -103,25 +102,6 @@ __device__ long long block_sum_ll(long long x, long long *red) {
     long long t = 0;
     for (int w = 0; w < kStreamThreads / 32; ++w) t += red[w];
     return t;
-}
-
-// write node e's mean key, mean value, alpha, beta into its pool slot (pg: its page if known)
-template <int D, typename T>
-__device__ void write_node(const StreamArgs &s, const UnitState<D, T> &st, int u, int e, uint8_t *pg = nullptr) {
-    if (!pg) pg = entry_page<D, T>(s, u, e);
-    if (!pg) return;
-    constexpr int VEC = kPageNodes * D * Elem<T>::SIZE;
-    const int slot = e % kPageNodes;
-    for (int dim = threadIdx.x; dim < D; dim += kStreamThreads) {
-        Elem<T>::put(pg + vec_off<D, T>(slot, dim), static_cast<float>(st.mk[static_cast<int64_t>(e) * D + dim]));
-        Elem<T>::put(pg + VEC + vec_off<D, T>(slot, dim), static_cast<float>(st.mv[static_cast<int64_t>(e) * D + dim]));
-    }
-    if (threadIdx.x == 0) {
-        const int m = st.m[e];
-        const double sig2 = st.M2[e] / (static_cast<double>(m) * D);
-        reinterpret_cast<float2 *>(pg + 2 * VEC)[slot] =
-            make_float2(m == 1 ? 0.0f : logf(static_cast<float>(m)), static_cast<float>(sig2 / (2.0 * D)));
-    }
 }
 
 // z = P [k; v] by the fixed recipe (z_i an fp32 fma chain over j ascending from 0); thread i < 16.
@@ -198,8 +178,18 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_init(const CoarsenArg
             st.m[e] = m;
             st.start[e] = tok;
             st.V[e] = V;
+            st.vord[i] = V;
             st.M2[e] = M2;
         }
+    }
+    // the recent window: ring position r holds token T - W + r in pool slot s_eff + n_mid + r
+    for (int r = 0; r < sr.w_eff; ++r) {
+        const int tok = sr.T - sr.w_eff + r;
+        for (int dim = tid; dim < D; dim += kStreamThreads) {
+            st.ring[(static_cast<int64_t>(r) * 2) * D + dim] = static_cast<float>(kraw[static_cast<int64_t>(tok) * D + dim]);
+            st.ring[(static_cast<int64_t>(r) * 2 + 1) * D + dim] = static_cast<float>(vraw[static_cast<int64_t>(tok) * D + dim]);
+        }
+        if (tid == 0) st.rpage[r] = s.page_table[static_cast<int64_t>(u) * s.max_pages + (sr.s_eff + n_mid + r) / kPageNodes];
     }
     // the projection, kept for the appends (small kernel parameters keep their launches cheap)
     if (u == 0)
@@ -221,6 +211,8 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_init(const CoarsenArg
         st.hdr->N = sr.N;
         st.hdr->S = sr.s_eff;
         st.hdr->W = sr.w_eff;
+        st.hdr->open = sr.s_eff + n_mid - 1;
+        st.hdr->open_page = s.page_table[static_cast<int64_t>(u) * s.max_pages + (sr.s_eff + n_mid - 1) / kPageNodes];
     }
 }
 
@@ -241,25 +233,30 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
     long long *sV = reinterpret_cast<long long *>(dsm + 2 * D * kProjDim * 4);  // [NM] V in node order
     int *sOrder = reinterpret_cast<int *>(sV + s.NM);                          // [NM] node order
     __shared__ float ky[D], vy[D];
-    __shared__ float zy[kProjDim];
+    __shared__ float zy[kProjDim], zl[kProjDim];
     __shared__ double red_d[kStreamThreads / 32];
-    __shared__ int sh_split, sh_merge_j, sh_pos, sh_ok, sh_yslot, sh_open, sh_mopen;
-    __shared__ long long sh_D, sh_Vopen;
-    __shared__ uint8_t *sh_opage;
+    __shared__ int sh_yslot, sh_ypage, sh_mopen, sh_newpage, sh_split, sh_merge_j, sh_pa, sh_pb, sh_ma, sh_mb;
+    __shared__ long long sh_D, sh_Vo;
+    __shared__ double sh_M2open, sh_M2a, sh_M2b;
     __shared__ unsigned long long sh_bmin;
-    __shared__ float zl[kProjDim];
     const int u = blockIdx.x;
     const int tid = threadIdx.x;
     UnitState<D, T> st(s, u);
     StreamHdr &H = *st.hdr;
     constexpr int VEC = kPageNodes * D * Elem<T>::SIZE;
-    // The loads are grouped into rounds of independent requests (every round is one L2 round trip):
-    // header; ring slot, open node, last feature and projection; page id and the open node's
-    // statistics; the leaving token.
-    const int W = H.W, N = H.N;
-    int n_nodes = H.n_nodes, n_ent = H.n_ent;
-    const int ring = H.ring;
-    {   // the projection: every load in flight at once
+    constexpr int PAGE = 2 * VEC + kPageNodes * 8;
+
+    // round trip 0: the header
+    const int W = H.W, N = H.N, n_nodes0 = H.n_nodes, n_ent0 = H.n_ent, ring = H.ring, Tcur = H.T;
+    const int open = H.open, open_page = H.open_page;
+    const long long cT0 = H.cT;
+
+    // round trip 1: every other input the append may need, all loads in flight together -- the
+    // projection, the last middle feature, the leaving token y (from the recent ring) and its pool
+    // slot, the new token, the open node's statistics, the page of the slot a new node would take,
+    // and, when the node count is at N (a split is then followed by a merge), the node order with
+    // the nodes' variations
+    {
         constexpr int NV4 = 2 * D * kProjDim / 4 / kStreamThreads;
         float4 p4[NV4];
 #pragma unroll
@@ -267,34 +264,58 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
 #pragma unroll
         for (int r = 0; r < NV4; ++r) reinterpret_cast<float4 *>(sP)[r * kStreamThreads + tid] = p4[r];
     }
-    if (tid == 0) sh_yslot = st.recent[ring];
-    if (tid == 32) sh_open = n_nodes >= 1 ? st.order[n_nodes - 1] : -1;
-    if (tid >= 64 && tid < 64 + kProjDim) zl[tid - 64] = H.z_last[tid - 64];
-    __syncthreads();
-    const int yslot = sh_yslot, open = sh_open;
-    if (tid == 0) sh_ok = open >= 0 && entry_page<D, T>(s, u, yslot) != nullptr;
-    if (tid == 32 && open >= 0) {
-        sh_Vopen = st.V[open];
-        sh_mopen = st.m[open];
-        sh_opage = entry_page<D, T>(s, u, open);
-    }
-    // the open node's running means (used if y joins it)
+    float kn = 0.0f, vn = 0.0f;   // the new token (dimension tid)
     double mk_o = 0.0, mv_o = 0.0;
-    if (tid < D && open >= 0) {
+    if (tid < D) {
+        ky[tid] = st.ring[(static_cast<int64_t>(ring) * 2) * D + tid];
+        vy[tid] = st.ring[(static_cast<int64_t>(ring) * 2 + 1) * D + tid];
+        kn = static_cast<float>(static_cast<const T *>(s.k_new)[static_cast<int64_t>(u) * D + tid]);
+        vn = static_cast<float>(static_cast<const T *>(s.v_new)[static_cast<int64_t>(u) * D + tid]);
         mk_o = st.mk[static_cast<int64_t>(open) * D + tid];
         mv_o = st.mv[static_cast<int64_t>(open) * D + tid];
     }
-    __syncthreads();
-    if (!sh_ok) return;
-
-    // 1. the oldest recent token y leaves the window: read it from its pool slot
-    const uint8_t *ypg = entry_page<D, T>(s, u, yslot);
-    for (int dim = tid; dim < D; dim += kStreamThreads) {
-        ky[dim] = Elem<T>::get(ypg + vec_off<D, T>(yslot % kPageNodes, dim));
-        vy[dim] = Elem<T>::get(ypg + VEC + vec_off<D, T>(yslot % kPageNodes, dim));
+    if (tid >= 64 && tid < 64 + kProjDim) zl[tid - 64] = H.z_last[tid - 64];
+    if (tid == 0) {
+        sh_yslot = st.recent[ring];
+        sh_ypage = st.rpage[ring];
+        sh_Vo = st.vord[n_nodes0 - 1];
+    }
+    if (tid == 32) {
+        sh_mopen = st.m[open];
+        sh_M2open = st.M2[open];
+        sh_newpage = n_ent0 < s.Ecap ? s.page_table[static_cast<int64_t>(u) * s.max_pages + n_ent0 / kPageNodes] : -1;
+    }
+    const bool may_merge = n_nodes0 >= N;
+    if (may_merge) {
+        for (int j0 = 0; j0 < n_nodes0; j0 += 4 * kStreamThreads) {
+            int o[4];
+            long long vv[4];
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int j = j0 + r * kStreamThreads + tid;
+                o[r] = j < n_nodes0 ? st.order[j] : 0;
+                vv[r] = j < n_nodes0 ? st.vord[j] : 0;
+            }
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                const int j = j0 + r * kStreamThreads + tid;
+                if (j < n_nodes0) {
+                    sOrder[j] = o[r];
+                    sV[j] = vv[r];
+                }
+            }
+        }
     }
     __syncthreads();
-    // 2. its variation step, then first hitting on the open node's budget
+    const int yslot = sh_yslot, ypage = sh_ypage, m_open = sh_mopen;
+    if (ypage < 0 || ypage >= s.num_pages) {
+        if (tid == 0) raise_flag(s.flags, FLAG_BAD_PAGE);
+        return;
+    }
+    uint8_t *ypg = s.pages + static_cast<int64_t>(ypage) * PAGE;
+
+    // the leaving token's step (the offline fixed fp32 recipe), then first hitting on the open
+    // node's budget
     if (tid < kProjDim) zy[tid] = feature_i(sP, ky, vy, D, tid);
     __syncthreads();
     if (tid == 0) {
@@ -303,28 +324,58 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
             raise_flag(s.flags, FLAG_OVERFLOW);
             Dy = 0;
         }
-        const long long cT = H.cT + Dy;
+        const long long cT = cT0 + Dy;
         H.cT = cT;
-        for (int i = 0; i < kProjDim; ++i) H.z_last[i] = zy[i];
-        const long long Vo = sh_Vopen;
-        sh_split = prod_ge(static_cast<unsigned long long>(N), static_cast<unsigned long long>(Vo + Dy), 1ull,
-                           static_cast<unsigned long long>(cT))
-                       ? 1
-                       : 0;
-        if (sh_split && n_ent >= s.Ecap) {   // no free slot: host-checked capacity, never true
+        int split = prod_ge(static_cast<unsigned long long>(N), static_cast<unsigned long long>(sh_Vo + Dy), 1ull,
+                            static_cast<unsigned long long>(cT))
+                        ? 1
+                        : 0;
+        if (split && n_ent0 >= s.Ecap) {   // no free slot: host-checked capacity, never true
             raise_flag(s.flags, FLAG_BAD_LENS);
-            sh_split = 0;
+            split = 0;
         }
+        sh_split = split;
         sh_D = Dy;
     }
+    if (tid < kProjDim) H.z_last[tid] = zy[tid];
     __syncthreads();
     const long long Dy = sh_D;
-    const int ypos = H.T - W;   // token index of y
-    if (sh_split) {
-        const int e = n_ent;
-        for (int dim = tid; dim < D; dim += kStreamThreads) {
-            st.mk[static_cast<int64_t>(e) * D + dim] = ky[dim];
-            st.mv[static_cast<int64_t>(e) * D + dim] = vy[dim];
+    const bool split = sh_split != 0;
+    const int ypos = Tcur - W;   // token index of y
+    int n_nodes = n_nodes0, n_ent = n_ent0;
+    int new_open = open, new_open_page = open_page;
+    // the node whose pool entry is rewritten at the end, with its statistics (dimension tid)
+    int wr_node = -1, wr_page = -1, wr_m = 0;
+    double wr_M2 = 0.0, wr_k = 0.0, wr_v = 0.0;
+
+    if (!split) {   // y joins the open node (pairwise update with a one-member node)
+        const double inv = 1.0 / (m_open + 1);
+        double q = 0.0;
+        if (tid < D) {
+            const double dk = static_cast<double>(ky[tid]) - mk_o;
+            q = dk * dk;
+            wr_k = mk_o + dk * inv;
+            wr_v = mv_o + (static_cast<double>(vy[tid]) - mv_o) * inv;
+            st.mk[static_cast<int64_t>(open) * D + tid] = wr_k;
+            st.mv[static_cast<int64_t>(open) * D + tid] = wr_v;
+        }
+        const double dd = block_sum(q, red_d);
+        wr_M2 = sh_M2open + dd * m_open * inv;
+        wr_m = m_open + 1;
+        if (tid == 0) {
+            st.M2[open] = wr_M2;
+            st.m[open] = wr_m;
+            st.V[open] = sh_Vo + Dy;
+            st.vord[n_nodes0 - 1] = sh_Vo + Dy;
+        }
+        wr_node = open;
+        wr_page = open_page;
+    } else {
+        // y starts a new node in the next free entry
+        const int e = n_ent0;
+        if (tid < D) {
+            st.mk[static_cast<int64_t>(e) * D + tid] = ky[tid];
+            st.mv[static_cast<int64_t>(e) * D + tid] = vy[tid];
         }
         if (tid == 0) {
             st.m[e] = 1;
@@ -332,182 +383,174 @@ __global__ void __launch_bounds__(kStreamThreads) k_stream_append(const StreamAr
             st.start[e] = ypos;
             st.M2[e] = 0.0;
             st.owner[e] = 0;
-            st.order[n_nodes] = e;
+            st.order[n_nodes0] = e;
+            st.vord[n_nodes0] = Dy;
+            if (may_merge) {
+                sOrder[n_nodes0] = e;
+                sV[n_nodes0] = Dy;
+            }
         }
-        ++n_nodes;
-        ++n_ent;
-    } else {   // y joins the open node (pairwise update with a one-member node)
-        const int e = open;
-        const int m = sh_mopen;
-        const double inv = 1.0 / (m + 1);
-        double q = 0.0;
+        n_nodes = n_nodes0 + 1;
+        n_ent = n_ent0 + 1;
+        new_open = e;
+        new_open_page = sh_newpage;
+        wr_node = e;
+        wr_page = sh_newpage;
+        wr_m = 1;
         if (tid < D) {
-            const double dk = static_cast<double>(ky[tid]) - mk_o;
-            q = dk * dk;
-            st.mk[static_cast<int64_t>(e) * D + tid] = mk_o + dk * inv;
-            st.mv[static_cast<int64_t>(e) * D + tid] = mv_o + (static_cast<double>(vy[tid]) - mv_o) * inv;
+            wr_k = ky[tid];
+            wr_v = vy[tid];
         }
-        const double dd = block_sum(q, red_d);
-        if (tid == 0) {
-            st.M2[e] += dd * m * inv;
-            st.m[e] = m + 1;
-            st.V[e] = sh_Vopen + Dy;
-        }
-    }
-    __syncthreads();
+        __syncthreads();
 
-    // 3. above N nodes: merge the adjacent pair with the smallest combined variation
-    int merged = -1, moved = -1;
-    if (n_nodes > N) {
-        // the node order, then the nodes' variations, to shared memory (batches of loads in flight)
-        for (int j0 = 0; j0 < n_nodes; j0 += 4 * kStreamThreads) {
-            int o[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int j = j0 + r * kStreamThreads + tid;
-                o[r] = j < n_nodes ? st.order[j] : 0;
+        // above N nodes: merge the adjacent pair with the smallest combined variation. The new
+        // node is the last entry and the last in node order, so it is never the left node of the
+        // pair; the slot a merge frees is refilled by the new node (unless the new node is the one
+        // merged away, which frees its own slot).
+        if (n_nodes > N) {
+            long long best = LLONG_MAX;
+            int bj = INT_MAX;
+            for (int j = tid; j < n_nodes - 1; j += kStreamThreads) {
+                const long long v2 = sV[j] + sV[j + 1];
+                if (v2 < best) {   // j ascending per thread: keeps the leftmost of equal sums
+                    best = v2;
+                    bj = j;
+                }
             }
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int j = j0 + r * kStreamThreads + tid;
-                if (j < n_nodes) sOrder[j] = o[r];
+            if (tid == 0) {
+                sh_bmin = static_cast<unsigned long long>(LLONG_MAX);
+                sh_merge_j = INT_MAX;
             }
-        }
-        __syncthreads();
-        for (int j0 = 0; j0 < n_nodes; j0 += 4 * kStreamThreads) {
-            long long vv[4];
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int j = j0 + r * kStreamThreads + tid;
-                vv[r] = j < n_nodes ? st.V[sOrder[j]] : 0;
+            __syncthreads();
+            atomicMin(&sh_bmin, static_cast<unsigned long long>(best));
+            __syncthreads();
+            if (static_cast<unsigned long long>(best) == sh_bmin) atomicMin(&sh_merge_j, bj);
+            __syncthreads();
+            const int j = sh_merge_j;
+            const int ea = sOrder[j], eb = sOrder[j + 1];
+            const bool b_new = eb == e;
+            // round trip 2: the pair's statistics and the page ids of their slots
+            double ak = 0.0, av = 0.0, bk = 0.0, bv = 0.0;
+            if (tid < D) {
+                ak = st.mk[static_cast<int64_t>(ea) * D + tid];
+                av = st.mv[static_cast<int64_t>(ea) * D + tid];
+                bk = b_new ? static_cast<double>(ky[tid]) : st.mk[static_cast<int64_t>(eb) * D + tid];
+                bv = b_new ? static_cast<double>(vy[tid]) : st.mv[static_cast<int64_t>(eb) * D + tid];
             }
-#pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                const int j = j0 + r * kStreamThreads + tid;
-                if (j < n_nodes) sV[j] = vv[r];
+            if (tid == 0) {
+                sh_ma = st.m[ea];
+                sh_mb = b_new ? 1 : st.m[eb];
+                sh_M2a = st.M2[ea];
+                sh_M2b = b_new ? 0.0 : st.M2[eb];
+                sh_pa = s.page_table[static_cast<int64_t>(u) * s.max_pages + ea / kPageNodes];
+                sh_pb = s.page_table[static_cast<int64_t>(u) * s.max_pages + eb / kPageNodes];
             }
-        }
-        __syncthreads();
-        // the smallest V_j + V_{j+1} (all >= 0), then the smallest j attaining it
-        long long best = LLONG_MAX;
-        int bj = INT_MAX;
-        for (int j = tid; j < n_nodes - 1; j += kStreamThreads) {
-            const long long v2 = sV[j] + sV[j + 1];
-            if (v2 < best) {   // j ascending per thread: keeps the leftmost of equal sums
-                best = v2;
-                bj = j;
+            __syncthreads();
+            const int ma = sh_ma, mb = sh_mb;
+            // pairwise update: a <- a + b (means and summed squared deviations)
+            const double wb = static_cast<double>(mb) / (ma + mb);
+            double q = 0.0, nk = 0.0, nv = 0.0;
+            if (tid < D) {
+                const double dk = bk - ak;
+                q = dk * dk;
+                nk = ak + dk * wb;
+                nv = av + (bv - av) * wb;
+                st.mk[static_cast<int64_t>(ea) * D + tid] = nk;
+                st.mv[static_cast<int64_t>(ea) * D + tid] = nv;
             }
-        }
-        if (tid == 0) {
-            sh_bmin = static_cast<unsigned long long>(LLONG_MAX);
-            sh_merge_j = INT_MAX;
-        }
-        __syncthreads();
-        atomicMin(&sh_bmin, static_cast<unsigned long long>(best));
-        __syncthreads();
-        if (static_cast<unsigned long long>(best) == sh_bmin) atomicMin(&sh_merge_j, bj);
-        __syncthreads();
-        const int j = sh_merge_j;
-        const int ea = sOrder[j], eb = sOrder[j + 1];
-        // pairwise update: a <- a + b
-        const int ma = st.m[ea], mb = st.m[eb];
-        const double wb = static_cast<double>(mb) / (ma + mb);
-        double q = 0.0;
-        for (int dim = tid; dim < D; dim += kStreamThreads) {
-            double &ak = st.mk[static_cast<int64_t>(ea) * D + dim];
-            double &av = st.mv[static_cast<int64_t>(ea) * D + dim];
-            const double dk = st.mk[static_cast<int64_t>(eb) * D + dim] - ak;
-            q += dk * dk;
-            ak += dk * wb;
-            av += (st.mv[static_cast<int64_t>(eb) * D + dim] - av) * wb;
-        }
-        const double dd = block_sum(q, red_d);
-        if (tid == 0) {
-            st.M2[ea] += st.M2[eb] + dd * static_cast<double>(ma) * mb / (ma + mb);
-            st.m[ea] = ma + mb;
-            st.V[ea] += st.V[eb];
-        }
-        // drop position j + 1 from the node order (from the shared copy)
-        for (int t = j + 1 + tid; t < n_nodes - 1; t += kStreamThreads) st.order[t] = sOrder[t + 1];
-        __syncthreads();
-        --n_nodes;
-        merged = ea;
-        // the freed slot eb takes the unit's last entry
-        const int last = n_ent - 1;
-        if (eb != last) {
-            const int kind = st.owner[last];
-            if (kind <= -2) {   // a recent token: copy its pool entry
-                const uint8_t *src = entry_page<D, T>(s, u, last);
-                uint8_t *dst = entry_page<D, T>(s, u, eb);
-                if (src && dst) {
-                    for (int dim = tid; dim < D; dim += kStreamThreads) {
-                        Elem<T>::put(dst + vec_off<D, T>(eb % kPageNodes, dim),
-                                     Elem<T>::get(src + vec_off<D, T>(last % kPageNodes, dim)));
-                        Elem<T>::put(dst + VEC + vec_off<D, T>(eb % kPageNodes, dim),
-                                     Elem<T>::get(src + VEC + vec_off<D, T>(last % kPageNodes, dim)));
-                    }
-                    if (tid == 0)
-                        reinterpret_cast<float2 *>(dst + 2 * VEC)[eb % kPageNodes] =
-                            reinterpret_cast<const float2 *>(src + 2 * VEC)[last % kPageNodes];
+            const double dd = block_sum(q, red_d);
+            const double M2ab = sh_M2a + sh_M2b + dd * static_cast<double>(ma) * mb / (ma + mb);
+            const long long Vab = sV[j] + sV[j + 1];
+            if (tid == 0) {
+                st.M2[ea] = M2ab;
+                st.m[ea] = ma + mb;
+                st.V[ea] = Vab;
+                st.vord[j] = Vab;
+            }
+            // drop position j + 1 from the node order (and its variation)
+            for (int t = j + 1 + tid; t < n_nodes - 1; t += kStreamThreads) {
+                st.order[t] = sOrder[t + 1];
+                st.vord[t] = sV[t + 1];
+            }
+            __syncthreads();
+            n_nodes -= 1;
+            n_ent -= 1;
+            if (b_new) {
+                // the new node merged into its left neighbour, which becomes the open node; the
+                // new node's slot (the last entry) is released
+                new_open = ea;
+                new_open_page = sh_pa;
+                wr_node = -1;
+            } else {
+                // the new node moves into the freed slot eb, at order position n_nodes - 1
+                if (tid < D) {
+                    st.mk[static_cast<int64_t>(eb) * D + tid] = ky[tid];
+                    st.mv[static_cast<int64_t>(eb) * D + tid] = vy[tid];
                 }
                 if (tid == 0) {
-                    st.recent[-2 - kind] = eb;
-                    st.owner[eb] = kind;
-                }
-            } else {   // a middle node: move its state; its pool slot is rewritten below
-                for (int dim = tid; dim < D; dim += kStreamThreads) {
-                    st.mk[static_cast<int64_t>(eb) * D + dim] = st.mk[static_cast<int64_t>(last) * D + dim];
-                    st.mv[static_cast<int64_t>(eb) * D + dim] = st.mv[static_cast<int64_t>(last) * D + dim];
-                }
-                if (tid == 0) {
-                    st.m[eb] = st.m[last];
-                    st.start[eb] = st.start[last];
-                    st.V[eb] = st.V[last];
-                    st.M2[eb] = st.M2[last];
+                    st.m[eb] = 1;
+                    st.start[eb] = ypos;
+                    st.V[eb] = Dy;
+                    st.M2[eb] = 0.0;
                     st.owner[eb] = 0;
-                    sh_pos = -1;
+                    st.order[n_nodes - 1] = eb;
                 }
-                __syncthreads();
-                // its position in the order before the shift (sOrder), then after it
-                for (int p = tid; p < n_nodes + 1; p += kStreamThreads)
-                    if (sOrder[p] == last) sh_pos = p > j + 1 ? p - 1 : p;
-                __syncthreads();
-                if (tid == 0 && sh_pos >= 0) st.order[sh_pos] = eb;
-                if (merged == last) merged = eb;
-                moved = eb;
+                new_open = eb;
+                new_open_page = sh_pb;
+                wr_node = eb;
+                wr_page = sh_pb;
+            }
+            // the merged node's pool entry
+            if (sh_pa >= 0 && sh_pa < s.num_pages) {
+                uint8_t *pg = s.pages + static_cast<int64_t>(sh_pa) * PAGE;
+                const int slot = ea % kPageNodes;
+                if (tid < D) {
+                    Elem<T>::put(pg + vec_off<D, T>(slot, tid), static_cast<float>(nk));
+                    Elem<T>::put(pg + VEC + vec_off<D, T>(slot, tid), static_cast<float>(nv));
+                }
+                if (tid == 0) {
+                    const int m = ma + mb;
+                    reinterpret_cast<float2 *>(pg + 2 * VEC)[slot] = make_float2(
+                        logf(static_cast<float>(m)), static_cast<float>(M2ab / (static_cast<double>(m) * D) / (2.0 * D)));
+                }
+            } else if (tid == 0) {
+                raise_flag(s.flags, FLAG_BAD_PAGE);
             }
         }
-        --n_ent;
-        __syncthreads();
     }
 
-    // 4. the new token takes y's (possibly moved) slot as an exact recent entry
-    {
-        const int ns = merged >= 0 ? st.recent[ring] : yslot;   // entries move only in a merge
-        uint8_t *pg = ns == yslot ? const_cast<uint8_t *>(ypg) : entry_page<D, T>(s, u, ns);
-        if (pg) {
-            const T *kn = static_cast<const T *>(s.k_new) + static_cast<int64_t>(u) * D;
-            const T *vn = static_cast<const T *>(s.v_new) + static_cast<int64_t>(u) * D;
-            for (int dim = tid; dim < D; dim += kStreamThreads) {
-                Elem<T>::put(pg + vec_off<D, T>(ns % kPageNodes, dim), static_cast<float>(kn[dim]));
-                Elem<T>::put(pg + VEC + vec_off<D, T>(ns % kPageNodes, dim), static_cast<float>(vn[dim]));
+    // the new token takes y's slot as an exact recent entry, and y's place in the ring
+    if (tid < D) {
+        Elem<T>::put(ypg + vec_off<D, T>(yslot % kPageNodes, tid), kn);
+        Elem<T>::put(ypg + VEC + vec_off<D, T>(yslot % kPageNodes, tid), vn);
+        st.ring[(static_cast<int64_t>(ring) * 2) * D + tid] = kn;
+        st.ring[(static_cast<int64_t>(ring) * 2 + 1) * D + tid] = vn;
+    }
+    if (tid == 0) reinterpret_cast<float2 *>(ypg + 2 * VEC)[yslot % kPageNodes] = make_float2(0.0f, 0.0f);
+    // the open node's (or the moved new node's) pool entry, from the statistics held here
+    if (wr_node >= 0) {
+        if (wr_page >= 0 && wr_page < s.num_pages) {
+            uint8_t *pg = s.pages + static_cast<int64_t>(wr_page) * PAGE;
+            const int slot = wr_node % kPageNodes;
+            if (tid < D) {
+                Elem<T>::put(pg + vec_off<D, T>(slot, tid), static_cast<float>(wr_k));
+                Elem<T>::put(pg + VEC + vec_off<D, T>(slot, tid), static_cast<float>(wr_v));
             }
-            if (tid == 0) reinterpret_cast<float2 *>(pg + 2 * VEC)[ns % kPageNodes] = make_float2(0.0f, 0.0f);
+            if (tid == 0)
+                reinterpret_cast<float2 *>(pg + 2 * VEC)[slot] = make_float2(
+                    wr_m == 1 ? 0.0f : logf(static_cast<float>(wr_m)),
+                    static_cast<float>(wr_M2 / (static_cast<double>(wr_m) * D) / (2.0 * D)));
+        } else if (tid == 0) {
+            raise_flag(s.flags, FLAG_BAD_PAGE);
         }
     }
-    // 5. changed middle nodes to the pool
-    {
-        const int last_node = merged >= 0 || sh_split ? st.order[n_nodes - 1] : open;
-        write_node<D, T>(s, st, u, last_node, last_node == open ? sh_opage : nullptr);
-    }
-    if (merged >= 0) write_node<D, T>(s, st, u, merged);
-    if (moved >= 0) write_node<D, T>(s, st, u, moved);
-    __syncthreads();
     if (tid == 0) {
         H.n_nodes = n_nodes;
         H.n_ent = n_ent;
+        H.open = new_open;
+        H.open_page = new_open_page;
         H.ring = (ring + 1) % W;
-        H.T = H.T + 1;
+        H.T = Tcur + 1;
         s.lens[u] = n_ent;
     }
 }
@@ -539,6 +582,12 @@ void stream_layout(int d, int Ecap, int W, StreamArgs *s) {
     off = up256(off + 8ll * Ecap * d);
     s->off_mv = off;
     off = up256(off + 8ll * Ecap * d);
+    s->off_vord = off;
+    off = up256(off + 8ll * Ecap);
+    s->off_rpage = off;
+    off = up256(off + 4ll * (W > 0 ? W : 1));
+    s->off_ring = off;
+    off = up256(off + 4ll * 2 * (W > 0 ? W : 1) * d);
     s->unit_bytes = off;
 }
 

@@ -26,7 +26,8 @@ def _layout(d, Ecap, W_):
     o, off = {}, up(128)
     for name, size in (("order", 4 * Ecap), ("recent", 4 * max(W_, 1)), ("owner", 4 * Ecap), ("m", 4 * Ecap),
                        ("start", 4 * Ecap), ("V", 8 * Ecap), ("M2", 8 * Ecap), ("mk", 8 * Ecap * d),
-                       ("mv", 8 * Ecap * d)):
+                       ("mv", 8 * Ecap * d), ("vord", 8 * Ecap), ("rpage", 4 * max(W_, 1)),
+                       ("ring", 4 * 2 * max(W_, 1) * d)):
         o[name] = off
         off = up(off + size)
     o["unit"] = off

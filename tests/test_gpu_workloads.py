@@ -119,3 +119,77 @@ def test_gqa7_32k_3p5pct_variation_weighted_full():
     r = _coarsen_full(w, representative="variation")
     _check_units(w, r, [(3, 1), (30, 2)], representative="variation")
     _check_decode(w, r, [3, 30])
+
+
+def test_coarsen_131k_tensor_projection_full():
+    """The coarsening workload with the tensor-core projection option, stage by stage on sampled
+    units: every step within the bound of the exact bf16 projection's step; boundaries, c_t and
+    statistics as the oracle computes them from those steps."""
+    w = workloads.WORKLOADS["coarsen_131k"]
+    T_list = workloads.seq_lengths(w)
+    N_list = workloads.segment_counts(w, T_list)
+    k, v, _ = workloads.make_kv(w, "cuda", T_list=T_list)
+    pages = [skv.pages_for(T, N, S, W) for T, N in zip(T_list, N_list)]
+    table, num_pages = workloads.page_assignment(w.B, w.Hkv, pages, False, w.seed)
+    table = table.cuda()
+    pool = skv.NodePool(num_pages, w.d, w.torch_dtype)
+    bnd = torch.full((w.B, w.Hkv, max(N_list) + 1), -7, dtype=torch.int32, device="cuda")
+    cum = torch.full((k.shape[0],), -7, dtype=torch.int64, device="cuda")
+    ws = torch.zeros(skv.coarsen_workspace_bytes(w.Hkv, w.d, T_list, N_list, S, W), dtype=torch.uint8, device="cuda")
+    lens = skv.coarsen(k, v, w.Hkv, T_list, N_list, S, W, w.seed, pool, table, boundaries=bnd, cumvar=cum,
+                       workspace=ws, projection="tensor")
+    st, flags = skv.workspace_error(ws)
+    assert st == 0, flags
+    P16 = oracle.projection_bf16(w.seed, w.d)
+    for (b, h) in [(0, 0), (3, 2), (7, 3)]:
+        kk = to_np32(workloads.unit_rows(k, T_list, w.Hkv, b, h))
+        vv = to_np32(workloads.unit_rows(v, T_list, w.Hkv, b, h))
+        M = T_list[b] - S - W
+        off = sum(T_list[:b]) * w.Hkv + h * T_list[b]
+        C = cum[off:off + M].cpu().numpy()
+        D = np.diff(C, prepend=0)
+        dref, bound = oracle.tensor_steps_reference(kk, vv, S, W, P16)
+        assert np.all(np.abs(D - dref) <= bound), f"unit ({b},{h}) steps"
+        u = oracle.coarsen_unit_from_steps(kk, vv, S, W, N_list[b], D)
+        assert np.array_equal(bnd[b, h, :N_list[b] + 1].cpu().numpy(), u.bounds)
+        assert int(lens[b, h]) == u.kt.shape[0]
+        kt, vt, al, be = skv.read_entries(pool, table, lens, b, h)
+
+        class G:
+            pass
+
+        g = G()
+        g.kt, g.vt = kt.double().cpu().numpy(), vt.double().cpu().numpy()
+        g.alpha, g.beta = al.double().cpu().numpy(), be.double().cpu().numpy()
+        check_nodes(g, u, w.torch_dtype, w.d, f"tensor projection unit ({b},{h})")
+
+
+def test_coarsen_131k_wave_pipeline_captured_equals_direct():
+    """The 131k workload's coarsening runs in waves of units (projection on the caller's stream,
+    later stages on the library's side stream). Captured into a CUDA graph and replayed, it gives
+    the direct call's boundaries, lens and stored nodes bit for bit (half the batch, 16 units)."""
+    import dataclasses
+    w = dataclasses.replace(workloads.WORKLOADS["coarsen_131k"], B=4)
+    r = _coarsen_full(w)
+    T_list, N_list = r["T"], r["N"]
+    pool2 = skv.NodePool(r["pool"].num_pages, w.d, w.torch_dtype)
+    lens2 = torch.full_like(r["lens"], -7)
+    bnd2 = torch.full_like(r["bnd"], -7)
+    ws2 = torch.zeros(skv.coarsen_workspace_bytes(w.Hkv, w.d, T_list, N_list, S, W), dtype=torch.uint8,
+                      device="cuda")
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        skv.coarsen(r["k"], r["v"], w.Hkv, T_list, N_list, S, W, w.seed, pool2, r["table"], lens=lens2,
+                    boundaries=bnd2, workspace=ws2)
+    g.replay()
+    torch.cuda.synchronize()
+    assert skv.workspace_error(ws2)[0] == 0
+    assert torch.equal(lens2, r["lens"]) and torch.equal(bnd2, r["bnd"])
+    for b in range(w.B):
+        for h in range(w.Hkv):
+            one = skv.read_entries(r["pool"], r["table"], r["lens"], b, h)
+            two = skv.read_entries(pool2, r["table"], lens2, b, h)
+            for x, y in zip(one, two):
+                assert torch.equal(x, y), f"unit ({b},{h}) differs"
+    del g

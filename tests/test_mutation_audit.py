@@ -1,16 +1,18 @@
-"""Mutation audit of the oracle's pins (test infrastructure; run by hand, not collected by pytest).
+"""Mutation audit of the oracle's pins (test infrastructure; collected, and skipped unless
+SKV_MUTATION_AUDIT=1 is set, because it rebuilds and re-tests the oracle once per mutation, which
+takes a few minutes).
 
 Each entry plants one plausible mistake -- a dropped term, a wrong index, order or operand, a wrong
 rounding, normaliser or comparison -- in a temporary copy of the oracle, rebuilds that copy and runs
-the oracle's CPU pins (tests/test_oracle_*.py) against it. A mistake that no pin catches is
-reported as SURVIVED. The repository's own files are never modified.
+the oracle's CPU pins (tests/test_oracle_*.py) against it. A mistake that no pin catches fails its
+test case. The repository's own files are never modified.
 
-    python tests/mutation_audit.py            # all mutations (a few minutes)
-    python tests/mutation_audit.py seg_gt     # selected ones
+    SKV_MUTATION_AUDIT=1 python -m pytest tests/test_mutation_audit.py -q       # every mutation
+    SKV_MUTATION_AUDIT=1 python -m pytest tests/test_mutation_audit.py -k seg_gt
 
 Conventions of the oracle's own readings that the pages do not fix are listed in CONVENTIONS:
 there a planted change alters only which (equally valid) convention is followed, so surviving it
-is expected.
+is expected (and asserted).
 """
 from __future__ import annotations
 
@@ -19,6 +21,8 @@ import shutil
 import subprocess
 import sys
 import tempfile
+
+import pytest
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 
@@ -85,6 +89,21 @@ MUTATIONS = [
      "sums = [self.nodes[j].V for j in range(len(self.nodes) - 1)]"),
     ("stream_merge_M2", STREAM, "M2 = a.M2 + b.M2 + float(dk @ dk) * a.m * b.m / m",
      "M2 = a.M2 + b.M2"),
+    # the centring option's fixed-order mean (reading R8)
+    ("mean_one_block", C, "const int b1 = b0 + ORC_MEAN_BLOCK < T ? b0 + ORC_MEAN_BLOCK : T;",
+     "const int b1 = T;"),
+    ("mean_div_tminus1", C, "mu[i] = T > 0 ? total / (float)T : 0.0f;",
+     "mu[i] = T > 1 ? total / (float)(T - 1) : 0.0f;"),
+    ("center_keys_noop", INIT, "    return (k - key_mean_f32(k)[None, :]).astype(np.float32)",
+     "    return k.astype(np.float32)"),
+    # the given-steps path and the tensor projection's checks
+    ("steps_prefix_exclusive", C, "            if (C) C[t] = run;\n            if (d64) d64[t] = 0.0;",
+     "            if (C) C[t] = run - D_in[t];\n            if (d64) d64[t] = 0.0;"),
+    ("steps_ignored", C, "            run += D_in[t];", "            run += 100;"),
+    ("bf16_truncate", INIT, "    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16", "    r = (u >> 16) << 16"),
+    ("tensor_ref_no_v", INIT, "    x = np.concatenate([k, v], axis=1)[s_eff:s_eff + M]",
+     "    x = np.concatenate([k, 0 * v], axis=1)[s_eff:s_eff + M]"),
+
 ]
 
 # the Box-Muller branch is part of reading R2's generator definition, which the pages leave open
@@ -112,38 +131,44 @@ def _copy_tree(dst):
             shutil.copy(os.path.join(ROOT, "tests", f), os.path.join(dst, "tests", f))
 
 
-def main(selected):
-    survivors = []
-    for name, rel, old, new in MUTATIONS:
-        if selected and name not in selected:
-            continue
-        with tempfile.TemporaryDirectory(prefix="oracle_mut_") as tmp:
-            _copy_tree(tmp)
-            path = os.path.join(tmp, rel)
-            src = open(path).read()
-            if src.count(old) != 1:
-                raise SystemExit(f"{name}: anchor found {src.count(old)} times")
-            src = src.replace(old, new)
-            if name in EXTRA:
-                a, b = EXTRA[name]
-                src = src.replace(a, b, 1)
-            open(path, "w").write(src)
-            env = dict(os.environ, PYTHONDONTWRITEBYTECODE="1")
-            subprocess.run([sys.executable, "-c", "import oracle; oracle.build(force=True)"], cwd=tmp, env=env,
-                           check=True, capture_output=True)
-            tests = sorted(os.path.join("tests", f) for f in os.listdir(os.path.join(tmp, "tests"))
-                           if f.startswith("test_oracle_"))
-            r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "not gpu", "-p", "no:cacheprovider",
-                                *tests], cwd=tmp, env=env, capture_output=True, text=True)
-            caught = r.returncode != 0
-            tail = (r.stdout.strip().splitlines() or [""])[-1]
-            note = " (convention of the oracle's reading)" if name in CONVENTIONS else ""
-            print(f"{name:26s} {'CAUGHT' if caught else 'SURVIVED'}{note}  {tail}", flush=True)
-            if not caught and name not in CONVENTIONS:
-                survivors.append(name)
-    if survivors:
-        raise SystemExit(f"mutations no pin catches: {survivors}")
 
 
-if __name__ == "__main__":
-    main(set(sys.argv[1:]))
+def _run_mutation(name, rel, old, new):
+    """True if the pins catch the planted mistake (the pin suite fails on the mutated copy)."""
+    with tempfile.TemporaryDirectory(prefix="oracle_mut_") as tmp:
+        _copy_tree(tmp)
+        path = os.path.join(tmp, rel)
+        src = open(path).read()
+        assert src.count(old) == 1, f"{name}: anchor found {src.count(old)} times"
+        src = src.replace(old, new)
+        if name in EXTRA:
+            a, b = EXTRA[name]
+            src = src.replace(a, b, 1)
+        open(path, "w").write(src)
+        env = dict(os.environ, PYTHONDONTWRITEBYTECODE="1")
+        env.pop("SKV_MUTATION_AUDIT", None)
+        subprocess.run([sys.executable, "-c", "import oracle; oracle.build(force=True)"], cwd=tmp, env=env,
+                       check=True, capture_output=True)
+        tests = sorted(os.path.join("tests", f) for f in os.listdir(os.path.join(tmp, "tests"))
+                       if f.startswith("test_oracle_"))
+        r = subprocess.run([sys.executable, "-m", "pytest", "-q", "-x", "-m", "not gpu", "-p", "no:cacheprovider",
+                            *tests], cwd=tmp, env=env, capture_output=True, text=True)
+        return r.returncode != 0
+
+
+@pytest.mark.skipif(not os.environ.get("SKV_MUTATION_AUDIT"),
+                    reason="rebuilds and re-tests the oracle per mutation (minutes): set SKV_MUTATION_AUDIT=1")
+@pytest.mark.parametrize("name,rel,old,new", MUTATIONS, ids=[m[0] for m in MUTATIONS])
+def test_planted_mistake_is_caught_by_a_pin(name, rel, old, new):
+    caught = _run_mutation(name, rel, old, new)
+    if name in CONVENTIONS:
+        assert not caught, f"{name}: a convention change should leave every pin green"
+    else:
+        assert caught, f"{name}: no oracle pin catches this planted mistake"
+
+
+def test_every_anchor_is_present_once():
+    """Each mutation's anchor text occurs exactly once in the current oracle sources (so the audit
+    keeps testing what it claims when the oracle is edited)."""
+    for name, rel, old, _ in MUTATIONS:
+        assert open(os.path.join(ROOT, rel)).read().count(old) == 1, name
