@@ -294,12 +294,15 @@ def l2_flush_buffer(device):
     return torch.zeros(64 << 20, dtype=torch.float32, device=device)   # 256 MB, twice the 126 MB L2
 
 
-def coarsen_stage(device, reps: int = 5):
-    """Coarsener throughput on the 8 x 4 x 131,072-token workload (tokens/s, GB/s of raw KV)."""
+def coarsen_stage(device, reps: int = 5, batch: int | None = None):
+    """Coarsener throughput on the 8 x 4 x 131,072-token workload (tokens/s, GB/s of raw KV);
+    `batch` < 8 takes the first sequences only (a profiling case)."""
     import torch
     import compressed_decode_attention_equal_b200 as skv
     import workloads
     w = workloads.WORKLOADS[COARSEN_WORKLOAD]
+    if batch is not None:
+        w = dataclasses.replace(w, B=batch)
     T_list = workloads.seq_lengths(w)
     N_list = workloads.segment_counts(w, T_list)
     k, v, _ = workloads.make_kv(w, device, T_list=T_list)
@@ -413,7 +416,7 @@ def cpu_baseline(w, caches, table, budget_s: float = 12.0):
                       f"{int(c['lens'].sum())} entries), fp64, nodes read back from the GPU"}
 
 
-def diagonal_closure_stage(w, device, layers: int, steps: int = 2000, regions: int = 5):
+def diagonal_closure_stage(w, device, layers: int, steps: int = 1000, regions: int = 3):
     """Decode with the diagonal closure (per-dimension variances in every node) on the same workload:
     layer caches coarsened into diagonal pools, graph replays, CUDA events (rank 0 only)."""
     import torch
@@ -447,7 +450,7 @@ def diagonal_closure_stage(w, device, layers: int, steps: int = 2000, regions: i
             "note": "same workload and call with diagonal-closure pools (per-dimension key variances)"}
 
 
-def other_decode_stage(device, steps: int = 2000, regions: int = 5):
+def other_decode_stage(device, steps: int = 1000, regions: int = 3):
     """Decode on the two other decode workloads, each cache built by the coarsener and replayed from
     CUDA graphs (rank 0 only):
     - gqa6_10k5_prefill_decode: 1 sequence, 2 KV heads, 421 entries each, a 0.45 MB cache, so the
@@ -502,7 +505,7 @@ def other_decode_stage(device, steps: int = 2000, regions: int = 5):
     return res
 
 
-def stream_stage(w, device, steps: int = 3000, distinct: int = 60, regions: int = 5):
+def stream_stage(w, device, steps: int = 1000, distinct: int = 60, regions: int = 3):
     """Streaming coarsening on the decode workload: skv_stream_init on the prompts, then appends of
     one token per unit replayed from CUDA graphs (rank 0 only). The append is latency-bound (one CTA
     per unit, a 4,096-FMA projection chain and O(N) merge search per call)."""
@@ -870,6 +873,10 @@ def main():
     ap.add_argument("--no-diagonal", action="store_true", help="skip the diagonal-closure decode timing")
     ap.add_argument("--no-stream", action="store_true", help="skip the streaming-append timing")
     ap.add_argument("--no-other", action="store_true", help="skip the decode timing on the other two workloads")
+    ap.add_argument("--only", choices=["coarsen", "diagonal", "stream", "other"],
+                    help="run this single-GPU stage alone (no headline line; a profiling aid)")
+    ap.add_argument("--coarsen-batch", type=int, default=None,
+                    help="sequences of the coarsening workload (default all 8; fewer for a profiling case)")
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
@@ -903,12 +910,21 @@ def main():
     init_ranks("nccl", device, world)
     from compressed_decode_attention_equal_b200 import build
     build.build()
+    if args.only:
+        import workloads
+        w = workloads.WORKLOADS[WORKLOAD]
+        stage = {"coarsen": lambda: coarsen_stage(device, batch=args.coarsen_batch),
+                 "diagonal": lambda: diagonal_closure_stage(w, device, args.layers, steps=args.steps),
+                 "stream": lambda: stream_stage(w, device, steps=args.steps),
+                 "other": lambda: other_decode_stage(device, steps=args.steps)}[args.only]
+        print(json.dumps({"stage": args.only, "result": stage()}), flush=True)
+        return
     res, caches, table, w = run_ours(args, rank, world, device)
     # the single-GPU characterisations and the CPU baseline run at N = 1 only: under torchrun the
     # other ranks would hold their GPUs idle at the closing barrier meanwhile
     if rank == 0 and world == 1:
         if not args.no_coarsen:
-            res["coarsen"] = coarsen_stage(device)
+            res["coarsen"] = coarsen_stage(device, batch=args.coarsen_batch)
         if not args.no_diagonal:
             res["diagonal_closure"] = diagonal_closure_stage(w, device, args.layers)
         if not args.no_stream:

@@ -19,8 +19,6 @@
 //                    recents) and write lens
 //   k_segment_reduce one warp per entry: two-pass mean / variance, node write
 //                    into the paged pool (swizzled 16-byte chunks)
-#include <vector>
-
 #include "skv_common.cuh"
 #include "skv_internal.h"
 
@@ -50,7 +48,7 @@ __device__ __forceinline__ float to_f32<float>(float x) { return x; }
 // one thread per key dimension, one CTA per (block of kMeanBlock tokens, unit)
 template <int D, typename T>
 __global__ void __launch_bounds__(D) k_key_block_sums(const CoarsenArgs a) {
-    const int u = a.unit0 + blockIdx.y, blk = blockIdx.x;
+    const int u = blockIdx.y, blk = blockIdx.x;
     const int b = u / a.Hkv, h = u % a.Hkv;
     const SeqRow sr = a.seq[b];
     const int t0 = blk * kMeanBlock;
@@ -65,7 +63,7 @@ __global__ void __launch_bounds__(D) k_key_block_sums(const CoarsenArgs a) {
 
 template <int D>
 __global__ void __launch_bounds__(D) k_key_mean(const CoarsenArgs a) {
-    const int u = a.unit0 + blockIdx.x;
+    const int u = blockIdx.x;
     const SeqRow sr = a.seq[u / a.Hkv];
     const int nblk = (sr.T + kMeanBlock - 1) / kMeanBlock;
     const float *bs = a.key_blk + static_cast<int64_t>(u) * a.max_blk * D + threadIdx.x;
@@ -192,7 +190,7 @@ __global__ void __launch_bounds__(kK1Threads, 2)
     long long *warp_sum = reinterpret_cast<long long *>(bar + 8);
     float *mus = reinterpret_cast<float *>(warp_sum + 8);   // the unit's mean key (CENTER)
 
-    const int u = a.unit0 + blockIdx.y;
+    const int u = blockIdx.y;
     const int tile = blockIdx.x;
     const int b = u / a.Hkv, h = u % a.Hkv;
     const SeqRow sr = a.seq[b];
@@ -331,7 +329,7 @@ __global__ void __launch_bounds__(kK1Threads, 2)
     uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kK1Stages * kK1StageBytes);
     long long *warp_sum = reinterpret_cast<long long *>(bar + 8);
 
-    const int u = a.unit0 + blockIdx.y;
+    const int u = blockIdx.y;
     const int tile = blockIdx.x;
     const int b = u / a.Hkv, h = u % a.Hkv;
     const SeqRow sr = a.seq[b];
@@ -428,7 +426,7 @@ __global__ void __launch_bounds__(kK1Threads, 2)
 __global__ void __launch_bounds__(256) k_tile_prefix(const CoarsenArgs a) {
     __shared__ long long wsum[8];
     __shared__ long long carry_s;
-    const int u = a.unit0 + blockIdx.x;
+    const int u = blockIdx.x;
     const int b = u / a.Hkv;
     const SeqRow sr = a.seq[b];
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
@@ -473,7 +471,7 @@ __device__ __forceinline__ long long floor_ratio(long long N, long long C, long 
 }
 
 __global__ void __launch_bounds__(kTileRows) k_boundaries(const CoarsenArgs a) {
-    const int u = a.unit0 + blockIdx.y, tile = blockIdx.x;
+    const int u = blockIdx.y, tile = blockIdx.x;
     const int b = u / a.Hkv, h = u % a.Hkv;
     const SeqRow sr = a.seq[b];
     if (tile >= sr.tiles || threadIdx.x >= kTileOut) return;
@@ -505,7 +503,7 @@ __global__ void __launch_bounds__(kTileRows) k_boundaries(const CoarsenArgs a) {
 __global__ void __launch_bounds__(512) k_plan_entries(const CoarsenArgs a) {
     __shared__ int wsum[16];
     __shared__ int carry_s;
-    const int u = a.unit0 + blockIdx.x;
+    const int u = blockIdx.x;
     const int b = u / a.Hkv, h = u % a.Hkv;
     const SeqRow sr = a.seq[b];
     const int N = sr.N, M = sr.M;
@@ -600,7 +598,7 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
     constexpr int EPL = 16 / ELEM;        // elements per lane
     static_assert(CH >= 8 && CH <= 32, "row must span 8..32 chunks");
 
-    const int u = a.unit0 + blockIdx.y;
+    const int u = blockIdx.y;
     const int b = u / a.Hkv, h = u % a.Hkv;
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int e = blockIdx.x * kK3Warps + warp;
@@ -781,7 +779,7 @@ static cudaError_t launch_project_tc(const CoarsenArgs &a, int n_units, const Pr
     return cudaSuccess;
 }
 
-// The projection of units [a.unit0, a.unit0 + n): quantised steps and tile scans.
+// The projection of the batch's n units: quantised steps and tile scans.
 template <int D, typename T, bool CENTER>
 static cudaError_t launch_projection(const CoarsenArgs &a, int n, const ProjT &proj, const ProjFrag &frag,
                                      const CUtensorMap &map_k, const CUtensorMap &map_v, cudaStream_t s) {
@@ -806,8 +804,8 @@ static cudaError_t launch_projection(const CoarsenArgs &a, int n, const ProjT &p
     return cudaSuccess;
 }
 
-// Everything after the projection for units [a.unit0, a.unit0 + n): prefix over tiles, boundaries,
-// entries, segment statistics.
+// Everything after the projection for the batch's n units: prefix over tiles, boundaries, entries,
+// segment statistics.
 template <int D, typename T, bool CENTER>
 static void launch_segments(const CoarsenArgs &a, int n, cudaStream_t s) {
     if (a.max_tiles > 0) {
@@ -824,45 +822,6 @@ static void launch_segments(const CoarsenArgs &a, int n, cudaStream_t s) {
     }
 }
 
-// Waves of units: the raw keys and values of one wave fit comfortably in the 126 MB L2, so the
-// segment statistics, which read them a second time, find them there if they run while (or just
-// after) the wave is projected. Consecutive units of at most kWaveBytes together (at least one).
-constexpr size_t kWaveBytes = 72u << 20;
-
-struct SideStream {
-    int dev = -1;
-    cudaStream_t s = nullptr;
-    std::vector<cudaEvent_t> ev;
-};
-
-// The library's side stream of the current device (created once, highest priority) and at least
-// `n` events, created on first use; guarded by the coarsening call's lock.
-static cudaError_t side_stream(size_t n, SideStream **out) {
-    static std::vector<SideStream> all;
-    int dev = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e != cudaSuccess) return e;
-    SideStream *ss = nullptr;
-    for (auto &x : all)
-        if (x.dev == dev) ss = &x;
-    if (!ss) {
-        SideStream x;
-        x.dev = dev;
-        int lo = 0, hi = 0;
-        if ((e = cudaDeviceGetStreamPriorityRange(&lo, &hi)) != cudaSuccess) return e;
-        if ((e = cudaStreamCreateWithPriority(&x.s, cudaStreamNonBlocking, hi)) != cudaSuccess) return e;
-        all.push_back(x);
-        ss = &all.back();
-    }
-    while (ss->ev.size() < n) {
-        cudaEvent_t ev;
-        if ((e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming)) != cudaSuccess) return e;
-        ss->ev.push_back(ev);
-    }
-    *out = ss;
-    return cudaSuccess;
-}
-
 template <int D, typename T, bool CENTER>
 static cudaError_t launch_typed(const CoarsenArgs &a, const SeqTable &table, const ProjT &proj, const ProjFrag &frag,
                                 const CUtensorMap &map_k, const CUtensorMap &map_v, cudaStream_t s) {
@@ -872,50 +831,11 @@ static cudaError_t launch_typed(const CoarsenArgs &a, const SeqTable &table, con
         k_key_block_sums<D, T><<<dim3(a.max_blk, units), D, 0, s>>>(a);
         k_key_mean<D><<<units, D, 0, s>>>(a);
     }
-    // waves of consecutive units (unit u = b * Hkv + h holds 2 T_b d elements)
-    std::vector<std::pair<int, int>> waves;   // (first unit, units)
-    size_t total = 0;
-    {
-        size_t wb = 0;
-        for (int u = 0; u < units; ++u) {
-            const size_t ub = 2ull * table.rows[u / a.Hkv].T * D * sizeof(T);
-            total += ub;
-            if (waves.empty() || wb + ub > kWaveBytes) {
-                waves.emplace_back(u, 0);
-                wb = 0;
-            }
-            waves.back().second += 1;
-            wb += ub;
-        }
+    if (a.max_tiles > 0) {
+        const cudaError_t e = launch_projection<D, T, CENTER>(a, units, proj, frag, map_k, map_v, s);
+        if (e != cudaSuccess) return e;
     }
-    cudaError_t e = cudaSuccess;
-    if (a.max_tiles == 0 || waves.size() < 3 || total < 3 * kWaveBytes) {
-        // one pass over the whole batch on the caller's stream
-        if (a.max_tiles > 0 && (e = launch_projection<D, T, CENTER>(a, units, proj, frag, map_k, map_v, s)) != cudaSuccess)
-            return e;
-        launch_segments<D, T, CENTER>(a, units, s);
-        return cudaGetLastError();
-    }
-    // Wave pipeline: the projection of wave w runs on the caller's stream while the library's side
-    // stream takes the later stages of wave w - 1, whose keys and values are still in L2. The
-    // projection of wave w waits for the side stream to finish wave w - 2, so that the side stream
-    // never falls more than one wave behind (and its reads stay L2 hits).
-    SideStream *ss = nullptr;
-    const size_t nw = waves.size();
-    if ((e = side_stream(2 * nw, &ss)) != cudaSuccess) return e;
-    cudaEvent_t *ev_proj = ss->ev.data(), *ev_side = ss->ev.data() + nw;
-    for (size_t w = 0; w < nw; ++w) {
-        CoarsenArgs aw = a;
-        aw.unit0 = waves[w].first;
-        const int n = waves[w].second;
-        if (w >= 2 && (e = cudaStreamWaitEvent(s, ev_side[w - 2], 0)) != cudaSuccess) return e;
-        if ((e = launch_projection<D, T, CENTER>(aw, n, proj, frag, map_k, map_v, s)) != cudaSuccess) return e;
-        if ((e = cudaEventRecord(ev_proj[w], s)) != cudaSuccess) return e;
-        if ((e = cudaStreamWaitEvent(ss->s, ev_proj[w], 0)) != cudaSuccess) return e;
-        launch_segments<D, T, CENTER>(aw, n, ss->s);
-        if ((e = cudaEventRecord(ev_side[w], ss->s)) != cudaSuccess) return e;
-    }
-    if ((e = cudaStreamWaitEvent(s, ev_side[nw - 1], 0)) != cudaSuccess) return e;   // join
+    launch_segments<D, T, CENTER>(a, units, s);
     return cudaGetLastError();
 }
 

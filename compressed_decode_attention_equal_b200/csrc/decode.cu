@@ -61,28 +61,21 @@ template <int D, int NT, bool DIAG = false>
 struct SplitSmem {
     static constexpr int QROWB = D * 2 + 16;              // padded query row: conflict-free ldmatrix
     static constexpr int QBUF = NT * 8 * QROWB;           // the query rows of one piece
-    // Row tiles per consumer warp. With 16 or more query rows per unit a warp takes two row
-    // tiles: the page's K and V fragments, loaded once, feed both tiles' MMAs (two independent
-    // accumulator chains), and each page passes through half as many warps.
-    static constexpr int TPW = (!DIAG && NT >= 2) ? 2 : 1;
     // Consumer warps. With the variances a page carries 1.5x the bytes and 3x the MMAs before PV:
     // one CTA per SM with 8 consumer warps and 8 stages takes a whole unit (measured 27.5 us
-    // against 32.2 us for 4 warps, 4 stages and 3 CTAs per SM on the 7B 3.5% shape). Two row
-    // tiles per warp need about 200 registers per thread; the register file is split over the
-    // SM's four schedulers, so at most two warps may share one: one CTA per SM of 6 consumer
-    // warps and the producer. One row tile: 4 consumer warps, two CTAs per SM.
-    static constexpr int CONS = DIAG ? 8 : (TPW == 2 ? 6 : kDecConsumers);
-    static constexpr int CTAS_PER_SM = CONS == kDecConsumers ? 2 : 1;
+    // against 32.2 us for 4 warps, 4 stages and 3 CTAs per SM on the 7B 3.5% shape). Otherwise
+    // 4 consumer warps and two CTAs per SM. (Two row tiles per warp sharing the K and V
+    // fragments, which needs one CTA of 6 consumer warps per SM for its registers, measured 94 us
+    // against 81 us on the ragged paged 2% workload.)
+    static constexpr int CONS = DIAG ? 8 : kDecConsumers;
+    static constexpr int CTAS_PER_SM = DIAG ? 1 : 2;
     static constexpr int THREADS = (CONS + 1) * 32;
-    static constexpr int WPP = NT / TPW;                  // consumer warps per page
-    static constexpr int PG = CONS / WPP;                 // page groups (pages i, i + PG, ... per warp)
-    // two row tiles per warp (3 or 6 page groups): 12 stages keep 100 KB of pages in flight per
-    // SM, about what two CTAs of the one-tile configuration keep
-    static constexpr int STAGES = DIAG ? 8 : (TPW == 2 ? 12 : kDecStages);
+    static constexpr int PG = CONS / NT;                  // page groups (pages i, i + PG, ... per warp)
+    static constexpr int STAGES = DIAG ? 8 : kDecStages;
     static_assert(STAGES % PG == 0, "a stage's successive pages must go to one consumer warp");
     static constexpr int STAGES_BYTES = STAGES * PageGeom<D, DIAG>::STAGE;
     static constexpr int MST = D + 4;                     // mbuf row stride: 16-byte rows
-    static constexpr int MBUF_FLOATS = PG * NT * 8 * MST; // per page group and query row: O, m, l
+    static constexpr int MBUF_FLOATS = CONS * 8 * MST;   // per page group and query row: O, m, l
     static constexpr int BARS = 2 * STAGES + 4;
     static constexpr int ROWS = NT * 8;                   // query rows of one piece
     static constexpr int WST = 9;                         // merge weights per row (<= 8) + log2 partition
@@ -296,9 +289,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     using L = SplitSmem<D, NT, DIAG>;
     constexpr int NCONS = L::CONS;           // consumer warps (the producer is warp NCONS)
     constexpr int NTHR = L::THREADS;
-    constexpr int TPW = L::TPW;              // row tiles per consumer warp
-    constexpr int WPP = L::WPP;              // consumer warps per page
-    constexpr int PG = L::PG;                // page groups: the warps of a group share each page
+    constexpr int PG = L::PG;                // page groups: warps sharing a row tile split the pages
     constexpr int NKS = D / 16;              // QK k-steps over dims == PV m-tiles over dims
     constexpr int NS = L::STAGES;            // ring depth
     static_assert(NS % PG == 0, "a stage's successive pages must go to one consumer warp");
@@ -329,7 +320,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     if (tid == 0) {   // independent of the inputs: overlaps the wait below
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], WPP);
+            mbar_init(&empty[s], NT);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&qfull[s], 1);
@@ -448,7 +439,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                 mbar_inval(&full[s2]);
                 mbar_inval(&empty[s2]);
                 mbar_init(&full[s2], 1);
-                mbar_init(&empty[s2], WPP);
+                mbar_init(&empty[s2], NT);
             }
             for (int s2 = 0; s2 < 2; ++s2) {
                 mbar_inval(&qfull[s2]);
@@ -559,7 +550,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     }
 
     // ------------------------------- consumers -------------------------------
-    const int wt = warp % WPP, pg = warp / WPP;   // row tiles wt*TPW .. wt*TPW+TPW-1; page group pg
+    const int nt = warp % NT, pg = warp / NT;   // row tile nt, page group pg
     const int g = lane >> 2, c = lane & 3;
     const int ctid = tid;   // 0 .. NCONS * 32 - 1
     const float c_scale = kLog2e * rsqrtf(static_cast<float>(D));
@@ -579,69 +570,55 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
             orow[ctid] = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
         }
 
-        // Q^T fragments of this warp's row tiles (rows (wt*TPW + tt)*8 + g of the piece), |q|^2
-        uint32_t qf[TPW][NKS][2];
-        float qn_r0[TPW], qn_r1[TPW];
+        // Q^T fragments of rows nt*8 + g of this piece (ldmatrix from the producer's copy), |q|^2
+        uint32_t qf[NKS][2];
+        float qn = 0.0f;
         {
             const int slot = pi & 1;
             if (alive && !mbar_wait(&qfull[slot], (pi >> 1) & 1)) {
                 if (lane == 0) raise_flag(a.flags, FLAG_TIMEOUT);
                 alive = false;
             }
+            const uint32_t qb = smem_u32(qbuf + slot * L::QBUF) + (nt * 8 + (lane & 7)) * L::QROWB;
 #pragma unroll
-            for (int tt = 0; tt < TPW; ++tt) {
-                const uint32_t qb =
-                    smem_u32(qbuf + slot * L::QBUF) + ((wt * TPW + tt) * 8 + (lane & 7)) * L::QROWB;
-#pragma unroll
-                for (int k2 = 0; k2 < NKS / 2; ++k2)
-                    ldsm_x4(qb + ((4 * k2 + (lane >> 3)) << 4), qf[tt][2 * k2][0], qf[tt][2 * k2][1],
-                            qf[tt][2 * k2 + 1][0], qf[tt][2 * k2 + 1][1]);
-            }
+            for (int k2 = 0; k2 < NKS / 2; ++k2)
+                ldsm_x4(qb + ((4 * k2 + (lane >> 3)) << 4), qf[2 * k2][0], qf[2 * k2][1], qf[2 * k2 + 1][0],
+                        qf[2 * k2 + 1][1]);
             __syncwarp();
             if (lane == 0) mbar_arrive(&qempty[slot]);
 #pragma unroll
-            for (int tt = 0; tt < TPW; ++tt) {
-                float qn = 0.0f;
-#pragma unroll
-                for (int ks = 0; ks < NKS; ++ks) {
-                    const uint32_t w0 = qf[tt][ks][0], w1 = qf[tt][ks][1];
-                    qn = fmaf(bf16lo(w0), bf16lo(w0), qn);
-                    qn = fmaf(bf16hi(w0), bf16hi(w0), qn);
-                    qn = fmaf(bf16lo(w1), bf16lo(w1), qn);
-                    qn = fmaf(bf16hi(w1), bf16hi(w1), qn);
-                }
-                qn += __shfl_xor_sync(0xffffffffu, qn, 1);
-                qn += __shfl_xor_sync(0xffffffffu, qn, 2);
-                qn_r0[tt] = __shfl_sync(0xffffffffu, qn, (2 * c) * 4);
-                qn_r1[tt] = __shfl_sync(0xffffffffu, qn, (2 * c + 1) * 4);
+            for (int ks = 0; ks < NKS; ++ks) {
+                const uint32_t w0 = qf[ks][0], w1 = qf[ks][1];
+                qn = fmaf(bf16lo(w0), bf16lo(w0), qn);
+                qn = fmaf(bf16hi(w0), bf16hi(w0), qn);
+                qn = fmaf(bf16lo(w1), bf16lo(w1), qn);
+                qn = fmaf(bf16hi(w1), bf16hi(w1), qn);
             }
         }
         // diagonal closure: q_i^2 as the B operand of Var (16 x D) (q^2)^T, split into bf16 hi + lo
         // (q^2 of a bf16 q has at most 16 significant bits: hi + lo holds it exactly)
         uint32_t q2h[DIAG ? NKS : 1][2], q2l[DIAG ? NKS : 1][2];
         if constexpr (DIAG) {
-            static_assert(!DIAG || TPW == 1, "the diagonal closure keeps one row tile per warp");
 #pragma unroll
             for (int ks = 0; ks < NKS; ++ks)
 #pragma unroll
                 for (int r2 = 0; r2 < 2; ++r2) {
-                    const float lo2 = bf16lo(qf[0][ks][r2]), hi2 = bf16hi(qf[0][ks][r2]);
+                    const float lo2 = bf16lo(qf[ks][r2]), hi2 = bf16hi(qf[ks][r2]);
                     const float slo = lo2 * lo2, shi = hi2 * hi2;
                     const uint32_t h2 = pack_bf16x2(slo, shi);
                     q2h[ks][r2] = h2;
                     q2l[ks][r2] = pack_bf16x2(slo - bf16lo(h2), shi - bf16hi(h2));
                 }
         }
+        qn += __shfl_xor_sync(0xffffffffu, qn, 1);
+        qn += __shfl_xor_sync(0xffffffffu, qn, 2);
+        const float qn_r0 = __shfl_sync(0xffffffffu, qn, (2 * c) * 4);
+        const float qn_r1 = __shfl_sync(0xffffffffu, qn, (2 * c + 1) * 4);
 
-        float m_run[TPW][2], l_run[TPW][2];
-        float o[TPW][NKS][4];
+        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+        float o[NKS][4];
 #pragma unroll
-        for (int tt = 0; tt < TPW; ++tt) {
-            m_run[tt][0] = m_run[tt][1] = -INFINITY;
-            l_run[tt][0] = l_run[tt][1] = 0.0f;
-#pragma unroll
-            for (int mt = 0; mt < NKS; ++mt) o[tt][mt][0] = o[tt][mt][1] = o[tt][mt][2] = o[tt][mt][3] = 0.0f;
-        }
+        for (int mt = 0; mt < NKS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.0f;
 
         // page i of the CTA's range goes to page group i % PG (global index, not piece-local)
         for (int k = ((pg - i0 % PG) + PG) % PG; k < npg && alive; k += PG) {
@@ -654,13 +631,9 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
             }
             const bool valid = svalid[s] != 0;
             const int nvalid = min(kPageNodes, Lent - (lo + k) * kPageNodes);
-            // S^T accumulators: two per row tile (even / odd k-steps), so that no chain of
-            // dependent MMAs is longer than NKS / 2
-            float sacc[TPW][2][4];
-#pragma unroll
-            for (int tt = 0; tt < TPW; ++tt)
-#pragma unroll
-                for (int hh = 0; hh < 2; ++hh) sacc[tt][hh][0] = sacc[tt][hh][1] = sacc[tt][hh][2] = sacc[tt][hh][3] = 0.0f;
+            // S^T accumulators: even and odd k-steps apart, so that no chain of dependent MMAs is
+            // longer than NKS / 2
+            float sacc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
             float cacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // diagonal closure: sum_i q_i^2 var_i
             uint32_t vf[NKS][4];
             float2 ab0 = make_float2(0.0f, 0.0f), ab1 = ab0;
@@ -668,35 +641,18 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                 const uint32_t kb = smem_u32(stages + s * G::STAGE);
                 const uint32_t vb = kb + G::VEC_BYTES;
                 const float2 *ab = reinterpret_cast<const float2 *>(stages + s * G::STAGE + 2 * G::VEC_BYTES);
-                // S^T (16 nodes x 8 rows) = K (16 x D) Q^T (D x 8), per row tile
+                // S^T (16 nodes x 8 rows) = K (16 x D) Q^T (D x 8): every K fragment first
+                // (independent shared loads), then the MMAs
                 {
                     const int mi = lane >> 3, node = (lane & 7) + 8 * (mi & 1);
-                    if constexpr (TPW == 1) {
-                        // every K fragment first (independent shared loads), then the MMAs
-                        uint32_t kf[NKS][4];
+                    uint32_t kf[NKS][4];
 #pragma unroll
-                        for (int ks = 0; ks < NKS; ++ks)
-                            ldsm_x4(kb + node * G::ROWB + (swz(2 * ks + (mi >> 1), node) << 4), kf[ks][0], kf[ks][1],
-                                    kf[ks][2], kf[ks][3]);
+                    for (int ks = 0; ks < NKS; ++ks)
+                        ldsm_x4(kb + node * G::ROWB + (swz(2 * ks + (mi >> 1), node) << 4), kf[ks][0], kf[ks][1],
+                                kf[ks][2], kf[ks][3]);
 #pragma unroll
-                        for (int ks = 0; ks < NKS; ++ks)
-                            mma_bf16(sacc[0][ks & 1], kf[ks][0], kf[ks][1], kf[ks][2], kf[ks][3], qf[0][ks][0],
-                                     qf[0][ks][1]);
-                    } else {
-                        // one K fragment feeds every row tile; the next one is loaded a step ahead
-                        uint32_t kn[4];
-                        ldsm_x4(kb + node * G::ROWB + (swz(mi >> 1, node) << 4), kn[0], kn[1], kn[2], kn[3]);
-#pragma unroll
-                        for (int ks = 0; ks < NKS; ++ks) {
-                            const uint32_t k0 = kn[0], k1 = kn[1], k2 = kn[2], k3 = kn[3];
-                            if (ks + 1 < NKS)
-                                ldsm_x4(kb + node * G::ROWB + (swz(2 * (ks + 1) + (mi >> 1), node) << 4), kn[0], kn[1],
-                                        kn[2], kn[3]);
-#pragma unroll
-                            for (int tt = 0; tt < TPW; ++tt)
-                                mma_bf16(sacc[tt][ks & 1], k0, k1, k2, k3, qf[tt][ks][0], qf[tt][ks][1]);
-                        }
-                    }
+                    for (int ks = 0; ks < NKS; ++ks)
+                        mma_bf16(sacc[ks & 1], kf[ks][0], kf[ks][1], kf[ks][2], kf[ks][3], qf[ks][0], qf[ks][1]);
                     if constexpr (DIAG) {   // C^T (16 nodes x 8 rows) = Var (16 x D) (q^2)^T
                         const uint32_t varb = kb + G::VAR_OFF;
 #pragma unroll
@@ -724,101 +680,87 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
             __syncwarp();
             if (lane == 0) mbar_arrive(&empty[s]);   // the page is in registers: release the stage
             if (valid) {
-                // slots past the unit's last entry may hold anything (NaN included): their V^T
-                // elements are zeroed, since P = 0 does not cancel NaN in the product. This
-                // thread's fragment holds nodes 2c, 2c+1 (a0..a3) and 2c+8, 2c+9 (a4..a7).
-                if (nvalid < kPageNodes) {
+                float sl[4];
+                // closure: |q|^2 beta, or sum_i q_i^2 var_i / (2d) with the diagonal variances
+                constexpr float kInv2d = 0.5f / D;
+                const float cl0 = DIAG ? fmaf(cacc[0], kInv2d, ab0.x) : fmaf(qn_r0, ab0.y, ab0.x);
+                const float cl1 = DIAG ? fmaf(cacc[1], kInv2d, ab0.x) : fmaf(qn_r1, ab0.y, ab0.x);
+                const float cl2 = DIAG ? fmaf(cacc[2], kInv2d, ab1.x) : fmaf(qn_r0, ab1.y, ab1.x);
+                const float cl3 = DIAG ? fmaf(cacc[3], kInv2d, ab1.x) : fmaf(qn_r1, ab1.y, ab1.x);
+                sl[0] = g < nvalid ? fmaf(sacc[0][0] + sacc[1][0], c_scale, kLog2e * cl0) : -INFINITY;
+                sl[1] = g < nvalid ? fmaf(sacc[0][1] + sacc[1][1], c_scale, kLog2e * cl1) : -INFINITY;
+                sl[2] = g + 8 < nvalid ? fmaf(sacc[0][2] + sacc[1][2], c_scale, kLog2e * cl2) : -INFINITY;
+                sl[3] = g + 8 < nvalid ? fmaf(sacc[0][3] + sacc[1][3], c_scale, kLog2e * cl3) : -INFINITY;
+                float mx0 = fmaxf(sl[0], sl[2]), mx1 = fmaxf(sl[1], sl[3]);
+#pragma unroll
+                for (int off = 4; off < 32; off <<= 1) {
+                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                }
+                const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+                const float base0 = mn0 == -INFINITY ? 0.0f : mn0;
+                const float base1 = mn1 == -INFINITY ? 0.0f : mn1;
+                const float corr0 = ex2(m_run[0] - base0), corr1 = ex2(m_run[1] - base1);
+                const float p0 = ex2(sl[0] - base0), p1 = ex2(sl[1] - base1);
+                const float p2 = ex2(sl[2] - base0), p3 = ex2(sl[3] - base1);
+                l_run[0] = fmaf(l_run[0], corr0, p0 + p2);
+                l_run[1] = fmaf(l_run[1], corr1, p1 + p3);
+                m_run[0] = mn0;
+                m_run[1] = mn1;
+                if (!__all_sync(0xffffffffu, corr0 == 1.0f && corr1 == 1.0f)) {
+#pragma unroll
+                    for (int mt = 0; mt < NKS; ++mt) {
+                        o[mt][0] *= corr0;
+                        o[mt][1] *= corr1;
+                        o[mt][2] *= corr0;
+                        o[mt][3] *= corr1;
+                    }
+                }
+                // P^T as the B operand (16 nodes x 8 rows): transpose the 8x8 halves in registers
+                const uint32_t bp0 = movmatrix_t(pack_bf16x2(p0, p1));
+                const uint32_t bp1 = movmatrix_t(pack_bf16x2(p2, p3));
+                // O^T (D x 8) += V^T (D x 16) P^T (16 x 8)
+                if (nvalid == kPageNodes) {
+#pragma unroll
+                    for (int mt = 0; mt < NKS; ++mt) mma_bf16(o[mt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], bp0, bp1);
+                } else {
+                    // slots past the unit's last entry may hold anything (NaN included): zero their
+                    // V^T elements, since P = 0 does not cancel NaN in the product. This thread's
+                    // fragment holds nodes 2c, 2c+1 (a0..a3) and 2c+8, 2c+9 (a4..a7).
                     const uint32_t m_lo =
                         (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
                     const uint32_t m_hi =
                         (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
 #pragma unroll
-                    for (int mt = 0; mt < NKS; ++mt) {
-                        vf[mt][0] &= m_lo;
-                        vf[mt][1] &= m_lo;
-                        vf[mt][2] &= m_hi;
-                        vf[mt][3] &= m_hi;
-                    }
+                    for (int mt = 0; mt < NKS; ++mt)
+                        mma_bf16(o[mt], vf[mt][0] & m_lo, vf[mt][1] & m_lo, vf[mt][2] & m_hi, vf[mt][3] & m_hi, bp0,
+                                 bp1);
                 }
-                uint32_t bp0[TPW], bp1[TPW];
-#pragma unroll
-                for (int tt = 0; tt < TPW; ++tt) {
-                    float sl[4];
-                    // closure: |q|^2 beta, or sum_i q_i^2 var_i / (2d) with the diagonal variances
-                    constexpr float kInv2d = 0.5f / D;
-                    const float cl0 = DIAG ? fmaf(cacc[0], kInv2d, ab0.x) : fmaf(qn_r0[tt], ab0.y, ab0.x);
-                    const float cl1 = DIAG ? fmaf(cacc[1], kInv2d, ab0.x) : fmaf(qn_r1[tt], ab0.y, ab0.x);
-                    const float cl2 = DIAG ? fmaf(cacc[2], kInv2d, ab1.x) : fmaf(qn_r0[tt], ab1.y, ab1.x);
-                    const float cl3 = DIAG ? fmaf(cacc[3], kInv2d, ab1.x) : fmaf(qn_r1[tt], ab1.y, ab1.x);
-                    const float s0 = sacc[tt][0][0] + sacc[tt][1][0], s1 = sacc[tt][0][1] + sacc[tt][1][1];
-                    const float s2 = sacc[tt][0][2] + sacc[tt][1][2], s3 = sacc[tt][0][3] + sacc[tt][1][3];
-                    sl[0] = g < nvalid ? fmaf(s0, c_scale, kLog2e * cl0) : -INFINITY;
-                    sl[1] = g < nvalid ? fmaf(s1, c_scale, kLog2e * cl1) : -INFINITY;
-                    sl[2] = g + 8 < nvalid ? fmaf(s2, c_scale, kLog2e * cl2) : -INFINITY;
-                    sl[3] = g + 8 < nvalid ? fmaf(s3, c_scale, kLog2e * cl3) : -INFINITY;
-                    float mx0 = fmaxf(sl[0], sl[2]), mx1 = fmaxf(sl[1], sl[3]);
-#pragma unroll
-                    for (int off = 4; off < 32; off <<= 1) {
-                        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
-                    }
-                    const float mn0 = fmaxf(m_run[tt][0], mx0), mn1 = fmaxf(m_run[tt][1], mx1);
-                    const float base0 = mn0 == -INFINITY ? 0.0f : mn0;
-                    const float base1 = mn1 == -INFINITY ? 0.0f : mn1;
-                    const float corr0 = ex2(m_run[tt][0] - base0), corr1 = ex2(m_run[tt][1] - base1);
-                    const float p0 = ex2(sl[0] - base0), p1 = ex2(sl[1] - base1);
-                    const float p2 = ex2(sl[2] - base0), p3 = ex2(sl[3] - base1);
-                    l_run[tt][0] = fmaf(l_run[tt][0], corr0, p0 + p2);
-                    l_run[tt][1] = fmaf(l_run[tt][1], corr1, p1 + p3);
-                    m_run[tt][0] = mn0;
-                    m_run[tt][1] = mn1;
-                    if (!__all_sync(0xffffffffu, corr0 == 1.0f && corr1 == 1.0f)) {
-#pragma unroll
-                        for (int mt = 0; mt < NKS; ++mt) {
-                            o[tt][mt][0] *= corr0;
-                            o[tt][mt][1] *= corr1;
-                            o[tt][mt][2] *= corr0;
-                            o[tt][mt][3] *= corr1;
-                        }
-                    }
-                    // P^T as the B operand (16 nodes x 8 rows): transpose the 8x8 halves in registers
-                    bp0[tt] = movmatrix_t(pack_bf16x2(p0, p1));
-                    bp1[tt] = movmatrix_t(pack_bf16x2(p2, p3));
-                }
-                // O^T (D x 8) += V^T (D x 16) P^T (16 x 8), per row tile
-#pragma unroll
-                for (int mt = 0; mt < NKS; ++mt)
-#pragma unroll
-                    for (int tt = 0; tt < TPW; ++tt)
-                        mma_bf16(o[tt][mt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], bp0[tt], bp1[tt]);
             }
         }
         i0 += npg;
         ++pi;
 
         // ---- piece epilogue: merge the page groups through shared memory ----
+#pragma unroll
+        for (int off = 4; off < 32; off <<= 1) {
+            l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
+            l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
+        }
         constexpr int MST = L::MST, WST = L::WST;
+        float *mw = mbuf + warp * 8 * MST;
 #pragma unroll
-        for (int tt = 0; tt < TPW; ++tt) {
-#pragma unroll
-            for (int off = 4; off < 32; off <<= 1) {
-                l_run[tt][0] += __shfl_xor_sync(0xffffffffu, l_run[tt][0], off);
-                l_run[tt][1] += __shfl_xor_sync(0xffffffffu, l_run[tt][1], off);
-            }
-            float *mw = mbuf + ((pg * NT + wt * TPW + tt) * 8) * MST;
-#pragma unroll
-            for (int mt = 0; mt < NKS; ++mt) {
-                mw[(2 * c) * MST + 16 * mt + g] = o[tt][mt][0];
-                mw[(2 * c + 1) * MST + 16 * mt + g] = o[tt][mt][1];
-                mw[(2 * c) * MST + 16 * mt + g + 8] = o[tt][mt][2];
-                mw[(2 * c + 1) * MST + 16 * mt + g + 8] = o[tt][mt][3];
-            }
-            if (g == 0) {
-                mw[(2 * c) * MST + D] = m_run[tt][0];
-                mw[(2 * c) * MST + D + 1] = l_run[tt][0];
-                mw[(2 * c + 1) * MST + D] = m_run[tt][1];
-                mw[(2 * c + 1) * MST + D + 1] = l_run[tt][1];
-            }
+        for (int mt = 0; mt < NKS; ++mt) {
+            mw[(2 * c) * MST + 16 * mt + g] = o[mt][0];
+            mw[(2 * c + 1) * MST + 16 * mt + g] = o[mt][1];
+            mw[(2 * c) * MST + 16 * mt + g + 8] = o[mt][2];
+            mw[(2 * c + 1) * MST + 16 * mt + g + 8] = o[mt][3];
+        }
+        if (g == 0) {
+            mw[(2 * c) * MST + D] = m_run[0];
+            mw[(2 * c) * MST + D + 1] = l_run[0];
+            mw[(2 * c + 1) * MST + D] = m_run[1];
+            mw[(2 * c + 1) * MST + D + 1] = l_run[1];
         }
         asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
         const bool complete = (ps >= ra) && (pe <= rb);

@@ -68,7 +68,6 @@ struct CoarsenArgs {
     int closure;         // skv_closure: SKV_CLOSURE_DIAGONAL also writes per-dimension variances
     int center;          // 1: keys enter every stage with the unit's mean key removed
     int projection;      // skv_projection: SKV_PROJECTION_TENSOR_BF16 selects k_project_tc
-    int unit0;           // first unit of the launch (the per-unit kernels run over a wave of units)
     int max_blk;         // largest ceil(T / kMeanBlock) over the batch
     float *key_blk;      // [units][max_blk][d] per-block key sums (centring only)
     float *key_mu;       // [units][d] mean key of each unit (centring only)

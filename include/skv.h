@@ -203,7 +203,7 @@ skv_status skv_coarsen(const void *k, const void *v, skv_dtype dtype, int B, int
  * closure: the pool's skv_closure; SKV_CLOSURE_DIAGONAL also writes each
  *   node's per-dimension key variances (zero for exact tokens).
  * center_keys: 1 selects the common-mode mean removal of "SPICY-KV"
- *   Independent Claim 1(b) (keys mapped into an anisotropy-reduced space
+ *   Independent Claim 1(b) (keys mapped into a less anisotropic space
  *   before coarsening): every key of a unit enters the pipeline -- the
  *   projection, the segment statistics and the exact tokens alike -- as
  *   fl32(k_t - mu) with mu the unit's mean key over all T_b tokens. mu follows

@@ -49,7 +49,7 @@
  *      population variance of key dimension i (orc_coarsen_unit2's var). With
  *      var_i = sigma^2 for every i it is the scalar form of R7.
  *  R8  Option (orc_key_mean_f32): common-mode mean removal of [SK]
- *      Independent Claim 1(b) (keys mapped into an anisotropy-reduced space
+ *      Independent Claim 1(b) (keys mapped into a less anisotropic space
  *      before coarsening): every key of a unit has the unit's mean key mu
  *      (over all T tokens) subtracted in fp32, and the coarsening then runs on
  *      the centred keys. Because the centred keys feed the fixed fp32

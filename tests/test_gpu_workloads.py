@@ -164,10 +164,9 @@ def test_coarsen_131k_tensor_projection_full():
         check_nodes(g, u, w.torch_dtype, w.d, f"tensor projection unit ({b},{h})")
 
 
-def test_coarsen_131k_wave_pipeline_captured_equals_direct():
-    """The 131k workload's coarsening runs in waves of units (projection on the caller's stream,
-    later stages on the library's side stream). Captured into a CUDA graph and replayed, it gives
-    the direct call's boundaries, lens and stored nodes bit for bit (half the batch, 16 units)."""
+def test_coarsen_131k_captured_equals_direct():
+    """Half the 131k coarsening workload (16 units of 131,072 tokens) captured into a CUDA graph and
+    replayed gives the direct call's boundaries, lens and stored nodes bit for bit."""
     import dataclasses
     w = dataclasses.replace(workloads.WORKLOADS["coarsen_131k"], B=4)
     r = _coarsen_full(w)
