@@ -261,8 +261,9 @@ def summarise_regions(times_ms, steps: int):
 def time_regions(fn, steps: int, dist_on: bool, regions: int, flush=None):
     """Device time (ms) of `regions` timed regions, each EXACTLY `steps` calls fn(0..steps-1)
     replayed from CUDA graphs and bracketed by a barrier (multi-rank) and a synchronize on both
-    sides. Between regions (outside the timed interval) `flush`, a buffer larger than L2, is
-    rewritten so that no region starts with the previous region's data in L2."""
+    sides. Between regions (outside the timed interval) `flush`, a buffer larger than L2, is read
+    (a sum) so that no region starts with the previous region's data in L2; reading leaves clean
+    lines behind, so the timed calls pay no write-back of the flush."""
     import torch
     graphs = region_graphs(fn, steps)
     for g in graphs:
@@ -271,7 +272,7 @@ def time_regions(fn, steps: int, dist_on: bool, regions: int, flush=None):
     times = []
     for _ in range(regions):
         if flush is not None:
-            flush.add_(1)
+            flush.sum()
         torch.cuda.synchronize()
         if dist_on:
             torch.distributed.barrier()
@@ -291,7 +292,7 @@ def time_regions(fn, steps: int, dist_on: bool, regions: int, flush=None):
 
 def l2_flush_buffer(device):
     import torch
-    return torch.zeros(64 << 20, dtype=torch.float32, device=device)   # 256 MB, twice the 126 MB L2
+    return torch.zeros(64 << 20, dtype=torch.float32, device=device)   # 256 MB, twice the 126 MB L2 (read)
 
 
 def coarsen_stage(device, reps: int = 5, batch: int | None = None):
@@ -560,7 +561,7 @@ def bench_config(w, world: int):
             "middle_nodes": w.N, "entries_per_head": workloads_entries(w), "query_rows_per_step": w.B * w.R * w.Hq,
             "parallelism": f"dp{world}" if world > 1 else "single",
             "l2": "inputs larger than L2: 6 layer caches of 76.8 MB decoded in rotation, and a 256 MB buffer "
-                  "rewritten between timed regions",
+                  "read between timed regions",
             "timing": "CUDA graphs of back-to-back decode calls; CUDA events around each region of exactly "
                       "`steps` calls; median over the regions, then max over ranks"}
 
@@ -653,7 +654,7 @@ def time_e2e_regions(step, fork, join, steps: int, dist_on: bool, regions: int, 
     torch.cuda.synchronize()
     times = []
     for _ in range(regions):
-        flush.add_(1)
+        flush.sum()
         torch.cuda.synchronize()
         if dist_on:
             torch.distributed.barrier()

@@ -82,8 +82,12 @@ constexpr int kK1Stages = 2;
 constexpr int kK1ColBytes = 64;                  // column chunk of every row per stage (64-byte swizzle)
 constexpr int kK1BoxRows = 256;                  // TMA box height (two boxes per stage)
 constexpr int kK1StageBytes = kTileRows * kK1ColBytes;
-constexpr int kZStride = 20;                     // floats per row of the z buffer (conflict-free)
-static_assert(kTileRows % kK1BoxRows == 0 && kTileRows * kZStride * 4 <= kK1Stages * kK1StageBytes, "tile");
+// floats per row of the z buffer: odd, so that 32 consecutive rows at one column hit 32 banks
+constexpr int kZStride = 17;
+// the steps of a tile's outputs, staged after the z buffer for the scan's thread mapping
+constexpr int kZBytes = kTileRows * kZStride * 4;
+static_assert(kTileRows % kK1BoxRows == 0 && kZBytes % 8 == 0 &&
+                  kZBytes + kTileRows * 8 <= kK1Stages * kK1StageBytes, "tile");
 
 template <int D>
 constexpr size_t k1_smem_bytes() {
@@ -126,11 +130,12 @@ __device__ __forceinline__ int k1_sub(int r, int cc) { return r * 4 + (cc ^ ((r 
 __device__ __forceinline__ void scan_tile(const CoarsenArgs &a, const SeqRow &sr, int u, int h, int tile,
                                           const float *zb, long long *warp_sum) {
     const int tid = threadIdx.x;
-    // outputs l = 4 tid + 1 .. 4 tid + 4 (rows of the tile; row 0 is the halo)
-    long long Dv[kK1Tok];
+    // steps of outputs l = tid + 1 + 128 q (rows l - 1 and l of the tile; row 0 is the halo):
+    // consecutive threads read consecutive z rows (conflict-free at the odd row stride)
+    long long *Ds = reinterpret_cast<long long *>(const_cast<float *>(zb) + kTileRows * kZStride);
 #pragma unroll
     for (int q = 0; q < kK1Tok; ++q) {
-        const int l = kK1Tok * tid + 1 + q;
+        const int l = tid + 1 + kK1Threads * q;
         const int t = tile * kTileOut + l - 1;
         long long D_ = 0;
         if (l <= kTileOut && t < sr.M && t > 0) {
@@ -140,7 +145,15 @@ __device__ __forceinline__ void scan_tile(const CoarsenArgs &a, const SeqRow &sr
                 D_ = 0;
             }
         }
-        Dv[q] = D_;
+        if (l <= kTileOut) Ds[l] = D_;
+    }
+    __syncthreads();
+    // the scan takes outputs l = 4 tid + 1 .. 4 tid + 4
+    long long Dv[kK1Tok];
+#pragma unroll
+    for (int q = 0; q < kK1Tok; ++q) {
+        const int l = kK1Tok * tid + 1 + q;
+        Dv[q] = l <= kTileOut ? Ds[l] : 0;
     }
     // block inclusive scan of the per-thread sums
     const int lane = tid & 31, warp = tid >> 5;

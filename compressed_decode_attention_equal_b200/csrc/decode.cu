@@ -70,12 +70,17 @@ struct SplitSmem {
     static constexpr int CONS = DIAG ? 8 : kDecConsumers;
     static constexpr int CTAS_PER_SM = DIAG ? 1 : 2;
     static constexpr int THREADS = (CONS + 1) * 32;
-    static constexpr int PG = CONS / NT;                  // page groups (pages i, i + PG, ... per warp)
-    static constexpr int STAGES = DIAG ? 8 : kDecStages;
+    // 16 or more query rows per unit (scalar closure): query rows are the MMA's M dimension, 16
+    // rows per warp, and the softmax's P feeds the PV product from the accumulators directly
+    static constexpr bool MR = !DIAG && NT >= 2;
+    static constexpr int WPP = MR ? NT / 2 : NT;          // consumer warps per page
+    static constexpr int PG = CONS / WPP;                 // page groups (pages i, i + PG, ... per warp)
+    // four row tiles with rows as M: the doubled page-group buffer leaves room for six stages
+    static constexpr int STAGES = DIAG ? 8 : (MR && NT == 4 ? 6 : kDecStages);
     static_assert(STAGES % PG == 0, "a stage's successive pages must go to one consumer warp");
     static constexpr int STAGES_BYTES = STAGES * PageGeom<D, DIAG>::STAGE;
     static constexpr int MST = D + 4;                     // mbuf row stride: 16-byte rows
-    static constexpr int MBUF_FLOATS = CONS * 8 * MST;   // per page group and query row: O, m, l
+    static constexpr int MBUF_FLOATS = PG * NT * 8 * MST; // per page group and query row: O, m, l
     static constexpr int BARS = 2 * STAGES + 4;
     static constexpr int ROWS = NT * 8;                   // query rows of one piece
     static constexpr int WST = 9;                         // merge weights per row (<= 8) + log2 partition
@@ -289,6 +294,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     using L = SplitSmem<D, NT, DIAG>;
     constexpr int NCONS = L::CONS;           // consumer warps (the producer is warp NCONS)
     constexpr int NTHR = L::THREADS;
+    constexpr bool MR = L::MR;               // query rows as the MMA's M dimension
     constexpr int PG = L::PG;                // page groups: warps sharing a row tile split the pages
     constexpr int NKS = D / 16;              // QK k-steps over dims == PV m-tiles over dims
     constexpr int NS = L::STAGES;            // ring depth
@@ -320,7 +326,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     if (tid == 0) {   // independent of the inputs: overlaps the wait below
         for (int s = 0; s < NS; ++s) {
             mbar_init(&full[s], 1);
-            mbar_init(&empty[s], NT);
+            mbar_init(&empty[s], L::WPP);
         }
         for (int s = 0; s < 2; ++s) {
             mbar_init(&qfull[s], 1);
@@ -439,7 +445,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                 mbar_inval(&full[s2]);
                 mbar_inval(&empty[s2]);
                 mbar_init(&full[s2], 1);
-                mbar_init(&empty[s2], NT);
+                mbar_init(&empty[s2], L::WPP);
             }
             for (int s2 = 0; s2 < 2; ++s2) {
                 mbar_inval(&qfull[s2]);
@@ -550,10 +556,14 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     }
 
     // ------------------------------- consumers -------------------------------
-    const int nt = warp % NT, pg = warp / NT;   // row tile nt, page group pg
+    // warp's row-tile group and page group (one n8 row tile nt = wt per warp; with rows as M, the
+    // 16 rows of tiles 2 wt and 2 wt + 1)
+    const int wt = warp % L::WPP, pg = warp / L::WPP;
+    const int nt = wt;
     const int g = lane >> 2, c = lane & 3;
     const int ctid = tid;   // 0 .. NCONS * 32 - 1
     const float c_scale = kLog2e * rsqrtf(static_cast<float>(D));
+    constexpr int MST = L::MST, WST = L::WST;
     int i0 = 0, pi = 0;
     int split_v[2] = {0, 0}, split_ps[2] = {0, 0}, split_pe[2] = {0, 0}, n_split = 0;   // (thread 0)
     for (int v = v0; v < nv && prefix[v] < rb; ++v) {
@@ -570,197 +580,371 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
             orow[ctid] = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
         }
 
-        // Q^T fragments of rows nt*8 + g of this piece (ldmatrix from the producer's copy), |q|^2
-        uint32_t qf[NKS][2];
-        float qn = 0.0f;
-        {
-            const int slot = pi & 1;
-            if (alive && !mbar_wait(&qfull[slot], (pi >> 1) & 1)) {
-                if (lane == 0) raise_flag(a.flags, FLAG_TIMEOUT);
-                alive = false;
-            }
-            const uint32_t qb = smem_u32(qbuf + slot * L::QBUF) + (nt * 8 + (lane & 7)) * L::QROWB;
-#pragma unroll
-            for (int k2 = 0; k2 < NKS / 2; ++k2)
-                ldsm_x4(qb + ((4 * k2 + (lane >> 3)) << 4), qf[2 * k2][0], qf[2 * k2][1], qf[2 * k2 + 1][0],
-                        qf[2 * k2 + 1][1]);
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&qempty[slot]);
-#pragma unroll
-            for (int ks = 0; ks < NKS; ++ks) {
-                const uint32_t w0 = qf[ks][0], w1 = qf[ks][1];
-                qn = fmaf(bf16lo(w0), bf16lo(w0), qn);
-                qn = fmaf(bf16hi(w0), bf16hi(w0), qn);
-                qn = fmaf(bf16lo(w1), bf16lo(w1), qn);
-                qn = fmaf(bf16hi(w1), bf16hi(w1), qn);
-            }
-        }
-        // diagonal closure: q_i^2 as the B operand of Var (16 x D) (q^2)^T, split into bf16 hi + lo
-        // (q^2 of a bf16 q has at most 16 significant bits: hi + lo holds it exactly)
-        uint32_t q2h[DIAG ? NKS : 1][2], q2l[DIAG ? NKS : 1][2];
-        if constexpr (DIAG) {
-#pragma unroll
-            for (int ks = 0; ks < NKS; ++ks)
-#pragma unroll
-                for (int r2 = 0; r2 < 2; ++r2) {
-                    const float lo2 = bf16lo(qf[ks][r2]), hi2 = bf16hi(qf[ks][r2]);
-                    const float slo = lo2 * lo2, shi = hi2 * hi2;
-                    const uint32_t h2 = pack_bf16x2(slo, shi);
-                    q2h[ks][r2] = h2;
-                    q2l[ks][r2] = pack_bf16x2(slo - bf16lo(h2), shi - bf16hi(h2));
+        if constexpr (MR) {
+            // ---- query rows as the MMA's M dimension (16 or more rows per unit) ----
+            // Warp (wt, pg) takes rows 16 wt .. 16 wt + 15 of the piece for every page of its page
+            // group: S (16 rows x 16 nodes) = Q K^T as two n8 tiles of nodes, the softmax on the
+            // accumulators (each row spread over a quad of lanes), and P -- whose accumulator
+            // layout is already the A operand of the next product -- times V into O (16 rows x D).
+            uint32_t qa[NKS][4];   // A fragments of Q: rows g / g + 8, dims 2c, 2c + 1 (+ 8) of each k-step
+            float qn_g = 0.0f, qn_h = 0.0f;   // |q|^2 of rows g and g + 8 (h: the row 8 below)
+            {
+                const int slot = pi & 1;
+                if (alive && !mbar_wait(&qfull[slot], (pi >> 1) & 1)) {
+                    if (lane == 0) raise_flag(a.flags, FLAG_TIMEOUT);
+                    alive = false;
                 }
-        }
-        qn += __shfl_xor_sync(0xffffffffu, qn, 1);
-        qn += __shfl_xor_sync(0xffffffffu, qn, 2);
-        const float qn_r0 = __shfl_sync(0xffffffffu, qn, (2 * c) * 4);
-        const float qn_r1 = __shfl_sync(0xffffffffu, qn, (2 * c + 1) * 4);
-
-        float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
-        float o[NKS][4];
+                const uint32_t qb =
+                    smem_u32(qbuf + slot * L::QBUF) + (wt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1)) * L::QROWB;
 #pragma unroll
-        for (int mt = 0; mt < NKS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.0f;
-
-        // page i of the CTA's range goes to page group i % PG (global index, not piece-local)
-        for (int k = ((pg - i0 % PG) + PG) % PG; k < npg && alive; k += PG) {
-            const int i = i0 + k;
-            const int s = i % NS;
-            if (!mbar_wait(&full[s], (i / NS) & 1)) {
-                if (lane == 0) raise_flag(a.flags, FLAG_TIMEOUT);
-                alive = false;
-                break;
+                for (int ks = 0; ks < NKS; ++ks)
+                    ldsm_x4(qb + ((2 * ks + (lane >> 4)) << 4), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&qempty[slot]);
+#pragma unroll
+                for (int ks = 0; ks < NKS; ++ks) {
+#pragma unroll
+                    for (int r2 = 0; r2 < 4; r2 += 2) {
+                        const uint32_t wg = qa[ks][r2], wh = qa[ks][r2 + 1];
+                        qn_g = fmaf(bf16lo(wg), bf16lo(wg), qn_g);
+                        qn_g = fmaf(bf16hi(wg), bf16hi(wg), qn_g);
+                        qn_h = fmaf(bf16lo(wh), bf16lo(wh), qn_h);
+                        qn_h = fmaf(bf16hi(wh), bf16hi(wh), qn_h);
+                    }
+                }
+#pragma unroll
+                for (int off = 1; off < 4; off <<= 1) {
+                    qn_g += __shfl_xor_sync(0xffffffffu, qn_g, off);
+                    qn_h += __shfl_xor_sync(0xffffffffu, qn_h, off);
+                }
             }
-            const bool valid = svalid[s] != 0;
-            const int nvalid = min(kPageNodes, Lent - (lo + k) * kPageNodes);
-            // S^T accumulators: even and odd k-steps apart, so that no chain of dependent MMAs is
-            // longer than NKS / 2
-            float sacc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
-            float cacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // diagonal closure: sum_i q_i^2 var_i
-            uint32_t vf[NKS][4];
-            float2 ab0 = make_float2(0.0f, 0.0f), ab1 = ab0;
-            if (valid) {
-                const uint32_t kb = smem_u32(stages + s * G::STAGE);
-                const uint32_t vb = kb + G::VEC_BYTES;
-                const float2 *ab = reinterpret_cast<const float2 *>(stages + s * G::STAGE + 2 * G::VEC_BYTES);
-                // S^T (16 nodes x 8 rows) = K (16 x D) Q^T (D x 8): every K fragment first
-                // (independent shared loads), then the MMAs
-                {
-                    const int mi = lane >> 3, node = (lane & 7) + 8 * (mi & 1);
-                    uint32_t kf[NKS][4];
+            float m_g = -INFINITY, m_h = -INFINITY, l_g = 0.0f, l_h = 0.0f;
+            float o[2 * NKS][4];   // d-tile j: rows g / g + 8, dims 8 j + 2c, 8 j + 2c + 1
 #pragma unroll
-                    for (int ks = 0; ks < NKS; ++ks)
-                        ldsm_x4(kb + node * G::ROWB + (swz(2 * ks + (mi >> 1), node) << 4), kf[ks][0], kf[ks][1],
-                                kf[ks][2], kf[ks][3]);
-#pragma unroll
-                    for (int ks = 0; ks < NKS; ++ks)
-                        mma_bf16(sacc[ks & 1], kf[ks][0], kf[ks][1], kf[ks][2], kf[ks][3], qf[ks][0], qf[ks][1]);
-                    if constexpr (DIAG) {   // C^T (16 nodes x 8 rows) = Var (16 x D) (q^2)^T
-                        const uint32_t varb = kb + G::VAR_OFF;
+            for (int j = 0; j < 2 * NKS; ++j) o[j][0] = o[j][1] = o[j][2] = o[j][3] = 0.0f;
+
+            for (int k = ((pg - i0 % PG) + PG) % PG; k < npg && alive; k += PG) {
+                const int i = i0 + k;
+                const int s = i % NS;
+                if (!mbar_wait(&full[s], (i / NS) & 1)) {
+                    if (lane == 0) raise_flag(a.flags, FLAG_TIMEOUT);
+                    alive = false;
+                    break;
+                }
+                const bool valid = svalid[s] != 0;
+                const int nvalid = min(kPageNodes, Lent - (lo + k) * kPageNodes);
+                if (valid) {
+                    const uint32_t kb = smem_u32(stages + s * G::STAGE);
+                    const uint32_t vb = kb + G::VEC_BYTES;
+                    const float4 *ab4 = reinterpret_cast<const float4 *>(stages + s * G::STAGE + 2 * G::VEC_BYTES);
+                    const int mi = lane >> 3;
+                    // S = Q K^T: the x4 load of K rows at a k-step holds nodes 0-7 (r0, r2) and 8-15
+                    // (r1, r3) as the B fragments of the two node tiles; the next k-step's load is
+                    // issued before this one's MMAs
+                    float sacc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+                    {
+                        const int node = (lane & 7) + 8 * (mi & 1);
+                        uint32_t kn[4];
+                        ldsm_x4(kb + node * G::ROWB + (swz(mi >> 1, node) << 4), kn[0], kn[1], kn[2], kn[3]);
 #pragma unroll
                         for (int ks = 0; ks < NKS; ++ks) {
-                            const int chunk = 2 * ks + (mi >> 1);
-                            uint32_t a0, a1, a2, a3;
-                            ldsm_x4(varb + node * G::ROWB + (swz(chunk, node) << 4), a0, a1, a2, a3);
-                            mma_bf16(cacc, a0, a1, a2, a3, q2h[ks][0], q2h[ks][1]);
-                            mma_bf16(cacc, a0, a1, a2, a3, q2l[ks][0], q2l[ks][1]);
+                            const uint32_t k0 = kn[0], k1 = kn[1], k2 = kn[2], k3 = kn[3];
+                            if (ks + 1 < NKS)
+                                ldsm_x4(kb + node * G::ROWB + (swz(2 * (ks + 1) + (mi >> 1), node) << 4), kn[0], kn[1],
+                                        kn[2], kn[3]);
+                            mma_bf16(sacc[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], k0, k2);
+                            mma_bf16(sacc[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], k1, k3);
+                        }
+                    }
+                    // logits of nodes 8 nt + 2c + e for rows g (accumulator e) and g + 8 (2 + e)
+                    const float4 abA = ab4[c], abB = ab4[4 + c];   // nodes 2c, 2c+1 and 8+2c, 9+2c
+                    const float al[2][2] = {{abA.x, abA.z}, {abB.x, abB.z}};
+                    const float be[2][2] = {{abA.y, abA.w}, {abB.y, abB.w}};
+                    float sg[2][2], sh[2][2];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            const bool in = 8 * nt + 2 * c + e < nvalid;
+                            sg[nt][e] = in ? fmaf(sacc[nt][e], c_scale, kLog2e * fmaf(qn_g, be[nt][e], al[nt][e])) : -INFINITY;
+                            sh[nt][e] = in ? fmaf(sacc[nt][2 + e], c_scale, kLog2e * fmaf(qn_h, be[nt][e], al[nt][e]))
+                                           : -INFINITY;
+                        }
+                    float mxg = fmaxf(fmaxf(sg[0][0], sg[0][1]), fmaxf(sg[1][0], sg[1][1]));
+                    float mxh = fmaxf(fmaxf(sh[0][0], sh[0][1]), fmaxf(sh[1][0], sh[1][1]));
+#pragma unroll
+                    for (int off = 1; off < 4; off <<= 1) {
+                        mxg = fmaxf(mxg, __shfl_xor_sync(0xffffffffu, mxg, off));
+                        mxh = fmaxf(mxh, __shfl_xor_sync(0xffffffffu, mxh, off));
+                    }
+                    const float ng = fmaxf(m_g, mxg), nh = fmaxf(m_h, mxh);
+                    const float bg = ng == -INFINITY ? 0.0f : ng, bh = nh == -INFINITY ? 0.0f : nh;
+                    const float cg = ex2(m_g - bg), ch = ex2(m_h - bh);
+                    float pg_[2][2], ph_[2][2];
+#pragma unroll
+                    for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                        for (int e = 0; e < 2; ++e) {
+                            pg_[nt][e] = ex2(sg[nt][e] - bg);
+                            ph_[nt][e] = ex2(sh[nt][e] - bh);
+                        }
+                    l_g = fmaf(l_g, cg, (pg_[0][0] + pg_[0][1]) + (pg_[1][0] + pg_[1][1]));
+                    l_h = fmaf(l_h, ch, (ph_[0][0] + ph_[0][1]) + (ph_[1][0] + ph_[1][1]));
+                    m_g = ng;
+                    m_h = nh;
+                    if (!__all_sync(0xffffffffu, cg == 1.0f && ch == 1.0f)) {
+#pragma unroll
+                        for (int j = 0; j < 2 * NKS; ++j) {
+                            o[j][0] *= cg;
+                            o[j][1] *= cg;
+                            o[j][2] *= ch;
+                            o[j][3] *= ch;
+                        }
+                    }
+                    // P (16 rows x 16 nodes) as the A operand: accumulator layout, packed to bf16
+                    const uint32_t pa0 = pack_bf16x2(pg_[0][0], pg_[0][1]), pa1 = pack_bf16x2(ph_[0][0], ph_[0][1]);
+                    const uint32_t pa2 = pack_bf16x2(pg_[1][0], pg_[1][1]), pa3 = pack_bf16x2(ph_[1][0], ph_[1][1]);
+                    // O += P V: the transposed x4 load of V at a pair of d-tiles holds nodes 0-7 of both
+                    // (r0, r1) and nodes 8-15 of both (r2, r3). Slots past the unit's last entry may
+                    // hold anything (NaN included): their V elements are zeroed, since P = 0 does not
+                    // cancel NaN (b0 holds nodes 2c, 2c + 1; b1 nodes 2c + 8, 2c + 9).
+                    const uint32_t m_lo = nvalid == kPageNodes ? 0xffffffffu
+                                          : (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
+                    const uint32_t m_hi = nvalid == kPageNodes ? 0xffffffffu
+                                          : (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
+                    {
+                        const int node = (lane & 7) + 8 * (mi >> 1);
+                        uint32_t vn[4];
+                        ldsm_x4_t(vb + node * G::ROWB + (swz(mi & 1, node) << 4), vn[0], vn[1], vn[2], vn[3]);
+#pragma unroll
+                        for (int mt = 0; mt < NKS; ++mt) {
+                            const uint32_t v0 = vn[0] & m_lo, v1 = vn[1] & m_lo, v2 = vn[2] & m_hi, v3 = vn[3] & m_hi;
+                            if (mt + 1 < NKS)
+                                ldsm_x4_t(vb + node * G::ROWB + (swz(2 * (mt + 1) + (mi & 1), node) << 4), vn[0], vn[1],
+                                          vn[2], vn[3]);
+                            mma_bf16(o[2 * mt], pa0, pa1, pa2, pa3, v0, v2);
+                            mma_bf16(o[2 * mt + 1], pa0, pa1, pa2, pa3, v1, v3);
                         }
                     }
                 }
-                // V^T fragments (A operand of O^T = V^T P^T) into registers now, so the stage goes
-                // back to the producer before the softmax
-                {
-                    const int mi = lane >> 3, node = (lane & 7) + 8 * (mi >> 1);
-#pragma unroll
-                    for (int mt = 0; mt < NKS; ++mt)
-                        ldsm_x4_t(vb + node * G::ROWB + (swz(2 * mt + (mi & 1), node) << 4), vf[mt][0], vf[mt][1],
-                                  vf[mt][2], vf[mt][3]);
-                }
-                ab0 = ab[g];
-                ab1 = ab[g + 8];
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);   // K and V read: release the stage
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&empty[s]);   // the page is in registers: release the stage
-            if (valid) {
-                float sl[4];
-                // closure: |q|^2 beta, or sum_i q_i^2 var_i / (2d) with the diagonal variances
-                constexpr float kInv2d = 0.5f / D;
-                const float cl0 = DIAG ? fmaf(cacc[0], kInv2d, ab0.x) : fmaf(qn_r0, ab0.y, ab0.x);
-                const float cl1 = DIAG ? fmaf(cacc[1], kInv2d, ab0.x) : fmaf(qn_r1, ab0.y, ab0.x);
-                const float cl2 = DIAG ? fmaf(cacc[2], kInv2d, ab1.x) : fmaf(qn_r0, ab1.y, ab1.x);
-                const float cl3 = DIAG ? fmaf(cacc[3], kInv2d, ab1.x) : fmaf(qn_r1, ab1.y, ab1.x);
-                sl[0] = g < nvalid ? fmaf(sacc[0][0] + sacc[1][0], c_scale, kLog2e * cl0) : -INFINITY;
-                sl[1] = g < nvalid ? fmaf(sacc[0][1] + sacc[1][1], c_scale, kLog2e * cl1) : -INFINITY;
-                sl[2] = g + 8 < nvalid ? fmaf(sacc[0][2] + sacc[1][2], c_scale, kLog2e * cl2) : -INFINITY;
-                sl[3] = g + 8 < nvalid ? fmaf(sacc[0][3] + sacc[1][3], c_scale, kLog2e * cl3) : -INFINITY;
-                float mx0 = fmaxf(sl[0], sl[2]), mx1 = fmaxf(sl[1], sl[3]);
+            i0 += npg;
+            ++pi;
+
+            // ---- piece epilogue: O, m, l of rows g and g + 8 into the page-group buffer (the
+            // n8 row tiles 2 wt and 2 wt + 1 of the one-tile layout) ----
 #pragma unroll
-                for (int off = 4; off < 32; off <<= 1) {
-                    mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
-                    mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+            for (int off = 1; off < 4; off <<= 1) {
+                l_g += __shfl_xor_sync(0xffffffffu, l_g, off);
+                l_h += __shfl_xor_sync(0xffffffffu, l_h, off);
+            }
+            float *mw0 = mbuf + ((pg * NT + 2 * wt) * 8 + g) * MST;
+            float *mw1 = mbuf + ((pg * NT + 2 * wt + 1) * 8 + g) * MST;
+#pragma unroll
+            for (int j = 0; j < 2 * NKS; ++j) {
+                *reinterpret_cast<float2 *>(mw0 + 8 * j + 2 * c) = make_float2(o[j][0], o[j][1]);
+                *reinterpret_cast<float2 *>(mw1 + 8 * j + 2 * c) = make_float2(o[j][2], o[j][3]);
+            }
+            if (c == 0) {
+                mw0[D] = m_g;
+                mw0[D + 1] = l_g;
+                mw1[D] = m_h;
+                mw1[D + 1] = l_h;
+            }
+        } else {
+            // Q^T fragments of rows nt*8 + g of this piece (ldmatrix from the producer's copy), |q|^2
+            uint32_t qf[NKS][2];
+            float qn = 0.0f;
+            {
+                const int slot = pi & 1;
+                if (alive && !mbar_wait(&qfull[slot], (pi >> 1) & 1)) {
+                    if (lane == 0) raise_flag(a.flags, FLAG_TIMEOUT);
+                    alive = false;
                 }
-                const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
-                const float base0 = mn0 == -INFINITY ? 0.0f : mn0;
-                const float base1 = mn1 == -INFINITY ? 0.0f : mn1;
-                const float corr0 = ex2(m_run[0] - base0), corr1 = ex2(m_run[1] - base1);
-                const float p0 = ex2(sl[0] - base0), p1 = ex2(sl[1] - base1);
-                const float p2 = ex2(sl[2] - base0), p3 = ex2(sl[3] - base1);
-                l_run[0] = fmaf(l_run[0], corr0, p0 + p2);
-                l_run[1] = fmaf(l_run[1], corr1, p1 + p3);
-                m_run[0] = mn0;
-                m_run[1] = mn1;
-                if (!__all_sync(0xffffffffu, corr0 == 1.0f && corr1 == 1.0f)) {
-#pragma unroll
-                    for (int mt = 0; mt < NKS; ++mt) {
-                        o[mt][0] *= corr0;
-                        o[mt][1] *= corr1;
-                        o[mt][2] *= corr0;
-                        o[mt][3] *= corr1;
+                const uint32_t qb = smem_u32(qbuf + slot * L::QBUF) + (nt * 8 + (lane & 7)) * L::QROWB;
+    #pragma unroll
+                for (int k2 = 0; k2 < NKS / 2; ++k2)
+                    ldsm_x4(qb + ((4 * k2 + (lane >> 3)) << 4), qf[2 * k2][0], qf[2 * k2][1], qf[2 * k2 + 1][0],
+                            qf[2 * k2 + 1][1]);
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&qempty[slot]);
+    #pragma unroll
+                for (int ks = 0; ks < NKS; ++ks) {
+                    const uint32_t w0 = qf[ks][0], w1 = qf[ks][1];
+                    qn = fmaf(bf16lo(w0), bf16lo(w0), qn);
+                    qn = fmaf(bf16hi(w0), bf16hi(w0), qn);
+                    qn = fmaf(bf16lo(w1), bf16lo(w1), qn);
+                    qn = fmaf(bf16hi(w1), bf16hi(w1), qn);
+                }
+            }
+            // diagonal closure: q_i^2 as the B operand of Var (16 x D) (q^2)^T, split into bf16 hi + lo
+            // (q^2 of a bf16 q has at most 16 significant bits: hi + lo holds it exactly)
+            uint32_t q2h[DIAG ? NKS : 1][2], q2l[DIAG ? NKS : 1][2];
+            if constexpr (DIAG) {
+    #pragma unroll
+                for (int ks = 0; ks < NKS; ++ks)
+    #pragma unroll
+                    for (int r2 = 0; r2 < 2; ++r2) {
+                        const float lo2 = bf16lo(qf[ks][r2]), hi2 = bf16hi(qf[ks][r2]);
+                        const float slo = lo2 * lo2, shi = hi2 * hi2;
+                        const uint32_t h2 = pack_bf16x2(slo, shi);
+                        q2h[ks][r2] = h2;
+                        q2l[ks][r2] = pack_bf16x2(slo - bf16lo(h2), shi - bf16hi(h2));
+                    }
+            }
+            qn += __shfl_xor_sync(0xffffffffu, qn, 1);
+            qn += __shfl_xor_sync(0xffffffffu, qn, 2);
+            const float qn_r0 = __shfl_sync(0xffffffffu, qn, (2 * c) * 4);
+            const float qn_r1 = __shfl_sync(0xffffffffu, qn, (2 * c + 1) * 4);
+
+            float m_run[2] = {-INFINITY, -INFINITY}, l_run[2] = {0.0f, 0.0f};
+            float o[NKS][4];
+    #pragma unroll
+            for (int mt = 0; mt < NKS; ++mt) o[mt][0] = o[mt][1] = o[mt][2] = o[mt][3] = 0.0f;
+
+            // page i of the CTA's range goes to page group i % PG (global index, not piece-local)
+            for (int k = ((pg - i0 % PG) + PG) % PG; k < npg && alive; k += PG) {
+                const int i = i0 + k;
+                const int s = i % NS;
+                if (!mbar_wait(&full[s], (i / NS) & 1)) {
+                    if (lane == 0) raise_flag(a.flags, FLAG_TIMEOUT);
+                    alive = false;
+                    break;
+                }
+                const bool valid = svalid[s] != 0;
+                const int nvalid = min(kPageNodes, Lent - (lo + k) * kPageNodes);
+                // S^T accumulators: even and odd k-steps apart, so that no chain of dependent MMAs is
+                // longer than NKS / 2
+                float sacc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+                float cacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // diagonal closure: sum_i q_i^2 var_i
+                uint32_t vf[NKS][4];
+                float2 ab0 = make_float2(0.0f, 0.0f), ab1 = ab0;
+                if (valid) {
+                    const uint32_t kb = smem_u32(stages + s * G::STAGE);
+                    const uint32_t vb = kb + G::VEC_BYTES;
+                    const float2 *ab = reinterpret_cast<const float2 *>(stages + s * G::STAGE + 2 * G::VEC_BYTES);
+                    // S^T (16 nodes x 8 rows) = K (16 x D) Q^T (D x 8): every K fragment first
+                    // (independent shared loads), then the MMAs
+                    {
+                        const int mi = lane >> 3, node = (lane & 7) + 8 * (mi & 1);
+                        uint32_t kf[NKS][4];
+    #pragma unroll
+                        for (int ks = 0; ks < NKS; ++ks)
+                            ldsm_x4(kb + node * G::ROWB + (swz(2 * ks + (mi >> 1), node) << 4), kf[ks][0], kf[ks][1],
+                                    kf[ks][2], kf[ks][3]);
+    #pragma unroll
+                        for (int ks = 0; ks < NKS; ++ks)
+                            mma_bf16(sacc[ks & 1], kf[ks][0], kf[ks][1], kf[ks][2], kf[ks][3], qf[ks][0], qf[ks][1]);
+                        if constexpr (DIAG) {   // C^T (16 nodes x 8 rows) = Var (16 x D) (q^2)^T
+                            const uint32_t varb = kb + G::VAR_OFF;
+    #pragma unroll
+                            for (int ks = 0; ks < NKS; ++ks) {
+                                const int chunk = 2 * ks + (mi >> 1);
+                                uint32_t a0, a1, a2, a3;
+                                ldsm_x4(varb + node * G::ROWB + (swz(chunk, node) << 4), a0, a1, a2, a3);
+                                mma_bf16(cacc, a0, a1, a2, a3, q2h[ks][0], q2h[ks][1]);
+                                mma_bf16(cacc, a0, a1, a2, a3, q2l[ks][0], q2l[ks][1]);
+                            }
+                        }
+                    }
+                    // V^T fragments (A operand of O^T = V^T P^T) into registers now, so the stage goes
+                    // back to the producer before the softmax
+                    {
+                        const int mi = lane >> 3, node = (lane & 7) + 8 * (mi >> 1);
+    #pragma unroll
+                        for (int mt = 0; mt < NKS; ++mt)
+                            ldsm_x4_t(vb + node * G::ROWB + (swz(2 * mt + (mi & 1), node) << 4), vf[mt][0], vf[mt][1],
+                                      vf[mt][2], vf[mt][3]);
+                    }
+                    ab0 = ab[g];
+                    ab1 = ab[g + 8];
+                }
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&empty[s]);   // the page is in registers: release the stage
+                if (valid) {
+                    float sl[4];
+                    // closure: |q|^2 beta, or sum_i q_i^2 var_i / (2d) with the diagonal variances
+                    constexpr float kInv2d = 0.5f / D;
+                    const float cl0 = DIAG ? fmaf(cacc[0], kInv2d, ab0.x) : fmaf(qn_r0, ab0.y, ab0.x);
+                    const float cl1 = DIAG ? fmaf(cacc[1], kInv2d, ab0.x) : fmaf(qn_r1, ab0.y, ab0.x);
+                    const float cl2 = DIAG ? fmaf(cacc[2], kInv2d, ab1.x) : fmaf(qn_r0, ab1.y, ab1.x);
+                    const float cl3 = DIAG ? fmaf(cacc[3], kInv2d, ab1.x) : fmaf(qn_r1, ab1.y, ab1.x);
+                    sl[0] = g < nvalid ? fmaf(sacc[0][0] + sacc[1][0], c_scale, kLog2e * cl0) : -INFINITY;
+                    sl[1] = g < nvalid ? fmaf(sacc[0][1] + sacc[1][1], c_scale, kLog2e * cl1) : -INFINITY;
+                    sl[2] = g + 8 < nvalid ? fmaf(sacc[0][2] + sacc[1][2], c_scale, kLog2e * cl2) : -INFINITY;
+                    sl[3] = g + 8 < nvalid ? fmaf(sacc[0][3] + sacc[1][3], c_scale, kLog2e * cl3) : -INFINITY;
+                    float mx0 = fmaxf(sl[0], sl[2]), mx1 = fmaxf(sl[1], sl[3]);
+    #pragma unroll
+                    for (int off = 4; off < 32; off <<= 1) {
+                        mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
+                        mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
+                    }
+                    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+                    const float base0 = mn0 == -INFINITY ? 0.0f : mn0;
+                    const float base1 = mn1 == -INFINITY ? 0.0f : mn1;
+                    const float corr0 = ex2(m_run[0] - base0), corr1 = ex2(m_run[1] - base1);
+                    const float p0 = ex2(sl[0] - base0), p1 = ex2(sl[1] - base1);
+                    const float p2 = ex2(sl[2] - base0), p3 = ex2(sl[3] - base1);
+                    l_run[0] = fmaf(l_run[0], corr0, p0 + p2);
+                    l_run[1] = fmaf(l_run[1], corr1, p1 + p3);
+                    m_run[0] = mn0;
+                    m_run[1] = mn1;
+                    if (!__all_sync(0xffffffffu, corr0 == 1.0f && corr1 == 1.0f)) {
+    #pragma unroll
+                        for (int mt = 0; mt < NKS; ++mt) {
+                            o[mt][0] *= corr0;
+                            o[mt][1] *= corr1;
+                            o[mt][2] *= corr0;
+                            o[mt][3] *= corr1;
+                        }
+                    }
+                    // P^T as the B operand (16 nodes x 8 rows): transpose the 8x8 halves in registers
+                    const uint32_t bp0 = movmatrix_t(pack_bf16x2(p0, p1));
+                    const uint32_t bp1 = movmatrix_t(pack_bf16x2(p2, p3));
+                    // O^T (D x 8) += V^T (D x 16) P^T (16 x 8)
+                    if (nvalid == kPageNodes) {
+    #pragma unroll
+                        for (int mt = 0; mt < NKS; ++mt) mma_bf16(o[mt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], bp0, bp1);
+                    } else {
+                        // slots past the unit's last entry may hold anything (NaN included): zero their
+                        // V^T elements, since P = 0 does not cancel NaN in the product. This thread's
+                        // fragment holds nodes 2c, 2c+1 (a0..a3) and 2c+8, 2c+9 (a4..a7).
+                        const uint32_t m_lo =
+                            (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
+                        const uint32_t m_hi =
+                            (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
+    #pragma unroll
+                        for (int mt = 0; mt < NKS; ++mt)
+                            mma_bf16(o[mt], vf[mt][0] & m_lo, vf[mt][1] & m_lo, vf[mt][2] & m_hi, vf[mt][3] & m_hi, bp0,
+                                     bp1);
                     }
                 }
-                // P^T as the B operand (16 nodes x 8 rows): transpose the 8x8 halves in registers
-                const uint32_t bp0 = movmatrix_t(pack_bf16x2(p0, p1));
-                const uint32_t bp1 = movmatrix_t(pack_bf16x2(p2, p3));
-                // O^T (D x 8) += V^T (D x 16) P^T (16 x 8)
-                if (nvalid == kPageNodes) {
-#pragma unroll
-                    for (int mt = 0; mt < NKS; ++mt) mma_bf16(o[mt], vf[mt][0], vf[mt][1], vf[mt][2], vf[mt][3], bp0, bp1);
-                } else {
-                    // slots past the unit's last entry may hold anything (NaN included): zero their
-                    // V^T elements, since P = 0 does not cancel NaN in the product. This thread's
-                    // fragment holds nodes 2c, 2c+1 (a0..a3) and 2c+8, 2c+9 (a4..a7).
-                    const uint32_t m_lo =
-                        (2 * c < nvalid ? 0x0000ffffu : 0u) | (2 * c + 1 < nvalid ? 0xffff0000u : 0u);
-                    const uint32_t m_hi =
-                        (2 * c + 8 < nvalid ? 0x0000ffffu : 0u) | (2 * c + 9 < nvalid ? 0xffff0000u : 0u);
-#pragma unroll
-                    for (int mt = 0; mt < NKS; ++mt)
-                        mma_bf16(o[mt], vf[mt][0] & m_lo, vf[mt][1] & m_lo, vf[mt][2] & m_hi, vf[mt][3] & m_hi, bp0,
-                                 bp1);
-                }
             }
-        }
-        i0 += npg;
-        ++pi;
+            i0 += npg;
+            ++pi;
 
-        // ---- piece epilogue: merge the page groups through shared memory ----
-#pragma unroll
-        for (int off = 4; off < 32; off <<= 1) {
-            l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
-            l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
-        }
-        constexpr int MST = L::MST, WST = L::WST;
-        float *mw = mbuf + warp * 8 * MST;
-#pragma unroll
-        for (int mt = 0; mt < NKS; ++mt) {
-            mw[(2 * c) * MST + 16 * mt + g] = o[mt][0];
-            mw[(2 * c + 1) * MST + 16 * mt + g] = o[mt][1];
-            mw[(2 * c) * MST + 16 * mt + g + 8] = o[mt][2];
-            mw[(2 * c + 1) * MST + 16 * mt + g + 8] = o[mt][3];
-        }
-        if (g == 0) {
-            mw[(2 * c) * MST + D] = m_run[0];
-            mw[(2 * c) * MST + D + 1] = l_run[0];
-            mw[(2 * c + 1) * MST + D] = m_run[1];
-            mw[(2 * c + 1) * MST + D + 1] = l_run[1];
+            // ---- piece epilogue: merge the page groups through shared memory ----
+    #pragma unroll
+            for (int off = 4; off < 32; off <<= 1) {
+                l_run[0] += __shfl_xor_sync(0xffffffffu, l_run[0], off);
+                l_run[1] += __shfl_xor_sync(0xffffffffu, l_run[1], off);
+            }
+            float *mw = mbuf + warp * 8 * MST;
+    #pragma unroll
+            for (int mt = 0; mt < NKS; ++mt) {
+                mw[(2 * c) * MST + 16 * mt + g] = o[mt][0];
+                mw[(2 * c + 1) * MST + 16 * mt + g] = o[mt][1];
+                mw[(2 * c) * MST + 16 * mt + g + 8] = o[mt][2];
+                mw[(2 * c + 1) * MST + 16 * mt + g + 8] = o[mt][3];
+            }
+            if (g == 0) {
+                mw[(2 * c) * MST + D] = m_run[0];
+                mw[(2 * c) * MST + D + 1] = l_run[0];
+                mw[(2 * c + 1) * MST + D] = m_run[1];
+                mw[(2 * c + 1) * MST + D + 1] = l_run[1];
+            }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
         const bool complete = (ps >= ra) && (pe <= rb);
