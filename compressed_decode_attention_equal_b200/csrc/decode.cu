@@ -357,10 +357,12 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     // While the preceding grid may still run, warm L2 with the guessed range's first pages: the
     // page ids read here may be stale (the preceding grid may write the table), so they feed only
     // L2 prefetches -- a stale id costs a wasted read, never a wrong result -- and are read again
-    // after the wait below. Ids outside the pool are not touched.
+    // after the wait below (this read is L2-only, so it leaves no stale line in L1). Ids outside
+    // the pool are not touched. (Issuing the first copies with these ids and checking them against
+    // the second read made the consumers wait for that read: measured slower.)
     if (warp == NCONS && try_spec && lane < n_first) {
         const long long u = vc / a.row_passes;
-        const int phys = ld_global_s32(a.page_table + u * a.max_pages + c0 + lane);
+        const int phys = ld_global_cg_s32(a.page_table + u * a.max_pages + c0 + lane);
         if (phys >= 0 && phys < a.num_pages)
             bulk_prefetch_l2(a.pages + static_cast<long long>(phys) * G::STAGE, G::STAGE);
     }

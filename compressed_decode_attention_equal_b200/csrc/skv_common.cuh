@@ -229,6 +229,14 @@ __device__ __forceinline__ int ld_global_s32(const int32_t *p) {
     return v;
 }
 
+// The same, cached in L2 only: for data another grid may still be writing (no stale copy is left
+// in this SM's L1 for a later read).
+__device__ __forceinline__ int ld_global_cg_s32(const int32_t *p) {
+    int v;
+    asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p));
+    return v;
+}
+
 __device__ __forceinline__ void st_dsmem(uint32_t addr, float v) {
     asm volatile("st.shared::cluster.f32 [%0], %1;" ::"r"(addr), "f"(v) : "memory");
 }
