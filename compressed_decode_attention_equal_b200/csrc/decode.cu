@@ -92,8 +92,7 @@ struct SplitSmem {
                                     16 * 4 + ((EPI_BYTES + 15) / 16) * 16;
 };
 
-__device__ __forceinline__ int clamp_entries(const DecodeArgs &a, int u) {
-    int L = a.lens[u];
+__device__ __forceinline__ int clamp_len(const DecodeArgs &a, int L) {
     const int cap = a.max_pages * kPageNodes;
     if (L > cap) {
         raise_flag(a.flags, FLAG_BAD_LENS);
@@ -101,6 +100,8 @@ __device__ __forceinline__ int clamp_entries(const DecodeArgs &a, int u) {
     }
     return L < 0 ? 0 : L;
 }
+
+__device__ __forceinline__ int clamp_entries(const DecodeArgs &a, int u) { return clamp_len(a, a.lens[u]); }
 
 // largest v with prefix[v] <= f
 __device__ __forceinline__ int find_vunit(const int *prefix, int nv, long long f) {
@@ -113,19 +114,29 @@ __device__ __forceinline__ int find_vunit(const int *prefix, int nv, long long f
     return lo;
 }
 
-// Every CTA rebuilds the page prefix over virtual units (lens are tiny and L2-resident). Run by
-// the consumer warps alone (named barrier 1), so the producer can start copies meanwhile.
+// Every CTA rebuilds the page prefix over virtual units (lens are tiny and L2-resident), and keeps
+// every virtual unit's (clamped) entry count in shared memory for the pieces. Run by the consumer
+// warps alone (named barrier 1), so the producer can start copies meanwhile.
 template <int NCONS>
-__device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, int *scratch) {
+__device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, int *ents, int *scratch) {
     const int nv = a.n_vunits;
     const int tid = threadIdx.x, nth = NCONS * 32;
     const int per = (nv + nth - 1) / nth;
     const int lo = min(tid * per, nv), hi = min(lo + per, nv);
     int local = 0;
-    for (int v = lo; v < hi; ++v) {
-        const int pages = (clamp_entries(a, v / a.row_passes) + kPageNodes - 1) / kPageNodes;
-        prefix[v] = pages;   // page count for now; made exclusive below
-        local += pages;
+    for (int v = lo; v < hi; v += 4) {
+        int raw[4];   // four loads in flight before any is used
+#pragma unroll
+        for (int j = 0; j < 4; ++j) raw[j] = v + j < hi ? a.lens[(v + j) / a.row_passes] : 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (v + j < hi) {
+                const int L = clamp_len(a, raw[j]);
+                const int pages = (L + kPageNodes - 1) / kPageNodes;
+                ents[v + j] = L;
+                prefix[v + j] = pages;   // page count for now; made exclusive below
+                local += pages;
+            }
     }
     const int lane = tid & 31, warp = tid >> 5;
     int x = local;
@@ -173,13 +184,21 @@ __device__ __forceinline__ int piece_code(int i, long long ps, long long ptot, i
 // pieces, every load of two rows is issued before any is used (one round trip to L2).
 constexpr int kFastPieces = 6;
 
+// What the merge of a split unit reads and writes
+struct MergeArgs {
+    const float *part_l, *part_v;
+    void *out;
+    float *lse;
+    int row_passes, Hkv, pass_rows, rows, R, Hq, G;
+};
+
 template <int D>
-__device__ __forceinline__ void merge_store(const DecodeArgs &a, int b, int h, int row, int lane, const float *acc,
+__device__ __forceinline__ void merge_store(const MergeArgs &m, int b, int h, int row, int lane, const float *acc,
                                             float M, float Ls) {
     constexpr int DPL = D / 32;
-    const long long oi = (static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G;
+    const long long oi = (static_cast<long long>(b) * m.R + row / m.G) * m.Hq + h * m.G + row % m.G;
     const float inv = Ls > 0.0f ? 1.0f / Ls : 0.0f;
-    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(a.out) + oi * D + lane * DPL;
+    __nv_bfloat16 *dst = static_cast<__nv_bfloat16 *>(m.out) + oi * D + lane * DPL;
     if constexpr (DPL == 4) {
         uint2 w;
         w.x = pack_bf16x2(acc[0] * inv, acc[1] * inv);
@@ -188,15 +207,59 @@ __device__ __forceinline__ void merge_store(const DecodeArgs &a, int b, int h, i
     } else {
         *reinterpret_cast<uint32_t *>(dst) = pack_bf16x2(acc[0] * inv, acc[1] * inv);
     }
-    if (lane == 0) a.lse[oi] = Ls > 0.0f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
+    if (lane == 0) m.lse[oi] = Ls > 0.0f ? (M + __log2f(Ls)) * kLn2 : -INFINITY;
 }
 
 template <int D, int NCONS>
-__device__ void merge_unit(const DecodeArgs &a, int v, const int *codes, int n, int warp, int lane) {
+__device__ void merge_unit(const MergeArgs m, int v, const int *codes, int n, int warp, int lane) {
     constexpr int DPL = D / 32;   // dimensions per lane
-    const int u = v / a.row_passes, rpass = v % a.row_passes;
-    const int b = u / a.Hkv, h = u % a.Hkv;
-    const int rows_here = min(a.pass_rows, a.rows - rpass * kRowsPerPass);
+    const int u = v / m.row_passes, rpass = v % m.row_passes;
+    const int b = u / m.Hkv, h = u % m.Hkv;
+    const int rows_here = min(m.pass_rows, m.rows - rpass * kRowsPerPass);
+    if (n <= 2) {
+        // the common split: two pieces. Rows in groups of four per warp (two with eight warps),
+        // every load of a group issued before any is used: one round trip to L2 per group.
+        constexpr int RPW = kRowsPerPass / NCONS, CH = NCONS >= 8 ? 2 : (RPW < 4 ? RPW : 4);
+#pragma unroll 1
+        for (int t0 = 0; t0 < RPW && warp + t0 * NCONS < rows_here; t0 += CH) {
+            float lv[CH][2], xv[CH][2][DPL];
+#pragma unroll
+            for (int t = 0; t < CH; ++t) {
+                const int rr = warp + (t0 + t) * NCONS;
+#pragma unroll
+                for (int i = 0; i < 2; ++i) {
+                    lv[t][i] = -INFINITY;
+#pragma unroll
+                    for (int j = 0; j < DPL; ++j) xv[t][i][j] = 0.0f;
+                    if (i < n && rr < rows_here) {
+                        const long long pr = static_cast<long long>(codes[i]) * m.pass_rows + rr;
+                        lv[t][i] = __ldcg(m.part_l + pr);
+                        const float *src = m.part_v + pr * D + lane * DPL;
+                        if constexpr (DPL == 4) {
+                            const float4 x = __ldcg(reinterpret_cast<const float4 *>(src));
+                            xv[t][i][0] = x.x; xv[t][i][1] = x.y; xv[t][i][2] = x.z; xv[t][i][3] = x.w;
+                        } else {
+                            const float2 x = __ldcg(reinterpret_cast<const float2 *>(src));
+                            xv[t][i][0] = x.x; xv[t][i][1] = x.y;
+                        }
+                    }
+                }
+            }
+#pragma unroll
+            for (int t = 0; t < CH; ++t) {
+                const int rr = warp + (t0 + t) * NCONS;
+                if (rr >= rows_here) continue;
+                const float M = fmaxf(lv[t][0], lv[t][1]);
+                const float Mb = M == -INFINITY ? 0.0f : M;
+                const float w0 = ex2(lv[t][0] - Mb), w1 = ex2(lv[t][1] - Mb);   // -inf (absent piece): 0
+                float acc[DPL];
+#pragma unroll
+                for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w1, xv[t][1][j], w0 * xv[t][0][j]);
+                merge_store<D>(m, b, h, rpass * kRowsPerPass + rr, lane, acc, M, w0 + w1);
+            }
+        }
+        return;
+    }
     if (n <= kFastPieces) {
         for (int r0 = warp; r0 < rows_here; r0 += 2 * NCONS) {
             float lv[2][kFastPieces], xv[2][kFastPieces][DPL];
@@ -209,9 +272,9 @@ __device__ void merge_unit(const DecodeArgs &a, int v, const int *codes, int n, 
 #pragma unroll
                     for (int j = 0; j < DPL; ++j) xv[t][i][j] = 0.0f;
                     if (i < n && rr < rows_here) {
-                        const long long pr = static_cast<long long>(codes[i]) * a.pass_rows + rr;
-                        lv[t][i] = __ldcg(a.part_l + pr);
-                        const float *src = a.part_v + pr * D + lane * DPL;
+                        const long long pr = static_cast<long long>(codes[i]) * m.pass_rows + rr;
+                        lv[t][i] = __ldcg(m.part_l + pr);
+                        const float *src = m.part_v + pr * D + lane * DPL;
                         if constexpr (DPL == 4) {
                             const float4 x = __ldcg(reinterpret_cast<const float4 *>(src));
                             xv[t][i][0] = x.x; xv[t][i][1] = x.y; xv[t][i][2] = x.z; xv[t][i][3] = x.w;
@@ -240,7 +303,7 @@ __device__ void merge_unit(const DecodeArgs &a, int v, const int *codes, int n, 
 #pragma unroll
                     for (int j = 0; j < DPL; ++j) acc[j] = fmaf(w, xv[t][i][j], acc[j]);
                 }
-                merge_store<D>(a, b, h, rpass * kRowsPerPass + rr, lane, acc, M, Ls);
+                merge_store<D>(m, b, h, rpass * kRowsPerPass + rr, lane, acc, M, Ls);
             }
         }
         return;
@@ -249,7 +312,7 @@ __device__ void merge_unit(const DecodeArgs &a, int v, const int *codes, int n, 
         float M = -INFINITY;
         for (int base = 0; base < n; base += 32) {
             const int i = base + lane;
-            M = fmaxf(M, i < n ? __ldcg(a.part_l + static_cast<long long>(codes[i]) * a.pass_rows + rr) : -INFINITY);
+            M = fmaxf(M, i < n ? __ldcg(m.part_l + static_cast<long long>(codes[i]) * m.pass_rows + rr) : -INFINITY);
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
@@ -260,14 +323,14 @@ __device__ void merge_unit(const DecodeArgs &a, int v, const int *codes, int n, 
         for (int base = 0; base < n; base += 32) {
             const int i = base + lane;
             const float wi =
-                i < n ? ex2(__ldcg(a.part_l + static_cast<long long>(codes[i]) * a.pass_rows + rr) - Mb) : 0.0f;
+                i < n ? ex2(__ldcg(m.part_l + static_cast<long long>(codes[i]) * m.pass_rows + rr) - Mb) : 0.0f;
             Ls += wi;
             const int cnt = min(32, n - base);
 #pragma unroll 4
             for (int k = 0; k < cnt; ++k) {
                 const float w = __shfl_sync(0xffffffffu, wi, k);
                 const float *src =
-                    a.part_v + (static_cast<long long>(codes[base + k]) * a.pass_rows + rr) * D + lane * DPL;
+                    m.part_v + (static_cast<long long>(codes[base + k]) * m.pass_rows + rr) * D + lane * DPL;
                 if constexpr (DPL == 4) {
                     const float4 x = __ldcg(reinterpret_cast<const float4 *>(src));
                     acc[0] = fmaf(w, x.x, acc[0]);
@@ -283,7 +346,7 @@ __device__ void merge_unit(const DecodeArgs &a, int v, const int *codes, int n, 
         }
 #pragma unroll
         for (int off = 16; off > 0; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
-        merge_store<D>(a, b, h, rpass * kRowsPerPass + rr, lane, acc, M, Ls);
+        merge_store<D>(m, b, h, rpass * kRowsPerPass + rr, lane, acc, M, Ls);
     }
 }
 
@@ -321,7 +384,8 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     const int nv = a.n_vunits;
     // aligned split: rank r > 0 of a cluster stores its piece into rank 0's receive buffer
     // (cluster - 1 blocks of pass_rows x (D + 1) floats behind the page prefix)
-    float *xbuf = reinterpret_cast<float *>(prefix + ((nv + 1 + 3) & ~3));   // 16-byte aligned
+    int *ents = prefix + ((nv + 1 + 3) & ~3);   // entries of every virtual unit
+    float *xbuf = reinterpret_cast<float *>(ents + ((nv + 3) & ~3));   // 16-byte aligned
     cluster_arrive_relaxed();   // this CTA has started (waited on before any remote access)
     if (tid == 0) {   // independent of the inputs: overlaps the wait below
         for (int s = 0; s < NS; ++s) {
@@ -395,8 +459,10 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                     } else {
                         svalid[k] = 1;
                         mbar_arrive_expect_tx(&full[k], G::STAGE);
-                        bulk_g2s(stages + k * G::STAGE, a.pages + static_cast<long long>(phys) * G::STAGE, G::STAGE,
-                                 &full[k]);
+                        // pages are read once per call: evict-first, so that they do not push the
+                        // small inputs (tables, lengths, queries) out of L2
+                        bulk_g2s_hint(stages + k * G::STAGE, a.pages + static_cast<long long>(phys) * G::STAGE,
+                                      G::STAGE, &full[k], createpolicy_evict_first());
                     }
                 }
                 __syncwarp();
@@ -405,7 +471,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
         cluster_wait();   // pairs with the arrival above (the producer touches no remote memory)
         asm volatile("bar.sync 2, %0;" ::"n"(NTHR));   // the consumers' verdict and prefix
     } else {
-        build_prefix<NCONS>(a, prefix, scan_scratch);
+        build_prefix<NCONS>(a, prefix, ents, scan_scratch);
         // Aligned split: when every unit has the same page count P0 and `cluster` CTAs per unit
         // fit in the grid, the k = cluster CTAs of a thread-block cluster take equal page ranges of
         // one unit and merge through distributed shared memory (no global partials, one piece per
@@ -496,6 +562,24 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
         int v = spec_ok ? vc : -1, pi = spec_ok ? 0 : -1;   // current (nonempty) piece
         const int i_first = spec_ok ? n_first : 0;
         if (spec_ok && spec_bad != 0 && lane == 0) raise_flag(a.flags, FLAG_BAD_PAGE);
+        // the query rows of piece vq into slot `slot` of the double buffer
+        auto copy_q = [&](int vq, int slot) {
+            const int u = vq / a.row_passes, rpass = vq % a.row_passes;
+            const int b = u / a.Hkv, h = u % a.Hkv;
+            const int p0 = rpass * kRowsPerPass, p1 = min(p0 + a.pass_rows, a.rows);
+            if (lane == 0) mbar_arrive_expect_tx(&qfull[slot], (p1 - p0) * D * 2);
+            __syncwarp();
+            for (int row = p0 + lane; row < p1; row += 32) {
+                const __nv_bfloat16 *src =
+                    q + ((static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G) * D;
+                bulk_g2s(qbuf + slot * L::QBUF + (row - p0) * L::QROWB, src, D * 2, &qfull[slot]);
+            }
+        };
+        if (!spec_ok && alive) {   // the first piece's query rows need no page id: copy them first
+            v = v0;
+            pi = 0;
+            copy_q(v, 0);
+        }
         for (int base = 0; base < n_my && alive; base += 32) {
             int my_page = -1;
             if (base == 0 && spec_ok) {
@@ -519,16 +603,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                         alive = false;
                         break;
                     }
-                    const int u = v / a.row_passes, rpass = v % a.row_passes;
-                    const int b = u / a.Hkv, h = u % a.Hkv;
-                    const int p0 = rpass * kRowsPerPass, p1 = min(p0 + a.pass_rows, a.rows);
-                    if (lane == 0) mbar_arrive_expect_tx(&qfull[slot], (p1 - p0) * D * 2);
-                    __syncwarp();
-                    for (int row = p0 + lane; row < p1; row += 32) {
-                        const __nv_bfloat16 *src =
-                            q + ((static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G) * D;
-                        bulk_g2s(qbuf + slot * L::QBUF + (row - p0) * L::QROWB, src, D * 2, &qfull[slot]);
-                    }
+                    copy_q(v, slot);
                 }
                 const int s = i % NS;
                 const int phys = __shfl_sync(0xffffffffu, my_page, k);
@@ -546,8 +621,8 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                         svalid[s] = 1;
                         mbar_arrive_expect_tx(&full[s], G::STAGE);
                         // a page is one contiguous [keys | values | alpha,beta] block: one copy
-                        bulk_g2s(stages + s * G::STAGE, a.pages + static_cast<long long>(phys) * G::STAGE, G::STAGE,
-                                 &full[s]);
+                        bulk_g2s_hint(stages + s * G::STAGE, a.pages + static_cast<long long>(phys) * G::STAGE,
+                                      G::STAGE, &full[s], createpolicy_evict_first());
                     }
                 }
                 __syncwarp();
@@ -575,7 +650,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
         if (npg <= 0) continue;   // an empty unit: written in the prologue
         const int u = v / a.row_passes, rpass = v % a.row_passes;
         const int b = u / a.Hkv, h = u % a.Hkv;
-        const int Lent = clamp_entries(a, u);
+        const int Lent = ents[v];
         const int rows_here = min(a.pass_rows, a.rows - rpass * kRowsPerPass);
         if (ctid < rows_here) {   // output row of each query row (read after the page loop)
             const int row = rpass * kRowsPerPass + ctid;
@@ -1093,7 +1168,9 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
         for (int i = ctid; i < n; i += NCONS * 32) codes[i] = piece_code(i, ps, ptot, a.ncta, c_first);
         __threadfence();   // acquire: the other pieces' partials are visible after their counts
         asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
-        merge_unit<D, NCONS>(a, v, codes, n, warp, lane);
+        merge_unit<D, NCONS>(MergeArgs{a.part_l, a.part_v, a.out, a.lse, a.row_passes, a.Hkv, a.pass_rows, a.rows, a.R,
+                                       a.Hq, a.G},
+                             v, codes, n, warp, lane);
         if (ctid == 0) a.counters[v] = 0;   // ready for the next call
         asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
     }
@@ -1183,6 +1260,7 @@ __global__ void __launch_bounds__(128) k_decode_f32(const DecodeArgs a) {
 template <int D, int NT, bool DIAG>
 static size_t split_smem(int n_vunits, int cluster) {
     return SplitSmem<D, NT, DIAG>::FIXED + static_cast<size_t>((n_vunits + 1 + 3) & ~3) * 4 +
+           static_cast<size_t>((n_vunits + 3) & ~3) * 4 +   // entries per virtual unit
            static_cast<size_t>(cluster - 1) * (NT * 8) * (D + 1) * 4;   // aligned-split receive buffer
 }
 
