@@ -88,7 +88,7 @@ struct SplitSmem {
     static constexpr int SVALID_INTS = (STAGES + 3) & ~3;   // padded: mbuf (read as float4) stays 16-byte aligned
     static constexpr int MBUF_OFF = STAGES_BYTES + 2 * QBUF + BARS * 8 + SVALID_INTS * 4;
     static_assert(MBUF_OFF % 16 == 0 && (MBUF_FLOATS * 4) % 16 == 0, "16-byte aligned epilogue buffers");
-    static constexpr size_t FIXED = 16 + STAGES_BYTES + 2 * QBUF + BARS * 8 + SVALID_INTS * 4 + MBUF_FLOATS * 4 +
+    static constexpr size_t FIXED = 128 + STAGES_BYTES + 2 * QBUF + BARS * 8 + SVALID_INTS * 4 + MBUF_FLOATS * 4 +
                                     16 * 4 + ((EPI_BYTES + 15) / 16) * 16;
 };
 
@@ -114,9 +114,15 @@ __device__ __forceinline__ int find_vunit(const int *prefix, int nv, long long f
     return lo;
 }
 
-// Every CTA rebuilds the page prefix over virtual units (lens are tiny and L2-resident), and keeps
-// every virtual unit's (clamped) entry count in shared memory for the pieces. Run by the consumer
-// warps alone (named barrier 1), so the producer can start copies meanwhile.
+// Work of one piece besides its pages, in pages: the stream-K split balances pages plus this much
+// per unit, since each piece costs its CTA a query-row load and an epilogue (the page-group merge
+// and the output or partial stores) on top of its pages -- measured about five pages' worth with
+// 28 query rows per unit, so a split by pages alone left the CTAs holding many short units last.
+constexpr int kPieceWork = 4;
+
+// Every CTA rebuilds the page prefix over virtual units (flat index of each unit's first page) and
+// keeps every unit's clamped entry count, both in shared memory (lens are tiny and L2-resident).
+// Run by the consumer warps alone (named barrier 1), so the producer can start copies meanwhile.
 template <int NCONS>
 __device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, int *ents, int *scratch) {
     const int nv = a.n_vunits;
@@ -159,16 +165,58 @@ __device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, i
     asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
 }
 
-// First flat page of CTA c's range, and the CTA whose (nonempty) range holds page f.
-__device__ __forceinline__ long long cta_begin(long long c, long long ptot, int ncta) { return ptot * c / ncta; }
+// The work prefix of the stream-K split (built only when the grid splits that way): a unit's work
+// is its pages plus kPieceWork if it has any, wpre[v] = prefix[v] + kPieceWork * (nonempty units
+// before v). Consumer warps alone, after build_prefix.
+template <int NCONS>
+__device__ __forceinline__ void build_work(const DecodeArgs &a, const int *prefix, int *wpre, int *scratch) {
+    const int nv = a.n_vunits;
+    const int tid = threadIdx.x, nth = NCONS * 32;
+    const int per = (nv + nth - 1) / nth;
+    const int lo = min(tid * per, nv), hi = min(lo + per, nv);
+    int local = 0;
+    for (int v = lo; v < hi; ++v) local += prefix[v + 1] > prefix[v] ? 1 : 0;
+    const int lane = tid & 31, warp = tid >> 5;
+    int x = local;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, x, off);
+        if (lane >= off) x += n;
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));   // scratch free (build_prefix read it)
+    if (lane == 31) scratch[warp] = x;
+    asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
+    int wp = 0;
+    for (int w = 0; w < warp; ++w) wp += scratch[w];
+    int run = wp + x - local;
+    for (int v = lo; v < hi; ++v) {
+        wpre[v] = prefix[v] + kPieceWork * run;
+        run += prefix[v + 1] > prefix[v] ? 1 : 0;
+    }
+    if (tid == nth - 1) wpre[nv] = prefix[nv] + kPieceWork * (wp + x);
+    asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
+}
+
+// Flat page index at work position w: the pages of the units before w's unit, plus those of w's
+// unit that lie before w (a unit's pages follow its kPieceWork in the work order).
+__device__ __forceinline__ long long flat_of_work(const int *wpre, const int *prefix, int nv, long long w) {
+    if (w >= wpre[nv]) return prefix[nv];
+    const int v = find_vunit(wpre, nv, w);
+    const long long pages = prefix[v + 1] - prefix[v];
+    const long long into = w - (wpre[v + 1] - pages);
+    return prefix[v] + (into < 0 ? 0 : (into > pages ? pages : into));
+}
+
+// The CTA whose (nonempty) range holds work position f.
 __device__ __forceinline__ long long cta_of(long long f, long long ptot, int ncta) {
     return ((f + 1) * ncta + ptot - 1) / ptot - 1;
 }
 
-// Pieces of the unit covering flat pages [ps, pe): their count, and the partial-slot code
-// (cta * 2 + slot) of piece i. With ptot >= ncta every CTA range is nonempty: the pieces sit in
-// CTAs c_first..c_last, the first in its tail slot (1), the others in their head slot (0). With
-// ptot < ncta every nonempty range holds exactly one page: piece i is page ps + i's CTA.
+// Pieces of the unit whose pages lie at work positions [ps, pe): their count, and the partial-slot
+// code (cta * 2 + slot) of piece i. With ptot >= ncta every CTA range is nonempty: the pieces sit
+// in CTAs c_first..c_last, the first in its tail slot (1), the others in their head slot (0). With
+// ptot < ncta every nonempty range holds exactly one work position: piece i is position ps + i's
+// CTA.
 __device__ __forceinline__ int piece_count(long long ps, long long pe, long long ptot, int ncta) {
     if (ptot < ncta) return static_cast<int>(pe - ps);
     return static_cast<int>(cta_of(pe - 1, ptot, ncta) - cta_of(ps, ptot, ncta) + 1);
@@ -364,7 +412,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     static_assert(NS % PG == 0, "a stage's successive pages must go to one consumer warp");
 
     extern __shared__ uint8_t smem_raw[];
-    uint8_t *smem = smem_raw + ((16 - (smem_u32(smem_raw) & 15)) & 15);
+    uint8_t *smem = smem_raw + ((128 - (smem_u32(smem_raw) & 127)) & 127);   // 128-byte aligned (measured faster)
     uint8_t *stages = smem;
     uint8_t *qbuf = stages + L::STAGES_BYTES;
     uint64_t *full = reinterpret_cast<uint64_t *>(qbuf + 2 * L::QBUF);
@@ -386,6 +434,9 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     // (cluster - 1 blocks of pass_rows x (D + 1) floats behind the page prefix)
     int *ents = prefix + ((nv + 1 + 3) & ~3);   // entries of every virtual unit
     float *xbuf = reinterpret_cast<float *>(ents + ((nv + 3) & ~3));   // 16-byte aligned
+    // the stream-K split's work prefix shares the receive buffer's storage (used only by the
+    // aligned split)
+    int *wpre = reinterpret_cast<int *>(xbuf);
     cluster_arrive_relaxed();   // this CTA has started (waited on before any remote access)
     if (tid == 0) {   // independent of the inputs: overlaps the wait below
         for (int s = 0; s < NS; ++s) {
@@ -484,12 +535,13 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                 uni &= (prefix[v + 1] - prefix[v] == P0);
         }
         uni = bar_and(1, NCONS * 32, uni);
+        const bool al = uni && (kcl > 1 || 4LL * nv >= 3LL * a.ncta) && P0 >= kcl &&
+                        static_cast<long long>(nv) * kcl <= a.ncta;
         if (tid == 0) {
-            const bool al = uni && (kcl > 1 || 4LL * nv >= 3LL * a.ncta) && P0 >= kcl &&
-                            static_cast<long long>(nv) * kcl <= a.ncta;
             misc[8] = al ? 1 : 0;
             misc[9] = (al && try_spec && P0 == a.max_pages) ? 1 : 0;
         }
+        if (!al) build_work<NCONS>(a, prefix, wpre, scan_scratch);
         cluster_wait();   // every CTA of the cluster has started
         asm volatile("bar.arrive 2, %0;" ::"n"(NTHR));
         asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));   // misc visible to every consumer
@@ -525,15 +577,15 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
         }
         __syncthreads();
     }
-    const long long ptot = prefix[nv];
+    const long long ptot = aligned ? 0 : wpre[nv];   // total work of the stream-K split
     const int P0 = prefix[1] - prefix[0];
-    long long ra, rb;
+    long long pa, pb;   // this CTA's flat pages
     if (aligned) {
-        ra = vc < nv ? prefix[vc] + P0 * crank / kcl : 0;
-        rb = vc < nv ? prefix[vc] + P0 * (crank + 1) / kcl : 0;
+        pa = vc < nv ? prefix[vc] + P0 * crank / kcl : 0;
+        pb = vc < nv ? prefix[vc] + P0 * (crank + 1) / kcl : 0;
     } else {
-        ra = ptot * blockIdx.x / a.ncta;
-        rb = ptot * (blockIdx.x + 1) / a.ncta;
+        pa = flat_of_work(wpre, prefix, nv, ptot * blockIdx.x / a.ncta);
+        pb = flat_of_work(wpre, prefix, nv, ptot * (blockIdx.x + 1) / a.ncta);
     }
     __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(a.out);
     if (warp < NCONS) {
@@ -552,9 +604,9 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
             }
         }
     }
-    if (ra >= rb) return;
-    const int v0 = aligned ? vc : find_vunit(prefix, nv, ra);
-    const int n_my = static_cast<int>(rb - ra);
+    if (pa >= pb) return;
+    const int v0 = aligned ? vc : find_vunit(prefix, nv, pa);
+    const int n_my = static_cast<int>(pb - pa);
 
     if (warp == NCONS) {
         // ----------------------------- producer -----------------------------
@@ -585,14 +637,14 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
             if (base == 0 && spec_ok) {
                 my_page = spec_page;   // the same columns, read before the lens were known
             } else if (base + lane < n_my) {
-                const long long f = ra + base + lane;
+                const long long f = pa + base + lane;
                 const int vv = find_vunit(prefix, nv, f);
                 my_page = a.page_table[static_cast<long long>(vv / a.row_passes) * a.max_pages + (f - prefix[vv])];
             }
             const int cnt = min(32, n_my - base);
             for (int k = base < i_first ? i_first - base : 0; k < cnt; ++k) {
                 const int i = base + k;
-                const long long f = ra + i;
+                const long long f = pa + i;
                 if (v < 0 || f >= prefix[v + 1]) {
                     // first page of the next piece: copy its query rows first
                     v = find_vunit(prefix, nv, f);
@@ -643,9 +695,9 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     constexpr int MST = L::MST, WST = L::WST;
     int i0 = 0, pi = 0;
     int split_v[2] = {0, 0}, split_ps[2] = {0, 0}, split_pe[2] = {0, 0}, n_split = 0;   // (thread 0)
-    for (int v = v0; v < nv && prefix[v] < rb; ++v) {
-        const long long ps = prefix[v], pe = prefix[v + 1];
-        const int lo = static_cast<int>(max(ra, ps) - ps), hi = static_cast<int>(min(rb, pe) - ps);
+    for (int v = v0; v < nv && prefix[v] < pb; ++v) {
+        const long long ps = prefix[v], pe = prefix[v + 1];   // the unit's flat pages
+        const int lo = static_cast<int>(max(pa, ps) - ps), hi = static_cast<int>(min(pb, pe) - ps);
         const int npg = hi - lo;
         if (npg <= 0) continue;   // an empty unit: written in the prologue
         const int u = v / a.row_passes, rpass = v % a.row_passes;
@@ -1024,8 +1076,8 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
             }
         }
         asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
-        const bool complete = (ps >= ra) && (pe <= rb);
-        const int slot = ps < ra ? 0 : 1;
+        const bool complete = (ps >= pa) && (pe <= pb);
+        const int slot = ps < pa ? 0 : 1;
         // per query row: normalised page-group weights, log2 partition and output row
         if (ctid < rows_here) {
             const int rr = ctid, ntr = rr >> 3, j = rr & 7;
@@ -1085,8 +1137,9 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
         }
         if (!complete && !aligned && ctid == 0 && n_split < 2) {
             split_v[n_split] = v;
-            split_ps[n_split] = static_cast<int>(ps);
-            split_pe[n_split] = static_cast<int>(pe);
+            // the unit's pages in work positions (the split's coordinates)
+            split_ps[n_split] = wpre[v + 1] - static_cast<int>(pe - ps);
+            split_pe[n_split] = wpre[v + 1];
             ++n_split;
         }
         asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));   // mbuf free for the next piece
@@ -1259,9 +1312,11 @@ __global__ void __launch_bounds__(128) k_decode_f32(const DecodeArgs a) {
 // ---------------------------------------------------------------------------
 template <int D, int NT, bool DIAG>
 static size_t split_smem(int n_vunits, int cluster) {
+    const size_t recv = static_cast<size_t>(cluster - 1) * (NT * 8) * (D + 1) * 4;   // aligned-split receive buffer
+    const size_t work = static_cast<size_t>(n_vunits + 1) * 4;                       // or the work prefix
     return SplitSmem<D, NT, DIAG>::FIXED + static_cast<size_t>((n_vunits + 1 + 3) & ~3) * 4 +
            static_cast<size_t>((n_vunits + 3) & ~3) * 4 +   // entries per virtual unit
-           static_cast<size_t>(cluster - 1) * (NT * 8) * (D + 1) * 4;   // aligned-split receive buffer
+           (recv > work ? recv : work);
 }
 
 constexpr int kMaxCluster = 8;   // portable cluster size limit
