@@ -45,6 +45,13 @@ constexpr int kDecConsumers = 4;
 // phase's parity as complete (mbarrier parity aliasing) and read stale data.
 constexpr int kDecStages = 8;
 constexpr float kLog2e = 1.4426950408889634f;
+// Lazy maximum of the online softmax: a row's reference maximum moves only when a page's maximum
+// exceeds it by more than this (log2 units). Until then the page's exponents are taken against the
+// stale reference, so they are at most 2^8 -- exact in fp32 and of unchanged relative precision in
+// bf16 -- and O, l and the reference stay consistent (the final normalisation and log-partition use
+// them together). The rescale of O, 64 multiplies per page, then runs rarely instead of on most
+// pages.
+constexpr float kLazyMax = 8.0f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 // DIAG: the page also carries per-dimension key variances (the diagonal closure) after alpha/beta
@@ -112,6 +119,30 @@ __device__ __forceinline__ int find_vunit(const int *prefix, int nv, long long f
         else hi = mid;
     }
     return lo;
+}
+
+// The same search by a whole warp (every lane gets the answer): each round tests 32 evenly spaced
+// entries at once, so nv = 8192 takes three rounds of shared loads instead of thirteen dependent ones.
+__device__ __forceinline__ int find_vunit_warp(const int *prefix, int nv, long long f, int lane) {
+    int lo = 0, hi = nv;   // prefix[lo] <= f < prefix[hi]
+    while (hi - lo > 32) {
+        const int step = (hi - lo + 31) / 32;
+        const int idx = lo + lane * step;
+        const unsigned ok = __ballot_sync(0xffffffffu, idx < hi && prefix[idx] <= f);   // lane 0 always
+        const int k = 31 - __clz(ok);
+        lo += k * step;
+        hi = min(lo + step, hi);
+    }
+    const unsigned ok = __ballot_sync(0xffffffffu, lo + lane < hi && prefix[lo + lane] <= f);
+    return lo + 31 - __clz(ok);
+}
+
+// floor(x / n) for 0 <= x < 2^53 and n > 0, exact: x and n are exact doubles and the division is
+// correctly rounded, so a quotient that is not an integer stays more than 1/n away from the next one
+// (far above the rounding error), and an integer quotient is exact. Much cheaper than a 64-bit integer
+// division.
+__device__ __forceinline__ long long floor_div(long long x, long long n) {
+    return static_cast<long long>(floor(static_cast<double>(x) / static_cast<double>(n)));
 }
 
 // Work of one piece besides its pages, in pages: the stream-K split balances pages plus this much
@@ -198,10 +229,11 @@ __device__ __forceinline__ void build_work(const DecodeArgs &a, const int *prefi
 }
 
 // Flat page index at work position w: the pages of the units before w's unit, plus those of w's
-// unit that lie before w (a unit's pages follow its kPieceWork in the work order).
-__device__ __forceinline__ long long flat_of_work(const int *wpre, const int *prefix, int nv, long long w) {
+// unit that lie before w (a unit's pages follow its kPieceWork in the work order). A whole warp.
+// (Not inlined: inlined twice, the searches' registers pushed the streaming loop into spills.)
+__device__ __noinline__ long long flat_of_work(const int *wpre, const int *prefix, int nv, long long w, int lane) {
     if (w >= wpre[nv]) return prefix[nv];
-    const int v = find_vunit(wpre, nv, w);
+    const int v = find_vunit_warp(wpre, nv, w, lane);
     const long long pages = prefix[v + 1] - prefix[v];
     const long long into = w - (wpre[v + 1] - pages);
     return prefix[v] + (into < 0 ? 0 : (into > pages ? pages : into));
@@ -209,7 +241,7 @@ __device__ __forceinline__ long long flat_of_work(const int *wpre, const int *pr
 
 // The CTA whose (nonempty) range holds work position f.
 __device__ __forceinline__ long long cta_of(long long f, long long ptot, int ncta) {
-    return ((f + 1) * ncta + ptot - 1) / ptot - 1;
+    return floor_div((f + 1) * ncta + ptot - 1, ptot) - 1;
 }
 
 // Pieces of the unit whose pages lie at work positions [ps, pe): their count, and the partial-slot
@@ -584,8 +616,8 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
         pa = vc < nv ? prefix[vc] + P0 * crank / kcl : 0;
         pb = vc < nv ? prefix[vc] + P0 * (crank + 1) / kcl : 0;
     } else {
-        pa = flat_of_work(wpre, prefix, nv, ptot * blockIdx.x / a.ncta);
-        pb = flat_of_work(wpre, prefix, nv, ptot * (blockIdx.x + 1) / a.ncta);
+        pa = flat_of_work(wpre, prefix, nv, floor_div(ptot * blockIdx.x, a.ncta), lane);
+        pb = flat_of_work(wpre, prefix, nv, floor_div(ptot * (blockIdx.x + 1), a.ncta), lane);
     }
     __nv_bfloat16 *outp = static_cast<__nv_bfloat16 *>(a.out);
     if (warp < NCONS) {
@@ -605,7 +637,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
         }
     }
     if (pa >= pb) return;
-    const int v0 = aligned ? vc : find_vunit(prefix, nv, pa);
+    const int v0 = aligned ? vc : find_vunit_warp(prefix, nv, pa, lane);
     const int n_my = static_cast<int>(pb - pa);
 
     if (warp == NCONS) {
@@ -695,6 +727,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     constexpr int MST = L::MST, WST = L::WST;
     int i0 = 0, pi = 0;
     int split_v[2] = {0, 0}, split_ps[2] = {0, 0}, split_pe[2] = {0, 0}, n_split = 0;   // (thread 0)
+    int early_prev = -1;   // (thread 0) the count returned for the range's first piece, if counted early
     for (int v = v0; v < nv && prefix[v] < pb; ++v) {
         const long long ps = prefix[v], pe = prefix[v + 1];   // the unit's flat pages
         const int lo = static_cast<int>(max(pa, ps) - ps), hi = static_cast<int>(min(pb, pe) - ps);
@@ -806,9 +839,10 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                         mxg = fmaxf(mxg, __shfl_xor_sync(0xffffffffu, mxg, off));
                         mxh = fmaxf(mxh, __shfl_xor_sync(0xffffffffu, mxh, off));
                     }
-                    const float ng = fmaxf(m_g, mxg), nh = fmaxf(m_h, mxh);
+                    const bool ug = mxg > m_g + kLazyMax, uh = mxh > m_h + kLazyMax;   // move the reference?
+                    const float ng = ug ? mxg : m_g, nh = uh ? mxh : m_h;
                     const float bg = ng == -INFINITY ? 0.0f : ng, bh = nh == -INFINITY ? 0.0f : nh;
-                    const float cg = ex2(m_g - bg), ch = ex2(m_h - bh);
+                    const float cg = ug ? ex2(m_g - bg) : 1.0f, ch = uh ? ex2(m_h - bh) : 1.0f;
                     float pg_[2][2], ph_[2][2];
 #pragma unroll
                     for (int nt = 0; nt < 2; ++nt)
@@ -821,7 +855,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                     l_h = fmaf(l_h, ch, (ph_[0][0] + ph_[0][1]) + (ph_[1][0] + ph_[1][1]));
                     m_g = ng;
                     m_h = nh;
-                    if (!__all_sync(0xffffffffu, cg == 1.0f && ch == 1.0f)) {
+                    if (__any_sync(0xffffffffu, ug || uh)) {
 #pragma unroll
                         for (int j = 0; j < 2 * NKS; ++j) {
                             o[j][0] *= cg;
@@ -1010,17 +1044,18 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                         mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, off));
                         mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, off));
                     }
-                    const float mn0 = fmaxf(m_run[0], mx0), mn1 = fmaxf(m_run[1], mx1);
+                    const bool u0 = mx0 > m_run[0] + kLazyMax, u1 = mx1 > m_run[1] + kLazyMax;   // move the reference?
+                    const float mn0 = u0 ? mx0 : m_run[0], mn1 = u1 ? mx1 : m_run[1];
                     const float base0 = mn0 == -INFINITY ? 0.0f : mn0;
                     const float base1 = mn1 == -INFINITY ? 0.0f : mn1;
-                    const float corr0 = ex2(m_run[0] - base0), corr1 = ex2(m_run[1] - base1);
+                    const float corr0 = u0 ? ex2(m_run[0] - base0) : 1.0f, corr1 = u1 ? ex2(m_run[1] - base1) : 1.0f;
                     const float p0 = ex2(sl[0] - base0), p1 = ex2(sl[1] - base1);
                     const float p2 = ex2(sl[2] - base0), p3 = ex2(sl[3] - base1);
                     l_run[0] = fmaf(l_run[0], corr0, p0 + p2);
                     l_run[1] = fmaf(l_run[1], corr1, p1 + p3);
                     m_run[0] = mn0;
                     m_run[1] = mn1;
-                    if (!__all_sync(0xffffffffu, corr0 == 1.0f && corr1 == 1.0f)) {
+                    if (__any_sync(0xffffffffu, u0 || u1)) {
     #pragma unroll
                         for (int mt = 0; mt < NKS; ++mt) {
                             o[mt][0] *= corr0;
@@ -1135,14 +1170,21 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                 if (d4 == 0) a.part_l[pr] = lse2;
             }
         }
+        asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));   // mbuf free; every partial of the piece stored
         if (!complete && !aligned && ctid == 0 && n_split < 2) {
             split_v[n_split] = v;
             // the unit's pages in work positions (the split's coordinates)
             split_ps[n_split] = wpre[v + 1] - static_cast<int>(pe - ps);
             split_pe[n_split] = wpre[v + 1];
+            if (n_split == 0 && pe < pb) {
+                // the range's first piece, with more of the range after it: its unit's other pieces
+                // end the previous CTAs' ranges, so count it now and let one of them merge the unit
+                // at its end (the count's result is read only at the end of this range)
+                __threadfence();
+                early_prev = atomicAdd(a.counters + v, 1);
+            }
             ++n_split;
         }
-        asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));   // mbuf free for the next piece
     }
 
     if (aligned && kcl > 1) {
@@ -1196,8 +1238,8 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
         int np = 0;
         if (n_split > 0) {
             __threadfence();
-            // both counters in flight at once: one round trip
-            const int prev0 = atomicAdd(a.counters + split_v[0], 1);
+            // the counters not counted yet, both in flight at once: one round trip
+            const int prev0 = early_prev >= 0 ? early_prev : atomicAdd(a.counters + split_v[0], 1);
             const int prev1 = n_split > 1 ? atomicAdd(a.counters + split_v[1], 1) : 0;
             for (int k = 0; k < n_split; ++k) {
                 if ((k == 0 ? prev0 : prev1) == piece_count(split_ps[k], split_pe[k], ptot, a.ncta) - 1) {
