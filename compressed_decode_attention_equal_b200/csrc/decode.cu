@@ -532,24 +532,23 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                     q + ((static_cast<long long>(b) * a.R + row / a.G) * a.Hq + h * a.G + row % a.G) * D;
                 bulk_g2s(qbuf + (row - p0) * L::QROWB, src, D * 2, &qfull[0]);
             }
-            for (int k = 0; k < n_first; ++k) {
-                const int phys = __shfl_sync(0xffffffffu, spec_page, k);
-                if (lane == 0) {
-                    if (phys < 0 || phys >= a.num_pages) {   // flagged only if the guess holds
-                        spec_bad |= 1u << k;
-                        svalid[k] = 0;
-                        mbar_arrive(&full[k]);
-                    } else {
-                        svalid[k] = 1;
-                        mbar_arrive_expect_tx(&full[k], G::STAGE);
-                        // pages are read once per call: evict-first, so that they do not push the
-                        // small inputs (tables, lengths, queries) out of L2
-                        bulk_g2s_hint(stages + k * G::STAGE, a.pages + static_cast<long long>(phys) * G::STAGE,
-                                      G::STAGE, &full[k], createpolicy_evict_first());
-                    }
+            // lane k copies page k of the range into stage k (all issued at once)
+            bool bad = false;
+            if (lane < n_first) {
+                if (spec_page < 0 || spec_page >= a.num_pages) {   // flagged only if the guess holds
+                    bad = true;
+                    svalid[lane] = 0;
+                    mbar_arrive(&full[lane]);
+                } else {
+                    svalid[lane] = 1;
+                    mbar_arrive_expect_tx(&full[lane], G::STAGE);
+                    // pages are read once per call: evict-first, so that they do not push the small
+                    // inputs (tables, lengths, queries) out of L2
+                    bulk_g2s_hint(stages + lane * G::STAGE, a.pages + static_cast<long long>(spec_page) * G::STAGE,
+                                  G::STAGE, &full[lane], createpolicy_evict_first());
                 }
-                __syncwarp();
             }
+            spec_bad = __ballot_sync(0xffffffffu, bad);
         }
         cluster_wait();   // pairs with the arrival above (the producer touches no remote memory)
         asm volatile("bar.sync 2, %0;" ::"n"(NTHR));   // the consumers' verdict and prefix
