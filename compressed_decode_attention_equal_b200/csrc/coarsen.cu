@@ -316,31 +316,90 @@ __global__ void __launch_bounds__(kK1Threads, 2)
 }
 
 // ---------------------------------------------------------------------------
-// k_project_tc (option SKV_PROJECTION_TENSOR_BF16): the same tiles, TMA staging and scan, but
-// z = P16 x on the tensor cores: P16 = bf16(P), x the bf16 features, fp32 accumulation
-// (mma.sync m16n8k16; tokens as M, the 16 outputs as two n8 tiles, features as K). Each warp owns
-// 128 rows of the tile (8 m-tiles); P16's B fragments stay in registers for the whole tile. The
-// products are exact; only the accumulation order and rounding differ from the fixed recipe, so
-// the quantised steps differ from it by a bounded amount and the boundaries follow the steps the
-// tensor cores produced.
+// k_project_tc (option SKV_PROJECTION_TENSOR_BF16): the same tiles and scan, with z = P16 x on the
+// fifth-generation tensor cores: P16 = bf16(P), x the bf16 features, fp32 accumulation in tensor
+// memory. The products are exact; only the accumulation order and rounding differ from the fixed
+// recipe, so the quantised steps differ from it by a bounded amount and the boundaries follow the
+// steps the tensor cores produced.
+//
+// One thread issues everything: the TMA copies of a tile's 64-byte feature chunks (512 rows each,
+// the 64-byte swizzle) into a kTcStages ring, and per chunk 8 MMAs (tcgen05.mma kind::f16, M = 128
+// tokens, N = 16 outputs, K = 16 features: 4 row blocks x 2 feature halves) that read the chunk and
+// P16's image straight from shared memory and accumulate z of the 4 row blocks in 64 columns of
+// tensor memory; tcgen05.commit releases a stage to the next copy when its MMAs are done. The four
+// warps then read z back (tcgen05.ld, one token row per thread) for the steps and the scan.
 // ---------------------------------------------------------------------------
+constexpr int kTcStages = 3;
+constexpr int kTcCols = 4 * kProjDim;   // tensor-memory columns: z of the tile's 4 row blocks of 128
+
+// Shared-memory matrix descriptor of a K-major operand in the 64-byte swizzle (rows of 64 bytes,
+// 16-byte granule g of row r at g ^ ((r >> 1) & 3)): start address, 8-row groups 512 bytes apart.
+__device__ __forceinline__ uint64_t tc_desc_sw64(uint32_t saddr) {
+    return static_cast<uint64_t>((saddr & 0x3FFFFu) >> 4) | (static_cast<uint64_t>(1u) << 16) |
+           (static_cast<uint64_t>(512u >> 4) << 32) | (static_cast<uint64_t>(1u) << 46) |
+           (static_cast<uint64_t>(4u) << 61);
+}
+
+// Instruction descriptor of kind::f16: fp32 accumulator, bf16 A and B, both K-major, N = 16, M = 128.
+constexpr uint32_t kTcIdesc = (1u << 4) | (1u << 7) | (1u << 10) | ((kProjDim >> 3) << 17) | ((128u >> 4) << 24);
+
+__device__ __forceinline__ void tc_mma(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, bool accumulate) {
+    asm volatile(
+        "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+            d_tmem),
+        "l"(adesc), "l"(bdesc), "r"(kTcIdesc), "r"(accumulate ? 1u : 0u));
+}
+
+// arrive on `bar` once every MMA this thread has issued so far has completed
+__device__ __forceinline__ void tc_commit(uint64_t *bar) {
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(smem_u32(bar))
+                 : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before_sync() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after_sync() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+
+// 16 consecutive fp32 columns of this thread's tensor-memory lane
+__device__ __forceinline__ void tc_ld16(uint32_t taddr, float *v) {
+    uint32_t r[16];
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, "
+        "%15}, [%16];"
+        : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]),
+          "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = __uint_as_float(r[j]);
+}
+
+template <int D>
+constexpr size_t tc_smem_bytes() {
+    // alignment slack + stage ring + P16 image + barriers, tensor-memory slot, scan scratch
+    return 1024 + kTcStages * kK1StageBytes + sizeof(ProjFrag) + 128 + 64;
+}
+
 template <int D>
 __global__ void __launch_bounds__(kK1Threads, 2)
     k_project_tc(const CoarsenArgs a, const __grid_constant__ CUtensorMap map_k,
                  const __grid_constant__ CUtensorMap map_v, const __grid_constant__ ProjFrag pf) {
-    constexpr int KCHUNK = D * 2 / kK1ColBytes;      // bf16 column chunks of one key row
-    constexpr int NCHUNK = 2 * KCHUNK;               // key chunks, then value chunks
-    constexpr int KPC = kK1ColBytes / 32;            // k-steps of 16 features per chunk
-    constexpr int NKS = NCHUNK * KPC;                // k-steps over the 2d features
-    constexpr int MT = kTileRows / 16 / (kK1Threads / 32);   // m-tiles of 16 rows per warp (8)
-    static_assert(NKS * 16 == 2 * D, "k-steps cover the features");
+    constexpr int KCHUNK = D * 2 / kK1ColBytes;   // bf16 column chunks of one key row
+    constexpr int NCHUNK = 2 * KCHUNK;            // key chunks, then value chunks
+    constexpr int PIMG = NCHUNK * kProjDim * kK1ColBytes;   // bytes of P16's image
+    static_assert(kTileRows == 4 * 128 && kK1StageBytes == kTileRows * kK1ColBytes, "4 row blocks of 128");
+    static_assert(PIMG <= static_cast<int>(sizeof(ProjFrag)) && kTcCols == 64, "image and columns");
 
     extern __shared__ uint8_t smem_raw[];
     const uint32_t raw = smem_u32(smem_raw);
-    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);
+    uint8_t *smem = smem_raw + (((raw + 1023u) & ~1023u) - raw);   // the swizzle atoms need 512-byte alignment
     uint8_t *stages = smem;
-    uint64_t *bar = reinterpret_cast<uint64_t *>(smem + kK1Stages * kK1StageBytes);
-    long long *warp_sum = reinterpret_cast<long long *>(bar + 8);
+    uint8_t *pimg = stages + kTcStages * kK1StageBytes;
+    uint64_t *full = reinterpret_cast<uint64_t *>(pimg + sizeof(ProjFrag));
+    uint64_t *consumed = full + kTcStages;
+    uint64_t *done = consumed + kTcStages;
+    uint32_t *tslot = reinterpret_cast<uint32_t *>(done + 1);
+    int *ok_flag = reinterpret_cast<int *>(tslot + 1);
+    long long *warp_sum = reinterpret_cast<long long *>(full + 16);
 
     const int u = blockIdx.y;
     const int tile = blockIdx.x;
@@ -350,86 +409,105 @@ __global__ void __launch_bounds__(kK1Threads, 2)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
     const int y0 = static_cast<int>(sr.row_off + static_cast<int64_t>(h) * sr.T + sr.s_eff) + tile * kTileOut - 1;
+    int n_issued = 0;   // (thread 0) chunks whose copy has been issued
     auto issue = [&](int c, int s) {
-        mbar_arrive_expect_tx(&bar[s], kK1StageBytes);
+        ++n_issued;
+        mbar_arrive_expect_tx(&full[s], kK1StageBytes);
         const CUtensorMap *map = c < KCHUNK ? &map_k : &map_v;
 #pragma unroll
         for (int hb = 0; hb < kTileRows / kK1BoxRows; ++hb)
             tma_load_2d(stages + s * kK1StageBytes + hb * kK1BoxRows * kK1ColBytes, map, (c % KCHUNK) * 32,
-                        y0 + hb * kK1BoxRows, &bar[s]);
+                        y0 + hb * kK1BoxRows, &full[s]);
     };
     if (tid == 0) {
         prefetch_tensormap(&map_k);
         prefetch_tensormap(&map_v);
-        for (int s = 0; s < kK1Stages; ++s) mbar_init(&bar[s], 1);
+        for (int s = 0; s < kTcStages; ++s) {
+            mbar_init(&full[s], 1);
+            mbar_init(&consumed[s], 1);
+        }
+        mbar_init(done, 1);
+        *ok_flag = 1;
         fence_mbar_init();
-        for (int c = 0; c < NCHUNK && c < kK1Stages; ++c) issue(c, c);
+        for (int c = 0; c < NCHUNK && c < kTcStages; ++c) issue(c, c);
     }
-    uint32_t bf[NKS][2][2];   // P16^T fragments: k-step, n-tile, register
-#pragma unroll
-    for (int ks = 0; ks < NKS; ++ks)
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            bf[ks][nt][0] = pf.w[((ks * 2 + nt) * 32 + lane) * 2];
-            bf[ks][nt][1] = pf.w[((ks * 2 + nt) * 32 + lane) * 2 + 1];
-        }
-    float zacc[MT][2][4];
-#pragma unroll
-    for (int mt = 0; mt < MT; ++mt)
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) zacc[mt][nt][0] = zacc[mt][nt][1] = zacc[mt][nt][2] = zacc[mt][nt][3] = 0.0f;
-    __syncthreads();   // barriers initialised
+    // P16's image (already in the 64-byte swizzle, chunk after chunk) into shared memory, then made
+    // visible to the tensor cores (async proxy)
+    for (int i = tid; i < PIMG / 16; i += kK1Threads)
+        reinterpret_cast<uint4 *>(pimg)[i] = reinterpret_cast<const uint4 *>(pf.w)[i];
+    fence_proxy_async_smem();
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(smem_u32(tslot)),
+                     "r"(static_cast<uint32_t>(kTcCols)));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+    tc_fence_before_sync();
+    __syncthreads();   // barriers, the image and the tensor-memory address are ready
+    tc_fence_after_sync();
+    const uint32_t tmem = *tslot;
 
-    // ldmatrix rows of this lane: matrices 0 / 1 are rows 0-7 / 8-15 of an m-tile at the k-step's
-    // first 8 features, matrices 2 / 3 the same rows at its last 8
-    const int lrow = (lane & 7) + 8 * ((lane >> 3) & 1), lhalf = lane >> 4;
+    if (tid == 0) {
+        bool ok = true;
+        int n_landed = 0;   // chunks whose copy this thread has seen land
+        for (int c = 0; c < NCHUNK; ++c) {
+            const int s = c % kTcStages;
+            if (!mbar_wait(&full[s], (c / kTcStages) & 1)) {
+                ok = false;
+                break;
+            }
+            ++n_landed;
+            tc_fence_after_sync();
+            const uint32_t sa = smem_u32(stages + s * kK1StageBytes);
+            const uint32_t sb = smem_u32(pimg + c * kProjDim * kK1ColBytes);
 #pragma unroll
-    for (int c = 0; c < NCHUNK; ++c) {
-        const int s = c % kK1Stages;
-        const bool got = mbar_wait(&bar[s], (c / kK1Stages) & 1);
-        const uint32_t sb = smem_u32(stages + s * kK1StageBytes);
+            for (int mb = 0; mb < 4; ++mb)
 #pragma unroll
-        for (int kk = 0; kk < KPC; ++kk) {
-            const int ks = c * KPC + kk;
-            const int cc = 2 * kk + lhalf;   // 16-byte sub-chunk of the 64-byte chunk row
-#pragma unroll
-            for (int mt = 0; mt < MT; ++mt) {
-                const int row = warp * (MT * 16) + mt * 16 + lrow;
-                uint32_t a0, a1, a2, a3;
-                ldsm_x4(sb + row * kK1ColBytes + ((cc ^ ((row >> 1) & 3)) << 4), a0, a1, a2, a3);
-                mma_bf16(zacc[mt][0], a0, a1, a2, a3, bf[ks][0][0], bf[ks][0][1]);
-                mma_bf16(zacc[mt][1], a0, a1, a2, a3, bf[ks][1][0], bf[ks][1][1]);
+                for (int ks = 0; ks < 2; ++ks)
+                    tc_mma(tmem + mb * kProjDim, tc_desc_sw64(sa + mb * 128 * kK1ColBytes + ks * 32),
+                           tc_desc_sw64(sb + ks * 32), c > 0 || ks > 0);
+            tc_commit(&consumed[s]);   // the stage is free once these MMAs have read it
+            if (c + kTcStages < NCHUNK) {
+                if (!mbar_wait(&consumed[s], (c / kTcStages) & 1)) {
+                    ok = false;
+                    break;
+                }
+                issue(c + kTcStages, s);
             }
         }
-        // as in k_project_scan: a wait that gave up stops the tile after the copies in flight land
-        if (!__syncthreads_and(got)) {
-            if (tid == 0) {
-                for (int c2 = c; c2 < NCHUNK && c2 <= c + 1; ++c2)
-                    (void)mbar_wait(&bar[c2 % kK1Stages], (c2 / kK1Stages) & 1);
-                raise_flag(a.flags, FLAG_TIMEOUT);
-            }
-            return;
+        tc_commit(done);   // every MMA issued, also after a failed wait
+        if (!ok) {
+            // a wait gave up: no further copy or MMA; the copies already in flight land first
+            for (int c2 = n_landed; c2 < n_issued; ++c2)
+                (void)mbar_wait(&full[c2 % kTcStages], (c2 / kTcStages) & 1);
+            *ok_flag = 0;
+            raise_flag(a.flags, FLAG_TIMEOUT);
         }
-        if (tid == 0 && c + kK1Stages < NCHUNK) issue(c + kK1Stages, s);
     }
-
-    // z of the rows -> shared: accumulator (mt, nt) holds tokens row0 + g, row0 + g + 8 and
-    // outputs 8 nt + 2 c4, 8 nt + 2 c4 + 1
+    const bool mma_done = mbar_wait(done, 0);
+    __syncthreads();   // thread 0's verdict
+    tc_fence_after_sync();
+    const bool good = mma_done && *ok_flag != 0;
+    // z of the tile's rows (the stages are free: every MMA has completed) -> shared, row after row
     float *zb = reinterpret_cast<float *>(stages);
-    const int g = lane >> 2, c4 = lane & 3;
+    if (good) {
+#pragma unroll 1
+        for (int mb = 0; mb < 4; ++mb) {
+            float z[kProjDim];
+            tc_ld16(tmem + ((static_cast<uint32_t>(warp) * 32u) << 16) + mb * kProjDim, z);
+            const int r = mb * 128 + warp * 32 + lane;
 #pragma unroll
-    for (int mt = 0; mt < MT; ++mt) {
-        const int r = warp * (MT * 16) + mt * 16 + g;
-#pragma unroll
-        for (int nt = 0; nt < 2; ++nt) {
-            const int i = nt * 8 + 2 * c4;
-            zb[r * kZStride + i] = zacc[mt][nt][0];
-            zb[r * kZStride + i + 1] = zacc[mt][nt][1];
-            zb[(r + 8) * kZStride + i] = zacc[mt][nt][2];
-            zb[(r + 8) * kZStride + i + 1] = zacc[mt][nt][3];
+            for (int i = 0; i < kProjDim; ++i) zb[r * kZStride + i] = z[i];
         }
     }
+    tc_fence_before_sync();
     __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(static_cast<uint32_t>(kTcCols)));
+    if (!good) {
+        if (tid == 0 && !mma_done) raise_flag(a.flags, FLAG_TIMEOUT);
+        return;
+    }
     scan_tile(a, sr, u, h, tile, zb, warp_sum);
 }
 
@@ -778,7 +856,7 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
 template <int D>
 static cudaError_t launch_project_tc(const CoarsenArgs &a, int n_units, const ProjFrag &frag,
                                     const CUtensorMap &map_k, const CUtensorMap &map_v, cudaStream_t s) {
-    constexpr size_t smem = 1024 + kK1Stages * kK1StageBytes + 64 + 64;
+    constexpr size_t smem = tc_smem_bytes<D>();
     static thread_local int configured_dev = -1;
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);

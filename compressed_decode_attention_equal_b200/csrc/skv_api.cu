@@ -84,22 +84,20 @@ uint16_t bf16_rne_bits(float x) {
     return static_cast<uint16_t>((u + 0x7fffu + ((u >> 16) & 1u)) >> 16);
 }
 
-// P16 = bf16(P) laid out as the tensor-core projection's B fragments (see ProjFrag): register r of
-// lane (g = lane / 4, c = lane % 4) in k-step ks and n-tile nt packs P16[8 nt + g][16 ks + 2 c + 8 r]
-// (low half) and P16[8 nt + g][16 ks + 2 c + 8 r + 1] (high half).
+// P16 = bf16(P) as the tensor-core projection's shared-memory image (see ProjFrag).
 void make_projection_fragments(uint64_t seed, int d, ProjFrag &out) {
     std::vector<float> P(static_cast<size_t>(kProjDim) * 2 * d);
     make_projection(seed, d, P.data());
     std::memset(&out, 0, sizeof out);
-    const int cols = 2 * d, nks = cols / 16;
-    for (int ks = 0; ks < nks; ++ks)
-        for (int nt = 0; nt < 2; ++nt)
-            for (int lane = 0; lane < 32; ++lane)
-                for (int r = 0; r < 2; ++r) {
-                    const int n = 8 * nt + lane / 4, k = 16 * ks + 2 * (lane % 4) + 8 * r;
-                    const uint32_t lo = bf16_rne_bits(P[static_cast<size_t>(n) * cols + k]);
-                    const uint32_t hi = bf16_rne_bits(P[static_cast<size_t>(n) * cols + k + 1]);
-                    out.w[((ks * 2 + nt) * 32 + lane) * 2 + r] = lo | (hi << 16);
+    const int cols = 2 * d, nchunk = cols / 32;
+    uint16_t *img = reinterpret_cast<uint16_t *>(out.w);
+    for (int c = 0; c < nchunk; ++c)
+        for (int n = 0; n < kProjDim; ++n)
+            for (int g = 0; g < 4; ++g)
+                for (int e = 0; e < 8; ++e) {
+                    const int k = 32 * c + 8 * g + e;   // feature
+                    img[c * 512 + n * 32 + ((g ^ ((n >> 1) & 3)) * 8) + e] =
+                        bf16_rne_bits(P[static_cast<size_t>(n) * cols + k]);
                 }
 }
 

@@ -39,11 +39,13 @@ struct ProjT {
     float pt[2 * 128 * SKV_PROJ_DIM];
 };
 
-// The tensor-core projection's operand: P16 = bf16(P) (round to nearest even) as mma.sync
-// m16n8k16 B fragments, w[((ks * 2 + nt) * 32 + lane) * 2 + r] for k-step ks (features 16 ks ..
-// 16 ks + 15), n-tile nt (outputs 8 nt .. 8 nt + 7) and the fragment's register r.
-struct ProjFrag {
-    uint32_t w[(2 * 128 / 16) * 2 * 32 * 2];
+// The tensor-core projection's B operand: P16 = bf16(P) (round to nearest even) as the image the
+// MMAs read from shared memory: for each 32-feature chunk c (features 32 c .. 32 c + 31 of [k; v]),
+// 16 rows of 64 bytes (row n = output n), the row's four 16-byte granules g (features 32 c + 8 g ..
+// + 7) stored at granule position g ^ ((n >> 1) & 3) -- the 64-byte swizzle of the TMA-loaded
+// token chunks. Chunk c's image starts at byte 1024 c; d = 64 uses the first half.
+struct alignas(16) ProjFrag {
+    uint32_t w[(2 * 128 / 32) * 16 * 64 / 4];
 };
 
 struct CoarsenArgs {
