@@ -548,9 +548,10 @@ __global__ void __launch_bounds__(256) k_tile_prefix(const CoarsenArgs a) {
 // ---------------------------------------------------------------------------
 // k_boundaries: b_j = first t with N c_t >= j c_T  (j = 1 .. N-1)
 // ---------------------------------------------------------------------------
-// floor(N * C / CT) for CT > 0, exact (the double estimate is off by at most one)
-__device__ __forceinline__ long long floor_ratio(long long N, long long C, long long CT) {
-    long long q = static_cast<long long>(static_cast<double>(N) * static_cast<double>(C) / static_cast<double>(CT));
+// floor(N * C / CT) for CT > 0, exact: the double estimate (inv_ct = 1 / CT) is off by at most one
+// and corrected with exact 128-bit products
+__device__ __forceinline__ long long floor_ratio(long long N, long long C, long long CT, double inv_ct) {
+    long long q = static_cast<long long>(static_cast<double>(N) * static_cast<double>(C) * inv_ct);
     if (q < 0) q = 0;
     while (prod_ge(static_cast<uint64_t>(N), static_cast<uint64_t>(C), static_cast<uint64_t>(q + 1),
                    static_cast<uint64_t>(CT)))
@@ -561,19 +562,21 @@ __device__ __forceinline__ long long floor_ratio(long long N, long long C, long 
     return q;
 }
 
+// One thread per middle token t: the thresholds j with floor(N c_{t-1} / c_T) < j <= floor(N c_t / c_T)
+// are first hit at t. Each thread computes its own floor once and takes its predecessor's from the
+// neighbouring lane (the first lane of a warp computes both).
 __global__ void __launch_bounds__(kTileRows) k_boundaries(const CoarsenArgs a) {
     const int u = blockIdx.y, tile = blockIdx.x;
     const int b = u / a.Hkv, h = u % a.Hkv;
     const SeqRow sr = a.seq[b];
-    if (tile >= sr.tiles || threadIdx.x >= kTileOut) return;
+    if (tile >= sr.tiles) return;
     const int t = tile * kTileOut + threadIdx.x;
-    if (t >= sr.M) return;
+    const bool act = threadIdx.x < kTileOut && t < sr.M;   // inactive threads sit at the tile's end
     const int64_t *ls = a.local_scan + sr.mid_off + static_cast<int64_t>(h) * sr.M;
     const long long tp = a.tile_prefix[static_cast<int64_t>(u) * a.max_tiles + tile];
     const long long CT = a.unit_total[u];
-    const long long Ct = tp + ls[t];
-    const long long Cprev = threadIdx.x == 0 ? tp : tp + ls[t - 1];
-    if (a.cumvar) a.cumvar[sr.row_off + static_cast<int64_t>(h) * sr.T + t] = Ct;
+    const long long Ct = act ? tp + ls[t] : 0;
+    if (act && a.cumvar) a.cumvar[sr.row_off + static_cast<int64_t>(h) * sr.T + t] = Ct;
     const int N = sr.N;
     int32_t *bnd = a.bounds + sr.bnd_off + static_cast<int64_t>(h) * (N + 1);
     if (CT == 0) {
@@ -581,11 +584,14 @@ __global__ void __launch_bounds__(kTileRows) k_boundaries(const CoarsenArgs a) {
             for (int j = 1; j < N; ++j) bnd[j] = 0;
         return;
     }
-    if (t == 0) return;
-    long long jhi = floor_ratio(N, Ct, CT);
-    if (jhi > N - 1) jhi = N - 1;
-    const long long jlo = floor_ratio(N, Cprev, CT) + 1;
-    for (long long j = jlo; j <= jhi; ++j) bnd[j] = t;
+    const double inv = 1.0 / static_cast<double>(CT);
+    const long long q = act ? floor_ratio(N, Ct, CT, inv) : 0;
+    long long qprev = __shfl_up_sync(0xffffffffu, q, 1);
+    if ((threadIdx.x & 31) == 0 && act)
+        qprev = floor_ratio(N, threadIdx.x == 0 ? tp : tp + ls[t - 1], CT, inv);
+    if (!act || t == 0) return;
+    const long long jhi = q > N - 1 ? N - 1 : q;
+    for (long long j = qprev + 1; j <= jhi; ++j) bnd[j] = t;
 }
 
 // ---------------------------------------------------------------------------

@@ -147,9 +147,10 @@ __device__ __forceinline__ long long floor_div(long long x, long long n) {
 
 // Work of one piece besides its pages, in pages: the stream-K split balances pages plus this much
 // per unit, since each piece costs its CTA a query-row load and an epilogue (the page-group merge
-// and the output or partial stores) on top of its pages -- measured about five pages' worth with
-// 28 query rows per unit, so a split by pages alone left the CTAs holding many short units last.
-constexpr int kPieceWork = 4;
+// and the output or partial stores) on top of its pages, so a split by pages alone left the CTAs
+// holding many short units last (28 query rows per unit: 2, 4, 6 and 8 measured 62.3, 58.0, 56.8
+// and 57.0 us on the ragged 2% workload).
+constexpr int kPieceWork = 6;
 
 // Every CTA rebuilds the page prefix over virtual units (flat index of each unit's first page) and
 // keeps every unit's clamped entry count, both in shared memory (lens are tiny and L2-resident).
