@@ -155,21 +155,27 @@ constexpr int kPieceWork = 6;
 // Every CTA rebuilds the page prefix over virtual units (flat index of each unit's first page) and
 // keeps every unit's clamped entry count, both in shared memory (lens are tiny and L2-resident).
 // Run by the consumer warps alone (named barrier 1), so the producer can start copies meanwhile.
+// `spec`: before the dependency wait, with lens that may still change: L2-only loads (no stale line
+// is left in L1) and no flag raised; the result is checked against a second read after the wait.
 template <int NCONS>
-__device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, int *ents, int *scratch) {
+__device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, int *ents, int *scratch, bool spec) {
     const int nv = a.n_vunits;
     const int tid = threadIdx.x, nth = NCONS * 32;
     const int per = (nv + nth - 1) / nth;
     const int lo = min(tid * per, nv), hi = min(lo + per, nv);
+    const int cap = a.max_pages * kPageNodes;
     int local = 0;
     for (int v = lo; v < hi; v += 4) {
         int raw[4];   // four loads in flight before any is used
 #pragma unroll
-        for (int j = 0; j < 4; ++j) raw[j] = v + j < hi ? a.lens[(v + j) / a.row_passes] : 0;
+        for (int j = 0; j < 4; ++j) {
+            const int32_t *p = a.lens + (v + j) / a.row_passes;
+            raw[j] = v + j < hi ? (spec ? ld_global_cg_s32(p) : *p) : 0;
+        }
 #pragma unroll
         for (int j = 0; j < 4; ++j)
             if (v + j < hi) {
-                const int L = clamp_len(a, raw[j]);
+                const int L = spec ? min(max(raw[j], 0), cap) : clamp_len(a, raw[j]);
                 const int pages = (L + kPageNodes - 1) / kPageNodes;
                 ents[v + j] = L;
                 prefix[v + j] = pages;   // page count for now; made exclusive below
@@ -195,6 +201,27 @@ __device__ __forceinline__ void build_prefix(const DecodeArgs &a, int *prefix, i
     }
     if (tid == nth - 1) prefix[nv] = wp + x;
     asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));
+}
+
+// After the dependency wait: read the lens again (flagging bad ones) and check every clamped count
+// against the one the speculative prefix was built from. Consumer warps alone; the verdict is
+// the same in every consumer thread.
+template <int NCONS>
+__device__ __forceinline__ bool lens_unchanged(const DecodeArgs &a, const int *ents) {
+    const int nv = a.n_vunits;
+    const int tid = threadIdx.x, nth = NCONS * 32;
+    const int per = (nv + nth - 1) / nth;
+    const int lo = min(tid * per, nv), hi = min(lo + per, nv);
+    bool same = true;
+    for (int v = lo; v < hi; v += 4) {
+        int raw[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) raw[j] = v + j < hi ? a.lens[(v + j) / a.row_passes] : 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+            if (v + j < hi) same &= clamp_len(a, raw[j]) == ents[v + j];
+    }
+    return bar_and(1, NCONS * 32, same);
 }
 
 // The work prefix of the stream-K split (built only when the grid splits that way): a unit's work
@@ -467,8 +494,11 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     // (cluster - 1 blocks of pass_rows x (D + 1) floats behind the page prefix)
     int *ents = prefix + ((nv + 1 + 3) & ~3);   // entries of every virtual unit
     float *xbuf = reinterpret_cast<float *>(ents + ((nv + 3) & ~3));   // 16-byte aligned
-    // the stream-K split's work prefix shares the receive buffer's storage (used only by the
-    // aligned split)
+    // The stream-K split's work prefix shares the receive buffer's storage. Only a busy CTA of an
+    // aligned cluster launch has its receive buffer written by other CTAs; such a CTA always takes
+    // the producer's guess (try_spec below), and with the guess the set-up, work prefix included,
+    // runs only after the dependency wait and is final -- it builds the work prefix only if the
+    // split is not aligned, when no CTA writes a receive buffer.
     int *wpre = reinterpret_cast<int *>(xbuf);
     cluster_arrive_relaxed();   // this CTA has started (waited on before any remote access)
     if (tid == 0) {   // independent of the inputs: overlaps the wait below
@@ -514,8 +544,9 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
         if (phys >= 0 && phys < a.num_pages)
             bulk_prefetch_l2(a.pages + static_cast<long long>(phys) * G::STAGE, G::STAGE);
     }
-    // wait for every preceding grid to complete (its writes visible) before reading any input
-    asm volatile("griddepcontrol.wait;" ::: "memory");
+    // wait for every preceding grid to complete (its writes visible) before reading any input (the
+    // consumer warps wait below, after their speculative set-up)
+    if (warp >= NCONS) asm volatile("griddepcontrol.wait;" ::: "memory");
     const __nv_bfloat16 *q = static_cast<const __nv_bfloat16 *>(a.q);
     int spec_page = -1;      // producer lane j: page id of column c0 + j
     uint32_t spec_bad = 0;   // producer: first pages whose id lies outside the pool
@@ -554,26 +585,73 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
         cluster_wait();   // pairs with the arrival above (the producer touches no remote memory)
         asm volatile("bar.sync 2, %0;" ::"n"(NTHR));   // the consumers' verdict and prefix
     } else {
-        build_prefix<NCONS>(a, prefix, ents, scan_scratch);
-        // Aligned split: when every unit has the same page count P0 and `cluster` CTAs per unit
-        // fit in the grid, the k = cluster CTAs of a thread-block cluster take equal page ranges of
-        // one unit and merge through distributed shared memory (no global partials, one piece per
-        // CTA). Otherwise the flat page space is cut into ncta equal ranges (stream-K style).
-        const int P0 = prefix[1] - prefix[0];
-        bool uni = true;
-        {
-            const int per = (nv + NCONS * 32 - 1) / (NCONS * 32);
-            for (int v = min(tid * per, nv); v < min(tid * per + per, nv); ++v)
-                uni &= (prefix[v + 1] - prefix[v] == P0);
+        // Without the producer's guess (the stream-K split is likely), the set-up -- page prefix,
+        // work prefix and this CTA's range -- first runs before the dependency wait on lens that
+        // may be stale (misc[11..13]: the range's first and end flat page and first virtual unit,
+        // misc[14] = 1), and is kept if the lens read after the wait are the same; otherwise, and
+        // with the guess, it runs after the wait (where the producer's copies, not the set-up, are
+        // the critical path).
+        bool have = false;
+        bool waited = false;
+        // (built for the many-row shapes only: the code slowed the 7-row decode measurably even
+        // where it did not run)
+        if constexpr (MR) {
+            if (!try_spec) {
+                waited = true;
+                build_prefix<NCONS>(a, prefix, ents, scan_scratch, true);
+                const int P0s = prefix[1] - prefix[0];
+                bool unis = true;
+                {
+                    const int per = (nv + NCONS * 32 - 1) / (NCONS * 32);
+                    for (int v = min(tid * per, nv); v < min(tid * per + per, nv); ++v)
+                        unis &= (prefix[v + 1] - prefix[v] == P0s);
+                }
+                unis = bar_and(1, NCONS * 32, unis);
+                const bool als = unis && (kcl > 1 || 4LL * nv >= 3LL * a.ncta) && P0s >= kcl &&
+                                 static_cast<long long>(nv) * kcl <= a.ncta;
+                if (!als) {
+                    build_work<NCONS>(a, prefix, wpre, scan_scratch);
+                    if (warp == 0) {
+                        const long long ptot_ = wpre[nv];
+                        const long long pa_ = flat_of_work(wpre, prefix, nv, floor_div(ptot_ * blockIdx.x, a.ncta), lane);
+                        const long long pb_ =
+                            flat_of_work(wpre, prefix, nv, floor_div(ptot_ * (blockIdx.x + 1), a.ncta), lane);
+                        const int v0_ = pa_ < pb_ ? find_vunit_warp(prefix, nv, pa_, lane) : 0;
+                        if (lane == 0) {
+                            misc[11] = static_cast<int>(pa_);
+                            misc[12] = static_cast<int>(pb_);
+                            misc[13] = v0_;
+                        }
+                    }
+                }
+                asm volatile("griddepcontrol.wait;" ::: "memory");
+                have = lens_unchanged<NCONS>(a, ents) && !als;
+                if (have && tid == 0) {
+                    misc[8] = 0;
+                    misc[9] = 0;
+                }
+            }
         }
-        uni = bar_and(1, NCONS * 32, uni);
-        const bool al = uni && (kcl > 1 || 4LL * nv >= 3LL * a.ncta) && P0 >= kcl &&
-                        static_cast<long long>(nv) * kcl <= a.ncta;
-        if (tid == 0) {
-            misc[8] = al ? 1 : 0;
-            misc[9] = (al && try_spec && P0 == a.max_pages) ? 1 : 0;
+        if (!waited) asm volatile("griddepcontrol.wait;" ::: "memory");
+        if (MR && tid == 0) misc[14] = have ? 1 : 0;
+        if (!have) {
+            build_prefix<NCONS>(a, prefix, ents, scan_scratch, false);
+            const int P0 = prefix[1] - prefix[0];
+            bool uni = true;
+            {
+                const int per = (nv + NCONS * 32 - 1) / (NCONS * 32);
+                for (int v = min(tid * per, nv); v < min(tid * per + per, nv); ++v)
+                    uni &= (prefix[v + 1] - prefix[v] == P0);
+            }
+            uni = bar_and(1, NCONS * 32, uni);
+            const bool al = uni && (kcl > 1 || 4LL * nv >= 3LL * a.ncta) && P0 >= kcl &&
+                            static_cast<long long>(nv) * kcl <= a.ncta;
+            if (tid == 0) {
+                misc[8] = al ? 1 : 0;
+                misc[9] = (al && try_spec && P0 == a.max_pages) ? 1 : 0;
+            }
+            if (!al) build_work<NCONS>(a, prefix, wpre, scan_scratch);
         }
-        if (!al) build_work<NCONS>(a, prefix, wpre, scan_scratch);
         cluster_wait();   // every CTA of the cluster has started
         asm volatile("bar.arrive 2, %0;" ::"n"(NTHR));
         asm volatile("bar.sync 1, %0;" ::"n"(NCONS * 32));   // misc visible to every consumer
@@ -611,10 +689,14 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
     }
     const long long ptot = aligned ? 0 : wpre[nv];   // total work of the stream-K split
     const int P0 = prefix[1] - prefix[0];
+    const bool have_range = MR && misc[14] != 0;
     long long pa, pb;   // this CTA's flat pages
     if (aligned) {
         pa = vc < nv ? prefix[vc] + P0 * crank / kcl : 0;
         pb = vc < nv ? prefix[vc] + P0 * (crank + 1) / kcl : 0;
+    } else if (have_range) {
+        pa = misc[11];
+        pb = misc[12];
     } else {
         pa = flat_of_work(wpre, prefix, nv, floor_div(ptot * blockIdx.x, a.ncta), lane);
         pb = flat_of_work(wpre, prefix, nv, floor_div(ptot * (blockIdx.x + 1), a.ncta), lane);
@@ -637,7 +719,7 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
         }
     }
     if (pa >= pb) return;
-    const int v0 = aligned ? vc : find_vunit_warp(prefix, nv, pa, lane);
+    const int v0 = aligned ? vc : (have_range ? misc[13] : find_vunit_warp(prefix, nv, pa, lane));
     const int n_my = static_cast<int>(pb - pa);
 
     if (warp == NCONS) {
