@@ -830,26 +830,25 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
             // group: S (16 rows x 16 nodes) = Q K^T as two n8 tiles of nodes, the softmax on the
             // accumulators (each row spread over a quad of lanes), and P -- whose accumulator
             // layout is already the A operand of the next product -- times V into O (16 rows x D).
-            uint32_t qa[NKS][4];   // A fragments of Q: rows g / g + 8, dims 2c, 2c + 1 (+ 8) of each k-step
+            // The A fragments of Q (rows g / g + 8, dims 2c, 2c + 1 (+ 8) of each k-step) are read
+            // from the piece's query slot at every k-step rather than held in 32 registers across
+            // the page loop; the slot is released at the piece's end.
             float qn_g = 0.0f, qn_h = 0.0f;   // |q|^2 of rows g and g + 8 (h: the row 8 below)
+            const int qslot = pi & 1;
+            const uint32_t qb =
+                smem_u32(qbuf + qslot * L::QBUF) + (wt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1)) * L::QROWB;
             {
-                const int slot = pi & 1;
-                if (alive && !mbar_wait(&qfull[slot], (pi >> 1) & 1)) {
+                if (alive && !mbar_wait(&qfull[qslot], (pi >> 1) & 1)) {
                     if (lane == 0) raise_flag(a.flags, FLAG_TIMEOUT);
                     alive = false;
                 }
-                const uint32_t qb =
-                    smem_u32(qbuf + slot * L::QBUF) + (wt * 16 + (lane & 7) + 8 * ((lane >> 3) & 1)) * L::QROWB;
-#pragma unroll
-                for (int ks = 0; ks < NKS; ++ks)
-                    ldsm_x4(qb + ((2 * ks + (lane >> 4)) << 4), qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3]);
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&qempty[slot]);
 #pragma unroll
                 for (int ks = 0; ks < NKS; ++ks) {
+                    uint32_t qf[4];
+                    ldsm_x4(qb + ((2 * ks + (lane >> 4)) << 4), qf[0], qf[1], qf[2], qf[3]);
 #pragma unroll
                     for (int r2 = 0; r2 < 4; r2 += 2) {
-                        const uint32_t wg = qa[ks][r2], wh = qa[ks][r2 + 1];
+                        const uint32_t wg = qf[r2], wh = qf[r2 + 1];
                         qn_g = fmaf(bf16lo(wg), bf16lo(wg), qn_g);
                         qn_g = fmaf(bf16hi(wg), bf16hi(wg), qn_g);
                         qn_h = fmaf(bf16lo(wh), bf16lo(wh), qn_h);
@@ -886,19 +885,29 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                     // (r1, r3) as the B fragments of the two node tiles; the next k-step's load is
                     // issued before this one's MMAs
                     float sacc[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
+                    // odd k-steps accumulate apart: two chains of four dependent MMAs per node tile
+                    float sodd[2][4] = {{0.0f, 0.0f, 0.0f, 0.0f}, {0.0f, 0.0f, 0.0f, 0.0f}};
                     {
                         const int node = (lane & 7) + 8 * (mi & 1);
-                        uint32_t kn[4];
+                        uint32_t kn[4], qn[4];
                         ldsm_x4(kb + node * G::ROWB + (swz(mi >> 1, node) << 4), kn[0], kn[1], kn[2], kn[3]);
+                        ldsm_x4(qb + ((lane >> 4) << 4), qn[0], qn[1], qn[2], qn[3]);
 #pragma unroll
                         for (int ks = 0; ks < NKS; ++ks) {
                             const uint32_t k0 = kn[0], k1 = kn[1], k2 = kn[2], k3 = kn[3];
-                            if (ks + 1 < NKS)
+                            const uint32_t q0 = qn[0], q1 = qn[1], q2 = qn[2], q3 = qn[3];
+                            if (ks + 1 < NKS) {
                                 ldsm_x4(kb + node * G::ROWB + (swz(2 * (ks + 1) + (mi >> 1), node) << 4), kn[0], kn[1],
                                         kn[2], kn[3]);
-                            mma_bf16(sacc[0], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], k0, k2);
-                            mma_bf16(sacc[1], qa[ks][0], qa[ks][1], qa[ks][2], qa[ks][3], k1, k3);
+                                ldsm_x4(qb + ((2 * (ks + 1) + (lane >> 4)) << 4), qn[0], qn[1], qn[2], qn[3]);
+                            }
+                            mma_bf16((ks & 1) ? sodd[0] : sacc[0], q0, q1, q2, q3, k0, k2);
+                            mma_bf16((ks & 1) ? sodd[1] : sacc[1], q0, q1, q2, q3, k1, k3);
                         }
+#pragma unroll
+                        for (int nt = 0; nt < 2; ++nt)
+#pragma unroll
+                            for (int r = 0; r < 4; ++r) sacc[nt][r] += sodd[nt][r];
                     }
                     // logits of nodes 8 nt + 2c + e for rows g (accumulator e) and g + 8 (2 + e)
                     const float4 abA = ab4[c], abB = ab4[4 + c];   // nodes 2c, 2c+1 and 8+2c, 9+2c
@@ -975,6 +984,8 @@ __global__ void __launch_bounds__(SplitSmem<D, NT, DIAG>::THREADS, SplitSmem<D, 
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&empty[s]);   // K and V read: release the stage
             }
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&qempty[qslot]);   // the piece's query rows are no longer read
             i0 += npg;
             ++pi;
 
