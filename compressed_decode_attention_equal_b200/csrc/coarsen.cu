@@ -12,8 +12,8 @@
 //   k_project_scan   TMA-staged tiles of 511 middle tokens (+1 halo): z via the
 //                    fixed fp32 fma recipe, D_t = rne(d_t 2^20), tile-local
 //                    inclusive int64 scan and tile totals
-//   k_tile_prefix    exclusive scan of tile totals per unit, c_T
-//   k_boundaries     every token writes the thresholds it crosses:
+//   k_boundaries     c_T and each tile's start from the tile totals; every token
+//                    writes the thresholds it crosses:
 //                    b_j = t for N c_{t-1} < j c_T <= N c_t (128-bit products)
 //   k_plan_entries   drop empty segments, lay out entries (sinks, segments,
 //                    recents) and write lens
@@ -512,40 +512,6 @@ __global__ void __launch_bounds__(kK1Threads, 2)
 }
 
 // ---------------------------------------------------------------------------
-// k_tile_prefix: exclusive scan of the tile totals of one unit; c_T
-// ---------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) k_tile_prefix(const CoarsenArgs a) {
-    __shared__ long long wsum[8];
-    __shared__ long long carry_s;
-    const int u = blockIdx.x;
-    const int b = u / a.Hkv;
-    const SeqRow sr = a.seq[b];
-    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-    const int64_t rowb = static_cast<int64_t>(u) * a.max_tiles;
-    long long carry = 0;
-    for (int base = 0; base < sr.tiles; base += 256) {
-        const int i = base + tid;
-        const long long x = i < sr.tiles ? a.tile_total[rowb + i] : 0;
-        long long v = x;
-#pragma unroll
-        for (int off = 1; off < 32; off <<= 1) {
-            const long long n = __shfl_up_sync(0xffffffffu, v, off);
-            if (lane >= off) v += n;
-        }
-        if (lane == 31) wsum[warp] = v;
-        __syncthreads();
-        long long wp = 0;
-        for (int w = 0; w < warp; ++w) wp += wsum[w];
-        if (i < sr.tiles) a.tile_prefix[rowb + i] = carry + wp + v - x;
-        if (tid == 255) carry_s = carry + wp + v;
-        __syncthreads();
-        carry = carry_s;
-        __syncthreads();
-    }
-    if (tid == 0) a.unit_total[u] = carry;
-}
-
-// ---------------------------------------------------------------------------
 // k_boundaries: b_j = first t with N c_t >= j c_T  (j = 1 .. N-1)
 // ---------------------------------------------------------------------------
 // floor(N * C / CT) for CT > 0, exact: the double estimate (inv_ct = 1 / CT) is off by at most one
@@ -562,44 +528,143 @@ __device__ __forceinline__ long long floor_ratio(long long N, long long C, long 
     return q;
 }
 
+// floor(N c / c_T) from the double estimate x = fl(fl(c) * scale), scale = fl(N * fl(1 / c_T)): four
+// roundings, so |x - N c / c_T| <= N 2^-51 (the ratio is at most N). When x lies farther than
+// guard = N 2^-48 from every integer its floor is the exact one (x - floor(x) is exact: both are
+// multiples of x's ulp); -1 otherwise (undecided: the exact floor_ratio decides).
+__device__ __forceinline__ int floor_estimate(long long c, double scale, double guard) {
+    const double x = static_cast<double>(c) * scale;
+    const double f = floor(x);
+    return x - f > guard && x - f < 1.0 - guard ? static_cast<int>(f) : -1;
+}
+
 // One thread per middle token t: the thresholds j with floor(N c_{t-1} / c_T) < j <= floor(N c_t / c_T)
-// are first hit at t. Each thread computes its own floor once and takes its predecessor's from the
-// neighbouring lane (the first lane of a warp computes both).
-__global__ void __launch_bounds__(kTileRows) k_boundaries(const CoarsenArgs a) {
-    const int u = blockIdx.y, tile = blockIdx.x;
+// are first hit at t. Each thread takes its own floor once; its predecessor's comes from the lane
+// below, across warps through shared memory, and for a tile's first token from the tile's start.
+// A CTA takes kBndTiles consecutive tiles of one unit: c at the start of its first tile and c_T are
+// sums of the unit's tile totals (exact integers), so no separate prefix pass over the tiles runs
+// before it. All its loads are issued before the first floor is taken and the floors stay in
+// registers: those of the double estimate first, then the exact ones for the few estimates that lie
+// too close to an integer.
+constexpr int kBndTiles = 4;
+
+__global__ void __launch_bounds__(kTileRows, 2) k_boundaries(const CoarsenArgs a) {
+    constexpr int WARPS = kTileRows / 32;
+    __shared__ long long red[2][WARPS];
+    __shared__ long long tts[kBndTiles];     // the CTA's tile totals
+    __shared__ int qlast[kBndTiles][WARPS];  // the floor of each warp's last token, per tile
+    __shared__ int qstart[kBndTiles];        // the floor at each tile's start (its first token's predecessor)
+    const int u = blockIdx.y, tile0 = blockIdx.x * kBndTiles;
     const int b = u / a.Hkv, h = u % a.Hkv;
     const SeqRow sr = a.seq[b];
-    if (tile >= sr.tiles) return;
-    const int t = tile * kTileOut + threadIdx.x;
-    const bool act = threadIdx.x < kTileOut && t < sr.M;   // inactive threads sit at the tile's end
+    if (tile0 >= sr.tiles) {
+        if (blockIdx.x == 0 && threadIdx.x == 0) a.unit_total[u] = 0;   // a unit without middle tokens
+        return;
+    }
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int64_t rowb = static_cast<int64_t>(u) * a.max_tiles;
     const int64_t *ls = a.local_scan + sr.mid_off + static_cast<int64_t>(h) * sr.M;
-    const long long tp = a.tile_prefix[static_cast<int64_t>(u) * a.max_tiles + tile];
-    const long long CT = a.unit_total[u];
-    const long long Ct = act ? tp + ls[t] : 0;
-    if (act && a.cumvar) a.cumvar[sr.row_off + static_cast<int64_t>(h) * sr.T + t] = Ct;
+    long long before = 0, total = 0;   // this thread's share of the tile totals before tile0 / of all
+    for (int i = tid; i < sr.tiles; i += kTileRows) {
+        const long long x = a.tile_total[rowb + i];
+        total += x;
+        if (i < tile0) before += x;
+    }
+    long long lsv[kBndTiles];   // the tile-local scan at this thread's token of each tile; -1: none
+#pragma unroll
+    for (int g = 0; g < kBndTiles; ++g) {
+        const int tile = tile0 + g;
+        const int t = tile * kTileOut + tid;
+        lsv[g] = tile < sr.tiles && tid < kTileOut && t < sr.M ? ls[t] : -1;   // inactive threads sit at the end
+    }
+    if (tid < kBndTiles) tts[tid] = tile0 + tid < sr.tiles ? a.tile_total[rowb + tile0 + tid] : 0;
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        before += __shfl_xor_sync(0xffffffffu, before, off);
+        total += __shfl_xor_sync(0xffffffffu, total, off);
+    }
+    if (lane == 0) {
+        red[0][warp] = before;
+        red[1][warp] = total;
+    }
+    __syncthreads();
+    before = total = 0;
+#pragma unroll
+    for (int w = 0; w < WARPS; ++w) {
+        before += red[0][w];
+        total += red[1][w];
+    }
+    const long long CT = total;   // c_T
+    if (blockIdx.x == 0 && tid == 0) a.unit_total[u] = CT;
     const int N = sr.N;
+    if (a.cumvar) {   // c_t of the tiles' middle tokens
+        long long tp = before;
+#pragma unroll
+        for (int g = 0; g < kBndTiles; ++g) {
+            const int t = (tile0 + g) * kTileOut + tid;
+            if (lsv[g] >= 0) a.cumvar[sr.row_off + static_cast<int64_t>(h) * sr.T + t] = tp + lsv[g];
+            tp += tts[g];
+        }
+    }
     int32_t *bnd = a.bounds + sr.bnd_off + static_cast<int64_t>(h) * (N + 1);
     if (CT == 0) {
-        if (t == 0)
+        if (tile0 == 0 && tid == 0)
             for (int j = 1; j < N; ++j) bnd[j] = 0;
         return;
     }
     const double inv = 1.0 / static_cast<double>(CT);
-    const long long q = act ? floor_ratio(N, Ct, CT, inv) : 0;
-    long long qprev = __shfl_up_sync(0xffffffffu, q, 1);
-    if ((threadIdx.x & 31) == 0 && act)
-        qprev = floor_ratio(N, threadIdx.x == 0 ? tp : tp + ls[t - 1], CT, inv);
-    if (!act || t == 0) return;
-    const long long jhi = q > N - 1 ? N - 1 : q;
-    for (long long j = qprev + 1; j <= jhi; ++j) bnd[j] = t;
+    const double scale = static_cast<double>(N) * inv, guard = static_cast<double>(N) * 0x1p-48;
+    int q[kBndTiles];
+    uint32_t undecided = 0;
+    {
+        long long tp = before;
+#pragma unroll
+        for (int g = 0; g < kBndTiles; ++g) {
+            q[g] = floor_estimate(lsv[g] >= 0 ? tp + lsv[g] : 0, scale, guard);
+            if (q[g] < 0) undecided |= 1u << g;
+            tp += tts[g];
+        }
+    }
+    if (undecided) {   // the exact floors with 128-bit products (rare)
+        long long tp = before;
+#pragma unroll
+        for (int g = 0; g < kBndTiles; ++g) {
+            if (undecided & (1u << g)) q[g] = static_cast<int>(floor_ratio(N, lsv[g] >= 0 ? tp + lsv[g] : 0, CT, inv));
+            tp += tts[g];
+        }
+    }
+    if (lane == 31) {
+#pragma unroll
+        for (int g = 0; g < kBndTiles; ++g) qlast[g][warp] = q[g];
+    }
+    if (tid < kBndTiles) {   // thread g: the floor at tile g's start
+        long long tp = before;
+        for (int g = 0; g < tid; ++g) tp += tts[g];
+        int f = floor_estimate(tp, scale, guard);
+        if (f < 0) f = static_cast<int>(floor_ratio(N, tp, CT, inv));
+        qstart[tid] = f;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int g = 0; g < kBndTiles; ++g) {
+        if (tile0 + g >= sr.tiles) break;   // (the same for the whole CTA)
+        const int t = (tile0 + g) * kTileOut + tid;
+        int qprev = __shfl_up_sync(0xffffffffu, q[g], 1);
+        if (lane == 0) qprev = warp > 0 ? qlast[g][warp - 1] : qstart[g];
+        if (lsv[g] >= 0 && t != 0) {
+            const int jhi = q[g] > N - 1 ? N - 1 : q[g];
+            for (int j = qprev + 1; j <= jhi; ++j) bnd[j] = t;
+        }
+    }
 }
 
 // ---------------------------------------------------------------------------
 // k_plan_entries: entries (start, mass) in the order sinks, nonempty segments, recents
 // ---------------------------------------------------------------------------
+constexpr int kPlanSeg = 8;   // segments per thread and round of k_plan_entries
+
 __global__ void __launch_bounds__(512) k_plan_entries(const CoarsenArgs a) {
     __shared__ int wsum[16];
-    __shared__ int carry_s;
     const int u = blockIdx.x;
     const int b = u / a.Hkv, h = u % a.Hkv;
     const SeqRow sr = a.seq[b];
@@ -615,16 +680,17 @@ __global__ void __launch_bounds__(512) k_plan_entries(const CoarsenArgs a) {
     __syncthreads();
     int2 *ents = a.ents + sr.ent_off + static_cast<int64_t>(h) * sr.emax;
     for (int e = tid; e < sr.s_eff; e += 512) ents[e] = make_int2(e, 1);
+    // each thread takes kPlanSeg consecutive segments of a round: all its boundaries are read at once
     int carry = 0;
-    for (int base = 0; base < N; base += 512) {
-        const int j = base + tid;
-        int lo = 0, hi = 0;
-        if (j < N) {
-            lo = bnd[j];
-            hi = bnd[j + 1];
-        }
-        const int f = (j < N && hi > lo) ? 1 : 0;
-        int v = f;
+    for (int base = 0; base < N; base += 512 * kPlanSeg) {
+        const int j0 = base + tid * kPlanSeg;
+        int bv[kPlanSeg + 1];
+#pragma unroll
+        for (int i = 0; i <= kPlanSeg; ++i) bv[i] = j0 + i <= N ? bnd[j0 + i] : 0;
+        int cnt = 0;
+#pragma unroll
+        for (int i = 0; i < kPlanSeg; ++i) cnt += (j0 + i < N && bv[i + 1] > bv[i]) ? 1 : 0;
+        int v = cnt;
 #pragma unroll
         for (int off = 1; off < 32; off <<= 1) {
             const int n = __shfl_up_sync(0xffffffffu, v, off);
@@ -632,13 +698,19 @@ __global__ void __launch_bounds__(512) k_plan_entries(const CoarsenArgs a) {
         }
         if (lane == 31) wsum[warp] = v;
         __syncthreads();
-        int wp = 0;
-        for (int w = 0; w < warp; ++w) wp += wsum[w];
-        if (f) ents[sr.s_eff + carry + wp + v - 1] = make_int2(sr.s_eff + lo, hi - lo);
-        if (tid == 511) carry_s = carry + wp + v;
-        __syncthreads();
-        carry = carry_s;
-        __syncthreads();
+        int wp = 0, all = 0;
+#pragma unroll
+        for (int w = 0; w < 16; ++w) {
+            const int x = wsum[w];
+            all += x;
+            if (w < warp) wp += x;
+        }
+        int e = sr.s_eff + carry + wp + v - cnt;   // this thread's first entry
+#pragma unroll
+        for (int i = 0; i < kPlanSeg; ++i)
+            if (j0 + i < N && bv[i + 1] > bv[i]) ents[e++] = make_int2(sr.s_eff + bv[i], bv[i + 1] - bv[i]);
+        carry += all;
+        __syncthreads();   // wsum is read before the next round writes it
     }
     for (int i = tid; i < sr.w_eff; i += 512) ents[sr.s_eff + carry + i] = make_int2(sr.s_eff + M + i, 1);
     if (tid == 0) a.lens[u] = sr.s_eff + carry + sr.w_eff;
@@ -682,6 +754,7 @@ struct Vec16<float> {
 };
 
 constexpr int kK3Warps = 8;
+constexpr int kSegPrefetchRows = 256;   // rows of a segment prefetched into L2 at its start
 
 // W: the variation-weighted representative is compiled in (a separate instantiation, so the
 // plain-mean kernel keeps its register budget).
@@ -712,6 +785,20 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
     const int64_t row0 = sr.row_off + static_cast<int64_t>(h) * sr.T + start;
     const uint8_t *kp = static_cast<const uint8_t *>(a.k) + row0 * ROWB + ch * 16;
     const uint8_t *vp = static_cast<const uint8_t *>(a.v) + row0 * ROWB + ch * 16;
+    // The segment's rows are contiguous: one bulk L2 prefetch per tensor (its first kSegPrefetchRows
+    // rows) puts the first pass's DRAM reads in flight at once, so that the warp's loads below wait
+    // on L2 rather than on a chain of DRAM round trips. Taken by the weighted kernel only, whose
+    // register budget leaves fewer warps per SM to cover the latency (the plain mean measured
+    // slower with it).
+    if (W && lane == 0 && m > 8) {
+        const uint8_t *k0 = static_cast<const uint8_t *>(a.k) + row0 * ROWB;
+        const uint8_t *v0 = static_cast<const uint8_t *>(a.v) + row0 * ROWB;
+        const uint32_t bytes = static_cast<uint32_t>(m < kSegPrefetchRows ? m : kSegPrefetchRows) * ROWB;
+        if (((reinterpret_cast<uintptr_t>(k0) | reinterpret_cast<uintptr_t>(v0)) & 15u) == 0) {
+            bulk_prefetch_l2(k0, bytes);
+            bulk_prefetch_l2(v0, bytes);
+        }
+    }
 
     // A middle segment with the variation-weighted representative ("Equal-Variation KV Cache",
     // "Implementation notes") also accumulates sum_r d_r k_r, sum_r d_r v_r and sum_r d_r with
@@ -905,10 +992,8 @@ static cudaError_t launch_projection(const CoarsenArgs &a, int n, const ProjT &p
 // segment statistics.
 template <int D, typename T, bool CENTER>
 static void launch_segments(const CoarsenArgs &a, int n, cudaStream_t s) {
-    if (a.max_tiles > 0) {
-        k_tile_prefix<<<n, 256, 0, s>>>(a);
-        k_boundaries<<<dim3(a.max_tiles, n), kTileRows, 0, s>>>(a);
-    }
+    const int bnd_ctas = (a.max_tiles + kBndTiles - 1) / kBndTiles;   // (one per unit writes c_T = 0 without tiles)
+    k_boundaries<<<dim3(bnd_ctas > 0 ? bnd_ctas : 1, n), kTileRows, 0, s>>>(a);
     k_plan_entries<<<n, 512, 0, s>>>(a);
     if (a.max_emax > 0) {
         const dim3 g3((a.max_emax + kK3Warps - 1) / kK3Warps, n);

@@ -189,8 +189,6 @@ skv_status plan_coarsen(int B, int Hkv, int d, const int32_t *T_host, const int3
     off += align256(sizeof(SeqRow) * B);
     p.lay.tile_total = off;
     off += align256(static_cast<size_t>(units) * p.max_tiles * 8);
-    p.lay.tile_prefix = off;
-    off += align256(static_cast<size_t>(units) * p.max_tiles * 8);
     p.lay.unit_total = off;
     off += align256(static_cast<size_t>(units) * 8);
     p.lay.local_scan = off;
@@ -430,7 +428,6 @@ static skv_status coarsen_impl(const void *k, const void *v, skv_dtype dtype, in
     a.Nmax = plan.Nmax;
     a.seq = reinterpret_cast<const SeqRow *>(ws + plan.lay.seq);
     a.tile_total = reinterpret_cast<int64_t *>(ws + plan.lay.tile_total);
-    a.tile_prefix = reinterpret_cast<int64_t *>(ws + plan.lay.tile_prefix);
     a.unit_total = reinterpret_cast<int64_t *>(ws + plan.lay.unit_total);
     a.local_scan = reinterpret_cast<int64_t *>(ws + plan.lay.local_scan);
     a.bounds = reinterpret_cast<int32_t *>(ws + plan.lay.bounds);

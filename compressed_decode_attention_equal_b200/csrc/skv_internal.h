@@ -55,7 +55,7 @@ struct CoarsenArgs {
     int max_emax;    // largest emax over the batch
     int Nmax;        // largest N over the batch
     const SeqRow *seq;
-    int64_t *tile_total, *tile_prefix, *unit_total, *local_scan;
+    int64_t *tile_total, *unit_total, *local_scan;
     int32_t *bounds;
     int2 *ents;
     uint32_t *flags;
@@ -79,7 +79,7 @@ constexpr int kMeanBlock = 256;   // tokens per block of the centring mean's fix
 
 // Workspace carve-up (offsets in bytes from the workspace start).
 struct CoarsenLayout {
-    size_t seq, tile_total, tile_prefix, unit_total, local_scan, bounds, ents, key_blk, key_mu, total;
+    size_t seq, tile_total, unit_total, local_scan, bounds, ents, key_blk, key_mu, total;
 };
 
 // Host-side launchers (coarsen.cu).
