@@ -192,6 +192,33 @@ def test_jump_crosses_many_thresholds():
     compare_units(r, orc, k, v, [T], 1, [30], torch.bfloat16)
 
 
+@pytest.mark.parametrize("projection", ["fixed", "tensor"])
+def test_thresholds_hit_exactly(projection):
+    """Keys alternating between two rows make every middle step the same D (fl(x - y) = -fl(y - x)),
+    so c_t = t D. With M - 1 = N k the ratio N c_t / c_T = t / k is an integer at every threshold:
+    the double estimate of each floor lies within its guard band of an integer and the exact
+    128-bit path decides. Closed form: b_j = j k, and (fixed recipe) bit-exact with the oracle."""
+    N, kstep, d = 16, 40, 128
+    M = N * kstep + 1                      # two projection tiles
+    T = S + M + W
+    g = torch.Generator(device="cuda").manual_seed(11)
+    k = (torch.randn(T, d, device="cuda", generator=g) * 0.3).bfloat16()
+    v = torch.zeros(T, d, dtype=torch.bfloat16, device="cuda")
+    a, b = k[S].clone(), (k[S] * -0.5 + 0.125).bfloat16()
+    k[S:S + M:2] = a
+    k[S + 1:S + M:2] = b
+    r = run_coarsen(k, v, 1, [T], [N], seed=5, projection=projection)
+    assert r["status"] == 0, r["flags"]
+    C = r["cum"][:M].cpu().numpy()        # c_t of the middle tokens t = 0 .. M - 1
+    D = int(C[1])
+    assert D > 0 and np.array_equal(C, np.arange(M, dtype=np.int64) * D), "steps are not all equal"
+    bnd = r["bnd"][0, 0, :N + 1].cpu().numpy()
+    assert np.array_equal(bnd, np.append(np.arange(N) * kstep, M)), bnd
+    if projection == "fixed":
+        orc = oracle_units(k, v, 1, [T], [N], seed=5)
+        compare_units(r, orc, k, v, [T], 1, [N], torch.bfloat16)
+
+
 def test_overflow_is_flagged():
     T, d = 300, 128
     k = torch.zeros(T, d, dtype=torch.float32, device="cuda")

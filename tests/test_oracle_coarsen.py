@@ -128,6 +128,25 @@ def test_identical_keys_zero_variance(orc):
     assert np.all(u.sigma2 == 0.0) and np.all(u.beta == 0.0)
 
 
+def test_alternating_keys_hit_every_threshold_exactly(orc):
+    """Keys alternating between two rows give every middle step the same D (the difference of the
+    two projections, negated, has the same square norm), so c_t = t D; with M - 1 = N k the
+    thresholds j c_T / N are hit exactly, at b_j = j k (the equality case of N c_t >= j c_T)."""
+    d, S, W, N, step = 64, 8, 48, 16, 40
+    M = N * step + 1
+    T = S + M + W
+    rng = np.random.default_rng(3)
+    k = (rng.standard_normal((T, d)) * 0.3).astype(np.float32)
+    v = np.zeros((T, d), np.float32)
+    a = k[S].copy()
+    k[S:S + M:2] = a
+    k[S + 1:S + M:2] = a * np.float32(-0.5) + np.float32(0.125)
+    u = orc.coarsen_unit(k, v, S, W, N, orc.projection(5, d))
+    assert u.C[1] > 0 and np.array_equal(u.C, np.arange(M, dtype=np.int64) * u.C[1])
+    assert np.array_equal(u.bounds, np.append(np.arange(N) * step, M))
+    assert np.all(u.mass[S:S + N - 1] == step) and u.mass[S + N - 1] == step + 1   # the last also takes t = M - 1
+
+
 def test_overflow_is_reported(orc):
     d, T = 64, 20
     k = np.zeros((T, d), np.float32)
