@@ -2,7 +2,7 @@
 
 Bit-exact: the projection P, every unit's cumulative quantised variation c_t, the segment
 boundaries, the entry counts. Within tolerance: node statistics (mean key / value, alpha = ln m,
-beta = sigma^2 / (2d)). Sizes span several projection tiles (255 tokens each) with ragged tails,
+beta = sigma^2 / (2d)). Sizes span several projection tiles (511 middle tokens each) with ragged tails,
 plus the degenerate cases: T <= n_sink + n_recent, empty middle, M < N (empty segments dropped),
 constant middle (c_T = 0), N = 1, one jump crossing many thresholds, d = 64 / 128, fp32 / bf16;
 every case also with the variation-weighted segment representative."""
@@ -91,8 +91,8 @@ CASES = [
     ("short_sequences", torch.bfloat16, 128, 2, [0, 1, 8, 55, 56, 57, 60, 63], [4, 4, 4, 4, 4, 4, 4, 4], "normal"),
     ("more_segments_than_tokens", torch.bfloat16, 128, 1, [70, 200], [40, 500], "normal"),
     ("single_segment", torch.bfloat16, 128, 2, [3000], [1], "normal"),
-    ("tile_edges", torch.bfloat16, 128, 1, [56 + 255, 56 + 256, 56 + 510, 56 + 511, 56 + 254], [7, 7, 7, 7, 7],
-     "normal"),
+    ("tile_edges", torch.bfloat16, 128, 1, [56 + 255, 56 + 510, 56 + 511, 56 + 512, 56 + 1022, 56 + 1023],
+     [7, 7, 7, 7, 7, 7], "normal"),
     # 21 units of ragged lengths: one sequence empty, one without a middle, one with N = 1
     ("many_units_ragged", torch.bfloat16, 128, 3, [900, 40, 1500, 0, 700, 2100, 333], [30, 4, 60, 4, 1, 80, 9],
      "normal"),
