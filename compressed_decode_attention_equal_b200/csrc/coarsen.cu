@@ -531,8 +531,10 @@ __device__ __forceinline__ long long floor_ratio(long long N, long long C, long 
 // floor(N c / c_T) from the double estimate x = fl(fl(c) * scale), scale = fl(N * fl(1 / c_T)): four
 // roundings, so |x - N c / c_T| <= N 2^-51 (the ratio is at most N). When x lies farther than
 // guard = N 2^-48 from every integer its floor is the exact one (x - floor(x) is exact: both are
-// multiples of x's ulp); -1 otherwise (undecided: the exact floor_ratio decides).
+// multiples of x's ulp); -1 otherwise (undecided: the exact floor_ratio decides). c = 0 (the unit's
+// first token, and threads without a token) is exact at once.
 __device__ __forceinline__ int floor_estimate(long long c, double scale, double guard) {
+    if (c == 0) return 0;
     const double x = static_cast<double>(c) * scale;
     const double f = floor(x);
     return x - f > guard && x - f < 1.0 - guard ? static_cast<int>(f) : -1;
@@ -548,7 +550,7 @@ __device__ __forceinline__ int floor_estimate(long long c, double scale, double 
 // too close to an integer.
 constexpr int kBndTiles = 4;
 
-__global__ void __launch_bounds__(kTileRows, 2) k_boundaries(const CoarsenArgs a) {
+__global__ void __launch_bounds__(kTileRows, 3) k_boundaries(const CoarsenArgs a) {
     constexpr int WARPS = kTileRows / 32;
     __shared__ long long red[2][WARPS];
     __shared__ long long tts[kBndTiles];     // the CTA's tile totals
