@@ -68,6 +68,8 @@ __global__ void __launch_bounds__(D) k_key_mean(const CoarsenArgs a) {
     const int nblk = (sr.T + kMeanBlock - 1) / kMeanBlock;
     const float *bs = a.key_blk + static_cast<int64_t>(u) * a.max_blk * D + threadIdx.x;
     float tot = 0.0f;
+    // (unrolled so that the loads run ahead of the additions, which keep the fixed block order)
+#pragma unroll 16
     for (int c = 0; c < nblk; ++c) tot = __fadd_rn(tot, bs[static_cast<int64_t>(c) * D]);
     a.key_mu[static_cast<int64_t>(u) * D + threadIdx.x] = sr.T > 0 ? __fdiv_rn(tot, static_cast<float>(sr.T)) : 0.0f;
 }
