@@ -219,6 +219,33 @@ def test_thresholds_hit_exactly(projection):
         compare_units(r, orc, k, v, [T], 1, [N], torch.bfloat16)
 
 
+@pytest.mark.parametrize("projection", ["fixed", "tensor"])
+def test_long_unit_over_512_tiles(projection):
+    """One unit of 600 full projection tiles plus a ragged tail (306,677 middle tokens): the
+    boundary kernel sums more than 512 tile totals per unit (two rounds of its CTA) for c_T and
+    each tile's start. Fixed recipe: c_t, boundaries and statistics against the oracle. Both
+    projections: the boundaries are the first hits of N c_t >= j c_T on the GPU's own c_t, in
+    exact integers."""
+    d, N = 64, 64
+    M = 600 * 511 + 77
+    T = S + M + W
+    g = torch.Generator(device="cuda").manual_seed(21)
+    k = (torch.randn(T, d, device="cuda", generator=g) * 0.05).cumsum(0).bfloat16()
+    v = (torch.randn(T, d, device="cuda", generator=g) * 0.5).bfloat16()
+    r = run_coarsen(k, v, 1, [T], [N], seed=3, projection=projection)
+    assert r["status"] == 0, r["flags"]
+    C = r["cum"][:M].cpu().numpy()
+    CT = int(C[-1])
+    assert CT > 0 and np.all(np.diff(C) >= 0)
+    # N c_t >= j c_T  <=>  c_t >= ceil(j c_T / N) for integer c_t: the first such t by bisection
+    thr = np.array([-(-j * CT // N) for j in range(1, N)], dtype=np.int64)
+    want = np.concatenate([[0], np.searchsorted(C, thr, side="left"), [M]])
+    assert np.array_equal(r["bnd"][0, 0, :N + 1].cpu().numpy(), want)
+    if projection == "fixed":
+        orc = oracle_units(k, v, 1, [T], [N], seed=3)
+        compare_units(r, orc, k, v, [T], 1, [N], torch.bfloat16)
+
+
 def test_overflow_is_flagged():
     T, d = 300, 128
     k = torch.zeros(T, d, dtype=torch.float32, device="cuda")
