@@ -246,6 +246,32 @@ def test_long_unit_over_512_tiles(projection):
         compare_units(r, orc, k, v, [T], 1, [N], torch.bfloat16)
 
 
+def test_more_than_4096_segments():
+    """N = 6,000 over 20,000 middle tokens: the entry planner runs two rounds of 4,096 segments
+    (the entry offset carried between them) and drops the empty segments of both (two jumps, each
+    crossing several thresholds at once); entries and statistics against the oracle."""
+    rows = _jump_walk()
+    T, d, N = rows.shape[0], rows.shape[1], 6000
+    k = rows.bfloat16().cuda()
+    v = (torch.randn(T, d, generator=torch.Generator().manual_seed(32)) * 0.5).bfloat16().cuda()
+    r = run_coarsen(k, v, 1, [T], [N], seed=4)
+    assert r["status"] == 0, r["flags"]
+    orc = oracle_units(k, v, 1, [T], [N], seed=4)
+    empty = np.diff(orc[(0, 0)].bounds) == 0
+    assert empty[:4096].any() and empty[4096:].any()   # empty segments in both rounds
+    compare_units(r, orc, k, v, [T], 1, [N], torch.bfloat16)
+
+
+def _jump_walk(M=20000, d=64):
+    """A random walk over S + M + W rows (CPU generator) with +30 jumps at middle tokens 3,000 and
+    17,000."""
+    g = torch.Generator().manual_seed(31)
+    k = (torch.randn(S + M + W, d, generator=g) * 0.05).cumsum(0)
+    k[S + 3000:] += 30.0
+    k[S + 17000:] += 30.0
+    return k
+
+
 def test_overflow_is_flagged():
     T, d = 300, 128
     k = torch.zeros(T, d, dtype=torch.float32, device="cuda")
