@@ -89,6 +89,8 @@ CASES = [
     ("f32_d128", torch.float32, 128, 2, [700], [21], "walk"),
     ("key_only_variation", torch.bfloat16, 128, 2, [2000, 900], [50, 30], "zero"),
     ("short_sequences", torch.bfloat16, 128, 2, [0, 1, 8, 55, 56, 57, 60, 63], [4, 4, 4, 4, 4, 4, 4, 4], "normal"),
+    # no unit of the batch has a middle token (no projection tile anywhere)
+    ("no_middle_anywhere", torch.bfloat16, 128, 2, [0, 8, 56], [4, 4, 4], "normal"),
     ("more_segments_than_tokens", torch.bfloat16, 128, 1, [70, 200], [40, 500], "normal"),
     ("single_segment", torch.bfloat16, 128, 2, [3000], [1], "normal"),
     ("tile_edges", torch.bfloat16, 128, 1, [56 + 255, 56 + 510, 56 + 511, 56 + 512, 56 + 1022, 56 + 1023],
