@@ -46,37 +46,6 @@ void make_projection(uint64_t seed, int d, float *P) {
     }
 }
 
-// Small cache of transposed projections, keyed by (seed, d).
-struct ProjCache {
-    std::mutex mu;
-    struct Entry {
-        uint64_t seed;
-        int d;
-        ProjT pt;
-    };
-    std::vector<Entry> entries;
-    void get(uint64_t seed, int d, ProjT &out) {
-        std::lock_guard<std::mutex> lock(mu);
-        for (auto &e : entries)
-            if (e.seed == seed && e.d == d) {
-                out = e.pt;
-                return;
-            }
-        std::vector<float> P(static_cast<size_t>(kProjDim) * 2 * d);
-        make_projection(seed, d, P.data());
-        Entry e;
-        e.seed = seed;
-        e.d = d;
-        std::memset(&e.pt, 0, sizeof e.pt);
-        for (int i = 0; i < kProjDim; ++i)
-            for (int j = 0; j < 2 * d; ++j) e.pt.pt[j * kProjDim + i] = P[static_cast<size_t>(i) * 2 * d + j];
-        if (entries.size() >= 16) entries.erase(entries.begin());
-        entries.push_back(e);
-        out = e.pt;
-    }
-};
-ProjCache g_proj;
-
 // bf16 bits of an fp32 value, rounded to nearest even (the inputs here are finite)
 uint16_t bf16_rne_bits(float x) {
     uint32_t u;
@@ -85,9 +54,7 @@ uint16_t bf16_rne_bits(float x) {
 }
 
 // P16 = bf16(P) as the tensor-core projection's shared-memory image (see ProjFrag).
-void make_projection_fragments(uint64_t seed, int d, ProjFrag &out) {
-    std::vector<float> P(static_cast<size_t>(kProjDim) * 2 * d);
-    make_projection(seed, d, P.data());
+void make_projection_fragments(const float *P, int d, ProjFrag &out) {
     std::memset(&out, 0, sizeof out);
     const int cols = 2 * d, nchunk = cols / 32;
     uint16_t *img = reinterpret_cast<uint16_t *>(out.w);
@@ -100,6 +67,42 @@ void make_projection_fragments(uint64_t seed, int d, ProjFrag &out) {
                         bf16_rne_bits(P[static_cast<size_t>(n) * cols + k]);
                 }
 }
+
+// Small cache of the projection in both device forms -- transposed fp32 for the fixed recipe, the
+// bf16 image for the tensor cores -- keyed by (seed, d), so that a call draws P only the first time.
+struct ProjCache {
+    std::mutex mu;
+    struct Entry {
+        uint64_t seed;
+        int d;
+        ProjT pt;
+        ProjFrag frag;
+    };
+    std::vector<Entry> entries;
+    void get(uint64_t seed, int d, ProjT *pt, ProjFrag *frag) {
+        std::lock_guard<std::mutex> lock(mu);
+        for (auto &e : entries)
+            if (e.seed == seed && e.d == d) {
+                if (pt) *pt = e.pt;
+                if (frag) *frag = e.frag;
+                return;
+            }
+        std::vector<float> P(static_cast<size_t>(kProjDim) * 2 * d);
+        make_projection(seed, d, P.data());
+        Entry e;
+        e.seed = seed;
+        e.d = d;
+        std::memset(&e.pt, 0, sizeof e.pt);
+        for (int i = 0; i < kProjDim; ++i)
+            for (int j = 0; j < 2 * d; ++j) e.pt.pt[j * kProjDim + i] = P[static_cast<size_t>(i) * 2 * d + j];
+        make_projection_fragments(P.data(), d, e.frag);
+        if (entries.size() >= 16) entries.erase(entries.begin());
+        entries.push_back(e);
+        if (pt) *pt = e.pt;
+        if (frag) *frag = e.frag;
+    }
+};
+ProjCache g_proj;
 
 // ---------------------------------------------------------------------------
 // driver entry point for TMA descriptors (resolved once through the runtime)
@@ -403,9 +406,9 @@ static skv_status coarsen_impl(const void *k, const void *v, skv_dtype dtype, in
     static ProjFrag frag;   // host staging (guarded by table_mu)
     if (projection == SKV_PROJECTION_TENSOR_BF16) {
         std::memset(&proj, 0, sizeof proj);
-        make_projection_fragments(proj_seed, d, frag);
+        g_proj.get(proj_seed, d, nullptr, &frag);
     } else {
-        g_proj.get(proj_seed, d, proj);
+        g_proj.get(proj_seed, d, &proj, nullptr);
         std::memset(&frag, 0, sizeof frag);
     }
     CUtensorMap map_k, map_v;
