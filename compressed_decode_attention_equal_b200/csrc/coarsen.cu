@@ -811,10 +811,12 @@ __global__ void __launch_bounds__(kK3Warps * 32) k_segment_reduce(const CoarsenA
     const bool weighted = W && m > 1 && t_mid >= 0 && t_mid < sr.M;
     const int64_t *ls = a.local_scan + sr.mid_off + static_cast<int64_t>(h) * sr.M;
 
-    // loads are issued kUnroll token steps at a time (2 x kUnroll 16-byte loads in flight per lane);
-    // the weighted kernel takes 2 (75 registers, 3 CTAs per SM: its L2 prefetch already has the
-    // segment's rows in flight; 4 steps took 93 registers and 2 CTAs per SM and measured slower)
-    constexpr int kUnroll = W ? 2 : 8;
+    // loads are issued kUnroll token steps at a time (2 x kUnroll 16-byte loads in flight per lane).
+    // The plain kernel takes 10 (74 registers, 3 CTAs per SM; 4, 6, 8, 12 and 16 measured slower),
+    // the centred one 8 (10 costs it a CTA per SM). The weighted kernel takes 2 (75 registers, 3
+    // CTAs per SM: its L2 prefetch already has the segment's rows in flight; 4 steps took 93
+    // registers and 2 CTAs per SM and measured slower).
+    constexpr int kUnroll = W ? 2 : (CENTER ? 8 : 10);
     float sk[EPL], sv[EPL], wk[EPL], wv[EPL], x[EPL], wsum = 0.0f;
 #pragma unroll
     for (int i = 0; i < EPL; ++i) sk[i] = sv[i] = wk[i] = wv[i] = 0.0f;
